@@ -1,0 +1,358 @@
+"""Benchmark of the gated delta-rule hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one chunk-parallel forward (gdr_chunk_fwd) over the training-shape
+workload bf16_b8_h16_t4096_d128 (B=8, H=16, T=4096, dk=dv=128, chunk 64,
+post-write read, zero initial state), inputs resident in HBM.  The same run also
+times the batched decode step (gdr_decode_step, 256 sequences x 32 v-heads,
+128x128 fp32 state, 64 steps with fresh inputs) and reports its HBM bandwidth.
+
+Prints ONE JSON line on rank 0.  Under torchrun (N > 1) every rank runs the same
+workload on its own GPU with its own seed (weak scaling, no collective on the data
+path); the step time is the max over ranks.
+
+Inputs (q, k, v, o: 537 MB; decode state: 537 MB) are larger than the 126 MB L2,
+so no flush is done between timed iterations.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gated-delta chunk-fwd tokens/s + %bf16 TC peak; decode state GB/s vs HBM peak"
+CHUNK_WORKLOAD = "bf16_b8_h16_t4096_d128"
+DECODE_WORKLOAD = "bf16_decode_n256_hk16_hv32_d128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def flops_per_head_token(C, dk, dv):
+    """Dense chunk-form FLOPs per token per head: KK^T, QK^T, W (2C dk each), U and the
+    intra output (2C dv each), W H, the state update and Q H (2 dk dv each)."""
+    return 6 * C * dk + 4 * C * dv + 6 * dk * dv
+
+
+# ------------------------------------------------------------------ clocks sampler
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ our implementation
+
+def bench_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import gated_delta_rule_146_b200 as gdr
+    import workloads
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks, peak_src = load_peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------- chunk-parallel forward
+    w = workloads.WORKLOADS[args.workload]
+    x = workloads.workload_inputs(w, seed=rank)
+    d = {n: (t.to(dev) if t is not None else None) for n, t in x.items()}
+    cargs = gdr.make_chunk_args(d["q"], d["v"], d["g"], d["cu_seqlens"], w.chunk, w.read_mode,
+                                w.scale)
+    path = gdr.chunk_fwd_path(cargs)
+    ws = torch.empty(gdr.chunk_fwd_workspace_size(cargs), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(d["v"])
+    S_final = torch.empty((cargs.n_seqs, w.Hv, w.dk, w.dv), dtype=torch.float32, device=dev)
+
+    def step():
+        gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], d["cu_seqlens"],
+                      chunk=w.chunk, read_mode=w.read_mode, scale=w.scale, o=o, S_final=S_final,
+                      workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)  # let the sampler come up before the timed region
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+
+    tokens = int(d["q"].shape[0] * d["q"].shape[1])
+    head_tokens = tokens * w.Hv
+    flops = head_tokens * flops_per_head_token(w.chunk, w.dk, w.dv)
+    algo_bytes = sum(t.numel() * t.element_size() for t in
+                     (d["q"], d["k"], d["v"], d["g"], d["beta"], o, S_final)) + (
+        d["S0"].numel() * 4 if d["S0"] is not None else 0)
+    value = world * tokens / (ms / 1e3)
+    tflops = flops / (ms / 1e3) / 1e12
+    hbm_gbs = algo_bytes / (ms / 1e3) / 1e9
+    launches_per_call = 2 if path == "tc" else 3
+
+    # ---------------- decode step
+    dec = None
+    if not args.no_decode:
+        dw = workloads.DECODE_WORKLOADS[DECODE_WORKLOAD]
+        dx = workloads.decode_workload_inputs(dw, seed=rank)
+        dd = {n: t.to(dev) for n, t in dx.items()}
+        od = torch.empty((dw.N, dw.Hv, dw.dv), dtype=torch.bfloat16, device=dev)
+
+        def dstep(t):
+            gdr.decode_step(dd["q"][t], dd["k"][t], dd["v"][t], dd["g"][t], dd["beta"][t],
+                            dd["S"], read_mode=dw.read_mode, scale=dw.scale, o=od)
+
+        for t in range(min(args.warmup, dw.steps)):
+            dstep(t)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for t in range(dw.steps):
+            dstep(t)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        dms = max_over_ranks(e0.elapsed_time(e1) / dw.steps)
+        dbytes = 2 * dd["S"].numel() * 4 + sum(
+            dd[n][0].numel() * dd[n].element_size() for n in ("q", "k", "v", "g", "beta")) + (
+            od.numel() * od.element_size())
+        dgbs = dbytes / (dms / 1e3) / 1e9
+        dec = {"workload": DECODE_WORKLOAD, "ms_per_step": dms, "bytes_per_step": dbytes,
+               "value": world * dgbs, "unit": "GB/s",
+               "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"],
+                            "unit": "GB/s", "frac": dgbs / peaks["hbm_gbs"],
+                            "peak_source": f"{peak_src} (hbm_gbs, copy)"}}
+    clocks = sampler.stop()
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        pin = {n: x[n].pin_memory() for n in ("q", "k", "v", "g", "beta")}
+        h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h_S = torch.empty(S_final.shape, dtype=S_final.dtype).pin_memory()
+        bufs = {n: torch.empty_like(d[n]) for n in pin}
+
+        def e2e_step():
+            for n in pin:
+                bufs[n].copy_(pin[n], non_blocking=True)
+            oo, SS = gdr.chunk_fwd(bufs["q"], bufs["k"], bufs["v"], bufs["g"], bufs["beta"],
+                                   None, None, chunk=w.chunk, read_mode=w.read_mode,
+                                   scale=w.scale, o=o, S_final=S_final, workspace=ws)
+            h_o.copy_(oo, non_blocking=True)
+            h_S.copy_(SS, non_blocking=True)
+
+        n_e2e = max(1, min(args.steps, 5))
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = max_over_ranks(a0.elapsed_time(a1) / n_e2e)
+        e2e = {"value": world * tokens / (ems / 1e3), "unit": "tokens/s", "ms_per_step": ems,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin.values()),
+               "d2h_bytes_per_step": h_o.numel() * h_o.element_size() + h_S.numel() * 4}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "Hk": w.Hk, "Hv": w.Hv, "dk": w.dk,
+                   "dv": w.dv, "chunk": w.chunk, "read_mode": w.read_mode,
+                   "state": "fp32", "path": path,
+                   "l2": "inputs larger than L2 (q,k,v,o 537 MB > 126 MB), no flush",
+                   "parallelism": f"replicas x{world}, no collective"},
+        "tflops": tflops, "pct_bf16_tc_peak": tflops * 1e3 / peaks["bf16_tflops"] * 100,
+        "roofline": {"bound": "hbm", "achieved": hbm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": hbm_gbs / peaks["hbm_gbs"], "traffic": args.traffic,
+                     "algorithmic_bytes": algo_bytes, "flops": flops,
+                     "tensor_frac": tflops * 1e3 / peaks["bf16_tflops"],
+                     "timed": "whole gdr_chunk_fwd call (plan + chunk kernels), CUDA events",
+                     "peak_source": f"{peak_src} (hbm_gbs copy; bf16_tflops burst)"},
+        "decode": dec, "e2e": e2e, "clocks": clocks,
+        "gpu_launches": launches_per_call * args.steps,
+    }
+    return line, x, w
+
+
+def cpu_oracle_sample(x, w, rows=1):
+    """Time the fp64 oracle, as it stands, on `rows` rows of the workload (all heads)."""
+    import oracle
+    sub = {n: (t[:rows] if t is not None else None) for n, t in x.items()
+           if n in ("q", "k", "v", "g", "beta")}
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.forward(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"], None, None,
+                   read_mode=w.read_mode, scale=w.scale)
+    dt = time.perf_counter() - t0
+    tokens = rows * w.T
+    cores = len(os.sched_getaffinity(0))
+    threads = int(os.environ.get("OMP_NUM_THREADS", cores))
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows} of {w.B} rows x {w.T} tokens x {w.Hv} heads of {w.name}, "
+                      f"fp64 per-token recurrence, {dt:.2f} s"}
+
+
+def bench_reference(args, rank, world):
+    """The oracle timed on the host cores: each step a bounded sample of the workload."""
+    import workloads
+    if rank != 0:
+        return None
+    w = workloads.WORKLOADS[args.workload]
+    x = workloads.workload_inputs(w)
+    rows = 1
+    for _ in range(args.warmup):
+        cpu_oracle_sample(x, w, rows)
+    vals, times = [], []
+    for _ in range(args.steps):
+        r = cpu_oracle_sample(x, w, rows)
+        vals.append(r["value"])
+        times.append(rows * w.T / r["value"])
+    value = statistics.median(vals)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(times) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "Hk": w.Hk, "Hv": w.Hv, "dk": w.dk,
+                   "dv": w.dv, "chunk": w.chunk, "read_mode": w.read_mode},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle", "cores": r["cores"],
+                         "sample": r["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=CHUNK_WORKLOAD)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per launch of the dominant kernel from an ncu capture")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = bench_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line, x, w = bench_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_oracle_sample(x, w, rows=1)
+        elif rank == 0:
+            line["cpu_baseline"] = None
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

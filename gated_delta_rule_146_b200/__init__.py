@@ -1,0 +1,147 @@
+"""B200 gated delta-rule library: thin Python binding over the C ABI of libgdr.so.
+
+Every computation runs in the library's CUDA kernels (include/gdr.h).  This
+module only marshals torch CUDA tensors into pointers, allocates the outputs and
+the workspace with torch, and passes the current CUDA stream.  There is no CPU
+fallback: if the compiled library is missing, importing the entry points raises.
+
+Entry points (names follow the C ABI):
+  chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, ...) -> (o, S_final)
+  decode_step(q, k, v, g, beta, S, ...) -> o           (S updated in place)
+  chunk_fwd_workspace_size(...), chunk_fwd_path(...), read_device_error(...)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+from . import _abi
+from ._abi import GdrError, ChunkArgs, DecodeArgs, F32, BF16, READ_POST, READ_PRE  # noqa: F401
+
+__all__ = ["chunk_fwd", "decode_step", "chunk_fwd_workspace_size", "chunk_fwd_path",
+           "read_device_error", "library", "GdrError"]
+
+
+def library():
+    """The loaded libgdr.so (raises if it has not been built)."""
+    return _abi.lib()
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("gdr kernels take CUDA tensors only (there is no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("gdr kernels take contiguous tensors")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_chunk_args(q, v, g, cu_seqlens=None, chunk=64, read_mode="post", scale=None,
+                    qk_l2norm=True, reverse=False, o_accumulate=False):
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    return ChunkArgs(B, T, Hk, Hv, dk, dv, n_seqs, chunk, _dtype_code(q), _dtype_code(g),
+                     READ_PRE if read_mode == "pre" else READ_POST, float(scale),
+                     int(bool(qk_l2norm)), int(bool(reverse)), int(bool(o_accumulate)))
+
+
+def chunk_fwd_workspace_size(args: ChunkArgs) -> int:
+    return int(_abi.lib().gdr_chunk_fwd_workspace_size(ctypes.byref(args)))
+
+
+def chunk_fwd_path(args: ChunkArgs):
+    r = _abi.lib().gdr_chunk_fwd_path(ctypes.byref(args))
+    return None if r is None else r.decode()
+
+
+def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, *, chunk=64, read_mode="post",
+              scale=None, qk_l2norm=True, reverse=False, o=None, o_accumulate=False,
+              output_final_state=True, S_final=None, workspace=None, stream=None):
+    """Chunk-parallel forward (gdr_chunk_fwd).  Shapes: q, k [B,T,Hk,dk]; v [B,T,Hv,dv];
+    g, beta [B,T,Hv]; S0 [n_seqs,Hv,dk,dv] fp32 or None; cu_seqlens int32 [n_seqs+1] or
+    None.  Returns (o [B,T,Hv,dv], S_final [n_seqs,Hv,dk,dv] fp32 or None)."""
+    import torch
+    _check_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_final, workspace)
+    args = make_chunk_args(q, v, g, cu_seqlens, chunk, read_mode, scale, qk_l2norm, reverse,
+                           o_accumulate)
+    if k.dtype != q.dtype or v.dtype != q.dtype or beta.dtype != g.dtype:
+        raise TypeError("q, k, v share one dtype and g, beta another")
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    if S0 is not None and S0.dtype != torch.float32:
+        raise TypeError("S0 must be float32")
+    if o is None:
+        if o_accumulate:
+            raise ValueError("o_accumulate needs an existing o")
+        o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    if S_final is None and output_final_state:
+        S_final = torch.empty((args.n_seqs, args.Hv, args.dk, args.dv), dtype=torch.float32,
+                              device=q.device)
+    need = chunk_fwd_workspace_size(args)
+    if need == 0:
+        raise GdrError(_abi.GDR_ERR_UNSUPPORTED, "no kernel path for these arguments")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = _abi.lib().gdr_chunk_fwd(
+        ctypes.byref(args), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+        _ptr(cu_seqlens), _ptr(o), _ptr(S_final), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
+    _abi.check(st)
+    return o, S_final
+
+
+def read_device_error(args: ChunkArgs, workspace, stream=None) -> int:
+    """Synchronising diagnostic: the device-side status recorded in `workspace`."""
+    return int(_abi.lib().gdr_read_device_error(ctypes.byref(args), _ptr(workspace),
+                                                _stream(stream)))
+
+
+def make_decode_args(q, v, g, read_mode="post", scale=None, qk_l2norm=True):
+    N, Hk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    return DecodeArgs(N, Hk, Hv, dk, dv, _dtype_code(q), _dtype_code(g),
+                      READ_PRE if read_mode == "pre" else READ_POST, float(scale),
+                      int(bool(qk_l2norm)))
+
+
+def decode_step(q, k, v, g, beta, S, *, read_mode="post", scale=None, qk_l2norm=True, o=None,
+                stream=None):
+    """One recurrent token per sequence (gdr_decode_step): q, k [N,Hk,dk]; v [N,Hv,dv];
+    g, beta [N,Hv]; S [N,Hv,dk,dv] fp32, updated in place.  Returns o [N,Hv,dv]."""
+    import torch
+    _check_cuda(q, k, v, g, beta, S, o)
+    if S.dtype != torch.float32:
+        raise TypeError("the state must be float32")
+    args = make_decode_args(q, v, g, read_mode, scale, qk_l2norm)
+    if o is None:
+        o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    st = _abi.lib().gdr_decode_step(ctypes.byref(args), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                    _ptr(beta), _ptr(S), _ptr(o), _stream(stream))
+    _abi.check(st)
+    return o

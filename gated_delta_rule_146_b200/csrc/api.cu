@@ -1,0 +1,148 @@
+// api.cu -- the C ABI declared in include/gdr.h: host-side validation and dispatch.
+//
+// Nothing here allocates device memory, synchronises (except the diagnostic
+// gdr_read_device_error) or keeps state between calls; every entry point only
+// checks its arguments and enqueues kernels on the caller's stream.
+#include <cstring>
+
+#include "common.cuh"
+
+namespace gdr {
+bool tc_supported(const gdr_chunk_args& a);
+gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k, const void* v,
+                           const void* g, const void* beta, const float* S0, void* o,
+                           float* S_final, void* ws, const WsLayout& L, cudaStream_t st);
+}  // namespace gdr
+
+using namespace gdr;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_dtype(gdr_dtype d) { return d == GDR_F32 || d == GDR_BF16; }
+
+// Shape/enum validation shared by workspace_size, path and chunk_fwd.
+gdr_status check_chunk_args(const gdr_chunk_args* a) {
+    if (!a) return GDR_ERR_INVALID_ARG;
+    if (a->B < 1 || a->T < 0 || a->Hk < 1 || a->Hv < 1 || a->Hv % a->Hk != 0)
+        return GDR_ERR_INVALID_ARG;
+    if (a->dk < 1 || a->dv < 1 || a->n_seqs < 1) return GDR_ERR_INVALID_ARG;
+    if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64 && a->chunk != 128)
+        return GDR_ERR_INVALID_ARG;
+    if (!valid_dtype(a->io_dtype) || !valid_dtype(a->gate_dtype)) return GDR_ERR_INVALID_ARG;
+    if (a->read_mode != GDR_READ_POST && a->read_mode != GDR_READ_PRE) return GDR_ERR_INVALID_ARG;
+    if ((a->qk_l2norm | a->reverse | a->o_accumulate) & ~1) return GDR_ERR_INVALID_ARG;
+    const long long T_tot = (long long)a->B * a->T;
+    if (T_tot * a->Hv * (a->dk > a->dv ? a->dk : a->dv) >= (1LL << 40)) return GDR_ERR_INVALID_ARG;
+    if (T_tot > 0x7fffffffLL || (long long)a->n_seqs * a->Hv > 0x7fffffffLL)
+        return GDR_ERR_INVALID_ARG;
+    if (a->Hv > 65535) return GDR_ERR_UNSUPPORTED;
+    return GDR_OK;
+}
+
+enum class Path { None, Tc, Simt };
+
+Path choose_path(const gdr_chunk_args& a) {
+    if (tc_supported(a)) return Path::Tc;
+    if (simt_supported(a)) return Path::Simt;
+    return Path::None;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gdr_chunk_fwd_workspace_size(const gdr_chunk_args* a) {
+    if (check_chunk_args(a) != GDR_OK) return 0;
+    const Path path = choose_path(*a);
+    if (path == Path::None) return 0;
+    return ws_layout(*a, path == Path::Simt).total;
+}
+
+const char* gdr_chunk_fwd_path(const gdr_chunk_args* a) {
+    if (check_chunk_args(a) != GDR_OK) return nullptr;
+    switch (choose_path(*a)) {
+        case Path::Tc: return "tc";
+        case Path::Simt: return "simt";
+        default: return nullptr;
+    }
+}
+
+gdr_status gdr_chunk_fwd(const gdr_chunk_args* a, const void* q, const void* k, const void* v,
+                         const void* g, const void* beta, const float* S0,
+                         const int32_t* cu_seqlens, void* o, float* S_final, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    gdr_status st = check_chunk_args(a);
+    if (st != GDR_OK) return st;
+    if (cu_seqlens) {
+        if (a->B != 1) return GDR_ERR_INVALID_ARG;
+    } else if (a->n_seqs != a->B) {
+        return GDR_ERR_INVALID_ARG;
+    }
+    const bool has_tokens = (long long)a->B * a->T > 0;
+    if (has_tokens && (!q || !k || !v || !g || !beta || !o)) return GDR_ERR_INVALID_ARG;
+    if (!workspace) return GDR_ERR_WORKSPACE;
+    const void* ptrs[] = {q, k, v, g, beta, S0, cu_seqlens, o, S_final, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDR_ERR_ALIGNMENT;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return GDR_ERR_ALIGNMENT;
+    const Path path = choose_path(*a);
+    if (path == Path::None) return GDR_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(*a, path == Path::Simt);
+    if (workspace_bytes < L.total) return GDR_ERR_WORKSPACE;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (launch_plan(*a, cu_seqlens, workspace, L, s) != cudaSuccess) return GDR_ERR_CUDA;
+    if (path == Path::Tc)
+        return launch_chunk_tc(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s);
+    return launch_chunk_simt(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s);
+}
+
+gdr_status gdr_decode_step(const gdr_decode_args* a, const void* q, const void* k, const void* v,
+                           const void* g, const void* beta, float* S_inout, void* o,
+                           void* stream) {
+    if (!a) return GDR_ERR_INVALID_ARG;
+    if (a->N < 0 || a->Hk < 1 || a->Hv < 1 || a->Hv % a->Hk != 0 || a->dk < 1 || a->dv < 1)
+        return GDR_ERR_INVALID_ARG;
+    if (!valid_dtype(a->io_dtype) || !valid_dtype(a->gate_dtype)) return GDR_ERR_INVALID_ARG;
+    if (a->read_mode != GDR_READ_POST && a->read_mode != GDR_READ_PRE) return GDR_ERR_INVALID_ARG;
+    if (a->qk_l2norm & ~1) return GDR_ERR_INVALID_ARG;
+    if ((long long)a->N * a->Hv > 0x7fffffffLL) return GDR_ERR_INVALID_ARG;
+    if (!decode_supported(*a)) return GDR_ERR_UNSUPPORTED;
+    if (a->N == 0) return GDR_OK;
+    if (!q || !k || !v || !g || !beta || !S_inout || !o) return GDR_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, beta, S_inout, o};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return GDR_ERR_ALIGNMENT;
+    return launch_decode(*a, q, k, v, g, beta, S_inout, o, static_cast<cudaStream_t>(stream));
+}
+
+const char* gdr_status_string(gdr_status s) {
+    switch (s) {
+        case GDR_OK: return "GDR_OK";
+        case GDR_ERR_INVALID_ARG: return "GDR_ERR_INVALID_ARG: invalid argument";
+        case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED: no kernel for these sizes/dtypes";
+        case GDR_ERR_ALIGNMENT: return "GDR_ERR_ALIGNMENT: pointer not 16-byte aligned";
+        case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE: workspace missing or too small";
+        case GDR_ERR_CUDA: return "GDR_ERR_CUDA: kernel launch failed";
+        case GDR_ERR_DEVICE_CHECK: return "GDR_ERR_DEVICE_CHECK: device-side check failed (cu_seqlens)";
+        case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT: a bounded device wait gave up";
+    }
+    return "unknown gdr_status";
+}
+
+gdr_status gdr_read_device_error(const gdr_chunk_args* a, const void* workspace, void* stream) {
+    (void)a;
+    if (!workspace) return GDR_ERR_INVALID_ARG;
+    int err = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&err, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GDR_ERR_CUDA;
+    return static_cast<gdr_status>(err);
+}
+
+const char* gdr_version(void) { return "gdr-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+// common.cuh -- device helpers and the workspace layout shared by the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdr.h"
+
+namespace gdr {
+
+constexpr float kNormEps = 1e-6f;  // x / max(||x||, eps), as F.normalize(eps=1e-6)
+
+// ---- element access ---------------------------------------------------------
+
+__device__ __forceinline__ float load_elem(const void* p, size_t i, gdr_dtype dt) {
+    return dt == GDR_BF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i])
+                          : static_cast<const float*>(p)[i];
+}
+
+__device__ __forceinline__ void store_elem(void* p, size_t i, float x, gdr_dtype dt) {
+    if (dt == GDR_BF16) static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(x);
+    else static_cast<float*>(p)[i] = x;
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// ---- workspace ----------------------------------------------------------------
+//
+// [header 256 B][cu (n_seqs+1) int32][chunk_off (n_seqs+1) int32][chunk_seq (max_chunks)
+// int32][fp32 W [T_tot][Hv][dk]][fp32 U [T_tot][Hv][dv]][fp32 G [T_tot][Hv]]
+// The three fp32 arrays exist only for the CUDA-core (SIMT) path.
+
+struct WsHeader {
+    int err;           // gdr_status recorded by a device-side check
+    int n_chunks;      // total chunks over all sequences
+    int pad[62];
+};
+
+struct WsLayout {
+    size_t cu, chunk_off, chunk_seq, W, U, G, total;
+    long long max_chunks;
+};
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline WsLayout ws_layout(const gdr_chunk_args& a, bool simt) {
+    WsLayout L{};
+    const long long T_tot = (long long)a.B * a.T;
+    L.max_chunks = (T_tot + a.chunk - 1) / a.chunk + a.n_seqs;
+    size_t off = sizeof(WsHeader);
+    L.cu = off;        off = align_up(off + sizeof(int32_t) * (a.n_seqs + 1), 256);
+    L.chunk_off = off; off = align_up(off + sizeof(int32_t) * (a.n_seqs + 1), 256);
+    L.chunk_seq = off; off = align_up(off + sizeof(int32_t) * (size_t)L.max_chunks, 256);
+    if (simt) {
+        L.W = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv * a.dk, 256);
+        L.U = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv * a.dv, 256);
+        L.G = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv, 256);
+    }
+    L.total = off;
+    return L;
+}
+
+// Device view of the chunk map built by plan_kernel.
+struct ChunkMap {
+    const WsHeader* hdr;
+    const int32_t* cu;         // [n_seqs+1] token offsets (validated)
+    const int32_t* chunk_off;  // [n_seqs+1] first global chunk of each sequence
+    const int32_t* chunk_seq;  // [max_chunks] sequence of each global chunk
+};
+
+// Physical token index of logical position p of a sequence spanning [t0, t1).
+__device__ __forceinline__ long long phys_token(long long t0, long long t1, int p, int reverse) {
+    return reverse ? (t1 - 1 - p) : (t0 + p);
+}
+
+}  // namespace gdr
+
+// Launchers implemented in the .cu files (host side).
+namespace gdr {
+cudaError_t launch_plan(const gdr_chunk_args& a, const int32_t* cu_in, void* ws, const WsLayout& L,
+                        cudaStream_t st);
+gdr_status launch_chunk_simt(const gdr_chunk_args& a, const void* q, const void* k,
+                             const void* v, const void* g, const void* beta, const float* S0,
+                             void* o, float* S_final, void* ws, const WsLayout& L,
+                             cudaStream_t st);
+bool simt_supported(const gdr_chunk_args& a);
+gdr_status launch_decode(const gdr_decode_args& a, const void* q, const void* k, const void* v,
+                         const void* g, const void* beta, float* S, void* o, cudaStream_t st);
+bool decode_supported(const gdr_decode_args& a);
+}  // namespace gdr

@@ -1,0 +1,181 @@
+// decode.cu -- one-token recurrent decode step, streaming the fp32 state once.
+//
+// Per (sequence n, value head h) and token (flashrt fused_layer.py `_decode_one`:
+// the recurrent core reads the cached state and writes the new one each token;
+// tiny_gdn/fugue.py `fused_recurrent_gdn2_fwd` call with an initial state):
+//     s_k = H^T k,  s_q = H^T q
+//     u   = beta (v - alpha s_k)
+//     H  <- alpha H + k u^T                         (in place)
+//     post: o = scale (alpha s_q + (k.q) u)   [= scale H_new^T q]
+//     pre:  o = scale s_q
+// The columns of H (dv) are independent, so a block owns a slice of DVS columns
+// and every row of it: it loads the whole slice into registers with 16-byte
+// streaming loads, reduces s_k and s_q over the dk rows (warp shuffles, then
+// shared memory across warps), and writes the updated slice back from the same
+// registers.  Each block reads all of its slice before writing any of it, so the
+// update in place needs no scratch copy of the state.
+#include "common.cuh"
+
+namespace gdr {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+struct DecodeParams {
+    const void* q; const void* k; const void* v; const void* g; const void* beta;
+    float* S; void* o;
+    int Hk, Hv, read_pre, qk_l2norm;
+    gdr_dtype io, gt;
+    float scale;
+};
+
+template <int DK, int DV, int DVS>
+__global__ void __launch_bounds__(kThreads)
+decode_kernel(DecodeParams p) {
+    constexpr int CPR = DVS / 4;           // float4 column groups per row slice
+    constexpr int RPW = 32 / CPR;          // rows a warp covers per pass
+    constexpr int RPP = RPW * kWarps;      // rows per pass over the block
+    constexpr int NP = DK / RPP;           // passes (float4 registers per thread)
+    static_assert(DK % RPP == 0, "dk must be a multiple of the rows per pass");
+
+    __shared__ float s_q[DK], s_k[DK];
+    __shared__ float s_red[2][kWarps][DVS];
+    __shared__ float s_u[DVS];
+    __shared__ float s_alpha, s_beta;
+
+    const int nh = blockIdx.x;                   // n * Hv + h
+    const int J = blockIdx.y;                    // column slice
+    const int n = nh / p.Hv, h = nh % p.Hv, hk = h / (p.Hv / p.Hk);
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int cg = lane % CPR, rw = lane / CPR;  // float4 column group, row within warp pass
+
+    // issue the state loads first: they are the whole cost of the kernel
+    float* Sblk = p.S + (size_t)nh * DK * DV + J * DVS + cg * 4;
+    float4 hreg[NP];
+#pragma unroll
+    for (int m = 0; m < NP; ++m) {
+        const int d = m * RPP + wid * RPW + rw;
+        hreg[m] = __ldcs(reinterpret_cast<const float4*>(Sblk + (size_t)d * DV));
+    }
+
+    // q, k (normalised), gates
+    const size_t qk_base = ((size_t)n * p.Hk + hk) * DK;
+    for (int d = tid; d < DK; d += kThreads) {
+        s_q[d] = load_elem(p.q, qk_base + d, p.io);
+        s_k[d] = load_elem(p.k, qk_base + d, p.io);
+    }
+    if (tid == 0) {
+        s_alpha = expf(load_elem(p.g, (size_t)nh, p.gt));
+        s_beta = load_elem(p.beta, (size_t)nh, p.gt);
+    }
+    __syncthreads();
+    if (wid < 3) {
+        // warp 0: ||q||, warp 1: ||k||, warp 2: raw k.q
+        float acc = 0.f;
+        for (int d = lane; d < DK; d += 32)
+            acc += wid == 0 ? s_q[d] * s_q[d] : (wid == 1 ? s_k[d] * s_k[d] : s_q[d] * s_k[d]);
+        acc = warp_sum(acc);
+        if (lane == 0) s_red[0][wid][0] = acc;
+    }
+    __syncthreads();
+    float inv_q = 1.f, inv_k = 1.f;
+    if (p.qk_l2norm) {
+        inv_q = 1.f / fmaxf(sqrtf(s_red[0][0][0]), kNormEps);
+        inv_k = 1.f / fmaxf(sqrtf(s_red[0][1][0]), kNormEps);
+    }
+    const float kq = s_red[0][2][0] * inv_q * inv_k;
+    __syncthreads();
+
+    // partial s_k, s_q over this thread's rows, 4 columns
+    float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sq = sk;
+    float kr[NP];
+#pragma unroll
+    for (int m = 0; m < NP; ++m) {
+        const int d = m * RPP + wid * RPW + rw;
+        const float kd = s_k[d] * inv_k, qd = s_q[d] * inv_q;
+        kr[m] = kd;
+        sk.x = fmaf(hreg[m].x, kd, sk.x); sk.y = fmaf(hreg[m].y, kd, sk.y);
+        sk.z = fmaf(hreg[m].z, kd, sk.z); sk.w = fmaf(hreg[m].w, kd, sk.w);
+        sq.x = fmaf(hreg[m].x, qd, sq.x); sq.y = fmaf(hreg[m].y, qd, sq.y);
+        sq.z = fmaf(hreg[m].z, qd, sq.z); sq.w = fmaf(hreg[m].w, qd, sq.w);
+    }
+    // reduce over the rows held by this warp (lanes sharing a column group)
+#pragma unroll
+    for (int o = CPR; o < 32; o <<= 1) {
+        sk.x += __shfl_xor_sync(0xffffffffu, sk.x, o); sk.y += __shfl_xor_sync(0xffffffffu, sk.y, o);
+        sk.z += __shfl_xor_sync(0xffffffffu, sk.z, o); sk.w += __shfl_xor_sync(0xffffffffu, sk.w, o);
+        sq.x += __shfl_xor_sync(0xffffffffu, sq.x, o); sq.y += __shfl_xor_sync(0xffffffffu, sq.y, o);
+        sq.z += __shfl_xor_sync(0xffffffffu, sq.z, o); sq.w += __shfl_xor_sync(0xffffffffu, sq.w, o);
+    }
+    if (rw == 0) {
+        s_red[0][wid][cg * 4 + 0] = sk.x; s_red[0][wid][cg * 4 + 1] = sk.y;
+        s_red[0][wid][cg * 4 + 2] = sk.z; s_red[0][wid][cg * 4 + 3] = sk.w;
+        s_red[1][wid][cg * 4 + 0] = sq.x; s_red[1][wid][cg * 4 + 1] = sq.y;
+        s_red[1][wid][cg * 4 + 2] = sq.z; s_red[1][wid][cg * 4 + 3] = sq.w;
+    }
+    __syncthreads();
+    const float alpha = s_alpha, beta = s_beta;
+    if (tid < DVS) {
+        float tk = 0.f, tq = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) { tk += s_red[0][w][tid]; tq += s_red[1][w][tid]; }
+        const int col = J * DVS + tid;
+        const float vj = load_elem(p.v, (size_t)nh * DV + col, p.io);
+        const float u = beta * (vj - alpha * tk);
+        s_u[tid] = u;
+        const float oj = p.read_pre ? p.scale * tq : p.scale * fmaf(alpha, tq, kq * u);
+        store_elem(p.o, (size_t)nh * DV + col, oj, p.io);
+    }
+    __syncthreads();
+    const float4 u4 = *reinterpret_cast<const float4*>(&s_u[cg * 4]);
+#pragma unroll
+    for (int m = 0; m < NP; ++m) {
+        const int d = m * RPP + wid * RPW + rw;
+        float4 r;
+        r.x = fmaf(alpha, hreg[m].x, kr[m] * u4.x); r.y = fmaf(alpha, hreg[m].y, kr[m] * u4.y);
+        r.z = fmaf(alpha, hreg[m].z, kr[m] * u4.z); r.w = fmaf(alpha, hreg[m].w, kr[m] * u4.w);
+        __stcs(reinterpret_cast<float4*>(Sblk + (size_t)d * DV), r);
+    }
+}
+
+template <int DK, int DV>
+gdr_status launch_dv(const gdr_decode_args& a, const DecodeParams& p, cudaStream_t st) {
+    constexpr int DVS = DV >= 64 ? 64 : 32;
+    dim3 grid((unsigned)(a.N * a.Hv), DV / DVS);
+    decode_kernel<DK, DV, DVS><<<grid, kThreads, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+template <int DK>
+gdr_status launch_dk(const gdr_decode_args& a, const DecodeParams& p, cudaStream_t st) {
+    switch (a.dv) {
+        case 32: return launch_dv<DK, 32>(a, p, st);
+        case 64: return launch_dv<DK, 64>(a, p, st);
+        case 128: return launch_dv<DK, 128>(a, p, st);
+        default: return GDR_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace
+
+bool decode_supported(const gdr_decode_args& a) {
+    return (a.dk == 32 || a.dk == 64 || a.dk == 128) && (a.dv == 32 || a.dv == 64 || a.dv == 128);
+}
+
+gdr_status launch_decode(const gdr_decode_args& a, const void* q, const void* k, const void* v,
+                         const void* g, const void* beta, float* S, void* o, cudaStream_t st) {
+    DecodeParams p;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.S = S; p.o = o;
+    p.Hk = a.Hk; p.Hv = a.Hv; p.read_pre = a.read_mode == GDR_READ_PRE;
+    p.qk_l2norm = a.qk_l2norm; p.io = a.io_dtype; p.gt = a.gate_dtype; p.scale = a.scale;
+    switch (a.dk) {
+        case 32: return launch_dk<32>(a, p, st);
+        case 64: return launch_dk<64>(a, p, st);
+        case 128: return launch_dk<128>(a, p, st);
+        default: return GDR_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace gdr

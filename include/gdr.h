@@ -1,0 +1,170 @@
+/*
+ * gdr.h -- C ABI of the B200 gated delta-rule library (libgdr.so).
+ *
+ * The recurrence, per (sequence n, value head h), with the state held
+ * transposed as H = S^T of shape [dk][dv] (dv contiguous):
+ *
+ *     u_t = beta_t (v_t - alpha_t H_{t-1}^T k_t)
+ *     H_t = alpha_t H_{t-1} + k_t u_t^T,            alpha_t = exp(g_t)
+ *     post-write read  o_t = scale * H_t^T q_t
+ *     pre-write read   o_t = scale * H_{t-1}^T q_t
+ *
+ * (Prizma "seq/delta.py", module docstring: S_t = alpha_t S_{t-1} + u_t k_t^T
+ * with u_t = beta_t (v_t - alpha_t S_{t-1} k_t) and the strictly causal read
+ * o_t = S_{t-1} q_t; sparse_delta_memory/layer.py, SparseDeltaMemory docstring:
+ * memory *= exp(g), memory += beta k (v - memory k)^T; tiny_gdn/fugue.py,
+ * BidirectionalGatedDeltaNet2 docstring: the forward read q_t^T S_t.)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every tensor argument is a DEVICE pointer owned by the caller.  The
+ *   library never allocates, frees or synchronises; every call only enqueues
+ *   kernels on `stream` (a cudaStream_t passed as void*; NULL = legacy default
+ *   stream) and returns.  Calls hold no host state between them.
+ * - All tensors are dense and row-major in the index order given.  Pointers
+ *   must be 16-byte aligned (GDR_ERR_ALIGNMENT otherwise).
+ * - Arguments are validated on the host before anything is enqueued; a call
+ *   that returns anything but GDR_OK has enqueued nothing (except
+ *   GDR_ERR_CUDA, returned when a launch itself fails).
+ * - Inconsistencies only visible on the device (a cu_seqlens array that is not
+ *   non-decreasing, does not start at 0 or does not end at T) are recorded in
+ *   an error word inside the workspace; the kernels then skip the work.  Read
+ *   it with gdr_read_device_error.  No kernel traps or waits without a bound.
+ */
+#ifndef GDR_H
+#define GDR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDR_OK = 0,
+    GDR_ERR_INVALID_ARG = 1,   /* null pointer, bad size, Hv % Hk != 0, bad enum ... */
+    GDR_ERR_UNSUPPORTED = 2,   /* valid, but no kernel for this (dk, dv, chunk, dtype) */
+    GDR_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
+    GDR_ERR_WORKSPACE = 4,     /* workspace missing or smaller than the required size */
+    GDR_ERR_CUDA = 5,          /* a CUDA launch failed (cudaGetLastError after launch) */
+    GDR_ERR_DEVICE_CHECK = 6,  /* device-side check failed (bad cu_seqlens) */
+    GDR_ERR_TIMEOUT = 7        /* a bounded device-side wait gave up */
+} gdr_status;
+
+typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
+
+/* Read mode.  POST: o_t = scale * S_t q_t (tiny_gdn/fugue.py forward scan,
+ * q_t^T S_t).  PRE: o_t = scale * S_{t-1} q_t (Prizma "seq/delta.py", the
+ * strictly causal pre-write read). */
+typedef enum { GDR_READ_POST = 0, GDR_READ_PRE = 1 } gdr_read_mode;
+
+/*
+ * Arguments of the chunk-parallel forward (training / prefill).
+ *
+ * The forward is evaluated in the exact chunk-wise WY/UT form (Prizma
+ * "seq/delta.py", chunked_delta: per chunk a unit-lower-triangular solve
+ * (I + A) U = ..., then the chunk-to-chunk state carry;
+ * sparse_delta_memory/layer.py module docstring: the chunk size changes the
+ * result only through floating-point rounding).
+ */
+typedef struct {
+    int B;                 /* rows; with cu_seqlens B must be 1 */
+    int T;                 /* tokens per row (with cu_seqlens: total packed tokens) */
+    int Hk, Hv;            /* key/query heads and value heads, Hv % Hk == 0; value head h
+                              reads key head h / (Hv / Hk)  (tiny_gdn/fugue.py `heads`) */
+    int dk, dv;            /* head dims; GPU kernels: dk, dv in {32, 64, 128} */
+    int n_seqs;            /* == B without cu_seqlens, else number of packed sequences */
+    int chunk;             /* 16, 32, 64 or 128 (64: the contract of flashrt fused_layer.py
+                              `_prefill_chain`); chunks restart at every sequence start */
+    gdr_dtype io_dtype;    /* dtype of q, k, v and o */
+    gdr_dtype gate_dtype;  /* dtype of g and beta */
+    gdr_read_mode read_mode;
+    float scale;           /* multiplies the read in both modes */
+    int qk_l2norm;         /* 1: q, k <- x / max(||x||_2, 1e-6) in fp32 inside the kernels
+                              (use_qk_l2norm_in_kernel of tiny_gdn/fugue.py `scan`) */
+    int reverse;           /* 1: scan every sequence from its last token to its first, in
+                              place (tiny_gdn/fugue.py `scan`, direction 1); o is written at
+                              each token's own position, S_final is the state after the
+                              sequence's FIRST token */
+    int o_accumulate;      /* 1: o += result (o is read, the sum written back in io_dtype);
+                              0: o = result */
+} gdr_chunk_args;
+
+/* Bytes of device workspace gdr_chunk_fwd needs for these arguments (0 on invalid
+ * arguments).  Depends on B, T, Hv, dk, dv, n_seqs, chunk and the dtypes only. */
+size_t gdr_chunk_fwd_workspace_size(const gdr_chunk_args* args);
+
+/*
+ * Chunk-parallel forward over every sequence and value head.
+ *
+ *   q, k        [B, T, Hk, dk]   io_dtype
+ *   v           [B, T, Hv, dv]   io_dtype
+ *   g, beta     [B, T, Hv]       gate_dtype; g = log(alpha) (<= 0 for a decay), beta
+ *                                 unrestricted (beta in (0, 2) gives negative
+ *                                 eigenvalues, tiny_gdn/fugue.py `project`)
+ *   S0          [n_seqs, Hv, dk, dv] fp32 initial state, or NULL for zero
+ *   cu_seqlens  [n_seqs + 1] int32 device offsets into the packed row (B == 1), or
+ *               NULL for B rows of T tokens (tiny_gdn/fugue.py `segment_layout`)
+ *   o           [B, T, Hv, dv]   io_dtype output (rounded to nearest even for bf16)
+ *   S_final     [n_seqs, Hv, dk, dv] fp32 final state, or NULL; may alias S0
+ *               (each state is read completely before its final value is written)
+ *   workspace   device scratch of at least gdr_chunk_fwd_workspace_size(args) bytes,
+ *               256-byte aligned; its contents need no initialisation
+ *
+ * Empty sequences are allowed (their S_final is S0, or zero).
+ */
+gdr_status gdr_chunk_fwd(const gdr_chunk_args* args,
+                         const void* q, const void* k, const void* v,
+                         const void* g, const void* beta,
+                         const float* S0, const int32_t* cu_seqlens,
+                         void* o, float* S_final,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Name of the kernel path gdr_chunk_fwd takes for these arguments: "tc" (tcgen05
+ * tensor-core kernels), "simt" (fp32 CUDA-core kernels) or NULL if unsupported. */
+const char* gdr_chunk_fwd_path(const gdr_chunk_args* args);
+
+/*
+ * One-token recurrent decode step (flashrt fused_layer.py `_decode_one`, the
+ * recurrent core that reads and writes the cached state once per token).
+ */
+typedef struct {
+    int N;                 /* independent sequences, one token each */
+    int Hk, Hv, dk, dv;    /* as in gdr_chunk_args; GPU kernel: dk in {32,64,128},
+                              dv a multiple of 32 up to 128 */
+    gdr_dtype io_dtype, gate_dtype;
+    gdr_read_mode read_mode;
+    float scale;
+    int qk_l2norm;
+} gdr_decode_args;
+
+/*
+ *   q, k     [N, Hk, dk]  io_dtype      v, o  [N, Hv, dv]  io_dtype
+ *   g, beta  [N, Hv]      gate_dtype
+ *   S_inout  [N, Hv, dk, dv] fp32, updated in place: every block reads its whole slice
+ *            of the state into registers before it writes any of it back, so no scratch
+ *            state is needed.
+ */
+gdr_status gdr_decode_step(const gdr_decode_args* args,
+                           const void* q, const void* k, const void* v,
+                           const void* g, const void* beta,
+                           float* S_inout, void* o, void* stream);
+
+/* Human-readable name of a status. */
+const char* gdr_status_string(gdr_status status);
+
+/* Test/diagnostic helper, NOT for the hot path: copies the device error word out of a
+ * workspace last used by gdr_chunk_fwd with `args`, SYNCHRONISES `stream`, and returns
+ * GDR_OK or the recorded device-side status. */
+gdr_status gdr_read_device_error(const gdr_chunk_args* args, const void* workspace,
+                                 void* stream);
+
+/* Library version string (also names the target architecture). */
+const char* gdr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H */

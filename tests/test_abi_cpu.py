@@ -1,0 +1,101 @@
+"""The C-ABI library loads, exports what include/gdr.h declares, and validates its
+arguments on the host (no GPU needed: every call here is refused before any launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_146_b200 import _abi, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "gdr.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdr_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) == set(_abi.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert b"sm_100a" in lib.gdr_version()
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert lib.gdr_status_string(s).startswith(b"GDR_")
+
+
+def args(**kw):
+    base = dict(B=2, T=100, Hk=2, Hv=4, dk=64, dv=64, n_seqs=2, chunk=64, io_dtype=_abi.BF16,
+                gate_dtype=_abi.BF16, read_mode=_abi.READ_POST, scale=0.125, qk_l2norm=1,
+                reverse=0, o_accumulate=0)
+    base.update(kw)
+    return _abi.ChunkArgs(**base)
+
+
+def test_workspace_size(lib):
+    a = args()
+    n = lib.gdr_chunk_fwd_workspace_size(ctypes.byref(a))
+    assert n > 0 and n % 256 == 0
+    assert lib.gdr_chunk_fwd_workspace_size(ctypes.byref(args(Hv=3))) == 0
+    assert lib.gdr_chunk_fwd_workspace_size(ctypes.byref(args(chunk=48))) == 0
+    assert lib.gdr_chunk_fwd_path(ctypes.byref(args(dk=100))) in (b"simt", None)
+
+
+FAKE = 0x10000  # a well-aligned address that is never dereferenced: every call below is
+                # refused by host validation before anything is enqueued
+
+
+def call(lib, a, **ptrs):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, S0=None, cu=None, o=FAKE,
+             S_final=FAKE, ws=FAKE)
+    p.update(ptrs)
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdr_chunk_fwd(ctypes.byref(a), vp(p["q"]), vp(p["k"]), vp(p["v"]), vp(p["g"]),
+                             vp(p["beta"]), vp(p["S0"]), vp(p["cu"]), vp(p["o"]),
+                             vp(p["S_final"]), vp(p["ws"]), ctypes.c_size_t(p.get("wsb", 0)),
+                             None)
+
+
+def test_host_validation(lib):
+    a = args()
+    need = lib.gdr_chunk_fwd_workspace_size(ctypes.byref(a))
+    assert call(lib, args(Hv=3)) == _abi.GDR_ERR_INVALID_ARG
+    assert call(lib, args(chunk=8)) == _abi.GDR_ERR_INVALID_ARG
+    assert call(lib, args(io_dtype=7)) == _abi.GDR_ERR_INVALID_ARG
+    assert call(lib, args(read_mode=2)) == _abi.GDR_ERR_INVALID_ARG
+    assert call(lib, a, q=None, wsb=need) == _abi.GDR_ERR_INVALID_ARG
+    assert call(lib, args(n_seqs=3), wsb=need) == _abi.GDR_ERR_INVALID_ARG  # n_seqs != B
+    assert call(lib, a, cu=FAKE, wsb=need) == _abi.GDR_ERR_INVALID_ARG      # varlen needs B=1
+    assert call(lib, a, k=FAKE + 4, wsb=need) == _abi.GDR_ERR_ALIGNMENT
+    assert call(lib, a, ws=FAKE + 16, wsb=need) == _abi.GDR_ERR_ALIGNMENT   # workspace 256 B
+    assert call(lib, a, ws=None, wsb=need) == _abi.GDR_ERR_WORKSPACE
+    assert call(lib, a, wsb=need - 1) == _abi.GDR_ERR_WORKSPACE
+
+
+def test_decode_host_validation(lib):
+    d = _abi.DecodeArgs(N=4, Hk=2, Hv=4, dk=128, dv=128, io_dtype=_abi.BF16,
+                        gate_dtype=_abi.BF16, read_mode=_abi.READ_POST, scale=0.1, qk_l2norm=1)
+    vp = ctypes.c_void_p
+    f = lambda a, **kw: lib.gdr_decode_step(ctypes.byref(a), *[vp(kw.get(n, FAKE)) for n in
+                                                              ("q", "k", "v", "g", "b", "S", "o")],
+                                            None)
+    bad = _abi.DecodeArgs(**{**{n: getattr(d, n) for n, _ in d._fields_}, "Hv": 5})
+    assert f(bad) == _abi.GDR_ERR_INVALID_ARG
+    unsup = _abi.DecodeArgs(**{**{n: getattr(d, n) for n, _ in d._fields_}, "dk": 96})
+    assert f(unsup) == _abi.GDR_ERR_UNSUPPORTED
+    assert f(d, S=FAKE + 8) == _abi.GDR_ERR_ALIGNMENT
+    empty = _abi.DecodeArgs(**{**{n: getattr(d, n) for n, _ in d._fields_}, "N": 0})
+    assert f(empty) == _abi.GDR_OK  # nothing to do, nothing launched
