@@ -10,6 +10,7 @@ LIB_PATH = os.path.join(_HERE, "libgdr.so")
 
 GDR_OK, GDR_ERR_INVALID_ARG, GDR_ERR_UNSUPPORTED, GDR_ERR_ALIGNMENT = 0, 1, 2, 3
 GDR_ERR_WORKSPACE, GDR_ERR_CUDA, GDR_ERR_DEVICE_CHECK, GDR_ERR_TIMEOUT = 4, 5, 6, 7
+GDR_ERR_RANGE = 8
 F32, BF16 = 0, 1
 READ_POST, READ_PRE = 0, 1
 

@@ -128,6 +128,7 @@ const char* gdr_status_string(gdr_status s) {
         case GDR_ERR_CUDA: return "GDR_ERR_CUDA: kernel launch failed";
         case GDR_ERR_DEVICE_CHECK: return "GDR_ERR_DEVICE_CHECK: device-side check failed (cu_seqlens)";
         case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT: a bounded device wait gave up";
+        case GDR_ERR_RANGE: return "GDR_ERR_RANGE: a tensor-core operand left the fp16 range";
     }
     return "unknown gdr_status";
 }

@@ -20,11 +20,17 @@
 // dimension (128): accumulators hold rows of W^T, U~^T, V'^T, O^T and H^T, one TMEM lane
 // per dk or dv index, one column per token (or per dk for the state).  Every MMA is then
 // M=128, N=64 or 128, and every TMEM->shared epilogue writes whole 128-byte rows.  A and
-// B operands are bf16 in shared memory in the 128-byte-swizzled canonical layouts
+// B operands are 16-bit in shared memory in the 128-byte-swizzled canonical layouts
 // (K-major or MN-major as each product needs); accumulation and the state are fp32.
 //
+// Operand precision: V and T diag(beta) are bf16 (V arrives in bf16); every other operand
+// (normalised q and k, T diag(beta e^G), W, the state copy, V', P) is rounded to fp16,
+// whose 11-bit significand keeps the chain of roundings well inside the bf16 parity bound
+// at long sequence lengths where bf16 operands do not.  The fp16 range is checked wherever
+// an operand is produced; a value beyond it sets GDR_ERR_RANGE.
+//
 // The state H is kept transposed in TMEM (lane = dv, column = dk).  After each chunk the
-// epilogue reads it once, writes the bf16 copy the next chunk's MMAs consume, and scales
+// epilogue reads it once, writes the fp16 copy the next chunk's MMAs consume, and scales
 // it in place by the next chunk's total decay, so the next state update accumulates onto
 // it directly.
 #include "common.cuh"
@@ -46,14 +52,14 @@ constexpr uint32_t OFF_KQ0 = 0;        // 2 x 16 KB atoms (dk halves): K rows 0-
 constexpr uint32_t OFF_KQ1 = 32768;    // second buffer (next chunk)
 constexpr uint32_t OFF_V0 = 65536;     // 2 x 8 KB (dv halves): V rows 0-63
 constexpr uint32_t OFF_V1 = 81920;
-constexpr uint32_t OFF_TW = 98304;     // T diag(beta e^G), [i][j] bf16
+constexpr uint32_t OFF_TW = 98304;     // T diag(beta e^G), [i][j] fp16
 constexpr uint32_t OFF_TU = 106496;    // T diag(beta), [i][j] bf16
 constexpr uint32_t OFF_OS = 98304;     // output staging [tok][dv] bf16 (aliases TW, TU)
-constexpr uint32_t OFF_P = 114688;     // P [i][j] bf16
-constexpr uint32_t OFF_WN = 122880;    // -W^T as [dk][tok] bf16
+constexpr uint32_t OFF_P = 114688;     // P [i][j] fp16
+constexpr uint32_t OFF_WN = 122880;    // -W^T as [dk][tok] fp16
 constexpr uint32_t OFF_AS = 122880;    // A fp32 [64][64] (aliases WN; dead before WN is written)
-constexpr uint32_t OFF_HB = 139264;    // H^T bf16 [dv][dk], 2 x 16 KB atoms (dk halves)
-constexpr uint32_t OFF_VP = 172032;    // V'^T bf16 [dv][tok]
+constexpr uint32_t OFF_HB = 139264;    // H^T fp16 [dv][dk], 2 x 16 KB atoms (dk halves)
+constexpr uint32_t OFF_VP = 172032;    // V'^T fp16 [dv][tok]
 constexpr uint32_t OFF_SMALL = 188416;
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + 2048 + 1024;
 
@@ -82,12 +88,26 @@ struct TcParams {
     float scale;
 };
 
-__device__ __forceinline__ uint4 scale_bf16x8(uint4 u, float f) {
+constexpr float kF16Max = 65000.f;  // operands at or beyond this (or NaN) raise GDR_ERR_RANGE
+
+// fp16 pair with a range check: `bad` is set when either value is not finite or too large
+__device__ __forceinline__ uint32_t h2(float a, float b, bool& bad) {
+    bad |= !(fabsf(a) < kF16Max) || !(fabsf(b) < kF16Max);
+    return pack_f16x2(a, b);
+}
+
+__device__ __forceinline__ uint4 h8(const float* f, bool& bad) {
+    return make_uint4(h2(f[0], f[1], bad), h2(f[2], f[3], bad), h2(f[4], f[5], bad),
+                      h2(f[6], f[7], bad));
+}
+
+// 8 fp16 scaled by f (|f| <= 1 at every call site, so the range cannot grow)
+__device__ __forceinline__ uint4 scale_f16x8(uint4 u, float f) {
     uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        const float2 x = unpack_bf16x2(w[e]);
-        w[e] = pack_bf16x2(x.x * f, x.y * f);
+        const float2 x = unpack_f16x2(w[e]);
+        w[e] = pack_f16x2(x.x * f, x.y * f);
     }
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
@@ -170,7 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
         return all != 0;
     };
 
-    // ---- prologue: chunk 0 in flight, initial state into TMEM (pre-scaled) and bf16 copy
+    // ---- prologue: chunk 0 in flight, initial state into TMEM (pre-scaled) and fp16 copy
+    bool bad = false;  // an fp16 operand out of range
     float g_nx, b_nx;
     load_chunk(0, 0);
     cp_async_commit();
@@ -197,8 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                 }
                 const int cd = (d0 >> 3) + e8;
                 *reinterpret_cast<uint4*>(sm + OFF_HB + (cd >> 3) * 16384 + sw128(j, cd & 7)) =
-                    make_uint4(pack_bf16x2(hv[0], hv[1]), pack_bf16x2(hv[2], hv[3]),
-                               pack_bf16x2(hv[4], hv[5]), pack_bf16x2(hv[6], hv[7]));
+                    h8(hv, bad);
             }
             tmem_st32(tlane + TM_HM + d0, r);
         }
@@ -222,8 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
         fence_proxy_async_smem();
         __syncthreads();
 
-        // ---- A: L2-normalise the 128 rows of [K; Q] in place; in-chunk cumsum of g
-        if (p.qk_l2norm) {
+        // ---- A: the 128 rows of [K; Q]: bf16 -> (L2-normalised) fp16 in place; cumsum of g
+        {
             uint4 vals[16];
             float ss = 0.f;
 #pragma unroll
@@ -237,11 +257,20 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                     ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
                 }
             }
-            const float inv = 1.f / fmaxf(sqrtf(ss), kNormEps);
+            const float inv = p.qk_l2norm ? 1.f / fmaxf(sqrtf(ss), kNormEps) : 1.f;
 #pragma unroll
-            for (int cd = 0; cd < 16; ++cd)
+            for (int cd = 0; cd < 16; ++cd) {
+                const uint32_t w[4] = {vals[cd].x, vals[cd].y, vals[cd].z, vals[cd].w};
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 x = unpack_bf16x2(w[e]);
+                    f[2 * e] = x.x * inv;
+                    f[2 * e + 1] = x.y * inv;
+                }
                 *reinterpret_cast<uint4*>(KQp + (cd >> 3) * 16384 + sw128(tid, cd & 7)) =
-                    scale_bf16x8(vals[cd], inv);
+                    h8(f, bad);
+            }
         }
         if (warp == 0) {
             const float a0 = SS.g[buf][2 * lane], a1 = SS.g[buf][2 * lane + 1];
@@ -265,18 +294,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
 
         // ---- B: D0 = [K;Q] K^T  (M=128, N=64, K=128)
         if (tid == 0) {
-            const uint32_t id = idesc_bf16_f32(128, 64, false, false);
+            const uint32_t id = idesc_f32acc(128, 64, false, false, false);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(tmem + TM_D0, sdesc_sw128(KQ + off, 16, 1024),
-                            sdesc_sw128(KQ + off, 16, 1024), id, kk > 0);
+                mma_f32acc_ss(tmem + TM_D0, sdesc_sw128(KQ + off, 16, 1024),
+                              sdesc_sw128(KQ + off, 16, 1024), id, kk > 0);
             }
             mma_commit(&SS.mbar[0]);
         }
         if (!wait_mma(0, par)) { failed = true; break; }
 
-        // ---- C: A (fp32, rows 0-63) and P (bf16, rows 64-127) from D0; Q -> Q~ in place
+        // ---- C: A (fp32, rows 0-63) and P (fp16, rows 64-127) from D0; Q -> Q~ in place
         {
             const int i = tid & 63;
             const bool isK = tid < C;
@@ -315,8 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                                        : 0.f;
                         }
                         *reinterpret_cast<uint4*>(sm + OFF_P + sw128(i, half * 4 + e8)) =
-                            make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]),
-                                       pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
+                            h8(pv, bad);
                     }
                 }
             }
@@ -326,7 +354,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                 for (int cd = 0; cd < 16; ++cd) {
                     uint4* ptr = reinterpret_cast<uint4*>(KQp + (cd >> 3) * 16384 + 8192 +
                                                           sw128(i, cd & 7));
-                    *ptr = scale_bf16x8(*ptr, f);
+                    const uint4 u = *ptr;
+                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                    float fv[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x = unpack_f16x2(w[e]);
+                        fv[2 * e] = x.x * f;
+                        fv[2 * e + 1] = x.y * f;
+                    }
+                    *ptr = h8(fv, bad);
                 }
             }
         }
@@ -361,7 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
 #pragma unroll
             for (int i = 0; i < C; ++i) {
                 const uint32_t off = sw128(i, c0 >> 3) + (c0 & 7) * 2;
-                *reinterpret_cast<__nv_bfloat16*>(tw + off) = __float2bfloat16_rn(x[i] * fw);
+                const float tw_v = x[i] * fw;
+                bad |= !(fabsf(tw_v) < kF16Max);
+                *reinterpret_cast<__half*>(tw + off) = __float2half_rn(tw_v);
                 *reinterpret_cast<__nv_bfloat16*>(tu + off) = __float2bfloat16_rn(x[i] * fu);
             }
         }
@@ -370,17 +409,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
         __syncthreads();
         tc_fence_after();
 
-        // ---- E: W^T = K^T T_w^T and U~^T = V^T T_u^T  (M=128, N=64, K=64, A MN-major)
+        // ---- E: W^T = K^T T_w^T (fp16) and U~^T = V^T T_u^T (bf16)  (M=128, N=64, K=64)
         if (tid == 0) {
-            const uint32_t id = idesc_bf16_f32(128, 64, true, false);
+            const uint32_t idw = idesc_f32acc(128, 64, true, false, false);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_DW, sdesc_sw128(KQ + kk * 2048, 16384, 1024),
-                            sdesc_sw128(sbase + OFF_TW + kk * 32, 16, 1024), id, kk > 0);
+                mma_f32acc_ss(tmem + TM_DW, sdesc_sw128(KQ + kk * 2048, 16384, 1024),
+                              sdesc_sw128(sbase + OFF_TW + kk * 32, 16, 1024), idw, kk > 0);
+            const uint32_t idu = idesc_f32acc(128, 64, true, false, true);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_DU, sdesc_sw128(VV + kk * 2048, 8192, 1024),
-                            sdesc_sw128(sbase + OFF_TU + kk * 32, 16, 1024), id, kk > 0);
+                mma_f32acc_ss(tmem + TM_DU, sdesc_sw128(VV + kk * 2048, 8192, 1024),
+                              sdesc_sw128(sbase + OFF_TU + kk * 32, 16, 1024), idu, kk > 0);
             mma_commit(&SS.mbar[1]);
         }
         if (!wait_mma(1, par)) { failed = true; break; }
@@ -395,10 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                 tmem_wait_ld();
 #pragma unroll
                 for (int e8 = 0; e8 < 4; ++e8) {
-                    const float* f = reinterpret_cast<const float*>(r + e8 * 8);
-                    *reinterpret_cast<uint4*>(sm + OFF_WN + sw128(d, half * 4 + e8)) =
-                        make_uint4(pack_bf16x2(-f[0], -f[1]), pack_bf16x2(-f[2], -f[3]),
-                                   pack_bf16x2(-f[4], -f[5]), pack_bf16x2(-f[6], -f[7]));
+                    float f[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) f[u] = -__uint_as_float(r[e8 * 8 + u]);
+                    *reinterpret_cast<uint4*>(sm + OFF_WN + sw128(d, half * 4 + e8)) = h8(f, bad);
                 }
             }
             if (tid < C) {
@@ -407,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                 for (int cd = 0; cd < 16; ++cd) {
                     uint4* ptr = reinterpret_cast<uint4*>(KQp + (cd >> 3) * 16384 +
                                                           sw128(tid, cd & 7));
-                    *ptr = scale_bf16x8(*ptr, f);
+                    *ptr = scale_f16x8(*ptr, f);
                 }
             }
         }
@@ -418,25 +458,25 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
 
         // ---- G: V'^T = U~^T + H^T (-W^T);  O^T = H^T Q~^T   (M=128, N=64, K=128)
         if (tid == 0) {
-            const uint32_t id1 = idesc_bf16_f32(128, 64, false, true);
+            const uint32_t id1 = idesc_f32acc(128, 64, false, true, false);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t hoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(tmem + TM_DU, sdesc_sw128(sbase + OFF_HB + hoff, 16, 1024),
-                            sdesc_sw128(sbase + OFF_WN + kk * 2048, 8192, 1024), id1, 1);
+                mma_f32acc_ss(tmem + TM_DU, sdesc_sw128(sbase + OFF_HB + hoff, 16, 1024),
+                              sdesc_sw128(sbase + OFF_WN + kk * 2048, 8192, 1024), id1, 1);
             }
-            const uint32_t id2 = idesc_bf16_f32(128, 64, false, false);
+            const uint32_t id2 = idesc_f32acc(128, 64, false, false, false);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t hoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(tmem + TM_DO, sdesc_sw128(sbase + OFF_HB + hoff, 16, 1024),
-                            sdesc_sw128(KQ + hoff + 8192, 16, 1024), id2, kk > 0);
+                mma_f32acc_ss(tmem + TM_DO, sdesc_sw128(sbase + OFF_HB + hoff, 16, 1024),
+                              sdesc_sw128(KQ + hoff + 8192, 16, 1024), id2, kk > 0);
             }
             mma_commit(&SS.mbar[2]);
         }
         if (!wait_mma(2, par)) { failed = true; break; }
 
-        // ---- H: V'^T rows -> VP (bf16); stage the next chunk's gates
+        // ---- H: V'^T rows -> VP (fp16); stage the next chunk's gates
         {
             const int j = tid;
 #pragma unroll
@@ -447,9 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
 #pragma unroll
                 for (int e8 = 0; e8 < 4; ++e8) {
                     const float* f = reinterpret_cast<const float*>(r + e8 * 8);
-                    *reinterpret_cast<uint4*>(sm + OFF_VP + sw128(j, half * 4 + e8)) =
-                        make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                   pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+                    *reinterpret_cast<uint4*>(sm + OFF_VP + sw128(j, half * 4 + e8)) = h8(f, bad);
                 }
             }
             if (has_next && tid < C) { SS.g[buf ^ 1][tid] = g_nx; SS.b[buf ^ 1][tid] = b_nx; }
@@ -465,21 +503,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
 
         // ---- I: O^T += V'^T P^T (N=64, K=64);  H^T += V'^T K~ (N=128, K=64, B MN-major)
         if (tid == 0) {
-            const uint32_t id3 = idesc_bf16_f32(128, 64, false, false);
+            const uint32_t id3 = idesc_f32acc(128, 64, false, false, false);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_DO, sdesc_sw128(sbase + OFF_VP + kk * 32, 16, 1024),
-                            sdesc_sw128(sbase + OFF_P + kk * 32, 16, 1024), id3, 1);
-            const uint32_t id4 = idesc_bf16_f32(128, 128, false, true);
+                mma_f32acc_ss(tmem + TM_DO, sdesc_sw128(sbase + OFF_VP + kk * 32, 16, 1024),
+                              sdesc_sw128(sbase + OFF_P + kk * 32, 16, 1024), id3, 1);
+            const uint32_t id4 = idesc_f32acc(128, 128, false, true, false);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_HM, sdesc_sw128(sbase + OFF_VP + kk * 32, 16, 1024),
-                            sdesc_sw128(KQ + kk * 2048, 16384, 1024), id4, 1);
+                mma_f32acc_ss(tmem + TM_HM, sdesc_sw128(sbase + OFF_VP + kk * 32, 16, 1024),
+                              sdesc_sw128(KQ + kk * 2048, 16384, 1024), id4, 1);
             mma_commit(&SS.mbar[3]);
         }
         if (!wait_mma(3, par)) { failed = true; break; }
 
-        // ---- J: O^T -> staging -> global; state -> bf16 copy, pre-scaled for the next chunk
+        // ---- J: O^T -> staging -> global; state -> fp16 copy, pre-scaled for the next chunk
         {
             const int j = tid;
 #pragma unroll
@@ -506,8 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                     const float* f = reinterpret_cast<const float*>(r + e8 * 8);
                     const int cd = (d0 >> 3) + e8;
                     *reinterpret_cast<uint4*>(sm + OFF_HB + (cd >> 3) * 16384 + sw128(j, cd & 7)) =
-                        make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                   pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+                        h8(f, bad);
                 }
                 if (has_next) {
 #pragma unroll
@@ -552,6 +589,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
         if (tid == 0) atomicExch(&p.hdr->err, (int)GDR_ERR_TIMEOUT);
         cp_async_wait<0>();
     }
+    if (__syncthreads_or(bad ? 1 : 0) && tid == 0)
+        atomicCAS(&p.hdr->err, (int)GDR_OK, (int)GDR_ERR_RANGE);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);

@@ -49,7 +49,9 @@ typedef enum {
     GDR_ERR_WORKSPACE = 4,     /* workspace missing or smaller than the required size */
     GDR_ERR_CUDA = 5,          /* a CUDA launch failed (cudaGetLastError after launch) */
     GDR_ERR_DEVICE_CHECK = 6,  /* device-side check failed (bad cu_seqlens) */
-    GDR_ERR_TIMEOUT = 7        /* a bounded device-side wait gave up */
+    GDR_ERR_TIMEOUT = 7,       /* a bounded device-side wait gave up */
+    GDR_ERR_RANGE = 8          /* tensor-core path: an internal operand left the fp16 range
+                                  (|x| >= 65000 or not finite); the outputs are not valid */
 } gdr_status;
 
 typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;

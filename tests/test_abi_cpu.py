@@ -33,7 +33,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for s in range(8):
+    for s in range(9):
         assert lib.gdr_status_string(s).startswith(b"GDR_")
 
 

@@ -97,3 +97,18 @@ def test_state_aliasing_in_place():
     _, S_r = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"],
                             scale=1 / math.sqrt(128))
     assert_close("S", S, S_r, torch.bfloat16)
+
+
+def test_fp16_range_is_reported():
+    """Values far beyond the fp16 range of the internal operands raise GDR_ERR_RANGE
+    instead of returning silently wrong results."""
+    x = workloads.chunk_inputs(1, 100, 1, 1, 128, 128, "bf16", seed=17)
+    x["v"] = (x["v"].float() * 1e6).to(torch.bfloat16)
+    d = {n: to_dev(x[n]) if x.get(n) is not None else None for n in x}
+    args = gdr.make_chunk_args(d["q"], d["v"], d["g"])
+    ws = torch.empty(gdr.chunk_fwd_workspace_size(args), dtype=torch.uint8, device="cuda")
+    gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], workspace=ws)
+    assert gdr.read_device_error(args, ws) == gdr._abi.GDR_ERR_RANGE
+    x["v"] = (x["v"].float() * 1e-6).to(torch.bfloat16)
+    gdr.chunk_fwd(d["q"], d["k"], to_dev(x["v"]), d["g"], d["beta"], workspace=ws)
+    assert gdr.read_device_error(args, ws) == gdr._abi.GDR_OK
