@@ -128,6 +128,9 @@ def bench_ours(args, rank, world, local_rank):
 
     # ---------------- chunk-parallel forward
     w = workloads.WORKLOADS[args.workload]
+    if args.rows:  # a smaller case of the same kernel (profiling): fewer rows of the workload
+        import dataclasses
+        w = dataclasses.replace(w, B=args.rows, name=f"{w.name}[rows={args.rows}]")
     x = workloads.workload_inputs(w, seed=rank)
     d = {n: (t.to(dev) if t is not None else None) for n, t in x.items()}
     cargs = gdr.make_chunk_args(d["q"], d["v"], d["g"], d["cu_seqlens"], w.chunk, w.read_mode,
@@ -248,11 +251,11 @@ def bench_ours(args, rank, world, local_rank):
                    "state": "fp32", "path": path,
                    "l2": "inputs larger than L2 (q,k,v,o 537 MB > 126 MB), no flush",
                    "parallelism": f"replicas x{world}, no collective"},
-        "tflops": tflops, "pct_bf16_tc_peak": tflops * 1e3 / peaks["bf16_tflops"] * 100,
+        "tflops": tflops, "pct_bf16_tc_peak": tflops / peaks["bf16_tflops"] * 100,
         "roofline": {"bound": "hbm", "achieved": hbm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": hbm_gbs / peaks["hbm_gbs"], "traffic": args.traffic,
                      "algorithmic_bytes": algo_bytes, "flops": flops,
-                     "tensor_frac": tflops * 1e3 / peaks["bf16_tflops"],
+                     "tensor_frac": tflops / peaks["bf16_tflops"],
                      "timed": "whole gdr_chunk_fwd call (plan + chunk kernels), CUDA events",
                      "peak_source": f"{peak_src} (hbm_gbs copy; bf16_tflops burst)"},
         "decode": dec, "e2e": e2e, "clocks": clocks,
@@ -320,6 +323,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="run only this many rows of the forward workload (profiling a small case)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the dominant kernel from an ncu capture")
     args = ap.parse_args()
