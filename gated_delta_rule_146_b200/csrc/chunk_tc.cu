@@ -36,8 +36,12 @@
 // Operand precision: V and T diag(beta) are bf16 (V arrives in bf16); every other operand
 // (normalised q and k, T diag(beta e^G), W, the state copy, V', P) is rounded to fp16,
 // whose 11-bit significand keeps the chain of roundings well inside the bf16 parity bound
-// at long sequence lengths where bf16 operands do not.  The fp16 range is checked wherever
-// an operand is produced; a value beyond it sets GDR_ERR_RANGE.
+// at long sequence lengths where bf16 operands do not.  Every fp16 operand is checked for
+// overflow (an infinite or NaN half); one sets GDR_ERR_RANGE.  Decay factors are
+// 2^(log2(e) (G_i - G_j)) by the hardware exp2 approximation (relative error ~2^-22).
+//
+// The state update uses V' with its rows scaled by e^(G_C - G_i) (a second fp16 copy in
+// tensor memory) against the unscaled K, so K is never rewritten after normalisation.
 //
 // The state H is kept transposed in TMEM (lane = dv, column = dk).  After each chunk the
 // chain reads it once, writes the fp16 copy the next chunk's MMAs consume, and scales it
@@ -56,7 +60,7 @@ constexpr int D = 128;           // dk = dv
 constexpr int kThreads = 256;    // warpgroup 0: state chain, warpgroup 1: chunk preparation
 constexpr int kBarChain = 1, kBarPrep = 2;  // named barriers of the two warpgroups
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr float kF16Max = 65000.f;  // operands at or beyond this (or NaN) raise GDR_ERR_RANGE
+constexpr float kLog2e = 1.4426950408889634f;
 
 // shared memory map (bytes from a 1024-byte-aligned base)
 constexpr uint32_t OFF_KQ = 0;         // 3 x 32 KB; per dk half (16 KB): K rows 0-63, Q rows 64-127
@@ -70,7 +74,7 @@ constexpr uint32_t OFF_RS = 163840;    // solve scratch: 4 warps x 16x16 fp32
 constexpr uint32_t OFF_P = 167936;     // 2 x 8 KB: P fp16 [i][j]
 constexpr uint32_t OFF_WN = 184320;    // 2 x 16 KB: -W^T fp16 [dk][tok]
 constexpr uint32_t OFF_SMALL = 217088;
-constexpr uint32_t SMEM_BYTES = OFF_SMALL + 2048 + 1024;
+constexpr uint32_t SMEM_BYTES = OFF_SMALL + 4096 + 1024;
 
 // TMEM columns (32-bit each)
 constexpr uint32_t TM_D0 = 0;     // [K;Q] K^T, then W^T (64)
@@ -78,7 +82,8 @@ constexpr uint32_t TM_DU = 64;    // 2 x 64: U~^T, then V'^T, by chunk parity
 constexpr uint32_t TM_DO = 192;   // O^T (64)
 constexpr uint32_t TM_HM = 256;   // state H^T, fp32 (128)
 constexpr uint32_t TM_HB = 384;   // state H^T, fp16 packed (64): A operand
-constexpr uint32_t TM_VP = 448;   // V'^T, fp16 packed (32): A operand
+constexpr uint32_t TM_VP = 448;   // V'^T, fp16 packed (32): A operand of the output product
+constexpr uint32_t TM_VS = 480;   // V'^T scaled by e^(G_C - G_i), fp16 packed (32): state update
 constexpr uint32_t TM_COLS = 512;
 
 // mbarriers
@@ -86,15 +91,15 @@ enum { MB_M0 = 0, MB_MW = 1, MB_M1 = 2, MB_M3 = 3 /* x2 */, MB_PREP = 5 /* x2 */
 
 struct Small {
     float g[2][C], b[2][C];  // raw gates by chunk parity (prep)
-    float G[C];              // in-chunk cumulative log decay of the chunk being prepared
-    float Kd[C];             // e^(G_last - G_i), 0 beyond the chunk
+    float G[C];              // log2(e) x in-chunk cumulative log decay (prep, chunk being prepared)
     float bg[C];             // beta_i e^(G_i)
+    float Kd[2][C];          // e^(G_last - G_i), 0 beyond the chunk, by chunk parity (for the chain)
     float gsum_part[2];      // chain: partial sums of the next chunk's g
     uint64_t mbar[MB_COUNT];
     uint32_t tmem_base;
     int abort;
 };
-static_assert(sizeof(Small) <= 2048, "small shared block");
+static_assert(sizeof(Small) <= 4096, "small shared block");
 
 struct TcParams {
     const __nv_bfloat16* q; const __nv_bfloat16* k; const __nv_bfloat16* v;
@@ -106,26 +111,17 @@ struct TcParams {
     float scale;
 };
 
-// fp16 pair with a range check: `bad` is set when either value is not finite or too large
-__device__ __forceinline__ uint32_t h2(float a, float b, bool& bad) {
-    bad |= !(fabsf(a) < kF16Max) || !(fabsf(b) < kF16Max);
-    return pack_f16x2(a, b);
+// fp16 pair; `flags` accumulates the overflow test: (exponent & 0x7C00) + 0x0400 carries into
+// bit 15 (31) exactly when a half is infinite or NaN.
+__device__ __forceinline__ uint32_t h2(float a, float b, uint32_t& flags) {
+    const uint32_t u = pack_f16x2(a, b);
+    flags |= (u & 0x7C007C00u) + 0x04000400u;
+    return u;
 }
 
-__device__ __forceinline__ uint4 h8(const float* f, bool& bad) {
-    return make_uint4(h2(f[0], f[1], bad), h2(f[2], f[3], bad), h2(f[4], f[5], bad),
-                      h2(f[6], f[7], bad));
-}
-
-// 8 fp16 scaled by f (|f| <= 1 at every call site, so the range cannot grow)
-__device__ __forceinline__ uint4 scale_f16x8(uint4 u, float f) {
-    uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float2 x = unpack_f16x2(w[e]);
-        w[e] = pack_f16x2(x.x * f, x.y * f);
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
+__device__ __forceinline__ uint4 h8(const float* f, uint32_t& flags) {
+    return make_uint4(h2(f[0], f[1], flags), h2(f[2], f[3], flags), h2(f[4], f[5], flags),
+                      h2(f[6], f[7], flags));
 }
 
 // element (i, j) of a fp32 [64][64] matrix stored with 16-byte chunks XOR-swizzled by row
@@ -152,6 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
     const int L = (int)(t1 - t0);
     const int nchunks = (L + C - 1) / C;
     const size_t sb = ((size_t)s * p.Hv + h) * D * D;
+    // physical token of logical position 0, and the step between consecutive positions
+    const long long tokA = p.reverse ? t1 - 1 : t0;
+    const long long tstep = p.reverse ? -1 : 1;
 
     if (nchunks == 0) {  // empty sequence: the state passes through
         if (p.S_final)
@@ -175,12 +174,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
     tc_fence_after();
     const uint32_t tmem = SS.tmem_base;
     const uint32_t tlane = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's lanes
-    bool bad = false;   // an fp16 operand out of range
-    bool fail = false;  // a bounded wait gave up
+    uint32_t rflags = 0;  // fp16 overflow test bits
+    bool fail = false;    // a bounded wait gave up
 
-    auto gate_at = [&](const void* arr, int c, int i) -> float {
-        const long long t = phys_token(t0, t1, c * C + i, p.reverse);
-        return load_elem(arr, (size_t)t * p.Hv + h, p.gt);
+    auto gate_at = [&](const void* arr, int pos) -> float {
+        return load_elem(arr, (size_t)(tokA + tstep * pos) * p.Hv + h, p.gt);
     };
     // wait for a phase of an mbarrier; the whole warpgroup agrees on the outcome
     auto wg_wait = [&](int idx, uint32_t parity, int bar_id) -> bool {
@@ -194,27 +192,25 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
     if (wg == 1) {
         // ============================ preparation warpgroup ============================
         const int t = lt;
+        // cp.async plan: this thread copies 16-byte column chunk `cd` of rows r0 + 8 m
+        const int cd = t & 15, r0 = t >> 4;
+        const __nv_bfloat16* kbase = p.k + (size_t)hk * D + cd * 8;
+        const __nv_bfloat16* qbase = p.q + (size_t)hk * D + cd * 8;
+        const __nv_bfloat16* vbase = p.v + (size_t)h * D + cd * 8;
+        const long long kq_tok = (long long)p.Hk * D, v_tok = (long long)p.Hv * D;
         auto load_chunk = [&](int c) {
             const int Cc = min(C, L - c * C);
-            const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
-            const uint32_t vv = sbase + OFF_V + (c & 1) * V_STRIDE;
-            for (int idx = t; idx < 3 * C * 16; idx += 128) {
-                const int tile = idx >> 10, rem = idx & 1023, i = rem >> 4, cd = rem & 15;
+            const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_STRIDE + (cd >> 3) * 16384;
+            const uint32_t vv = sbase + OFF_V + (c & 1) * V_STRIDE + (cd >> 3) * 8192;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int i = r0 + 8 * m;
                 const bool valid = i < Cc;
-                const long long tok = valid ? phys_token(t0, t1, c * C + i, p.reverse) : t0;
-                const __nv_bfloat16* src;
-                uint32_t dst;
-                if (tile == 0) {
-                    src = p.k + ((size_t)tok * p.Hk + hk) * D + cd * 8;
-                    dst = kq + (cd >> 3) * 16384 + sw128(i, cd & 7);
-                } else if (tile == 1) {
-                    src = p.q + ((size_t)tok * p.Hk + hk) * D + cd * 8;
-                    dst = kq + (cd >> 3) * 16384 + 8192 + sw128(i, cd & 7);
-                } else {
-                    src = p.v + ((size_t)tok * p.Hv + h) * D + cd * 8;
-                    dst = vv + (cd >> 3) * 8192 + sw128(i, cd & 7);
-                }
-                cp_async16(dst, src, valid);
+                const long long tok = valid ? tokA + tstep * (c * C + i) : t0;
+                const uint32_t off = sw128(i, cd & 7);
+                cp_async16(kq + off, kbase + tok * kq_tok, valid);
+                cp_async16(kq + 8192 + off, qbase + tok * kq_tok, valid);
+                cp_async16(vv + off, vbase + tok * v_tok, valid);
             }
         };
         load_chunk(0);
@@ -222,8 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
         {
             const int Cc0 = min(C, L);
             if (t < C) {
-                SS.g[0][t] = t < Cc0 ? gate_at(p.g, 0, t) : 0.f;
-                SS.b[0][t] = t < Cc0 ? gate_at(p.beta, 0, t) : 0.f;
+                SS.g[0][t] = t < Cc0 ? gate_at(p.g, t) : 0.f;
+                SS.b[0][t] = t < Cc0 ? gate_at(p.beta, t) : 0.f;
             }
         }
         float g_nx = 0.f, b_nx = 0.f;
@@ -240,46 +236,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             if (has_next) {
                 load_chunk(c + 1);
                 const int Cn = min(C, L - (c + 1) * C);
-                g_nx = t < Cn ? gate_at(p.g, c + 1, t) : 0.f;
-                b_nx = t < Cn ? gate_at(p.beta, c + 1, t) : 0.f;
+                g_nx = t < Cn ? gate_at(p.g, (c + 1) * C + t) : 0.f;
+                b_nx = t < Cn ? gate_at(p.beta, (c + 1) * C + t) : 0.f;
             }
             cp_async_commit();
-            cp_async_wait<1>();
-            fence_proxy_async_smem();
-            named_bar(kBarPrep, 128);
-
-            // P1: row t of [K; Q]: bf16 -> (L2-normalised) fp16 in place; cumsum of g
-            {
-                uint4 vals[16];
-                float ss = 0.f;
-#pragma unroll
-                for (int cd = 0; cd < 16; ++cd) {
-                    vals[cd] = *reinterpret_cast<const uint4*>(KQp + (cd >> 3) * 16384 +
-                                                               sw128(t, cd & 7));
-                    const uint32_t w[4] = {vals[cd].x, vals[cd].y, vals[cd].z, vals[cd].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 x = unpack_bf16x2(w[e]);
-                        ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
-                    }
-                }
-                const float inv = p.qk_l2norm ? 1.f / fmaxf(sqrtf(ss), kNormEps) : 1.f;
-#pragma unroll
-                for (int cd = 0; cd < 16; ++cd) {
-                    const uint32_t w[4] = {vals[cd].x, vals[cd].y, vals[cd].z, vals[cd].w};
-                    float f[8];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 x = unpack_bf16x2(w[e]);
-                        f[2 * e] = x.x * inv;
-                        f[2 * e + 1] = x.y * inv;
-                    }
-                    *reinterpret_cast<uint4*>(KQp + (cd >> 3) * 16384 + sw128(t, cd & 7)) =
-                        h8(f, bad);
-                }
-            }
+            // in-chunk cumsum of g (log2 units) while the copies land
             if (warp == 4) {
-                const float a0 = SS.g[pb][2 * lane], a1 = SS.g[pb][2 * lane + 1];
+                const float a0 = SS.g[pb][2 * lane] * kLog2e, a1 = SS.g[pb][2 * lane + 1] * kLog2e;
                 const float pair = a0 + a1;
                 float incl = pair;
 #pragma unroll
@@ -291,10 +254,43 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                 SS.G[2 * lane] = excl + a0;
                 SS.G[2 * lane + 1] = excl + a0 + a1;
             }
+            cp_async_wait<1>();
+            fence_proxy_async_smem();
             named_bar(kBarPrep, 128);
-            if (t < C) {
-                SS.Kd[t] = t < Cc ? expf(SS.G[Cc - 1] - SS.G[t]) : 0.f;
-                SS.bg[t] = SS.b[pb][t] * expf(SS.G[t]);
+
+            // P1: row t of [K; Q]: bf16 -> (L2-normalised) fp16 in place; per-row factors
+            {
+                uint4 vals[16];
+                float ss = 0.f;
+#pragma unroll
+                for (int c16 = 0; c16 < 16; ++c16) {
+                    vals[c16] = *reinterpret_cast<const uint4*>(KQp + (c16 >> 3) * 16384 +
+                                                                sw128(t, c16 & 7));
+                    const uint32_t w[4] = {vals[c16].x, vals[c16].y, vals[c16].z, vals[c16].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x = unpack_bf16x2(w[e]);
+                        ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
+                    }
+                }
+                const float inv = p.qk_l2norm ? 1.f / fmaxf(sqrtf(ss), kNormEps) : 1.f;
+#pragma unroll
+                for (int c16 = 0; c16 < 16; ++c16) {
+                    const uint32_t w[4] = {vals[c16].x, vals[c16].y, vals[c16].z, vals[c16].w};
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x = unpack_bf16x2(w[e]);
+                        f[2 * e] = x.x * inv;
+                        f[2 * e + 1] = x.y * inv;
+                    }
+                    *reinterpret_cast<uint4*>(KQp + (c16 >> 3) * 16384 + sw128(t, c16 & 7)) =
+                        h8(f, rflags);
+                }
+                if (t < C) {
+                    SS.Kd[pb][t] = t < Cc ? ex2(SS.G[Cc - 1] - SS.G[t]) : 0.f;
+                    SS.bg[t] = SS.b[pb][t] * ex2(SS.G[t]);
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -314,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             }
             if (!wg_wait(MB_M0, c & 1, kBarPrep)) { fail = true; break; }
 
-            // P3: A rows (fp32) and P rows (fp16) from D0; Q -> Q~ in place
+            // P3: A rows (fp32) and P rows (fp16) from D0; Q -> Q~ = scale e^(G') Q in place
             {
                 const int i = t & 63;
                 const bool isK = t < C;
@@ -334,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
                                 const int j = half * 32 + e4 * 4 + u;
-                                a[u] = j < i ? bi * u2f(r[e4 * 4 + u]) * expf(Gi - SS.G[j]) : 0.f;
+                                a[u] = j < i ? bi * u2f(r[e4 * 4 + u]) * ex2(Gi - SS.G[j]) : 0.f;
                             }
                             *reinterpret_cast<float4*>(f32sw(As, i, half * 32 + e4 * 4)) =
                                 make_float4(a[0], a[1], a[2], a[3]);
@@ -347,29 +343,24 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                             for (int u = 0; u < 8; ++u) {
                                 const int j = half * 32 + e8 * 8 + u;
                                 const bool on = p.read_pre ? (j < i) : (j <= i);
-                                pv[u] = on ? p.scale * u2f(r[e8 * 8 + u]) * expf(Gr - SS.G[j]) : 0.f;
+                                pv[u] = on ? p.scale * u2f(r[e8 * 8 + u]) * ex2(Gr - SS.G[j]) : 0.f;
                             }
                             *reinterpret_cast<uint4*>(sm + OFF_P + pb * 8192 +
-                                                      sw128(i, half * 4 + e8)) = h8(pv, bad);
+                                                      sw128(i, half * 4 + e8)) = h8(pv, rflags);
                         }
                     }
                 }
                 if (!isK) {
-                    const float f = p.scale * expf(Gr);
+                    const __half2 f2 = __float2half2_rn(p.scale * ex2(Gr));
 #pragma unroll
-                    for (int cd = 0; cd < 16; ++cd) {
-                        uint4* ptr = reinterpret_cast<uint4*>(KQp + (cd >> 3) * 16384 + 8192 +
-                                                              sw128(i, cd & 7));
-                        const uint4 u = *ptr;
-                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-                        float fv[8];
+                    for (int c16 = 0; c16 < 16; ++c16) {
+                        uint4* ptr = reinterpret_cast<uint4*>(KQp + (c16 >> 3) * 16384 + 8192 +
+                                                              sw128(i, c16 & 7));
+                        uint4 u = *ptr;
+                        __half2* hv = reinterpret_cast<__half2*>(&u);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 x = unpack_f16x2(w[e]);
-                            fv[2 * e] = x.x * f;
-                            fv[2 * e + 1] = x.y * f;
-                        }
-                        *ptr = h8(fv, bad);
+                        for (int e = 0; e < 4; ++e) hv[e] = __hmul2(hv[e], f2);
+                        *ptr = u;
                     }
                 }
             }
@@ -383,18 +374,20 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                 float* Ts = reinterpret_cast<float*>(sm + OFF_TWU);
                 const int wp = warp - 4;
                 if (lane < 16) {
+                    // column `cl` of the inverse of the unit-lower 16x16 block `wp`, by
+                    // right-looking substitution (each new x_j is pushed into later rows)
                     const int b0 = wp * 16, cl = lane;
-                    float x[16];
+                    float acc[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float acc = 0.f;
+                    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
 #pragma unroll
-                        for (int jj = 0; jj < i; ++jj)
-                            acc = fmaf(*f32sw(As, b0 + i, b0 + jj), x[jj], acc);
-                        x[i] = i < cl ? 0.f : (i == cl ? 1.f : -acc);
+                    for (int jc = 0; jc < 16; ++jc) {
+                        const float xj = jc < cl ? 0.f : (jc == cl ? 1.f : -acc[jc]);
+                        *f32sw(Ts, b0 + jc, b0 + cl) = xj;
+#pragma unroll
+                        for (int i = jc + 1; i < 16; ++i)
+                            acc[i] = fmaf(*f32sw(As, b0 + i, b0 + jc), xj, acc[i]);
                     }
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) *f32sw(Ts, b0 + i, b0 + cl) = x[i];
                 }
                 named_bar(kBarPrep, 128);
                 const int gq = lane >> 2, tq = lane & 3;
@@ -456,14 +449,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                     }
                     named_bar(kBarPrep, 128);
                 }
-                // T -> T diag(beta e^G) (fp16) and T diag(beta) (bf16), row i, 32 columns
+                // T -> T diag(beta e^G) (fp16) and T diag(beta) (bf16): row i, 32 columns
                 const int i = t >> 1, half = t & 1;
                 float tv[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int j = half * 32 + e;
-                    tv[e] = j <= i ? *f32sw(Ts, i, j) : 0.f;
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 v4 = *reinterpret_cast<const float4*>(f32sw(Ts, i, half * 32 + e4 * 4));
+                    tv[e4 * 4 + 0] = v4.x; tv[e4 * 4 + 1] = v4.y;
+                    tv[e4 * 4 + 2] = v4.z; tv[e4 * 4 + 3] = v4.w;
                 }
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if (half * 32 + e > i) tv[e] = 0.f;  // blocks above the diagonal are never written
                 named_bar(kBarPrep, 128);  // T is read completely before the 16-bit tiles overwrite it
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
@@ -471,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int jj = m * 8 + 2 * e, j = half * 32 + jj;
-                        w4[e] = h2(tv[jj] * SS.bg[j], tv[jj + 1] * SS.bg[j + 1], bad);
+                        w4[e] = h2(tv[jj] * SS.bg[j], tv[jj + 1] * SS.bg[j + 1], rflags);
                         u4[e] = pack_bf16x2(tv[jj] * SS.b[pb][j], tv[jj + 1] * SS.b[pb][j + 1]);
                     }
                     *reinterpret_cast<uint4*>(sm + OFF_TWU + sw128(i, half * 4 + m)) =
@@ -502,35 +499,24 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             }
             if (!wg_wait(MB_MW, c & 1, kBarPrep)) { fail = true; break; }
 
-            // P6: -W^T rows -> WN[pb] (B operand, MN-major); K -> K~ = diag(Kd) K in place
-            {
+            // P6: -W^T rows -> WN[pb] (B operand, MN-major); hand the chunk to the chain
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32];
-                    tmem_ld32(tlane + TM_D0 + half * 32, r);
-                    tmem_wait_ld();
+            for (int half = 0; half < 2; ++half) {
+                uint32_t r[32];
+                tmem_ld32(tlane + TM_D0 + half * 32, r);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int e8 = 0; e8 < 4; ++e8) {
-                        float f[8];
+                for (int e8 = 0; e8 < 4; ++e8) {
+                    float f[8];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) f[u] = -u2f(r[e8 * 8 + u]);
-                        *reinterpret_cast<uint4*>(sm + OFF_WN + pb * 16384 +
-                                                  sw128(t, half * 4 + e8)) = h8(f, bad);
-                    }
+                    for (int u = 0; u < 8; ++u) f[u] = -u2f(r[e8 * 8 + u]);
+                    *reinterpret_cast<uint4*>(sm + OFF_WN + pb * 16384 + sw128(t, half * 4 + e8)) =
+                        h8(f, rflags);
                 }
-                if (t < C) {
-                    const float f = SS.Kd[t];
-#pragma unroll
-                    for (int cd = 0; cd < 16; ++cd) {
-                        uint4* ptr = reinterpret_cast<uint4*>(KQp + (cd >> 3) * 16384 +
-                                                              sw128(t, cd & 7));
-                        *ptr = scale_f16x8(*ptr, f);
-                    }
-                }
-                if (has_next && t < C) {
-                    SS.g[pb ^ 1][t] = g_nx;
-                    SS.b[pb ^ 1][t] = b_nx;
-                }
+            }
+            if (has_next && t < C) {
+                SS.g[pb ^ 1][t] = g_nx;
+                SS.b[pb ^ 1][t] = b_nx;
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -540,13 +526,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
     } else {
         // =============================== chain warpgroup ===============================
         const int j = lt;  // dv column = TMEM lane
+        const long long o_step = tstep * (long long)p.Hv * D;  // elements between consecutive positions
         {
             // initial state -> TM_HM (pre-scaled by chunk 0's total decay), TM_HB (fp16)
-            const float gv = lt < min(C, L) ? gate_at(p.g, 0, lt) : 0.f;
+            const float gv = lt < min(C, L) ? gate_at(p.g, lt) : 0.f;
             const float part = warp_sum(gv);
             if (lane == 0 && warp < 2) SS.gsum_part[warp] = part;
             named_bar(kBarChain, 128);
-            const float gam = expf(SS.gsum_part[0] + SS.gsum_part[1]);
+            const float gam = ex2((SS.gsum_part[0] + SS.gsum_part[1]) * kLog2e);
 #pragma unroll
             for (int d0 = 0; d0 < D; d0 += 32) {
                 uint32_t r[32], hb[16];
@@ -556,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                     const float x1 = p.S0 ? p.S0[sb + (size_t)(d0 + e + 1) * D + j] : 0.f;
                     r[e] = __float_as_uint(x0 * gam);
                     r[e + 1] = __float_as_uint(x1 * gam);
-                    hb[e >> 1] = h2(x0, x1, bad);
+                    hb[e >> 1] = h2(x0, x1, rflags);
                 }
                 tmem_st32(tlane + TM_HM + d0, r);
                 tmem_st16(tlane + TM_HB + d0 / 2, hb);
@@ -572,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             const int Cc = min(C, L - c * C);
             const bool has_next = c + 1 < nchunks;
             const int Cn = has_next ? min(C, L - (c + 1) * C) : 0;
-            const float g_nx = lt < Cn ? gate_at(p.g, c + 1, lt) : 0.f;
+            const float g_nx = lt < Cn ? gate_at(p.g, (c + 1) * C + lt) : 0.f;
 
             if (!wg_wait(MB_PREP + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
             // C1: V'^T = U~^T + H^T (-W^T);  O^T = H^T Q~^T   (A = state copy in TMEM)
@@ -594,16 +581,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             }
             if (!wg_wait(MB_M1, c & 1, kBarChain)) { fail = true; break; }
 
-            // C2: V'^T -> fp16 packed in TMEM (A operand of the next two products)
+            // C2: V'^T -> fp16 packed in TMEM, plain (output) and scaled by Kd (state update)
             {
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32], pk[16];
+                    uint32_t r[32], pk[16], ps[16];
                     tmem_ld32(tlane + TM_DU + pb * 64 + half * 32, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = h2(u2f(r[2 * e]), u2f(r[2 * e + 1]), bad);
+                    for (int e = 0; e < 16; ++e) {
+                        const float a = u2f(r[2 * e]), b = u2f(r[2 * e + 1]);
+                        pk[e] = h2(a, b, rflags);
+                        ps[e] = h2(a * SS.Kd[pb][half * 32 + 2 * e], b * SS.Kd[pb][half * 32 + 2 * e + 1],
+                                   rflags);
+                    }
                     tmem_st16(tlane + TM_VP + half * 16, pk);
+                    tmem_st16(tlane + TM_VS + half * 16, ps);
                 }
                 tmem_wait_st();
                 if (warp < 2) {
@@ -615,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             named_bar(kBarChain, 128);
             tc_fence_after();
 
-            // C3: O^T += V'^T P^T (N=64, K=64);  H^T += V'^T K~ (N=128, K=64, B MN-major)
+            // C3: O^T += V'^T P^T (N=64, K=64);  H^T += (Kd V')^T K (N=128, K=64, B MN-major)
             if (lt == 0) {
                 const uint32_t id3 = idesc_f32acc(128, 64, false, false, false);
 #pragma unroll
@@ -625,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                 const uint32_t id4 = idesc_f32acc(128, 128, false, true, false);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f32acc_ts(tmem + TM_HM, tmem + TM_VP + kk * 8,
+                    mma_f32acc_ts(tmem + TM_HM, tmem + TM_VS + kk * 8,
                                   sdesc_sw128(KQ + kk * 2048, 16384, 1024), id4, 1);
                 mma_commit(&SS.mbar[MB_M3 + pb]);
             }
@@ -633,23 +626,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
 
             // C4: O -> global (bf16 pairs); state -> fp16 copy, pre-scaled for the next chunk
             {
+                __nv_bfloat16* orow = p.o + (tokA + tstep * (long long)(c * C)) * p.Hv * D +
+                                      (size_t)h * D + (j & ~1);
+                const bool odd = j & 1;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t r[32];
                     tmem_ld32(tlane + TM_DO + half * 32, r);
                     tmem_wait_ld();
-                    const bool odd = j & 1;
 #pragma unroll
                     for (int m = 0; m < 16; ++m) {
                         const float a = u2f(r[2 * m]), b = u2f(r[2 * m + 1]);  // O[i0][j], O[i0+1][j]
                         const float recv = __shfl_xor_sync(0xffffffffu, odd ? a : b, 1);
                         const int i = half * 32 + 2 * m + (odd ? 1 : 0);
-                        const float lo = odd ? recv : a, hi = odd ? b : recv;
                         if (i < Cc) {
-                            const long long tok = phys_token(t0, t1, c * C + i, p.reverse);
-                            uint32_t* dst = reinterpret_cast<uint32_t*>(
-                                p.o + ((size_t)tok * p.Hv + h) * D + (j & ~1));
-                            float2 val = make_float2(lo, hi);
+                            uint32_t* dst = reinterpret_cast<uint32_t*>(orow + o_step * i);
+                            float2 val = odd ? make_float2(recv, b) : make_float2(a, recv);
                             if (p.o_acc) {
                                 const float2 old = unpack_bf16x2(*dst);
                                 val.x += old.x;
@@ -659,14 +651,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                         }
                     }
                 }
-                const float gam = has_next ? expf(SS.gsum_part[0] + SS.gsum_part[1]) : 1.f;
+                const float gam = has_next ? ex2((SS.gsum_part[0] + SS.gsum_part[1]) * kLog2e) : 1.f;
 #pragma unroll
                 for (int d0 = 0; d0 < D; d0 += 32) {
                     uint32_t r[32], hb[16];
                     tmem_ld32(tlane + TM_HM + d0, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) hb[e] = h2(u2f(r[2 * e]), u2f(r[2 * e + 1]), bad);
+                    for (int e = 0; e < 16; ++e) hb[e] = h2(u2f(r[2 * e]), u2f(r[2 * e + 1]), rflags);
                     tmem_st16(tlane + TM_HB + d0 / 2, hb);
                     if (has_next) {
 #pragma unroll
@@ -686,10 +678,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
         }
     }
 
-    if (fail && tid == 0) atomicExch(&p.hdr->err, (int)GDR_ERR_TIMEOUT);
-    if (fail && tid == 128) atomicExch(&p.hdr->err, (int)GDR_ERR_TIMEOUT);
+    if (fail && (tid == 0 || tid == 128)) atomicExch(&p.hdr->err, (int)GDR_ERR_TIMEOUT);
     tc_fence_before();
-    if (__syncthreads_or(bad ? 1 : 0) && tid == 0)
+    if (__syncthreads_or((rflags & 0x80008000u) ? 1 : 0) && tid == 0)
         atomicCAS(&p.hdr->err, (int)GDR_OK, (int)GDR_ERR_RANGE);
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 }

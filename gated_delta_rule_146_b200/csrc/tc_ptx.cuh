@@ -204,6 +204,13 @@ __device__ __forceinline__ void named_bar(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// ---- fast base-2 exponential (hardware approximation, flushes subnormal results to 0) ----
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---- warp-level tf32 MMA (m16n8k8, fp32 accumulate) for the small blocked solve ---------
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
