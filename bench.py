@@ -100,6 +100,27 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+# ------------------------------------------------------------------ replica bookkeeping
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank float over all ranks (the step time of the slowest replica)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" \
+        else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Units per second over all replicas: every rank does the same work per step (weak
+    scaling) and the step takes as long as the slowest rank."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 # ------------------------------------------------------------------ our implementation
 
 def bench_ours(args, rank, world, local_rank):
@@ -118,13 +139,6 @@ def bench_ours(args, rank, world, local_rank):
     def barrier():
         if world > 1:
             dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # ---------------- chunk-parallel forward
     w = workloads.WORKLOADS[args.workload]
@@ -160,7 +174,7 @@ def bench_ours(args, rank, world, local_rank):
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world)
 
     tokens = int(d["q"].shape[0] * d["q"].shape[1])
     head_tokens = tokens * w.Hv
@@ -168,7 +182,7 @@ def bench_ours(args, rank, world, local_rank):
     algo_bytes = sum(t.numel() * t.element_size() for t in
                      (d["q"], d["k"], d["v"], d["g"], d["beta"], o, S_final)) + (
         d["S0"].numel() * 4 if d["S0"] is not None else 0)
-    value = world * tokens / (ms / 1e3)
+    value = whole_job_rate(tokens, world, ms)
     tflops = flops / (ms / 1e3) / 1e12
     hbm_gbs = algo_bytes / (ms / 1e3) / 1e9
     launches_per_call = 2 if path == "tc" else 3
@@ -196,7 +210,7 @@ def bench_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        dms = max_over_ranks(e0.elapsed_time(e1) / dw.steps)
+        dms = max_over_ranks(e0.elapsed_time(e1) / dw.steps, world)
         dbytes = 2 * dd["S"].numel() * 4 + sum(
             dd[n][0].numel() * dd[n].element_size() for n in ("q", "k", "v", "g", "beta")) + (
             od.numel() * od.element_size())
@@ -236,8 +250,8 @@ def bench_ours(args, rank, world, local_rank):
         a1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ems = max_over_ranks(a0.elapsed_time(a1) / n_e2e)
-        e2e = {"value": world * tokens / (ems / 1e3), "unit": "tokens/s", "ms_per_step": ems,
+        ems = max_over_ranks(a0.elapsed_time(a1) / n_e2e, world)
+        e2e = {"value": whole_job_rate(tokens, world, ems), "unit": "tokens/s", "ms_per_step": ems,
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin.values()),
                "d2h_bytes_per_step": h_o.numel() * h_o.element_size() + h_S.numel() * 4}
 

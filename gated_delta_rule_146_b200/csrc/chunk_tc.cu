@@ -18,10 +18,11 @@
 //   o = diag(scale e^G') Q H + P V',  P = scale (Q K^T)(.)decay mask   (MMA x2)
 //   H <- e^(G_C) H + (diag(e^(G_C - G)) K)^T V'     (MMA into the TMEM state)
 //
-// Two warpgroups work on consecutive chunks at once.  The "prep" warpgroup (warps 4-7)
-// loads chunk c+1 and does everything that does not depend on the state: normalisation,
-// [K;Q]K^T, the solve, W and U~.  The "chain" warpgroup (warps 0-3) runs the state
-// recursion of chunk c: V', the output and the state update.  They hand chunks over
+// Three warpgroups work on consecutive chunks at once.  The two "prep" warpgroups (warps
+// 4-11, splitting each step by rows or column halves) load chunk c+1 and do everything that
+// does not depend on the state: normalisation, [K;Q]K^T, the solve, W and U~.  The "chain"
+// warpgroup (warps 0-3) runs the state recursion of chunk c: V', the output and the state
+// update.  They hand chunks over
 // through mbarriers; K/Q tiles are triple-buffered and every other per-chunk buffer is
 // double-buffered by chunk parity.
 //
@@ -57,8 +58,9 @@ using namespace tc;
 
 constexpr int C = 64;            // chunk length
 constexpr int D = 128;           // dk = dv
-constexpr int kThreads = 256;    // warpgroup 0: state chain, warpgroup 1: chunk preparation
-constexpr int kBarChain = 1, kBarPrep = 2;  // named barriers of the two warpgroups
+constexpr int kThreads = 384;    // warpgroup 0: state chain; warpgroups 1-2: chunk preparation
+constexpr int kPrep = 256;       // preparation threads
+constexpr int kBarChain = 1, kBarPrep = 2;  // named barriers of the chain and of the preparation
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -74,7 +76,7 @@ constexpr uint32_t OFF_RS = 163840;    // solve scratch: 4 warps x 16x16 fp32
 constexpr uint32_t OFF_P = 167936;     // 2 x 8 KB: P fp16 [i][j]
 constexpr uint32_t OFF_WN = 184320;    // 2 x 16 KB: -W^T fp16 [dk][tok]
 constexpr uint32_t OFF_SMALL = 217088;
-constexpr uint32_t SMEM_BYTES = OFF_SMALL + 4096 + 1024;
+constexpr uint32_t SMEM_BYTES = OFF_SMALL + 5120 + 1024;
 
 // TMEM columns (32-bit each)
 constexpr uint32_t TM_D0 = 0;     // [K;Q] K^T, then W^T (64)
@@ -94,12 +96,17 @@ struct Small {
     float G[C];              // log2(e) x in-chunk cumulative log decay (prep, chunk being prepared)
     float bg[C];             // beta_i e^(G_i)
     float Kd[2][C];          // e^(G_last - G_i), 0 beyond the chunk, by chunk parity (for the chain)
+    float Er[C];             // 2^(G_i - G_ref): row factor of the decay (K rows)
+    float Eq[C];             // 2^(G'_i - G_ref): row factor for the read (G' = G_i or G_{i-1})
+    float Ec[C];             // 2^(G_ref - G_j): column factor
+    float ssp[2][128];       // partial sums of squares of the [K;Q] row halves
     float gsum_part[2];      // chain: partial sums of the next chunk's g
     uint64_t mbar[MB_COUNT];
     uint32_t tmem_base;
     int abort;
+    int split_ok;            // the chunk's decay factors factor into row x column exactly
 };
-static_assert(sizeof(Small) <= 4096, "small shared block");
+static_assert(sizeof(Small) <= 5120, "small shared block");
 
 struct TcParams {
     const __nv_bfloat16* q; const __nv_bfloat16* k; const __nv_bfloat16* v;
@@ -138,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
     const uint32_t sbase = smem_u32(sm);
     Small& SS = *reinterpret_cast<Small*>(sm + OFF_SMALL);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wg = tid >> 7;     // 0: chain, 1: prep
+    const int wg = tid >> 7;     // 0: chain, 1-2: prep
     const int lt = tid & 127;    // index within the warpgroup = TMEM lane
     if (p.hdr->err != GDR_OK) return;
 
@@ -165,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
     }
     if (tid == 0) {
         for (int i = 0; i < MB_COUNT; ++i)
-            mbar_init(&SS.mbar[i], (i == MB_PREP || i == MB_PREP + 1) ? 128 : 1);
+            mbar_init(&SS.mbar[i], (i == MB_PREP || i == MB_PREP + 1) ? kPrep : 1);
         SS.abort = 0;
         mbar_init_fence();
     }
@@ -183,17 +190,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
     // wait for a phase of an mbarrier; the whole warpgroup agrees on the outcome
     auto wg_wait = [&](int idx, uint32_t parity, int bar_id) -> bool {
         const bool ok = mbar_wait_bounded(&SS.mbar[idx], parity, kWaitLimitNs);
-        const bool all = named_bar_and(bar_id, 128, (ok && !SS.abort) ? 1 : 0) != 0;
+        const int n = bar_id == kBarPrep ? kPrep : 128;
+        const bool all = named_bar_and(bar_id, n, (ok && !SS.abort) ? 1 : 0) != 0;
         if (!all) SS.abort = 1;
         tc_fence_after();
         return all;
     };
 
-    if (wg == 1) {
-        // ============================ preparation warpgroup ============================
-        const int t = lt;
-        // cp.async plan: this thread copies 16-byte column chunk `cd` of rows r0 + 8 m
-        const int cd = t & 15, r0 = t >> 4;
+    if (wg >= 1) {
+        // ============================ preparation warpgroups ===========================
+        const int pt = tid - 128;      // 0..255
+        const int r = pt & 127;        // TMEM lane / row of [K;Q] / dk or dv row
+        const int hf = pt >> 7;        // which half of the columns this thread takes
+        const int pw = pt >> 5;        // preparation warp 0..7
+        // cp.async plan: this thread copies 16-byte column chunk `cd` of rows r0 + 16 m
+        const int cd = pt & 15, r0 = pt >> 4;
         const __nv_bfloat16* kbase = p.k + (size_t)hk * D + cd * 8;
         const __nv_bfloat16* qbase = p.q + (size_t)hk * D + cd * 8;
         const __nv_bfloat16* vbase = p.v + (size_t)h * D + cd * 8;
@@ -203,8 +214,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_STRIDE + (cd >> 3) * 16384;
             const uint32_t vv = sbase + OFF_V + (c & 1) * V_STRIDE + (cd >> 3) * 8192;
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int i = r0 + 8 * m;
+            for (int m = 0; m < 4; ++m) {
+                const int i = r0 + 16 * m;
                 const bool valid = i < Cc;
                 const long long tok = valid ? tokA + tstep * (c * C + i) : t0;
                 const uint32_t off = sw128(i, cd & 7);
@@ -217,9 +228,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
         cp_async_commit();
         {
             const int Cc0 = min(C, L);
-            if (t < C) {
-                SS.g[0][t] = t < Cc0 ? gate_at(p.g, t) : 0.f;
-                SS.b[0][t] = t < Cc0 ? gate_at(p.beta, t) : 0.f;
+            if (pt < C) {
+                SS.g[0][pt] = pt < Cc0 ? gate_at(p.g, pt) : 0.f;
+                SS.b[0][pt] = pt < Cc0 ? gate_at(p.beta, pt) : 0.f;
             }
         }
         float g_nx = 0.f, b_nx = 0.f;
@@ -236,12 +247,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             if (has_next) {
                 load_chunk(c + 1);
                 const int Cn = min(C, L - (c + 1) * C);
-                g_nx = t < Cn ? gate_at(p.g, (c + 1) * C + t) : 0.f;
-                b_nx = t < Cn ? gate_at(p.beta, (c + 1) * C + t) : 0.f;
+                g_nx = pt < Cn ? gate_at(p.g, (c + 1) * C + pt) : 0.f;
+                b_nx = pt < Cn ? gate_at(p.beta, (c + 1) * C + pt) : 0.f;
             }
             cp_async_commit();
-            // in-chunk cumsum of g (log2 units) while the copies land
-            if (warp == 4) {
+            // in-chunk cumsum of g (log2 units) while the copies land, and whether every decay
+            // factor 2^(G_i - G_j) splits into 2^(G_i - G_ref) 2^(G_ref - G_j) inside the normal
+            // fp32 range (true unless the log2 decay strays more than 110 from G_ref = G_31)
+            if (pw == 0) {
                 const float a0 = SS.g[pb][2 * lane] * kLog2e, a1 = SS.g[pb][2 * lane + 1] * kLog2e;
                 const float pair = a0 + a1;
                 float incl = pair;
@@ -251,32 +264,52 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                     if (lane >= o) incl += y;
                 }
                 const float excl = incl - pair;
-                SS.G[2 * lane] = excl + a0;
-                SS.G[2 * lane + 1] = excl + a0 + a1;
+                const float G0 = excl + a0, G1 = excl + a0 + a1;
+                SS.G[2 * lane] = G0;
+                SS.G[2 * lane + 1] = G1;
+                const float Gref = __shfl_sync(0xffffffffu, G1, 15);  // G_31
+                float dev = fmaxf(fabsf(G0 - Gref), fabsf(G1 - Gref));
+                dev = fmaxf(dev, fabsf(excl - Gref));                // G_{i-1} of the pre-read
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, o));
+                if (lane == 0) SS.split_ok = dev <= 110.f;
             }
             cp_async_wait<1>();
             fence_proxy_async_smem();
-            named_bar(kBarPrep, 128);
+            named_bar(kBarPrep, kPrep);
 
-            // P1: row t of [K; Q]: bf16 -> (L2-normalised) fp16 in place; per-row factors
+            // P1: half row of [K; Q]: bf16 -> (L2-normalised) fp16 in place; per-row factors
             {
-                uint4 vals[16];
+                uint4 vals[8];
                 float ss = 0.f;
+                uint8_t* rowp = KQp + hf * 16384;
 #pragma unroll
-                for (int c16 = 0; c16 < 16; ++c16) {
-                    vals[c16] = *reinterpret_cast<const uint4*>(KQp + (c16 >> 3) * 16384 +
-                                                                sw128(t, c16 & 7));
-                    const uint32_t w[4] = {vals[c16].x, vals[c16].y, vals[c16].z, vals[c16].w};
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    vals[c8] = *reinterpret_cast<const uint4*>(rowp + sw128(r, c8));
+                    const uint32_t w[4] = {vals[c8].x, vals[c8].y, vals[c8].z, vals[c8].w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 x = unpack_bf16x2(w[e]);
                         ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
                     }
                 }
-                const float inv = p.qk_l2norm ? 1.f / fmaxf(sqrtf(ss), kNormEps) : 1.f;
+                SS.ssp[hf][r] = ss;
+                if (pt < C) {
+                    const float Gref = SS.G[31];
+                    const float Gi = SS.G[pt];
+                    const float Gr = p.read_pre ? (pt > 0 ? SS.G[pt - 1] : 0.f) : Gi;
+                    SS.Kd[pb][pt] = pt < Cc ? ex2(SS.G[Cc - 1] - Gi) : 0.f;
+                    SS.bg[pt] = SS.b[pb][pt] * ex2(Gi);
+                    SS.Er[pt] = ex2(Gi - Gref);
+                    SS.Eq[pt] = ex2(Gr - Gref);
+                    SS.Ec[pt] = ex2(Gref - Gi);
+                }
+                named_bar(kBarPrep, kPrep);
+                const float tot = SS.ssp[0][r] + SS.ssp[1][r];
+                const float inv = p.qk_l2norm ? 1.f / fmaxf(sqrtf(tot), kNormEps) : 1.f;
 #pragma unroll
-                for (int c16 = 0; c16 < 16; ++c16) {
-                    const uint32_t w[4] = {vals[c16].x, vals[c16].y, vals[c16].z, vals[c16].w};
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const uint32_t w[4] = {vals[c8].x, vals[c8].y, vals[c8].z, vals[c8].w};
                     float f[8];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -284,21 +317,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                         f[2 * e] = x.x * inv;
                         f[2 * e + 1] = x.y * inv;
                     }
-                    *reinterpret_cast<uint4*>(KQp + (c16 >> 3) * 16384 + sw128(t, c16 & 7)) =
-                        h8(f, rflags);
-                }
-                if (t < C) {
-                    SS.Kd[pb][t] = t < Cc ? ex2(SS.G[Cc - 1] - SS.G[t]) : 0.f;
-                    SS.bg[t] = SS.b[pb][t] * ex2(SS.G[t]);
+                    *reinterpret_cast<uint4*>(rowp + sw128(r, c8)) = h8(f, rflags);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            named_bar(kBarPrep, 128);
+            named_bar(kBarPrep, kPrep);
             tc_fence_after();
 
             // P2: D0 = [K;Q] K^T  (M=128, N=64, K=128)
-            if (t == 0) {
+            if (pt == 0) {
                 const uint32_t id = idesc_f32acc(128, 64, false, false, false);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -310,52 +338,54 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             }
             if (!wg_wait(MB_M0, c & 1, kBarPrep)) { fail = true; break; }
 
-            // P3: A rows (fp32) and P rows (fp16) from D0; Q -> Q~ = scale e^(G') Q in place
+            // P3: columns [32 hf, 32 hf + 32) of row r of D0: A (fp32, rows 0-63) and
+            //     P (fp16, rows 64-127); half of Q -> Q~ = scale e^(G') Q in place
             {
-                const int i = t & 63;
-                const bool isK = t < C;
-                const float Gi = SS.G[i];
-                const float Gr = p.read_pre ? (i > 0 ? SS.G[i - 1] : 0.f) : Gi;
-                const float bi = SS.b[pb][i];
+                const int i = r & 63;
+                const bool isK = r < C;
+                const bool split = SS.split_ok;
                 float* As = reinterpret_cast<float*>(sm + OFF_AS);
+                uint32_t rr[32];
+                tmem_ld32(tlane + TM_D0 + hf * 32, rr);
+                tmem_wait_ld();
+                if (isK) {
+                    const float Gi = SS.G[i];
+                    const float bi = SS.b[pb][i];
+                    const float fi = bi * SS.Er[i];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32];
-                    tmem_ld32(tlane + TM_D0 + half * 32, r);
-                    tmem_wait_ld();
-                    if (isK) {
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        float a[4];
 #pragma unroll
-                        for (int e4 = 0; e4 < 8; ++e4) {
-                            float a[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const int j = half * 32 + e4 * 4 + u;
-                                a[u] = j < i ? bi * u2f(r[e4 * 4 + u]) * ex2(Gi - SS.G[j]) : 0.f;
-                            }
-                            *reinterpret_cast<float4*>(f32sw(As, i, half * 32 + e4 * 4)) =
-                                make_float4(a[0], a[1], a[2], a[3]);
+                        for (int u = 0; u < 4; ++u) {
+                            const int j = hf * 32 + e4 * 4 + u;
+                            const float v = split ? fi * u2f(rr[e4 * 4 + u]) * SS.Ec[j]
+                                                  : bi * u2f(rr[e4 * 4 + u]) * ex2(Gi - SS.G[j]);
+                            a[u] = j < i ? v : 0.f;
                         }
-                    } else {
-#pragma unroll
-                        for (int e8 = 0; e8 < 4; ++e8) {
-                            float pv[8];
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) {
-                                const int j = half * 32 + e8 * 8 + u;
-                                const bool on = p.read_pre ? (j < i) : (j <= i);
-                                pv[u] = on ? p.scale * u2f(r[e8 * 8 + u]) * ex2(Gr - SS.G[j]) : 0.f;
-                            }
-                            *reinterpret_cast<uint4*>(sm + OFF_P + pb * 8192 +
-                                                      sw128(i, half * 4 + e8)) = h8(pv, rflags);
-                        }
+                        *reinterpret_cast<float4*>(f32sw(As, i, hf * 32 + e4 * 4)) =
+                            make_float4(a[0], a[1], a[2], a[3]);
                     }
-                }
-                if (!isK) {
+                } else {
+                    const float Gr = p.read_pre ? (i > 0 ? SS.G[i - 1] : 0.f) : SS.G[i];
+                    const float fi = p.scale * SS.Eq[i];
+#pragma unroll
+                    for (int e8 = 0; e8 < 4; ++e8) {
+                        float pv[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int j = hf * 32 + e8 * 8 + u;
+                            const bool on = p.read_pre ? (j < i) : (j <= i);
+                            const float v = split ? fi * u2f(rr[e8 * 8 + u]) * SS.Ec[j]
+                                                  : p.scale * u2f(rr[e8 * 8 + u]) * ex2(Gr - SS.G[j]);
+                            pv[u] = on ? v : 0.f;
+                        }
+                        *reinterpret_cast<uint4*>(sm + OFF_P + pb * 8192 + sw128(i, hf * 4 + e8)) =
+                            h8(pv, rflags);
+                    }
                     const __half2 f2 = __float2half2_rn(p.scale * ex2(Gr));
 #pragma unroll
-                    for (int c16 = 0; c16 < 16; ++c16) {
-                        uint4* ptr = reinterpret_cast<uint4*>(KQp + (c16 >> 3) * 16384 + 8192 +
-                                                              sw128(i, c16 & 7));
+                    for (int c8 = 0; c8 < 8; ++c8) {
+                        uint4* ptr = reinterpret_cast<uint4*>(KQp + hf * 16384 + 8192 + sw128(i, c8));
                         uint4 u = *ptr;
                         __half2* hv = reinterpret_cast<__half2*>(&u);
 #pragma unroll
@@ -365,18 +395,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                 }
             }
             tc_fence_before();
-            named_bar(kBarPrep, 128);
+            named_bar(kBarPrep, kPrep);
 
             // P4: T = (I + A)^-1, blocked by 16: diagonal blocks by substitution, then the
             //     off-diagonal blocks T_rs = -T_rr sum_{l=s}^{r-1} A_rl T_ls by block distance
             {
                 float* As = reinterpret_cast<float*>(sm + OFF_AS);
                 float* Ts = reinterpret_cast<float*>(sm + OFF_TWU);
-                const int wp = warp - 4;
-                if (lane < 16) {
-                    // column `cl` of the inverse of the unit-lower 16x16 block `wp`, by
+                if (pw < 4 && lane < 16) {
+                    // column `cl` of the inverse of the unit-lower 16x16 block `pw`, by
                     // right-looking substitution (each new x_j is pushed into later rows)
-                    const int b0 = wp * 16, cl = lane;
+                    const int b0 = pw * 16, cl = lane;
                     float acc[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) acc[i] = 0.f;
@@ -389,12 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                             acc[i] = fmaf(*f32sw(As, b0 + i, b0 + jc), xj, acc[i]);
                     }
                 }
-                named_bar(kBarPrep, 128);
+                named_bar(kBarPrep, kPrep);
                 const int gq = lane >> 2, tq = lane & 3;
-                float* Rs = reinterpret_cast<float*>(sm + OFF_RS) + wp * 256;
+                float* Rs = reinterpret_cast<float*>(sm + OFF_RS) + (pw & 3) * 256;
                 for (int dist = 1; dist < 4; ++dist) {
-                    if (wp < 4 - dist) {
-                        const int sblk = wp, rblk = wp + dist;
+                    if (pw < 4 - dist) {
+                        const int sblk = pw, rblk = pw + dist;
                         float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                         for (int l = sblk; l < rblk; ++l) {
 #pragma unroll
@@ -439,51 +468,51 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                         }
 #pragma unroll
                         for (int nt = 0; nt < 2; ++nt) {
-                            const int rr = 16 * rblk + gq, cc = 16 * sblk + 8 * nt + 2 * tq;
-                            *f32sw(Ts, rr, cc) = -acc2[nt][0];
-                            *f32sw(Ts, rr, cc + 1) = -acc2[nt][1];
-                            *f32sw(Ts, rr + 8, cc) = -acc2[nt][2];
-                            *f32sw(Ts, rr + 8, cc + 1) = -acc2[nt][3];
+                            const int rr2 = 16 * rblk + gq, cc = 16 * sblk + 8 * nt + 2 * tq;
+                            *f32sw(Ts, rr2, cc) = -acc2[nt][0];
+                            *f32sw(Ts, rr2, cc + 1) = -acc2[nt][1];
+                            *f32sw(Ts, rr2 + 8, cc) = -acc2[nt][2];
+                            *f32sw(Ts, rr2 + 8, cc + 1) = -acc2[nt][3];
                         }
                         __syncwarp();
                     }
-                    named_bar(kBarPrep, 128);
+                    named_bar(kBarPrep, kPrep);
                 }
-                // T -> T diag(beta e^G) (fp16) and T diag(beta) (bf16): row i, 32 columns
-                const int i = t >> 1, half = t & 1;
-                float tv[32];
+                // T -> T diag(beta e^G) (fp16) and T diag(beta) (bf16): row i, 16 columns
+                const int i = pt >> 2, qq = pt & 3;
+                float tv[16];
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 v4 = *reinterpret_cast<const float4*>(f32sw(Ts, i, half * 32 + e4 * 4));
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float4 v4 = *reinterpret_cast<const float4*>(f32sw(Ts, i, qq * 16 + e4 * 4));
                     tv[e4 * 4 + 0] = v4.x; tv[e4 * 4 + 1] = v4.y;
                     tv[e4 * 4 + 2] = v4.z; tv[e4 * 4 + 3] = v4.w;
                 }
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if (half * 32 + e > i) tv[e] = 0.f;  // blocks above the diagonal are never written
-                named_bar(kBarPrep, 128);  // T is read completely before the 16-bit tiles overwrite it
+                for (int e = 0; e < 16; ++e)
+                    if (qq * 16 + e > i) tv[e] = 0.f;  // blocks above the diagonal are never written
+                named_bar(kBarPrep, kPrep);  // T is read completely before the 16-bit tiles overwrite it
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
+                for (int m = 0; m < 2; ++m) {
                     uint32_t w4[4], u4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int jj = m * 8 + 2 * e, j = half * 32 + jj;
+                        const int jj = m * 8 + 2 * e, j = qq * 16 + jj;
                         w4[e] = h2(tv[jj] * SS.bg[j], tv[jj + 1] * SS.bg[j + 1], rflags);
                         u4[e] = pack_bf16x2(tv[jj] * SS.b[pb][j], tv[jj + 1] * SS.b[pb][j + 1]);
                     }
-                    *reinterpret_cast<uint4*>(sm + OFF_TWU + sw128(i, half * 4 + m)) =
+                    *reinterpret_cast<uint4*>(sm + OFF_TWU + sw128(i, qq * 2 + m)) =
                         make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    *reinterpret_cast<uint4*>(sm + OFF_TWU + 8192 + sw128(i, half * 4 + m)) =
+                    *reinterpret_cast<uint4*>(sm + OFF_TWU + 8192 + sw128(i, qq * 2 + m)) =
                         make_uint4(u4[0], u4[1], u4[2], u4[3]);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            named_bar(kBarPrep, 128);
+            named_bar(kBarPrep, kPrep);
             tc_fence_after();
 
             // P5: W^T = K^T T_w^T (fp16, into D0) and U~^T = V^T T_u^T (bf16, into DU[pb])
-            if (t == 0) {
+            if (pt == 0) {
                 const uint32_t idw = idesc_f32acc(128, 64, true, false, false);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
@@ -499,24 +528,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             }
             if (!wg_wait(MB_MW, c & 1, kBarPrep)) { fail = true; break; }
 
-            // P6: -W^T rows -> WN[pb] (B operand, MN-major); hand the chunk to the chain
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r[32];
-                tmem_ld32(tlane + TM_D0 + half * 32, r);
+            // P6: columns [32 hf, +32) of -W^T row r -> WN[pb] (B operand, MN-major)
+            {
+                uint32_t rr[32];
+                tmem_ld32(tlane + TM_D0 + hf * 32, rr);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e8 = 0; e8 < 4; ++e8) {
                     float f[8];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) f[u] = -u2f(r[e8 * 8 + u]);
-                    *reinterpret_cast<uint4*>(sm + OFF_WN + pb * 16384 + sw128(t, half * 4 + e8)) =
+                    for (int u = 0; u < 8; ++u) f[u] = -u2f(rr[e8 * 8 + u]);
+                    *reinterpret_cast<uint4*>(sm + OFF_WN + pb * 16384 + sw128(r, hf * 4 + e8)) =
                         h8(f, rflags);
                 }
             }
-            if (has_next && t < C) {
-                SS.g[pb ^ 1][t] = g_nx;
-                SS.b[pb ^ 1][t] = b_nx;
+            if (has_next && pt < C) {
+                SS.g[pb ^ 1][pt] = g_nx;
+                SS.b[pb ^ 1][pt] = b_nx;
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -583,11 +611,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
 
             // C2: V'^T -> fp16 packed in TMEM, plain (output) and scaled by Kd (state update)
             {
+                uint32_t rv[2][32];
+                tmem_ld32(tlane + TM_DU + pb * 64, rv[0]);
+                tmem_ld32(tlane + TM_DU + pb * 64 + 32, rv[1]);
+                tmem_wait_ld();
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32], pk[16], ps[16];
-                    tmem_ld32(tlane + TM_DU + pb * 64 + half * 32, r);
-                    tmem_wait_ld();
+                    uint32_t pk[16], ps[16];
+                    const uint32_t* r = rv[half];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const float a = u2f(r[2 * e]), b = u2f(r[2 * e + 1]);
@@ -629,11 +660,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                 __nv_bfloat16* orow = p.o + (tokA + tstep * (long long)(c * C)) * p.Hv * D +
                                       (size_t)h * D + (j & ~1);
                 const bool odd = j & 1;
+                uint32_t ro[2][32];
+                tmem_ld32(tlane + TM_DO, ro[0]);
+                tmem_ld32(tlane + TM_DO + 32, ro[1]);
+                tmem_wait_ld();
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32];
-                    tmem_ld32(tlane + TM_DO + half * 32, r);
-                    tmem_wait_ld();
+                    const uint32_t* r = ro[half];
 #pragma unroll
                     for (int m = 0; m < 16; ++m) {
                         const float a = u2f(r[2 * m]), b = u2f(r[2 * m + 1]);  // O[i0][j], O[i0+1][j]
@@ -653,21 +686,28 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                 }
                 const float gam = has_next ? ex2((SS.gsum_part[0] + SS.gsum_part[1]) * kLog2e) : 1.f;
 #pragma unroll
-                for (int d0 = 0; d0 < D; d0 += 32) {
-                    uint32_t r[32], hb[16];
-                    tmem_ld32(tlane + TM_HM + d0, r);
+                for (int d0 = 0; d0 < D; d0 += 64) {
+                    uint32_t r2[2][32];
+                    tmem_ld32(tlane + TM_HM + d0, r2[0]);
+                    tmem_ld32(tlane + TM_HM + d0 + 32, r2[1]);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) hb[e] = h2(u2f(r[2 * e]), u2f(r[2 * e + 1]), rflags);
-                    tmem_st16(tlane + TM_HB + d0 / 2, hb);
-                    if (has_next) {
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t (&r)[32] = r2[hh];
+                        const int dd = d0 + hh * 32;
+                        uint32_t hb[16];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(u2f(r[e]) * gam);
-                        tmem_st32(tlane + TM_HM + d0, r);
-                    } else if (p.S_final) {
+                        for (int e = 0; e < 16; ++e) hb[e] = h2(u2f(r[2 * e]), u2f(r[2 * e + 1]), rflags);
+                        tmem_st16(tlane + TM_HB + dd / 2, hb);
+                        if (has_next) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            p.S_final[sb + (size_t)(d0 + e) * D + j] = u2f(r[e]);
+                            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(u2f(r[e]) * gam);
+                            tmem_st32(tlane + TM_HM + dd, r);
+                        } else if (p.S_final) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                p.S_final[sb + (size_t)(dd + e) * D + j] = u2f(r[e]);
+                        }
                     }
                 }
                 tmem_wait_st();
@@ -678,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
         }
     }
 
-    if (fail && (tid == 0 || tid == 128)) atomicExch(&p.hdr->err, (int)GDR_ERR_TIMEOUT);
+    if (fail && (tid == 0 || tid == 128 || tid == 256)) atomicExch(&p.hdr->err, (int)GDR_ERR_TIMEOUT);
     tc_fence_before();
     if (__syncthreads_or((rflags & 0x80008000u) ? 1 : 0) && tid == 0)
         atomicCAS(&p.hdr->err, (int)GDR_OK, (int)GDR_ERR_RANGE);
