@@ -15,7 +15,8 @@ F32, BF16 = 0, 1
 READ_POST, READ_PRE = 0, 1
 
 # every symbol include/gdr.h declares
-EXPORTS = ["gdr_chunk_fwd_workspace_size", "gdr_chunk_fwd", "gdr_chunk_fwd_path",
+EXPORTS = ["gdr_chunk_fwd_workspace_size", "gdr_chunk_fwd", "gdr_chunk_fwd_noalloc",
+           "gdr_chunk_fwd_path",
            "gdr_decode_step", "gdr_status_string", "gdr_read_device_error", "gdr_version"]
 
 
@@ -51,6 +52,8 @@ def _declare(lib):
     lib.gdr_chunk_fwd_workspace_size.restype = sz
     lib.gdr_chunk_fwd.argtypes = [ctypes.POINTER(ChunkArgs)] + [vp] * 10 + [sz, vp]
     lib.gdr_chunk_fwd.restype = ctypes.c_int
+    lib.gdr_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(ChunkArgs)] + [vp] * 10
+    lib.gdr_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.gdr_chunk_fwd_path.argtypes = [ctypes.POINTER(ChunkArgs)]
     lib.gdr_chunk_fwd_path.restype = ctypes.c_char_p
     lib.gdr_decode_step.argtypes = [ctypes.POINTER(DecodeArgs)] + [vp] * 8

@@ -123,6 +123,37 @@ gdr_status gdr_chunk_fwd(const gdr_chunk_args* args,
                          void* o, float* S_final,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * gdr_chunk_fwd without a caller-provided workspace.  (No counterpart on the pages: this is
+ * a convenience of this library.)
+ *
+ * For callers that cannot allocate device memory: a serving process whose GPU memory is
+ * reserved up front by its own pool (cudaMalloc may fail there, and it synchronises the
+ * device), code inside a framework hook or callback where the CUDA allocator may not be
+ * called, or a plain-C caller without a device allocator.  The caller still passes the
+ * inputs and outputs exactly as for gdr_chunk_fwd; the scratch is a static device array of
+ * GDR_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until exit.
+ *
+ * - Calls whose scratch need (gdr_chunk_fwd_workspace_size) exceeds the array return
+ *   GDR_ERR_WORKSPACE and enqueue nothing.  The tensor-core path needs only
+ *   256 + 8 (n_seqs + 1) + 4 (ceil(B*T / chunk) + n_seqs) bytes; the CUDA-core path
+ *   additionally 4 B*T Hv (dk + dv + 1) bytes, so it fits only small problems.
+ * - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *   with that device current; make that first call before any stream capture.
+ * - All calls on a device share the one array: calls that overlap on the GPU (different
+ *   streams, or different host threads, without ordering between them) race and may
+ *   corrupt each other's results.  Each call rewrites every scratch field it reads, so a
+ *   previous call's contents never leak into the next.
+ * - The device error word lives in the shared array, so gdr_read_device_error cannot be
+ *   used with this entry point.
+ */
+#define GDR_NOALLOC_SCRATCH_BYTES (4u << 20)
+gdr_status gdr_chunk_fwd_noalloc(const gdr_chunk_args* args,
+                                 const void* q, const void* k, const void* v,
+                                 const void* g, const void* beta,
+                                 const float* S0, const int32_t* cu_seqlens,
+                                 void* o, float* S_final, void* stream);
+
 /* Name of the kernel path gdr_chunk_fwd takes for these arguments: "tc" (tcgen05
  * tensor-core kernels), "simt" (fp32 CUDA-core kernels) or NULL if unsupported. */
 const char* gdr_chunk_fwd_path(const gdr_chunk_args* args);
