@@ -47,6 +47,10 @@
 // The state H is kept transposed in TMEM (lane = dv, column = dk).  After each chunk the
 // chain reads it once, writes the fp16 copy the next chunk's MMAs consume, and scales it
 // in place by the next chunk's total decay, so the next state update accumulates onto it.
+#include <cuda.h>
+
+#include <cstring>
+
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -89,7 +93,14 @@ constexpr uint32_t TM_VS = 480;   // V'^T scaled by e^(G_C - G_i), fp16 packed (
 constexpr uint32_t TM_COLS = 512;
 
 // mbarriers
-enum { MB_M0 = 0, MB_MW = 1, MB_M1 = 2, MB_M3 = 3 /* x2 */, MB_PREP = 5 /* x2 */, MB_COUNT = 7 };
+enum {
+    MB_M0 = 0, MB_MW = 1, MB_M1 = 2,
+    MB_M3 = 3,    // x2: state update of a chunk done (by chunk parity)
+    MB_PREP = 5,  // x2: chunk prepared (by chunk parity)
+    MB_LD = 7,    // x3: K, Q, V tiles of a chunk landed (by K/Q buffer)
+    MB_CD = 10,   // x2: chain finished with a chunk's buffers (by chunk parity)
+    MB_COUNT = 12
+};
 
 struct Small {
     float g[2][C], b[2][C];  // raw gates by chunk parity (prep)
@@ -113,7 +124,7 @@ struct TcParams {
     const void* g; const void* beta; const float* S0;
     __nv_bfloat16* o; float* S_final;
     WsHeader* hdr; const int32_t* cu;
-    int Hk, Hv, read_pre, qk_l2norm, reverse, o_acc;
+    int Hk, Hv, read_pre, qk_l2norm, reverse, o_acc, use_tma;
     gdr_dtype gt;
     float scale;
 };
@@ -138,7 +149,9 @@ __device__ __forceinline__ float* f32sw(float* base, int i, int j) {
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
-__global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
+               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -172,7 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
     }
     if (tid == 0) {
         for (int i = 0; i < MB_COUNT; ++i)
-            mbar_init(&SS.mbar[i], (i == MB_PREP || i == MB_PREP + 1) ? kPrep : 1);
+            mbar_init(&SS.mbar[i], (i == MB_PREP || i == MB_PREP + 1) ? kPrep
+                                   : (i == MB_CD || i == MB_CD + 1)  ? 128
+                                                                     : 1);
         SS.abort = 0;
         mbar_init_fence();
     }
@@ -210,6 +225,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
         const __nv_bfloat16* vbase = p.v + (size_t)h * D + cd * 8;
         const long long kq_tok = (long long)p.Hk * D, v_tok = (long long)p.Hv * D;
         auto load_chunk = [&](int c) {
+            if (p.use_tma) {  // forward scans: six 8 KB tensor tiles, issued by one thread
+                if (pt == 0) {
+                    uint64_t* bar = &SS.mbar[MB_LD + c % 3];
+                    const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
+                    const uint32_t vv = sbase + OFF_V + (c & 1) * V_STRIDE;
+                    const int z = (int)(t0 + (long long)c * C);
+                    mbar_expect_tx(bar, 6 * 8192);
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        tma_load_3d(kq + half * 16384, &tm_k, half * 64, hk, z, bar);
+                        tma_load_3d(kq + half * 16384 + 8192, &tm_q, half * 64, hk, z, bar);
+                        tma_load_3d(vv + half * 8192, &tm_v, half * 64, h, z, bar);
+                    }
+                }
+                return;
+            }
             const int Cc = min(C, L - c * C);
             const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_STRIDE + (cd >> 3) * 16384;
             const uint32_t vv = sbase + OFF_V + (c & 1) * V_STRIDE + (cd >> 3) * 8192;
@@ -225,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             }
         };
         load_chunk(0);
-        cp_async_commit();
+        if (!p.use_tma) cp_async_commit();
         {
             const int Cc0 = min(C, L);
             if (pt < C) {
@@ -242,15 +273,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             const int Cc = min(C, L - c * C);
             const bool has_next = c + 1 < nchunks;
 
-            // P0: the buffers of chunk c-2 are released once its state update completed
-            if (c >= 2 && !wg_wait(MB_M3 + pb, ((c >> 1) & 1) ^ 1, kBarPrep)) { fail = true; break; }
+            // P0: the buffers of chunk c-2 are released once the chain is done with them
+            if (c >= 2 && !wg_wait(MB_CD + pb, ((c >> 1) & 1) ^ 1, kBarPrep)) { fail = true; break; }
             if (has_next) {
                 load_chunk(c + 1);
                 const int Cn = min(C, L - (c + 1) * C);
                 g_nx = pt < Cn ? gate_at(p.g, (c + 1) * C + pt) : 0.f;
                 b_nx = pt < Cn ? gate_at(p.beta, (c + 1) * C + pt) : 0.f;
             }
-            cp_async_commit();
+            if (!p.use_tma) cp_async_commit();
             // in-chunk cumsum of g (log2 units) while the copies land, and whether every decay
             // factor 2^(G_i - G_j) splits into 2^(G_i - G_ref) 2^(G_ref - G_j) inside the normal
             // fp32 range (true unless the log2 decay strays more than 110 from G_ref = G_31)
@@ -274,9 +305,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                 for (int o = 16; o > 0; o >>= 1) dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, o));
                 if (lane == 0) SS.split_ok = dev <= 110.f;
             }
-            cp_async_wait<1>();
+            bool landed = true;
+            if (p.use_tma)
+                landed = mbar_wait_bounded(&SS.mbar[MB_LD + c % 3], (uint32_t)((c / 3) & 1),
+                                           kWaitLimitNs);
+            else
+                cp_async_wait<1>();
             fence_proxy_async_smem();
-            named_bar(kBarPrep, kPrep);
+            if (!named_bar_and(kBarPrep, kPrep, (landed && !SS.abort) ? 1 : 0)) {
+                SS.abort = 1;
+                fail = true;
+                break;
+            }
 
             // P1: half row of [K; Q]: bf16 -> (L2-normalised) fp16 in place; per-row factors
             {
@@ -307,6 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                 named_bar(kBarPrep, kPrep);
                 const float tot = SS.ssp[0][r] + SS.ssp[1][r];
                 const float inv = p.qk_l2norm ? 1.f / fmaxf(sqrtf(tot), kNormEps) : 1.f;
+                // rows past the chunk (tensor tiles carry the following tokens there) become 0
+                const bool live = (r & 63) < Cc;
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
                     const uint32_t w[4] = {vals[c8].x, vals[c8].y, vals[c8].z, vals[c8].w};
@@ -314,10 +356,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 x = unpack_bf16x2(w[e]);
-                        f[2 * e] = x.x * inv;
-                        f[2 * e + 1] = x.y * inv;
+                        f[2 * e] = live ? x.x * inv : 0.f;
+                        f[2 * e + 1] = live ? x.y * inv : 0.f;
                     }
                     *reinterpret_cast<uint4*>(rowp + sw128(r, c8)) = h8(f, rflags);
+                }
+                for (int idx = pt; idx < (C - Cc) * 16; idx += kPrep) {  // V rows past the chunk
+                    const int i = Cc + (idx >> 4), c16 = idx & 15;
+                    *reinterpret_cast<uint4*>(sm + OFF_V + pb * V_STRIDE + (c16 >> 3) * 8192 +
+                                              sw128(i, c16 & 7)) = make_uint4(0, 0, 0, 0);
                 }
             }
             fence_proxy_async_smem();
@@ -554,7 +601,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
     } else {
         // =============================== chain warpgroup ===============================
         const int j = lt;  // dv column = TMEM lane
-        const long long o_step = tstep * (long long)p.Hv * D;  // elements between consecutive positions
         {
             // initial state -> TM_HM (pre-scaled by chunk 0's total decay), TM_HB (fp16)
             const float gv = lt < min(C, L) ? gate_at(p.g, lt) : 0.f;
@@ -655,32 +701,42 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
             }
             if (!wg_wait(MB_M3 + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
 
-            // C4: O -> global (bf16 pairs); state -> fp16 copy, pre-scaled for the next chunk
+            // C4: O -> staged in WN[pb] (row per token) -> bulk copies to global; state ->
+            //     fp16 copy, pre-scaled for the next chunk
             {
-                __nv_bfloat16* orow = p.o + (tokA + tstep * (long long)(c * C)) * p.Hv * D +
-                                      (size_t)h * D + (j & ~1);
-                const bool odd = j & 1;
+                uint8_t* stage = sm + OFF_WN + pb * 16384;
                 uint32_t ro[2][32];
                 tmem_ld32(tlane + TM_DO, ro[0]);
                 tmem_ld32(tlane + TM_DO + 32, ro[1]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const uint32_t* r = ro[half];
+                for (int half = 0; half < 2; ++half)
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        const float a = u2f(r[2 * m]), b = u2f(r[2 * m + 1]);  // O[i0][j], O[i0+1][j]
-                        const float recv = __shfl_xor_sync(0xffffffffu, odd ? a : b, 1);
-                        const int i = half * 32 + 2 * m + (odd ? 1 : 0);
-                        if (i < Cc) {
-                            uint32_t* dst = reinterpret_cast<uint32_t*>(orow + o_step * i);
-                            float2 val = odd ? make_float2(recv, b) : make_float2(a, recv);
-                            if (p.o_acc) {
-                                const float2 old = unpack_bf16x2(*dst);
-                                val.x += old.x;
-                                val.y += old.y;
+                    for (int m = 0; m < 32; ++m)
+                        *reinterpret_cast<__nv_bfloat16*>(stage + (half * 32 + m) * 256 + j * 2) =
+                            __float2bfloat16_rn(u2f(ro[half][m]));
+                fence_proxy_async_smem();
+                named_bar(kBarChain, 128);
+                if (lt < Cc) {
+                    const long long tok = tokA + tstep * (long long)(c * C + lt);
+                    __nv_bfloat16* dst = p.o + ((size_t)tok * p.Hv + h) * D;
+                    if (!p.o_acc) {
+                        bulk_store(dst, sbase + OFF_WN + pb * 16384 + lt * 256, 256);
+                        bulk_commit();
+                    } else {
+#pragma unroll 4
+                        for (int c16 = 0; c16 < 16; ++c16) {
+                            const uint4 a = *reinterpret_cast<const uint4*>(stage + lt * 256 + c16 * 16);
+                            uint4* dp = reinterpret_cast<uint4*>(dst + c16 * 8);
+                            const uint4 b = *dp;
+                            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+                            uint32_t ow[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 x = unpack_bf16x2(aw[e]), y = unpack_bf16x2(bw[e]);
+                                ow[e] = pack_bf16x2(x.x + y.x, x.y + y.y);
                             }
-                            *dst = pack_bf16x2(val.x, val.y);
+                            *dp = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                         }
                     }
                 }
@@ -711,6 +767,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
                     }
                 }
                 tmem_wait_st();
+                if (lt < Cc && !p.o_acc) bulk_wait_read();
+                mbar_arrive(&SS.mbar[MB_CD + pb]);
             }
             tc_fence_before();
             named_bar(kBarChain, 128);
@@ -723,6 +781,41 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fused_tc(TcParams p) {
     if (__syncthreads_or((rflags & 0x80008000u) ? 1 : 0) && tid == 0)
         atomicCAS(&p.hdr->err, (int)GDR_OK, (int)GDR_ERR_RANGE);
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda)
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static bool looked = false;
+    if (!looked) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+        looked = true;
+    }
+    return fn;
+}
+
+// [tokens][heads][128] bf16 viewed as a 3-D tensor (128, heads, tokens); box 64 x 1 x 64
+// with the 128-byte swizzle, i.e. one 8 KB K-major atom stack of the kernel's layout.
+bool make_tile_map(CUtensorMap* m, const void* base, int heads, long long tokens) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)tokens};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -746,11 +839,23 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
     p.Hk = a.Hk; p.Hv = a.Hv; p.read_pre = a.read_mode == GDR_READ_PRE;
     p.qk_l2norm = a.qk_l2norm; p.reverse = a.reverse; p.o_acc = a.o_accumulate;
     p.gt = a.gate_dtype; p.scale = a.scale;
+    CUtensorMap tq, tk, tv;
+    memset(&tq, 0, sizeof(tq));
+    memset(&tk, 0, sizeof(tk));
+    memset(&tv, 0, sizeof(tv));
+    const long long T_tot = (long long)a.B * a.T;
+    p.use_tma = 0;
+    if (!a.reverse && T_tot > 0) {  // reversed scans gather rows with cp.async instead
+        if (!make_tile_map(&tq, q, a.Hk, T_tot) || !make_tile_map(&tk, k, a.Hk, T_tot) ||
+            !make_tile_map(&tv, v, a.Hv, T_tot))
+            return GDR_ERR_CUDA;
+        p.use_tma = 1;
+    }
     if (cudaFuncSetAttribute(chunk_fused_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
     dim3 grid((unsigned)a.n_seqs, (unsigned)a.Hv);
-    chunk_fused_tc<<<grid, kThreads, SMEM_BYTES, st>>>(p);
+    chunk_fused_tc<<<grid, kThreads, SMEM_BYTES, st>>>(p, tq, tk, tv);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 
