@@ -76,9 +76,9 @@ constexpr uint32_t V_STRIDE = 16384;
 constexpr uint32_t OFF_TWU = 131072;   // T diag(beta e^G) fp16 [i][j] | T diag(beta) bf16 [i][j];
                                        // holds the fp32 T [64][64] during the solve
 constexpr uint32_t OFF_AS = 147456;    // A fp32 [64][64]
-constexpr uint32_t OFF_RS = 163840;    // solve scratch: 4 warps x 16x16 fp32
+constexpr uint32_t OFF_RS = 163840;    // the four diagonal 16x16 blocks of A, transposed (fp32)
 constexpr uint32_t OFF_P = 167936;     // 2 x 8 KB: P fp16 [i][j]
-constexpr uint32_t OFF_WN = 184320;    // 2 x 16 KB: -W^T fp16 [dk][tok]
+constexpr uint32_t OFF_WN = 184320;    // 2 x 16 KB: -W^T fp16 [dk][tok]; output staging
 constexpr uint32_t OFF_SMALL = 217088;
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + 5120 + 1024;
 
@@ -411,6 +411,13 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         }
                         *reinterpret_cast<float4*>(f32sw(As, i, hf * 32 + e4 * 4)) =
                             make_float4(a[0], a[1], a[2], a[3]);
+                        // the diagonal 16x16 block of row i, transposed, for the substitution
+                        const int jb = hf * 32 + e4 * 4;
+                        if ((jb >> 4) == (i >> 4)) {
+                            float* at = reinterpret_cast<float*>(sm + OFF_RS) + (i >> 4) * 256;
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) at[((jb + u) & 15) * 16 + (i & 15)] = a[u];
+                        }
                     }
                 } else {
                     const float Gr = p.read_pre ? (i > 0 ? SS.G[i - 1] : 0.f) : SS.G[i];
@@ -444,15 +451,19 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             tc_fence_before();
             named_bar(kBarPrep, kPrep);
 
-            // P4: T = (I + A)^-1, blocked by 16: diagonal blocks by substitution, then the
-            //     off-diagonal blocks T_rs = -T_rr sum_{l=s}^{r-1} A_rl T_ls by block distance
+            // P4: T = (I + A)^-1 by 16-blocks.  Stage 0: the four diagonal inverses T_bb by
+            //     right-looking substitution (one warp each, on the transposed block);
+            //     stage A: E_rl = T_rr A_rl for r > l, in place over A (six warps);
+            //     stage d = 1..3: T_rs = -sum_{l=s}^{r-1} E_rl T_ls for r - s = d.
+            //     The warp MMAs (tf32, m16n8k8) pair each thread's two k slots with two
+            //     adjacent columns, so every A fragment comes in two 8-byte loads.
             {
                 float* As = reinterpret_cast<float*>(sm + OFF_AS);
                 float* Ts = reinterpret_cast<float*>(sm + OFF_TWU);
+                const float* AsT = reinterpret_cast<const float*>(sm + OFF_RS);
                 if (pw < 4 && lane < 16) {
-                    // column `cl` of the inverse of the unit-lower 16x16 block `pw`, by
-                    // right-looking substitution (each new x_j is pushed into later rows)
                     const int b0 = pw * 16, cl = lane;
+                    const float* at = AsT + pw * 256;
                     float acc[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) acc[i] = 0.f;
@@ -461,67 +472,60 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         const float xj = jc < cl ? 0.f : (jc == cl ? 1.f : -acc[jc]);
                         *f32sw(Ts, b0 + jc, b0 + cl) = xj;
 #pragma unroll
-                        for (int i = jc + 1; i < 16; ++i)
-                            acc[i] = fmaf(*f32sw(As, b0 + i, b0 + jc), xj, acc[i]);
+                        for (int i4 = (jc + 1) >> 2; i4 < 4; ++i4) {
+                            const float4 a4 = *reinterpret_cast<const float4*>(at + jc * 16 + 4 * i4);
+                            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                if (4 * i4 + u > jc) acc[4 * i4 + u] = fmaf(av[u], xj, acc[4 * i4 + u]);
+                        }
                     }
                 }
                 named_bar(kBarPrep, kPrep);
                 const int gq = lane >> 2, tq = lane & 3;
-                float* Rs = reinterpret_cast<float*>(sm + OFF_RS) + (pw & 3) * 256;
+                // one 16x16x16 product step: acc[nt] += X(rows 16 xr.., cols 16 xc + 8 ks..)
+                //                                      * Z(rows 16 zr + 8 ks.., cols 16 zc + 8 nt..)
+                auto mma_block = [&](float (&acc)[2][4], const float* X, int xr, int xc,
+                                     const float* Z, int zr, int zc) {
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const int col = 16 * xc + 8 * ks + 2 * tq;
+                        const float2 lo = *reinterpret_cast<const float2*>(f32sw(const_cast<float*>(X), 16 * xr + gq, col));
+                        const float2 hi = *reinterpret_cast<const float2*>(f32sw(const_cast<float*>(X), 16 * xr + gq + 8, col));
+                        const uint32_t a[4] = {to_tf32(lo.x), to_tf32(hi.x), to_tf32(lo.y), to_tf32(hi.y)};
+                        const int zrow = 16 * zr + 8 * ks + 2 * tq;
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt) {
+                            const int zc_ = 16 * zc + 8 * nt + gq;
+                            const uint32_t bf[2] = {to_tf32(*f32sw(const_cast<float*>(Z), zrow, zc_)),
+                                                    to_tf32(*f32sw(const_cast<float*>(Z), zrow + 1, zc_))};
+                            mma_tf32_16x8x8(acc[nt], a, bf);
+                        }
+                    }
+                };
+                auto store_block = [&](float* Y, int yr, int yc, const float (&acc)[2][4], float sgn) {
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const int rr = 16 * yr + gq, cc = 16 * yc + 8 * nt + 2 * tq;
+                        *reinterpret_cast<float2*>(f32sw(Y, rr, cc)) = make_float2(sgn * acc[nt][0], sgn * acc[nt][1]);
+                        *reinterpret_cast<float2*>(f32sw(Y, rr + 8, cc)) = make_float2(sgn * acc[nt][2], sgn * acc[nt][3]);
+                    }
+                };
+                if (pw < 6) {  // stage A: (1,0) (2,0) (3,0) (2,1) (3,1) (3,2)
+                    const int rblk = pw < 3 ? pw + 1 : (pw < 5 ? pw - 1 : 3);
+                    const int lblk = pw < 3 ? 0 : (pw < 5 ? 1 : 2);
+                    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                    mma_block(acc, Ts, rblk, rblk, As, rblk, lblk);
+                    __syncwarp();
+                    store_block(As, rblk, lblk, acc, 1.f);
+                }
+                named_bar(kBarPrep, kPrep);
                 for (int dist = 1; dist < 4; ++dist) {
                     if (pw < 4 - dist) {
                         const int sblk = pw, rblk = pw + dist;
                         float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                        for (int l = sblk; l < rblk; ++l) {
-#pragma unroll
-                            for (int ks = 0; ks < 2; ++ks) {
-                                const int ar = 16 * rblk + gq, ac = 16 * l + 8 * ks + tq;
-                                const uint32_t a[4] = {to_tf32(*f32sw(As, ar, ac)),
-                                                       to_tf32(*f32sw(As, ar + 8, ac)),
-                                                       to_tf32(*f32sw(As, ar, ac + 4)),
-                                                       to_tf32(*f32sw(As, ar + 8, ac + 4))};
-#pragma unroll
-                                for (int nt = 0; nt < 2; ++nt) {
-                                    const int br = 16 * l + 8 * ks + tq, bc = 16 * sblk + 8 * nt + gq;
-                                    const uint32_t bf[2] = {to_tf32(*f32sw(Ts, br, bc)),
-                                                            to_tf32(*f32sw(Ts, br + 4, bc))};
-                                    mma_tf32_16x8x8(acc[nt], a, bf);
-                                }
-                            }
-                        }
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt) {
-                            Rs[gq * 16 + 8 * nt + 2 * tq] = acc[nt][0];
-                            Rs[gq * 16 + 8 * nt + 2 * tq + 1] = acc[nt][1];
-                            Rs[(gq + 8) * 16 + 8 * nt + 2 * tq] = acc[nt][2];
-                            Rs[(gq + 8) * 16 + 8 * nt + 2 * tq + 1] = acc[nt][3];
-                        }
-                        __syncwarp();
-                        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-                        for (int ks = 0; ks < 2; ++ks) {
-                            const int ar = 16 * rblk + gq, ac = 16 * rblk + 8 * ks + tq;
-                            const uint32_t a[4] = {to_tf32(*f32sw(Ts, ar, ac)),
-                                                   to_tf32(*f32sw(Ts, ar + 8, ac)),
-                                                   to_tf32(*f32sw(Ts, ar, ac + 4)),
-                                                   to_tf32(*f32sw(Ts, ar + 8, ac + 4))};
-#pragma unroll
-                            for (int nt = 0; nt < 2; ++nt) {
-                                const uint32_t bf[2] = {
-                                    to_tf32(Rs[(8 * ks + tq) * 16 + 8 * nt + gq]),
-                                    to_tf32(Rs[(8 * ks + tq + 4) * 16 + 8 * nt + gq])};
-                                mma_tf32_16x8x8(acc2[nt], a, bf);
-                            }
-                        }
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt) {
-                            const int rr2 = 16 * rblk + gq, cc = 16 * sblk + 8 * nt + 2 * tq;
-                            *f32sw(Ts, rr2, cc) = -acc2[nt][0];
-                            *f32sw(Ts, rr2, cc + 1) = -acc2[nt][1];
-                            *f32sw(Ts, rr2 + 8, cc) = -acc2[nt][2];
-                            *f32sw(Ts, rr2 + 8, cc + 1) = -acc2[nt][3];
-                        }
-                        __syncwarp();
+                        for (int l = sblk; l < rblk; ++l) mma_block(acc, As, rblk, l, Ts, l, sblk);
+                        store_block(Ts, rblk, sblk, acc, -1.f);
                     }
                     named_bar(kBarPrep, kPrep);
                 }
@@ -537,15 +541,23 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
                     if (qq * 16 + e > i) tv[e] = 0.f;  // blocks above the diagonal are never written
+                float bgv[16], bv[16];
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float4 x = *reinterpret_cast<const float4*>(&SS.bg[qq * 16 + 4 * e4]);
+                    const float4 y = *reinterpret_cast<const float4*>(&SS.b[pb][qq * 16 + 4 * e4]);
+                    bgv[4 * e4] = x.x; bgv[4 * e4 + 1] = x.y; bgv[4 * e4 + 2] = x.z; bgv[4 * e4 + 3] = x.w;
+                    bv[4 * e4] = y.x; bv[4 * e4 + 1] = y.y; bv[4 * e4 + 2] = y.z; bv[4 * e4 + 3] = y.w;
+                }
                 named_bar(kBarPrep, kPrep);  // T is read completely before the 16-bit tiles overwrite it
 #pragma unroll
                 for (int m = 0; m < 2; ++m) {
                     uint32_t w4[4], u4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int jj = m * 8 + 2 * e, j = qq * 16 + jj;
-                        w4[e] = h2(tv[jj] * SS.bg[j], tv[jj + 1] * SS.bg[j + 1], rflags);
-                        u4[e] = pack_bf16x2(tv[jj] * SS.b[pb][j], tv[jj + 1] * SS.b[pb][j + 1]);
+                        const int jj = m * 8 + 2 * e;
+                        w4[e] = h2(tv[jj] * bgv[jj], tv[jj + 1] * bgv[jj + 1], rflags);
+                        u4[e] = pack_bf16x2(tv[jj] * bv[jj], tv[jj + 1] * bv[jj + 1]);
                     }
                     *reinterpret_cast<uint4*>(sm + OFF_TWU + sw128(i, qq * 2 + m)) =
                         make_uint4(w4[0], w4[1], w4[2], w4[3]);
