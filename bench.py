@@ -159,7 +159,9 @@ def bench_ours(args, rank, world, local_rank):
                       chunk=w.chunk, read_mode=w.read_mode, scale=w.scale, o=o, S_final=S_final,
                       workspace=ws)
 
-    for _ in range(args.warmup):
+    if args.only == "decode":
+        args.steps = max(1, min(args.steps, 1))
+    for _ in range(args.warmup if args.only != "decode" else 0):
         step()
     torch.cuda.synchronize()
     sampler = ClockSampler(local_rank)
@@ -189,8 +191,12 @@ def bench_ours(args, rank, world, local_rank):
 
     # ---------------- decode step
     dec = None
-    if not args.no_decode:
+    if not args.no_decode and args.only != "chunk":
         dw = workloads.DECODE_WORKLOADS[DECODE_WORKLOAD]
+        if args.decode_seqs:
+            import dataclasses
+            dw = dataclasses.replace(dw, N=args.decode_seqs,
+                                     name=f"{dw.name}[seqs={args.decode_seqs}]")
         dx = workloads.decode_workload_inputs(dw, seed=rank)
         dd = {n: t.to(dev) for n, t in dx.items()}
         od = torch.empty((dw.N, dw.Hv, dw.dv), dtype=torch.bfloat16, device=dev)
@@ -215,7 +221,7 @@ def bench_ours(args, rank, world, local_rank):
             dd[n][0].numel() * dd[n].element_size() for n in ("q", "k", "v", "g", "beta")) + (
             od.numel() * od.element_size())
         dgbs = dbytes / (dms / 1e3) / 1e9
-        dec = {"workload": DECODE_WORKLOAD, "ms_per_step": dms, "bytes_per_step": dbytes,
+        dec = {"workload": dw.name, "ms_per_step": dms, "bytes_per_step": dbytes,
                "value": world * dgbs, "unit": "GB/s",
                "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"],
                             "unit": "GB/s", "frac": dgbs / peaks["hbm_gbs"],
@@ -337,6 +343,10 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["all", "chunk", "decode"], default="all",
+                    help="profiling: time only one of the two hot paths")
+    ap.add_argument("--decode-seqs", type=int, default=0,
+                    help="profiling: run the decode step on this many sequences only")
     ap.add_argument("--rows", type=int, default=0,
                     help="run only this many rows of the forward workload (profiling a small case)")
     ap.add_argument("--traffic", type=float, default=None,

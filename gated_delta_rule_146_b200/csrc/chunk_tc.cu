@@ -149,6 +149,16 @@ __device__ __forceinline__ float* f32sw(float* base, int i, int j) {
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
+// Raw bits of a gate element (bf16 zero-extended, or fp32): loading without converting lets
+// the load stay in flight until the value is consumed much later.
+__device__ __forceinline__ uint32_t load_gate_bits(const void* p, size_t i, gdr_dtype dt) {
+    return dt == GDR_BF16 ? (uint32_t)static_cast<const unsigned short*>(p)[i]
+                          : static_cast<const uint32_t*>(p)[i];
+}
+__device__ __forceinline__ float gate_bits_to_float(uint32_t b, gdr_dtype dt) {
+    return __uint_as_float(dt == GDR_BF16 ? b << 16 : b);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
@@ -202,6 +212,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     auto gate_at = [&](const void* arr, int pos) -> float {
         return load_elem(arr, (size_t)(tokA + tstep * pos) * p.Hv + h, p.gt);
     };
+    auto gate_bits_at = [&](const void* arr, int pos) -> uint32_t {
+        return load_gate_bits(arr, (size_t)(tokA + tstep * pos) * p.Hv + h, p.gt);
+    };
     // wait for a phase of an mbarrier; the whole warpgroup agrees on the outcome
     auto wg_wait = [&](int idx, uint32_t parity, int bar_id) -> bool {
         const bool ok = mbar_wait_bounded(&SS.mbar[idx], parity, kWaitLimitNs);
@@ -226,7 +239,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
         const long long kq_tok = (long long)p.Hk * D, v_tok = (long long)p.Hv * D;
         auto load_chunk = [&](int c) {
             if (p.use_tma) {  // forward scans: six 8 KB tensor tiles, issued by one thread
-                if (pt == 0) {
+                if (pt == 32) {
                     uint64_t* bar = &SS.mbar[MB_LD + c % 3];
                     const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
                     const uint32_t vv = sbase + OFF_V + (c & 1) * V_STRIDE;
@@ -255,6 +268,11 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 cp_async16(vv + off, vbase + tok * v_tok, valid);
             }
         };
+        if (p.use_tma && pt == 32) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
+        }
         load_chunk(0);
         if (!p.use_tma) cp_async_commit();
         {
@@ -264,7 +282,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 SS.b[0][pt] = pt < Cc0 ? gate_at(p.beta, pt) : 0.f;
             }
         }
-        float g_nx = 0.f, b_nx = 0.f;
+        uint32_t g_nx = 0, b_nx = 0;  // raw bits of the next chunk's gates
         for (int c = 0; c < nchunks; ++c) {
             const int pb = c & 1;
             const uint32_t KQ = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
@@ -275,11 +293,15 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
 
             // P0: the buffers of chunk c-2 are released once the chain is done with them
             if (c >= 2 && !wg_wait(MB_CD + pb, ((c >> 1) & 1) ^ 1, kBarPrep)) { fail = true; break; }
+            int Cn = 0;
             if (has_next) {
                 load_chunk(c + 1);
-                const int Cn = min(C, L - (c + 1) * C);
-                g_nx = pt < Cn ? gate_at(p.g, (c + 1) * C + pt) : 0.f;
-                b_nx = pt < Cn ? gate_at(p.beta, (c + 1) * C + pt) : 0.f;
+                // in-bounds position for every thread, masked only where the value is stored
+                // (a select on a just-loaded value would wait for the load right here)
+                Cn = min(C, L - (c + 1) * C);
+                const int pos = (c + 1) * C + min(pt & 63, Cn - 1);
+                g_nx = gate_bits_at(p.g, pos);
+                b_nx = gate_bits_at(p.beta, pos);
             }
             if (!p.use_tma) cp_async_commit();
             // in-chunk cumsum of g (log2 units) while the copies land, and whether every decay
@@ -321,19 +343,21 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             // P1: half row of [K; Q]: bf16 -> (L2-normalised) fp16 in place; per-row factors
             {
                 uint4 vals[8];
-                float ss = 0.f;
+                float ssq[4] = {0.f, 0.f, 0.f, 0.f};
                 uint8_t* rowp = KQp + hf * 16384;
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
+                for (int c8 = 0; c8 < 8; ++c8)
                     vals[c8] = *reinterpret_cast<const uint4*>(rowp + sw128(r, c8));
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
                     const uint32_t w[4] = {vals[c8].x, vals[c8].y, vals[c8].z, vals[c8].w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 x = unpack_bf16x2(w[e]);
-                        ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
+                        ssq[e] = fmaf(x.x, x.x, fmaf(x.y, x.y, ssq[e]));
                     }
                 }
-                SS.ssp[hf][r] = ss;
+                SS.ssp[hf][r] = (ssq[0] + ssq[1]) + (ssq[2] + ssq[3]);
                 if (pt < C) {
                     const float Gref = SS.G[31];
                     const float Gi = SS.G[pt];
@@ -602,8 +626,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 }
             }
             if (has_next && pt < C) {
-                SS.g[pb ^ 1][pt] = g_nx;
-                SS.b[pb ^ 1][pt] = b_nx;
+                SS.g[pb ^ 1][pt] = pt < Cn ? gate_bits_to_float(g_nx, p.gt) : 0.f;
+                SS.b[pb ^ 1][pt] = pt < Cn ? gate_bits_to_float(b_nx, p.gt) : 0.f;
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -645,7 +669,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             const int Cc = min(C, L - c * C);
             const bool has_next = c + 1 < nchunks;
             const int Cn = has_next ? min(C, L - (c + 1) * C) : 0;
-            const float g_nx = lt < Cn ? gate_at(p.g, (c + 1) * C + lt) : 0.f;
+            // loaded unconditionally from an in-bounds position, masked when reduced in C2
+            uint32_t g_raw = 0;
+            if (has_next) g_raw = gate_bits_at(p.g, (c + 1) * C + min(lt & 63, Cn - 1));
 
             if (!wg_wait(MB_PREP + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
             // C1: V'^T = U~^T + H^T (-W^T);  O^T = H^T Q~^T   (A = state copy in TMEM)
@@ -689,7 +715,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 }
                 tmem_wait_st();
                 if (warp < 2) {
-                    const float part = warp_sum(g_nx);
+                    const float part = warp_sum(lt < Cn ? gate_bits_to_float(g_raw, p.gt) : 0.f);
                     if (lane == 0) SS.gsum_part[warp] = part;
                 }
             }
@@ -713,8 +739,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             }
             if (!wg_wait(MB_M3 + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
 
-            // C4: O -> staged in WN[pb] (row per token) -> bulk copies to global; state ->
-            //     fp16 copy, pre-scaled for the next chunk
+            // C4: O -> staged in WN[pb] (row per token) -> coalesced stores; state -> fp16
+            //     copy, pre-scaled for the next chunk
             {
                 uint8_t* stage = sm + OFF_WN + pb * 16384;
                 uint32_t ro[2][32];
@@ -729,17 +755,15 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                             __float2bfloat16_rn(u2f(ro[half][m]));
                 fence_proxy_async_smem();
                 named_bar(kBarChain, 128);
-                if (lt < Cc) {
-                    const long long tok = tokA + tstep * (long long)(c * C + lt);
-                    __nv_bfloat16* dst = p.o + ((size_t)tok * p.Hv + h) * D;
-                    if (!p.o_acc) {
-                        bulk_store(dst, sbase + OFF_WN + pb * 16384 + lt * 256, 256);
-                        bulk_commit();
-                    } else {
-#pragma unroll 4
-                        for (int c16 = 0; c16 < 16; ++c16) {
-                            const uint4 a = *reinterpret_cast<const uint4*>(stage + lt * 256 + c16 * 16);
-                            uint4* dp = reinterpret_cast<uint4*>(dst + c16 * 8);
+                // 16-byte chunks, consecutive threads on consecutive chunks of a row
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const int idx = m * 128 + lt, row = idx >> 4, c16 = idx & 15;
+                    if (row < Cc) {
+                        const long long tok = tokA + tstep * (long long)(c * C + row);
+                        uint4* dp = reinterpret_cast<uint4*>(p.o + ((size_t)tok * p.Hv + h) * D + c16 * 8);
+                        uint4 a = *reinterpret_cast<const uint4*>(stage + row * 256 + c16 * 16);
+                        if (p.o_acc) {
                             const uint4 b = *dp;
                             const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
                             uint32_t ow[4];
@@ -748,8 +772,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                                 const float2 x = unpack_bf16x2(aw[e]), y = unpack_bf16x2(bw[e]);
                                 ow[e] = pack_bf16x2(x.x + y.x, x.y + y.y);
                             }
-                            *dp = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                            a = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                         }
+                        *dp = a;
                     }
                 }
                 const float gam = has_next ? ex2((SS.gsum_part[0] + SS.gsum_part[1]) * kLog2e) : 1.f;
@@ -779,7 +804,6 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 tmem_wait_st();
-                if (lt < Cc && !p.o_acc) bulk_wait_read();
                 mbar_arrive(&SS.mbar[MB_CD + pb]);
             }
             tc_fence_before();
