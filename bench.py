@@ -45,6 +45,23 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def measured_traffic(kernel: str, source: str, units: float):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu summary
+    (profiles/traffic.json), scaled from the captured case to `units` (rows or sequences);
+    None when the kernel source has changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "gated_delta_rule_146_b200", "csrc", source)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != rec["source_sha256_16"]:
+        return None
+    captured = rec.get("rows_captured") or rec.get("seqs_captured")
+    return (rec["dram_read_bytes"] + rec["dram_write_bytes"]) * units / captured
+
+
 def flops_per_head_token(C, dk, dv):
     """Dense chunk-form FLOPs per token per head: KK^T, QK^T, W (2C dk each), U and the
     intra output (2C dv each), W H, the state update and Q H (2 dk dv each)."""
@@ -225,6 +242,7 @@ def bench_ours(args, rank, world, local_rank):
                "value": world * dgbs, "unit": "GB/s",
                "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"],
                             "unit": "GB/s", "frac": dgbs / peaks["hbm_gbs"],
+                            "traffic": measured_traffic("decode_kernel", "decode.cu", dw.N),
                             "peak_source": f"{peak_src} (hbm_gbs, copy)"}}
     clocks = sampler.stop()
 
@@ -273,7 +291,10 @@ def bench_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}, no collective"},
         "tflops": tflops, "pct_bf16_tc_peak": tflops / peaks["bf16_tflops"] * 100,
         "roofline": {"bound": "hbm", "achieved": hbm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": hbm_gbs / peaks["hbm_gbs"], "traffic": args.traffic,
+                     "frac": hbm_gbs / peaks["hbm_gbs"],
+                     "traffic": args.traffic if args.traffic is not None else (
+                         measured_traffic("chunk_fused_tc", "chunk_tc.cu", w.B)
+                         if path == "tc" and not w.n_varlen else None),
                      "algorithmic_bytes": algo_bytes, "flops": flops,
                      "tensor_frac": tflops / peaks["bf16_tflops"],
                      "timed": "whole gdr_chunk_fwd call (plan + chunk kernels), CUDA events",
