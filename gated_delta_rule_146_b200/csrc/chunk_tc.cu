@@ -34,8 +34,10 @@
 // shared memory in the 128-byte-swizzled canonical layouts (K-major or MN-major as each
 // product needs).  Accumulation and the state are fp32.
 //
-// Operand precision: V and T diag(beta) are bf16 (V arrives in bf16); every other operand
-// (normalised q and k, T diag(beta e^G), W, the state copy, V', P) is rounded to fp16,
+// Operand precision: [K;Q] K^T is formed from the bf16 inputs as they arrive (exact
+// products, fp32 sums) and the L2 norms are applied to its rows and columns in fp32.
+// V and T diag(beta) are bf16 (V arrives in bf16); every other operand
+// (normalised k, Q~, T diag(beta e^G), W, the state copy, V', P) is rounded to fp16,
 // whose 11-bit significand keeps the chain of roundings well inside the bf16 parity bound
 // at long sequence lengths where bf16 operands do not.  Every fp16 operand is checked for
 // overflow (an infinite or NaN half); one sets GDR_ERR_RANGE.  Decay factors are
@@ -109,7 +111,7 @@ struct Small {
     float Kd[2][C];          // e^(G_last - G_i), 0 beyond the chunk, by chunk parity (for the chain)
     float Er[C];             // 2^(G_i - G_ref): row factor of the decay (K rows)
     float Eq[C];             // 2^(G'_i - G_ref): row factor for the read (G' = G_i or G_{i-1})
-    float Ec[C];             // 2^(G_ref - G_j): column factor
+    float ck[C];             // column factor of [K;Q]K^T: 1/||k_j|| (x 2^(G_ref - G_j) when split)
     float ssp[2][128];       // partial sums of squares of the [K;Q] row halves
     float gsum_part[2];      // chain: partial sums of the next chunk's g
     uint64_t mbar[MB_COUNT];
@@ -125,6 +127,7 @@ struct TcParams {
     __nv_bfloat16* o; float* S_final;
     WsHeader* hdr; const int32_t* cu;
     int Hk, Hv, read_pre, qk_l2norm, reverse, o_acc, use_tma;
+    int tma_store;  // full output chunks leave through the output tensor map
     gdr_dtype gt;
     float scale;
 };
@@ -161,7 +164,8 @@ __device__ __forceinline__ float gate_bits_to_float(uint32_t b, gdr_dtype dt) {
 
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
-               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+               const __grid_constant__ CUtensorMap tm_o) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -291,8 +295,14 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             const int Cc = min(C, L - c * C);
             const bool has_next = c + 1 < nchunks;
 
-            // P0: the buffers of chunk c-2 are released once the chain is done with them
-            if (c >= 2 && !wg_wait(MB_CD + pb, ((c >> 1) & 1) ^ 1, kBarPrep)) { fail = true; break; }
+            // P0: the buffers of chunk c-2 are released once the chain is done with them.  Either
+            //     barrier also publishes this chunk's gates (stored by warps 4 and 5) to the
+            //     cumulative sum below.
+            if (c >= 2) {
+                if (!wg_wait(MB_CD + pb, ((c >> 1) & 1) ^ 1, kBarPrep)) { fail = true; break; }
+            } else {
+                named_bar(kBarPrep, kPrep);
+            }
             int Cn = 0;
             if (has_next) {
                 load_chunk(c + 1);
@@ -340,11 +350,30 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 break;
             }
 
-            // P1: half row of [K; Q]: bf16 -> (L2-normalised) fp16 in place; per-row factors
+            // P1: D0 = [K;Q] K^T straight from the bf16 tiles (M=128, N=64, K=128).  The L2
+            //     norms scale D0's rows and columns afterwards, so the product starts as soon
+            //     as the tiles land and runs while the operands are normalised.
+            tc_fence_after();
+            if (pt == 0) {
+                const uint32_t id = idesc_f32acc(128, 64, false, false, true);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_f32acc_ss(tmem + TM_D0, sdesc_sw128(KQ + off, 16, 1024),
+                                  sdesc_sw128(KQ + off, 16, 1024), id, kk > 0);
+                }
+                mma_commit(&SS.mbar[MB_M0]);
+            }
+            // P2: half row of [K; Q] -> sum of squares -> fp16 operand in registers: K rows
+            //     L2-normalised, Q rows as Q~ = scale e^(G') q / ||q||; rows past the chunk
+            //     (tensor tiles carry the following tokens there) become 0.  Stored over the
+            //     bf16 tile once the product has read it.
+            uint32_t hv[32];
+            float inv;  // 1 / ||row|| (1 without normalisation)
+            uint8_t* rowp = KQp + hf * 16384;
             {
                 uint4 vals[8];
                 float ssq[4] = {0.f, 0.f, 0.f, 0.f};
-                uint8_t* rowp = KQp + hf * 16384;
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8)
                     vals[c8] = *reinterpret_cast<const uint4*>(rowp + sw128(r, c8));
@@ -358,6 +387,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 SS.ssp[hf][r] = (ssq[0] + ssq[1]) + (ssq[2] + ssq[3]);
+                float ec = 0.f;
                 if (pt < C) {
                     const float Gref = SS.G[31];
                     const float Gi = SS.G[pt];
@@ -366,72 +396,80 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     SS.bg[pt] = SS.b[pb][pt] * ex2(Gi);
                     SS.Er[pt] = ex2(Gi - Gref);
                     SS.Eq[pt] = ex2(Gr - Gref);
-                    SS.Ec[pt] = ex2(Gref - Gi);
+                    ec = ex2(Gref - Gi);
                 }
                 named_bar(kBarPrep, kPrep);
                 const float tot = SS.ssp[0][r] + SS.ssp[1][r];
-                const float inv = p.qk_l2norm ? 1.f / fmaxf(sqrtf(tot), kNormEps) : 1.f;
-                // rows past the chunk (tensor tiles carry the following tokens there) become 0
-                const bool live = (r & 63) < Cc;
+                inv = p.qk_l2norm ? rsqrtf(fmaxf(tot, kNormEps * kNormEps)) : 1.f;
+                // column factor of D0 (K rows): 1/||k_j||, times 2^(G_ref - G_j) when split
+                if (pt < C) SS.ck[pt] = SS.split_ok ? ec * inv : inv;
+                const int i = r & 63;
+                float f = inv;
+                if (r >= C) {
+                    const float Gr = p.read_pre ? (i > 0 ? SS.G[i - 1] : 0.f) : SS.G[i];
+                    f = p.scale * ex2(Gr) * inv;
+                }
+                if (i >= Cc) f = 0.f;
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
                     const uint32_t w[4] = {vals[c8].x, vals[c8].y, vals[c8].z, vals[c8].w};
-                    float f[8];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 x = unpack_bf16x2(w[e]);
-                        f[2 * e] = live ? x.x * inv : 0.f;
-                        f[2 * e + 1] = live ? x.y * inv : 0.f;
+                        hv[c8 * 4 + e] = h2(x.x * f, x.y * f, rflags);
                     }
-                    *reinterpret_cast<uint4*>(rowp + sw128(r, c8)) = h8(f, rflags);
                 }
                 for (int idx = pt; idx < (C - Cc) * 16; idx += kPrep) {  // V rows past the chunk
-                    const int i = Cc + (idx >> 4), c16 = idx & 15;
+                    const int iv = Cc + (idx >> 4), c16 = idx & 15;
                     *reinterpret_cast<uint4*>(sm + OFF_V + pb * V_STRIDE + (c16 >> 3) * 8192 +
-                                              sw128(i, c16 & 7)) = make_uint4(0, 0, 0, 0);
+                                              sw128(iv, c16 & 7)) = make_uint4(0, 0, 0, 0);
                 }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar(kBarPrep, kPrep);
-            tc_fence_after();
-
-            // P2: D0 = [K;Q] K^T  (M=128, N=64, K=128)
-            if (pt == 0) {
-                const uint32_t id = idesc_f32acc(128, 64, false, false, false);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_f32acc_ss(tmem + TM_D0, sdesc_sw128(KQ + off, 16, 1024),
-                                  sdesc_sw128(KQ + off, 16, 1024), id, kk > 0);
-                }
-                mma_commit(&SS.mbar[MB_M0]);
             }
             if (!wg_wait(MB_M0, c & 1, kBarPrep)) { fail = true; break; }
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8)
+                *reinterpret_cast<uint4*>(rowp + sw128(r, c8)) =
+                    make_uint4(hv[c8 * 4], hv[c8 * 4 + 1], hv[c8 * 4 + 2], hv[c8 * 4 + 3]);
 
-            // P3: columns [32 hf, 32 hf + 32) of row r of D0: A (fp32, rows 0-63) and
-            //     P (fp16, rows 64-127); half of Q -> Q~ = scale e^(G') Q in place
+            // P3: columns [32 hf, 32 hf + 32) of row r of D0, with the norms applied: A (fp32,
+            //     rows 0-63) and P (fp16, rows 64-127)
             {
                 const int i = r & 63;
-                const bool isK = r < C;
+                const bool live = i < Cc;
                 const bool split = SS.split_ok;
                 float* As = reinterpret_cast<float*>(sm + OFF_AS);
                 uint32_t rr[32];
                 tmem_ld32(tlane + TM_D0 + hf * 32, rr);
                 tmem_wait_ld();
-                if (isK) {
-                    const float Gi = SS.G[i];
-                    const float bi = SS.b[pb][i];
-                    const float fi = bi * SS.Er[i];
+                float ckv[32];
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 x = *reinterpret_cast<const float4*>(&SS.ck[hf * 32 + e4 * 4]);
+                    ckv[e4 * 4] = x.x; ckv[e4 * 4 + 1] = x.y; ckv[e4 * 4 + 2] = x.z; ckv[e4 * 4 + 3] = x.w;
+                }
+                // row factor (beta_i / ||k_i|| or scale / ||q_i||, times 2^(G'_i - G_ref) when
+                // split) and, without the split, the per-element decay exponent's row part
+                const float Gi = r < C ? SS.G[i]
+                                       : (p.read_pre ? (i > 0 ? SS.G[i - 1] : 0.f) : SS.G[i]);
+                float fi = live ? (r < C ? SS.b[pb][i] : p.scale) * inv : 0.f;
+                if (split) fi *= r < C ? SS.Er[i] : SS.Eq[i];
+                float vals[32];
+                if (split) {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) vals[u] = fi * u2f(rr[u]) * ckv[u];
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        vals[u] = fi * u2f(rr[u]) * ckv[u] * ex2(Gi - SS.G[hf * 32 + u]);
+                }
+                if (r < C) {
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
                         float a[4];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             const int j = hf * 32 + e4 * 4 + u;
-                            const float v = split ? fi * u2f(rr[e4 * 4 + u]) * SS.Ec[j]
-                                                  : bi * u2f(rr[e4 * 4 + u]) * ex2(Gi - SS.G[j]);
-                            a[u] = j < i ? v : 0.f;
+                            a[u] = j < i ? vals[e4 * 4 + u] : 0.f;
                         }
                         *reinterpret_cast<float4*>(f32sw(As, i, hf * 32 + e4 * 4)) =
                             make_float4(a[0], a[1], a[2], a[3]);
@@ -444,8 +482,6 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         }
                     }
                 } else {
-                    const float Gr = p.read_pre ? (i > 0 ? SS.G[i - 1] : 0.f) : SS.G[i];
-                    const float fi = p.scale * SS.Eq[i];
 #pragma unroll
                     for (int e8 = 0; e8 < 4; ++e8) {
                         float pv[8];
@@ -453,22 +489,10 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         for (int u = 0; u < 8; ++u) {
                             const int j = hf * 32 + e8 * 8 + u;
                             const bool on = p.read_pre ? (j < i) : (j <= i);
-                            const float v = split ? fi * u2f(rr[e8 * 8 + u]) * SS.Ec[j]
-                                                  : p.scale * u2f(rr[e8 * 8 + u]) * ex2(Gr - SS.G[j]);
-                            pv[u] = on ? v : 0.f;
+                            pv[u] = on ? vals[e8 * 8 + u] : 0.f;
                         }
                         *reinterpret_cast<uint4*>(sm + OFF_P + pb * 8192 + sw128(i, hf * 4 + e8)) =
                             h8(pv, rflags);
-                    }
-                    const __half2 f2 = __float2half2_rn(p.scale * ex2(Gr));
-#pragma unroll
-                    for (int c8 = 0; c8 < 8; ++c8) {
-                        uint4* ptr = reinterpret_cast<uint4*>(KQp + hf * 16384 + 8192 + sw128(i, c8));
-                        uint4 u = *ptr;
-                        __half2* hv = reinterpret_cast<__half2*>(&u);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) hv[e] = __hmul2(hv[e], f2);
-                        *ptr = u;
                     }
                 }
             }
@@ -476,25 +500,24 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             named_bar(kBarPrep, kPrep);
 
             // P4: T = (I + A)^-1 by 16-blocks.  Stage 0: the four diagonal inverses T_bb by
-            //     right-looking substitution (one warp each, on the transposed block);
-            //     stage A: E_rl = T_rr A_rl for r > l, in place over A (six warps);
-            //     stage d = 1..3: T_rs = -sum_{l=s}^{r-1} E_rl T_ls for r - s = d.
-            //     The warp MMAs (tf32, m16n8k8) pair each thread's two k slots with two
-            //     adjacent columns, so every A fragment comes in two 8-byte loads.
+            //     substitution (one warp each); then the blocks below the diagonal in three
+            //     phases of tf32 warp MMAs.
             {
                 float* As = reinterpret_cast<float*>(sm + OFF_AS);
                 float* Ts = reinterpret_cast<float*>(sm + OFF_TWU);
                 const float* AsT = reinterpret_cast<const float*>(sm + OFF_RS);
                 if (pw < 4 && lane < 16) {
+                    // column cl of T_bb: x_m = [m == cl] - sum_{n<m} A_mn x_n, in registers
+                    // (no shared-memory store between the loads, so they all issue early)
                     const int b0 = pw * 16, cl = lane;
-                    const float* at = AsT + pw * 256;
+                    const float* __restrict__ at = AsT + pw * 256;
                     float acc[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) acc[i] = 0.f;
 #pragma unroll
                     for (int jc = 0; jc < 16; ++jc) {
                         const float xj = jc < cl ? 0.f : (jc == cl ? 1.f : -acc[jc]);
-                        *f32sw(Ts, b0 + jc, b0 + cl) = xj;
+                        acc[jc] = xj;
 #pragma unroll
                         for (int i4 = (jc + 1) >> 2; i4 < 4; ++i4) {
                             const float4 a4 = *reinterpret_cast<const float4*>(at + jc * 16 + 4 * i4);
@@ -504,52 +527,95 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                                 if (4 * i4 + u > jc) acc[4 * i4 + u] = fmaf(av[u], xj, acc[4 * i4 + u]);
                         }
                     }
+#pragma unroll
+                    for (int jc = 0; jc < 16; ++jc) *f32sw(Ts, b0 + jc, b0 + cl) = acc[jc];
                 }
                 named_bar(kBarPrep, kPrep);
                 const int gq = lane >> 2, tq = lane & 3;
-                // one 16x16x16 product step: acc[nt] += X(rows 16 xr.., cols 16 xc + 8 ks..)
-                //                                      * Z(rows 16 zr + 8 ks.., cols 16 zc + 8 nt..)
-                auto mma_block = [&](float (&acc)[2][4], const float* X, int xr, int xc,
-                                     const float* Z, int zr, int zc) {
+                // 16x16 blocks in warp-MMA fragments (tf32, m16n8k8).  Each thread's two k slots
+                // are paired with two adjacent columns, so an accumulator block (rows gq, gq + 8;
+                // columns 8 nt + 2 tq, +1) is itself the A fragment of its own k half nt.
+                using Frag = uint32_t[2][4];  // A fragments of the two k halves
+                using Blk = float[2][4];      // accumulator block, by column half
+                auto frag_smem = [&](Frag& a, const float* X, int xr, int xc) {
 #pragma unroll
                     for (int ks = 0; ks < 2; ++ks) {
                         const int col = 16 * xc + 8 * ks + 2 * tq;
                         const float2 lo = *reinterpret_cast<const float2*>(f32sw(const_cast<float*>(X), 16 * xr + gq, col));
                         const float2 hi = *reinterpret_cast<const float2*>(f32sw(const_cast<float*>(X), 16 * xr + gq + 8, col));
-                        const uint32_t a[4] = {to_tf32(lo.x), to_tf32(hi.x), to_tf32(lo.y), to_tf32(hi.y)};
-                        const int zrow = 16 * zr + 8 * ks + 2 * tq;
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt) {
-                            const int zc_ = 16 * zc + 8 * nt + gq;
-                            const uint32_t bf[2] = {to_tf32(*f32sw(const_cast<float*>(Z), zrow, zc_)),
-                                                    to_tf32(*f32sw(const_cast<float*>(Z), zrow + 1, zc_))};
-                            mma_tf32_16x8x8(acc[nt], a, bf);
-                        }
+                        a[ks][0] = to_tf32(lo.x); a[ks][1] = to_tf32(hi.x);
+                        a[ks][2] = to_tf32(lo.y); a[ks][3] = to_tf32(hi.y);
                     }
                 };
-                auto store_block = [&](float* Y, int yr, int yc, const float (&acc)[2][4], float sgn) {
+                auto frag_reg = [&](Frag& a, const Blk& e) {
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        a[ks][0] = to_tf32(e[ks][0]); a[ks][1] = to_tf32(e[ks][2]);
+                        a[ks][2] = to_tf32(e[ks][1]); a[ks][3] = to_tf32(e[ks][3]);
+                    }
+                };
+                // R (+)= X Z, Z the 16x16 block (zr, zc) in shared memory; the four MMAs are
+                // independent (one accumulator per k half) and summed at the end
+                auto bprod = [&](Blk& R, const Frag& a, const float* Z, int zr, int zc, bool add) {
+                    float t[2][2][4];
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt) {
+                            const int zrow = 16 * zr + 8 * ks + 2 * tq, zcol = 16 * zc + 8 * nt + gq;
+                            const uint32_t bf[2] = {to_tf32(*f32sw(const_cast<float*>(Z), zrow, zcol)),
+                                                    to_tf32(*f32sw(const_cast<float*>(Z), zrow + 1, zcol))};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) t[ks][nt][e] = 0.f;
+                            mma_tf32_16x8x8(t[ks][nt], a[ks], bf);
+                        }
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            R[nt][e] = (add ? R[nt][e] : 0.f) + (t[0][nt][e] + t[1][nt][e]);
+                };
+                auto store_neg = [&](float* Y, int yr, int yc, const Blk& acc) {
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
                         const int rr = 16 * yr + gq, cc = 16 * yc + 8 * nt + 2 * tq;
-                        *reinterpret_cast<float2*>(f32sw(Y, rr, cc)) = make_float2(sgn * acc[nt][0], sgn * acc[nt][1]);
-                        *reinterpret_cast<float2*>(f32sw(Y, rr + 8, cc)) = make_float2(sgn * acc[nt][2], sgn * acc[nt][3]);
+                        *reinterpret_cast<float2*>(f32sw(Y, rr, cc)) = make_float2(-acc[nt][0], -acc[nt][1]);
+                        *reinterpret_cast<float2*>(f32sw(Y, rr + 8, cc)) = make_float2(-acc[nt][2], -acc[nt][3]);
                     }
                 };
-                if (pw < 6) {  // stage A: (1,0) (2,0) (3,0) (2,1) (3,1) (3,2)
-                    const int rblk = pw < 3 ? pw + 1 : (pw < 5 ? pw - 1 : 3);
-                    const int lblk = pw < 3 ? 0 : (pw < 5 ? 1 : 2);
-                    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                    mma_block(acc, Ts, rblk, rblk, As, rblk, lblk);
-                    __syncwarp();
-                    store_block(As, rblk, lblk, acc, 1.f);
-                }
-                named_bar(kBarPrep, kPrep);
-                for (int dist = 1; dist < 4; ++dist) {
-                    if (pw < 4 - dist) {
-                        const int sblk = pw, rblk = pw + dist;
-                        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                        for (int l = sblk; l < rblk; ++l) mma_block(acc, As, rblk, l, Ts, l, sblk);
-                        store_block(Ts, rblk, sblk, acc, -1.f);
+                // E_rl = T_rr A_rl (r > l);  T_rs = -sum_{l=s}^{r-1} E_rl T_ls.
+                //   phase 1: T_10, T_21, T_32 (warps 0-2); Y_20 = E_20 T_00, Y_31 = E_31 T_11,
+                //            Y_30 = E_30 T_00 (warps 3-5, which also form the E they need next)
+                //   phase 2: T_20 = -(Y_20 + E_21 T_10), T_31 = -(Y_31 + E_32 T_21),
+                //            Y_30 += E_31 T_10
+                //   phase 3: T_30 = -(Y_30 + E_32 T_20)
+                {
+                    Frag a;
+                    Blk Y, E1, E2;  // E1, E2: the E blocks a warp keeps for phases 2 and 3
+                    if (pw < 6) {
+                        const int r = pw < 3 ? pw + 1 : (pw == 3 ? 2 : 3);
+                        const int l = pw < 3 ? pw : (pw == 4 ? 1 : 0);
+                        Blk E;
+                        frag_smem(a, Ts, r, r);
+                        bprod(E, a, As, r, l, false);
+                        if (pw >= 3) bprod(E1, a, As, r, l + 1, false);  // E_21, E_32, E_31
+                        if (pw == 5) bprod(E2, a, As, r, 2, false);       // E_32
+                        frag_reg(a, E);
+                        bprod(Y, a, Ts, l, l, false);
+                        if (pw < 3) store_neg(Ts, r, l, Y);
+                    }
+                    named_bar(kBarPrep, kPrep);
+                    if (pw >= 3 && pw < 6) {
+                        frag_reg(a, E1);
+                        if (pw == 3) { bprod(Y, a, Ts, 1, 0, true); store_neg(Ts, 2, 0, Y); }
+                        if (pw == 4) { bprod(Y, a, Ts, 2, 1, true); store_neg(Ts, 3, 1, Y); }
+                        if (pw == 5) bprod(Y, a, Ts, 1, 0, true);
+                    }
+                    named_bar(kBarPrep, kPrep);
+                    if (pw == 5) {
+                        frag_reg(a, E2);
+                        bprod(Y, a, Ts, 2, 0, true);
+                        store_neg(Ts, 3, 0, Y);
                     }
                     named_bar(kBarPrep, kPrep);
                 }
@@ -682,6 +748,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     mma_f32acc_ts(tmem + TM_DU + pb * 64, tmem + TM_HB + kk * 8,
                                   sdesc_sw128(sbase + OFF_WN + pb * 16384 + kk * 2048, 8192, 1024),
                                   id1, 1);
+                // V' is all C2 needs: its barrier fires before the output product runs; the
+                // commit after C3 covers the output product
+                mma_commit(&SS.mbar[MB_M1]);
                 const uint32_t id2 = idesc_f32acc(128, 64, false, false, false);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -689,7 +758,6 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     mma_f32acc_ts(tmem + TM_DO, tmem + TM_HB + kk * 8,
                                   sdesc_sw128(KQ + off + 8192, 16, 1024), id2, kk > 0);
                 }
-                mma_commit(&SS.mbar[MB_M1]);
             }
             if (!wg_wait(MB_M1, c & 1, kBarChain)) { fail = true; break; }
 
@@ -739,10 +807,14 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             }
             if (!wg_wait(MB_M3 + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
 
-            // C4: O -> staged in WN[pb] (row per token) -> coalesced stores; state -> fp16
-            //     copy, pre-scaled for the next chunk
+            // C4: O -> staged in WN[pb] -> global (two tensor stores for a full chunk, else
+            //     coalesced 16-byte stores); state -> fp16 copy, pre-scaled for the next chunk
             {
+                // staging: two [token][64] bf16 tiles (dv halves) in the 128-byte-swizzled
+                // layout of the output tensor map's box
                 uint8_t* stage = sm + OFF_WN + pb * 16384;
+                uint8_t* stage_j = stage + (j >> 6) * 8192 + (j & 7) * 2;
+                const int cj = (j & 63) >> 3;
                 uint32_t ro[2][32];
                 tmem_ld32(tlane + TM_DO, ro[0]);
                 tmem_ld32(tlane + TM_DO + 32, ro[1]);
@@ -751,10 +823,19 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 for (int half = 0; half < 2; ++half)
 #pragma unroll
                     for (int m = 0; m < 32; ++m)
-                        *reinterpret_cast<__nv_bfloat16*>(stage + (half * 32 + m) * 256 + j * 2) =
+                        *reinterpret_cast<__nv_bfloat16*>(stage_j + sw128(half * 32 + m, cj)) =
                             __float2bfloat16_rn(u2f(ro[half][m]));
                 fence_proxy_async_smem();
                 named_bar(kBarChain, 128);
+                if (p.tma_store && Cc == C) {
+                    if (lt == 0) {
+                        const int z = (int)(t0 + (long long)c * C);
+                        const uint32_t src = sbase + OFF_WN + pb * 16384;
+                        tma_store_3d(&tm_o, src, 0, h, z);
+                        tma_store_3d(&tm_o, src + 8192, 64, h, z);
+                        bulk_commit();
+                    }
+                } else {
                 // 16-byte chunks, consecutive threads on consecutive chunks of a row
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {
@@ -762,7 +843,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     if (row < Cc) {
                         const long long tok = tokA + tstep * (long long)(c * C + row);
                         uint4* dp = reinterpret_cast<uint4*>(p.o + ((size_t)tok * p.Hv + h) * D + c16 * 8);
-                        uint4 a = *reinterpret_cast<const uint4*>(stage + row * 256 + c16 * 16);
+                        uint4 a = *reinterpret_cast<const uint4*>(stage + (c16 >> 3) * 8192 +
+                                                                  sw128(row, c16 & 7));
                         if (p.o_acc) {
                             const uint4 b = *dp;
                             const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
@@ -776,6 +858,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         }
                         *dp = a;
                     }
+                }
                 }
                 const float gam = has_next ? ex2((SS.gsum_part[0] + SS.gsum_part[1]) * kLog2e) : 1.f;
 #pragma unroll
@@ -804,6 +887,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 tmem_wait_st();
+                if (lt == 0) bulk_wait_read();  // the staging buffer is free for reuse
                 mbar_arrive(&SS.mbar[MB_CD + pb]);
             }
             tc_fence_before();
@@ -812,6 +896,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
         }
     }
 
+    if (tid == 0) bulk_wait_all();  // output tiles written before the CTA exits
     if (fail && (tid == 0 || tid == 128 || tid == 256)) atomicExch(&p.hdr->err, (int)GDR_ERR_TIMEOUT);
     tc_fence_before();
     if (__syncthreads_or((rflags & 0x80008000u) ? 1 : 0) && tid == 0)
@@ -875,23 +960,27 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
     p.Hk = a.Hk; p.Hv = a.Hv; p.read_pre = a.read_mode == GDR_READ_PRE;
     p.qk_l2norm = a.qk_l2norm; p.reverse = a.reverse; p.o_acc = a.o_accumulate;
     p.gt = a.gate_dtype; p.scale = a.scale;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     memset(&tq, 0, sizeof(tq));
     memset(&tk, 0, sizeof(tk));
     memset(&tv, 0, sizeof(tv));
+    memset(&to, 0, sizeof(to));
     const long long T_tot = (long long)a.B * a.T;
     p.use_tma = 0;
+    p.tma_store = 0;
     if (!a.reverse && T_tot > 0) {  // reversed scans gather rows with cp.async instead
         if (!make_tile_map(&tq, q, a.Hk, T_tot) || !make_tile_map(&tk, k, a.Hk, T_tot) ||
             !make_tile_map(&tv, v, a.Hv, T_tot))
             return GDR_ERR_CUDA;
         p.use_tma = 1;
+        // accumulating outputs are read back, so they keep the plain stores
+        p.tma_store = !a.o_accumulate && make_tile_map(&to, o, a.Hv, T_tot);
     }
     if (cudaFuncSetAttribute(chunk_fused_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
     dim3 grid((unsigned)a.n_seqs, (unsigned)a.Hv);
-    chunk_fused_tc<<<grid, kThreads, SMEM_BYTES, st>>>(p, tq, tk, tv);
+    chunk_fused_tc<<<grid, kThreads, SMEM_BYTES, st>>>(p, tq, tk, tv, to);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

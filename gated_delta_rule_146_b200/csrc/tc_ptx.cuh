@@ -257,9 +257,10 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int 
 }
 
 // ---- bulk copy shared -> global (contiguous bytes, 16-byte aligned, size % 16 == 0) ------
-__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
-                 "r"(ssrc), "r"(bytes)
+// tensor tile store from shared memory (bulk-group completion)
+__device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(src), "r"(x), "r"(y), "r"(z)
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit() {
@@ -268,6 +269,10 @@ __device__ __forceinline__ void bulk_commit() {
 // wait until the shared-memory sources of this thread's bulk copies have been read
 __device__ __forceinline__ void bulk_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// wait until this thread's bulk copies have completed (their global writes performed)
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // ---- cp.async (16 bytes, zero-filled when !valid) ----------------------------------------
