@@ -75,9 +75,9 @@ constexpr uint32_t OFF_KQ = 0;         // 3 x 32 KB; per dk half (16 KB): K rows
 constexpr uint32_t KQ_STRIDE = 32768;
 constexpr uint32_t OFF_V = 98304;      // 2 x 16 KB; per dv half (8 KB): V rows 0-63 (bf16)
 constexpr uint32_t V_STRIDE = 16384;
-constexpr uint32_t OFF_TWU = 131072;   // T diag(beta e^G) fp16 [i][j] | T diag(beta) bf16 [i][j];
-                                       // holds the fp32 T [64][64] during the solve
-constexpr uint32_t OFF_AS = 147456;    // A fp32 [64][64]
+constexpr uint32_t OFF_TWU = 131072;   // T fp32 [64][64] (the solve)
+constexpr uint32_t OFF_AS = 147456;    // A fp32 [64][64]; after the solve's first phase:
+                                       // T diag(beta e^G) fp16 [i][j] | T diag(beta) bf16 [i][j]
 constexpr uint32_t OFF_RS = 163840;    // the four diagonal 16x16 blocks of A, transposed (fp32)
 constexpr uint32_t OFF_P = 167936;     // 2 x 8 KB: P fp16 [i][j]
 constexpr uint32_t OFF_WN = 184320;    // 2 x 16 KB: -W^T fp16 [dk][tok]; output staging
@@ -132,15 +132,15 @@ struct TcParams {
     float scale;
 };
 
-// fp16 pair; `flags` accumulates the overflow test: (exponent & 0x7C00) + 0x0400 carries into
-// bit 15 (31) exactly when a half is infinite or NaN.
-__device__ __forceinline__ uint32_t h2(float a, float b, uint32_t& flags) {
-    const uint32_t u = pack_f16x2(a, b);
-    flags |= (u & 0x7C007C00u) + 0x04000400u;
-    return u;
+// fp16 pair; `mx` keeps the running maximum magnitude of every half produced (NaN sticks),
+// tested once at the end: an infinite or NaN half means the value left the fp16 range.
+__device__ __forceinline__ uint32_t h2(float a, float b, __half2& mx) {
+    const __half2 v = __floats2half2_rn(a, b);
+    mx = __hmax2_nan(mx, __habs2(v));
+    return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-__device__ __forceinline__ uint4 h8(const float* f, uint32_t& flags) {
+__device__ __forceinline__ uint4 h8(const float* f, __half2& flags) {
     return make_uint4(h2(f[0], f[1], flags), h2(f[2], f[3], flags), h2(f[4], f[5], flags),
                       h2(f[6], f[7], flags));
 }
@@ -210,7 +210,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     tc_fence_after();
     const uint32_t tmem = SS.tmem_base;
     const uint32_t tlane = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's lanes
-    uint32_t rflags = 0;  // fp16 overflow test bits
+    __half2 rflags = __float2half2_rn(0.f);  // running max |fp16 operand| (overflow test)
+    bool rbad = false;                       // a bound showed an operand out of the fp16 range
     bool fail = false;    // a bounded wait gave up
 
     auto gate_at = [&](const void* arr, int pos) -> float {
@@ -314,9 +315,43 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 b_nx = gate_bits_at(p.beta, pos);
             }
             if (!p.use_tma) cp_async_commit();
-            // in-chunk cumsum of g (log2 units) while the copies land, and whether every decay
-            // factor 2^(G_i - G_j) splits into 2^(G_i - G_ref) 2^(G_ref - G_j) inside the normal
-            // fp32 range (true unless the log2 decay strays more than 110 from G_ref = G_31)
+            bool landed = true;
+            if (p.use_tma)
+                landed = mbar_wait_bounded(&SS.mbar[MB_LD + c % 3], (uint32_t)((c / 3) & 1),
+                                           kWaitLimitNs);
+            else
+                cp_async_wait<1>();
+            fence_proxy_async_smem();
+            if (!named_bar_and(kBarPrep, kPrep, (landed && !SS.abort) ? 1 : 0)) {
+                SS.abort = 1;
+                fail = true;
+                break;
+            }
+
+            // P1: D0 = [K;Q] K^T straight from the bf16 tiles (M=128, N=64, K=128).  The L2
+            //     norms scale D0's rows and columns afterwards, so the product starts as soon
+            //     as the tiles land and runs while the operands are normalised.
+            tc_fence_after();
+            if (pt == kPrep - 32) {  // warp 11: the cumsum below keeps warp 4 busy
+                const uint32_t id = idesc_f32acc(128, 64, false, false, true);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_f32acc_ss(tmem + TM_D0, sdesc_sw128(KQ + off, 16, 1024),
+                                  sdesc_sw128(KQ + off, 16, 1024), id, kk > 0);
+                }
+                mma_commit(&SS.mbar[MB_M0]);
+            }
+            // P2: half row of [K; Q] -> sum of squares -> fp16 operand in registers: K rows
+            //     L2-normalised, Q rows as Q~ = scale e^(G') q / ||q||; rows past the chunk
+            //     (tensor tiles carry the following tokens there) become 0.  Stored over the
+            //     bf16 tile once the product has read it.
+            uint32_t hv[32];
+            float inv;  // 1 / ||row|| (1 without normalisation)
+            uint8_t* rowp = KQp + hf * 16384;
+            // in-chunk cumsum of g (log2 units; warp 4, while the other warps load), and whether
+            // every decay factor 2^(G_i - G_j) splits into 2^(G_i - G_ref) 2^(G_ref - G_j) inside
+            // the normal fp32 range (true unless the log2 decay strays more than 110 from G_31)
             if (pw == 0) {
                 const float a0 = SS.g[pb][2 * lane] * kLog2e, a1 = SS.g[pb][2 * lane + 1] * kLog2e;
                 const float pair = a0 + a1;
@@ -337,40 +372,6 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 for (int o = 16; o > 0; o >>= 1) dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, o));
                 if (lane == 0) SS.split_ok = dev <= 110.f;
             }
-            bool landed = true;
-            if (p.use_tma)
-                landed = mbar_wait_bounded(&SS.mbar[MB_LD + c % 3], (uint32_t)((c / 3) & 1),
-                                           kWaitLimitNs);
-            else
-                cp_async_wait<1>();
-            fence_proxy_async_smem();
-            if (!named_bar_and(kBarPrep, kPrep, (landed && !SS.abort) ? 1 : 0)) {
-                SS.abort = 1;
-                fail = true;
-                break;
-            }
-
-            // P1: D0 = [K;Q] K^T straight from the bf16 tiles (M=128, N=64, K=128).  The L2
-            //     norms scale D0's rows and columns afterwards, so the product starts as soon
-            //     as the tiles land and runs while the operands are normalised.
-            tc_fence_after();
-            if (pt == 0) {
-                const uint32_t id = idesc_f32acc(128, 64, false, false, true);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_f32acc_ss(tmem + TM_D0, sdesc_sw128(KQ + off, 16, 1024),
-                                  sdesc_sw128(KQ + off, 16, 1024), id, kk > 0);
-                }
-                mma_commit(&SS.mbar[MB_M0]);
-            }
-            // P2: half row of [K; Q] -> sum of squares -> fp16 operand in registers: K rows
-            //     L2-normalised, Q rows as Q~ = scale e^(G') q / ||q||; rows past the chunk
-            //     (tensor tiles carry the following tokens there) become 0.  Stored over the
-            //     bf16 tile once the product has read it.
-            uint32_t hv[32];
-            float inv;  // 1 / ||row|| (1 without normalisation)
-            uint8_t* rowp = KQp + hf * 16384;
             {
                 uint4 vals[8];
                 float ssq[4] = {0.f, 0.f, 0.f, 0.f};
@@ -387,8 +388,11 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 SS.ssp[hf][r] = (ssq[0] + ssq[1]) + (ssq[2] + ssq[3]);
-                float ec = 0.f;
-                if (pt < C) {
+                named_bar(kBarPrep, kPrep);
+                const float tot = SS.ssp[0][r] + SS.ssp[1][r];
+                inv = p.qk_l2norm ? rsqrtf(fmaxf(tot, kNormEps * kNormEps)) : 1.f;
+                if (pt < C) {  // per-token factors; the column factor of D0 (K rows) is 1/||k_j||,
+                               // times 2^(G_ref - G_j) when split
                     const float Gref = SS.G[31];
                     const float Gi = SS.G[pt];
                     const float Gr = p.read_pre ? (pt > 0 ? SS.G[pt - 1] : 0.f) : Gi;
@@ -396,13 +400,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     SS.bg[pt] = SS.b[pb][pt] * ex2(Gi);
                     SS.Er[pt] = ex2(Gi - Gref);
                     SS.Eq[pt] = ex2(Gr - Gref);
-                    ec = ex2(Gref - Gi);
+                    SS.ck[pt] = SS.split_ok ? ex2(Gref - Gi) * inv : inv;
                 }
-                named_bar(kBarPrep, kPrep);
-                const float tot = SS.ssp[0][r] + SS.ssp[1][r];
-                inv = p.qk_l2norm ? rsqrtf(fmaxf(tot, kNormEps * kNormEps)) : 1.f;
-                // column factor of D0 (K rows): 1/||k_j||, times 2^(G_ref - G_j) when split
-                if (pt < C) SS.ck[pt] = SS.split_ok ? ec * inv : inv;
                 const int i = r & 63;
                 float f = inv;
                 if (r >= C) {
@@ -410,13 +409,15 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     f = p.scale * ex2(Gr) * inv;
                 }
                 if (i >= Cc) f = 0.f;
+                // every element of the row is at most ||row|| f in magnitude (NaN fails too)
+                if (!(sqrtf(tot) * fabsf(f) < 65504.f)) rbad = true;
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
                     const uint32_t w[4] = {vals[c8].x, vals[c8].y, vals[c8].z, vals[c8].w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 x = unpack_bf16x2(w[e]);
-                        hv[c8 * 4 + e] = h2(x.x * f, x.y * f, rflags);
+                        hv[c8 * 4 + e] = pack_f16x2(x.x * f, x.y * f);
                     }
                 }
                 for (int idx = pt; idx < (C - Cc) * 16; idx += kPrep) {  // V rows past the chunk
@@ -639,7 +640,6 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     bgv[4 * e4] = x.x; bgv[4 * e4 + 1] = x.y; bgv[4 * e4 + 2] = x.z; bgv[4 * e4 + 3] = x.w;
                     bv[4 * e4] = y.x; bv[4 * e4 + 1] = y.y; bv[4 * e4 + 2] = y.z; bv[4 * e4 + 3] = y.w;
                 }
-                named_bar(kBarPrep, kPrep);  // T is read completely before the 16-bit tiles overwrite it
 #pragma unroll
                 for (int m = 0; m < 2; ++m) {
                     uint32_t w4[4], u4[4];
@@ -649,9 +649,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         w4[e] = h2(tv[jj] * bgv[jj], tv[jj + 1] * bgv[jj + 1], rflags);
                         u4[e] = pack_bf16x2(tv[jj] * bv[jj], tv[jj + 1] * bv[jj + 1]);
                     }
-                    *reinterpret_cast<uint4*>(sm + OFF_TWU + sw128(i, qq * 2 + m)) =
+                    *reinterpret_cast<uint4*>(sm + OFF_AS + sw128(i, qq * 2 + m)) =
                         make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    *reinterpret_cast<uint4*>(sm + OFF_TWU + 8192 + sw128(i, qq * 2 + m)) =
+                    *reinterpret_cast<uint4*>(sm + OFF_AS + 8192 + sw128(i, qq * 2 + m)) =
                         make_uint4(u4[0], u4[1], u4[2], u4[3]);
                 }
             }
@@ -666,12 +666,12 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f32acc_ss(tmem + TM_D0, sdesc_sw128(KQ + kk * 2048, 16384, 1024),
-                                  sdesc_sw128(sbase + OFF_TWU + kk * 32, 16, 1024), idw, kk > 0);
+                                  sdesc_sw128(sbase + OFF_AS + kk * 32, 16, 1024), idw, kk > 0);
                 const uint32_t idu = idesc_f32acc(128, 64, true, false, true);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f32acc_ss(tmem + TM_DU + pb * 64, sdesc_sw128(VV + kk * 2048, 8192, 1024),
-                                  sdesc_sw128(sbase + OFF_TWU + 8192 + kk * 32, 16, 1024), idu,
+                                  sdesc_sw128(sbase + OFF_AS + 8192 + kk * 32, 16, 1024), idu,
                                   kk > 0);
                 mma_commit(&SS.mbar[MB_MW]);
             }
@@ -772,11 +772,14 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     uint32_t pk[16], ps[16];
                     const uint32_t* r = rv[half];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float a = u2f(r[2 * e]), b = u2f(r[2 * e + 1]);
-                        pk[e] = h2(a, b, rflags);
-                        ps[e] = h2(a * SS.Kd[pb][half * 32 + 2 * e], b * SS.Kd[pb][half * 32 + 2 * e + 1],
-                                   rflags);
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 kd = *reinterpret_cast<const float4*>(&SS.Kd[pb][half * 32 + 4 * e4]);
+                        const float a0 = u2f(r[4 * e4]), b0 = u2f(r[4 * e4 + 1]);
+                        const float a1 = u2f(r[4 * e4 + 2]), b1 = u2f(r[4 * e4 + 3]);
+                        pk[2 * e4] = h2(a0, b0, rflags);
+                        pk[2 * e4 + 1] = h2(a1, b1, rflags);
+                        ps[2 * e4] = h2(a0 * kd.x, b0 * kd.y, rflags);
+                        ps[2 * e4 + 1] = h2(a1 * kd.z, b1 * kd.w, rflags);
                     }
                     tmem_st16(tlane + TM_VP + half * 16, pk);
                     tmem_st16(tlane + TM_VS + half * 16, ps);
@@ -899,7 +902,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     if (tid == 0) bulk_wait_all();  // output tiles written before the CTA exits
     if (fail && (tid == 0 || tid == 128 || tid == 256)) atomicExch(&p.hdr->err, (int)GDR_ERR_TIMEOUT);
     tc_fence_before();
-    if (__syncthreads_or((rflags & 0x80008000u) ? 1 : 0) && tid == 0)
+    rbad = rbad || !(__low2float(rflags) <= 65504.f) || !(__high2float(rflags) <= 65504.f);
+    if (__syncthreads_or(rbad ? 1 : 0) && tid == 0)
         atomicCAS(&p.hdr->err, (int)GDR_OK, (int)GDR_ERR_RANGE);
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 }
