@@ -167,8 +167,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const __grid_constant__ CUtensorMap tm_o) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+    // 1024-byte aligned base, as a byte offset from the shared array so that every access
+    // through it stays a shared-memory access (an integer round trip would make them generic)
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
     Small& SS = *reinterpret_cast<Small*>(sm + OFF_SMALL);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -464,22 +465,20 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         vals[u] = fi * u2f(rr[u]) * ckv[u] * ex2(Gi - SS.G[hf * 32 + u]);
                 }
                 if (r < C) {
+                    // the solve reads the 16x16 blocks below the diagonal from A and the
+                    // diagonal blocks (strictly lower part) transposed; the rest is never read
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
-                        float a[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int j = hf * 32 + e4 * 4 + u;
-                            a[u] = j < i ? vals[e4 * 4 + u] : 0.f;
-                        }
-                        *reinterpret_cast<float4*>(f32sw(As, i, hf * 32 + e4 * 4)) =
-                            make_float4(a[0], a[1], a[2], a[3]);
-                        // the diagonal 16x16 block of row i, transposed, for the substitution
                         const int jb = hf * 32 + e4 * 4;
-                        if ((jb >> 4) == (i >> 4)) {
+                        if ((jb >> 4) < (i >> 4)) {
+                            *reinterpret_cast<float4*>(f32sw(As, i, jb)) =
+                                make_float4(vals[e4 * 4], vals[e4 * 4 + 1], vals[e4 * 4 + 2],
+                                            vals[e4 * 4 + 3]);
+                        } else if ((jb >> 4) == (i >> 4)) {
                             float* at = reinterpret_cast<float*>(sm + OFF_RS) + (i >> 4) * 256;
 #pragma unroll
-                            for (int u = 0; u < 4; ++u) at[((jb + u) & 15) * 16 + (i & 15)] = a[u];
+                            for (int u = 0; u < 4; ++u)
+                                at[((jb + u) & 15) * 16 + (i & 15)] = jb + u < i ? vals[e4 * 4 + u] : 0.f;
                         }
                     }
                 } else {
@@ -497,21 +496,22 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
             }
-            tc_fence_before();
-            named_bar(kBarPrep, kPrep);
 
             // P4: T = (I + A)^-1 by 16-blocks.  Stage 0: the four diagonal inverses T_bb by
-            //     substitution (one warp each); then the blocks below the diagonal in three
-            //     phases of tf32 warp MMAs.
+            //     substitution, each by the warp that wrote its block of A (warps 4 and 9, two
+            //     blocks each) while the Q-row warps are still forming P; then the blocks
+            //     below the diagonal in three phases of tf32 warp MMAs.
             {
                 float* As = reinterpret_cast<float*>(sm + OFF_AS);
                 float* Ts = reinterpret_cast<float*>(sm + OFF_TWU);
                 const float* AsT = reinterpret_cast<const float*>(sm + OFF_RS);
-                if (pw < 4 && lane < 16) {
-                    // column cl of T_bb: x_m = [m == cl] - sum_{n<m} A_mn x_n, in registers
-                    // (no shared-memory store between the loads, so they all issue early)
-                    const int b0 = pw * 16, cl = lane;
-                    const float* __restrict__ at = AsT + pw * 256;
+                if (pw == 0 || pw == 5) {
+                    // column cl of T_bb: x_m = [m == cl] - sum_{n<m} A_mn x_n, in registers, one
+                    // column per lane; warp 4 holds blocks 0 and 1, warp 9 blocks 2 and 3
+                    __syncwarp();  // the warp's transposed diagonal blocks are complete
+                    const int blk = (pw == 0 ? 0 : 2) + (lane >> 4);
+                    const int b0 = blk * 16, cl = lane & 15;
+                    const float* __restrict__ at = AsT + blk * 256;  // at[j * 16 + i] = A_ij
                     float acc[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) acc[i] = 0.f;
