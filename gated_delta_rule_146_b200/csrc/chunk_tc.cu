@@ -428,13 +428,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 }
             }
             if (!wg_wait(MB_M0, c & 1, kBarPrep)) { fail = true; break; }
-#pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8)
-                *reinterpret_cast<uint4*>(rowp + sw128(r, c8)) =
-                    make_uint4(hv[c8 * 4], hv[c8 * 4 + 1], hv[c8 * 4 + 2], hv[c8 * 4 + 3]);
-
             // P3: columns [32 hf, 32 hf + 32) of row r of D0, with the norms applied: A (fp32,
-            //     rows 0-63) and P (fp16, rows 64-127)
+            //     rows 0-63) and P (fp16, rows 64-127); the fp16 operands go over the bf16 tile
+            //     (read by the product) while the accumulator load is in flight
             {
                 const int i = r & 63;
                 const bool live = i < Cc;
@@ -442,19 +438,23 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 float* As = reinterpret_cast<float*>(sm + OFF_AS);
                 uint32_t rr[32];
                 tmem_ld32(tlane + TM_D0 + hf * 32, rr);
-                tmem_wait_ld();
                 float ckv[32];
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
                     const float4 x = *reinterpret_cast<const float4*>(&SS.ck[hf * 32 + e4 * 4]);
                     ckv[e4 * 4] = x.x; ckv[e4 * 4 + 1] = x.y; ckv[e4 * 4 + 2] = x.z; ckv[e4 * 4 + 3] = x.w;
                 }
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8)
+                    *reinterpret_cast<uint4*>(rowp + sw128(r, c8)) =
+                        make_uint4(hv[c8 * 4], hv[c8 * 4 + 1], hv[c8 * 4 + 2], hv[c8 * 4 + 3]);
                 // row factor (beta_i / ||k_i|| or scale / ||q_i||, times 2^(G'_i - G_ref) when
                 // split) and, without the split, the per-element decay exponent's row part
                 const float Gi = r < C ? SS.G[i]
                                        : (p.read_pre ? (i > 0 ? SS.G[i - 1] : 0.f) : SS.G[i]);
                 float fi = live ? (r < C ? SS.b[pb][i] : p.scale) * inv : 0.f;
                 if (split) fi *= r < C ? SS.Er[i] : SS.Eq[i];
+                tmem_wait_ld();
                 float vals[32];
                 if (split) {
 #pragma unroll
@@ -464,24 +464,56 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     for (int u = 0; u < 32; ++u)
                         vals[u] = fi * u2f(rr[u]) * ckv[u] * ex2(Gi - SS.G[hf * 32 + u]);
                 }
-                if (r < C) {
-                    // the solve reads the 16x16 blocks below the diagonal from A and the
-                    // diagonal blocks (strictly lower part) transposed; the rest is never read
+                // The solve reads the 16x16 blocks of A below the diagonal and the diagonal
+                // blocks (strictly lower part, transposed); the rest of A is never read.  Warp 5
+                // (rows 32-63, columns 0-31) holds only blocks below the diagonal; warps 4 and
+                // 9 hold the diagonal blocks (0, 1 and 2, 3), which they invert at once, and in
+                // lanes 16-31 one block below them (A_10, A_32); warp 8 holds none of them.
+                if (pw == 1) {
 #pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        const int jb = hf * 32 + e4 * 4;
-                        if ((jb >> 4) < (i >> 4)) {
-                            *reinterpret_cast<float4*>(f32sw(As, i, jb)) =
-                                make_float4(vals[e4 * 4], vals[e4 * 4 + 1], vals[e4 * 4 + 2],
-                                            vals[e4 * 4 + 3]);
-                        } else if ((jb >> 4) == (i >> 4)) {
-                            float* at = reinterpret_cast<float*>(sm + OFF_RS) + (i >> 4) * 256;
+                    for (int e4 = 0; e4 < 8; ++e4)
+                        *reinterpret_cast<float4*>(f32sw(As, i, e4 * 4)) =
+                            make_float4(vals[e4 * 4], vals[e4 * 4 + 1], vals[e4 * 4 + 2], vals[e4 * 4 + 3]);
+                } else if (pw == 0 || pw == 5) {
+                    const bool hi = lane >= 16;
+                    const int il = i & 15;
+                    float* at = reinterpret_cast<float*>(sm + OFF_RS) + (i >> 4) * 256;
 #pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                at[((jb + u) & 15) * 16 + (i & 15)] = jb + u < i ? vals[e4 * 4 + u] : 0.f;
+                    for (int u = 0; u < 16; ++u)
+                        at[u * 16 + il] = u < il ? (hi ? vals[16 + u] : vals[u]) : 0.f;
+                    __syncwarp();
+                    // P4 stage 0, column il of T_bb (b = i >> 4, one block per half warp):
+                    //   x_m = [m == il] - sum_{n<m} A_mn x_n, in registers
+                    {
+                        const int b0 = i & ~15;
+                        const float* __restrict__ atr = at;  // atr[j * 16 + m] = A_mj
+                        float* Ts = reinterpret_cast<float*>(sm + OFF_TWU);
+                        float acc[16];
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) acc[m] = 0.f;
+#pragma unroll
+                        for (int jc = 0; jc < 16; ++jc) {
+                            const float xj = jc < il ? 0.f : (jc == il ? 1.f : -acc[jc]);
+                            acc[jc] = xj;
+#pragma unroll
+                            for (int i4 = (jc + 1) >> 2; i4 < 4; ++i4) {
+                                const float4 a4 = *reinterpret_cast<const float4*>(atr + jc * 16 + 4 * i4);
+                                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                                for (int u = 0; u < 4; ++u)
+                                    if (4 * i4 + u > jc) acc[4 * i4 + u] = fmaf(av[u], xj, acc[4 * i4 + u]);
+                            }
                         }
+#pragma unroll
+                        for (int jc = 0; jc < 16; ++jc) *f32sw(Ts, b0 + jc, b0 + il) = acc[jc];
                     }
-                } else {
+                    if (hi) {
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4)
+                            *reinterpret_cast<float4*>(f32sw(As, i, hf * 32 + e4 * 4)) =
+                                make_float4(vals[e4 * 4], vals[e4 * 4 + 1], vals[e4 * 4 + 2], vals[e4 * 4 + 3]);
+                    }
+                } else if (r >= C) {
 #pragma unroll
                     for (int e8 = 0; e8 < 4; ++e8) {
                         float pv[8];
@@ -497,40 +529,12 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 }
             }
 
-            // P4: T = (I + A)^-1 by 16-blocks.  Stage 0: the four diagonal inverses T_bb by
-            //     substitution, each by the warp that wrote its block of A (warps 4 and 9, two
-            //     blocks each) while the Q-row warps are still forming P; then the blocks
-            //     below the diagonal in three phases of tf32 warp MMAs.
+            // P4: T = (I + A)^-1 by 16-blocks.  Stage 0 (the four diagonal inverses, above,
+            //     while the Q-row warps form P), then the blocks below the diagonal in three
+            //     phases of tf32 warp MMAs.
             {
                 float* As = reinterpret_cast<float*>(sm + OFF_AS);
                 float* Ts = reinterpret_cast<float*>(sm + OFF_TWU);
-                const float* AsT = reinterpret_cast<const float*>(sm + OFF_RS);
-                if (pw == 0 || pw == 5) {
-                    // column cl of T_bb: x_m = [m == cl] - sum_{n<m} A_mn x_n, in registers, one
-                    // column per lane; warp 4 holds blocks 0 and 1, warp 9 blocks 2 and 3
-                    __syncwarp();  // the warp's transposed diagonal blocks are complete
-                    const int blk = (pw == 0 ? 0 : 2) + (lane >> 4);
-                    const int b0 = blk * 16, cl = lane & 15;
-                    const float* __restrict__ at = AsT + blk * 256;  // at[j * 16 + i] = A_ij
-                    float acc[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-#pragma unroll
-                    for (int jc = 0; jc < 16; ++jc) {
-                        const float xj = jc < cl ? 0.f : (jc == cl ? 1.f : -acc[jc]);
-                        acc[jc] = xj;
-#pragma unroll
-                        for (int i4 = (jc + 1) >> 2; i4 < 4; ++i4) {
-                            const float4 a4 = *reinterpret_cast<const float4*>(at + jc * 16 + 4 * i4);
-                            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                if (4 * i4 + u > jc) acc[4 * i4 + u] = fmaf(av[u], xj, acc[4 * i4 + u]);
-                        }
-                    }
-#pragma unroll
-                    for (int jc = 0; jc < 16; ++jc) *f32sw(Ts, b0 + jc, b0 + cl) = acc[jc];
-                }
                 named_bar(kBarPrep, kPrep);
                 const int gq = lane >> 2, tq = lane & 3;
                 // 16x16 blocks in warp-MMA fragments (tf32, m16n8k8).  Each thread's two k slots

@@ -230,10 +230,11 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // ---- warp-level tf32 MMA (m16n8k8, fp32 accumulate) for the small blocked solve ---------
+// fp32 -> tf32 (10 explicit significand bits), rounded to nearest with ties away from zero:
+// add half a tf32 unit in the last place to the bit pattern and clear the 13 dropped bits
+// (a carry into the exponent is the correct rounding up; infinities stay infinite)
 __device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+    return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
 }
 __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4],
                                                 const uint32_t (&b)[2]) {
