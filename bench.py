@@ -45,18 +45,35 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def measured_traffic(kernel: str, source: str, units: float):
+CHUNK_TC_SOURCES = ("chunk_tc.cu", "tc_ptx.cuh", "common.cuh")
+DECODE_SOURCES = ("decode.cu", "common.cuh")
+
+
+def source_digest(sources) -> str:
+    """First 16 hex digits of the SHA-256 of the concatenated kernel sources (the .cu file
+    and the headers it includes), the revision key of a traffic record."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in sources:
+        with open(os.path.join(ROOT, "gated_delta_rule_146_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, sources, units: float):
     """DRAM bytes (read + write) per launch of `kernel` from the committed ncu summary
     (profiles/traffic.json), scaled from the captured case to `units` (rows or sequences);
-    None when the kernel source has changed since the counters were taken."""
-    import hashlib
+    None when a kernel source has changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    src = os.path.join(ROOT, "gated_delta_rule_146_b200", "csrc", source)
-    if not (os.path.exists(path) and os.path.exists(src)):
+    if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f).get(kernel)
-    if not rec or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != rec["source_sha256_16"]:
+    try:
+        digest = source_digest(sources)
+    except OSError:
+        return None
+    if not rec or digest != rec["source_sha256_16"]:
         return None
     captured = rec.get("rows_captured") or rec.get("seqs_captured")
     return (rec["dram_read_bytes"] + rec["dram_write_bytes"]) * units / captured
@@ -242,7 +259,7 @@ def bench_ours(args, rank, world, local_rank):
                "value": world * dgbs, "unit": "GB/s",
                "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"],
                             "unit": "GB/s", "frac": dgbs / peaks["hbm_gbs"],
-                            "traffic": measured_traffic("decode_kernel", "decode.cu", dw.N),
+                            "traffic": measured_traffic("decode_kernel", DECODE_SOURCES, dw.N),
                             "peak_source": f"{peak_src} (hbm_gbs, copy)"}}
     clocks = sampler.stop()
 
@@ -293,7 +310,7 @@ def bench_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": hbm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": hbm_gbs / peaks["hbm_gbs"],
                      "traffic": args.traffic if args.traffic is not None else (
-                         measured_traffic("chunk_fused_tc", "chunk_tc.cu", w.B)
+                         measured_traffic("chunk_fused_tc", CHUNK_TC_SOURCES, w.B)
                          if path == "tc" and not w.n_varlen else None),
                      "algorithmic_bytes": algo_bytes, "flops": flops,
                      "tensor_frac": tflops / peaks["bf16_tflops"],
