@@ -76,11 +76,12 @@ constexpr uint32_t KQ_STRIDE = 32768;
 constexpr uint32_t OFF_V = 98304;      // 2 x 16 KB; per dv half (8 KB): V rows 0-63 (bf16)
 constexpr uint32_t V_STRIDE = 16384;
 constexpr uint32_t OFF_TWU = 131072;   // T fp32 [64][64] (the solve)
-constexpr uint32_t OFF_AS = 147456;    // A fp32 [64][64]; after the solve's first phase:
-                                       // T diag(beta e^G) fp16 [i][j] | T diag(beta) bf16 [i][j]
+constexpr uint32_t OFF_AS = 147456;    // A fp32 [64][64]
 constexpr uint32_t OFF_RS = 163840;    // the four diagonal 16x16 blocks of A, transposed (fp32)
 constexpr uint32_t OFF_P = 167936;     // 2 x 8 KB: P fp16 [i][j]
-constexpr uint32_t OFF_WN = 184320;    // 2 x 16 KB: -W^T fp16 [dk][tok]; output staging
+constexpr uint32_t OFF_WN = 184320;    // 2 x 16 KB: T diag(beta e^G) fp16 | T diag(beta) bf16
+                                       // during the solve, then -W^T fp16 [dk][tok]; output
+                                       // staging
 constexpr uint32_t OFF_SMALL = 217088;
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + 5120 + 1024;
 
@@ -580,6 +581,26 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         for (int e = 0; e < 4; ++e)
                             R[nt][e] = (add ? R[nt][e] : 0.f) + (t[0][nt][e] + t[1][nt][e]);
                 };
+                // T_w = T diag(beta e^G) (fp16) and T_u = T diag(beta) (bf16) as [i][j] K-major
+                // tiles, the B operands of the W and U~ products, in the -W^T buffer of this
+                // chunk (free from the chunk's start until the products have run); each block of
+                // T is written there by the warp that completes it
+                uint8_t* twu = sm + OFF_WN + pb * 16384;
+                auto put_twu = [&](int yr, int yc, const Blk& acc) {  // block (yr, yc) = -acc
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const int cc = 16 * yc + 8 * nt + 2 * tq;
+                        const float2 bgp = *reinterpret_cast<const float2*>(&SS.bg[cc]);
+                        const float2 bp = *reinterpret_cast<const float2*>(&SS.b[pb][cc]);
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const float t0 = -acc[nt][2 * hh], t1 = -acc[nt][2 * hh + 1];
+                            const uint32_t off = sw128(16 * yr + gq + 8 * hh, cc >> 3) + (cc & 7) * 2;
+                            *reinterpret_cast<uint32_t*>(twu + off) = h2(t0 * bgp.x, t1 * bgp.y, rflags);
+                            *reinterpret_cast<uint32_t*>(twu + 8192 + off) = pack_bf16x2(t0 * bp.x, t1 * bp.y);
+                        }
+                    }
+                };
                 auto store_neg = [&](float* Y, int yr, int yc, const Blk& acc) {
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
@@ -594,6 +615,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 //   phase 2: T_20 = -(Y_20 + E_21 T_10), T_31 = -(Y_31 + E_32 T_21),
                 //            Y_30 += E_31 T_10
                 //   phase 3: T_30 = -(Y_30 + E_32 T_20)
+                // Warps 6 and 7 write the diagonal and upper blocks of T_w, T_u in phase 1.
                 {
                     Frag a;
                     Blk Y, E1, E2;  // E1, E2: the E blocks a warp keeps for phases 2 and 3
@@ -607,56 +629,50 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         if (pw == 5) bprod(E2, a, As, r, 2, false);       // E_32
                         frag_reg(a, E);
                         bprod(Y, a, Ts, l, l, false);
-                        if (pw < 3) store_neg(Ts, r, l, Y);
+                        if (pw < 2) store_neg(Ts, r, l, Y);  // T_10, T_21: read in phase 2
+                        if (pw < 3) put_twu(r, l, Y);
+                    } else {
+                        // row i: its diagonal block from the fp32 T, zeros to its right
+                        const int i = pt - 192, b = i >> 4;
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) {
+                            const int j0 = 16 * b + 8 * m;
+                            const float4 t0 = *reinterpret_cast<const float4*>(f32sw(Ts, i, j0));
+                            const float4 t1 = *reinterpret_cast<const float4*>(f32sw(Ts, i, j0 + 4));
+                            const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+                            const float4 g0 = *reinterpret_cast<const float4*>(&SS.bg[j0]);
+                            const float4 g1 = *reinterpret_cast<const float4*>(&SS.bg[j0 + 4]);
+                            const float4 b0 = *reinterpret_cast<const float4*>(&SS.b[pb][j0]);
+                            const float4 b1 = *reinterpret_cast<const float4*>(&SS.b[pb][j0 + 4]);
+                            const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                            uint32_t w4[4], u4[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                w4[e] = h2(tv[2 * e] * gv[2 * e], tv[2 * e + 1] * gv[2 * e + 1], rflags);
+                                u4[e] = pack_bf16x2(tv[2 * e] * bv[2 * e], tv[2 * e + 1] * bv[2 * e + 1]);
+                            }
+                            *reinterpret_cast<uint4*>(twu + sw128(i, 2 * b + m)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                            *reinterpret_cast<uint4*>(twu + 8192 + sw128(i, 2 * b + m)) = make_uint4(u4[0], u4[1], u4[2], u4[3]);
+                        }
+                        for (int c8 = 2 * b + 2; c8 < 8; ++c8) {
+                            *reinterpret_cast<uint4*>(twu + sw128(i, c8)) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4*>(twu + 8192 + sw128(i, c8)) = make_uint4(0, 0, 0, 0);
+                        }
                     }
                     named_bar(kBarPrep, kPrep);
                     if (pw >= 3 && pw < 6) {
                         frag_reg(a, E1);
-                        if (pw == 3) { bprod(Y, a, Ts, 1, 0, true); store_neg(Ts, 2, 0, Y); }
-                        if (pw == 4) { bprod(Y, a, Ts, 2, 1, true); store_neg(Ts, 3, 1, Y); }
+                        if (pw == 3) { bprod(Y, a, Ts, 1, 0, true); store_neg(Ts, 2, 0, Y); put_twu(2, 0, Y); }
+                        if (pw == 4) { bprod(Y, a, Ts, 2, 1, true); put_twu(3, 1, Y); }
                         if (pw == 5) bprod(Y, a, Ts, 1, 0, true);
                     }
                     named_bar(kBarPrep, kPrep);
                     if (pw == 5) {
                         frag_reg(a, E2);
                         bprod(Y, a, Ts, 2, 0, true);
-                        store_neg(Ts, 3, 0, Y);
+                        put_twu(3, 0, Y);
                     }
-                    named_bar(kBarPrep, kPrep);
-                }
-                // T -> T diag(beta e^G) (fp16) and T diag(beta) (bf16): row i, 16 columns
-                const int i = pt >> 2, qq = pt & 3;
-                float tv[16];
-#pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {
-                    const float4 v4 = *reinterpret_cast<const float4*>(f32sw(Ts, i, qq * 16 + e4 * 4));
-                    tv[e4 * 4 + 0] = v4.x; tv[e4 * 4 + 1] = v4.y;
-                    tv[e4 * 4 + 2] = v4.z; tv[e4 * 4 + 3] = v4.w;
-                }
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    if (qq * 16 + e > i) tv[e] = 0.f;  // blocks above the diagonal are never written
-                float bgv[16], bv[16];
-#pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {
-                    const float4 x = *reinterpret_cast<const float4*>(&SS.bg[qq * 16 + 4 * e4]);
-                    const float4 y = *reinterpret_cast<const float4*>(&SS.b[pb][qq * 16 + 4 * e4]);
-                    bgv[4 * e4] = x.x; bgv[4 * e4 + 1] = x.y; bgv[4 * e4 + 2] = x.z; bgv[4 * e4 + 3] = x.w;
-                    bv[4 * e4] = y.x; bv[4 * e4 + 1] = y.y; bv[4 * e4 + 2] = y.z; bv[4 * e4 + 3] = y.w;
-                }
-#pragma unroll
-                for (int m = 0; m < 2; ++m) {
-                    uint32_t w4[4], u4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int jj = m * 8 + 2 * e;
-                        w4[e] = h2(tv[jj] * bgv[jj], tv[jj + 1] * bgv[jj + 1], rflags);
-                        u4[e] = pack_bf16x2(tv[jj] * bv[jj], tv[jj + 1] * bv[jj + 1]);
-                    }
-                    *reinterpret_cast<uint4*>(sm + OFF_AS + sw128(i, qq * 2 + m)) =
-                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    *reinterpret_cast<uint4*>(sm + OFF_AS + 8192 + sw128(i, qq * 2 + m)) =
-                        make_uint4(u4[0], u4[1], u4[2], u4[3]);
                 }
             }
             fence_proxy_async_smem();
@@ -670,12 +686,12 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f32acc_ss(tmem + TM_D0, sdesc_sw128(KQ + kk * 2048, 16384, 1024),
-                                  sdesc_sw128(sbase + OFF_AS + kk * 32, 16, 1024), idw, kk > 0);
+                                  sdesc_sw128(sbase + OFF_WN + pb * 16384 + kk * 32, 16, 1024), idw, kk > 0);
                 const uint32_t idu = idesc_f32acc(128, 64, true, false, true);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f32acc_ss(tmem + TM_DU + pb * 64, sdesc_sw128(VV + kk * 2048, 8192, 1024),
-                                  sdesc_sw128(sbase + OFF_AS + 8192 + kk * 32, 16, 1024), idu,
+                                  sdesc_sw128(sbase + OFF_WN + pb * 16384 + 8192 + kk * 32, 16, 1024), idu,
                                   kk > 0);
                 mma_commit(&SS.mbar[MB_MW]);
             }
