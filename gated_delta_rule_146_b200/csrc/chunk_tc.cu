@@ -106,8 +106,8 @@ enum {
 };
 
 struct Small {
-    float g[2][C], b[2][C];  // raw gates by chunk parity (prep)
-    float G[C];              // log2(e) x in-chunk cumulative log decay (prep, chunk being prepared)
+    float b[2][C];           // beta by chunk parity (prep)
+    float G[2][C];           // log2(e) x in-chunk cumulative log decay, by chunk parity (prep)
     float bg[C];             // beta_i e^(G_i)
     float Kd[2][C];          // e^(G_last - G_i), 0 beyond the chunk, by chunk parity (for the chain)
     float Er[C];             // 2^(G_i - G_ref): row factor of the decay (K rows)
@@ -117,8 +117,8 @@ struct Small {
     float gsum_part[2];      // chain: partial sums of the next chunk's g
     uint64_t mbar[MB_COUNT];
     uint32_t tmem_base;
-    int abort;
-    int split_ok;            // the chunk's decay factors factor into row x column exactly
+    int gflag[2][2];         // a bounded wait gave up: [chain, preparation][alternate waits]
+    int split_ok[2];         // the chunk's decay factors factor into row x column exactly
 };
 static_assert(sizeof(Small) <= 5120, "small shared block");
 
@@ -204,7 +204,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             mbar_init(&SS.mbar[i], (i == MB_PREP || i == MB_PREP + 1) ? kPrep
                                    : (i == MB_CD || i == MB_CD + 1)  ? 128
                                                                      : 1);
-        SS.abort = 0;
+        SS.gflag[0][0] = SS.gflag[0][1] = SS.gflag[1][0] = SS.gflag[1][1] = 0;
         mbar_init_fence();
     }
     tc_fence_before();
@@ -222,12 +222,23 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     auto gate_bits_at = [&](const void* arr, int pos) -> uint32_t {
         return load_gate_bits(arr, (size_t)(tokA + tstep * pos) * p.Hv + h, p.gt);
     };
+    // the warpgroup agrees that every thread's wait succeeded: a thread whose wait gave up
+    // raises its group's flag before a plain barrier and every thread reads it after.  Flags
+    // alternate between consecutive waits, so a thread that has passed this barrier and fails
+    // its next wait never raises the flag a slower thread is still about to read; flags only
+    // ever go up, and a raised one ends the group.
+    int wk = 0;
+    auto group_agree = [&](bool ok, int bar_id) -> bool {
+        volatile int* f = &SS.gflag[bar_id == kBarPrep ? 1 : 0][wk & 1];
+        ++wk;
+        if (!ok) *f = 1;
+        named_bar(bar_id, bar_id == kBarPrep ? kPrep : 128);
+        return *f == 0;
+    };
     // wait for a phase of an mbarrier; the whole warpgroup agrees on the outcome
     auto wg_wait = [&](int idx, uint32_t parity, int bar_id) -> bool {
         const bool ok = mbar_wait_bounded(&SS.mbar[idx], parity, kWaitLimitNs);
-        const int n = bar_id == kBarPrep ? kPrep : 128;
-        const bool all = named_bar_and(bar_id, n, (ok && !SS.abort) ? 1 : 0) != 0;
-        if (!all) SS.abort = 1;
+        const bool all = group_agree(ok, bar_id);
         tc_fence_after();
         return all;
     };
@@ -245,19 +256,17 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
         const __nv_bfloat16* vbase = p.v + (size_t)h * D + cd * 8;
         const long long kq_tok = (long long)p.Hk * D, v_tok = (long long)p.Hv * D;
         auto load_chunk = [&](int c) {
-            if (p.use_tma) {  // forward scans: six 8 KB tensor tiles, issued by one thread
-                if (pt == 32) {
-                    uint64_t* bar = &SS.mbar[MB_LD + c % 3];
-                    const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
-                    const uint32_t vv = sbase + OFF_V + (c & 1) * V_STRIDE;
-                    const int z = (int)(t0 + (long long)c * C);
-                    mbar_expect_tx(bar, 6 * 8192);
+            if (p.use_tma) {  // forward scans: six 8 KB tensor tiles, issued by one thread (pt 128)
+                uint64_t* bar = &SS.mbar[MB_LD + c % 3];
+                const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
+                const uint32_t vv = sbase + OFF_V + (c & 1) * V_STRIDE;
+                const int z = (int)(t0 + (long long)c * C);
+                mbar_expect_tx(bar, 6 * 8192);
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        tma_load_3d(kq + half * 16384, &tm_k, half * 64, hk, z, bar);
-                        tma_load_3d(kq + half * 16384 + 8192, &tm_q, half * 64, hk, z, bar);
-                        tma_load_3d(vv + half * 8192, &tm_v, half * 64, h, z, bar);
-                    }
+                for (int half = 0; half < 2; ++half) {
+                    tma_load_3d(kq + half * 16384, &tm_k, half * 64, hk, z, bar);
+                    tma_load_3d(kq + half * 16384 + 8192, &tm_q, half * 64, hk, z, bar);
+                    tma_load_3d(vv + half * 8192, &tm_v, half * 64, h, z, bar);
                 }
                 return;
             }
@@ -275,21 +284,47 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 cp_async16(vv + off, vbase + tok * v_tok, valid);
             }
         };
-        if (p.use_tma && pt == 32) {
+        if (p.use_tma && pt == 128) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
         }
-        load_chunk(0);
+        if (!p.use_tma || pt == 128) load_chunk(0);
         if (!p.use_tma) cp_async_commit();
+        // in-chunk cumulative log decay (log2 units) of one chunk from its gates, two per lane
+        // (positions 2 lane, 2 lane + 1; 0 past the chunk), into G[par], and whether every
+        // decay factor 2^(G_i - G_j) splits into 2^(G_i - G_ref) 2^(G_ref - G_j) inside the
+        // normal fp32 range (true unless the log2 decay strays more than 110 from G_ref = G_31)
+        auto chunk_cumsum = [&](float a0, float a1, int par) {
+            a0 *= kLog2e;
+            a1 *= kLog2e;
+            const float pair = a0 + a1;
+            float incl = pair;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const float excl = incl - pair;
+            const float G0 = excl + a0, G1 = excl + a0 + a1;
+            SS.G[par][2 * lane] = G0;
+            SS.G[par][2 * lane + 1] = G1;
+            const float Gref = __shfl_sync(0xffffffffu, G1, 15);  // G_31
+            float dev = fmaxf(fabsf(G0 - Gref), fabsf(G1 - Gref));
+            dev = fmaxf(dev, fabsf(excl - Gref));                // G_{i-1} of the pre-read
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, o));
+            if (lane == 0) SS.split_ok[par] = dev <= 110.f;
+        };
         {
             const int Cc0 = min(C, L);
-            if (pt < C) {
-                SS.g[0][pt] = pt < Cc0 ? gate_at(p.g, pt) : 0.f;
-                SS.b[0][pt] = pt < Cc0 ? gate_at(p.beta, pt) : 0.f;
-            }
+            if (pt < C) SS.b[0][pt] = pt < Cc0 ? gate_at(p.beta, pt) : 0.f;
+            if (pw == 1)
+                chunk_cumsum(2 * lane < Cc0 ? gate_at(p.g, 2 * lane) : 0.f,
+                             2 * lane + 1 < Cc0 ? gate_at(p.g, 2 * lane + 1) : 0.f, 0);
         }
-        uint32_t g_nx = 0, b_nx = 0;  // raw bits of the next chunk's gates
+        // raw bits of the next chunk's gates: beta (one per thread), g (two per lane, warp 5)
+        uint32_t b_nx = 0, g_nx0 = 0, g_nx1 = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int pb = c & 1;
             const uint32_t KQ = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
@@ -299,8 +334,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             const bool has_next = c + 1 < nchunks;
 
             // P0: the buffers of chunk c-2 are released once the chain is done with them.  Either
-            //     barrier also publishes this chunk's gates (stored by warps 4 and 5) to the
-            //     cumulative sum below.
+            //     barrier also publishes this chunk's beta and cumulative decay (stored during
+            //     the previous chunk's preparation, or before the loop).
             if (c >= 2) {
                 if (!wg_wait(MB_CD + pb, ((c >> 1) & 1) ^ 1, kBarPrep)) { fail = true; break; }
             } else {
@@ -308,33 +343,22 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             }
             int Cn = 0;
             if (has_next) {
-                load_chunk(c + 1);
-                // in-bounds position for every thread, masked only where the value is stored
+                if (!p.use_tma) load_chunk(c + 1);  // reversed scans: every thread's row copies
+                // in-bounds positions for every thread, masked only where the values are used
                 // (a select on a just-loaded value would wait for the load right here)
                 Cn = min(C, L - (c + 1) * C);
-                const int pos = (c + 1) * C + min(pt & 63, Cn - 1);
-                g_nx = gate_bits_at(p.g, pos);
-                b_nx = gate_bits_at(p.beta, pos);
+                b_nx = gate_bits_at(p.beta, (c + 1) * C + min(pt & 63, Cn - 1));
+                if (pw == 1) {
+                    g_nx0 = gate_bits_at(p.g, (c + 1) * C + min(2 * lane, Cn - 1));
+                    g_nx1 = gate_bits_at(p.g, (c + 1) * C + min(2 * lane + 1, Cn - 1));
+                }
             }
             if (!p.use_tma) cp_async_commit();
-            bool landed = true;
-            if (p.use_tma)
-                landed = mbar_wait_bounded(&SS.mbar[MB_LD + c % 3], (uint32_t)((c / 3) & 1),
-                                           kWaitLimitNs);
-            else
-                cp_async_wait<1>();
-            fence_proxy_async_smem();
-            if (!named_bar_and(kBarPrep, kPrep, (landed && !SS.abort) ? 1 : 0)) {
-                SS.abort = 1;
-                fail = true;
-                break;
-            }
-
-            // P1: D0 = [K;Q] K^T straight from the bf16 tiles (M=128, N=64, K=128).  The L2
-            //     norms scale D0's rows and columns afterwards, so the product starts as soon
-            //     as the tiles land and runs while the operands are normalised.
-            tc_fence_after();
-            if (pt == kPrep - 32) {  // warp 11: the cumsum below keeps warp 4 busy
+            // P1: D0 = [K;Q] K^T straight from the bf16 tiles (M=128, N=64, K=128), issued by
+            //     warp 11 once the tiles have landed.  The L2 norms scale D0's rows and columns
+            //     afterwards, so the product runs while the operands are normalised.
+            auto issue_mma0 = [&]() {
+                tc_fence_after();
                 const uint32_t id = idesc_f32acc(128, 64, false, false, true);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -343,7 +367,19 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                                   sdesc_sw128(KQ + off, 16, 1024), id, kk > 0);
                 }
                 mma_commit(&SS.mbar[MB_M0]);
+            };
+            bool landed = true;
+            if (p.use_tma)
+                landed = mbar_wait_bounded(&SS.mbar[MB_LD + c % 3], (uint32_t)((c / 3) & 1),
+                                           kWaitLimitNs);
+            else
+                cp_async_wait<1>();
+            if (!p.use_tma) fence_proxy_async_smem();  // row copies land through the generic proxy
+            if (!group_agree(landed, kBarPrep)) {
+                fail = true;
+                break;
             }
+            if (pt == kPrep - 32) issue_mma0();
             // P2: half row of [K; Q] -> sum of squares -> fp16 operand in registers: K rows
             //     L2-normalised, Q rows as Q~ = scale e^(G') q / ||q||; rows past the chunk
             //     (tensor tiles carry the following tokens there) become 0.  Stored over the
@@ -351,29 +387,6 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             uint32_t hv[32];
             float inv;  // 1 / ||row|| (1 without normalisation)
             uint8_t* rowp = KQp + hf * 16384;
-            // in-chunk cumsum of g (log2 units; warp 4, while the other warps load), and whether
-            // every decay factor 2^(G_i - G_j) splits into 2^(G_i - G_ref) 2^(G_ref - G_j) inside
-            // the normal fp32 range (true unless the log2 decay strays more than 110 from G_31)
-            if (pw == 0) {
-                const float a0 = SS.g[pb][2 * lane] * kLog2e, a1 = SS.g[pb][2 * lane + 1] * kLog2e;
-                const float pair = a0 + a1;
-                float incl = pair;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += y;
-                }
-                const float excl = incl - pair;
-                const float G0 = excl + a0, G1 = excl + a0 + a1;
-                SS.G[2 * lane] = G0;
-                SS.G[2 * lane + 1] = G1;
-                const float Gref = __shfl_sync(0xffffffffu, G1, 15);  // G_31
-                float dev = fmaxf(fabsf(G0 - Gref), fabsf(G1 - Gref));
-                dev = fmaxf(dev, fabsf(excl - Gref));                // G_{i-1} of the pre-read
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, o));
-                if (lane == 0) SS.split_ok = dev <= 110.f;
-            }
             {
                 uint4 vals[8];
                 float ssq[4] = {0.f, 0.f, 0.f, 0.f};
@@ -395,19 +408,19 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 inv = p.qk_l2norm ? rsqrtf(fmaxf(tot, kNormEps * kNormEps)) : 1.f;
                 if (pt < C) {  // per-token factors; the column factor of D0 (K rows) is 1/||k_j||,
                                // times 2^(G_ref - G_j) when split
-                    const float Gref = SS.G[31];
-                    const float Gi = SS.G[pt];
-                    const float Gr = p.read_pre ? (pt > 0 ? SS.G[pt - 1] : 0.f) : Gi;
-                    SS.Kd[pb][pt] = pt < Cc ? ex2(SS.G[Cc - 1] - Gi) : 0.f;
+                    const float Gref = SS.G[pb][31];
+                    const float Gi = SS.G[pb][pt];
+                    const float Gr = p.read_pre ? (pt > 0 ? SS.G[pb][pt - 1] : 0.f) : Gi;
+                    SS.Kd[pb][pt] = pt < Cc ? ex2(SS.G[pb][Cc - 1] - Gi) : 0.f;
                     SS.bg[pt] = SS.b[pb][pt] * ex2(Gi);
                     SS.Er[pt] = ex2(Gi - Gref);
                     SS.Eq[pt] = ex2(Gr - Gref);
-                    SS.ck[pt] = SS.split_ok ? ex2(Gref - Gi) * inv : inv;
+                    SS.ck[pt] = SS.split_ok[pb] ? ex2(Gref - Gi) * inv : inv;
                 }
                 const int i = r & 63;
                 float f = inv;
                 if (r >= C) {
-                    const float Gr = p.read_pre ? (i > 0 ? SS.G[i - 1] : 0.f) : SS.G[i];
+                    const float Gr = p.read_pre ? (i > 0 ? SS.G[pb][i - 1] : 0.f) : SS.G[pb][i];
                     f = p.scale * ex2(Gr) * inv;
                 }
                 if (i >= Cc) f = 0.f;
@@ -433,9 +446,11 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             //     rows 0-63) and P (fp16, rows 64-127); the fp16 operands go over the bf16 tile
             //     (read by the product) while the accumulator load is in flight
             {
+                // warp 8 has no store here: it issues the next chunk's tensor loads
+                if (p.use_tma && has_next && pt == 128) load_chunk(c + 1);
                 const int i = r & 63;
                 const bool live = i < Cc;
-                const bool split = SS.split_ok;
+                const bool split = SS.split_ok[pb];
                 float* As = reinterpret_cast<float*>(sm + OFF_AS);
                 uint32_t rr[32];
                 tmem_ld32(tlane + TM_D0 + hf * 32, rr);
@@ -451,8 +466,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         make_uint4(hv[c8 * 4], hv[c8 * 4 + 1], hv[c8 * 4 + 2], hv[c8 * 4 + 3]);
                 // row factor (beta_i / ||k_i|| or scale / ||q_i||, times 2^(G'_i - G_ref) when
                 // split) and, without the split, the per-element decay exponent's row part
-                const float Gi = r < C ? SS.G[i]
-                                       : (p.read_pre ? (i > 0 ? SS.G[i - 1] : 0.f) : SS.G[i]);
+                const float Gi = r < C ? SS.G[pb][i]
+                                       : (p.read_pre ? (i > 0 ? SS.G[pb][i - 1] : 0.f) : SS.G[pb][i]);
                 float fi = live ? (r < C ? SS.b[pb][i] : p.scale) * inv : 0.f;
                 if (split) fi *= r < C ? SS.Er[i] : SS.Eq[i];
                 tmem_wait_ld();
@@ -463,7 +478,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 } else {
 #pragma unroll
                     for (int u = 0; u < 32; ++u)
-                        vals[u] = fi * u2f(rr[u]) * ckv[u] * ex2(Gi - SS.G[hf * 32 + u]);
+                        vals[u] = fi * u2f(rr[u]) * ckv[u] * ex2(Gi - SS.G[pb][hf * 32 + u]);
                 }
                 // The solve reads the 16x16 blocks of A below the diagonal and the diagonal
                 // blocks (strictly lower part, transposed); the rest of A is never read.  Warp 5
@@ -475,6 +490,10 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     for (int e4 = 0; e4 < 8; ++e4)
                         *reinterpret_cast<float4*>(f32sw(As, i, e4 * 4)) =
                             make_float4(vals[e4 * 4], vals[e4 * 4 + 1], vals[e4 * 4 + 2], vals[e4 * 4 + 3]);
+                    // then the next chunk's cumulative decay, off the critical path
+                    if (has_next)
+                        chunk_cumsum(2 * lane < Cn ? gate_bits_to_float(g_nx0, p.gt) : 0.f,
+                                     2 * lane + 1 < Cn ? gate_bits_to_float(g_nx1, p.gt) : 0.f, pb ^ 1);
                 } else if (pw == 0 || pw == 5) {
                     const bool hi = lane >= 16;
                     const int il = i & 15;
@@ -711,10 +730,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         h8(f, rflags);
                 }
             }
-            if (has_next && pt < C) {
-                SS.g[pb ^ 1][pt] = pt < Cn ? gate_bits_to_float(g_nx, p.gt) : 0.f;
-                SS.b[pb ^ 1][pt] = pt < Cn ? gate_bits_to_float(b_nx, p.gt) : 0.f;
-            }
+            if (has_next && pt < C) SS.b[pb ^ 1][pt] = pt < Cn ? gate_bits_to_float(b_nx, p.gt) : 0.f;
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&SS.mbar[MB_PREP + pb]);

@@ -202,24 +202,11 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
                      smem_u32(bar))
                  : "memory");
 }
-// Named barriers in the non-aligned form, which counts arriving threads one by one: the
-// lanes of a warp may reach them apart (after a lane-divergent branch) without the warp
-// being counted twice or early.
-// Barrier over `n` threads with id `id` (1..15); returns 1 iff `ok` holds on every thread.
-__device__ __forceinline__ int named_bar_and(int id, int n, int ok) {
-    uint32_t out;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 q, %1, 0;\n\t"
-        "barrier.red.and.pred p, %2, %3, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(out)
-        : "r"(ok), "r"(id), "r"(n)
-        : "memory");
-    return (int)out;
-}
+// Named barrier over `n` threads with id `id` (1..15), through the compiler's barrier
+// intrinsic, so that every warp reaches it converged (lanes returning from a lane-divergent
+// branch included).
 __device__ __forceinline__ void named_bar(int id, int n) {
-    asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+    __barrier_sync_count((unsigned)id, (unsigned)n);
 }
 
 // ---- fast base-2 exponential (hardware approximation, flushes subnormal results to 0) ----
