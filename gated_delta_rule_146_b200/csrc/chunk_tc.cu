@@ -102,7 +102,8 @@ enum {
     MB_PREP = 5,  // x2: chunk prepared (by chunk parity)
     MB_LD = 7,    // x3: K, Q, V tiles of a chunk landed (by K/Q buffer)
     MB_CD = 10,   // x2: chain finished with a chunk's buffers (by chunk parity)
-    MB_COUNT = 12
+    MB_MU = 12,   // U~ product of a chunk done (awaited by the chain's MMA issuer)
+    MB_COUNT = 13
 };
 
 struct Small {
@@ -638,6 +639,10 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 {
                     Frag a;
                     Blk Y, E1, E2;  // E1, E2: the E blocks a warp keeps for phases 2 and 3
+                    // E_32 passes from warp 8 (which forms it) to warp 9 (which needs it in phase
+                    // 3) through the transposed-diagonal buffer, free after stage 0, one
+                    // accumulator block per lane
+                    float* e32 = reinterpret_cast<float*>(sm + OFF_RS) + lane * 8;
                     if (pw < 6) {
                         const int r = pw < 3 ? pw + 1 : (pw == 3 ? 2 : 3);
                         const int l = pw < 3 ? pw : (pw == 4 ? 1 : 0);
@@ -645,7 +650,10 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         frag_smem(a, Ts, r, r);
                         bprod(E, a, As, r, l, false);
                         if (pw >= 3) bprod(E1, a, As, r, l + 1, false);  // E_21, E_32, E_31
-                        if (pw == 5) bprod(E2, a, As, r, 2, false);       // E_32
+                        if (pw == 4) {
+                            *reinterpret_cast<float4*>(e32) = make_float4(E1[0][0], E1[0][1], E1[0][2], E1[0][3]);
+                            *reinterpret_cast<float4*>(e32 + 4) = make_float4(E1[1][0], E1[1][1], E1[1][2], E1[1][3]);
+                        }
                         frag_reg(a, E);
                         bprod(Y, a, Ts, l, l, false);
                         if (pw < 2) store_neg(Ts, r, l, Y);  // T_10, T_21: read in phase 2
@@ -688,6 +696,10 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     }
                     named_bar(kBarPrep, kPrep);
                     if (pw == 5) {
+                        const float4 x0 = *reinterpret_cast<const float4*>(e32);
+                        const float4 x1 = *reinterpret_cast<const float4*>(e32 + 4);
+                        E2[0][0] = x0.x; E2[0][1] = x0.y; E2[0][2] = x0.z; E2[0][3] = x0.w;
+                        E2[1][0] = x1.x; E2[1][1] = x1.y; E2[1][2] = x1.z; E2[1][3] = x1.w;
                         frag_reg(a, E2);
                         bprod(Y, a, Ts, 2, 0, true);
                         put_twu(3, 0, Y);
@@ -706,13 +718,14 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f32acc_ss(tmem + TM_D0, sdesc_sw128(KQ + kk * 2048, 16384, 1024),
                                   sdesc_sw128(sbase + OFF_WN + pb * 16384 + kk * 32, 16, 1024), idw, kk > 0);
+                mma_commit(&SS.mbar[MB_MW]);  // W^T: all P6 needs
                 const uint32_t idu = idesc_f32acc(128, 64, true, false, true);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f32acc_ss(tmem + TM_DU + pb * 64, sdesc_sw128(VV + kk * 2048, 8192, 1024),
                                   sdesc_sw128(sbase + OFF_WN + pb * 16384 + 8192 + kk * 32, 16, 1024), idu,
                                   kk > 0);
-                mma_commit(&SS.mbar[MB_MW]);
+                mma_commit(&SS.mbar[MB_MU]);  // U~^T: awaited by the chain before V' accumulates
             }
             if (!wg_wait(MB_MW, c & 1, kBarPrep)) { fail = true; break; }
 
@@ -776,8 +789,12 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             if (has_next) g_raw = gate_bits_at(p.g, (c + 1) * C + min(lt & 63, Cn - 1));
 
             if (!wg_wait(MB_PREP + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
-            // C1: V'^T = U~^T + H^T (-W^T);  O^T = H^T Q~^T   (A = state copy in TMEM)
-            if (lt == 0) {
+            // C1: V'^T = U~^T + H^T (-W^T);  O^T = H^T Q~^T   (A = state copy in TMEM), once the
+            //     preparation's U~ product has landed (a failed wait skips the products: the
+            //     chain's next wait then gives up and the group agrees to stop)
+            if (lt == 0 &&
+                mbar_wait_bounded(&SS.mbar[MB_MU], (uint32_t)(c & 1), kWaitLimitNs)) {
+                tc_fence_after();
                 const uint32_t id1 = idesc_f32acc(128, 64, false, true, false);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
