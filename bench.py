@@ -223,6 +223,34 @@ def bench_ours(args, rank, world, local_rank):
     hbm_gbs = algo_bytes / (ms / 1e3) / 1e9
     launches_per_call = 2 if path == "tc" else 3
 
+    # ---------------- same forward through the fused gating prologue (raw a, b projections)
+    gating = None
+    if not args.no_gating and args.only != "decode":
+        a_raw, b_raw, A_h, dt_h = (t.to(dev) for t in workloads.raw_gate_inputs(
+            tuple(d["g"].shape), w.Hv, w.gate_dtype, seed=rank))
+
+        def gstep():
+            gdr.chunk_fwd(d["q"], d["k"], d["v"], a_raw, b_raw, d["S0"], d["cu_seqlens"],
+                          chunk=w.chunk, read_mode=w.read_mode, scale=w.scale, o=o,
+                          S_final=S_final, workspace=ws, gate_A=A_h, gate_dt_bias=dt_h)
+
+        for _ in range(args.warmup):
+            gstep()
+        torch.cuda.synchronize()
+        barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            gstep()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        gms = max_over_ranks(g0.elapsed_time(g1) / args.steps, world)
+        gating = {"ms_per_step": gms, "value": whole_job_rate(tokens, world, gms),
+                  "unit": "tokens/s", "overhead_vs_given_gates": gms / ms - 1.0,
+                  "inputs": "raw a ~ N(-2,1), b ~ N(0,1) with A = -1, dt_bias = 0 "
+                            "(same gate distributions as the workload)"}
+
     # ---------------- decode step
     dec = None
     if not args.no_decode and args.only != "chunk":
@@ -316,7 +344,7 @@ def bench_ours(args, rank, world, local_rank):
                      "tensor_frac": tflops / peaks["bf16_tflops"],
                      "timed": "whole gdr_chunk_fwd call (plan + chunk kernels), CUDA events",
                      "peak_source": f"{peak_src} (hbm_gbs copy; bf16_tflops burst)"},
-        "decode": dec, "e2e": e2e, "clocks": clocks,
+        "decode": dec, "gating_prologue": gating, "e2e": e2e, "clocks": clocks,
         "gpu_launches": launches_per_call * args.steps,
     }
     return line, x, w
@@ -379,6 +407,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=CHUNK_WORKLOAD)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-gating", action="store_true",
+                    help="skip the forward through the fused gating prologue")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["all", "chunk", "decode"], default="all",

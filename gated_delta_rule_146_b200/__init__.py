@@ -57,8 +57,25 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _gating_fields(gate_A, gate_dt_bias, beta_scale):
+    """(gate_raw, A pointer, dt_bias pointer, beta_scale) of the fused gating prologue:
+    with gate_A ([Hv] fp32, = -exp(A_log)) and gate_dt_bias ([Hv] fp32) given, g and beta
+    are the raw projections a, b and the kernels form g = A softplus(a + dt_bias),
+    beta = beta_scale sigmoid(b)."""
+    if (gate_A is None) != (gate_dt_bias is None):
+        raise ValueError("gate_A and gate_dt_bias come together")
+    if gate_A is None:
+        return 0, None, None, float(beta_scale)
+    import torch
+    for t in (gate_A, gate_dt_bias):
+        if t.dtype != torch.float32 or t.dim() != 1 or not t.is_contiguous():
+            raise TypeError("gate_A and gate_dt_bias are contiguous float32 [Hv] tensors")
+    return 1, gate_A.data_ptr(), gate_dt_bias.data_ptr(), float(beta_scale)
+
+
 def make_chunk_args(q, v, g, cu_seqlens=None, chunk=64, read_mode="post", scale=None,
-                    qk_l2norm=True, reverse=False, o_accumulate=False):
+                    qk_l2norm=True, reverse=False, o_accumulate=False, gate_A=None,
+                    gate_dt_bias=None, beta_scale=1.0):
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
@@ -66,7 +83,8 @@ def make_chunk_args(q, v, g, cu_seqlens=None, chunk=64, read_mode="post", scale=
         scale = 1.0 / math.sqrt(dk)
     return ChunkArgs(B, T, Hk, Hv, dk, dv, n_seqs, chunk, _dtype_code(q), _dtype_code(g),
                      READ_PRE if read_mode == "pre" else READ_POST, float(scale),
-                     int(bool(qk_l2norm)), int(bool(reverse)), int(bool(o_accumulate)))
+                     int(bool(qk_l2norm)), int(bool(reverse)), int(bool(o_accumulate)),
+                     *_gating_fields(gate_A, gate_dt_bias, beta_scale))
 
 
 def chunk_fwd_workspace_size(args: ChunkArgs) -> int:
@@ -80,14 +98,17 @@ def chunk_fwd_path(args: ChunkArgs):
 
 def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, *, chunk=64, read_mode="post",
               scale=None, qk_l2norm=True, reverse=False, o=None, o_accumulate=False,
-              output_final_state=True, S_final=None, workspace=None, stream=None):
+              output_final_state=True, S_final=None, workspace=None, stream=None,
+              gate_A=None, gate_dt_bias=None, beta_scale=1.0):
     """Chunk-parallel forward (gdr_chunk_fwd).  Shapes: q, k [B,T,Hk,dk]; v [B,T,Hv,dv];
     g, beta [B,T,Hv]; S0 [n_seqs,Hv,dk,dv] fp32 or None; cu_seqlens int32 [n_seqs+1] or
-    None.  Returns (o [B,T,Hv,dv], S_final [n_seqs,Hv,dk,dv] fp32 or None)."""
+    None.  With gate_A and gate_dt_bias ([Hv] fp32) given, g and beta are the raw
+    projections a and b of the fused gating prologue.  Returns (o [B,T,Hv,dv],
+    S_final [n_seqs,Hv,dk,dv] fp32 or None)."""
     import torch
-    _check_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_final, workspace)
+    _check_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_final, workspace, gate_A, gate_dt_bias)
     args = make_chunk_args(q, v, g, cu_seqlens, chunk, read_mode, scale, qk_l2norm, reverse,
-                           o_accumulate)
+                           o_accumulate, gate_A, gate_dt_bias, beta_scale)
     if k.dtype != q.dtype or v.dtype != q.dtype or beta.dtype != g.dtype:
         raise TypeError("q, k, v share one dtype and g, beta another")
     if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
@@ -120,25 +141,29 @@ def read_device_error(args: ChunkArgs, workspace, stream=None) -> int:
                                                 _stream(stream)))
 
 
-def make_decode_args(q, v, g, read_mode="post", scale=None, qk_l2norm=True):
+def make_decode_args(q, v, g, read_mode="post", scale=None, qk_l2norm=True, gate_A=None,
+                     gate_dt_bias=None, beta_scale=1.0):
     N, Hk, dk = q.shape
     Hv, dv = v.shape[1], v.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(dk)
     return DecodeArgs(N, Hk, Hv, dk, dv, _dtype_code(q), _dtype_code(g),
                       READ_PRE if read_mode == "pre" else READ_POST, float(scale),
-                      int(bool(qk_l2norm)))
+                      int(bool(qk_l2norm)), *_gating_fields(gate_A, gate_dt_bias, beta_scale))
 
 
 def decode_step(q, k, v, g, beta, S, *, read_mode="post", scale=None, qk_l2norm=True, o=None,
-                stream=None):
+                stream=None, gate_A=None, gate_dt_bias=None, beta_scale=1.0):
     """One recurrent token per sequence (gdr_decode_step): q, k [N,Hk,dk]; v [N,Hv,dv];
-    g, beta [N,Hv]; S [N,Hv,dk,dv] fp32, updated in place.  Returns o [N,Hv,dv]."""
+    g, beta [N,Hv]; S [N,Hv,dk,dv] fp32, updated in place.  With gate_A and gate_dt_bias
+    ([Hv] fp32) given, g and beta are the raw projections of the fused gating prologue.
+    Returns o [N,Hv,dv]."""
     import torch
-    _check_cuda(q, k, v, g, beta, S, o)
+    _check_cuda(q, k, v, g, beta, S, o, gate_A, gate_dt_bias)
     if S.dtype != torch.float32:
         raise TypeError("the state must be float32")
-    args = make_decode_args(q, v, g, read_mode, scale, qk_l2norm)
+    args = make_decode_args(q, v, g, read_mode, scale, qk_l2norm, gate_A, gate_dt_bias,
+                            beta_scale)
     if o is None:
         o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     st = _abi.lib().gdr_decode_step(ctypes.byref(args), _ptr(q), _ptr(k), _ptr(v), _ptr(g),

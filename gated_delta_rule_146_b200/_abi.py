@@ -26,14 +26,18 @@ class ChunkArgs(ctypes.Structure):
                 ("n_seqs", ctypes.c_int), ("chunk", ctypes.c_int), ("io_dtype", ctypes.c_int),
                 ("gate_dtype", ctypes.c_int), ("read_mode", ctypes.c_int),
                 ("scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int),
-                ("reverse", ctypes.c_int), ("o_accumulate", ctypes.c_int)]
+                ("reverse", ctypes.c_int), ("o_accumulate", ctypes.c_int),
+                ("gate_raw", ctypes.c_int), ("gate_A", ctypes.c_void_p),
+                ("gate_dt_bias", ctypes.c_void_p), ("beta_scale", ctypes.c_float)]
 
 
 class DecodeArgs(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int), ("Hk", ctypes.c_int), ("Hv", ctypes.c_int),
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("io_dtype", ctypes.c_int),
                 ("gate_dtype", ctypes.c_int), ("read_mode", ctypes.c_int),
-                ("scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int)]
+                ("scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int),
+                ("gate_raw", ctypes.c_int), ("gate_A", ctypes.c_void_p),
+                ("gate_dt_bias", ctypes.c_void_p), ("beta_scale", ctypes.c_float)]
 
 
 class GdrError(RuntimeError):

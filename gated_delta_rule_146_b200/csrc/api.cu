@@ -3,6 +3,7 @@
 // Nothing here allocates device memory, synchronises (except the diagnostic
 // gdr_read_device_error) or keeps state between calls; every entry point only
 // checks its arguments and enqueues kernels on the caller's stream.
+#include <cmath>
 #include <cstring>
 
 #include "common.cuh"
@@ -22,6 +23,20 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool valid_dtype(gdr_dtype d) { return d == GDR_F32 || d == GDR_BF16; }
 
+// Fused gating fields: flags, the scale, and (for a call) the per-head arrays.
+template <typename Args>
+gdr_status check_gating(const Args* a, bool pointers) {
+    if (a->gate_raw & ~1) return GDR_ERR_INVALID_ARG;
+    if (!a->gate_raw) return GDR_OK;
+    if (!std::isfinite(a->beta_scale)) return GDR_ERR_INVALID_ARG;
+    if (pointers) {
+        if (!a->gate_A || !a->gate_dt_bias) return GDR_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(a->gate_A) | reinterpret_cast<uintptr_t>(a->gate_dt_bias)) & 3u)
+            return GDR_ERR_ALIGNMENT;
+    }
+    return GDR_OK;
+}
+
 // Shape/enum validation shared by workspace_size, path and chunk_fwd.
 gdr_status check_chunk_args(const gdr_chunk_args* a) {
     if (!a) return GDR_ERR_INVALID_ARG;
@@ -33,6 +48,7 @@ gdr_status check_chunk_args(const gdr_chunk_args* a) {
     if (!valid_dtype(a->io_dtype) || !valid_dtype(a->gate_dtype)) return GDR_ERR_INVALID_ARG;
     if (a->read_mode != GDR_READ_POST && a->read_mode != GDR_READ_PRE) return GDR_ERR_INVALID_ARG;
     if ((a->qk_l2norm | a->reverse | a->o_accumulate) & ~1) return GDR_ERR_INVALID_ARG;
+    if (check_gating(a, false) != GDR_OK) return GDR_ERR_INVALID_ARG;
     const long long T_tot = (long long)a->B * a->T;
     if (T_tot * a->Hv * (a->dk > a->dv ? a->dk : a->dv) >= (1LL << 40)) return GDR_ERR_INVALID_ARG;
     if (T_tot > 0x7fffffffLL || (long long)a->n_seqs * a->Hv > 0x7fffffffLL)
@@ -82,6 +98,7 @@ gdr_status gdr_chunk_fwd(const gdr_chunk_args* a, const void* q, const void* k, 
     }
     const bool has_tokens = (long long)a->B * a->T > 0;
     if (has_tokens && (!q || !k || !v || !g || !beta || !o)) return GDR_ERR_INVALID_ARG;
+    if ((st = check_gating(a, true)) != GDR_OK) return st;
     if (!workspace) return GDR_ERR_WORKSPACE;
     const void* ptrs[] = {q, k, v, g, beta, S0, cu_seqlens, o, S_final, workspace};
     for (const void* p : ptrs)
@@ -108,10 +125,12 @@ gdr_status gdr_decode_step(const gdr_decode_args* a, const void* q, const void* 
     if (!valid_dtype(a->io_dtype) || !valid_dtype(a->gate_dtype)) return GDR_ERR_INVALID_ARG;
     if (a->read_mode != GDR_READ_POST && a->read_mode != GDR_READ_PRE) return GDR_ERR_INVALID_ARG;
     if (a->qk_l2norm & ~1) return GDR_ERR_INVALID_ARG;
+    if (check_gating(a, false) != GDR_OK) return GDR_ERR_INVALID_ARG;
     if ((long long)a->N * a->Hv > 0x7fffffffLL) return GDR_ERR_INVALID_ARG;
     if (!decode_supported(*a)) return GDR_ERR_UNSUPPORTED;
     if (a->N == 0) return GDR_OK;
     if (!q || !k || !v || !g || !beta || !S_inout || !o) return GDR_ERR_INVALID_ARG;
+    if (const gdr_status gs = check_gating(a, true); gs != GDR_OK) return gs;
     const void* ptrs[] = {q, k, v, g, beta, S_inout, o};
     for (const void* p : ptrs)
         if (!aligned16(p)) return GDR_ERR_ALIGNMENT;

@@ -40,6 +40,9 @@ struct SimtParams {
     int Hk, Hv, dk, dv, chunk, read_pre, qk_l2norm, reverse, o_acc;
     gdr_dtype io, gt;
     float scale;
+    int gate_raw;                 // fused gating prologue (see gate_xform)
+    const float* gate_A; const float* gate_dt_bias;
+    float beta_scale;
 };
 
 // Normalise `rows` rows of length n (row stride ld) in shared memory, one warp per row.
@@ -87,8 +90,8 @@ chunk_local_simt(SimtParams p) {
     }
     for (int i = tid; i < Cc; i += kThreads) {
         const long long t = phys_token(t0, t1, p0 + i, p.reverse);
-        Gs[i] = load_elem(p.g, (size_t)t * p.Hv + h, p.gt);
-        Bs[i] = load_elem(p.beta, (size_t)t * p.Hv + h, p.gt);
+            Gs[i] = xform_g(p, h, load_elem(p.g, (size_t)t * p.Hv + h, p.gt));
+        Bs[i] = xform_beta(p, load_elem(p.beta, (size_t)t * p.Hv + h, p.gt));
     }
     __syncthreads();
     if (p.qk_l2norm) l2norm_rows(R, Cc, dk, ld);
@@ -278,6 +281,8 @@ gdr_status launch_chunk_simt(const gdr_chunk_args& a, const void* q, const void*
     p.Hk = a.Hk; p.Hv = a.Hv; p.dk = a.dk; p.dv = a.dv; p.chunk = a.chunk;
     p.read_pre = a.read_mode == GDR_READ_PRE; p.qk_l2norm = a.qk_l2norm; p.reverse = a.reverse;
     p.o_acc = a.o_accumulate; p.io = a.io_dtype; p.gt = a.gate_dtype; p.scale = a.scale;
+    p.gate_raw = a.gate_raw; p.gate_A = a.gate_A; p.gate_dt_bias = a.gate_dt_bias;
+    p.beta_scale = a.beta_scale;
 
     const size_t sm1 = local_smem(a), sm2 = scan_smem(a);
     if ((cudaFuncSetAttribute(chunk_local_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,

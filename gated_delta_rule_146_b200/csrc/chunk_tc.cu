@@ -134,6 +134,13 @@ struct TcParams {
     float scale;
 };
 
+// The fused gating prologue's per-head arrays, a kernel argument of its own that only the
+// gated instantiation reads (the plain kernel's parameter block stays as it is).
+struct GateParams {
+    const float* A; const float* dt_bias;
+    float beta_scale;
+};
+
 // fp16 pair; `mx` keeps the running maximum magnitude of every half produced (NaN sticks),
 // tested once at the end: an infinite or NaN half means the value left the fp16 range.
 __device__ __forceinline__ uint32_t h2(float a, float b, __half2& mx) {
@@ -164,10 +171,13 @@ __device__ __forceinline__ float gate_bits_to_float(uint32_t b, gdr_dtype dt) {
     return __uint_as_float(dt == GDR_BF16 ? b << 16 : b);
 }
 
+// kRaw: the fused gating prologue is compiled into this instantiation only, so the plain-gate
+// kernel carries none of its code or register pressure.
+template <bool kRaw>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-               const __grid_constant__ CUtensorMap tm_o) {
+               const __grid_constant__ CUtensorMap tm_o, const GateParams gp) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base, as a byte offset from the shared array so that every access
     // through it stays a shared-memory access (an integer round trip would make them generic)
@@ -180,6 +190,15 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     if (p.hdr->err != GDR_OK) return;
 
     const int s = blockIdx.x, h = blockIdx.y;
+    // the gates as the recurrence uses them (fused gating prologue when kRaw)
+    auto XG = [&](float a) -> float {
+        if constexpr (kRaw) return gate_g_from_raw(gp.A[h], gp.dt_bias[h], a);
+        else return a;
+    };
+    auto XB = [&](float b) -> float {
+        if constexpr (kRaw) return gate_beta_from_raw(gp.beta_scale, b);
+        else return b;
+    };
     const int hk = h / (p.Hv / p.Hk);
     const long long t0 = p.cu[s], t1 = p.cu[s + 1];
     const int L = (int)(t1 - t0);
@@ -319,10 +338,10 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
         };
         {
             const int Cc0 = min(C, L);
-            if (pt < C) SS.b[0][pt] = pt < Cc0 ? gate_at(p.beta, pt) : 0.f;
+            if (pt < C) SS.b[0][pt] = pt < Cc0 ? XB(gate_at(p.beta, pt)) : 0.f;
             if (pw == 1)
-                chunk_cumsum(2 * lane < Cc0 ? gate_at(p.g, 2 * lane) : 0.f,
-                             2 * lane + 1 < Cc0 ? gate_at(p.g, 2 * lane + 1) : 0.f, 0);
+                chunk_cumsum(2 * lane < Cc0 ? XG(gate_at(p.g, 2 * lane)) : 0.f,
+                             2 * lane + 1 < Cc0 ? XG(gate_at(p.g, 2 * lane + 1)) : 0.f, 0);
         }
         // raw bits of the next chunk's gates: beta (one per thread), g (two per lane, warp 5)
         uint32_t b_nx = 0, g_nx0 = 0, g_nx1 = 0;
@@ -493,8 +512,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                             make_float4(vals[e4 * 4], vals[e4 * 4 + 1], vals[e4 * 4 + 2], vals[e4 * 4 + 3]);
                     // then the next chunk's cumulative decay, off the critical path
                     if (has_next)
-                        chunk_cumsum(2 * lane < Cn ? gate_bits_to_float(g_nx0, p.gt) : 0.f,
-                                     2 * lane + 1 < Cn ? gate_bits_to_float(g_nx1, p.gt) : 0.f, pb ^ 1);
+                        chunk_cumsum(2 * lane < Cn ? XG(gate_bits_to_float(g_nx0, p.gt)) : 0.f,
+                                     2 * lane + 1 < Cn ? XG(gate_bits_to_float(g_nx1, p.gt)) : 0.f,
+                                     pb ^ 1);
                 } else if (pw == 0 || pw == 5) {
                     const bool hi = lane >= 16;
                     const int il = i & 15;
@@ -743,7 +763,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         h8(f, rflags);
                 }
             }
-            if (has_next && pt < C) SS.b[pb ^ 1][pt] = pt < Cn ? gate_bits_to_float(b_nx, p.gt) : 0.f;
+            if (has_next && pt < C)
+                SS.b[pb ^ 1][pt] = pt < Cn ? XB(gate_bits_to_float(b_nx, p.gt)) : 0.f;
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&SS.mbar[MB_PREP + pb]);
@@ -754,7 +775,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
         const int j = lt;  // dv column = TMEM lane
         {
             // initial state -> TM_HM (pre-scaled by chunk 0's total decay), TM_HB (fp16)
-            const float gv = lt < min(C, L) ? gate_at(p.g, lt) : 0.f;
+            const float gv = lt < min(C, L) ? XG(gate_at(p.g, lt)) : 0.f;
             const float part = warp_sum(gv);
             if (lane == 0 && warp < 2) SS.gsum_part[warp] = part;
             named_bar(kBarChain, 128);
@@ -839,7 +860,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 }
                 tmem_wait_st();
                 if (warp < 2) {
-                    const float part = warp_sum(lt < Cn ? gate_bits_to_float(g_raw, p.gt) : 0.f);
+                    const float part = warp_sum(lt < Cn ? XG(gate_bits_to_float(g_raw, p.gt)) : 0.f);
                     if (lane == 0) SS.gsum_part[warp] = part;
                 }
             }
@@ -1017,6 +1038,7 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
     p.Hk = a.Hk; p.Hv = a.Hv; p.read_pre = a.read_mode == GDR_READ_PRE;
     p.qk_l2norm = a.qk_l2norm; p.reverse = a.reverse; p.o_acc = a.o_accumulate;
     p.gt = a.gate_dtype; p.scale = a.scale;
+    const GateParams gp{a.gate_A, a.gate_dt_bias, a.beta_scale};
     CUtensorMap tq, tk, tv, to;
     memset(&tq, 0, sizeof(tq));
     memset(&tk, 0, sizeof(tk));
@@ -1033,11 +1055,12 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
         // accumulating outputs are read back, so they keep the plain stores
         p.tma_store = !a.o_accumulate && make_tile_map(&to, o, a.Hv, T_tot);
     }
-    if (cudaFuncSetAttribute(chunk_fused_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto kernel = a.gate_raw ? chunk_fused_tc<true> : chunk_fused_tc<false>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
     dim3 grid((unsigned)a.n_seqs, (unsigned)a.Hv);
-    chunk_fused_tc<<<grid, kThreads, SMEM_BYTES, st>>>(p, tq, tk, tv, to);
+    kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p, tq, tk, tv, to, gp);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

@@ -23,6 +23,32 @@ __device__ __forceinline__ void store_elem(void* p, size_t i, float x, gdr_dtype
     else static_cast<float*>(p)[i] = x;
 }
 
+// ---- fused gating prologue ---------------------------------------------------
+// Raw per-token projections a, b -> g = A softplus(a + dt_bias), beta = beta_scale sigmoid(b)
+// (sparse_delta_memory/layer.py compute_gates, with the doubled beta of tiny_gdn/fugue.py
+// `project`); the identity when the gates are given.  `P` is a kernel's parameter block
+// (fields gate_raw, gate_A, gate_dt_bias, beta_scale), read where used so that nothing stays
+// live in registers, and the math is out of line, so that the kernels' register allocation
+// does not carry a branch that plain gates never take.
+static __device__ __noinline__ float gate_g_from_raw(float A, float dt, float a) {
+    const float x = a + dt;
+    return A * (x > 20.f ? x : log1pf(expf(x)));
+}
+
+static __device__ __noinline__ float gate_beta_from_raw(float scale, float b) {
+    return scale / (1.f + expf(-b));
+}
+
+template <typename P>
+__device__ __forceinline__ float xform_g(const P& p, int h, float a) {
+    return p.gate_raw ? gate_g_from_raw(p.gate_A[h], p.gate_dt_bias[h], a) : a;
+}
+
+template <typename P>
+__device__ __forceinline__ float xform_beta(const P& p, float b) {
+    return p.gate_raw ? gate_beta_from_raw(p.beta_scale, b) : b;
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);

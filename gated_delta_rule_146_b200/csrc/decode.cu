@@ -29,6 +29,9 @@ struct DecodeParams {
     int Hk, Hv, read_pre, qk_l2norm;
     gdr_dtype io, gt;
     float scale;
+    int gate_raw;                 // fused gating prologue (see gate_xform)
+    const float* gate_A; const float* gate_dt_bias;
+    float beta_scale;
 };
 
 template <int DK, int DV, int DVS>
@@ -67,8 +70,8 @@ decode_kernel(DecodeParams p) {
         s_k[d] = load_elem(p.k, qk_base + d, p.io);
     }
     if (tid == 0) {
-        s_alpha = expf(load_elem(p.g, (size_t)nh, p.gt));
-        s_beta = load_elem(p.beta, (size_t)nh, p.gt);
+            s_alpha = expf(xform_g(p, h, load_elem(p.g, (size_t)nh, p.gt)));
+        s_beta = xform_beta(p, load_elem(p.beta, (size_t)nh, p.gt));
     }
     __syncthreads();
     if (wid < 3) {
@@ -170,6 +173,8 @@ gdr_status launch_decode(const gdr_decode_args& a, const void* q, const void* k,
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.S = S; p.o = o;
     p.Hk = a.Hk; p.Hv = a.Hv; p.read_pre = a.read_mode == GDR_READ_PRE;
     p.qk_l2norm = a.qk_l2norm; p.io = a.io_dtype; p.gt = a.gate_dtype; p.scale = a.scale;
+    p.gate_raw = a.gate_raw; p.gate_A = a.gate_A; p.gate_dt_bias = a.gate_dt_bias;
+    p.beta_scale = a.beta_scale;
     switch (a.dk) {
         case 32: return launch_dk<32>(a, p, st);
         case 64: return launch_dk<64>(a, p, st);

@@ -91,6 +91,21 @@ typedef struct {
                               sequence's FIRST token */
     int o_accumulate;      /* 1: o += result (o is read, the sum written back in io_dtype);
                               0: o = result */
+    /* Fused gating prologue (sparse_delta_memory/layer.py `compute_gates`: A = -exp(A_log),
+     * g = A * softplus(a + dt_bias), beta = sigmoid(b); tiny_gdn/fugue.py `project`: beta
+     * doubled to allow negative eigenvalues; flashrt fused_layer.py `gdn_gating`).
+     *   gate_raw = 0: g and beta are the gates themselves; the three fields below are unused.
+     *   gate_raw = 1: the g and beta arguments hold the raw per-token projections a and b
+     *                 (same shape and gate_dtype), and the kernels form, in fp32,
+     *                   g    = gate_A[h] * softplus(a + gate_dt_bias[h])
+     *                   beta = beta_scale * sigmoid(b)
+     *                 with softplus(x) = x for x > 20 (as torch's softplus threshold). */
+    int gate_raw;
+    const float* gate_A;        /* [Hv] fp32 device array, A = -exp(A_log) (<= 0 for a decay);
+                                   4-byte aligned; required when gate_raw */
+    const float* gate_dt_bias;  /* [Hv] fp32 device array; 4-byte aligned; required when
+                                   gate_raw */
+    float beta_scale;           /* 1, or 2 for negative eigenvalues; must be finite */
 } gdr_chunk_args;
 
 /* Bytes of device workspace gdr_chunk_fwd needs for these arguments (0 on invalid
@@ -170,6 +185,10 @@ typedef struct {
     gdr_read_mode read_mode;
     float scale;
     int qk_l2norm;
+    int gate_raw;               /* fused gating prologue, exactly as in gdr_chunk_args */
+    const float* gate_A;
+    const float* gate_dt_bias;
+    float beta_scale;
 } gdr_decode_args;
 
 /*

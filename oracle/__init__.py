@@ -17,6 +17,9 @@ Three independent implementations live here:
 * ``exact.forward_exact`` -- exact rational arithmetic through the
   product-of-transitions form; used only to pin the oracle on tiny inputs.
 
+``gating`` forms the gates from raw projections (the fused gating prologue)
+in fp64; the recurrence oracles take its output like any other gates.
+
 Every input arrives already rounded to the dtype the GPU sees (bf16 / fp32);
 it is widened exactly to fp64 here.
 """
@@ -141,3 +144,24 @@ def bidirectional(q, k, v, g_fwd, beta_fwd, g_bwd, beta_bwd, cu_seqlens, read_mo
     o_b, _ = forward(q, k, v, g_bwd, beta_bwd, None, cu_seqlens, read_mode_bwd or read_mode,
                      scale, qk_l2norm, reverse=True)
     return combine * (o_f + o_b)
+
+
+def gating(a, b, A, dt_bias, beta_scale: float = 1.0):
+    """Gates from the raw per-token projections (the fused gating prologue), fp64.
+
+    sparse-delta-memory 2.0.0 ``sparse_delta_memory/layer.py``, ``compute_gates``:
+    ``A = -exp(A_log)`` per head, ``g = A * softplus(a + dt_bias)``, ``beta = sigmoid(b)``;
+    Rondo-Exp ``tiny_gdn/fugue.py``, ``project``: beta doubled to allow negative eigenvalues
+    (``beta_scale = 2``).  ``a``, ``b`` are ``[..., Hv]`` (any dtype, widened exactly);
+    ``A``, ``dt_bias`` are ``[Hv]``.  softplus and sigmoid are evaluated in closed form
+    (``log(1 + e^x)`` and ``1 / (1 + e^-x)``) through their overflow-free rearrangements;
+    torch's softplus returns ``x`` itself above 20, within 2e-9 relative of this.
+    Returns ``(g, beta)`` as fp64 arrays of ``a``'s shape.
+    """
+    a, b = _f64(a), _f64(b)
+    A, dt_bias = _f64(A), _f64(dt_bias)
+    x = a + dt_bias
+    softplus = np.logaddexp(0.0, x)            # log(1 + e^x)
+    g = A * softplus
+    beta = beta_scale * np.exp(-np.logaddexp(0.0, -b))  # 1 / (1 + e^-b)
+    return g, beta

@@ -99,3 +99,49 @@ def test_decode_host_validation(lib):
     assert f(d, S=FAKE + 8) == _abi.GDR_ERR_ALIGNMENT
     empty = _abi.DecodeArgs(**{**{n: getattr(d, n) for n, _ in d._fields_}, "N": 0})
     assert f(empty) == _abi.GDR_OK  # nothing to do, nothing launched
+
+
+def test_gating_host_validation(lib):
+    """The fused gating fields: flags, scale and per-head arrays are checked on the host."""
+    ok = args(gate_raw=1, gate_A=FAKE, gate_dt_bias=FAKE, beta_scale=2.0)
+    need = lib.gdr_chunk_fwd_workspace_size(ctypes.byref(ok))
+    assert need > 0
+    assert lib.gdr_chunk_fwd_workspace_size(ctypes.byref(args(gate_raw=2))) == 0
+    assert lib.gdr_chunk_fwd_workspace_size(
+        ctypes.byref(args(gate_raw=1, beta_scale=float("inf")))) == 0
+    assert call(lib, args(gate_raw=1, gate_dt_bias=FAKE, beta_scale=1.0),
+                wsb=need) == _abi.GDR_ERR_INVALID_ARG                       # no gate_A
+    assert call(lib, args(gate_raw=1, gate_A=FAKE + 2, gate_dt_bias=FAKE, beta_scale=1.0),
+                wsb=need) == _abi.GDR_ERR_ALIGNMENT
+    assert call(lib, ok, wsb=need - 1) == _abi.GDR_ERR_WORKSPACE            # gating accepted
+    d = _abi.DecodeArgs(N=4, Hk=2, Hv=4, dk=128, dv=128, io_dtype=_abi.BF16,
+                        gate_dtype=_abi.BF16, read_mode=_abi.READ_POST, scale=0.1, qk_l2norm=1,
+                        gate_raw=1, gate_A=None, gate_dt_bias=FAKE, beta_scale=1.0)
+    vp = ctypes.c_void_p
+    assert lib.gdr_decode_step(ctypes.byref(d), *[vp(FAKE)] * 7, None) == _abi.GDR_ERR_INVALID_ARG
+
+
+def test_struct_layout_matches_header(tmp_path):
+    """ctypes mirrors of the argument structs have the C header's size and field offsets."""
+    import shutil
+    import subprocess
+    if not shutil.which("gcc"):
+        pytest.skip("no host C compiler")
+    fields = {"gdr_chunk_args": _abi.ChunkArgs, "gdr_decode_args": _abi.DecodeArgs}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "gdr.h"', "int main(void) {"]
+    for cname, py in fields.items():
+        lines.append(f'printf("%zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'printf("%zu\\n", offsetof({cname}, {fname}));')
+    lines.append("return 0; }")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    want = []
+    for py in fields.values():
+        want.append(ctypes.sizeof(py))
+        want.extend(getattr(py, n).offset for n, _ in py._fields_)
+    assert got == want

@@ -166,3 +166,15 @@ def decode_inputs(N, Hk, Hv, dk, dv, steps, dtype="bf16", gate_dtype=None, s_std
 def decode_workload_inputs(w: DecodeWorkload, seed: int = 0):
     return decode_inputs(w.N, w.Hk, w.Hv, w.dk, w.dv, w.steps, w.dtype, w.gate_dtype, w.s_std,
                          seed)
+
+
+def raw_gate_inputs(shape, Hv, gate_dtype="bf16", seed=0):
+    """Raw gate projections for the fused gating prologue: a ~ N(-2, 1) and b ~ N(0, 1) in
+    the gate dtype, with per-head A = -1 and dt_bias = 0 (fp32), so that the gates the
+    kernels form, g = A softplus(a + dt_bias) and beta = sigmoid(b), follow the same
+    distributions as the workloads' direct gates."""
+    gen = _gen(seed + 7919)
+    dt = DTYPES[gate_dtype]
+    a = (torch.randn(shape, generator=gen) - 2.0).to(dt)
+    b = torch.randn(shape, generator=gen).to(dt)
+    return a, b, torch.full((Hv,), -1.0), torch.zeros(Hv)
