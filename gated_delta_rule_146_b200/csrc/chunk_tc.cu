@@ -173,7 +173,10 @@ __device__ __forceinline__ float gate_bits_to_float(uint32_t b, gdr_dtype dt) {
 
 // kRaw: the fused gating prologue is compiled into this instantiation only, so the plain-gate
 // kernel carries none of its code or register pressure.
-template <bool kRaw>
+// kDh: the head size dk = dv in memory, 128 or 64.  A 64-wide head runs in the same 128-wide
+// tiles with feature columns 64-127 zero (never loaded): the normalisation is unchanged and
+// the state's extra rows and columns receive only zero updates, so they stay zero.
+template <bool kRaw, int kDh>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -203,14 +206,15 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     const long long t0 = p.cu[s], t1 = p.cu[s + 1];
     const int L = (int)(t1 - t0);
     const int nchunks = (L + C - 1) / C;
-    const size_t sb = ((size_t)s * p.Hv + h) * D * D;
+    static_assert(kDh == 64 || kDh == D, "head size");
+    const size_t sb = ((size_t)s * p.Hv + h) * kDh * kDh;
     // physical token of logical position 0, and the step between consecutive positions
     const long long tokA = p.reverse ? t1 - 1 : t0;
     const long long tstep = p.reverse ? -1 : 1;
 
     if (nchunks == 0) {  // empty sequence: the state passes through
         if (p.S_final)
-            for (int e = tid; e < D * D; e += kThreads)
+            for (int e = tid; e < kDh * kDh; e += kThreads)
                 p.S_final[sb + e] = p.S0 ? p.S0[sb + e] : 0.f;
         return;
     }
@@ -226,6 +230,15 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                                                                      : 1);
         SS.gflag[0][0] = SS.gflag[0][1] = SS.gflag[1][0] = SS.gflag[1][1] = 0;
         mbar_init_fence();
+    }
+    if constexpr (kDh < D) {  // feature columns 64-127 of every K/Q and V tile stay zero
+        for (int e = tid; e < 3 * 1024 + 2 * 512; e += kThreads) {
+            const uint32_t off = e < 3072
+                ? OFF_KQ + (e >> 10) * KQ_STRIDE + 16384 + (e & 1023) * 16
+                : OFF_V + ((e - 3072) >> 9) * V_STRIDE + 8192 + ((e - 3072) & 511) * 16;
+            *reinterpret_cast<uint4*>(sm + off) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -271,19 +284,20 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
         const int pw = pt >> 5;        // preparation warp 0..7
         // cp.async plan: this thread copies 16-byte column chunk `cd` of rows r0 + 16 m
         const int cd = pt & 15, r0 = pt >> 4;
-        const __nv_bfloat16* kbase = p.k + (size_t)hk * D + cd * 8;
-        const __nv_bfloat16* qbase = p.q + (size_t)hk * D + cd * 8;
-        const __nv_bfloat16* vbase = p.v + (size_t)h * D + cd * 8;
-        const long long kq_tok = (long long)p.Hk * D, v_tok = (long long)p.Hv * D;
+        const bool cd_in = cd < kDh / 8;  // column chunks past a 64-wide head are zero-filled
+        const __nv_bfloat16* kbase = p.k + (size_t)hk * kDh + (cd_in ? cd : 0) * 8;
+        const __nv_bfloat16* qbase = p.q + (size_t)hk * kDh + (cd_in ? cd : 0) * 8;
+        const __nv_bfloat16* vbase = p.v + (size_t)h * kDh + (cd_in ? cd : 0) * 8;
+        const long long kq_tok = (long long)p.Hk * kDh, v_tok = (long long)p.Hv * kDh;
         auto load_chunk = [&](int c) {
             if (p.use_tma) {  // forward scans: six 8 KB tensor tiles, issued by one thread (pt 128)
                 uint64_t* bar = &SS.mbar[MB_LD + c % 3];
                 const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
                 const uint32_t vv = sbase + OFF_V + (c & 1) * V_STRIDE;
                 const int z = (int)(t0 + (long long)c * C);
-                mbar_expect_tx(bar, 6 * 8192);
+                mbar_expect_tx(bar, 3 * (kDh / 64) * 8192);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
+                for (int half = 0; half < kDh / 64; ++half) {
                     tma_load_3d(kq + half * 16384, &tm_k, half * 64, hk, z, bar);
                     tma_load_3d(kq + half * 16384 + 8192, &tm_q, half * 64, hk, z, bar);
                     tma_load_3d(vv + half * 8192, &tm_v, half * 64, h, z, bar);
@@ -296,7 +310,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int i = r0 + 16 * m;
-                const bool valid = i < Cc;
+                const bool valid = i < Cc && cd_in;
                 const long long tok = valid ? tokA + tstep * (c * C + i) : t0;
                 const uint32_t off = sw128(i, cd & 7);
                 cp_async16(kq + off, kbase + tok * kq_tok, valid);
@@ -310,6 +324,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
         }
         if (!p.use_tma || pt == 128) load_chunk(0);
+        // the chunk whose tensor loads this thread issued and nobody has waited for yet (-1:
+        // none); on an early exit it waits for them, so no copy lands in released memory
+        int ld_pending = p.use_tma && pt == 128 ? 0 : -1;
         if (!p.use_tma) cp_async_commit();
         // in-chunk cumulative log decay (log2 units) of one chunk from its gates, two per lane
         // (positions 2 lane, 2 lane + 1; 0 past the chunk), into G[par], and whether every
@@ -395,6 +412,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             else
                 cp_async_wait<1>();
             if (!p.use_tma) fence_proxy_async_smem();  // row copies land through the generic proxy
+            if (landed && ld_pending == c) ld_pending = -1;
             if (!group_agree(landed, kBarPrep)) {
                 fail = true;
                 break;
@@ -467,7 +485,10 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             //     (read by the product) while the accumulator load is in flight
             {
                 // warp 8 has no store here: it issues the next chunk's tensor loads
-                if (p.use_tma && has_next && pt == 128) load_chunk(c + 1);
+                if (p.use_tma && has_next && pt == 128) {
+                    load_chunk(c + 1);
+                    ld_pending = c + 1;
+                }
                 const int i = r & 63;
                 const bool live = i < Cc;
                 const bool split = SS.split_ok[pb];
@@ -770,6 +791,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             mbar_arrive(&SS.mbar[MB_PREP + pb]);
         }
         cp_async_wait<0>();
+        if (ld_pending >= 0)
+            mbar_wait_bounded(&SS.mbar[MB_LD + ld_pending % 3], (uint32_t)((ld_pending / 3) & 1),
+                              kWaitLimitNs);
     } else {
         // =============================== chain warpgroup ===============================
         const int j = lt;  // dv column = TMEM lane
@@ -785,8 +809,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 uint32_t r[32], hb[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const float x0 = p.S0 ? p.S0[sb + (size_t)(d0 + e) * D + j] : 0.f;
-                    const float x1 = p.S0 ? p.S0[sb + (size_t)(d0 + e + 1) * D + j] : 0.f;
+                    const bool in = p.S0 && d0 + e < kDh && j < kDh;
+                    const float x0 = in ? p.S0[sb + (size_t)(d0 + e) * kDh + j] : 0.f;
+                    const float x1 = in ? p.S0[sb + (size_t)(d0 + e + 1) * kDh + j] : 0.f;
                     r[e] = __float_as_uint(x0 * gam);
                     r[e + 1] = __float_as_uint(x1 * gam);
                     hb[e >> 1] = h2(x0, x1, rflags);
@@ -909,7 +934,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         const int z = (int)(t0 + (long long)c * C);
                         const uint32_t src = sbase + OFF_WN + pb * 16384;
                         tma_store_3d(&tm_o, src, 0, h, z);
-                        tma_store_3d(&tm_o, src + 8192, 64, h, z);
+                        if (kDh > 64) tma_store_3d(&tm_o, src + 8192, 64, h, z);
                         bulk_commit();
                     }
                 } else {
@@ -917,9 +942,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {
                     const int idx = m * 128 + lt, row = idx >> 4, c16 = idx & 15;
-                    if (row < Cc) {
+                    if (row < Cc && c16 < kDh / 8) {
                         const long long tok = tokA + tstep * (long long)(c * C + row);
-                        uint4* dp = reinterpret_cast<uint4*>(p.o + ((size_t)tok * p.Hv + h) * D + c16 * 8);
+                        uint4* dp = reinterpret_cast<uint4*>(p.o + ((size_t)tok * p.Hv + h) * kDh + c16 * 8);
                         uint4 a = *reinterpret_cast<const uint4*>(stage + (c16 >> 3) * 8192 +
                                                                   sw128(row, c16 & 7));
                         if (p.o_acc) {
@@ -959,7 +984,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         } else if (p.S_final) {
 #pragma unroll
                             for (int e = 0; e < 32; ++e)
-                                p.S_final[sb + (size_t)(dd + e) * D + j] = u2f(r[e]);
+                                if (dd + e < kDh && j < kDh)
+                                    p.S_final[sb + (size_t)(dd + e) * kDh + j] = u2f(r[e]);
                         }
                     }
                 }
@@ -1003,13 +1029,13 @@ EncodeTiledFn encode_tiled() {
     return fn;
 }
 
-// [tokens][heads][128] bf16 viewed as a 3-D tensor (128, heads, tokens); box 64 x 1 x 64
+// [tokens][heads][dim] bf16 viewed as a 3-D tensor (dim, heads, tokens); box 64 x 1 x 64
 // with the 128-byte swizzle, i.e. one 8 KB K-major atom stack of the kernel's layout.
-bool make_tile_map(CUtensorMap* m, const void* base, int heads, long long tokens) {
+bool make_tile_map(CUtensorMap* m, const void* base, int heads, long long tokens, int dim) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)tokens};
-    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+    const cuuint64_t dims[3] = {(cuuint64_t)dim, (cuuint64_t)heads, (cuuint64_t)tokens};
+    const cuuint64_t strides[2] = {(cuuint64_t)dim * 2, (cuuint64_t)heads * dim * 2};
     const cuuint32_t box[3] = {64, 1, 64};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
@@ -1020,7 +1046,7 @@ bool make_tile_map(CUtensorMap* m, const void* base, int heads, long long tokens
 }  // namespace
 
 bool tc_supported(const gdr_chunk_args& a) {
-    return a.io_dtype == GDR_BF16 && a.dk == D && a.dv == D && a.chunk == C;
+    return a.io_dtype == GDR_BF16 && a.dk == a.dv && (a.dk == D || a.dk == 64) && a.chunk == C;
 }
 
 gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k, const void* v,
@@ -1048,14 +1074,15 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
     p.use_tma = 0;
     p.tma_store = 0;
     if (!a.reverse && T_tot > 0) {  // reversed scans gather rows with cp.async instead
-        if (!make_tile_map(&tq, q, a.Hk, T_tot) || !make_tile_map(&tk, k, a.Hk, T_tot) ||
-            !make_tile_map(&tv, v, a.Hv, T_tot))
+        if (!make_tile_map(&tq, q, a.Hk, T_tot, a.dk) || !make_tile_map(&tk, k, a.Hk, T_tot, a.dk) ||
+            !make_tile_map(&tv, v, a.Hv, T_tot, a.dv))
             return GDR_ERR_CUDA;
         p.use_tma = 1;
         // accumulating outputs are read back, so they keep the plain stores
-        p.tma_store = !a.o_accumulate && make_tile_map(&to, o, a.Hv, T_tot);
+        p.tma_store = !a.o_accumulate && make_tile_map(&to, o, a.Hv, T_tot, a.dv);
     }
-    auto kernel = a.gate_raw ? chunk_fused_tc<true> : chunk_fused_tc<false>;
+    auto kernel = a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D> : chunk_fused_tc<false, D>)
+                            : (a.gate_raw ? chunk_fused_tc<true, 64> : chunk_fused_tc<false, 64>);
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;

@@ -1,4 +1,4 @@
-"""Parity of the tcgen05 tensor-core path (bf16, dk = dv = 128, chunk 64) against the
+"""Parity of the tcgen05 tensor-core path (bf16, dk = dv = 128 or 64, chunk 64) against the
 oracle, on shapes that exercise every branch of the fused kernel."""
 import math
 
@@ -21,17 +21,19 @@ def run(x, **kw):
     return o, S
 
 
-def test_path_is_tensor_core():
-    x = workloads.chunk_inputs(1, 64, 1, 1, 128, 128, "bf16")
+@pytest.mark.parametrize("d", [128, 64])
+def test_path_is_tensor_core(d):
+    x = workloads.chunk_inputs(1, 64, 1, 1, d, d, "bf16")
     a = gdr.make_chunk_args(to_dev(x["q"]), to_dev(x["v"]), to_dev(x["g"]))
     assert gdr.chunk_fwd_path(a) == "tc"
 
 
 @pytest.mark.parametrize("read_mode", ["post", "pre"])
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 1000])
-def test_lengths(read_mode, T):
-    x = workloads.chunk_inputs(2, T, 2, 4, 128, 128, "bf16", s0_std=0.02, seed=T)
-    scale = 1 / math.sqrt(128)
+@pytest.mark.parametrize("d", [128, 64])
+def test_lengths(read_mode, T, d):
+    x = workloads.chunk_inputs(2, T, 2, 4, d, d, "bf16", s0_std=0.02, seed=T + d)
+    scale = 1 / math.sqrt(d)
     o, S = run(x, read_mode=read_mode, scale=scale)
     o_r, S_r = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"],
                               read_mode=read_mode, scale=scale)
@@ -40,10 +42,11 @@ def test_lengths(read_mode, T):
 
 
 @pytest.mark.parametrize("reverse", [False, True])
-def test_varlen_reverse(reverse):
+@pytest.mark.parametrize("d", [128, 64])
+def test_varlen_reverse(reverse, d):
     lengths = [1, 0, 64, 65, 130, 0, 7, 300, 129]
-    x = workloads.chunk_inputs(1, 0, 2, 2, 128, 128, "bf16", lengths=lengths, s0_std=0.05,
-                               seed=11)
+    x = workloads.chunk_inputs(1, 0, 2, 2, d, d, "bf16", lengths=lengths, s0_std=0.05,
+                               seed=11 + d)
     o, S = run(x, read_mode="pre", scale=0.3, reverse=reverse)
     o_r, S_r = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"],
                               x["cu_seqlens"], read_mode="pre", scale=0.3, reverse=reverse)
@@ -113,3 +116,18 @@ def test_fp16_range_is_reported():
     x["v"] = (x["v"].float() * 1e-6).to(torch.bfloat16)
     gdr.chunk_fwd(d["q"], d["k"], to_dev(x["v"]), d["g"], d["beta"], workspace=ws)
     assert gdr.read_device_error(args, ws) == gdr._abi.GDR_OK
+
+
+def test_head_size_64_accumulate_and_aliasing():
+    """64-wide heads: accumulation into o (plain stores) and S_final aliasing S0."""
+    x = workloads.chunk_inputs(2, 150, 1, 3, 64, 64, "bf16", s0_std=0.1, seed=18)
+    d = {n: to_dev(x[n]) if x.get(n) is not None else None for n in x}
+    base = (0.01 * torch.randn(d["v"].shape, device="cuda")).to(torch.bfloat16)
+    o = base.clone()
+    S = d["S0"].clone()
+    gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S, o=o, o_accumulate=True,
+                  S_final=S, scale=0.125)
+    torch.cuda.synchronize()
+    o_r, S_r = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], scale=0.125)
+    assert_close("o", o, o_r + base.double().cpu().numpy(), torch.bfloat16)
+    assert_close("S", S, S_r, torch.bfloat16)
