@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 METRIC = "gated-delta chunk-fwd tokens/s + %bf16 TC peak; decode state GB/s vs HBM peak"
 CHUNK_WORKLOAD = "bf16_b8_h16_t4096_d128"
 DECODE_WORKLOAD = "bf16_decode_n256_hk16_hv32_d128"
+BIDIR_WORKLOAD = "bf16_bidir_16x2048_h12_d64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -251,6 +252,50 @@ def bench_ours(args, rank, world, local_rank):
                   "inputs": "raw a ~ N(-2,1), b ~ N(0,1) with A = -1, dt_bias = 0 "
                             "(same gate distributions as the workload)"}
 
+    # ---------------- bidirectional workload: both directions summed, two calls (reverse scan
+    # with accumulation for the second), same parity-tested configuration
+    bidir = None
+    if not args.no_bidir and args.only != "decode" and not args.rows:
+        bw = workloads.WORKLOADS[BIDIR_WORKLOAD]
+        bx = workloads.workload_inputs(bw, seed=rank)
+        bd = {n: (t.to(dev) if t is not None else None) for n, t in bx.items()}
+        bo = torch.empty_like(bd["v"])
+        bargs = gdr.make_chunk_args(bd["q"], bd["v"], bd["g"], bd["cu_seqlens"], bw.chunk,
+                                    bw.read_mode, bw.scale)
+        bws = torch.empty(gdr.chunk_fwd_workspace_size(bargs), dtype=torch.uint8, device=dev)
+
+        def bstep():
+            gdr.chunk_fwd(bd["q"], bd["k"], bd["v"], bd["g"], bd["beta"], None, bd["cu_seqlens"],
+                          chunk=bw.chunk, read_mode=bw.read_mode, scale=bw.scale, o=bo,
+                          output_final_state=False, workspace=bws)
+            gdr.chunk_fwd(bd["q"], bd["k"], bd["v"], bd["g_bwd"], bd["beta_bwd"], None,
+                          bd["cu_seqlens"], chunk=bw.chunk, read_mode=bw.read_mode,
+                          scale=bw.scale, reverse=True, o=bo, o_accumulate=True,
+                          output_final_state=False, workspace=bws)
+
+        for _ in range(args.warmup):
+            bstep()
+        torch.cuda.synchronize()
+        barrier()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(args.steps):
+            bstep()
+        b1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        bms = max_over_ranks(b0.elapsed_time(b1) / args.steps, world)
+        btok = int(bd["q"].shape[1])
+        # per direction: q, k, v and both gates read, o written (the accumulating pass also
+        # reads it back)
+        bbytes = 2 * sum(bd[n].numel() * bd[n].element_size() for n in ("q", "k", "v")) + sum(
+            bd[n].numel() * bd[n].element_size() for n in ("g", "beta", "g_bwd", "beta_bwd")) + (
+            3 * bo.numel() * bo.element_size())
+        bidir = {"workload": bw.name, "ms_per_step": bms, "value": whole_job_rate(btok, world, bms),
+                 "unit": "tokens/s", "path": gdr.chunk_fwd_path(bargs),
+                 "algorithmic_bytes": bbytes,
+                 "hbm_frac": bbytes / (bms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+
     # ---------------- decode step
     dec = None
     if not args.no_decode and args.only != "chunk":
@@ -344,7 +389,8 @@ def bench_ours(args, rank, world, local_rank):
                      "tensor_frac": tflops / peaks["bf16_tflops"],
                      "timed": "whole gdr_chunk_fwd call (plan + chunk kernels), CUDA events",
                      "peak_source": f"{peak_src} (hbm_gbs copy; bf16_tflops burst)"},
-        "decode": dec, "gating_prologue": gating, "e2e": e2e, "clocks": clocks,
+        "decode": dec, "gating_prologue": gating, "bidirectional": bidir, "e2e": e2e,
+        "clocks": clocks,
         "gpu_launches": launches_per_call * args.steps,
     }
     return line, x, w
@@ -407,6 +453,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=CHUNK_WORKLOAD)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-bidir", action="store_true",
+                    help="skip the bidirectional workload (both directions summed)")
     ap.add_argument("--no-gating", action="store_true",
                     help="skip the forward through the fused gating prologue")
     ap.add_argument("--no-e2e", action="store_true")
