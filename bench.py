@@ -334,6 +334,31 @@ def bench_ours(args, rank, world, local_rank):
                             "unit": "GB/s", "frac": dgbs / peaks["hbm_gbs"],
                             "traffic": measured_traffic("decode_kernel", DECODE_SOURCES, dw.N),
                             "peak_source": f"{peak_src} (hbm_gbs, copy)"}}
+        # the same steps with the decode chain's output epilogue fused (gated RMSNorm of o)
+        zn = torch.randn((dw.N, dw.Hv, dw.dv), device=dev).to(torch.bfloat16)
+        wn = torch.ones(dw.dv, device=dev)
+
+        def nstep(t):
+            gdr.decode_step(dd["q"][t], dd["k"][t], dd["v"][t], dd["g"][t], dd["beta"][t],
+                            dd["S"], read_mode=dw.read_mode, scale=dw.scale, o=od, norm_z=zn,
+                            norm_weight=wn, norm_eps=1e-6)
+
+        for t in range(min(args.warmup, dw.steps)):
+            nstep(t)
+        torch.cuda.synchronize()
+        barrier()
+        n0, n1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n0.record(stream)
+        for t in range(dw.steps):
+            nstep(t)
+        n1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        nms = max_over_ranks(n0.elapsed_time(n1) / dw.steps, world)
+        nbytes = dbytes + zn.numel() * zn.element_size()
+        ngbs = nbytes / (nms / 1e3) / 1e9
+        dec["fused_output_norm"] = {"ms_per_step": nms, "value": world * ngbs, "unit": "GB/s",
+                                    "frac": ngbs / peaks["hbm_gbs"]}
     clocks = sampler.stop()
 
     # ---------------- end to end through the public API with host buffers

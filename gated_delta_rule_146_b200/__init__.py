@@ -141,29 +141,47 @@ def read_device_error(args: ChunkArgs, workspace, stream=None) -> int:
                                                 _stream(stream)))
 
 
+def _norm_fields(q, norm_z, norm_weight, norm_eps):
+    """(out_norm, z pointer, weight pointer, eps) of the fused gated RMSNorm epilogue."""
+    if (norm_z is None) != (norm_weight is None):
+        raise ValueError("norm_z and norm_weight come together")
+    if norm_z is None:
+        return 0, None, None, float(norm_eps)
+    import torch
+    if norm_z.dtype != q.dtype:
+        raise TypeError("norm_z has the dtype of q, k, v and o")
+    if norm_weight.dtype != torch.float32 or norm_weight.dim() != 1:
+        raise TypeError("norm_weight is a float32 [dv] tensor")
+    return 1, norm_z.data_ptr(), norm_weight.data_ptr(), float(norm_eps)
+
+
 def make_decode_args(q, v, g, read_mode="post", scale=None, qk_l2norm=True, gate_A=None,
-                     gate_dt_bias=None, beta_scale=1.0):
+                     gate_dt_bias=None, beta_scale=1.0, norm_z=None, norm_weight=None,
+                     norm_eps=1e-6):
     N, Hk, dk = q.shape
     Hv, dv = v.shape[1], v.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(dk)
     return DecodeArgs(N, Hk, Hv, dk, dv, _dtype_code(q), _dtype_code(g),
                       READ_PRE if read_mode == "pre" else READ_POST, float(scale),
-                      int(bool(qk_l2norm)), *_gating_fields(gate_A, gate_dt_bias, beta_scale))
+                      int(bool(qk_l2norm)), *_gating_fields(gate_A, gate_dt_bias, beta_scale),
+                      *_norm_fields(q, norm_z, norm_weight, norm_eps))
 
 
 def decode_step(q, k, v, g, beta, S, *, read_mode="post", scale=None, qk_l2norm=True, o=None,
-                stream=None, gate_A=None, gate_dt_bias=None, beta_scale=1.0):
+                stream=None, gate_A=None, gate_dt_bias=None, beta_scale=1.0, norm_z=None,
+                norm_weight=None, norm_eps=1e-6):
     """One recurrent token per sequence (gdr_decode_step): q, k [N,Hk,dk]; v [N,Hv,dv];
     g, beta [N,Hv]; S [N,Hv,dk,dv] fp32, updated in place.  With gate_A and gate_dt_bias
-    ([Hv] fp32) given, g and beta are the raw projections of the fused gating prologue.
-    Returns o [N,Hv,dv]."""
+    ([Hv] fp32) given, g and beta are the raw projections of the fused gating prologue;
+    with norm_z ([N,Hv,dv]) and norm_weight ([dv] fp32) given, o is the gated RMSNorm of
+    the recurrent output.  Returns o [N,Hv,dv]."""
     import torch
-    _check_cuda(q, k, v, g, beta, S, o, gate_A, gate_dt_bias)
+    _check_cuda(q, k, v, g, beta, S, o, gate_A, gate_dt_bias, norm_z, norm_weight)
     if S.dtype != torch.float32:
         raise TypeError("the state must be float32")
     args = make_decode_args(q, v, g, read_mode, scale, qk_l2norm, gate_A, gate_dt_bias,
-                            beta_scale)
+                            beta_scale, norm_z, norm_weight, norm_eps)
     if o is None:
         o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     st = _abi.lib().gdr_decode_step(ctypes.byref(args), _ptr(q), _ptr(k), _ptr(v), _ptr(g),

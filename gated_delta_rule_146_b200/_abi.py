@@ -37,7 +37,9 @@ class DecodeArgs(ctypes.Structure):
                 ("gate_dtype", ctypes.c_int), ("read_mode", ctypes.c_int),
                 ("scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int),
                 ("gate_raw", ctypes.c_int), ("gate_A", ctypes.c_void_p),
-                ("gate_dt_bias", ctypes.c_void_p), ("beta_scale", ctypes.c_float)]
+                ("gate_dt_bias", ctypes.c_void_p), ("beta_scale", ctypes.c_float),
+                ("out_norm", ctypes.c_int), ("norm_z", ctypes.c_void_p),
+                ("norm_weight", ctypes.c_void_p), ("norm_eps", ctypes.c_float)]
 
 
 class GdrError(RuntimeError):

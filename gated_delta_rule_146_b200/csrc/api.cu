@@ -126,11 +126,18 @@ gdr_status gdr_decode_step(const gdr_decode_args* a, const void* q, const void* 
     if (a->read_mode != GDR_READ_POST && a->read_mode != GDR_READ_PRE) return GDR_ERR_INVALID_ARG;
     if (a->qk_l2norm & ~1) return GDR_ERR_INVALID_ARG;
     if (check_gating(a, false) != GDR_OK) return GDR_ERR_INVALID_ARG;
+    if (a->out_norm & ~1) return GDR_ERR_INVALID_ARG;
+    if (a->out_norm && !(std::isfinite(a->norm_eps) && a->norm_eps >= 0.f)) return GDR_ERR_INVALID_ARG;
     if ((long long)a->N * a->Hv > 0x7fffffffLL) return GDR_ERR_INVALID_ARG;
     if (!decode_supported(*a)) return GDR_ERR_UNSUPPORTED;
     if (a->N == 0) return GDR_OK;
     if (!q || !k || !v || !g || !beta || !S_inout || !o) return GDR_ERR_INVALID_ARG;
     if (const gdr_status gs = check_gating(a, true); gs != GDR_OK) return gs;
+    if (a->out_norm) {
+        if (!a->norm_z || !a->norm_weight) return GDR_ERR_INVALID_ARG;
+        if (!aligned16(a->norm_z) || (reinterpret_cast<uintptr_t>(a->norm_weight) & 3u))
+            return GDR_ERR_ALIGNMENT;
+    }
     const void* ptrs[] = {q, k, v, g, beta, S_inout, o};
     for (const void* p : ptrs)
         if (!aligned16(p)) return GDR_ERR_ALIGNMENT;

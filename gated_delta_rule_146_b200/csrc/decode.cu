@@ -8,6 +8,9 @@
 //     H  <- alpha H + k u^T                         (in place)
 //     post: o = scale (alpha s_q + (k.q) u)   [= scale H_new^T q]
 //     pre:  o = scale s_q
+// and, when the output epilogue is fused (the decode chain's gated RMSNorm, flashrt
+// fused_layer.py `_decode_one`), o <- o / sqrt(mean(o^2) + eps) * weight * silu(z) over
+// the head's dv values; that variant gives each block a whole head (DVS = DV).
 // The columns of H (dv) are independent, so a block owns a slice of DVS columns
 // and every row of it: it loads the whole slice into registers with 16-byte
 // streaming loads, reduces s_k and s_q over the dk rows (warp shuffles, then
@@ -32,11 +35,14 @@ struct DecodeParams {
     int gate_raw;                 // fused gating prologue (see gate_xform)
     const float* gate_A; const float* gate_dt_bias;
     float beta_scale;
+    const void* norm_z; const float* norm_weight;  // fused gated RMSNorm epilogue
+    float norm_eps;
 };
 
-template <int DK, int DV, int DVS>
+template <int DK, int DV, int DVS, bool kNorm>
 __global__ void __launch_bounds__(kThreads)
 decode_kernel(DecodeParams p) {
+    static_assert(!kNorm || DVS == DV, "the normed epilogue needs the whole head in a block");
     constexpr int CPR = DVS / 4;           // float4 column groups per row slice
     constexpr int RPW = 32 / CPR;          // rows a warp covers per pass
     constexpr int RPP = RPW * kWarps;      // rows per pass over the block
@@ -47,6 +53,8 @@ decode_kernel(DecodeParams p) {
     __shared__ float s_red[2][kWarps][DVS];
     __shared__ float s_u[DVS];
     __shared__ float s_alpha, s_beta;
+    __shared__ float s_o[kNorm ? DVS : 1];        // recurrent output of the head (epilogue)
+    __shared__ float s_ss[kWarps];
 
     const int nh = blockIdx.x;                   // n * Hv + h
     const int J = blockIdx.y;                    // column slice
@@ -129,9 +137,28 @@ decode_kernel(DecodeParams p) {
         const float u = beta * (vj - alpha * tk);
         s_u[tid] = u;
         const float oj = p.read_pre ? p.scale * tq : p.scale * fmaf(alpha, tq, kq * u);
-        store_elem(p.o, (size_t)nh * DV + col, oj, p.io);
+        if constexpr (kNorm) s_o[tid] = oj;
+        else store_elem(p.o, (size_t)nh * DV + col, oj, p.io);
     }
     __syncthreads();
+    if constexpr (kNorm) {
+        // gated RMSNorm over the head: o_j / sqrt(mean(o^2) + eps) * weight_j * silu(z_j)
+        if (wid * 32 < DV) {
+            const float x = tid < DV ? s_o[tid] : 0.f;
+            const float ss = warp_sum(x * x);
+            if (lane == 0) s_ss[wid] = ss;
+        }
+        __syncthreads();
+        if (tid < DV) {
+            float ss = 0.f;
+#pragma unroll
+            for (int w = 0; w < (DV + 31) / 32; ++w) ss += s_ss[w];
+            const float r = rsqrtf(ss / DV + p.norm_eps);
+            const float z = load_elem(p.norm_z, (size_t)nh * DV + tid, p.io);
+            const float silu = z / (1.f + expf(-z));
+            store_elem(p.o, (size_t)nh * DV + tid, s_o[tid] * r * p.norm_weight[tid] * silu, p.io);
+        }
+    }
     const float4 u4 = *reinterpret_cast<const float4*>(&s_u[cg * 4]);
 #pragma unroll
     for (int m = 0; m < NP; ++m) {
@@ -145,9 +172,13 @@ decode_kernel(DecodeParams p) {
 
 template <int DK, int DV>
 gdr_status launch_dv(const gdr_decode_args& a, const DecodeParams& p, cudaStream_t st) {
-    constexpr int DVS = DV >= 64 ? 64 : 32;
-    dim3 grid((unsigned)(a.N * a.Hv), DV / DVS);
-    decode_kernel<DK, DV, DVS><<<grid, kThreads, 0, st>>>(p);
+    if (a.out_norm) {  // one block per (sequence, head): the epilogue reduces over dv
+        decode_kernel<DK, DV, DV, true><<<dim3((unsigned)(a.N * a.Hv), 1), kThreads, 0, st>>>(p);
+    } else {
+        constexpr int DVS = DV >= 64 ? 64 : 32;
+        dim3 grid((unsigned)(a.N * a.Hv), DV / DVS);
+        decode_kernel<DK, DV, DVS, false><<<grid, kThreads, 0, st>>>(p);
+    }
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 
@@ -175,6 +206,7 @@ gdr_status launch_decode(const gdr_decode_args& a, const void* q, const void* k,
     p.qk_l2norm = a.qk_l2norm; p.io = a.io_dtype; p.gt = a.gate_dtype; p.scale = a.scale;
     p.gate_raw = a.gate_raw; p.gate_A = a.gate_A; p.gate_dt_bias = a.gate_dt_bias;
     p.beta_scale = a.beta_scale;
+    p.norm_z = a.norm_z; p.norm_weight = a.norm_weight; p.norm_eps = a.norm_eps;
     switch (a.dk) {
         case 32: return launch_dk<32>(a, p, st);
         case 64: return launch_dk<64>(a, p, st);

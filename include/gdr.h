@@ -189,6 +189,19 @@ typedef struct {
     const float* gate_A;
     const float* gate_dt_bias;
     float beta_scale;
+    /* Fused output epilogue of the decode chain (flashrt fused_layer.py `_decode_one`:
+     * rms_norm_gated_silu(core_out, z, norm.weight, eps) applied per head to the
+     * recurrent core's output).
+     *   out_norm = 0: o is the recurrent output itself; the three fields below are unused.
+     *   out_norm = 1: o_j = c_j / sqrt(mean_j(c_j^2) + norm_eps) * norm_weight[j] * silu(z_j)
+     *                 per (sequence, head), c the recurrent output in fp32, the mean over the
+     *                 dv values of the head, silu(x) = x / (1 + e^-x). */
+    int out_norm;
+    const void* norm_z;         /* [N, Hv, dv] io_dtype; 16-byte aligned; required when
+                                   out_norm */
+    const float* norm_weight;   /* [dv] fp32, shared by the heads; 4-byte aligned; required
+                                   when out_norm */
+    float norm_eps;             /* >= 0, finite */
 } gdr_decode_args;
 
 /*

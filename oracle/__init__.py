@@ -19,6 +19,7 @@ Three independent implementations live here:
 
 ``gating`` forms the gates from raw projections (the fused gating prologue)
 in fp64; the recurrence oracles take its output like any other gates.
+``gated_rmsnorm`` is the decode chain's output epilogue in fp64.
 
 Every input arrives already rounded to the dtype the GPU sees (bf16 / fp32);
 it is widened exactly to fp64 here.
@@ -165,3 +166,16 @@ def gating(a, b, A, dt_bias, beta_scale: float = 1.0):
     g = A * softplus
     beta = beta_scale * np.exp(-np.logaddexp(0.0, -b))  # 1 / (1 + e^-b)
     return g, beta
+
+
+def gated_rmsnorm(o, z, weight, eps: float):
+    """Output epilogue of the decode chain, fp64: per head (last axis, dv values)
+    ``o / sqrt(mean(o^2) + eps) * weight * silu(z)``, ``silu(x) = x sigmoid(x)``
+    (flashrt-structures 0.2.0 ``impls/gated_delta_core/fused_layer.py``, ``_decode_one``:
+    ``rms_norm_gated_silu(core_out, z, norm.weight, eps)``; the normalisation is read as
+    coming before the gate and the weight as one [dv] vector shared by the heads).
+    ``o``, ``z`` are ``[..., dv]``; returns fp64 of that shape."""
+    o, z, weight = _f64(o), _f64(z), _f64(weight)
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps)
+    silu = z * np.exp(-np.logaddexp(0.0, -z))
+    return o / rms * weight * silu

@@ -145,3 +145,17 @@ def test_struct_layout_matches_header(tmp_path):
         want.append(ctypes.sizeof(py))
         want.extend(getattr(py, n).offset for n, _ in py._fields_)
     assert got == want
+
+
+def test_decode_norm_host_validation(lib):
+    """The fused output epilogue's flag, eps and arrays are checked on the host."""
+    base = dict(N=4, Hk=2, Hv=4, dk=128, dv=128, io_dtype=_abi.BF16, gate_dtype=_abi.BF16,
+                read_mode=_abi.READ_POST, scale=0.1, qk_l2norm=1)
+    vp = ctypes.c_void_p
+    f = lambda **kw: lib.gdr_decode_step(ctypes.byref(_abi.DecodeArgs(**{**base, **kw})),
+                                         *[vp(FAKE)] * 7, None)
+    assert f(out_norm=2) == _abi.GDR_ERR_INVALID_ARG
+    assert f(out_norm=1, norm_z=FAKE, norm_weight=FAKE, norm_eps=-1.0) == _abi.GDR_ERR_INVALID_ARG
+    assert f(out_norm=1, norm_weight=FAKE, norm_eps=1e-6) == _abi.GDR_ERR_INVALID_ARG
+    assert f(out_norm=1, norm_z=FAKE + 8, norm_weight=FAKE, norm_eps=1e-6) == _abi.GDR_ERR_ALIGNMENT
+    assert f(out_norm=1, norm_z=FAKE, norm_weight=FAKE + 2, norm_eps=1e-6) == _abi.GDR_ERR_ALIGNMENT

@@ -67,3 +67,26 @@ def test_decode_workload_sampled():
         torch.cuda.synchronize()
         assert_close(f"o step {t}", o[seqs], o_ref, torch.bfloat16)
     assert_close("S final", S[seqs], S_ref, torch.bfloat16)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 32)])
+def test_decode_fused_gated_rmsnorm(dtype, dk, dv):
+    """o = gated RMSNorm of the recurrent output (the decode chain's epilogue), the state
+    updated exactly as without it."""
+    x = workloads.decode_inputs(5, 2, 4, dk, dv, steps=3, dtype=dtype, s_std=0.1, seed=50 + dv)
+    S = x["S"].clone().cuda()
+    S_ref = x["S"].double().numpy()
+    gen = torch.Generator("cpu").manual_seed(dk + dv)
+    w = 1.0 + 0.2 * torch.randn(dv, generator=gen)
+    scale = 1 / math.sqrt(dk)
+    for t in range(3):
+        z = torch.randn((5, 4, dv), generator=gen).to(workloads.DTYPES[dtype])
+        o = gdr.decode_step(*(to_dev(x[n][t]) for n in ("q", "k", "v", "g", "beta")), S,
+                            scale=scale, norm_z=to_dev(z), norm_weight=to_dev(w), norm_eps=1e-6)
+        o_core, S_ref = oracle.decode_step(*(x[n][t] for n in ("q", "k", "v", "g", "beta")),
+                                           S_ref, scale=scale)
+        ref = oracle.gated_rmsnorm(o_core, z, w, 1e-6)
+        torch.cuda.synchronize()
+        assert_close(f"o step {t}", o, ref, workloads.DTYPES[dtype])
+    assert_close("S", S, S_ref, torch.float32 if dtype == "f32" else torch.bfloat16)
