@@ -179,3 +179,55 @@ def gated_rmsnorm(o, z, weight, eps: float):
     rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps)
     silu = z * np.exp(-np.logaddexp(0.0, -z))
     return o / rms * weight * silu
+
+
+def _l2n(x):
+    n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+    return x / np.maximum(n, 1e-6)
+
+
+def gdn2_forward(q, k, v, g, b, w, S0=None, cu_seqlens=None, read_mode: str = "post",
+                 scale: float = 1.0, qk_l2norm: bool = True, reverse: bool = False):
+    """GDN-2 recurrence with decoupled gates, per-token loop in fp64 (Rondo-Exp
+    ``tiny_gdn/fugue.py``, ``BidirectionalGatedDeltaNet2`` docstring:
+    ``S_t = (I - k_t (b_t * k_t)^T) Diag(exp g_t) S_{t-1} + k_t (w_t * v_t)^T`` with S of
+    shape [dk, dv], the forward read ``q_t^T S_t``).
+
+    q, k [B, T, Hk, dk]; v [B, T, Hv, dv]; g, b [B, T, Hv, dk] (per key channel: log decay
+    and erase gate); w [B, T, Hv, dv] (per value channel write gate); S0 [n_seqs, Hv, dk,
+    dv] or None.  Same conventions as ``forward`` (H = S^T layout, GQA by repeating key
+    heads, varlen, the read modes, reversal within each sequence).  With g = log(alpha),
+    b = w = beta on every channel this is the scalar gated delta rule.
+    Returns (o [B, T, Hv, dv], S_final [n_seqs, Hv, dk, dv]) in fp64.
+    """
+    q, k, v, g, b, w = (_f64(x) for x in (q, k, v, g, b, w))
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    group = Hv // Hk
+    if cu_seqlens is None:
+        segs = [(n, 0, T) for n in range(B)]
+    else:
+        cu = np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+                        dtype=np.int64)
+        segs = [(0, int(cu[s]), int(cu[s + 1])) for s in range(len(cu) - 1)]
+    o = np.zeros((B, T, Hv, dv))
+    S_out = np.zeros((len(segs), Hv, dk, dv))
+    S0 = _f64(S0)
+    for si, (row, t0, t1) in enumerate(segs):
+        H = np.zeros((Hv, dk, dv)) if S0 is None else S0[si].copy()
+        order = range(t1 - 1, t0 - 1, -1) if reverse else range(t0, t1)
+        for t in order:
+            qt = np.repeat(q[row, t], group, axis=0)          # [Hv, dk]
+            kt = np.repeat(k[row, t], group, axis=0)
+            if qk_l2norm:
+                qt, kt = _l2n(qt), _l2n(kt)
+            if read_mode == "pre":
+                o[row, t] = scale * np.einsum("hd,hde->he", qt, H)
+            D = np.exp(g[row, t])                             # [Hv, dk]
+            DH = D[:, :, None] * H
+            u = w[row, t] * v[row, t] - np.einsum("hd,hde->he", b[row, t] * kt, DH)
+            H = DH + kt[:, :, None] * u[:, None, :]
+            if read_mode == "post":
+                o[row, t] = scale * np.einsum("hd,hde->he", qt, H)
+        S_out[si] = H
+    return o, S_out
