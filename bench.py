@@ -359,6 +359,68 @@ def bench_ours(args, rank, world, local_rank):
         ngbs = nbytes / (nms / 1e3) / 1e9
         dec["fused_output_norm"] = {"ms_per_step": nms, "value": world * ngbs, "unit": "GB/s",
                                     "frac": ngbs / peaks["hbm_gbs"]}
+    # ---------------- GDN-2 (decoupled per-channel gates): the chunk workload on the CUDA-core
+    # path and the decode steps, same inputs with g, beta per key channel and a write gate
+    gdn2 = None
+    if args.gdn2 and not args.rows:
+        gdn2 = {}
+        if args.only != "decode":
+            gg, gb, gw = (t.to(dev) for t in workloads.gdn2_gate_inputs(
+                tuple(d["v"].shape[:3]), w.dk, w.dv, w.gate_dtype, seed=rank))
+            g2args = gdr.make_chunk_args(d["q"], d["v"], gg, d["cu_seqlens"], w.chunk,
+                                         w.read_mode, w.scale, gdn2_w=gw)
+            g2ws = torch.empty(gdr.chunk_fwd_workspace_size(g2args), dtype=torch.uint8,
+                               device=dev)
+
+            def g2step():
+                gdr.chunk_fwd(d["q"], d["k"], d["v"], gg, gb, d["S0"], d["cu_seqlens"],
+                              chunk=w.chunk, read_mode=w.read_mode, scale=w.scale, o=o,
+                              S_final=S_final, workspace=g2ws, gdn2_w=gw)
+
+            g2steps = min(args.steps, 3)
+            for _ in range(min(args.warmup, 3)):
+                g2step()
+            torch.cuda.synchronize()
+            barrier()
+            c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            c0.record(stream)
+            for _ in range(g2steps):
+                g2step()
+            c1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            cms = max_over_ranks(c0.elapsed_time(c1) / g2steps, world)
+            gdn2["chunk"] = {"workload": w.name, "ms_per_step": cms, "steps": g2steps,
+                             "value": whole_job_rate(tokens, world, cms), "unit": "tokens/s",
+                             "path": gdr.chunk_fwd_path(g2args)}
+            del g2ws
+        if dec is not None:
+            dg, db, dwg = (t.to(dev) for t in workloads.gdn2_gate_inputs(
+                (dw.steps, dw.N, dw.Hv), dw.dk, dw.dv, dw.gate_dtype, seed=rank))
+
+            def g2dstep(t):
+                gdr.decode_step(dd["q"][t], dd["k"][t], dd["v"][t], dg[t], db[t], dd["S"],
+                                read_mode=dw.read_mode, scale=dw.scale, o=od, gdn2_w=dwg[t])
+
+            for t in range(min(args.warmup, dw.steps)):
+                g2dstep(t)
+            torch.cuda.synchronize()
+            barrier()
+            e0.record(stream)
+            for t in range(dw.steps):
+                g2dstep(t)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            g2ms = max_over_ranks(e0.elapsed_time(e1) / dw.steps, world)
+            g2bytes = 2 * dd["S"].numel() * 4 + sum(
+                dd[n][0].numel() * dd[n].element_size() for n in ("q", "k", "v")) + sum(
+                t[0].numel() * t.element_size() for t in (dg, db, dwg)) + (
+                od.numel() * od.element_size())
+            g2gbs = g2bytes / (g2ms / 1e3) / 1e9
+            gdn2["decode"] = {"workload": dw.name, "ms_per_step": g2ms,
+                              "bytes_per_step": g2bytes, "value": world * g2gbs, "unit": "GB/s",
+                              "frac": g2gbs / peaks["hbm_gbs"]}
     clocks = sampler.stop()
 
     # ---------------- end to end through the public API with host buffers
@@ -414,7 +476,7 @@ def bench_ours(args, rank, world, local_rank):
                      "tensor_frac": tflops / peaks["bf16_tflops"],
                      "timed": "whole gdr_chunk_fwd call (plan + chunk kernels), CUDA events",
                      "peak_source": f"{peak_src} (hbm_gbs copy; bf16_tflops burst)"},
-        "decode": dec, "gating_prologue": gating, "bidirectional": bidir, "e2e": e2e,
+        "decode": dec, "gating_prologue": gating, "bidirectional": bidir, "gdn2": gdn2, "e2e": e2e,
         "clocks": clocks,
         "gpu_launches": launches_per_call * args.steps,
     }
@@ -478,6 +540,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=CHUNK_WORKLOAD)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-gdn2", dest="gdn2", action="store_false",
+                    help="skip the GDN-2 (decoupled gates) chunk and decode measurements")
     ap.add_argument("--no-bidir", action="store_true",
                     help="skip the bidirectional workload (both directions summed)")
     ap.add_argument("--no-gating", action="store_true",

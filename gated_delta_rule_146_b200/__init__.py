@@ -73,9 +73,21 @@ def _gating_fields(gate_A, gate_dt_bias, beta_scale):
     return 1, gate_A.data_ptr(), gate_dt_bias.data_ptr(), float(beta_scale)
 
 
+def _gdn2_fields(g, v, gdn2_w):
+    """(gdn2, write-gate pointer): with gdn2_w ([.., Hv, dv], gate dtype) given, g and beta
+    are the per-key-channel log decay and erase gate of GDN-2 ([.., Hv, dk])."""
+    if gdn2_w is None:
+        return 0, None
+    if gdn2_w.dtype != g.dtype or tuple(gdn2_w.shape) != tuple(v.shape):
+        raise TypeError("gdn2_w has the shape of v and the dtype of g")
+    if g.dim() != v.dim():
+        raise TypeError("with gdn2_w, g and beta carry a key-channel axis")
+    return 1, gdn2_w.data_ptr()
+
+
 def make_chunk_args(q, v, g, cu_seqlens=None, chunk=64, read_mode="post", scale=None,
                     qk_l2norm=True, reverse=False, o_accumulate=False, gate_A=None,
-                    gate_dt_bias=None, beta_scale=1.0):
+                    gate_dt_bias=None, beta_scale=1.0, gdn2_w=None):
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
@@ -84,7 +96,7 @@ def make_chunk_args(q, v, g, cu_seqlens=None, chunk=64, read_mode="post", scale=
     return ChunkArgs(B, T, Hk, Hv, dk, dv, n_seqs, chunk, _dtype_code(q), _dtype_code(g),
                      READ_PRE if read_mode == "pre" else READ_POST, float(scale),
                      int(bool(qk_l2norm)), int(bool(reverse)), int(bool(o_accumulate)),
-                     *_gating_fields(gate_A, gate_dt_bias, beta_scale))
+                     *_gating_fields(gate_A, gate_dt_bias, beta_scale), *_gdn2_fields(g, v, gdn2_w))
 
 
 def chunk_fwd_workspace_size(args: ChunkArgs) -> int:
@@ -99,16 +111,19 @@ def chunk_fwd_path(args: ChunkArgs):
 def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, *, chunk=64, read_mode="post",
               scale=None, qk_l2norm=True, reverse=False, o=None, o_accumulate=False,
               output_final_state=True, S_final=None, workspace=None, stream=None,
-              gate_A=None, gate_dt_bias=None, beta_scale=1.0):
+              gate_A=None, gate_dt_bias=None, beta_scale=1.0, gdn2_w=None):
     """Chunk-parallel forward (gdr_chunk_fwd).  Shapes: q, k [B,T,Hk,dk]; v [B,T,Hv,dv];
     g, beta [B,T,Hv]; S0 [n_seqs,Hv,dk,dv] fp32 or None; cu_seqlens int32 [n_seqs+1] or
     None.  With gate_A and gate_dt_bias ([Hv] fp32) given, g and beta are the raw
-    projections a and b of the fused gating prologue.  Returns (o [B,T,Hv,dv],
-    S_final [n_seqs,Hv,dk,dv] fp32 or None)."""
+    projections a and b of the fused gating prologue.  With gdn2_w ([B,T,Hv,dv]) given, the
+    gates are GDN-2's: g the per-key-channel log decay and beta the erase gate, both
+    [B,T,Hv,dk], gdn2_w the write gate.  Returns (o [B,T,Hv,dv], S_final [n_seqs,Hv,dk,dv]
+    fp32 or None)."""
     import torch
-    _check_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_final, workspace, gate_A, gate_dt_bias)
+    _check_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_final, workspace, gate_A, gate_dt_bias,
+                gdn2_w)
     args = make_chunk_args(q, v, g, cu_seqlens, chunk, read_mode, scale, qk_l2norm, reverse,
-                           o_accumulate, gate_A, gate_dt_bias, beta_scale)
+                           o_accumulate, gate_A, gate_dt_bias, beta_scale, gdn2_w)
     if k.dtype != q.dtype or v.dtype != q.dtype or beta.dtype != g.dtype:
         raise TypeError("q, k, v share one dtype and g, beta another")
     if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
@@ -157,7 +172,7 @@ def _norm_fields(q, norm_z, norm_weight, norm_eps):
 
 def make_decode_args(q, v, g, read_mode="post", scale=None, qk_l2norm=True, gate_A=None,
                      gate_dt_bias=None, beta_scale=1.0, norm_z=None, norm_weight=None,
-                     norm_eps=1e-6):
+                     norm_eps=1e-6, gdn2_w=None):
     N, Hk, dk = q.shape
     Hv, dv = v.shape[1], v.shape[2]
     if scale is None:
@@ -165,23 +180,24 @@ def make_decode_args(q, v, g, read_mode="post", scale=None, qk_l2norm=True, gate
     return DecodeArgs(N, Hk, Hv, dk, dv, _dtype_code(q), _dtype_code(g),
                       READ_PRE if read_mode == "pre" else READ_POST, float(scale),
                       int(bool(qk_l2norm)), *_gating_fields(gate_A, gate_dt_bias, beta_scale),
-                      *_norm_fields(q, norm_z, norm_weight, norm_eps))
+                      *_norm_fields(q, norm_z, norm_weight, norm_eps), *_gdn2_fields(g, v, gdn2_w))
 
 
 def decode_step(q, k, v, g, beta, S, *, read_mode="post", scale=None, qk_l2norm=True, o=None,
                 stream=None, gate_A=None, gate_dt_bias=None, beta_scale=1.0, norm_z=None,
-                norm_weight=None, norm_eps=1e-6):
+                norm_weight=None, norm_eps=1e-6, gdn2_w=None):
     """One recurrent token per sequence (gdr_decode_step): q, k [N,Hk,dk]; v [N,Hv,dv];
     g, beta [N,Hv]; S [N,Hv,dk,dv] fp32, updated in place.  With gate_A and gate_dt_bias
     ([Hv] fp32) given, g and beta are the raw projections of the fused gating prologue;
     with norm_z ([N,Hv,dv]) and norm_weight ([dv] fp32) given, o is the gated RMSNorm of
-    the recurrent output.  Returns o [N,Hv,dv]."""
+    the recurrent output; with gdn2_w ([N,Hv,dv]) given, g and beta are GDN-2's
+    per-key-channel log decay and erase gate ([N,Hv,dk]).  Returns o [N,Hv,dv]."""
     import torch
-    _check_cuda(q, k, v, g, beta, S, o, gate_A, gate_dt_bias, norm_z, norm_weight)
+    _check_cuda(q, k, v, g, beta, S, o, gate_A, gate_dt_bias, norm_z, norm_weight, gdn2_w)
     if S.dtype != torch.float32:
         raise TypeError("the state must be float32")
     args = make_decode_args(q, v, g, read_mode, scale, qk_l2norm, gate_A, gate_dt_bias,
-                            beta_scale, norm_z, norm_weight, norm_eps)
+                            beta_scale, norm_z, norm_weight, norm_eps, gdn2_w)
     if o is None:
         o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     st = _abi.lib().gdr_decode_step(ctypes.byref(args), _ptr(q), _ptr(k), _ptr(v), _ptr(g),

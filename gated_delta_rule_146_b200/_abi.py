@@ -28,7 +28,8 @@ class ChunkArgs(ctypes.Structure):
                 ("scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int),
                 ("reverse", ctypes.c_int), ("o_accumulate", ctypes.c_int),
                 ("gate_raw", ctypes.c_int), ("gate_A", ctypes.c_void_p),
-                ("gate_dt_bias", ctypes.c_void_p), ("beta_scale", ctypes.c_float)]
+                ("gate_dt_bias", ctypes.c_void_p), ("beta_scale", ctypes.c_float),
+                ("gdn2", ctypes.c_int), ("gdn2_w", ctypes.c_void_p)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -39,7 +40,8 @@ class DecodeArgs(ctypes.Structure):
                 ("gate_raw", ctypes.c_int), ("gate_A", ctypes.c_void_p),
                 ("gate_dt_bias", ctypes.c_void_p), ("beta_scale", ctypes.c_float),
                 ("out_norm", ctypes.c_int), ("norm_z", ctypes.c_void_p),
-                ("norm_weight", ctypes.c_void_p), ("norm_eps", ctypes.c_float)]
+                ("norm_weight", ctypes.c_void_p), ("norm_eps", ctypes.c_float),
+                ("gdn2", ctypes.c_int), ("gdn2_w", ctypes.c_void_p)]
 
 
 class GdrError(RuntimeError):

@@ -26,7 +26,13 @@ bool valid_dtype(gdr_dtype d) { return d == GDR_F32 || d == GDR_BF16; }
 // Fused gating fields: flags, the scale, and (for a call) the per-head arrays.
 template <typename Args>
 gdr_status check_gating(const Args* a, bool pointers) {
-    if (a->gate_raw & ~1) return GDR_ERR_INVALID_ARG;
+    if ((a->gate_raw | a->gdn2) & ~1) return GDR_ERR_INVALID_ARG;
+    if (a->gdn2) {
+        if (a->gate_raw) return GDR_ERR_INVALID_ARG;  // the decoupled gates come as they are
+        if (pointers && !a->gdn2_w) return GDR_ERR_INVALID_ARG;
+        if (pointers && !aligned16(a->gdn2_w)) return GDR_ERR_ALIGNMENT;
+        return GDR_OK;
+    }
     if (!a->gate_raw) return GDR_OK;
     if (!std::isfinite(a->beta_scale)) return GDR_ERR_INVALID_ARG;
     if (pointers) {

@@ -43,6 +43,7 @@ struct SimtParams {
     int gate_raw;                 // fused gating prologue (see gate_xform)
     const float* gate_A; const float* gate_dt_bias;
     float beta_scale;
+    const void* w;                // GDN-2 write gate [T][Hv][dv]; g, beta are then [T][Hv][dk]
 };
 
 // Normalise `rows` rows of length n (row stride ld) in shared memory, one warp per row.
@@ -244,15 +245,196 @@ chunk_scan_simt(SimtParams p) {
             p.S_final[sbase + (size_t)d * dv + col] = Hs[d * kSlice + lane];
 }
 
+// ---- GDN-2: decoupled per-channel gates ------------------------------------------
+// (tiny_gdn/fugue.py BidirectionalGatedDeltaNet2: S_t = (I - k_t (b_t . k_t)^T) Diag(e^{g_t})
+// S_{t-1} + k_t (w_t . v_t)^T.)  With G_t the per-key-channel cumulative log decay of the
+// chunk and H (= S^T) the state at its start, the chunk's u_t solve one unit-lower system
+//     u_t + sum_{s<t} A_ts u_s = w_t . v_t - H^T (e^{G_t} . b_t . k_t),
+//     A_ts = sum_d b_td k_td k_sd e^{G_td - G_sd},
+// so W = T (e^{G} . b . K) and U~ = T (w . V) with T = (I + A)^-1, and then
+//     o_t = q_t^T (e^{G'_t} . H) + sum_{s<=t} (sum_d q_td k_sd e^{G'_td - G_sd}) (U~ - W H)_s,
+//     H  <- e^{G_C} . H + sum_s (e^{G_C - G_s} . k_s) (U~ - W H)_s^T.
+
+__global__ void __launch_bounds__(kThreads)
+chunk_local_simt_g2(SimtParams p) {
+    extern __shared__ float sm[];
+    const WsHeader* hdr = p.hdr;
+    if (hdr->err != GDR_OK) return;
+    const int c = blockIdx.x, h = blockIdx.y;
+    if (c >= hdr->n_chunks) return;
+    const int s = p.chunk_seq[c];
+    const long long t0 = p.cu[s], t1 = p.cu[s + 1];
+    const int jc = c - p.chunk_off[s];
+    const int p0 = jc * p.chunk;
+    const int Cc = (int)min((long long)p.chunk, (t1 - t0) - p0);
+    const int dk = p.dk, dv = p.dv, ld = dk + dv + 1, C = p.chunk;
+    const int hk = h / (p.Hv / p.Hk);
+
+    float* R = sm;                       // [C][ld]: K | V, then W | U~ in place
+    float* A = R + C * ld;               // [C][C+1]
+    float* Gc = A + C * (C + 1);         // [C][dk] cumulative log decay per key channel
+    float* Bc = Gc + C * dk;             // [C][dk] erase gate
+    const int tid = threadIdx.x;
+
+    for (int idx = tid; idx < Cc * dk; idx += kThreads) {
+        const int i = idx / dk, d = idx % dk;
+        const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+        R[i * ld + d] = load_elem(p.k, (size_t)(t * p.Hk + hk) * dk + d, p.io);
+        Gc[i * dk + d] = load_elem(p.g, (size_t)(t * p.Hv + h) * dk + d, p.gt);
+        Bc[i * dk + d] = load_elem(p.beta, (size_t)(t * p.Hv + h) * dk + d, p.gt);
+    }
+    for (int idx = tid; idx < Cc * dv; idx += kThreads) {
+        const int i = idx / dv, d = idx % dv;
+        const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+        const size_t e = (size_t)(t * p.Hv + h) * dv + d;
+        R[i * ld + dk + d] = load_elem(p.v, e, p.io) * load_elem(p.w, e, p.gt);  // w . v
+    }
+    __syncthreads();
+    if (p.qk_l2norm) l2norm_rows(R, Cc, dk, ld);
+    for (int d = tid; d < dk; d += kThreads) {
+        float run = 0.f;
+        for (int i = 0; i < Cc; ++i) { run += Gc[i * dk + d]; Gc[i * dk + d] = run; }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < Cc * Cc; idx += kThreads) {
+        const int i = idx / Cc, j = idx % Cc;
+        float val = 0.f;
+        if (j < i)
+            for (int d = 0; d < dk; ++d)
+                val = fmaf(Bc[i * dk + d] * R[i * ld + d] * R[j * ld + d],
+                           expf(Gc[i * dk + d] - Gc[j * dk + d]), val);
+        A[i * (C + 1) + j] = val;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < Cc * dk; idx += kThreads) {  // K rows -> e^{G} . b . k
+        const int i = idx / dk, d = idx % dk;
+        R[i * ld + d] *= Bc[i * dk + d] * expf(Gc[i * dk + d]);
+    }
+    __syncthreads();
+    for (int col = tid; col < dk + dv; col += kThreads) {
+        for (int i = 1; i < Cc; ++i) {
+            float x = R[i * ld + col];
+            for (int j = 0; j < i; ++j) x = fmaf(-A[i * (C + 1) + j], R[j * ld + col], x);
+            R[i * ld + col] = x;
+        }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < Cc * dk; idx += kThreads) {
+        const int i = idx / dk, d = idx % dk;
+        const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+        p.W[(size_t)(t * p.Hv + h) * dk + d] = R[i * ld + d];
+        p.G[(size_t)(t * p.Hv + h) * dk + d] = Gc[i * dk + d];
+    }
+    for (int idx = tid; idx < Cc * dv; idx += kThreads) {
+        const int i = idx / dv, d = idx % dv;
+        const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+        p.U[(size_t)(t * p.Hv + h) * dv + d] = R[i * ld + dk + d];
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+chunk_scan_simt_g2(SimtParams p) {
+    extern __shared__ float sm[];
+    if (p.hdr->err != GDR_OK) return;
+    const int s = blockIdx.x, h = blockIdx.y, J = blockIdx.z;
+    const int dk = p.dk, dv = p.dv, C = p.chunk, ldk = dk + 1;
+    const int hk = h / (p.Hv / p.Hk);
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int col = J * kSlice + lane;  // this lane's dv column
+    const long long t0 = p.cu[s], t1 = p.cu[s + 1];
+    const int L = (int)(t1 - t0);
+
+    float* Hs = sm;                    // [dk][32]
+    float* Qs = Hs + dk * kSlice;      // [C][dk+1]
+    float* Ks = Qs + C * ldk;          // [C][dk+1]
+    float* Ws = Ks + C * ldk;          // [C][dk+1]
+    float* Us = Ws + C * ldk;          // [C][33]  U~ then V'
+    float* Os = Us + C * (kSlice + 1); // [C][33]  inter-chunk read
+    float* P = Os + C * (kSlice + 1);  // [C][C+1]
+    float* Gc = P + C * (C + 1);       // [C][dk] cumulative log decay per key channel
+
+    const size_t sbase = ((size_t)s * p.Hv + h) * dk * dv;
+    for (int d = wid; d < dk; d += kThreads / 32)
+        Hs[d * kSlice + lane] = p.S0 ? p.S0[sbase + (size_t)d * dv + col] : 0.f;
+
+    for (int p0 = 0; p0 < L; p0 += C) {
+        const int Cc = min(C, L - p0);
+        __syncthreads();
+        for (int idx = tid; idx < Cc * dk; idx += kThreads) {
+            const int i = idx / dk, d = idx % dk;
+            const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+            Qs[i * ldk + d] = load_elem(p.q, (size_t)(t * p.Hk + hk) * dk + d, p.io);
+            Ks[i * ldk + d] = load_elem(p.k, (size_t)(t * p.Hk + hk) * dk + d, p.io);
+            Ws[i * ldk + d] = p.W[(size_t)(t * p.Hv + h) * dk + d];
+            Gc[i * dk + d] = p.G[(size_t)(t * p.Hv + h) * dk + d];
+        }
+        for (int i = wid; i < Cc; i += kThreads / 32) {
+            const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+            Us[i * (kSlice + 1) + lane] = p.U[(size_t)(t * p.Hv + h) * dv + col];
+        }
+        __syncthreads();
+        if (p.qk_l2norm) { l2norm_rows(Qs, Cc, dk, ldk); l2norm_rows(Ks, Cc, dk, ldk); }
+        __syncthreads();
+        // the read decay G'_i: G_i (post-write) or G_{i-1} (pre-write, 0 for the first token)
+        auto gread = [&](int i, int d) -> float {
+            return p.read_pre ? (i > 0 ? Gc[(i - 1) * dk + d] : 0.f) : Gc[i * dk + d];
+        };
+        for (int idx = tid; idx < Cc * Cc; idx += kThreads) {
+            const int i = idx / Cc, j = idx % Cc;
+            float val = 0.f;
+            if (p.read_pre ? (j < i) : (j <= i))
+                for (int d = 0; d < dk; ++d)
+                    val = fmaf(Qs[i * ldk + d] * Ks[j * ldk + d], expf(gread(i, d) - Gc[j * dk + d]),
+                               val);
+            P[i * (C + 1) + j] = p.scale * val;
+        }
+        for (int i = wid; i < Cc; i += kThreads / 32) {
+            float wh = 0.f, qh = 0.f;
+            for (int d = 0; d < dk; ++d) {
+                const float hv = Hs[d * kSlice + lane];
+                wh = fmaf(Ws[i * ldk + d], hv, wh);
+                qh = fmaf(Qs[i * ldk + d] * expf(gread(i, d)), hv, qh);
+            }
+            Us[i * (kSlice + 1) + lane] -= wh;
+            Os[i * (kSlice + 1) + lane] = p.scale * qh;
+        }
+        __syncthreads();
+        for (int i = wid; i < Cc; i += kThreads / 32) {
+            float acc = Os[i * (kSlice + 1) + lane];
+            const int jmax = p.read_pre ? i - 1 : i;
+            for (int j = 0; j <= jmax; ++j)
+                acc = fmaf(P[i * (C + 1) + j], Us[j * (kSlice + 1) + lane], acc);
+            const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+            const size_t oi = (size_t)(t * p.Hv + h) * dv + col;
+            if (p.o_acc) acc += load_elem(p.o, oi, p.io);
+            store_elem(p.o, oi, acc, p.io);
+        }
+        for (int d = wid; d < dk; d += kThreads / 32) {
+            const float Gl = Gc[(Cc - 1) * dk + d];
+            float acc = 0.f;
+            for (int i = 0; i < Cc; ++i)
+                acc = fmaf(expf(Gl - Gc[i * dk + d]) * Ks[i * ldk + d], Us[i * (kSlice + 1) + lane],
+                           acc);
+            Hs[d * kSlice + lane] = fmaf(expf(Gl), Hs[d * kSlice + lane], acc);
+        }
+    }
+    __syncthreads();
+    if (p.S_final)
+        for (int d = wid; d < dk; d += kThreads / 32)
+            p.S_final[sbase + (size_t)d * dv + col] = Hs[d * kSlice + lane];
+}
+
 size_t local_smem(const gdr_chunk_args& a) {
     const int C = a.chunk;
-    return sizeof(float) * ((size_t)C * (a.dk + a.dv + 1) + (size_t)C * (C + 1) + 2 * C);
+    return sizeof(float) * ((size_t)C * (a.dk + a.dv + 1) + (size_t)C * (C + 1) +
+                            (a.gdn2 ? 2 * (size_t)C * a.dk : 2 * (size_t)C));
 }
 
 size_t scan_smem(const gdr_chunk_args& a) {
     const int C = a.chunk, ldk = a.dk + 1;
     return sizeof(float) * ((size_t)a.dk * kSlice + 3 * (size_t)C * ldk +
-                            2 * (size_t)C * (kSlice + 1) + (size_t)C * (C + 1) + 3 * C);
+                            2 * (size_t)C * (kSlice + 1) + (size_t)C * (C + 1) +
+                            (a.gdn2 ? (size_t)C * a.dk : 3 * (size_t)C));
 }
 
 constexpr size_t kMaxSmem = 227 * 1024;
@@ -283,19 +465,22 @@ gdr_status launch_chunk_simt(const gdr_chunk_args& a, const void* q, const void*
     p.o_acc = a.o_accumulate; p.io = a.io_dtype; p.gt = a.gate_dtype; p.scale = a.scale;
     p.gate_raw = a.gate_raw; p.gate_A = a.gate_A; p.gate_dt_bias = a.gate_dt_bias;
     p.beta_scale = a.beta_scale;
+    p.w = a.gdn2_w;
 
+    auto local = a.gdn2 ? chunk_local_simt_g2 : chunk_local_simt;
+    auto scan = a.gdn2 ? chunk_scan_simt_g2 : chunk_scan_simt;
     const size_t sm1 = local_smem(a), sm2 = scan_smem(a);
-    if ((cudaFuncSetAttribute(chunk_local_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((cudaFuncSetAttribute(local, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)sm1)) != cudaSuccess) return GDR_ERR_CUDA;
-    if ((cudaFuncSetAttribute(chunk_scan_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)sm2)) != cudaSuccess) return GDR_ERR_CUDA;
     if (L.max_chunks > 0) {
         dim3 g1((unsigned)L.max_chunks, (unsigned)a.Hv);
-        chunk_local_simt<<<g1, kThreads, sm1, st>>>(p);
+        local<<<g1, kThreads, sm1, st>>>(p);
         if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
     }
     dim3 g2((unsigned)a.n_seqs, (unsigned)a.Hv, (unsigned)(a.dv / kSlice));
-    chunk_scan_simt<<<g2, kThreads, sm2, st>>>(p);
+    scan<<<g2, kThreads, sm2, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
     return GDR_OK;
 }

@@ -1046,7 +1046,8 @@ bool make_tile_map(CUtensorMap* m, const void* base, int heads, long long tokens
 }  // namespace
 
 bool tc_supported(const gdr_chunk_args& a) {
-    return a.io_dtype == GDR_BF16 && a.dk == a.dv && (a.dk == D || a.dk == 64) && a.chunk == C;
+    return a.io_dtype == GDR_BF16 && a.dk == a.dv && (a.dk == D || a.dk == 64) && a.chunk == C &&
+           !a.gdn2;
 }
 
 gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k, const void* v,

@@ -85,7 +85,9 @@ inline WsLayout ws_layout(const gdr_chunk_args& a, bool simt) {
     if (simt) {
         L.W = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv * a.dk, 256);
         L.U = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv * a.dv, 256);
-        L.G = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv, 256);
+        // in-chunk log decay: one per token and head, or one per key channel for GDN-2
+        L.G = off;
+        off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv * (a.gdn2 ? a.dk : 1), 256);
     }
     L.total = off;
     return L;

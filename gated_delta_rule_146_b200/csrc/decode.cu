@@ -11,6 +11,10 @@
 // and, when the output epilogue is fused (the decode chain's gated RMSNorm, flashrt
 // fused_layer.py `_decode_one`), o <- o / sqrt(mean(o^2) + eps) * weight * silu(z) over
 // the head's dv values; that variant gives each block a whole head (DVS = DV).
+// GDN-2 (decoupled gates, tiny_gdn/fugue.py BidirectionalGatedDeltaNet2) in the same pass:
+// with per-row decay e^{g_d} and erase gate b_d and per-column write gate w_j,
+//     s_k = H^T (e^g . b . k),  u = w . v - s_k,  H <- e^g . H + k u^T,
+//     post: o = scale (H^T (e^g . q) + (k.q) u),  pre: o = scale H^T q.
 // The columns of H (dv) are independent, so a block owns a slice of DVS columns
 // and every row of it: it loads the whole slice into registers with 16-byte
 // streaming loads, reduces s_k and s_q over the dk rows (warp shuffles, then
@@ -37,9 +41,10 @@ struct DecodeParams {
     float beta_scale;
     const void* norm_z; const float* norm_weight;  // fused gated RMSNorm epilogue
     float norm_eps;
+    const void* w;                // GDN-2 write gate [N][Hv][dv]; g, beta are then [N][Hv][dk]
 };
 
-template <int DK, int DV, int DVS, bool kNorm>
+template <int DK, int DV, int DVS, bool kNorm, bool kG2>
 __global__ void __launch_bounds__(kThreads)
 decode_kernel(DecodeParams p) {
     static_assert(!kNorm || DVS == DV, "the normed epilogue needs the whole head in a block");
@@ -54,6 +59,7 @@ decode_kernel(DecodeParams p) {
     __shared__ float s_u[DVS];
     __shared__ float s_alpha, s_beta;
     __shared__ float s_o[kNorm ? DVS : 1];        // recurrent output of the head (epilogue)
+    __shared__ float s_eg[kG2 ? DK : 1], s_b[kG2 ? DK : 1];  // GDN-2: e^{g_d}, b_d per row
     __shared__ float s_ss[kWarps];
 
     const int nh = blockIdx.x;                   // n * Hv + h
@@ -77,8 +83,13 @@ decode_kernel(DecodeParams p) {
         s_q[d] = load_elem(p.q, qk_base + d, p.io);
         s_k[d] = load_elem(p.k, qk_base + d, p.io);
     }
-    if (tid == 0) {
-            s_alpha = expf(xform_g(p, h, load_elem(p.g, (size_t)nh, p.gt)));
+    if constexpr (kG2) {
+        for (int d = tid; d < DK; d += kThreads) {
+            s_eg[d] = expf(load_elem(p.g, (size_t)nh * DK + d, p.gt));
+            s_b[d] = load_elem(p.beta, (size_t)nh * DK + d, p.gt);
+        }
+    } else if (tid == 0) {
+        s_alpha = expf(xform_g(p, h, load_elem(p.g, (size_t)nh, p.gt)));
         s_beta = xform_beta(p, load_elem(p.beta, (size_t)nh, p.gt));
     }
     __syncthreads();
@@ -101,12 +112,17 @@ decode_kernel(DecodeParams p) {
 
     // partial s_k, s_q over this thread's rows, 4 columns
     float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sq = sk;
-    float kr[NP];
+    float kr[NP], er[NP];  // normalised k and (GDN-2) the row decay, per held row
 #pragma unroll
     for (int m = 0; m < NP; ++m) {
         const int d = m * RPP + wid * RPW + rw;
-        const float kd = s_k[d] * inv_k, qd = s_q[d] * inv_q;
+        float kd = s_k[d] * inv_k, qd = s_q[d] * inv_q;
         kr[m] = kd;
+        if constexpr (kG2) {  // weights of this row in s_k and s_q
+            er[m] = s_eg[d];
+            kd *= er[m] * s_b[d];
+            if (!p.read_pre) qd *= er[m];
+        }
         sk.x = fmaf(hreg[m].x, kd, sk.x); sk.y = fmaf(hreg[m].y, kd, sk.y);
         sk.z = fmaf(hreg[m].z, kd, sk.z); sk.w = fmaf(hreg[m].w, kd, sk.w);
         sq.x = fmaf(hreg[m].x, qd, sq.x); sq.y = fmaf(hreg[m].y, qd, sq.y);
@@ -134,9 +150,15 @@ decode_kernel(DecodeParams p) {
         for (int w = 0; w < kWarps; ++w) { tk += s_red[0][w][tid]; tq += s_red[1][w][tid]; }
         const int col = J * DVS + tid;
         const float vj = load_elem(p.v, (size_t)nh * DV + col, p.io);
-        const float u = beta * (vj - alpha * tk);
+        float u, oj;
+        if constexpr (kG2) {
+            u = load_elem(p.w, (size_t)nh * DV + col, p.gt) * vj - tk;
+            oj = p.read_pre ? p.scale * tq : p.scale * fmaf(kq, u, tq);
+        } else {
+            u = beta * (vj - alpha * tk);
+            oj = p.read_pre ? p.scale * tq : p.scale * fmaf(alpha, tq, kq * u);
+        }
         s_u[tid] = u;
-        const float oj = p.read_pre ? p.scale * tq : p.scale * fmaf(alpha, tq, kq * u);
         if constexpr (kNorm) s_o[tid] = oj;
         else store_elem(p.o, (size_t)nh * DV + col, oj, p.io);
     }
@@ -164,21 +186,22 @@ decode_kernel(DecodeParams p) {
     for (int m = 0; m < NP; ++m) {
         const int d = m * RPP + wid * RPW + rw;
         float4 r;
-        r.x = fmaf(alpha, hreg[m].x, kr[m] * u4.x); r.y = fmaf(alpha, hreg[m].y, kr[m] * u4.y);
-        r.z = fmaf(alpha, hreg[m].z, kr[m] * u4.z); r.w = fmaf(alpha, hreg[m].w, kr[m] * u4.w);
+        const float a = kG2 ? er[m] : alpha;
+        r.x = fmaf(a, hreg[m].x, kr[m] * u4.x); r.y = fmaf(a, hreg[m].y, kr[m] * u4.y);
+        r.z = fmaf(a, hreg[m].z, kr[m] * u4.z); r.w = fmaf(a, hreg[m].w, kr[m] * u4.w);
         __stcs(reinterpret_cast<float4*>(Sblk + (size_t)d * DV), r);
     }
 }
 
 template <int DK, int DV>
 gdr_status launch_dv(const gdr_decode_args& a, const DecodeParams& p, cudaStream_t st) {
-    if (a.out_norm) {  // one block per (sequence, head): the epilogue reduces over dv
-        decode_kernel<DK, DV, DV, true><<<dim3((unsigned)(a.N * a.Hv), 1), kThreads, 0, st>>>(p);
-    } else {
-        constexpr int DVS = DV >= 64 ? 64 : 32;
-        dim3 grid((unsigned)(a.N * a.Hv), DV / DVS);
-        decode_kernel<DK, DV, DVS, false><<<grid, kThreads, 0, st>>>(p);
-    }
+    constexpr int DVS = DV >= 64 ? 64 : 32;
+    const dim3 whole((unsigned)(a.N * a.Hv), 1), sliced((unsigned)(a.N * a.Hv), DV / DVS);
+    // the normed epilogue takes one block per (sequence, head): it reduces over dv
+    if (a.out_norm && a.gdn2) decode_kernel<DK, DV, DV, true, true><<<whole, kThreads, 0, st>>>(p);
+    else if (a.out_norm) decode_kernel<DK, DV, DV, true, false><<<whole, kThreads, 0, st>>>(p);
+    else if (a.gdn2) decode_kernel<DK, DV, DVS, false, true><<<sliced, kThreads, 0, st>>>(p);
+    else decode_kernel<DK, DV, DVS, false, false><<<sliced, kThreads, 0, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 
@@ -207,6 +230,7 @@ gdr_status launch_decode(const gdr_decode_args& a, const void* q, const void* k,
     p.gate_raw = a.gate_raw; p.gate_A = a.gate_A; p.gate_dt_bias = a.gate_dt_bias;
     p.beta_scale = a.beta_scale;
     p.norm_z = a.norm_z; p.norm_weight = a.norm_weight; p.norm_eps = a.norm_eps;
+    p.w = a.gdn2_w;
     switch (a.dk) {
         case 32: return launch_dk<32>(a, p, st);
         case 64: return launch_dk<64>(a, p, st);

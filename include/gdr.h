@@ -106,6 +106,16 @@ typedef struct {
     const float* gate_dt_bias;  /* [Hv] fp32 device array; 4-byte aligned; required when
                                    gate_raw */
     float beta_scale;           /* 1, or 2 for negative eigenvalues; must be finite */
+    /* GDN-2 decoupled gates (tiny_gdn/fugue.py BidirectionalGatedDeltaNet2:
+     * S_t = (I - k_t (b_t * k_t)^T) Diag(exp g_t) S_{t-1} + k_t (w_t * v_t)^T).
+     *   gdn2 = 0: scalar gates, g and beta of one value per token and value head.
+     *   gdn2 = 1: g is the per-key-channel log decay [.., Hv, dk], beta the per-key-channel
+     *             erase gate b [.., Hv, dk], and gdn2_w the per-value-channel write gate
+     *             [.., Hv, dv], all gate_dtype and 16-byte aligned.  With g = log(alpha),
+     *             b = w = beta on every channel this is the scalar rule.  Not combined with
+     *             gate_raw. */
+    int gdn2;
+    const void* gdn2_w;
 } gdr_chunk_args;
 
 /* Bytes of device workspace gdr_chunk_fwd needs for these arguments (0 on invalid
@@ -152,7 +162,8 @@ gdr_status gdr_chunk_fwd(const gdr_chunk_args* args,
  * - Calls whose scratch need (gdr_chunk_fwd_workspace_size) exceeds the array return
  *   GDR_ERR_WORKSPACE and enqueue nothing.  The tensor-core path needs only
  *   256 + 8 (n_seqs + 1) + 4 (ceil(B*T / chunk) + n_seqs) bytes; the CUDA-core path
- *   additionally 4 B*T Hv (dk + dv + 1) bytes, so it fits only small problems.
+ *   additionally 4 B*T Hv (dk + dv + 1) bytes (4 B*T Hv (2 dk + dv) with gdn2), so it fits
+ *   only small problems.
  * - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  *   with that device current; make that first call before any stream capture.
  * - All calls on a device share the one array: calls that overlap on the GPU (different
@@ -202,6 +213,16 @@ typedef struct {
     const float* norm_weight;   /* [dv] fp32, shared by the heads; 4-byte aligned; required
                                    when out_norm */
     float norm_eps;             /* >= 0, finite */
+    /* GDN-2 decoupled gates (tiny_gdn/fugue.py BidirectionalGatedDeltaNet2:
+     * S_t = (I - k_t (b_t * k_t)^T) Diag(exp g_t) S_{t-1} + k_t (w_t * v_t)^T).
+     *   gdn2 = 0: scalar gates, g and beta of one value per token and value head.
+     *   gdn2 = 1: g is the per-key-channel log decay [N, Hv, dk], beta the per-key-channel
+     *             erase gate b [N, Hv, dk], and gdn2_w the per-value-channel write gate
+     *             [N, Hv, dv], all gate_dtype and 16-byte aligned.  With g = log(alpha),
+     *             b = w = beta on every channel this is the scalar rule.  Not combined with
+     *             gate_raw. */
+    int gdn2;
+    const void* gdn2_w;
 } gdr_decode_args;
 
 /*

@@ -159,3 +159,29 @@ def test_decode_norm_host_validation(lib):
     assert f(out_norm=1, norm_weight=FAKE, norm_eps=1e-6) == _abi.GDR_ERR_INVALID_ARG
     assert f(out_norm=1, norm_z=FAKE + 8, norm_weight=FAKE, norm_eps=1e-6) == _abi.GDR_ERR_ALIGNMENT
     assert f(out_norm=1, norm_z=FAKE, norm_weight=FAKE + 2, norm_eps=1e-6) == _abi.GDR_ERR_ALIGNMENT
+
+
+def test_gdn2_host_validation(lib):
+    """GDN-2's flag and write-gate pointer are checked on the host; the decoupled gates take
+    the CUDA-core chunk path and a workspace with per-key-channel cumulative decays."""
+    scalar = args()
+    g2 = args(gdn2=1, gdn2_w=FAKE)
+    need = lib.gdr_chunk_fwd_workspace_size(ctypes.byref(g2))
+    assert need > lib.gdr_chunk_fwd_workspace_size(ctypes.byref(scalar))
+    assert lib.gdr_chunk_fwd_path(ctypes.byref(g2)) == b"simt"
+    assert lib.gdr_chunk_fwd_workspace_size(ctypes.byref(args(gdn2=2))) == 0
+    assert lib.gdr_chunk_fwd_workspace_size(
+        ctypes.byref(args(gdn2=1, gate_raw=1, gate_A=FAKE, gate_dt_bias=FAKE))) == 0
+    assert call(lib, args(gdn2=1), wsb=need) == _abi.GDR_ERR_INVALID_ARG     # no write gate
+    assert call(lib, args(gdn2=1, gdn2_w=FAKE + 4), wsb=need) == _abi.GDR_ERR_ALIGNMENT
+    assert call(lib, g2, wsb=need - 1) == _abi.GDR_ERR_WORKSPACE             # GDN-2 accepted
+    base = dict(N=4, Hk=2, Hv=4, dk=128, dv=128, io_dtype=_abi.BF16, gate_dtype=_abi.BF16,
+                read_mode=_abi.READ_POST, scale=0.1, qk_l2norm=1)
+    vp = ctypes.c_void_p
+    f = lambda **kw: lib.gdr_decode_step(ctypes.byref(_abi.DecodeArgs(**{**base, **kw})),
+                                         *[vp(FAKE)] * 7, None)
+    assert f(gdn2=3, gdn2_w=FAKE) == _abi.GDR_ERR_INVALID_ARG
+    assert f(gdn2=1) == _abi.GDR_ERR_INVALID_ARG
+    assert f(gdn2=1, gdn2_w=FAKE + 8) == _abi.GDR_ERR_ALIGNMENT
+    assert f(gdn2=1, gdn2_w=FAKE, gate_raw=1, gate_A=FAKE, gate_dt_bias=FAKE) \
+        == _abi.GDR_ERR_INVALID_ARG

@@ -178,3 +178,16 @@ def raw_gate_inputs(shape, Hv, gate_dtype="bf16", seed=0):
     a = (torch.randn(shape, generator=gen) - 2.0).to(dt)
     b = torch.randn(shape, generator=gen).to(dt)
     return a, b, torch.full((Hv,), -1.0), torch.zeros(Hv)
+
+
+def gdn2_gate_inputs(shape, dk, dv, gate_dtype="bf16", seed=0):
+    """Decoupled GDN-2 gates for tokens of ``shape`` (e.g. [B, T, Hv]): per key channel the
+    log decay g = -softplus(N(-2, 1)) and erase gate b = sigmoid(N(0, 1)) [*shape, dk], per
+    value channel the write gate w = sigmoid(N(0, 1)) [*shape, dv], in the gate dtype."""
+    gen = _gen(seed + 104729)
+    dt = DTYPES[gate_dtype]
+    shape = tuple(shape)
+    g = -torch.nn.functional.softplus(torch.randn(shape + (dk,), generator=gen) - 2.0)
+    b = torch.sigmoid(torch.randn(shape + (dk,), generator=gen))
+    w = torch.sigmoid(torch.randn(shape + (dv,), generator=gen))
+    return g.to(dt), b.to(dt), w.to(dt)
