@@ -19,7 +19,8 @@ import os
 from . import _abi
 from ._abi import GdrError, ChunkArgs, DecodeArgs, F32, BF16, READ_POST, READ_PRE  # noqa: F401
 
-__all__ = ["chunk_fwd", "decode_step", "chunk_fwd_workspace_size", "chunk_fwd_path",
+__all__ = ["chunk_fwd", "chunk_bwd", "decode_step", "chunk_fwd_workspace_size",
+           "chunk_bwd_workspace_size", "chunk_fwd_path",
            "read_device_error", "library", "GdrError"]
 
 
@@ -148,6 +149,47 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, *, chunk=64, read_mode
         ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
     _abi.check(st)
     return o, S_final
+
+
+def chunk_bwd_workspace_size(args: ChunkArgs) -> int:
+    return int(_abi.lib().gdr_chunk_bwd_workspace_size(ctypes.byref(args)))
+
+
+def chunk_bwd(q, k, v, g, beta, dO, S0=None, cu_seqlens=None, dS_final=None, *, chunk=64,
+              read_mode="post", scale=None, qk_l2norm=True, reverse=False, dS0=True,
+              workspace=None, stream=None):
+    """Backward pass of ``chunk_fwd`` (gdr_chunk_bwd): the gradients of
+    <dO, o> + <dS_final, S_final> for the same inputs.  dO has the shape of v (io dtype);
+    dS_final [n_seqs,Hv,dk,dv] fp32 or None.  Returns (dq, dk, dv, dg, dbeta, dS0) with the
+    shapes and dtypes of q, k, v, g, beta and S0 (dS0 fp32, None when ``dS0=False``)."""
+    import torch
+    _check_cuda(q, k, v, g, beta, dO, S0, cu_seqlens, dS_final, workspace)
+    args = make_chunk_args(q, v, g, cu_seqlens, chunk, read_mode, scale, qk_l2norm, reverse)
+    if k.dtype != q.dtype or v.dtype != q.dtype or dO.dtype != q.dtype or beta.dtype != g.dtype:
+        raise TypeError("q, k, v, dO share one dtype and g, beta another")
+    if tuple(dO.shape) != tuple(v.shape):
+        raise TypeError("dO has the shape of v")
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    for t in (S0, dS_final):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError("S0 and dS_final must be float32")
+    need = chunk_bwd_workspace_size(args)
+    if need == 0:
+        raise GdrError(_abi.GDR_ERR_UNSUPPORTED, "no backward kernel for these arguments")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg, dbeta = torch.empty_like(g), torch.empty_like(beta)
+    dS0_t = (torch.empty((args.n_seqs, args.Hv, args.dk, args.dv), dtype=torch.float32,
+                         device=q.device) if dS0 else None)
+    st = _abi.lib().gdr_chunk_bwd(
+        ctypes.byref(args), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+        _ptr(cu_seqlens), _ptr(dO), _ptr(dS_final), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+        _ptr(dbeta), _ptr(dS0_t), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
+    _abi.check(st)
+    return dq, dk, dv, dg, dbeta, dS0_t
 
 
 def read_device_error(args: ChunkArgs, workspace, stream=None) -> int:

@@ -122,6 +122,42 @@ gdr_status gdr_chunk_fwd(const gdr_chunk_args* a, const void* q, const void* k, 
     return launch_chunk_simt(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s);
 }
 
+size_t gdr_chunk_bwd_workspace_size(const gdr_chunk_args* a) {
+    if (check_chunk_args(a) != GDR_OK || !bwd_supported(*a)) return 0;
+    return bwd_layout(*a).total;
+}
+
+gdr_status gdr_chunk_bwd(const gdr_chunk_args* a, const void* q, const void* k, const void* v,
+                         const void* g, const void* beta, const float* S0,
+                         const int32_t* cu_seqlens, const void* dO, const float* dS_final,
+                         void* dq, void* dk, void* dv, void* dg, void* dbeta, float* dS0,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+    gdr_status st = check_chunk_args(a);
+    if (st != GDR_OK) return st;
+    if (cu_seqlens) {
+        if (a->B != 1) return GDR_ERR_INVALID_ARG;
+    } else if (a->n_seqs != a->B) {
+        return GDR_ERR_INVALID_ARG;
+    }
+    if (a->gate_raw || a->gdn2 || a->o_accumulate) return GDR_ERR_UNSUPPORTED;
+    const bool has_tokens = (long long)a->B * a->T > 0;
+    if (has_tokens && (!q || !k || !v || !g || !beta || !dO || !dq || !dk || !dv || !dg || !dbeta))
+        return GDR_ERR_INVALID_ARG;
+    if (!workspace) return GDR_ERR_WORKSPACE;
+    const void* ptrs[] = {q, k, v, g, beta, S0, cu_seqlens, dO, dS_final, dq, dk, dv, dg, dbeta,
+                          dS0, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDR_ERR_ALIGNMENT;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return GDR_ERR_ALIGNMENT;
+    if (!bwd_supported(*a)) return GDR_ERR_UNSUPPORTED;
+    const BwdLayout B = bwd_layout(*a);
+    if (workspace_bytes < B.total) return GDR_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (launch_plan(*a, cu_seqlens, workspace, B.base, s) != cudaSuccess) return GDR_ERR_CUDA;
+    const BwdPtrs x{q, k, v, g, beta, dO, S0, dS_final, dq, dk, dv, dg, dbeta, dS0};
+    return launch_chunk_bwd(*a, x, workspace, B, s);
+}
+
 gdr_status gdr_decode_step(const gdr_decode_args* a, const void* q, const void* k, const void* v,
                            const void* g, const void* beta, float* S_inout, void* o,
                            void* stream) {

@@ -485,4 +485,28 @@ gdr_status launch_chunk_simt(const gdr_chunk_args& a, const void* q, const void*
     return GDR_OK;
 }
 
+gdr_status launch_wy_local_simt(const gdr_chunk_args& a, const void* k, const void* v,
+                                const void* g, const void* beta, void* ws, const WsLayout& L,
+                                float* W, float* U, float* G, cudaStream_t st) {
+    if (a.gdn2 || L.max_chunks == 0) return a.gdn2 ? GDR_ERR_UNSUPPORTED : GDR_OK;
+    char* base = static_cast<char*>(ws);
+    SimtParams p{};
+    p.k = k; p.v = v; p.g = g; p.beta = beta;
+    p.hdr = reinterpret_cast<const WsHeader*>(base);
+    p.cu = reinterpret_cast<const int32_t*>(base + L.cu);
+    p.chunk_off = reinterpret_cast<const int32_t*>(base + L.chunk_off);
+    p.chunk_seq = reinterpret_cast<const int32_t*>(base + L.chunk_seq);
+    p.W = W; p.U = U; p.G = G;
+    p.Hk = a.Hk; p.Hv = a.Hv; p.dk = a.dk; p.dv = a.dv; p.chunk = a.chunk;
+    p.qk_l2norm = a.qk_l2norm; p.reverse = a.reverse;
+    p.io = a.io_dtype; p.gt = a.gate_dtype;
+    p.gate_raw = a.gate_raw; p.gate_A = a.gate_A; p.gate_dt_bias = a.gate_dt_bias;
+    p.beta_scale = a.beta_scale;
+    const size_t sm1 = local_smem(a);
+    if (cudaFuncSetAttribute(chunk_local_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sm1) != cudaSuccess) return GDR_ERR_CUDA;
+    chunk_local_simt<<<dim3((unsigned)L.max_chunks, (unsigned)a.Hv), kThreads, sm1, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
 }  // namespace gdr

@@ -117,6 +117,26 @@ gdr_status launch_chunk_simt(const gdr_chunk_args& a, const void* q, const void*
                              void* o, float* S_final, void* ws, const WsLayout& L,
                              cudaStream_t st);
 bool simt_supported(const gdr_chunk_args& a);
+// W, U~, G of every chunk (the CUDA-core forward's first kernel) into the given arrays.
+gdr_status launch_wy_local_simt(const gdr_chunk_args& a, const void* k, const void* v,
+                                const void* g, const void* beta, void* ws, const WsLayout& L,
+                                float* W, float* U, float* G, cudaStream_t st);
+
+// Backward pass (chunk_bwd.cu).
+struct BwdLayout {
+    WsLayout base;  // the forward's plan and CUDA-core arrays
+    size_t Hc, dHc, Vp, dVp, dW, dKp, dqh, dkh, dGp, total;
+};
+struct BwdPtrs {
+    const void *q, *k, *v, *g, *beta, *dO;
+    const float *S0, *dS_final;
+    void *dq, *dk, *dv, *dg, *dbeta;
+    float* dS0;
+};
+BwdLayout bwd_layout(const gdr_chunk_args& a);
+bool bwd_supported(const gdr_chunk_args& a);
+gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
+                            const BwdLayout& B, cudaStream_t st);
 gdr_status launch_decode(const gdr_decode_args& a, const void* q, const void* k, const void* v,
                          const void* g, const void* beta, float* S, void* o, cudaStream_t st);
 bool decode_supported(const gdr_decode_args& a);

@@ -185,6 +185,38 @@ gdr_status gdr_chunk_fwd_noalloc(const gdr_chunk_args* args,
 const char* gdr_chunk_fwd_path(const gdr_chunk_args* args);
 
 /*
+ * Backward pass of gdr_chunk_fwd: the gradients of
+ *     L = <dO, o> + <dS_final, S_final>
+ * with respect to q, k, v, g, beta and S0, for the same arguments (Prizma "seq/delta.py",
+ * module docstring: the chunk-parallel form agrees with the per-token recurrence on the
+ * forward and on the gradients; the gradient is the per-token recurrence's).  The forward's
+ * intermediate values are recomputed from the inputs; nothing from a forward call is kept.
+ *
+ *   args        as for gdr_chunk_fwd, with gate_raw = 0, gdn2 = 0, o_accumulate = 0;
+ *               kernels: chunk in {16, 32, 64}, dk <= 128, dv a multiple of 32 up to 128
+ *   q .. cu_seqlens   the forward's inputs, layouts as for gdr_chunk_fwd
+ *   dO          [B, T, Hv, dv]   io_dtype, gradient of o
+ *   dS_final    [n_seqs, Hv, dk, dv] fp32 gradient of S_final, or NULL for zero
+ *   dq, dk      [B, T, Hk, dk]   io_dtype outputs (summed over the v-heads of a key head)
+ *   dv          [B, T, Hv, dv]   io_dtype output
+ *   dg, dbeta   [B, T, Hv]       gate_dtype outputs (dg is the gradient of g = log alpha)
+ *   dS0         [n_seqs, Hv, dk, dv] fp32 output, or NULL
+ *   workspace   device scratch of at least gdr_chunk_bwd_workspace_size(args) bytes,
+ *               256-byte aligned, no initialisation needed
+ *
+ * Outputs are written, never accumulated.  Errors: as gdr_chunk_fwd; GDR_ERR_UNSUPPORTED
+ * for sizes or options outside the kernels' range.
+ */
+size_t gdr_chunk_bwd_workspace_size(const gdr_chunk_args* args);
+gdr_status gdr_chunk_bwd(const gdr_chunk_args* args,
+                         const void* q, const void* k, const void* v,
+                         const void* g, const void* beta,
+                         const float* S0, const int32_t* cu_seqlens,
+                         const void* dO, const float* dS_final,
+                         void* dq, void* dk, void* dv, void* dg, void* dbeta, float* dS0,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * One-token recurrent decode step (flashrt fused_layer.py `_decode_one`, the
  * recurrent core that reads and writes the cached state once per token).
  */

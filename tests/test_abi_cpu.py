@@ -185,3 +185,33 @@ def test_gdn2_host_validation(lib):
     assert f(gdn2=1, gdn2_w=FAKE + 8) == _abi.GDR_ERR_ALIGNMENT
     assert f(gdn2=1, gdn2_w=FAKE, gate_raw=1, gate_A=FAKE, gate_dt_bias=FAKE) \
         == _abi.GDR_ERR_INVALID_ARG
+
+
+def test_backward_host_validation(lib):
+    """gdr_chunk_bwd: sizes, options and pointers are checked on the host."""
+    a = args(dk=128, dv=128)
+    need = lib.gdr_chunk_bwd_workspace_size(ctypes.byref(a))
+    assert need > lib.gdr_chunk_fwd_workspace_size(ctypes.byref(a))
+    assert lib.gdr_chunk_bwd_workspace_size(ctypes.byref(args(chunk=128))) == 0
+    assert lib.gdr_chunk_bwd_workspace_size(ctypes.byref(args(dv=48))) == 0
+    assert lib.gdr_chunk_bwd_workspace_size(ctypes.byref(args(gdn2=1, gdn2_w=FAKE))) == 0
+    assert lib.gdr_chunk_bwd_workspace_size(
+        ctypes.byref(args(gate_raw=1, gate_A=FAKE, gate_dt_bias=FAKE))) == 0
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def bwd(a, wsb=need, **kw):
+        p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, S0=None, cu=None, dO=FAKE,
+                 dS=None, dq=FAKE, dk=FAKE, dv=FAKE, dg=FAKE, db=FAKE, dS0=FAKE, ws=FAKE)
+        p.update(kw)
+        return lib.gdr_chunk_bwd(ctypes.byref(a), *[vp(p[n]) for n in (
+            "q", "k", "v", "g", "beta", "S0", "cu", "dO", "dS", "dq", "dk", "dv", "dg", "db",
+            "dS0", "ws")], ctypes.c_size_t(wsb), None)
+
+    assert bwd(args(dk=128, dv=128, Hv=3)) == _abi.GDR_ERR_INVALID_ARG
+    assert bwd(a, dO=None) == _abi.GDR_ERR_INVALID_ARG
+    assert bwd(a, dg=FAKE + 4) == _abi.GDR_ERR_ALIGNMENT
+    assert bwd(a, ws=FAKE + 16) == _abi.GDR_ERR_ALIGNMENT
+    assert bwd(args(dk=128, dv=128, o_accumulate=1)) == _abi.GDR_ERR_UNSUPPORTED
+    assert bwd(args(dk=128, dv=128, chunk=128)) == _abi.GDR_ERR_UNSUPPORTED
+    assert bwd(a, ws=None) == _abi.GDR_ERR_WORKSPACE
+    assert bwd(a, wsb=need - 1) == _abi.GDR_ERR_WORKSPACE

@@ -1,0 +1,94 @@
+"""GPU parity of the backward pass (gdr_chunk_bwd) against the fp64 reverse-mode oracle
+``oracle.backward``, on the same seeded inputs and upstream gradients.
+
+Tolerance: bf16 as for the forward (2e-2 RMS(ref) + 2^-7 |ref| element-wise).  fp32: the
+pages ask the two forms to agree to 1e-4 on the forward and on the gradients; gradients
+scale with dO, T and the state, so the bound used is 1e-4 max(1, RMS(ref))."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.backward as obw
+import workloads
+import gated_delta_rule_146_b200 as gdr
+from gpu_helpers import assert_close, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def grad_close(name, gpu, ref, dtype):
+    if dtype == torch.bfloat16:
+        return assert_close(name, gpu, ref, dtype)
+    g = gpu.detach().double().cpu().numpy()
+    if not ref.size:
+        return
+    tol = 1e-4 * max(1.0, float(np.sqrt(np.mean(ref * ref))))
+    err = np.abs(g - ref)
+    assert err.max() <= tol, f"{name}: max err {err.max():.3e} > {tol:.3e}"
+
+
+def upstream(x, dtype, seed, with_dS=True):
+    gen = torch.Generator("cpu").manual_seed(seed)
+    dO = torch.randn(x["v"].shape, generator=gen).to(workloads.DTYPES[dtype])
+    n = x["S0"].shape[0] if x["S0"] is not None else (
+        x["v"].shape[0] if x["cu_seqlens"] is None else x["cu_seqlens"].numel() - 1)
+    Hv, dk, dv = x["v"].shape[2], x["q"].shape[3], x["v"].shape[3]
+    dS = torch.randn((n, Hv, dk, dv), generator=gen) if with_dS else None
+    return dO, dS
+
+
+def run_and_check(x, dO, dS, dtype, *, read_mode="post", scale=0.1, reverse=False, chunk=64,
+                  qk_l2norm=True):
+    dev = {n: to_dev(t) if t is not None else None for n, t in x.items()}
+    got = gdr.chunk_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], to_dev(dO),
+                        dev["S0"], dev["cu_seqlens"], to_dev(dS), chunk=chunk,
+                        read_mode=read_mode, scale=scale, reverse=reverse, qk_l2norm=qk_l2norm)
+    torch.cuda.synchronize()
+    ref = obw.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], dO, x["S0"], dS,
+                       x["cu_seqlens"], read_mode=read_mode, scale=scale, reverse=reverse,
+                       qk_l2norm=qk_l2norm)
+    dt = workloads.DTYPES[dtype]
+    for name, g in zip(("dq", "dk", "dv", "dg", "dbeta", "dS0"), got):
+        grad_close(name, g, ref[name], dt)
+
+
+@pytest.mark.parametrize("read_mode", ["post", "pre"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_gqa_several_chunks_ragged_tail(dtype, read_mode):
+    x = workloads.chunk_inputs(2, 150, 2, 4, 128, 128, dtype, s0_std=0.05, seed=61)
+    dO, dS = upstream(x, dtype, 62)
+    run_and_check(x, dO, dS, dtype, read_mode=read_mode, scale=1 / math.sqrt(128))
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_varlen_empty_and_one_token_sequences(reverse):
+    lengths = [1, 0, 64, 65, 130, 7]
+    x = workloads.chunk_inputs(1, 0, 1, 2, 64, 64, "f32", lengths=lengths, s0_std=0.1, seed=63)
+    dO, dS = upstream(x, "f32", 64)
+    run_and_check(x, dO, dS, "f32", read_mode="pre", scale=0.3, reverse=reverse)
+
+
+@pytest.mark.parametrize("chunk", [16, 32])
+def test_smaller_chunks_rectangular_heads(chunk):
+    x = workloads.chunk_inputs(1, 100, 1, 1, 96, 64, "f32", s0_std=0.05, seed=65)
+    dO, dS = upstream(x, "f32", 66)
+    run_and_check(x, dO, dS, "f32", chunk=chunk, scale=0.2)
+
+
+def test_no_state_gradients_and_no_norm():
+    """S0 = None and dS_final = None (zero), without the in-kernel normalisation."""
+    x = workloads.chunk_inputs(1, 80, 2, 2, 32, 32, "f32", seed=67)
+    x["q"] = x["q"] * 0.2
+    x["k"] = x["k"] * 0.2
+    dO, _ = upstream(x, "f32", 68, with_dS=False)
+    run_and_check(x, dO, None, "f32", scale=1.0, qk_l2norm=False)
+
+
+def test_bidirectional_workload_rows():
+    """Two sequences of the bidirectional workload's shape (2048 tokens, H=12, d=64,
+    pre-write read, scale 1): the reverse direction's backward."""
+    x = workloads.chunk_inputs(1, 0, 12, 12, 64, 64, "bf16", lengths=[2048, 2048], seed=69)
+    dO, dS = upstream(x, "bf16", 70, with_dS=False)
+    run_and_check(x, dO, None, "bf16", read_mode="pre", scale=1.0, reverse=True)
