@@ -359,6 +359,46 @@ def bench_ours(args, rank, world, local_rank):
         ngbs = nbytes / (nms / 1e3) / 1e9
         dec["fused_output_norm"] = {"ms_per_step": nms, "value": world * ngbs, "unit": "GB/s",
                                     "frac": ngbs / peaks["hbm_gbs"]}
+    # ---------------- backward pass (gdr_chunk_bwd) on the same workload and inputs, with a
+    # seeded upstream gradient dO; gradients of q, k, v, g, beta and S0
+    backward = None
+    if args.backward and args.only != "decode" and not args.rows:
+        gen = torch.Generator("cpu").manual_seed(1000 + rank)
+        dOb = torch.randn(tuple(d["v"].shape), generator=gen).to(d["v"].dtype).to(dev)
+        bargs_ = gdr.make_chunk_args(d["q"], d["v"], d["g"], d["cu_seqlens"], w.chunk,
+                                     w.read_mode, w.scale)
+        bws_ = torch.empty(gdr.chunk_bwd_workspace_size(bargs_), dtype=torch.uint8, device=dev)
+
+        def bwstep():
+            gdr.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], dOb, d["S0"],
+                          d["cu_seqlens"], None, chunk=w.chunk, read_mode=w.read_mode,
+                          scale=w.scale, workspace=bws_)
+
+        bwsteps = min(args.steps, 5)
+        for _ in range(min(args.warmup, 3)):
+            bwstep()
+        torch.cuda.synchronize()
+        barrier()
+        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        k0.record(stream)
+        for _ in range(bwsteps):
+            bwstep()
+        k1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        kms = max_over_ranks(k0.elapsed_time(k1) / bwsteps, world)
+        # read q, k, v, g, beta, dO (and S0); write dq, dk, dv, dg, dbeta (and dS0)
+        kbytes = 2 * sum(d[n].numel() * d[n].element_size() for n in ("q", "k", "v", "g", "beta"))
+        kbytes += dOb.numel() * dOb.element_size()
+        if d["S0"] is not None:
+            kbytes += 2 * d["S0"].numel() * 4
+        backward = {"workload": w.name, "ms_per_step": kms, "steps": bwsteps,
+                    "value": whole_job_rate(tokens, world, kms), "unit": "tokens/s",
+                    "path": "simt (fp32 CUDA cores)", "algorithmic_bytes": kbytes,
+                    "hbm_frac": kbytes / (kms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                    "workspace_bytes": bws_.numel()}
+        del bws_
+
     # ---------------- GDN-2 (decoupled per-channel gates): the chunk workload on the CUDA-core
     # path and the decode steps, same inputs with g, beta per key channel and a write gate
     gdn2 = None
@@ -476,7 +516,7 @@ def bench_ours(args, rank, world, local_rank):
                      "tensor_frac": tflops / peaks["bf16_tflops"],
                      "timed": "whole gdr_chunk_fwd call (plan + chunk kernels), CUDA events",
                      "peak_source": f"{peak_src} (hbm_gbs copy; bf16_tflops burst)"},
-        "decode": dec, "gating_prologue": gating, "bidirectional": bidir, "gdn2": gdn2, "e2e": e2e,
+        "decode": dec, "gating_prologue": gating, "bidirectional": bidir, "gdn2": gdn2, "backward": backward, "e2e": e2e,
         "clocks": clocks,
         "gpu_launches": launches_per_call * args.steps,
     }
@@ -540,6 +580,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=CHUNK_WORKLOAD)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-backward", dest="backward", action="store_false",
+                    help="skip the backward-pass measurement")
     ap.add_argument("--no-gdn2", dest="gdn2", action="store_false",
                     help="skip the GDN-2 (decoupled gates) chunk and decode measurements")
     ap.add_argument("--no-bidir", action="store_true",

@@ -92,3 +92,28 @@ def test_bidirectional_workload_rows():
     x = workloads.chunk_inputs(1, 0, 12, 12, 64, 64, "bf16", lengths=[2048, 2048], seed=69)
     dO, dS = upstream(x, "bf16", 70, with_dS=False)
     run_and_check(x, dO, None, "bf16", read_mode="pre", scale=1.0, reverse=True)
+
+
+def test_training_shape_workload_sampled():
+    """The backward at the training workload's full size (8 x 4096 tokens, 16 heads, d=128,
+    bf16), checked on sampled (sequence, head) units that the oracle computes one by one
+    (key heads = value heads here, so dq and dk of a unit are its own)."""
+    w = workloads.WORKLOADS["bf16_b8_h16_t4096_d128"]
+    assert w.Hk == w.Hv
+    x = workloads.workload_inputs(w)
+    gen = torch.Generator("cpu").manual_seed(71)
+    dO = torch.randn(x["v"].shape, generator=gen).to(torch.bfloat16)
+    dev = {n: to_dev(t) if t is not None else None for n, t in x.items()}
+    got = gdr.chunk_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], to_dev(dO),
+                        dev["S0"], None, None, chunk=w.chunk, read_mode=w.read_mode,
+                        scale=w.scale)
+    torch.cuda.synchronize()
+    assert all(torch.isfinite(t.float()).all() for t in got)
+    for b, h in [(0, 0), (w.B - 1, w.Hv - 1), (3, 7)]:
+        sl = lambda t: t[b:b + 1, :, h:h + 1]
+        ref = obw.backward(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]), sl(x["beta"]),
+                           sl(dO), None if x["S0"] is None else x["S0"][b:b + 1, h:h + 1],
+                           None, read_mode=w.read_mode, scale=w.scale)
+        for name, g in zip(("dq", "dk", "dv", "dg", "dbeta"), got[:5]):
+            grad_close(f"{name}[{b},{h}]", sl(g), ref[name], torch.bfloat16)
+        grad_close(f"dS0[{b},{h}]", got[5][b:b + 1, h:h + 1], ref["dS0"], torch.bfloat16)
