@@ -25,6 +25,7 @@
 // Kernels, in order on the stream:
 //   plan_kernel            chunk map (shared with the forward)
 //   chunk_local_simt       W, U~, G per chunk (shared with the forward's CUDA-core path)
+//   bwd_chunk_prep         per (chunk, head): s e^{G'} q^, e^{G_C - G} k^ and P
 //   bwd_states_fwd         per (sequence, head, 32-column slice): H at every chunk start, V'
 //   bwd_states_bwd         same grid, chunks in reverse: dH+ at every chunk, dV', dS0
 //   bwd_chunk_dqk          per (chunk, head): dq (normalised adjoint), the P and carry parts
@@ -53,6 +54,9 @@ struct BwdParams {
     float *Vp, *dVp;                // [T][Hv][dv]: V', dV'
     float *dW, *dKp, *dqh, *dkh;    // [T][Hv][dk]
     float* dGp;                     // [T][Hv]
+    float *Qt, *Kt;                 // [T][Hv][dk]: s e^{G'} q^, e^{G_C - G} k^ (state passes;
+                                    // they share the storage of dqh, dkh, written later)
+    float* Pc;                      // [max_chunks][Hv][C][C]: P, zero off the mask
     int Hk, Hv, dk, dv, chunk, read_pre, qk_l2norm, reverse;
     gdr_dtype io, gt;
     float scale;
@@ -117,26 +121,41 @@ __device__ __forceinline__ bool chunk_pos(const BwdParams& p, ChunkPos& cp) {
 }
 
 // ---- state passes: one block per (sequence, v-head, 32-column slice of dv) ---------------
+//
+// Lane l of every warp owns column l of the slice.  Warp w owns rows w*RP .. w*RP+RP-1 of
+// the chunk's [C x 32] products (RP = C/8) and rows w*DR .. w*DR+DR-1 of the [dk x 32]
+// state (DR = dk/8), so each lane keeps RP or DR independent accumulators and reads the
+// row operands as float4 broadcasts.  K~ = e^{G_C - G} k^, Q~ = s e^{G'} q^ and P come from
+// bwd_chunk_prep, so the passes hold no normalisation or exponential.
 
+__device__ __forceinline__ void load_rows4(float* dst, const float* src, size_t row_stride,
+                                           int rows, int n, const BwdParams& p, long long t0,
+                                           long long t1, int p0, int h) {
+    const int n4 = n / 4;
+    for (int idx = threadIdx.x; idx < rows * n4; idx += kThreads) {
+        const int i = idx / n4, d4 = idx % n4;
+        const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+        reinterpret_cast<float4*>(dst + (size_t)i * n)[d4] =
+            reinterpret_cast<const float4*>(src + ((size_t)t * p.Hv + h) * row_stride)[d4];
+    }
+}
+
+template <int RP, int DR>
 __global__ void __launch_bounds__(kThreads)
 bwd_states_fwd(BwdParams p) {
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     if (p.hdr->err != GDR_OK) return;
     const int s = blockIdx.x, h = blockIdx.y, J = blockIdx.z;
-    const int dk = p.dk, dv = p.dv, C = p.chunk, ldk = dk + 1;
-    const int hk = h / (p.Hv / p.Hk);
+    const int dk = p.dk, dv = p.dv, C = p.chunk;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int col = J * kSlice + lane;
     const long long t0 = p.cu[s], t1 = p.cu[s + 1];
     const int L = (int)(t1 - t0);
 
     float* Hs = sm;                     // [dk][32]
-    float* Ks = Hs + dk * kSlice;       // [C][dk+1]
-    float* Ws = Ks + C * ldk;           // [C][dk+1]
-    float* Us = Ws + C * ldk;           // [C][33]  U~ then V'
-    float* Gs = Us + C * (kSlice + 1);  // [C]
-    float* Kd = Gs + C;                 // [C] e^{G_C - G_i}
-    float* nr = Kd + C;                 // [C] norms (unused here)
+    float* Kt = Hs + dk * kSlice;       // [C][dk] K~
+    float* Ws = Kt + C * dk;            // [C][dk] W
+    float* Us = Ws + C * dk;            // [C][33] U~ then V'
 
     const size_t sbase = ((size_t)s * p.Hv + h) * dk * dv;
     for (int d = wid; d < dk; d += kThreads / 32)
@@ -148,47 +167,69 @@ bwd_states_fwd(BwdParams p) {
         __syncthreads();
         for (int d = wid; d < dk; d += kThreads / 32)
             p.Hc[cbase + (size_t)d * dv + col] = Hs[d * kSlice + lane];
-        for (int idx = tid; idx < Cc * dk; idx += kThreads) {
-            const int i = idx / dk, d = idx % dk;
-            const long long t = phys_token(t0, t1, p0 + i, p.reverse);
-            Ks[i * ldk + d] = load_elem(p.k, (size_t)(t * p.Hk + hk) * dk + d, p.io);
-            Ws[i * ldk + d] = p.W[(size_t)(t * p.Hv + h) * dk + d];
-        }
+        load_rows4(Kt, p.Kt, dk, Cc, dk, p, t0, t1, p0, h);
+        load_rows4(Ws, p.W, dk, Cc, dk, p, t0, t1, p0, h);
         for (int i = wid; i < Cc; i += kThreads / 32) {
             const long long t = phys_token(t0, t1, p0 + i, p.reverse);
             Us[i * (kSlice + 1) + lane] = p.U[(size_t)(t * p.Hv + h) * dv + col];
-            if (lane == 0) Gs[i] = p.G[(size_t)t * p.Hv + h];
+        }
+        const float gC = expf(p.G[(size_t)phys_token(t0, t1, p0 + Cc - 1, p.reverse) * p.Hv + h]);
+        __syncthreads();
+        // V' = U~ - W H, rows wid*RP + r
+        {
+            float acc[RP];
+#pragma unroll
+            for (int r = 0; r < RP; ++r) acc[r] = 0.f;
+            for (int d = 0; d < dk; d += 4) {
+                const float h0 = Hs[(d + 0) * kSlice + lane], h1 = Hs[(d + 1) * kSlice + lane];
+                const float h2 = Hs[(d + 2) * kSlice + lane], h3 = Hs[(d + 3) * kSlice + lane];
+#pragma unroll
+                for (int r = 0; r < RP; ++r) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(Ws + (wid * RP + r) * dk + d);
+                    acc[r] = fmaf(w4.x, h0, fmaf(w4.y, h1, fmaf(w4.z, h2, fmaf(w4.w, h3, acc[r]))));
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+                const int i = wid * RP + r;
+                if (i < Cc) {
+                    const float vp = Us[i * (kSlice + 1) + lane] - acc[r];
+                    Us[i * (kSlice + 1) + lane] = vp;
+                    const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+                    p.Vp[(size_t)(t * p.Hv + h) * dv + col] = vp;
+                }
+            }
         }
         __syncthreads();
-        l2norm_rows_keep(Ks, nr, Cc, dk, ldk, p.qk_l2norm);
-        for (int i = tid; i < Cc; i += kThreads) Kd[i] = expf(Gs[Cc - 1] - Gs[i]);
-        // V' = U~ - W H
-        for (int i = wid; i < Cc; i += kThreads / 32) {
-            float wh = 0.f;
-            for (int d = 0; d < dk; ++d) wh = fmaf(Ws[i * ldk + d], Hs[d * kSlice + lane], wh);
-            const float vp = Us[i * (kSlice + 1) + lane] - wh;
-            Us[i * (kSlice + 1) + lane] = vp;
-            const long long t = phys_token(t0, t1, p0 + i, p.reverse);
-            p.Vp[(size_t)(t * p.Hv + h) * dv + col] = vp;
-        }
-        __syncthreads();
-        const float gC = expf(Gs[Cc - 1]);
-        for (int d = wid; d < dk; d += kThreads / 32) {
-            float acc = 0.f;
-            for (int i = 0; i < Cc; ++i)
-                acc = fmaf(Kd[i] * Ks[i * ldk + d], Us[i * (kSlice + 1) + lane], acc);
-            Hs[d * kSlice + lane] = fmaf(gC, Hs[d * kSlice + lane], acc);
+        // H <- e^{G_C} H + K~^T V', rows wid*DR + dr
+        {
+            float acc[DR];
+#pragma unroll
+            for (int r = 0; r < DR; ++r) acc[r] = gC * Hs[(wid * DR + r) * kSlice + lane];
+            for (int i = 0; i < Cc; ++i) {
+                const float v = Us[i * (kSlice + 1) + lane];
+#pragma unroll
+                for (int r = 0; r < DR; r += 4) {
+                    const float4 k4 = *reinterpret_cast<const float4*>(Kt + i * dk + wid * DR + r);
+                    acc[r] = fmaf(k4.x, v, acc[r]);
+                    acc[r + 1] = fmaf(k4.y, v, acc[r + 1]);
+                    acc[r + 2] = fmaf(k4.z, v, acc[r + 2]);
+                    acc[r + 3] = fmaf(k4.w, v, acc[r + 3]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < DR; ++r) Hs[(wid * DR + r) * kSlice + lane] = acc[r];
         }
     }
 }
 
+template <int RP, int DR>
 __global__ void __launch_bounds__(kThreads)
 bwd_states_bwd(BwdParams p) {
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     if (p.hdr->err != GDR_OK) return;
     const int s = blockIdx.x, h = blockIdx.y, J = blockIdx.z;
-    const int dk = p.dk, dv = p.dv, C = p.chunk, ldk = dk + 1;
-    const int hk = h / (p.Hv / p.Hk);
+    const int dk = p.dk, dv = p.dv, C = p.chunk;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int col = J * kSlice + lane;
     const long long t0 = p.cu[s], t1 = p.cu[s + 1];
@@ -196,16 +237,12 @@ bwd_states_bwd(BwdParams p) {
     const int nC = (L + C - 1) / C;
 
     float* dHs = sm;                    // [dk][32]
-    float* Qs = dHs + dk * kSlice;      // [C][dk+1]
-    float* Ks = Qs + C * ldk;           // [C][dk+1]
-    float* Ws = Ks + C * ldk;           // [C][dk+1]
-    float* dOs = Ws + C * ldk;          // [C][33]
+    float* Kt = dHs + dk * kSlice;      // [C][dk] K~
+    float* Qt = Kt + C * dk;            // [C][dk] Q~
+    float* Ws = Qt + C * dk;            // [C][dk] W
+    float* Ps = Ws + C * dk;            // [C][C]  P (scaled, decayed, masked)
+    float* dOs = Ps + C * C;            // [C][33]
     float* dVs = dOs + C * (kSlice + 1);// [C][33]
-    float* P = dVs + C * (kSlice + 1);  // [C][C+1]
-    float* Gs = P + C * (C + 1);        // [C]
-    float* Rd = Gs + C;                 // [C] e^{G'_i}
-    float* Kd = Rd + C;                 // [C] e^{G_C - G_i}
-    float* nr = Kd + C;                 // [C] norms (unused here)
 
     const size_t sbase = ((size_t)s * p.Hv + h) * dk * dv;
     for (int d = wid; d < dk; d += kThreads / 32)
@@ -213,63 +250,74 @@ bwd_states_bwd(BwdParams p) {
 
     for (int jc = nC - 1; jc >= 0; --jc) {
         const int p0 = jc * C, Cc = min(C, L - p0);
-        const size_t cbase = ((size_t)(p.chunk_off[s] + jc) * p.Hv + h) * dk * dv;
+        const int c = p.chunk_off[s] + jc;
+        const size_t cbase = ((size_t)c * p.Hv + h) * dk * dv;
         __syncthreads();
         for (int d = wid; d < dk; d += kThreads / 32)
             p.dHc[cbase + (size_t)d * dv + col] = dHs[d * kSlice + lane];
-        for (int idx = tid; idx < Cc * dk; idx += kThreads) {
-            const int i = idx / dk, d = idx % dk;
-            const long long t = phys_token(t0, t1, p0 + i, p.reverse);
-            Qs[i * ldk + d] = load_elem(p.q, (size_t)(t * p.Hk + hk) * dk + d, p.io);
-            Ks[i * ldk + d] = load_elem(p.k, (size_t)(t * p.Hk + hk) * dk + d, p.io);
-            Ws[i * ldk + d] = p.W[(size_t)(t * p.Hv + h) * dk + d];
+        load_rows4(Kt, p.Kt, dk, Cc, dk, p, t0, t1, p0, h);
+        load_rows4(Qt, p.Qt, dk, Cc, dk, p, t0, t1, p0, h);
+        load_rows4(Ws, p.W, dk, Cc, dk, p, t0, t1, p0, h);
+        {
+            const float4* src = reinterpret_cast<const float4*>(p.Pc + ((size_t)c * p.Hv + h) * C * C);
+            for (int idx = tid; idx < C * C / 4; idx += kThreads)
+                reinterpret_cast<float4*>(Ps)[idx] = src[idx];
         }
         for (int i = wid; i < Cc; i += kThreads / 32) {
             const long long t = phys_token(t0, t1, p0 + i, p.reverse);
             dOs[i * (kSlice + 1) + lane] = load_elem(p.dO, (size_t)(t * p.Hv + h) * dv + col, p.io);
-            if (lane == 0) Gs[i] = p.G[(size_t)t * p.Hv + h];
         }
+        const float gC = expf(p.G[(size_t)phys_token(t0, t1, p0 + Cc - 1, p.reverse) * p.Hv + h]);
         __syncthreads();
-        l2norm_rows_keep(Qs, nr, Cc, dk, ldk, p.qk_l2norm);
-        l2norm_rows_keep(Ks, nr, Cc, dk, ldk, p.qk_l2norm);
-        for (int i = tid; i < Cc; i += kThreads) {
-            Rd[i] = expf(p.read_pre ? (i > 0 ? Gs[i - 1] : 0.f) : Gs[i]);
-            Kd[i] = expf(Gs[Cc - 1] - Gs[i]);
-        }
-        __syncthreads();
-        for (int idx = tid; idx < Cc * Cc; idx += kThreads) {
-            const int i = idx / Cc, j = idx % Cc;
-            float val = 0.f;
-            if (p.read_pre ? (j < i) : (j <= i)) {
-                float dot = 0.f;
-                for (int d = 0; d < dk; ++d) dot = fmaf(Qs[i * ldk + d], Ks[j * ldk + d], dot);
-                const float Gi = p.read_pre ? (i > 0 ? Gs[i - 1] : 0.f) : Gs[i];
-                val = p.scale * dot * expf(Gi - Gs[j]);
-            }
-            P[i * (C + 1) + j] = val;
-        }
-        __syncthreads();
-        // dV'_j = sum_i P_ij dO_i + e^{G_C - G_j} k^_j^T dH+
-        for (int j = wid; j < Cc; j += kThreads / 32) {
-            float acc = 0.f;
-            for (int i = j; i < Cc; ++i) acc = fmaf(P[i * (C + 1) + j], dOs[i * (kSlice + 1) + lane], acc);
-            float kh = 0.f;
-            for (int d = 0; d < dk; ++d) kh = fmaf(Ks[j * ldk + d], dHs[d * kSlice + lane], kh);
-            const float dvp = fmaf(Kd[j], kh, acc);
-            dVs[j * (kSlice + 1) + lane] = dvp;
-            const long long t = phys_token(t0, t1, p0 + j, p.reverse);
-            p.dVp[(size_t)(t * p.Hv + h) * dv + col] = dvp;
-        }
-        __syncthreads();
-        // dH = e^{G_C} dH+ + s (diag(e^{G'}) Q^)^T dO - W^T dV'
-        const float gC = expf(Gs[Cc - 1]);
-        for (int d = wid; d < dk; d += kThreads / 32) {
-            float acc = 0.f;
+        // dV'_j = sum_i P_ij dO_i + K~_j . dH+, rows j = wid*RP + r
+        {
+            float acc[RP];
+#pragma unroll
+            for (int r = 0; r < RP; ++r) acc[r] = 0.f;
             for (int i = 0; i < Cc; ++i) {
-                acc = fmaf(p.scale * Rd[i] * Qs[i * ldk + d], dOs[i * (kSlice + 1) + lane], acc);
-                acc = fmaf(-Ws[i * ldk + d], dVs[i * (kSlice + 1) + lane], acc);
+                const float a = dOs[i * (kSlice + 1) + lane];
+#pragma unroll
+                for (int r = 0; r < RP; ++r) acc[r] = fmaf(Ps[i * C + wid * RP + r], a, acc[r]);
             }
-            dHs[d * kSlice + lane] = fmaf(gC, dHs[d * kSlice + lane], acc);
+            for (int d = 0; d < dk; d += 4) {
+                const float h0 = dHs[(d + 0) * kSlice + lane], h1 = dHs[(d + 1) * kSlice + lane];
+                const float h2 = dHs[(d + 2) * kSlice + lane], h3 = dHs[(d + 3) * kSlice + lane];
+#pragma unroll
+                for (int r = 0; r < RP; ++r) {
+                    const float4 k4 = *reinterpret_cast<const float4*>(Kt + (wid * RP + r) * dk + d);
+                    acc[r] = fmaf(k4.x, h0, fmaf(k4.y, h1, fmaf(k4.z, h2, fmaf(k4.w, h3, acc[r]))));
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+                const int j = wid * RP + r;
+                if (j < Cc) {
+                    dVs[j * (kSlice + 1) + lane] = acc[r];
+                    const long long t = phys_token(t0, t1, p0 + j, p.reverse);
+                    p.dVp[(size_t)(t * p.Hv + h) * dv + col] = acc[r];
+                }
+            }
+        }
+        __syncthreads();
+        // dH = e^{G_C} dH+ + Q~^T dO - W^T dV', rows wid*DR + dr
+        {
+            float acc[DR];
+#pragma unroll
+            for (int r = 0; r < DR; ++r) acc[r] = gC * dHs[(wid * DR + r) * kSlice + lane];
+            for (int i = 0; i < Cc; ++i) {
+                const float a = dOs[i * (kSlice + 1) + lane], b = dVs[i * (kSlice + 1) + lane];
+#pragma unroll
+                for (int r = 0; r < DR; r += 4) {
+                    const float4 q4 = *reinterpret_cast<const float4*>(Qt + i * dk + wid * DR + r);
+                    const float4 w4 = *reinterpret_cast<const float4*>(Ws + i * dk + wid * DR + r);
+                    acc[r] = fmaf(q4.x, a, fmaf(-w4.x, b, acc[r]));
+                    acc[r + 1] = fmaf(q4.y, a, fmaf(-w4.y, b, acc[r + 1]));
+                    acc[r + 2] = fmaf(q4.z, a, fmaf(-w4.z, b, acc[r + 2]));
+                    acc[r + 3] = fmaf(q4.w, a, fmaf(-w4.w, b, acc[r + 3]));
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < DR; ++r) dHs[(wid * DR + r) * kSlice + lane] = acc[r];
         }
     }
     __syncthreads();
@@ -288,6 +336,68 @@ __device__ void load_rows(float* dst, int C, int Cc, int n, int ld, F&& get) {
         const int i = idx / n, d = idx % n;
         dst[i * ld + d] = i < Cc ? get(i, d) : 0.f;
     }
+}
+
+// Q~ = s e^{G'} q^, K~ = e^{G_C - G} k^ and P = s (Q^ K^T) . e^{G'_i - G_j} on the mask, for
+// the state passes.
+__global__ void __launch_bounds__(kThreads)
+bwd_chunk_prep(BwdParams p) {
+    extern __shared__ float sm[];
+    if (p.hdr->err != GDR_OK) return;
+    ChunkPos cp;
+    if (!chunk_pos(p, cp)) return;
+    const int h = blockIdx.y, hk = h / (p.Hv / p.Hk);
+    const int dk = p.dk, C = p.chunk, ldk = dk + 1, Cc = cp.Cc;
+    const Tile tl;
+
+    float* Qs = sm;                     // [C][dk+1]
+    float* Ks = Qs + C * ldk;           // [C][dk+1]
+    float* Gs = Ks + C * ldk;           // [C]
+    float* Gr = Gs + C;                 // [C] G'
+    float* nr = Gr + C;                 // [C] norms (unused)
+
+    auto tok = [&](int i) { return phys_token(cp.t0, cp.t1, cp.p0 + i, p.reverse); };
+    load_rows(Qs, C, Cc, dk, ldk, [&](int i, int d) {
+        return load_elem(p.q, (size_t)(tok(i) * p.Hk + hk) * dk + d, p.io); });
+    load_rows(Ks, C, Cc, dk, ldk, [&](int i, int d) {
+        return load_elem(p.k, (size_t)(tok(i) * p.Hk + hk) * dk + d, p.io); });
+    for (int i = threadIdx.x; i < C; i += kThreads)
+        Gs[i] = i < Cc ? p.G[(size_t)tok(i) * p.Hv + h] : 0.f;
+    __syncthreads();
+    l2norm_rows_keep(Qs, nr, Cc, dk, ldk, p.qk_l2norm);
+    l2norm_rows_keep(Ks, nr, Cc, dk, ldk, p.qk_l2norm);
+    for (int i = threadIdx.x; i < C; i += kThreads)
+        Gr[i] = p.read_pre ? (i > 0 ? Gs[i - 1] : 0.f) : Gs[i];
+    __syncthreads();
+    const float GC = Gs[Cc - 1];
+    for (int idx = threadIdx.x; idx < Cc * dk; idx += kThreads) {
+        const int i = idx / dk, d = idx % dk;
+        const size_t o = (size_t)(tok(i) * p.Hv + h) * dk + d;
+        p.Qt[o] = p.scale * expf(Gr[i]) * Qs[i * ldk + d];
+        p.Kt[o] = expf(GC - Gs[i]) * Ks[i * ldk + d];
+    }
+    float S[4][4] = {};
+    for (int d = 0; d < dk; ++d) {
+        float a[4], b[4];
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) a[ii] = tl.row(ii) < C ? Qs[tl.row(ii) * ldk + d] : 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) b[jj] = tl.col(jj) < C ? Ks[tl.col(jj) * ldk + d] : 0.f;
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) S[ii][jj] = fmaf(a[ii], b[jj], S[ii][jj]);
+    }
+    float* Pout = p.Pc + ((size_t)cp.c * p.Hv + h) * C * C;
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const int i = tl.row(ii), j = tl.col(jj);
+            if (i >= C || j >= C) continue;
+            const bool m = i < Cc && j < Cc && (p.read_pre ? j < i : j <= i);
+            Pout[i * C + j] = m ? p.scale * S[ii][jj] * expf(Gr[i] - Gs[j]) : 0.f;
+        }
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -796,15 +906,19 @@ __global__ void bwd_reduce_heads(BwdParams p, long long n) {
 }
 
 size_t states_fwd_smem(const gdr_chunk_args& a) {
-    const int C = a.chunk, ldk = a.dk + 1;
-    return sizeof(float) * ((size_t)a.dk * kSlice + 2 * (size_t)C * ldk + (size_t)C * (kSlice + 1) +
-                            3 * (size_t)C);
+    const int C = a.chunk;
+    return sizeof(float) * ((size_t)a.dk * kSlice + 2 * (size_t)C * a.dk + (size_t)C * (kSlice + 1));
 }
 
 size_t states_bwd_smem(const gdr_chunk_args& a) {
-    const int C = a.chunk, ldk = a.dk + 1;
-    return sizeof(float) * ((size_t)a.dk * kSlice + 3 * (size_t)C * ldk +
-                            2 * (size_t)C * (kSlice + 1) + (size_t)C * (C + 1) + 4 * (size_t)C);
+    const int C = a.chunk;
+    return sizeof(float) * ((size_t)a.dk * kSlice + 3 * (size_t)C * a.dk + (size_t)C * C +
+                            2 * (size_t)C * (kSlice + 1));
+}
+
+size_t prep_smem(const gdr_chunk_args& a) {
+    const int C = a.chunk;
+    return sizeof(float) * (2 * (size_t)C * (a.dk + 1) + 3 * (size_t)C);
 }
 
 size_t dqk_smem(const gdr_chunk_args& a) {
@@ -821,6 +935,43 @@ size_t wy_smem(const gdr_chunk_args& a) {
 }
 
 constexpr size_t kMaxSmem = 227 * 1024;
+
+template <int RP, int DR>
+gdr_status launch_states_t(const gdr_chunk_args& a, const BwdParams& p, dim3 grid,
+                           cudaStream_t st) {
+    const size_t sf = states_fwd_smem(a), sb = states_bwd_smem(a);
+    if (cudaFuncSetAttribute(bwd_states_fwd<RP, DR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sf) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd_states_bwd<RP, DR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sb) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    bwd_states_fwd<RP, DR><<<grid, kThreads, sf, st>>>(p);
+    bwd_states_bwd<RP, DR><<<grid, kThreads, sb, st>>>(p);
+    return GDR_OK;
+}
+
+template <int RP>
+gdr_status launch_states_dk(const gdr_chunk_args& a, const BwdParams& p, dim3 grid,
+                            cudaStream_t st) {
+    switch (a.dk) {
+        case 32: return launch_states_t<RP, 4>(a, p, grid, st);
+        case 64: return launch_states_t<RP, 8>(a, p, grid, st);
+        case 96: return launch_states_t<RP, 12>(a, p, grid, st);
+        case 128: return launch_states_t<RP, 16>(a, p, grid, st);
+    }
+    return GDR_ERR_UNSUPPORTED;
+}
+
+// State passes for C rows per chunk (C/8 per warp) and dk state rows (dk/8 per warp).
+gdr_status launch_states(const gdr_chunk_args& a, const BwdParams& p, dim3 grid,
+                         cudaStream_t st) {
+    switch (a.chunk) {
+        case 16: return launch_states_dk<2>(a, p, grid, st);
+        case 32: return launch_states_dk<4>(a, p, grid, st);
+        case 64: return launch_states_dk<8>(a, p, grid, st);
+    }
+    return GDR_ERR_UNSUPPORTED;
+}
 
 }  // namespace
 
@@ -842,15 +993,18 @@ BwdLayout bwd_layout(const gdr_chunk_args& a) {
     B.dqh = off; off = align_up(off + tk, 256);
     B.dkh = off; off = align_up(off + tk, 256);
     B.dGp = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv, 256);
+    B.Pc = off;  off = align_up(off + sizeof(float) * (size_t)B.base.max_chunks * a.Hv * a.chunk * a.chunk, 256);
     B.total = off;
     return B;
 }
 
 bool bwd_supported(const gdr_chunk_args& a) {
     if (a.gate_raw || a.gdn2 || a.o_accumulate) return false;
-    if (a.chunk > 64 || a.dk > 128 || a.dv > 128 || a.dv % kSlice != 0) return false;
+    // the state passes split C rows and dk state rows over 8 warps, the latter in float4s
+    if (a.chunk > 64 || a.dk > 128 || a.dk % 32 != 0 || a.dv > 128 || a.dv % kSlice != 0)
+        return false;
     return states_fwd_smem(a) <= kMaxSmem && states_bwd_smem(a) <= kMaxSmem &&
-           dqk_smem(a) <= kMaxSmem && wy_smem(a) <= kMaxSmem;
+           prep_smem(a) <= kMaxSmem && dqk_smem(a) <= kMaxSmem && wy_smem(a) <= kMaxSmem;
 }
 
 gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
@@ -879,24 +1033,24 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
     p.dqh = reinterpret_cast<float*>(base + B.dqh);
     p.dkh = reinterpret_cast<float*>(base + B.dkh);
     p.dGp = reinterpret_cast<float*>(base + B.dGp);
+    p.Qt = p.dqh; p.Kt = p.dkh;
+    p.Pc = reinterpret_cast<float*>(base + B.Pc);
     p.Hk = a.Hk; p.Hv = a.Hv; p.dk = a.dk; p.dv = a.dv; p.chunk = a.chunk;
     p.read_pre = a.read_mode == GDR_READ_PRE; p.qk_l2norm = a.qk_l2norm; p.reverse = a.reverse;
     p.io = a.io_dtype; p.gt = a.gate_dtype; p.scale = a.scale;
 
     gdr_status s = launch_wy_local_simt(a, x.k, x.v, x.g, x.beta, ws, L, W, U, G, st);
     if (s != GDR_OK) return s;
-    const size_t sm_sf = states_fwd_smem(a), sm_sb = states_bwd_smem(a);
-    const size_t sm_q = dqk_smem(a), sm_w = wy_smem(a);
-    if (cudaFuncSetAttribute(bwd_states_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_sf) != cudaSuccess ||
-        cudaFuncSetAttribute(bwd_states_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_sb) != cudaSuccess ||
+    const size_t sm_p = prep_smem(a), sm_q = dqk_smem(a), sm_w = wy_smem(a);
+    if (cudaFuncSetAttribute(bwd_chunk_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_p) != cudaSuccess ||
         cudaFuncSetAttribute(bwd_chunk_dqk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_q) != cudaSuccess ||
         cudaFuncSetAttribute(bwd_chunk_wy, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_w) != cudaSuccess)
         return GDR_ERR_CUDA;
+    const dim3 gc((unsigned)L.max_chunks, (unsigned)a.Hv);
+    if (L.max_chunks > 0) bwd_chunk_prep<<<gc, kThreads, sm_p, st>>>(p);
     const dim3 gs((unsigned)a.n_seqs, (unsigned)a.Hv, (unsigned)(a.dv / kSlice));
-    bwd_states_fwd<<<gs, kThreads, sm_sf, st>>>(p);
-    bwd_states_bwd<<<gs, kThreads, sm_sb, st>>>(p);
+    if ((s = launch_states(a, p, gs, st)) != GDR_OK) return s;
     if (L.max_chunks > 0) {
-        const dim3 gc((unsigned)L.max_chunks, (unsigned)a.Hv);
         bwd_chunk_dqk<<<gc, kThreads, sm_q, st>>>(p);
         bwd_chunk_wy<<<gc, kThreads, sm_w, st>>>(p);
         const long long n = (long long)a.B * a.T * a.Hk * a.dk;

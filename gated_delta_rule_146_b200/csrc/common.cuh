@@ -125,7 +125,7 @@ gdr_status launch_wy_local_simt(const gdr_chunk_args& a, const void* k, const vo
 // Backward pass (chunk_bwd.cu).
 struct BwdLayout {
     WsLayout base;  // the forward's plan and CUDA-core arrays
-    size_t Hc, dHc, Vp, dVp, dW, dKp, dqh, dkh, dGp, total;
+    size_t Hc, dHc, Vp, dVp, dW, dKp, dqh, dkh, dGp, Pc, total;
 };
 struct BwdPtrs {
     const void *q, *k, *v, *g, *beta, *dO;
