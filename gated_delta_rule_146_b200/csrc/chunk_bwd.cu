@@ -25,7 +25,7 @@
 // Kernels, in order on the stream:
 //   plan_kernel            chunk map (shared with the forward)
 //   chunk_local_simt       W, U~, G per chunk (shared with the forward's CUDA-core path)
-//   bwd_chunk_prep         per (chunk, head): s e^{G'} q^, e^{G_C - G} k^ and P
+//   chunk_prep_simt        per (chunk, head): s e^{G'} q^, e^{G_C - G} k^ and P (shared too)
 //   bwd_states_fwd         per (sequence, head, 32-column slice): H at every chunk start, V'
 //   bwd_states_bwd         same grid, chunks in reverse: dH+ at every chunk, dV', dS0
 //   bwd_chunk_dqk          per (chunk, head): dq (normalised adjoint), the P and carry parts
@@ -54,9 +54,8 @@ struct BwdParams {
     float *Vp, *dVp;                // [T][Hv][dv]: V', dV'
     float *dW, *dKp, *dqh, *dkh;    // [T][Hv][dk]
     float* dGp;                     // [T][Hv]
-    float *Qt, *Kt;                 // [T][Hv][dk]: s e^{G'} q^, e^{G_C - G} k^ (state passes;
-                                    // they share the storage of dqh, dkh, written later)
-    float* Pc;                      // [max_chunks][Hv][C][C]: P, zero off the mask
+    const float *Qt, *Kt;           // [T][Hv][dk]: s e^{G'} q^, e^{G_C - G} k^ (chunk_prep_simt)
+    const float* Pc;                // [max_chunks][Hv][C][C]: P, zero off the mask
     int Hk, Hv, dk, dv, chunk, read_pre, qk_l2norm, reverse;
     gdr_dtype io, gt;
     float scale;
@@ -126,7 +125,7 @@ __device__ __forceinline__ bool chunk_pos(const BwdParams& p, ChunkPos& cp) {
 // the chunk's [C x 32] products (RP = C/8) and rows w*DR .. w*DR+DR-1 of the [dk x 32]
 // state (DR = dk/8), so each lane keeps RP or DR independent accumulators and reads the
 // row operands as float4 broadcasts.  K~ = e^{G_C - G} k^, Q~ = s e^{G'} q^ and P come from
-// bwd_chunk_prep, so the passes hold no normalisation or exponential.
+// chunk_prep_simt, so the passes hold no normalisation or exponential.
 
 __device__ __forceinline__ void load_rows4(float* dst, const float* src, size_t row_stride,
                                            int rows, int n, const BwdParams& p, long long t0,
@@ -336,68 +335,6 @@ __device__ void load_rows(float* dst, int C, int Cc, int n, int ld, F&& get) {
         const int i = idx / n, d = idx % n;
         dst[i * ld + d] = i < Cc ? get(i, d) : 0.f;
     }
-}
-
-// Q~ = s e^{G'} q^, K~ = e^{G_C - G} k^ and P = s (Q^ K^T) . e^{G'_i - G_j} on the mask, for
-// the state passes.
-__global__ void __launch_bounds__(kThreads)
-bwd_chunk_prep(BwdParams p) {
-    extern __shared__ float sm[];
-    if (p.hdr->err != GDR_OK) return;
-    ChunkPos cp;
-    if (!chunk_pos(p, cp)) return;
-    const int h = blockIdx.y, hk = h / (p.Hv / p.Hk);
-    const int dk = p.dk, C = p.chunk, ldk = dk + 1, Cc = cp.Cc;
-    const Tile tl;
-
-    float* Qs = sm;                     // [C][dk+1]
-    float* Ks = Qs + C * ldk;           // [C][dk+1]
-    float* Gs = Ks + C * ldk;           // [C]
-    float* Gr = Gs + C;                 // [C] G'
-    float* nr = Gr + C;                 // [C] norms (unused)
-
-    auto tok = [&](int i) { return phys_token(cp.t0, cp.t1, cp.p0 + i, p.reverse); };
-    load_rows(Qs, C, Cc, dk, ldk, [&](int i, int d) {
-        return load_elem(p.q, (size_t)(tok(i) * p.Hk + hk) * dk + d, p.io); });
-    load_rows(Ks, C, Cc, dk, ldk, [&](int i, int d) {
-        return load_elem(p.k, (size_t)(tok(i) * p.Hk + hk) * dk + d, p.io); });
-    for (int i = threadIdx.x; i < C; i += kThreads)
-        Gs[i] = i < Cc ? p.G[(size_t)tok(i) * p.Hv + h] : 0.f;
-    __syncthreads();
-    l2norm_rows_keep(Qs, nr, Cc, dk, ldk, p.qk_l2norm);
-    l2norm_rows_keep(Ks, nr, Cc, dk, ldk, p.qk_l2norm);
-    for (int i = threadIdx.x; i < C; i += kThreads)
-        Gr[i] = p.read_pre ? (i > 0 ? Gs[i - 1] : 0.f) : Gs[i];
-    __syncthreads();
-    const float GC = Gs[Cc - 1];
-    for (int idx = threadIdx.x; idx < Cc * dk; idx += kThreads) {
-        const int i = idx / dk, d = idx % dk;
-        const size_t o = (size_t)(tok(i) * p.Hv + h) * dk + d;
-        p.Qt[o] = p.scale * expf(Gr[i]) * Qs[i * ldk + d];
-        p.Kt[o] = expf(GC - Gs[i]) * Ks[i * ldk + d];
-    }
-    float S[4][4] = {};
-    for (int d = 0; d < dk; ++d) {
-        float a[4], b[4];
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii) a[ii] = tl.row(ii) < C ? Qs[tl.row(ii) * ldk + d] : 0.f;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) b[jj] = tl.col(jj) < C ? Ks[tl.col(jj) * ldk + d] : 0.f;
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) S[ii][jj] = fmaf(a[ii], b[jj], S[ii][jj]);
-    }
-    float* Pout = p.Pc + ((size_t)cp.c * p.Hv + h) * C * C;
-#pragma unroll
-    for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const int i = tl.row(ii), j = tl.col(jj);
-            if (i >= C || j >= C) continue;
-            const bool m = i < Cc && j < Cc && (p.read_pre ? j < i : j <= i);
-            Pout[i * C + j] = m ? p.scale * S[ii][jj] * expf(Gr[i] - Gs[j]) : 0.f;
-        }
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -916,11 +853,6 @@ size_t states_bwd_smem(const gdr_chunk_args& a) {
                             2 * (size_t)C * (kSlice + 1));
 }
 
-size_t prep_smem(const gdr_chunk_args& a) {
-    const int C = a.chunk;
-    return sizeof(float) * (2 * (size_t)C * (a.dk + 1) + 3 * (size_t)C);
-}
-
 size_t dqk_smem(const gdr_chunk_args& a) {
     const int C = a.chunk;
     return sizeof(float) * (2 * (size_t)C * (a.dk + 1) + 2 * (size_t)C * (a.dv + 1) +
@@ -993,7 +925,6 @@ BwdLayout bwd_layout(const gdr_chunk_args& a) {
     B.dqh = off; off = align_up(off + tk, 256);
     B.dkh = off; off = align_up(off + tk, 256);
     B.dGp = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv, 256);
-    B.Pc = off;  off = align_up(off + sizeof(float) * (size_t)B.base.max_chunks * a.Hv * a.chunk * a.chunk, 256);
     B.total = off;
     return B;
 }
@@ -1003,8 +934,8 @@ bool bwd_supported(const gdr_chunk_args& a) {
     // the state passes split C rows and dk state rows over 8 warps, the latter in float4s
     if (a.chunk > 64 || a.dk > 128 || a.dk % 32 != 0 || a.dv > 128 || a.dv % kSlice != 0)
         return false;
-    return states_fwd_smem(a) <= kMaxSmem && states_bwd_smem(a) <= kMaxSmem &&
-           prep_smem(a) <= kMaxSmem && dqk_smem(a) <= kMaxSmem && wy_smem(a) <= kMaxSmem;
+    return simt_supported(a) && simt_rb(a) && states_fwd_smem(a) <= kMaxSmem &&
+           states_bwd_smem(a) <= kMaxSmem && dqk_smem(a) <= kMaxSmem && wy_smem(a) <= kMaxSmem;
 }
 
 gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
@@ -1033,21 +964,21 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
     p.dqh = reinterpret_cast<float*>(base + B.dqh);
     p.dkh = reinterpret_cast<float*>(base + B.dkh);
     p.dGp = reinterpret_cast<float*>(base + B.dGp);
-    p.Qt = p.dqh; p.Kt = p.dkh;
-    p.Pc = reinterpret_cast<float*>(base + B.Pc);
+    p.Qt = reinterpret_cast<const float*>(base + L.Qt);
+    p.Kt = reinterpret_cast<const float*>(base + L.Kt);
+    p.Pc = reinterpret_cast<const float*>(base + L.Pc);
     p.Hk = a.Hk; p.Hv = a.Hv; p.dk = a.dk; p.dv = a.dv; p.chunk = a.chunk;
     p.read_pre = a.read_mode == GDR_READ_PRE; p.qk_l2norm = a.qk_l2norm; p.reverse = a.reverse;
     p.io = a.io_dtype; p.gt = a.gate_dtype; p.scale = a.scale;
 
     gdr_status s = launch_wy_local_simt(a, x.k, x.v, x.g, x.beta, ws, L, W, U, G, st);
+    if (s == GDR_OK) s = launch_prep_simt(a, x.q, x.k, ws, L, st);
     if (s != GDR_OK) return s;
-    const size_t sm_p = prep_smem(a), sm_q = dqk_smem(a), sm_w = wy_smem(a);
-    if (cudaFuncSetAttribute(bwd_chunk_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_p) != cudaSuccess ||
-        cudaFuncSetAttribute(bwd_chunk_dqk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_q) != cudaSuccess ||
+    const size_t sm_q = dqk_smem(a), sm_w = wy_smem(a);
+    if (cudaFuncSetAttribute(bwd_chunk_dqk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_q) != cudaSuccess ||
         cudaFuncSetAttribute(bwd_chunk_wy, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_w) != cudaSuccess)
         return GDR_ERR_CUDA;
     const dim3 gc((unsigned)L.max_chunks, (unsigned)a.Hv);
-    if (L.max_chunks > 0) bwd_chunk_prep<<<gc, kThreads, sm_p, st>>>(p);
     const dim3 gs((unsigned)a.n_seqs, (unsigned)a.Hv, (unsigned)(a.dv / kSlice));
     if ((s = launch_states(a, p, gs, st)) != GDR_OK) return s;
     if (L.max_chunks > 0) {

@@ -44,6 +44,7 @@ struct SimtParams {
     const float* gate_A; const float* gate_dt_bias;
     float beta_scale;
     const void* w;                // GDN-2 write gate [T][Hv][dv]; g, beta are then [T][Hv][dk]
+    float *Qt, *Kt, *Pc;          // register-blocked scan operands (chunk_prep_simt)
 };
 
 // Normalise `rows` rows of length n (row stride ld) in shared memory, one warp per row.
@@ -424,6 +425,307 @@ chunk_scan_simt_g2(SimtParams p) {
             p.S_final[sbase + (size_t)d * dv + col] = Hs[d * kSlice + lane];
 }
 
+// ---- register-blocked scan -----------------------------------------------------------
+//
+// chunk_prep_simt (one block per (chunk, value head), all chunks in parallel) forms, from the
+// normalised rows and the in-chunk log decays (per token, or per key channel for GDN-2),
+//     Q~_i = scale e^{G'_i} . q^_i,   K~_i = e^{G_C - G_i} . k^_i,
+//     P_ij = scale sum_d q^_id k^_jd e^{G'_id - G_jd}  on the causal mask (0 elsewhere),
+// so that the sequential scan is three dense fp32 products per chunk and column slice:
+//     V' = U~ - W H,   O = Q~ H + P V',   H <- e^{G_C} . H + K~^T V'.
+// In chunk_scan_rb lane l owns column l of the slice; warp w owns chunk rows w*RP ..
+// w*RP+RP-1 (RP = C/8) and state rows w*DR .. w*DR+DR-1 (DR = dk/8), with float4 broadcast
+// reads of the row operands and RP or DR independent accumulators per lane.
+
+template <bool kG2>
+__global__ void __launch_bounds__(kThreads)
+chunk_prep_simt(SimtParams p) {
+    extern __shared__ float sm[];
+    const WsHeader* hdr = p.hdr;
+    if (hdr->err != GDR_OK) return;
+    const int c = blockIdx.x, h = blockIdx.y;
+    if (c >= hdr->n_chunks) return;
+    const int s = p.chunk_seq[c];
+    const long long t0 = p.cu[s], t1 = p.cu[s + 1];
+    const int p0 = (c - p.chunk_off[s]) * p.chunk;
+    const int C = p.chunk, dk = p.dk, ldk = dk + 1;
+    const int Cc = (int)min((long long)C, (t1 - t0) - p0);
+    const int hk = h / (p.Hv / p.Hk);
+    const int tid = threadIdx.x, rg = tid >> 4, cg = tid & 15;
+    const int lg = kG2 ? ldk : 1;       // stride of a row of G: per channel or per token
+
+    float* Qs = sm;                     // [C][dk+1] q^
+    float* Ks = Qs + C * ldk;           // [C][dk+1] k^
+    float* Gs = Ks + C * ldk;           // [C][lg] G
+    float* Gr = Gs + C * lg;            // [C][lg] G' (read decay)
+
+    for (int idx = tid; idx < C * dk; idx += kThreads) {
+        const int i = idx / dk, d = idx % dk;
+        float qv = 0.f, kv = 0.f;
+        if (i < Cc) {
+            const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+            qv = load_elem(p.q, (size_t)(t * p.Hk + hk) * dk + d, p.io);
+            kv = load_elem(p.k, (size_t)(t * p.Hk + hk) * dk + d, p.io);
+        }
+        Qs[i * ldk + d] = qv;
+        Ks[i * ldk + d] = kv;
+    }
+    for (int idx = tid; idx < C * (kG2 ? dk : 1); idx += kThreads) {
+        const int i = kG2 ? idx / dk : idx, d = kG2 ? idx % dk : 0;
+        float gv = 0.f;
+        if (i < Cc) {
+            const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+            gv = kG2 ? p.G[(size_t)(t * p.Hv + h) * dk + d] : p.G[(size_t)t * p.Hv + h];
+        }
+        Gs[i * lg + d] = gv;
+    }
+    __syncthreads();
+    if (p.qk_l2norm) { l2norm_rows(Qs, Cc, dk, ldk); l2norm_rows(Ks, Cc, dk, ldk); }
+    for (int idx = tid; idx < C * (kG2 ? dk : 1); idx += kThreads) {
+        const int i = kG2 ? idx / dk : idx, d = kG2 ? idx % dk : 0;
+        Gr[i * lg + d] = p.read_pre ? (i > 0 ? Gs[(i - 1) * lg + d] : 0.f) : Gs[i * lg + d];
+    }
+    __syncthreads();
+    for (int idx = tid; idx < Cc * dk; idx += kThreads) {
+        const int i = idx / dk, d = idx % dk, e = kG2 ? d : 0;
+        const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+        const size_t o = (size_t)(t * p.Hv + h) * dk + d;
+        p.Qt[o] = p.scale * expf(Gr[i * lg + e]) * Qs[i * ldk + d];
+        p.Kt[o] = expf(Gs[(Cc - 1) * lg + e] - Gs[i * lg + e]) * Ks[i * ldk + d];
+    }
+    // P over this thread's rows 4 rg + ii and columns cg + 16 jj (C <= 64)
+    float acc[4][4] = {};
+    for (int d = 0; d < dk; ++d) {
+        float a[4], b[4];
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) a[ii] = 4 * rg + ii < C ? Qs[(4 * rg + ii) * ldk + d] : 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) b[jj] = cg + 16 * jj < C ? Ks[(cg + 16 * jj) * ldk + d] : 0.f;
+        if constexpr (kG2) {  // the decay differs per channel: one exp per (i, j, d)
+            float ga[4], gb[4];
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) ga[ii] = 4 * rg + ii < C ? Gr[(4 * rg + ii) * lg + d] : 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) gb[jj] = cg + 16 * jj < C ? Gs[(cg + 16 * jj) * lg + d] : 0.f;
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj)
+                    if (cg + 16 * jj <= 4 * rg + ii)  // past the mask the factor may overflow
+                        acc[ii][jj] = fmaf(a[ii] * b[jj], expf(ga[ii] - gb[jj]), acc[ii][jj]);
+        } else {
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) acc[ii][jj] = fmaf(a[ii], b[jj], acc[ii][jj]);
+        }
+    }
+    float* Pout = p.Pc + ((size_t)c * p.Hv + h) * C * C;
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const int i = 4 * rg + ii, j = cg + 16 * jj;
+            if (i >= C || j >= C) continue;
+            const bool m = i < Cc && j < Cc && (p.read_pre ? j < i : j <= i);
+            float v = 0.f;
+            if (m) v = kG2 ? p.scale * acc[ii][jj] : p.scale * acc[ii][jj] * expf(Gr[i] - Gs[j]);
+            Pout[i * C + j] = v;
+        }
+}
+
+// Rows [0, rows) of a token-major fp32 array [T][Hv][n] into shared rows of stride n.
+__device__ __forceinline__ void load_rows4(float* dst, const float* src, int rows, int n,
+                                           const SimtParams& p, long long t0, long long t1,
+                                           int p0, int h) {
+    const int n4 = n / 4;
+    for (int idx = threadIdx.x; idx < rows * n4; idx += kThreads) {
+        const int i = idx / n4, d4 = idx % n4;
+        const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+        reinterpret_cast<float4*>(dst + (size_t)i * n)[d4] =
+            reinterpret_cast<const float4*>(src + ((size_t)t * p.Hv + h) * n)[d4];
+    }
+}
+
+template <int RP, int DR, bool kG2>
+__global__ void __launch_bounds__(kThreads)
+chunk_scan_rb(SimtParams p) {
+    extern __shared__ __align__(16) float smr[];
+    if (p.hdr->err != GDR_OK) return;
+    const int s = blockIdx.x, h = blockIdx.y, J = blockIdx.z;
+    const int dk = p.dk, dv = p.dv, C = p.chunk;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int col = J * kSlice + lane;
+    const long long t0 = p.cu[s], t1 = p.cu[s + 1];
+    const int L = (int)(t1 - t0);
+
+    float* Hs = smr;                    // [dk][32] state slice
+    float* Kt = Hs + dk * kSlice;       // [C][dk] K~
+    float* Qt = Kt + C * dk;            // [C][dk] Q~
+    float* Ws = Qt + C * dk;            // [C][dk] W
+    float* Ps = Ws + C * dk;            // [C][C]  P
+    float* Us = Ps + C * C;             // [C][33] U~ then V'
+
+    const size_t sbase = ((size_t)s * p.Hv + h) * dk * dv;
+    for (int d = wid; d < dk; d += kThreads / 32)
+        Hs[d * kSlice + lane] = p.S0 ? p.S0[sbase + (size_t)d * dv + col] : 0.f;
+
+    for (int p0 = 0, jc = 0; p0 < L; p0 += C, ++jc) {
+        const int Cc = min(C, L - p0);
+        const int c = p.chunk_off[s] + jc;
+        __syncthreads();
+        load_rows4(Kt, p.Kt, Cc, dk, p, t0, t1, p0, h);
+        load_rows4(Qt, p.Qt, Cc, dk, p, t0, t1, p0, h);
+        load_rows4(Ws, p.W, Cc, dk, p, t0, t1, p0, h);
+        {
+            const float4* src = reinterpret_cast<const float4*>(p.Pc + ((size_t)c * p.Hv + h) * C * C);
+            for (int idx = tid; idx < C * C / 4; idx += kThreads)
+                reinterpret_cast<float4*>(Ps)[idx] = src[idx];
+        }
+        for (int i = wid; i < Cc; i += kThreads / 32) {
+            const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+            Us[i * (kSlice + 1) + lane] = p.U[(size_t)(t * p.Hv + h) * dv + col];
+        }
+        // the carry's decay of this warp's state rows: e^{G_C} (per channel for GDN-2)
+        float dc[DR];
+        {
+            const long long tl = phys_token(t0, t1, p0 + Cc - 1, p.reverse);
+#pragma unroll
+            for (int r = 0; r < DR; ++r)
+                dc[r] = expf(kG2 ? p.G[(size_t)(tl * p.Hv + h) * dk + wid * DR + r]
+                                 : p.G[(size_t)tl * p.Hv + h]);
+        }
+        __syncthreads();
+        // V' = U~ - W H
+        {
+            float acc[RP];
+#pragma unroll
+            for (int r = 0; r < RP; ++r) acc[r] = 0.f;
+            for (int d = 0; d < dk; d += 4) {
+                const float h0 = Hs[(d + 0) * kSlice + lane], h1 = Hs[(d + 1) * kSlice + lane];
+                const float h2 = Hs[(d + 2) * kSlice + lane], h3 = Hs[(d + 3) * kSlice + lane];
+#pragma unroll
+                for (int r = 0; r < RP; ++r) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(Ws + (wid * RP + r) * dk + d);
+                    acc[r] = fmaf(w4.x, h0, fmaf(w4.y, h1, fmaf(w4.z, h2, fmaf(w4.w, h3, acc[r]))));
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+                const int i = wid * RP + r;
+                if (i < Cc) Us[i * (kSlice + 1) + lane] -= acc[r];
+            }
+        }
+        __syncthreads();
+        // O = Q~ H + P V' and the new state, both from the old H
+        float hacc[DR];
+        {
+            float acc[RP];
+#pragma unroll
+            for (int r = 0; r < RP; ++r) acc[r] = 0.f;
+            for (int d = 0; d < dk; d += 4) {
+                const float h0 = Hs[(d + 0) * kSlice + lane], h1 = Hs[(d + 1) * kSlice + lane];
+                const float h2 = Hs[(d + 2) * kSlice + lane], h3 = Hs[(d + 3) * kSlice + lane];
+#pragma unroll
+                for (int r = 0; r < RP; ++r) {
+                    const float4 q4 = *reinterpret_cast<const float4*>(Qt + (wid * RP + r) * dk + d);
+                    acc[r] = fmaf(q4.x, h0, fmaf(q4.y, h1, fmaf(q4.z, h2, fmaf(q4.w, h3, acc[r]))));
+                }
+            }
+            for (int j = 0; j < Cc; ++j) {
+                const float a = Us[j * (kSlice + 1) + lane];
+#pragma unroll
+                for (int r = 0; r < RP; ++r) acc[r] = fmaf(Ps[(wid * RP + r) * C + j], a, acc[r]);
+            }
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+                const int i = wid * RP + r;
+                if (i < Cc) {
+                    const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+                    const size_t oi = (size_t)(t * p.Hv + h) * dv + col;
+                    float o = acc[r];
+                    if (p.o_acc) o += load_elem(p.o, oi, p.io);
+                    store_elem(p.o, oi, o, p.io);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < DR; ++r) hacc[r] = dc[r] * Hs[(wid * DR + r) * kSlice + lane];
+            for (int i = 0; i < Cc; ++i) {
+                const float v = Us[i * (kSlice + 1) + lane];
+#pragma unroll
+                for (int r = 0; r < DR; r += 4) {
+                    const float4 k4 = *reinterpret_cast<const float4*>(Kt + i * dk + wid * DR + r);
+                    hacc[r] = fmaf(k4.x, v, hacc[r]);
+                    hacc[r + 1] = fmaf(k4.y, v, hacc[r + 1]);
+                    hacc[r + 2] = fmaf(k4.z, v, hacc[r + 2]);
+                    hacc[r + 3] = fmaf(k4.w, v, hacc[r + 3]);
+                }
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < DR; ++r) Hs[(wid * DR + r) * kSlice + lane] = hacc[r];
+    }
+    __syncthreads();
+    if (p.S_final)
+        for (int d = wid; d < dk; d += kThreads / 32)
+            p.S_final[sbase + (size_t)d * dv + col] = Hs[d * kSlice + lane];
+}
+
+size_t prep_smem(const gdr_chunk_args& a) {
+    const size_t C = a.chunk, ldk = a.dk + 1;
+    return sizeof(float) * (2 * C * ldk + 2 * C * (a.gdn2 ? ldk : 1));
+}
+
+size_t scan_rb_smem(const gdr_chunk_args& a) {
+    const size_t C = a.chunk;
+    return sizeof(float) * ((size_t)a.dk * kSlice + 3 * C * a.dk + C * C + C * (kSlice + 1));
+}
+
+template <int RP, int DR>
+gdr_status launch_scan_rb_t(const gdr_chunk_args& a, const SimtParams& p, cudaStream_t st) {
+    auto kern = a.gdn2 ? chunk_scan_rb<RP, DR, true> : chunk_scan_rb<RP, DR, false>;
+    const size_t smem = scan_rb_smem(a);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return GDR_ERR_CUDA;
+    kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.Hv, (unsigned)(a.dv / kSlice)), kThreads, smem,
+           st>>>(p);
+    return GDR_OK;
+}
+
+template <int RP>
+gdr_status launch_scan_rb_dk(const gdr_chunk_args& a, const SimtParams& p, cudaStream_t st) {
+    switch (a.dk) {
+        case 32: return launch_scan_rb_t<RP, 4>(a, p, st);
+        case 64: return launch_scan_rb_t<RP, 8>(a, p, st);
+        case 96: return launch_scan_rb_t<RP, 12>(a, p, st);
+        case 128: return launch_scan_rb_t<RP, 16>(a, p, st);
+    }
+    return GDR_ERR_UNSUPPORTED;
+}
+
+gdr_status launch_scan_rb(const gdr_chunk_args& a, const SimtParams& p, cudaStream_t st) {
+    switch (a.chunk) {
+        case 16: return launch_scan_rb_dk<2>(a, p, st);
+        case 32: return launch_scan_rb_dk<4>(a, p, st);
+        case 64: return launch_scan_rb_dk<8>(a, p, st);
+    }
+    return GDR_ERR_UNSUPPORTED;
+}
+
+gdr_status launch_prep(const gdr_chunk_args& a, const SimtParams& p, const WsLayout& L,
+                       cudaStream_t st) {
+    if (L.max_chunks == 0) return GDR_OK;
+    auto kern = a.gdn2 ? chunk_prep_simt<true> : chunk_prep_simt<false>;
+    const size_t smem = prep_smem(a);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return GDR_ERR_CUDA;
+    kern<<<dim3((unsigned)L.max_chunks, (unsigned)a.Hv), kThreads, smem, st>>>(p);
+    return GDR_OK;
+}
+
 size_t local_smem(const gdr_chunk_args& a) {
     const int C = a.chunk;
     return sizeof(float) * ((size_t)C * (a.dk + a.dv + 1) + (size_t)C * (C + 1) +
@@ -443,6 +745,7 @@ constexpr size_t kMaxSmem = 227 * 1024;
 
 bool simt_supported(const gdr_chunk_args& a) {
     if (a.dv % kSlice != 0 || a.dk < 1 || a.dk > 256 || a.dv > 256) return false;
+    if (simt_rb(a) && (prep_smem(a) > kMaxSmem || scan_rb_smem(a) > kMaxSmem)) return false;
     return local_smem(a) <= kMaxSmem && scan_smem(a) <= kMaxSmem;
 }
 
@@ -466,6 +769,12 @@ gdr_status launch_chunk_simt(const gdr_chunk_args& a, const void* q, const void*
     p.gate_raw = a.gate_raw; p.gate_A = a.gate_A; p.gate_dt_bias = a.gate_dt_bias;
     p.beta_scale = a.beta_scale;
     p.w = a.gdn2_w;
+    const bool rb = simt_rb(a);
+    if (rb) {
+        p.Qt = reinterpret_cast<float*>(base + L.Qt);
+        p.Kt = reinterpret_cast<float*>(base + L.Kt);
+        p.Pc = reinterpret_cast<float*>(base + L.Pc);
+    }
 
     auto local = a.gdn2 ? chunk_local_simt_g2 : chunk_local_simt;
     auto scan = a.gdn2 ? chunk_scan_simt_g2 : chunk_scan_simt;
@@ -479,10 +788,38 @@ gdr_status launch_chunk_simt(const gdr_chunk_args& a, const void* q, const void*
         local<<<g1, kThreads, sm1, st>>>(p);
         if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
     }
+    if (rb) {
+        gdr_status s = launch_prep(a, p, L, st);
+        if (s == GDR_OK) s = launch_scan_rb(a, p, st);
+        if (s != GDR_OK) return s;
+        return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+    }
     dim3 g2((unsigned)a.n_seqs, (unsigned)a.Hv, (unsigned)(a.dv / kSlice));
     scan<<<g2, kThreads, sm2, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
     return GDR_OK;
+}
+
+gdr_status launch_prep_simt(const gdr_chunk_args& a, const void* q, const void* k, void* ws,
+                            const WsLayout& L, cudaStream_t st) {
+    if (a.gdn2 || !simt_rb(a)) return GDR_ERR_UNSUPPORTED;
+    char* base = static_cast<char*>(ws);
+    SimtParams p{};
+    p.q = q; p.k = k;
+    p.hdr = reinterpret_cast<const WsHeader*>(base);
+    p.cu = reinterpret_cast<const int32_t*>(base + L.cu);
+    p.chunk_off = reinterpret_cast<const int32_t*>(base + L.chunk_off);
+    p.chunk_seq = reinterpret_cast<const int32_t*>(base + L.chunk_seq);
+    p.G = reinterpret_cast<float*>(base + L.G);
+    p.Qt = reinterpret_cast<float*>(base + L.Qt);
+    p.Kt = reinterpret_cast<float*>(base + L.Kt);
+    p.Pc = reinterpret_cast<float*>(base + L.Pc);
+    p.Hk = a.Hk; p.Hv = a.Hv; p.dk = a.dk; p.dv = a.dv; p.chunk = a.chunk;
+    p.read_pre = a.read_mode == GDR_READ_PRE; p.qk_l2norm = a.qk_l2norm; p.reverse = a.reverse;
+    p.io = a.io_dtype; p.gt = a.gate_dtype; p.scale = a.scale;
+    const gdr_status s = launch_prep(a, p, L, st);
+    if (s != GDR_OK) return s;
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 
 gdr_status launch_wy_local_simt(const gdr_chunk_args& a, const void* k, const void* v,

@@ -58,8 +58,10 @@ __device__ __forceinline__ float warp_sum(float x) {
 // ---- workspace ----------------------------------------------------------------
 //
 // [header 256 B][cu (n_seqs+1) int32][chunk_off (n_seqs+1) int32][chunk_seq (max_chunks)
-// int32][fp32 W [T_tot][Hv][dk]][fp32 U [T_tot][Hv][dv]][fp32 G [T_tot][Hv]]
-// The three fp32 arrays exist only for the CUDA-core (SIMT) path.
+// int32][fp32 W [T_tot][Hv][dk]][fp32 U [T_tot][Hv][dv]][fp32 G [T_tot][Hv] (x dk for GDN-2)]
+// [fp32 Q~, K~ [T_tot][Hv][dk]][fp32 P [max_chunks][Hv][C][C]]
+// The fp32 arrays exist only for the CUDA-core (SIMT) path; Q~, K~, P only for its
+// register-blocked scan.
 
 struct WsHeader {
     int err;           // gdr_status recorded by a device-side check
@@ -68,9 +70,16 @@ struct WsHeader {
 };
 
 struct WsLayout {
-    size_t cu, chunk_off, chunk_seq, W, U, G, total;
+    size_t cu, chunk_off, chunk_seq, W, U, G, Qt, Kt, Pc, total;
     long long max_chunks;
 };
+
+// The register-blocked CUDA-core scan (chunk_scan_rb) splits a chunk's rows and the state's
+// dk rows over 8 warps, the latter in float4s: chunk <= 64, dk a multiple of 32 up to 128.
+// It reads the decayed, scaled Q~, K~ and P that chunk_prep_simt writes.
+inline bool simt_rb(const gdr_chunk_args& a) {
+    return a.chunk <= 64 && a.dk % 32 == 0 && a.dk <= 128 && a.dv % 32 == 0;
+}
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -88,6 +97,12 @@ inline WsLayout ws_layout(const gdr_chunk_args& a, bool simt) {
         // in-chunk log decay: one per token and head, or one per key channel for GDN-2
         L.G = off;
         off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv * (a.gdn2 ? a.dk : 1), 256);
+        if (simt_rb(a)) {  // operands of the register-blocked scan
+            L.Qt = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv * a.dk, 256);
+            L.Kt = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv * a.dk, 256);
+            L.Pc = off;
+            off = align_up(off + sizeof(float) * (size_t)L.max_chunks * a.Hv * a.chunk * a.chunk, 256);
+        }
     }
     L.total = off;
     return L;
@@ -122,10 +137,14 @@ gdr_status launch_wy_local_simt(const gdr_chunk_args& a, const void* k, const vo
                                 const void* g, const void* beta, void* ws, const WsLayout& L,
                                 float* W, float* U, float* G, cudaStream_t st);
 
+// Q~, K~ and P of every chunk (scalar gates) into the workspace arrays of ws_layout.
+gdr_status launch_prep_simt(const gdr_chunk_args& a, const void* q, const void* k, void* ws,
+                            const WsLayout& L, cudaStream_t st);
+
 // Backward pass (chunk_bwd.cu).
 struct BwdLayout {
     WsLayout base;  // the forward's plan and CUDA-core arrays
-    size_t Hc, dHc, Vp, dVp, dW, dKp, dqh, dkh, dGp, Pc, total;
+    size_t Hc, dHc, Vp, dVp, dW, dKp, dqh, dkh, dGp, total;
 };
 struct BwdPtrs {
     const void *q, *k, *v, *g, *beta, *dO;

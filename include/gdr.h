@@ -162,8 +162,9 @@ gdr_status gdr_chunk_fwd(const gdr_chunk_args* args,
  * - Calls whose scratch need (gdr_chunk_fwd_workspace_size) exceeds the array return
  *   GDR_ERR_WORKSPACE and enqueue nothing.  The tensor-core path needs only
  *   256 + 8 (n_seqs + 1) + 4 (ceil(B*T / chunk) + n_seqs) bytes; the CUDA-core path
- *   additionally 4 B*T Hv (dk + dv + 1) bytes (4 B*T Hv (2 dk + dv) with gdn2), so it fits
- *   only small problems.
+ *   additionally 4 B*T Hv (dk + dv + 1) bytes (4 B*T Hv (2 dk + dv) with gdn2), and for
+ *   chunk <= 64 with dk a multiple of 32 up to 128 another 8 B*T Hv dk +
+ *   4 (ceil(B*T / chunk) + n_seqs) Hv chunk^2 bytes, so it fits only small problems.
  * - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  *   with that device current; make that first call before any stream capture.
  * - All calls on a device share the one array: calls that overlap on the GPU (different
