@@ -271,18 +271,25 @@ chunk_local_simt_g2(SimtParams p) {
     const int dk = p.dk, dv = p.dv, ld = dk + dv + 1, C = p.chunk;
     const int hk = h / (p.Hv / p.Hk);
 
+    const int lg = dk + 1;               // padded rows: column reads hit distinct banks
     float* R = sm;                       // [C][ld]: K | V, then W | U~ in place
     float* A = R + C * ld;               // [C][C+1]
-    float* Gc = A + C * (C + 1);         // [C][dk] cumulative log decay per key channel
-    float* Bc = Gc + C * dk;             // [C][dk] erase gate
+    float* Gc = A + C * (C + 1);         // [C][dk+1] cumulative log decay per key channel
+    float* Bc = Gc + C * lg;             // [C][dk+1] erase gate
     const int tid = threadIdx.x;
 
-    for (int idx = tid; idx < Cc * dk; idx += kThreads) {
+    for (int idx = tid; idx < C * dk; idx += kThreads) {
         const int i = idx / dk, d = idx % dk;
-        const long long t = phys_token(t0, t1, p0 + i, p.reverse);
-        R[i * ld + d] = load_elem(p.k, (size_t)(t * p.Hk + hk) * dk + d, p.io);
-        Gc[i * dk + d] = load_elem(p.g, (size_t)(t * p.Hv + h) * dk + d, p.gt);
-        Bc[i * dk + d] = load_elem(p.beta, (size_t)(t * p.Hv + h) * dk + d, p.gt);
+        float kv = 0.f, gv = 0.f, bv = 0.f;
+        if (i < Cc) {
+            const long long t = phys_token(t0, t1, p0 + i, p.reverse);
+            kv = load_elem(p.k, (size_t)(t * p.Hk + hk) * dk + d, p.io);
+            gv = load_elem(p.g, (size_t)(t * p.Hv + h) * dk + d, p.gt);
+            bv = load_elem(p.beta, (size_t)(t * p.Hv + h) * dk + d, p.gt);
+        }
+        R[i * ld + d] = kv;
+        Gc[i * lg + d] = gv;
+        Bc[i * lg + d] = bv;
     }
     for (int idx = tid; idx < Cc * dv; idx += kThreads) {
         const int i = idx / dv, d = idx % dv;
@@ -294,22 +301,56 @@ chunk_local_simt_g2(SimtParams p) {
     if (p.qk_l2norm) l2norm_rows(R, Cc, dk, ld);
     for (int d = tid; d < dk; d += kThreads) {
         float run = 0.f;
-        for (int i = 0; i < Cc; ++i) { run += Gc[i * dk + d]; Gc[i * dk + d] = run; }
+        for (int i = 0; i < Cc; ++i) { run += Gc[i * lg + d]; Gc[i * lg + d] = run; }
     }
     __syncthreads();
-    for (int idx = tid; idx < Cc * Cc; idx += kThreads) {
-        const int i = idx / Cc, j = idx % Cc;
-        float val = 0.f;
-        if (j < i)
-            for (int d = 0; d < dk; ++d)
-                val = fmaf(Bc[i * dk + d] * R[i * ld + d] * R[j * ld + d],
-                           expf(Gc[i * dk + d] - Gc[j * dk + d]), val);
-        A[i * (C + 1) + j] = val;
+    // A over rows 4 rg + ii and columns cg + 16 jj of this thread (C <= 64; larger chunks
+    // take the rows in passes of 64)
+    {
+        const int rg = tid >> 4, cg = tid & 15;
+        for (int i0 = 0; i0 < C; i0 += 64)
+            for (int j0 = 0; j0 <= i0; j0 += 64) {
+                float acc[4][4] = {};
+                for (int d = 0; d < dk; ++d) {
+                    float a[4], b[4], ga[4], gb[4];
+#pragma unroll
+                    for (int ii = 0; ii < 4; ++ii) {
+                        const int i = i0 + 4 * rg + ii;
+                        a[ii] = i < C ? Bc[i * lg + d] * R[i * ld + d] : 0.f;
+                        ga[ii] = i < C ? Gc[i * lg + d] : 0.f;
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = j0 + cg + 16 * jj;
+                        b[jj] = j < C ? R[j * ld + d] : 0.f;
+                        gb[jj] = j < C ? Gc[j * lg + d] : 0.f;
+                    }
+#pragma unroll
+                    for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj)
+                            if (j0 + cg + 16 * jj < i0 + 4 * rg + ii)  // beyond the mask the
+                                acc[ii][jj] = fmaf(a[ii] * b[jj],   // factor may overflow
+                                                   expf(ga[ii] - gb[jj]), acc[ii][jj]);
+                }
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int i = i0 + 4 * rg + ii, j = j0 + cg + 16 * jj;
+                        if (i < C && j < C) A[i * (C + 1) + j] = (j < i && i < Cc) ? acc[ii][jj] : 0.f;
+                    }
+            }
+        // blocks above the diagonal (j0 > i0) of a 128-token chunk are zero
+        for (int idx = tid; idx < C * C; idx += kThreads) {
+            const int i = idx / C, j = idx % C;
+            if ((j / 64) > (i / 64)) A[i * (C + 1) + j] = 0.f;
+        }
     }
     __syncthreads();
     for (int idx = tid; idx < Cc * dk; idx += kThreads) {  // K rows -> e^{G} . b . k
         const int i = idx / dk, d = idx % dk;
-        R[i * ld + d] *= Bc[i * dk + d] * expf(Gc[i * dk + d]);
+        R[i * ld + d] *= Bc[i * lg + d] * expf(Gc[i * lg + d]);
     }
     __syncthreads();
     for (int col = tid; col < dk + dv; col += kThreads) {
@@ -324,7 +365,7 @@ chunk_local_simt_g2(SimtParams p) {
         const int i = idx / dk, d = idx % dk;
         const long long t = phys_token(t0, t1, p0 + i, p.reverse);
         p.W[(size_t)(t * p.Hv + h) * dk + d] = R[i * ld + d];
-        p.G[(size_t)(t * p.Hv + h) * dk + d] = Gc[i * dk + d];
+        p.G[(size_t)(t * p.Hv + h) * dk + d] = Gc[i * lg + d];
     }
     for (int idx = tid; idx < Cc * dv; idx += kThreads) {
         const int i = idx / dv, d = idx % dv;
@@ -729,7 +770,7 @@ gdr_status launch_prep(const gdr_chunk_args& a, const SimtParams& p, const WsLay
 size_t local_smem(const gdr_chunk_args& a) {
     const int C = a.chunk;
     return sizeof(float) * ((size_t)C * (a.dk + a.dv + 1) + (size_t)C * (C + 1) +
-                            (a.gdn2 ? 2 * (size_t)C * a.dk : 2 * (size_t)C));
+                            (a.gdn2 ? 2 * (size_t)C * (a.dk + 1) : 2 * (size_t)C));
 }
 
 size_t scan_smem(const gdr_chunk_args& a) {
