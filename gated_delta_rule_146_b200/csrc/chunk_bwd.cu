@@ -40,8 +40,9 @@ namespace gdr {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kSlice = 32;  // dv columns per state-pass block (one per lane)
+constexpr int kThreads = 256;  // state passes and the head reduction
+constexpr int kNT = 512;       // per-(chunk, head) kernels: 16 warps over 64 rows
+constexpr int kSlice = 32;     // dv columns per state-pass block (one per lane)
 
 struct BwdParams {
     const void *q, *k, *v, *g, *beta, *dO;
@@ -65,7 +66,7 @@ struct BwdParams {
 // record each row's norm |x| (needed by the adjoint).
 __device__ void l2norm_rows_keep(float* x, float* norms, int rows, int n, int ld, bool on) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    for (int i = wid; i < rows; i += kThreads / 32) {
+    for (int i = wid; i < rows; i += kNT / 32) {
         float ss = 0.f;
         for (int d = lane; d < n; d += 32) ss += x[i * ld + d] * x[i * ld + d];
         ss = warp_sum(ss);
@@ -78,13 +79,6 @@ __device__ void l2norm_rows_keep(float* x, float* norms, int rows, int n, int ld
     }
 }
 
-// Sum over the 16 lanes of a half-warp (the lanes that share a row group below).
-__device__ __forceinline__ float half_sum(float x) {
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
-}
-
 // Adjoint of x^ = x / max(|x|, eps) for one element, with proj = x^ . dx^ over the row.
 __device__ __forceinline__ float norm_adjoint(float dxh, float xh, float proj, float nrm,
                                               bool on) {
@@ -92,14 +86,15 @@ __device__ __forceinline__ float norm_adjoint(float dxh, float xh, float proj, f
     return nrm > kNormEps ? (dxh - xh * proj) / nrm : dxh / kNormEps;
 }
 
-// Register tiles of the per-chunk kernels: thread (rg = tid / 16, cg = tid % 16) owns rows
-// i = 4 rg + ii (ii < 4) and columns c = cg + 16 jj, so a half-warp reads 16 consecutive
-// columns of a row (no bank conflicts) and shares its rows (broadcast).
+// Register tiles of the per-chunk kernels (kNT threads): thread (rg = warp, cg = lane) owns
+// rows i = 4 rg + ii (ii < 4) and columns c = cg + 32 jj (jj < 2 for a [C x C] product,
+// jj < 4 for [C x dk]), so a warp reads 32 consecutive columns of a row (no bank
+// conflicts), shares its rows (broadcast) and reduces a row with warp shuffles.
 struct Tile {
     int rg, cg;
-    __device__ Tile() : rg(threadIdx.x >> 4), cg(threadIdx.x & 15) {}
+    __device__ Tile() : rg(threadIdx.x >> 5), cg(threadIdx.x & 31) {}
     __device__ int row(int ii) const { return 4 * rg + ii; }
-    __device__ int col(int jj) const { return cg + 16 * jj; }
+    __device__ int col(int jj) const { return cg + 32 * jj; }
 };
 
 struct ChunkPos {
@@ -331,13 +326,13 @@ bwd_states_bwd(BwdParams p) {
 // [Cc, C) so that products over the chunk need no bounds.
 template <typename F>
 __device__ void load_rows(float* dst, int C, int Cc, int n, int ld, F&& get) {
-    for (int idx = threadIdx.x; idx < C * n; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < C * n; idx += kNT) {
         const int i = idx / n, d = idx % n;
         dst[i * ld + d] = i < Cc ? get(i, d) : 0.f;
     }
 }
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kNT, 1)
 bwd_chunk_dqk(BwdParams p) {
     extern __shared__ float sm[];
     if (p.hdr->err != GDR_OK) return;
@@ -373,7 +368,7 @@ bwd_chunk_dqk(BwdParams p) {
         return load_elem(p.dO, (size_t)(tok(i) * p.Hv + h) * dv + e, p.io); });
     load_rows(Vps, C, Cc, dv, ldv, [&](int i, int e) {
         return p.Vp[(size_t)(tok(i) * p.Hv + h) * dv + e]; });
-    for (int i = threadIdx.x; i < C; i += kThreads) {
+    for (int i = threadIdx.x; i < C; i += kNT) {
         Gs[i] = i < Cc ? p.G[(size_t)tok(i) * p.Hv + h] : 0.f;
         dGr[i] = 0.f; dGs[i] = 0.f;
     }
@@ -381,42 +376,42 @@ bwd_chunk_dqk(BwdParams p) {
     __syncthreads();
     l2norm_rows_keep(Qs, qn, Cc, dk, ldk, on);
     l2norm_rows_keep(Ks, kn, Cc, dk, ldk, on);
-    for (int i = threadIdx.x; i < C; i += kThreads)
+    for (int i = threadIdx.x; i < C; i += kNT)
         Gr[i] = p.read_pre ? (i > 0 ? Gs[i - 1] : 0.f) : Gs[i];
     __syncthreads();
 
     // dP_ij = dO_i . V'_j and S_ij = q^_i . k^_j; D1 = s dP e^{G'_i - G_j} on the mask;
     // E = D1 S carries the decay gradient of the intra-chunk read.
     {
-        float dP[4][4] = {}, S[4][4] = {};
+        float dP[4][2] = {}, S[4][2] = {};
         for (int e = 0; e < dv; ++e) {
-            float a[4], b[4];
+            float a[4], b[2];
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii) a[ii] = tl.row(ii) < C ? dOs[tl.row(ii) * ldv + e] : 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) b[jj] = tl.col(jj) < C ? Vps[tl.col(jj) * ldv + e] : 0.f;
+            for (int jj = 0; jj < 2; ++jj) b[jj] = tl.col(jj) < C ? Vps[tl.col(jj) * ldv + e] : 0.f;
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) dP[ii][jj] = fmaf(a[ii], b[jj], dP[ii][jj]);
+                for (int jj = 0; jj < 2; ++jj) dP[ii][jj] = fmaf(a[ii], b[jj], dP[ii][jj]);
         }
         for (int d = 0; d < dk; ++d) {
-            float a[4], b[4];
+            float a[4], b[2];
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii) a[ii] = tl.row(ii) < C ? Qs[tl.row(ii) * ldk + d] : 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) b[jj] = tl.col(jj) < C ? Ks[tl.col(jj) * ldk + d] : 0.f;
+            for (int jj = 0; jj < 2; ++jj) b[jj] = tl.col(jj) < C ? Ks[tl.col(jj) * ldk + d] : 0.f;
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) S[ii][jj] = fmaf(a[ii], b[jj], S[ii][jj]);
+                for (int jj = 0; jj < 2; ++jj) S[ii][jj] = fmaf(a[ii], b[jj], S[ii][jj]);
         }
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii) {
             const int i = tl.row(ii);
             float rsum = 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < 2; ++jj) {
                 const int j = tl.col(jj);
                 const bool m = i < Cc && j < Cc && (p.read_pre ? j < i : j <= i);
                 const float d1 = m ? p.scale * dP[ii][jj] * expf(Gr[i] - Gs[j]) : 0.f;
@@ -425,7 +420,7 @@ bwd_chunk_dqk(BwdParams p) {
                 rsum += e;
                 if (m) atomicAdd(&dGs[j], -e);
             }
-            rsum = half_sum(rsum);
+            rsum = warp_sum(rsum);
             if (tl.cg == 0 && i < Cc) dGr[i] += rsum;
         }
     }
@@ -434,35 +429,35 @@ bwd_chunk_dqk(BwdParams p) {
     // Phase A: dQ^ = D1 K^ + s e^{G'} dO H^T; the inter read's decay gradient.
     const size_t cbase = ((size_t)cp.c * p.Hv + h) * dk * dv;
     {
-        float acc[4][8] = {}, X[4][8] = {};
+        float acc[4][4] = {}, X[4][4] = {};
         for (int j = 0; j < C; ++j) {
-            float a[4], b[8];
+            float a[4], b[4];
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii) a[ii] = tl.row(ii) < C ? D1[tl.row(ii) * ldc + j] : 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) b[jj] = tl.col(jj) < dk ? Ks[j * ldk + tl.col(jj)] : 0.f;
+            for (int jj = 0; jj < 4; ++jj) b[jj] = tl.col(jj) < dk ? Ks[j * ldk + tl.col(jj)] : 0.f;
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) acc[ii][jj] = fmaf(a[ii], b[jj], acc[ii][jj]);
+                for (int jj = 0; jj < 4; ++jj) acc[ii][jj] = fmaf(a[ii], b[jj], acc[ii][jj]);
         }
         for (int e0 = 0; e0 < dv; e0 += kSlice) {
             __syncthreads();
-            for (int idx = threadIdx.x; idx < dk * kSlice; idx += kThreads) {
+            for (int idx = threadIdx.x; idx < dk * kSlice; idx += kNT) {
                 const int d = idx / kSlice, e = idx % kSlice;
                 Tl[e * ldt + d] = p.Hc[cbase + (size_t)d * dv + e0 + e];
             }
             __syncthreads();
             for (int e = 0; e < kSlice; ++e) {
-                float a[4], b[8];
+                float a[4], b[4];
 #pragma unroll
                 for (int ii = 0; ii < 4; ++ii) a[ii] = tl.row(ii) < C ? dOs[tl.row(ii) * ldv + e0 + e] : 0.f;
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) b[jj] = tl.col(jj) < dk ? Tl[e * ldt + tl.col(jj)] : 0.f;
+                for (int jj = 0; jj < 4; ++jj) b[jj] = tl.col(jj) < dk ? Tl[e * ldt + tl.col(jj)] : 0.f;
 #pragma unroll
                 for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) X[ii][jj] = fmaf(a[ii], b[jj], X[ii][jj]);
+                    for (int jj = 0; jj < 4; ++jj) X[ii][jj] = fmaf(a[ii], b[jj], X[ii][jj]);
             }
         }
 #pragma unroll
@@ -472,7 +467,7 @@ bwd_chunk_dqk(BwdParams p) {
             const float rd = live ? p.scale * expf(Gr[i]) : 0.f;
             float gsum = 0.f, proj = 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
+            for (int jj = 0; jj < 4; ++jj) {
                 const int d = tl.col(jj);
                 if (d < dk && live) {
                     const float qh = Qs[i * ldk + d];
@@ -481,13 +476,13 @@ bwd_chunk_dqk(BwdParams p) {
                     proj = fmaf(qh, acc[ii][jj], proj);
                 }
             }
-            gsum = half_sum(gsum);
-            proj = half_sum(proj);
+            gsum = warp_sum(gsum);
+            proj = warp_sum(proj);
             if (tl.cg == 0 && live) dGr[i] += rd * gsum;
             if (live) {
                 const size_t base = (size_t)(tok(i) * p.Hv + h) * dk;
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
+                for (int jj = 0; jj < 4; ++jj) {
                     const int d = tl.col(jj);
                     if (d < dk)
                         p.dqh[base + d] = norm_adjoint(acc[ii][jj], Qs[i * ldk + d], proj, qn[i], on);
@@ -500,22 +495,22 @@ bwd_chunk_dqk(BwdParams p) {
     // gradient.
     const float GC = Gs[Cc - 1];
     {
-        float acc[4][8] = {}, Z[4][8] = {};
+        float acc[4][4] = {}, Z[4][4] = {};
         for (int j = 0; j < C; ++j) {
-            float a[4], b[8];
+            float a[4], b[4];
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii) a[ii] = tl.row(ii) < C ? D1[j * ldc + tl.row(ii)] : 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) b[jj] = tl.col(jj) < dk ? Qs[j * ldk + tl.col(jj)] : 0.f;
+            for (int jj = 0; jj < 4; ++jj) b[jj] = tl.col(jj) < dk ? Qs[j * ldk + tl.col(jj)] : 0.f;
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) acc[ii][jj] = fmaf(a[ii], b[jj], acc[ii][jj]);
+                for (int jj = 0; jj < 4; ++jj) acc[ii][jj] = fmaf(a[ii], b[jj], acc[ii][jj]);
         }
         float hdot = 0.f;
         for (int e0 = 0; e0 < dv; e0 += kSlice) {
             __syncthreads();
-            for (int idx = threadIdx.x; idx < dk * kSlice; idx += kThreads) {
+            for (int idx = threadIdx.x; idx < dk * kSlice; idx += kNT) {
                 const int d = idx / kSlice, e = idx % kSlice;
                 const size_t gi = cbase + (size_t)d * dv + e0 + e;
                 const float dh = p.dHc[gi];
@@ -524,15 +519,15 @@ bwd_chunk_dqk(BwdParams p) {
             }
             __syncthreads();
             for (int e = 0; e < kSlice; ++e) {
-                float a[4], b[8];
+                float a[4], b[4];
 #pragma unroll
                 for (int ii = 0; ii < 4; ++ii) a[ii] = tl.row(ii) < C ? Vps[tl.row(ii) * ldv + e0 + e] : 0.f;
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) b[jj] = tl.col(jj) < dk ? Tl[e * ldt + tl.col(jj)] : 0.f;
+                for (int jj = 0; jj < 4; ++jj) b[jj] = tl.col(jj) < dk ? Tl[e * ldt + tl.col(jj)] : 0.f;
 #pragma unroll
                 for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) Z[ii][jj] = fmaf(a[ii], b[jj], Z[ii][jj]);
+                    for (int jj = 0; jj < 4; ++jj) Z[ii][jj] = fmaf(a[ii], b[jj], Z[ii][jj]);
             }
         }
         hdot = warp_sum(hdot);
@@ -545,19 +540,19 @@ bwd_chunk_dqk(BwdParams p) {
             const float kd = live ? expf(GC - Gs[i]) : 0.f;
             float c = 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
+            for (int jj = 0; jj < 4; ++jj) {
                 const int d = tl.col(jj);
                 if (d < dk && live) {
                     c = fmaf(Ks[i * ldk + d], Z[ii][jj], c);
                     acc[ii][jj] = fmaf(kd, Z[ii][jj], acc[ii][jj]);
                 }
             }
-            c = half_sum(c) * kd;
+            c = warp_sum(c) * kd;
             if (tl.cg == 0 && live) { atomicAdd(&dGs[i], -c); csum += c; }
             if (live) {
                 const size_t base = (size_t)(tok(i) * p.Hv + h) * dk;
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
+                for (int jj = 0; jj < 4; ++jj) {
                     const int d = tl.col(jj);
                     if (d < dk) p.dKp[base + d] = acc[ii][jj];
                 }
@@ -568,29 +563,29 @@ bwd_chunk_dqk(BwdParams p) {
 
     // Phase C: dW = -dV' H^T.
     {
-        float acc[4][8] = {};
+        float acc[4][4] = {};
         for (int e0 = 0; e0 < dv; e0 += kSlice) {
             __syncthreads();
-            for (int idx = threadIdx.x; idx < dk * kSlice; idx += kThreads) {
+            for (int idx = threadIdx.x; idx < dk * kSlice; idx += kNT) {
                 const int d = idx / kSlice, e = idx % kSlice;
                 Tl[e * ldt + d] = p.Hc[cbase + (size_t)d * dv + e0 + e];
             }
-            for (int idx = threadIdx.x; idx < C * kSlice; idx += kThreads) {
+            for (int idx = threadIdx.x; idx < C * kSlice; idx += kNT) {
                 const int i = idx / kSlice, e = idx % kSlice;
                 dVt[i * (kSlice + 1) + e] =
                     i < Cc ? p.dVp[(size_t)(tok(i) * p.Hv + h) * dv + e0 + e] : 0.f;
             }
             __syncthreads();
             for (int e = 0; e < kSlice; ++e) {
-                float a[4], b[8];
+                float a[4], b[4];
 #pragma unroll
                 for (int ii = 0; ii < 4; ++ii) a[ii] = tl.row(ii) < C ? dVt[tl.row(ii) * (kSlice + 1) + e] : 0.f;
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) b[jj] = tl.col(jj) < dk ? Tl[e * ldt + tl.col(jj)] : 0.f;
+                for (int jj = 0; jj < 4; ++jj) b[jj] = tl.col(jj) < dk ? Tl[e * ldt + tl.col(jj)] : 0.f;
 #pragma unroll
                 for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) acc[ii][jj] = fmaf(a[ii], b[jj], acc[ii][jj]);
+                    for (int jj = 0; jj < 4; ++jj) acc[ii][jj] = fmaf(a[ii], b[jj], acc[ii][jj]);
             }
         }
 #pragma unroll
@@ -599,7 +594,7 @@ bwd_chunk_dqk(BwdParams p) {
             if (i >= Cc) continue;
             const size_t base = (size_t)(tok(i) * p.Hv + h) * dk;
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
+            for (int jj = 0; jj < 4; ++jj) {
                 const int d = tl.col(jj);
                 if (d < dk) p.dW[base + d] = -acc[ii][jj];
             }
@@ -615,10 +610,10 @@ bwd_chunk_dqk(BwdParams p) {
         }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < Cc; i += kThreads) p.dGp[(size_t)tok(i) * p.Hv + h] = dGs[i];
+    for (int i = threadIdx.x; i < Cc; i += kNT) p.dGp[(size_t)tok(i) * p.Hv + h] = dGs[i];
 }
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kNT, 1)
 bwd_chunk_wy(BwdParams p) {
     extern __shared__ float sm[];
     if (p.hdr->err != GDR_OK) return;
@@ -652,7 +647,7 @@ bwd_chunk_wy(BwdParams p) {
     load_rows(R, C, Cc, dk + dv, ldr, [&](int i, int x) {
         const size_t t = (size_t)tok(i) * p.Hv + h;
         return x < dk ? p.dW[t * dk + x] : p.dVp[t * dv + (x - dk)]; });
-    for (int i = threadIdx.x; i < C; i += kThreads) {
+    for (int i = threadIdx.x; i < C; i += kNT) {
         const bool live = i < Cc;
         Gs[i] = live ? p.G[(size_t)tok(i) * p.Hv + h] : 0.f;
         Bs[i] = live ? load_elem(p.beta, (size_t)tok(i) * p.Hv + h, p.gt) : 0.f;
@@ -664,22 +659,22 @@ bwd_chunk_wy(BwdParams p) {
     __syncthreads();
     // A_ij = beta_i (k^_i . k^_j) e^{G_i - G_j}, j < i
     {
-        float S[4][4] = {};
+        float S[4][2] = {};
         for (int d = 0; d < dk; ++d) {
-            float a[4], b[4];
+            float a[4], b[2];
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii) a[ii] = tl.row(ii) < C ? Ks[tl.row(ii) * ldk + d] : 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) b[jj] = tl.col(jj) < C ? Ks[tl.col(jj) * ldk + d] : 0.f;
+            for (int jj = 0; jj < 2; ++jj) b[jj] = tl.col(jj) < C ? Ks[tl.col(jj) * ldk + d] : 0.f;
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) S[ii][jj] = fmaf(a[ii], b[jj], S[ii][jj]);
+                for (int jj = 0; jj < 2; ++jj) S[ii][jj] = fmaf(a[ii], b[jj], S[ii][jj]);
         }
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < 2; ++jj) {
                 const int i = tl.row(ii), j = tl.col(jj);
                 if (i >= C || j >= C) continue;
                 const bool m = i < Cc && j < i;
@@ -689,7 +684,7 @@ bwd_chunk_wy(BwdParams p) {
     }
     __syncthreads();
     // [dR_w | dR_u] = (I + A)^-T [dW | dV']: x_i = r_i - sum_{j > i} A_ji x_j, from the last row
-    for (int x = threadIdx.x; x < dk + dv; x += kThreads) {
+    for (int x = threadIdx.x; x < dk + dv; x += kNT) {
         for (int i = Cc - 2; i >= 0; --i) {
             float r = R[i * ldr + x];
             for (int j = i + 1; j < Cc; ++j) r = fmaf(-A[j * ldc + i], R[j * ldr + x], r);
@@ -699,29 +694,29 @@ bwd_chunk_wy(BwdParams p) {
     __syncthreads();
     // dA_ij = -(dR_w,i . W_j + dR_u,i . U~_j) on j < i, and what it carries to beta, G, k^
     {
-        float dA[4][4] = {};
+        float dA[4][2] = {};
         for (int x = 0; x < dk + dv; ++x) {
-            float a[4], b[4];
+            float a[4], b[2];
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii) a[ii] = tl.row(ii) < C ? R[tl.row(ii) * ldr + x] : 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < 2; ++jj) {
                 const int j = tl.col(jj);
                 b[jj] = j < C ? (x < dk ? Ws[j * ldk + x] : Us[j * ldv + (x - dk)]) : 0.f;
             }
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) dA[ii][jj] = fmaf(-a[ii], b[jj], dA[ii][jj]);
+                for (int jj = 0; jj < 2; ++jj) dA[ii][jj] = fmaf(-a[ii], b[jj], dA[ii][jj]);
         }
         __syncthreads();  // every thread has read R, W, U~; Sk is rewritten below
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii) {
             const int i = tl.row(ii);
             float db = 0.f, dg = 0.f;
-            float sk[4], dd[4];
+            float sk[2], dd[2];
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < 2; ++jj) {
                 const int j = tl.col(jj);
                 const bool m = i < Cc && j < i;
                 sk[jj] = (i < C && j < C) ? Sk[i * ldc + j] : 0.f;
@@ -732,12 +727,12 @@ bwd_chunk_wy(BwdParams p) {
                 dg += ga;
                 if (m) atomicAdd(&dGs[j], -ga);
             }
-            db = half_sum(db);
-            dg = half_sum(dg);
+            db = warp_sum(db);
+            dg = warp_sum(dg);
             if (tl.cg == 0 && i < Cc) { atomicAdd(&dBs[i], db); atomicAdd(&dGs[i], dg); }
             const float bi = i < C ? Bs[i] : 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < 2; ++jj) {
                 const int j = tl.col(jj);
                 if (i < C && j < C) Sk[i * ldc + j] = bi * dd[jj];
             }
@@ -746,9 +741,9 @@ bwd_chunk_wy(BwdParams p) {
     __syncthreads();
     // dK^ = (beta D) K^ + (beta D)^T K^ + diag(beta e^G) dR_w + the P and carry parts
     {
-        float acc[4][8] = {};
+        float acc[4][4] = {};
         for (int j = 0; j < C; ++j) {
-            float a1[4], a2[4], b[8];
+            float a1[4], a2[4], b[4];
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii) {
                 const int i = tl.row(ii);
@@ -756,11 +751,11 @@ bwd_chunk_wy(BwdParams p) {
                 a2[ii] = i < C ? Sk[j * ldc + i] : 0.f;
             }
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) b[jj] = tl.col(jj) < dk ? Ks[j * ldk + tl.col(jj)] : 0.f;
+            for (int jj = 0; jj < 4; ++jj) b[jj] = tl.col(jj) < dk ? Ks[j * ldk + tl.col(jj)] : 0.f;
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) acc[ii][jj] = fmaf(a1[ii] + a2[ii], b[jj], acc[ii][jj]);
+                for (int jj = 0; jj < 4; ++jj) acc[ii][jj] = fmaf(a1[ii] + a2[ii], b[jj], acc[ii][jj]);
         }
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii) {
@@ -770,7 +765,7 @@ bwd_chunk_wy(BwdParams p) {
             const size_t base = live ? (size_t)(tok(i) * p.Hv + h) * dk : 0;
             float r = 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
+            for (int jj = 0; jj < 4; ++jj) {
                 const int d = tl.col(jj);
                 if (d < dk && live) {
                     const float rw = R[i * ldr + d];
@@ -778,18 +773,18 @@ bwd_chunk_wy(BwdParams p) {
                     acc[ii][jj] = fmaf(be, rw, acc[ii][jj]) + p.dKp[base + d];
                 }
             }
-            r = half_sum(r);
+            r = warp_sum(r);
             if (tl.cg == 0 && live) { atomicAdd(&dBs[i], eg * r); atomicAdd(&dGs[i], be * r); }
             float proj = 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
+            for (int jj = 0; jj < 4; ++jj) {
                 const int d = tl.col(jj);
                 if (d < dk && live) proj = fmaf(Ks[i * ldk + d], acc[ii][jj], proj);
             }
-            proj = half_sum(proj);
+            proj = warp_sum(proj);
             if (live) {
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
+                for (int jj = 0; jj < 4; ++jj) {
                     const int d = tl.col(jj);
                     if (d < dk)
                         p.dkh[base + d] = norm_adjoint(acc[ii][jj], Ks[i * ldk + d], proj, kn[i], on);
@@ -800,7 +795,7 @@ bwd_chunk_wy(BwdParams p) {
     // dv = beta dR_u; dbeta += v . dR_u (one warp per row)
     {
         const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-        for (int i = wid; i < Cc; i += kThreads / 32) {
+        for (int i = wid; i < Cc; i += kNT / 32) {
             const size_t base = (size_t)(tok(i) * p.Hv + h) * dv;
             float db = 0.f;
             for (int e = lane; e < dv; e += 32) {
@@ -982,8 +977,8 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
     const dim3 gs((unsigned)a.n_seqs, (unsigned)a.Hv, (unsigned)(a.dv / kSlice));
     if ((s = launch_states(a, p, gs, st)) != GDR_OK) return s;
     if (L.max_chunks > 0) {
-        bwd_chunk_dqk<<<gc, kThreads, sm_q, st>>>(p);
-        bwd_chunk_wy<<<gc, kThreads, sm_w, st>>>(p);
+        bwd_chunk_dqk<<<gc, kNT, sm_q, st>>>(p);
+        bwd_chunk_wy<<<gc, kNT, sm_w, st>>>(p);
         const long long n = (long long)a.B * a.T * a.Hk * a.dk;
         const unsigned blocks = (unsigned)std::min<long long>((n + kThreads - 1) / kThreads, 148LL * 16);
         if (n > 0) bwd_reduce_heads<<<blocks, kThreads, 0, st>>>(p, n);
