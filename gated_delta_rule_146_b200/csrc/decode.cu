@@ -77,11 +77,6 @@ decode_kernel(DecodeParams p) {
         hreg[m] = __ldcs(reinterpret_cast<const float4*>(Sblk + (size_t)d * DV));
     }
 
-    // the epilogue's gate z, fetched early so that its latency hides under the state loads
-    float zj = 0.f;
-    if constexpr (kNorm)
-        if (tid < DV) zj = load_elem(p.norm_z, (size_t)nh * DV + tid, p.io);
-
     // q, k (normalised), gates
     const size_t qk_base = ((size_t)n * p.Hk + hk) * DK;
     for (int d = tid; d < DK; d += kThreads) {
@@ -168,18 +163,6 @@ decode_kernel(DecodeParams p) {
         else store_elem(p.o, (size_t)nh * DV + col, oj, p.io);
     }
     __syncthreads();
-    // the state's write-back first: it needs only u, and the output epilogue below then
-    // overlaps the stores draining
-    const float4 u4 = *reinterpret_cast<const float4*>(&s_u[cg * 4]);
-#pragma unroll
-    for (int m = 0; m < NP; ++m) {
-        const int d = m * RPP + wid * RPW + rw;
-        float4 r;
-        const float a = kG2 ? s_eg[d] : alpha;  // the row's decay (re-read: fewer registers)
-        r.x = fmaf(a, hreg[m].x, kr[m] * u4.x); r.y = fmaf(a, hreg[m].y, kr[m] * u4.y);
-        r.z = fmaf(a, hreg[m].z, kr[m] * u4.z); r.w = fmaf(a, hreg[m].w, kr[m] * u4.w);
-        __stcs(reinterpret_cast<float4*>(Sblk + (size_t)d * DV), r);
-    }
     if constexpr (kNorm) {
         // gated RMSNorm over the head: o_j / sqrt(mean(o^2) + eps) * weight_j * silu(z_j)
         if (wid * 32 < DV) {
@@ -193,9 +176,20 @@ decode_kernel(DecodeParams p) {
 #pragma unroll
             for (int w = 0; w < (DV + 31) / 32; ++w) ss += s_ss[w];
             const float r = rsqrtf(ss / DV + p.norm_eps);
-            const float silu = zj / (1.f + expf(-zj));
+            const float z = load_elem(p.norm_z, (size_t)nh * DV + tid, p.io);
+            const float silu = z / (1.f + expf(-z));
             store_elem(p.o, (size_t)nh * DV + tid, s_o[tid] * r * p.norm_weight[tid] * silu, p.io);
         }
+    }
+    const float4 u4 = *reinterpret_cast<const float4*>(&s_u[cg * 4]);
+#pragma unroll
+    for (int m = 0; m < NP; ++m) {
+        const int d = m * RPP + wid * RPW + rw;
+        float4 r;
+        const float a = kG2 ? s_eg[d] : alpha;  // the row's decay (re-read: fewer registers)
+        r.x = fmaf(a, hreg[m].x, kr[m] * u4.x); r.y = fmaf(a, hreg[m].y, kr[m] * u4.y);
+        r.z = fmaf(a, hreg[m].z, kr[m] * u4.z); r.w = fmaf(a, hreg[m].w, kr[m] * u4.w);
+        __stcs(reinterpret_cast<float4*>(Sblk + (size_t)d * DV), r);
     }
 }
 
