@@ -45,6 +45,7 @@ struct SimtParams {
     float beta_scale;
     const void* w;                // GDN-2 write gate [T][Hv][dv]; g, beta are then [T][Hv][dk]
     float *Qt, *Kt, *Pc;          // register-blocked scan operands (chunk_prep_simt)
+    int g2_factor;                // GDN-2: factored off-diagonal blocks (see decayed_pairs)
 };
 
 // Normalise `rows` rows of length n (row stride ld) in shared memory, one warp per row.
@@ -246,6 +247,78 @@ chunk_scan_simt(SimtParams p) {
             p.S_final[sbase + (size_t)d * dv + col] = Hs[d * kSlice + lane];
 }
 
+// ---- decayed pair sums over key channels (GDN-2's A and P) ----------------------------
+//
+//     out_ij = sum_d X_id Y_jd e^{GX_id - GY_jd}   for j <= i,  a [C x C] tile, C <= 64,
+//
+// thread (rg = tid / 16, cg = tid % 16) owning rows 4 rg + ii and columns cg + 16 jj.  In
+// 16-row blocks the thread's rows lie in block I = rg / 4 (the same for both row groups of a
+// warp, so branches on it are warp-uniform) and column jj in block J = jj.
+//  - Diagonal blocks (J = I): one exp per term, only where j <= i (above, the factor may
+//    overflow).
+//  - Blocks below them (J < I), when `factor`: with the reference R_I = GY_{16 I - 1} (the
+//    decay just before row block I), e^{GX_i - GY_j} = e^{GX_i - R_I} e^{R_I - GY_j}.  While the
+//    decay never grows (every g <= 0), GX_i <= R_I <= GY_j, so both factors are <= 1 (no
+//    overflow; a factor that underflows belongs to a term that is smaller still), and the
+//    block is a plain product of rows scaled once: Xs (rows 16 .. C-1) and Ys (for each I,
+//    the rows j < 16 I, stacked from row 8 I (I - 1)).  Without `factor` these blocks take
+//    one exp per term as well.
+constexpr int kSub = 16;
+__host__ __device__ constexpr int ys_rows(int C) { return 8 * (C / kSub) * (C / kSub - 1); }
+
+struct PairOps {
+    const float *X, *Y, *GX, *GY;
+    int ldx, ldy, lgx, lgy;
+};
+
+__device__ void build_factored(float* Xs, float* Ys, int lds, const PairOps& o, int C, int dk) {
+    for (int idx = threadIdx.x; idx < (C - kSub) * dk; idx += kThreads) {
+        const int i = kSub + idx / dk, d = idx % dk, ref = kSub * (i / kSub) - 1;
+        Xs[(i - kSub) * lds + d] =
+            o.X[i * o.ldx + d] * expf(o.GX[i * o.lgx + d] - o.GY[ref * o.lgy + d]);
+    }
+    for (int I = 1; I < C / kSub; ++I)
+        for (int idx = threadIdx.x; idx < kSub * I * dk; idx += kThreads) {
+            const int j = idx / dk, d = idx % dk, ref = kSub * I - 1;
+            Ys[(8 * I * (I - 1) + j) * lds + d] =
+                o.Y[j * o.ldy + d] * expf(o.GY[ref * o.lgy + d] - o.GY[j * o.lgy + d]);
+        }
+}
+
+__device__ __forceinline__ void decayed_pairs(float (&acc)[4][4], const PairOps& o,
+                                              const float* Xs, const float* Ys, int lds,
+                                              bool factor, int C, int dk) {
+    const int rg = threadIdx.x >> 4, cg = threadIdx.x & 15, I = rg >> 2;
+    if (4 * rg >= C) return;
+    const bool fac = factor && I > 0;
+    const float* xs = Xs + (4 * rg - kSub) * lds;  // read only when fac
+    const float* ys = Ys + 8 * I * (I - 1) * lds;
+    for (int d = 0; d < dk; ++d) {
+        float a[4], ga[4], xa[4];
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) {
+            a[ii] = o.X[(4 * rg + ii) * o.ldx + d];
+            ga[ii] = o.GX[(4 * rg + ii) * o.lgx + d];
+            xa[ii] = fac ? xs[ii * lds + d] : 0.f;
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            if (jj > I) continue;
+            const int j = cg + 16 * jj;
+            if (fac && jj < I) {
+                const float b = ys[j * lds + d];
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) acc[ii][jj] = fmaf(xa[ii], b, acc[ii][jj]);
+            } else {
+                const float b = o.Y[j * o.ldy + d], gb = o.GY[j * o.lgy + d];
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii)
+                    if (j <= 4 * rg + ii) acc[ii][jj] = fmaf(a[ii] * b, expf(ga[ii] - gb), acc[ii][jj]);
+            }
+        }
+    }
+}
+
 // ---- GDN-2: decoupled per-channel gates ------------------------------------------
 // (tiny_gdn/fugue.py BidirectionalGatedDeltaNet2: S_t = (I - k_t (b_t . k_t)^T) Diag(e^{g_t})
 // S_{t-1} + k_t (w_t . v_t)^T.)  With G_t the per-key-channel cumulative log decay of the
@@ -275,9 +348,12 @@ chunk_local_simt_g2(SimtParams p) {
     float* R = sm;                       // [C][ld]: K | V, then W | U~ in place
     float* A = R + C * ld;               // [C][C+1]
     float* Gc = A + C * (C + 1);         // [C][dk+1] cumulative log decay per key channel
-    float* Bc = Gc + C * lg;             // [C][dk+1] erase gate
+    float* Bc = Gc + C * lg;             // [C][dk+1] erase gate, then b . k^
+    float* Xs = Bc + C * lg;             // [C-16][dk+1]  factored rows (g2_factor)
+    float* Ys = Xs + (C - kSub) * lg;    // [ys_rows(C)][dk+1]
     const int tid = threadIdx.x;
 
+    bool grows = false;                  // some g > 0: the factored blocks do not apply
     for (int idx = tid; idx < C * dk; idx += kThreads) {
         const int i = idx / dk, d = idx % dk;
         float kv = 0.f, gv = 0.f, bv = 0.f;
@@ -287,6 +363,7 @@ chunk_local_simt_g2(SimtParams p) {
             gv = load_elem(p.g, (size_t)(t * p.Hv + h) * dk + d, p.gt);
             bv = load_elem(p.beta, (size_t)(t * p.Hv + h) * dk + d, p.gt);
         }
+        grows |= gv > 0.f;
         R[i * ld + d] = kv;
         Gc[i * lg + d] = gv;
         Bc[i * lg + d] = bv;
@@ -297,15 +374,43 @@ chunk_local_simt_g2(SimtParams p) {
         const size_t e = (size_t)(t * p.Hv + h) * dv + d;
         R[i * ld + dk + d] = load_elem(p.v, e, p.io) * load_elem(p.w, e, p.gt);  // w . v
     }
-    __syncthreads();
+    const bool any_grows = __syncthreads_or(grows);  // also the barrier after the loads
+    const bool factor = p.g2_factor && !any_grows;
     if (p.qk_l2norm) l2norm_rows(R, Cc, dk, ld);
     for (int d = tid; d < dk; d += kThreads) {
         float run = 0.f;
         for (int i = 0; i < Cc; ++i) { run += Gc[i * lg + d]; Gc[i * lg + d] = run; }
     }
     __syncthreads();
-    // A over rows 4 rg + ii and columns cg + 16 jj of this thread (C <= 64; larger chunks
-    // take the rows in passes of 64)
+    if (C <= 64) {
+        // A_ij = sum_d (b . k^)_id k^_jd e^{G_id - G_jd}, j < i
+        for (int idx = tid; idx < C * dk; idx += kThreads) {
+            const int i = idx / dk, d = idx % dk;
+            Bc[i * lg + d] *= R[i * ld + d];
+        }
+        __syncthreads();
+        const PairOps ops{Bc, R, Gc, Gc, lg, ld, lg, lg};
+        if (factor) {
+            build_factored(Xs, Ys, lg, ops, C, dk);
+            __syncthreads();
+        }
+        float acc[4][4] = {};
+        decayed_pairs(acc, ops, Xs, Ys, lg, factor, C, dk);
+        const int rg = tid >> 4, cg = tid & 15;
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int i = 4 * rg + ii, j = cg + 16 * jj;
+                if (i < C && j < C) A[i * (C + 1) + j] = (j < i && i < Cc) ? acc[ii][jj] : 0.f;
+            }
+        __syncthreads();
+        for (int idx = tid; idx < Cc * dk; idx += kThreads) {  // K rows -> e^{G} . b . k
+            const int i = idx / dk, d = idx % dk;
+            R[i * ld + d] = Bc[i * lg + d] * expf(Gc[i * lg + d]);
+        }
+    } else {
+    // A over rows 4 rg + ii and columns cg + 16 jj of this thread, in passes of 64 rows
     {
         const int rg = tid >> 4, cg = tid & 15;
         for (int i0 = 0; i0 < C; i0 += 64)
@@ -351,6 +456,7 @@ chunk_local_simt_g2(SimtParams p) {
     for (int idx = tid; idx < Cc * dk; idx += kThreads) {  // K rows -> e^{G} . b . k
         const int i = idx / dk, d = idx % dk;
         R[i * ld + d] *= Bc[i * lg + d] * expf(Gc[i * lg + d]);
+    }
     }
     __syncthreads();
     for (int col = tid; col < dk + dv; col += kThreads) {
@@ -499,6 +605,8 @@ chunk_prep_simt(SimtParams p) {
     float* Ks = Qs + C * ldk;           // [C][dk+1] k^
     float* Gs = Ks + C * ldk;           // [C][lg] G
     float* Gr = Gs + C * lg;            // [C][lg] G' (read decay)
+    float* Xs = Gr + C * lg;            // GDN-2, g2_factor: [C-16][dk+1] factored rows
+    float* Ys = Xs + (C - kSub) * ldk;  //                    [ys_rows(C)][dk+1]
 
     for (int idx = tid; idx < C * dk; idx += kThreads) {
         const int i = idx / dk, d = idx % dk;
@@ -536,25 +644,27 @@ chunk_prep_simt(SimtParams p) {
     }
     // P over this thread's rows 4 rg + ii and columns cg + 16 jj (C <= 64)
     float acc[4][4] = {};
-    for (int d = 0; d < dk; ++d) {
-        float a[4], b[4];
+    if constexpr (kG2) {  // the decay differs per channel (decayed_pairs)
+        bool grows = false;  // the decay grows somewhere (some g > 0): no factored blocks
+        for (int idx = tid; idx < Cc * dk; idx += kThreads) {
+            const int i = idx / dk, d = idx % dk;
+            grows |= Gs[i * lg + d] > (i > 0 ? Gs[(i - 1) * lg + d] : 0.f);
+        }
+        const bool any_grows = __syncthreads_or(grows);
+        const bool factor = p.g2_factor && !any_grows;
+        const PairOps ops{Qs, Ks, Gr, Gs, ldk, ldk, lg, lg};
+        if (factor) {
+            build_factored(Xs, Ys, ldk, ops, C, dk);
+            __syncthreads();
+        }
+        decayed_pairs(acc, ops, Xs, Ys, ldk, factor, C, dk);
+    } else {
+        for (int d = 0; d < dk; ++d) {
+            float a[4], b[4];
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) a[ii] = 4 * rg + ii < C ? Qs[(4 * rg + ii) * ldk + d] : 0.f;
+            for (int ii = 0; ii < 4; ++ii) a[ii] = 4 * rg + ii < C ? Qs[(4 * rg + ii) * ldk + d] : 0.f;
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) b[jj] = cg + 16 * jj < C ? Ks[(cg + 16 * jj) * ldk + d] : 0.f;
-        if constexpr (kG2) {  // the decay differs per channel: one exp per (i, j, d)
-            float ga[4], gb[4];
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii) ga[ii] = 4 * rg + ii < C ? Gr[(4 * rg + ii) * lg + d] : 0.f;
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) gb[jj] = cg + 16 * jj < C ? Gs[(cg + 16 * jj) * lg + d] : 0.f;
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj)
-                    if (cg + 16 * jj <= 4 * rg + ii)  // past the mask the factor may overflow
-                        acc[ii][jj] = fmaf(a[ii] * b[jj], expf(ga[ii] - gb[jj]), acc[ii][jj]);
-        } else {
+            for (int jj = 0; jj < 4; ++jj) b[jj] = cg + 16 * jj < C ? Ks[(cg + 16 * jj) * ldk + d] : 0.f;
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
@@ -713,10 +823,36 @@ chunk_scan_rb(SimtParams p) {
             p.S_final[sbase + (size_t)d * dv + col] = Hs[d * kSlice + lane];
 }
 
-size_t prep_smem(const gdr_chunk_args& a) {
+constexpr size_t kMaxSmem = 227 * 1024;
+
+// GDN-2's factored blocks: rows of the Xs and Ys buffers, for 32 <= chunk <= 64
+size_t g2_factor_rows(const gdr_chunk_args& a) {
+    return (a.gdn2 && a.chunk >= 32 && a.chunk <= 64) ? (size_t)(a.chunk - kSub + ys_rows(a.chunk)) : 0;
+}
+
+size_t prep_smem_base(const gdr_chunk_args& a) {
     const size_t C = a.chunk, ldk = a.dk + 1;
     return sizeof(float) * (2 * C * ldk + 2 * C * (a.gdn2 ? ldk : 1));
 }
+
+size_t local_smem_base(const gdr_chunk_args& a) {
+    const int C = a.chunk;
+    return sizeof(float) * ((size_t)C * (a.dk + a.dv + 1) + (size_t)C * (C + 1) +
+                            (a.gdn2 ? 2 * (size_t)C * (a.dk + 1) : 2 * (size_t)C));
+}
+
+// whether the factored blocks' buffers fit next to both kernels' own
+bool g2_factor(const gdr_chunk_args& a) {
+    const size_t extra = sizeof(float) * g2_factor_rows(a) * (a.dk + 1);
+    return extra > 0 && local_smem_base(a) + extra <= kMaxSmem &&
+           (!simt_rb(a) || prep_smem_base(a) + extra <= kMaxSmem);
+}
+
+size_t g2_extra(const gdr_chunk_args& a) {
+    return g2_factor(a) ? sizeof(float) * g2_factor_rows(a) * (a.dk + 1) : 0;
+}
+
+size_t prep_smem(const gdr_chunk_args& a) { return prep_smem_base(a) + g2_extra(a); }
 
 size_t scan_rb_smem(const gdr_chunk_args& a) {
     const size_t C = a.chunk;
@@ -767,11 +903,7 @@ gdr_status launch_prep(const gdr_chunk_args& a, const SimtParams& p, const WsLay
     return GDR_OK;
 }
 
-size_t local_smem(const gdr_chunk_args& a) {
-    const int C = a.chunk;
-    return sizeof(float) * ((size_t)C * (a.dk + a.dv + 1) + (size_t)C * (C + 1) +
-                            (a.gdn2 ? 2 * (size_t)C * (a.dk + 1) : 2 * (size_t)C));
-}
+size_t local_smem(const gdr_chunk_args& a) { return local_smem_base(a) + g2_extra(a); }
 
 size_t scan_smem(const gdr_chunk_args& a) {
     const int C = a.chunk, ldk = a.dk + 1;
@@ -779,8 +911,6 @@ size_t scan_smem(const gdr_chunk_args& a) {
                             2 * (size_t)C * (kSlice + 1) + (size_t)C * (C + 1) +
                             (a.gdn2 ? (size_t)C * a.dk : 3 * (size_t)C));
 }
-
-constexpr size_t kMaxSmem = 227 * 1024;
 
 }  // namespace
 
@@ -810,6 +940,7 @@ gdr_status launch_chunk_simt(const gdr_chunk_args& a, const void* q, const void*
     p.gate_raw = a.gate_raw; p.gate_A = a.gate_A; p.gate_dt_bias = a.gate_dt_bias;
     p.beta_scale = a.beta_scale;
     p.w = a.gdn2_w;
+    p.g2_factor = g2_factor(a);
     const bool rb = simt_rb(a);
     if (rb) {
         p.Qt = reinterpret_cast<float*>(base + L.Qt);

@@ -90,3 +90,33 @@ def test_decode(dtype, read_mode, fused_norm):
         torch.cuda.synchronize()
         assert_close(f"o step {t}", o, o_ref, workloads.DTYPES[dtype])
     assert_close("S", S, S_ref, torch.float32 if dtype == "f32" else torch.bfloat16)
+
+
+@pytest.mark.parametrize("chunk", [16, 32])
+def test_chunk_sizes(chunk):
+    """Chunks of 32 (one factored block below the diagonal blocks) and 16 (diagonal only)."""
+    x = workloads.chunk_inputs(1, 150, 2, 2, 64, 64, "f32", s0_std=0.05, seed=73)
+    g, b, w = workloads.gdn2_gate_inputs(x["v"].shape[:3], 64, 64, "f32", seed=74)
+    o, S = run_chunk(x, g, b, w, chunk=chunk, scale=0.125)
+    o_r, S_r = oracle.gdn2_forward(x["q"], x["k"], x["v"], g, b, w, x["S0"], scale=0.125)
+    assert_close("o", o, o_r, torch.float32)
+    assert_close("S", S, S_r, torch.float32)
+
+
+def test_growing_and_strong_decays():
+    """Head 0: log decays of either sign (a chunk where the decay grows takes one exp per
+    term everywhere); head 1: strong decays (g ~ -2 per token, factors that underflow)."""
+    x = workloads.chunk_inputs(1, 130, 1, 2, 64, 64, "f32", s0_std=0.1, seed=75)
+    gen = torch.Generator("cpu").manual_seed(76)
+    shape = (1, 130, 2, 64)
+    g = torch.empty(shape)
+    g[:, :, 0] = torch.randn((1, 130, 64), generator=gen) * 0.05
+    g[:, :, 1] = -torch.nn.functional.softplus(torch.randn((1, 130, 64), generator=gen) + 2.0)
+    b = torch.sigmoid(torch.randn(shape, generator=gen))
+    w = torch.sigmoid(torch.randn((1, 130, 2, 64), generator=gen))
+    for mode in ("post", "pre"):
+        o, S = run_chunk(x, g, b, w, read_mode=mode, scale=0.125)
+        o_r, S_r = oracle.gdn2_forward(x["q"], x["k"], x["v"], g, b, w, x["S0"], read_mode=mode,
+                                       scale=0.125)
+        assert_close(f"o {mode}", o, o_r, torch.float32)
+        assert_close(f"S {mode}", S, S_r, torch.float32)
