@@ -19,7 +19,8 @@ import os
 from . import _abi
 from ._abi import GdrError, ChunkArgs, DecodeArgs, F32, BF16, READ_POST, READ_PRE  # noqa: F401
 
-__all__ = ["chunk_fwd", "chunk_bwd", "decode_step", "chunk_fwd_workspace_size",
+__all__ = ["chunk_fwd", "chunk_fwd_bidir", "chunk_bwd", "decode_step",
+           "chunk_fwd_workspace_size", "chunk_fwd_bidir_workspace_size",
            "chunk_bwd_workspace_size", "chunk_fwd_path",
            "read_device_error", "library", "GdrError"]
 
@@ -149,6 +150,42 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, *, chunk=64, read_mode
         ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
     _abi.check(st)
     return o, S_final
+
+
+def chunk_fwd_bidir(q, k, v, g_fwd, beta_fwd, g_bwd, beta_bwd, cu_seqlens=None, *, chunk=64,
+                    read_mode="pre", scale=None, qk_l2norm=True, o=None, workspace=None,
+                    stream=None, gate_A=None, gate_dt_bias=None, beta_scale=1.0, gdn2_w=None):
+    """Bidirectional forward (gdr_chunk_fwd_bidir): o = forward scan with (g_fwd, beta_fwd)
+    + reverse scan within each sequence with (g_bwd, beta_bwd), from zero states, in one
+    call.  Shapes as for ``chunk_fwd``.  Returns o."""
+    import torch
+    _check_cuda(q, k, v, g_fwd, beta_fwd, g_bwd, beta_bwd, cu_seqlens, o, workspace, gate_A,
+                gate_dt_bias, gdn2_w)
+    args = make_chunk_args(q, v, g_fwd, cu_seqlens, chunk, read_mode, scale, qk_l2norm, False,
+                           False, gate_A, gate_dt_bias, beta_scale, gdn2_w)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v share one dtype")
+    if len({t.dtype for t in (g_fwd, beta_fwd, g_bwd, beta_bwd)}) != 1:
+        raise TypeError("the gates of both directions share one dtype")
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    if o is None:
+        o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    need = int(_abi.lib().gdr_chunk_fwd_bidir_workspace_size(ctypes.byref(args)))
+    if need == 0:
+        raise GdrError(_abi.GDR_ERR_UNSUPPORTED, "no kernel path for these arguments")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = _abi.lib().gdr_chunk_fwd_bidir(
+        ctypes.byref(args), _ptr(q), _ptr(k), _ptr(v), _ptr(g_fwd), _ptr(beta_fwd), _ptr(g_bwd),
+        _ptr(beta_bwd), _ptr(cu_seqlens), _ptr(o), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
+    _abi.check(st)
+    return o
+
+
+def chunk_fwd_bidir_workspace_size(args: ChunkArgs) -> int:
+    return int(_abi.lib().gdr_chunk_fwd_bidir_workspace_size(ctypes.byref(args)))
 
 
 def chunk_bwd_workspace_size(args: ChunkArgs) -> int:

@@ -17,6 +17,7 @@ READ_POST, READ_PRE = 0, 1
 # every symbol include/gdr.h declares
 EXPORTS = ["gdr_chunk_fwd_workspace_size", "gdr_chunk_fwd", "gdr_chunk_fwd_noalloc",
            "gdr_chunk_bwd_workspace_size", "gdr_chunk_bwd",
+           "gdr_chunk_fwd_bidir_workspace_size", "gdr_chunk_fwd_bidir",
            "gdr_chunk_fwd_path",
            "gdr_decode_step", "gdr_status_string", "gdr_read_device_error", "gdr_version"]
 
@@ -63,6 +64,10 @@ def _declare(lib):
     lib.gdr_chunk_fwd.restype = ctypes.c_int
     lib.gdr_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(ChunkArgs)] + [vp] * 10
     lib.gdr_chunk_fwd_noalloc.restype = ctypes.c_int
+    lib.gdr_chunk_fwd_bidir_workspace_size.argtypes = [ctypes.POINTER(ChunkArgs)]
+    lib.gdr_chunk_fwd_bidir_workspace_size.restype = sz
+    lib.gdr_chunk_fwd_bidir.argtypes = [ctypes.POINTER(ChunkArgs)] + [vp] * 10 + [sz, vp]
+    lib.gdr_chunk_fwd_bidir.restype = ctypes.c_int
     lib.gdr_chunk_bwd_workspace_size.argtypes = [ctypes.POINTER(ChunkArgs)]
     lib.gdr_chunk_bwd_workspace_size.restype = sz
     lib.gdr_chunk_bwd.argtypes = [ctypes.POINTER(ChunkArgs)] + [vp] * 16 + [sz, vp]

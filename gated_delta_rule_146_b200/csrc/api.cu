@@ -10,9 +10,12 @@
 
 namespace gdr {
 bool tc_supported(const gdr_chunk_args& a);
+// `dependent`: launched as the programmatic dependent of the stream's previous grid
 gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k, const void* v,
                            const void* g, const void* beta, const float* S0, void* o,
-                           float* S_final, void* ws, const WsLayout& L, cudaStream_t st);
+                           float* S_final, void* ws, const WsLayout& L, cudaStream_t st,
+                           bool dependent = false);
+gdr_status launch_add_bf16(void* o, const void* x, long long n, cudaStream_t st);
 }  // namespace gdr
 
 using namespace gdr;
@@ -120,6 +123,75 @@ gdr_status gdr_chunk_fwd(const gdr_chunk_args* a, const void* q, const void* k, 
     if (path == Path::Tc)
         return launch_chunk_tc(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s);
     return launch_chunk_simt(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s);
+}
+
+// Bidirectional forward: the plan, then the two scans; on the tensor-core path the reverse
+// scan is the forward scan's programmatic dependent (it fills the SMs the first grid leaves
+// free) and writes a scratch output that one more kernel adds into o.
+namespace {
+size_t bidir_scratch_offset(const gdr_chunk_args& a, Path path) {
+    return align_up(ws_layout(a, path == Path::Simt).total, 256);
+}
+size_t bidir_workspace(const gdr_chunk_args& a, Path path) {
+    const size_t base = bidir_scratch_offset(a, path);
+    if (path != Path::Tc) return base;
+    return align_up(base + (size_t)2 * a.B * a.T * a.Hv * a.dv, 256);
+}
+}  // namespace
+
+size_t gdr_chunk_fwd_bidir_workspace_size(const gdr_chunk_args* a) {
+    if (check_chunk_args(a) != GDR_OK || a->reverse || a->o_accumulate) return 0;
+    const Path path = choose_path(*a);
+    if (path == Path::None) return 0;
+    return bidir_workspace(*a, path);
+}
+
+gdr_status gdr_chunk_fwd_bidir(const gdr_chunk_args* a, const void* q, const void* k,
+                               const void* v, const void* g_fwd, const void* beta_fwd,
+                               const void* g_bwd, const void* beta_bwd,
+                               const int32_t* cu_seqlens, void* o, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    gdr_status st = check_chunk_args(a);
+    if (st != GDR_OK) return st;
+    if (a->reverse || a->o_accumulate) return GDR_ERR_INVALID_ARG;
+    if (cu_seqlens) {
+        if (a->B != 1) return GDR_ERR_INVALID_ARG;
+    } else if (a->n_seqs != a->B) {
+        return GDR_ERR_INVALID_ARG;
+    }
+    const bool has_tokens = (long long)a->B * a->T > 0;
+    if (has_tokens && (!q || !k || !v || !g_fwd || !beta_fwd || !g_bwd || !beta_bwd || !o))
+        return GDR_ERR_INVALID_ARG;
+    if ((st = check_gating(a, true)) != GDR_OK) return st;
+    if (!workspace) return GDR_ERR_WORKSPACE;
+    const void* ptrs[] = {q, k, v, g_fwd, beta_fwd, g_bwd, beta_bwd, cu_seqlens, o, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDR_ERR_ALIGNMENT;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return GDR_ERR_ALIGNMENT;
+    const Path path = choose_path(*a);
+    if (path == Path::None) return GDR_ERR_UNSUPPORTED;
+    if (workspace_bytes < bidir_workspace(*a, path)) return GDR_ERR_WORKSPACE;
+    const WsLayout L = ws_layout(*a, path == Path::Simt);
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (launch_plan(*a, cu_seqlens, workspace, L, s) != cudaSuccess) return GDR_ERR_CUDA;
+    gdr_chunk_args rev = *a;
+    rev.reverse = 1;
+    if (path == Path::Tc) {
+        void* scratch = static_cast<char*>(workspace) + bidir_scratch_offset(*a, path);
+        if ((st = launch_chunk_tc(*a, q, k, v, g_fwd, beta_fwd, nullptr, o, nullptr, workspace,
+                                  L, s)) != GDR_OK)
+            return st;
+        if ((st = launch_chunk_tc(rev, q, k, v, g_bwd, beta_bwd, nullptr, scratch, nullptr,
+                                  workspace, L, s, /*dependent=*/true)) != GDR_OK)
+            return st;
+        return launch_add_bf16(o, scratch, (long long)a->B * a->T * a->Hv * a->dv, s);
+    }
+    if ((st = launch_chunk_simt(*a, q, k, v, g_fwd, beta_fwd, nullptr, o, nullptr, workspace, L,
+                                s)) != GDR_OK)
+        return st;
+    rev.o_accumulate = 1;  // the CUDA-core scan adds the reverse direction into o itself
+    return launch_chunk_simt(rev, q, k, v, g_bwd, beta_bwd, nullptr, o, nullptr, workspace, L, s);
 }
 
 size_t gdr_chunk_bwd_workspace_size(const gdr_chunk_args* a) {

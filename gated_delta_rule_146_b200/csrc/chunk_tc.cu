@@ -51,9 +51,11 @@
 // in place by the next chunk's total decay, so the next state update accumulates onto it.
 #include <cuda.h>
 
+#include <algorithm>
 #include <cstring>
 
 #include "common.cuh"
+
 #include "tc_ptx.cuh"
 
 namespace gdr {
@@ -190,7 +192,11 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wg = tid >> 7;     // 0: chain, 1-2: prep
     const int lt = tid & 127;    // index within the warpgroup = TMEM lane
-    if (p.hdr->err != GDR_OK) return;
+    // a grid launched after this one as its dependent (the reverse direction of a
+    // bidirectional call) may start on the SMs this grid leaves free; every CTA waits for the
+    // grid it depends on before it exits, so a later ordinary launch sees both grids' results
+    griddep_launch_dependents();
+    if (p.hdr->err != GDR_OK) { griddep_wait(); return; }
 
     const int s = blockIdx.x, h = blockIdx.y;
     // the gates as the recurrence uses them (fused gating prologue when kRaw)
@@ -216,6 +222,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
         if (p.S_final)
             for (int e = tid; e < kDh * kDh; e += kThreads)
                 p.S_final[sb + e] = p.S0 ? p.S0[sb + e] : 0.f;
+        griddep_wait();
         return;
     }
 
@@ -1006,6 +1013,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     if (__syncthreads_or(rbad ? 1 : 0) && tid == 0)
         atomicCAS(&p.hdr->err, (int)GDR_OK, (int)GDR_ERR_RANGE);
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+    griddep_wait();
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -1050,9 +1058,36 @@ bool tc_supported(const gdr_chunk_args& a) {
            !a.gdn2;
 }
 
+// sum of two bf16 arrays of n8 groups of 8, rounded once: o += x
+__global__ void add_bf16_kernel(__nv_bfloat16* o, const __nv_bfloat16* x, long long n8) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
+         i += (long long)gridDim.x * blockDim.x) {
+        uint4 a = reinterpret_cast<uint4*>(o)[i];
+        const uint4 b = reinterpret_cast<const uint4*>(x)[i];
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+        uint32_t ow[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 u = unpack_bf16x2(aw[e]), w = unpack_bf16x2(bw[e]);
+            ow[e] = pack_bf16x2(u.x + w.x, u.y + w.y);
+        }
+        reinterpret_cast<uint4*>(o)[i] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+    }
+}
+
+gdr_status launch_add_bf16(void* o, const void* x, long long n, cudaStream_t st) {
+    const long long n8 = n / 8;
+    if (n8 == 0) return GDR_OK;
+    const unsigned blocks = (unsigned)std::min<long long>((n8 + 255) / 256, 148LL * 8);
+    add_bf16_kernel<<<blocks, 256, 0, st>>>(static_cast<__nv_bfloat16*>(o),
+                                            static_cast<const __nv_bfloat16*>(x), n8);
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
 gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k, const void* v,
                            const void* g, const void* beta, const float* S0, void* o,
-                           float* S_final, void* ws, const WsLayout& L, cudaStream_t st) {
+                           float* S_final, void* ws, const WsLayout& L, cudaStream_t st,
+                           bool dependent) {
     char* base = static_cast<char*>(ws);
     TcParams p;
     p.q = static_cast<const __nv_bfloat16*>(q);
@@ -1088,7 +1123,22 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
                              (int)SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
     dim3 grid((unsigned)a.n_seqs, (unsigned)a.Hv);
-    kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p, tq, tk, tv, to, gp);
+    if (dependent) {  // may start while the stream's previous grid finishes (see the kernel)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kernel, p, tq, tk, tv, to, gp) != cudaSuccess)
+            return GDR_ERR_CUDA;
+    } else {
+        kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p, tq, tk, tv, to, gp);
+    }
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

@@ -254,6 +254,15 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int
                  ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(src), "r"(x), "r"(y), "r"(z)
                  : "memory");
 }
+// Programmatic dependent launch.  launch_dependents lets the stream's next grid, when it was
+// launched with programmatic stream serialisation, start its CTAs once every CTA of this grid
+// has issued it (or exited); wait blocks until the grid this one was launched after has
+// completed with its memory visible.  Both do nothing for grids launched the ordinary way.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

@@ -186,6 +186,34 @@ gdr_status gdr_chunk_fwd_noalloc(const gdr_chunk_args* args,
 const char* gdr_chunk_fwd_path(const gdr_chunk_args* args);
 
 /*
+ * Bidirectional forward (Rondo-Exp tiny_gdn/fugue.py, the bidirectional token mixer): one
+ * forward scan with (g_fwd, beta_fwd) and one scan over each sequence's tokens in reverse
+ * order with (g_bwd, beta_bwd), both from a zero state with the same q, k, v, read mode and
+ * scale, their outputs summed into o:  o = o_fwd + o_bwd  (o_bwd at each token's own
+ * position).  No state is returned.
+ *
+ *   args        as for gdr_chunk_fwd, with reverse = 0 and o_accumulate = 0
+ *   g_*, beta_* [B, T, Hv] gate_dtype, or the raw projections with gate_raw (both
+ *               directions share gate_A, gate_dt_bias, beta_scale); GDN-2 layouts with gdn2
+ *               (both directions share gdn2_w)
+ *   o           [B, T, Hv, dv] io_dtype; with bf16 on the tensor-core path each direction's
+ *               output is rounded to bf16 and the sum rounded once more, as two gdr_chunk_fwd
+ *               calls (the second with reverse and o_accumulate) give
+ *   workspace   at least gdr_chunk_fwd_bidir_workspace_size(args) bytes, 256-byte aligned
+ *
+ * On the tensor-core path the reverse scan's CTAs start while the forward scan's last CTAs
+ * run (programmatic dependent launch) and write a scratch output in the workspace, which a
+ * final kernel adds into o.  Errors: as gdr_chunk_fwd.
+ */
+size_t gdr_chunk_fwd_bidir_workspace_size(const gdr_chunk_args* args);
+gdr_status gdr_chunk_fwd_bidir(const gdr_chunk_args* args,
+                               const void* q, const void* k, const void* v,
+                               const void* g_fwd, const void* beta_fwd,
+                               const void* g_bwd, const void* beta_bwd,
+                               const int32_t* cu_seqlens, void* o,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Backward pass of gdr_chunk_fwd: the gradients of
  *     L = <dO, o> + <dS_final, S_final>
  * with respect to q, k, v, g, beta and S0, for the same arguments (Prizma "seq/delta.py",

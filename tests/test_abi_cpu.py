@@ -215,3 +215,26 @@ def test_backward_host_validation(lib):
     assert bwd(args(dk=128, dv=128, chunk=128)) == _abi.GDR_ERR_UNSUPPORTED
     assert bwd(a, ws=None) == _abi.GDR_ERR_WORKSPACE
     assert bwd(a, wsb=need - 1) == _abi.GDR_ERR_WORKSPACE
+
+
+def test_bidirectional_host_validation(lib):
+    """gdr_chunk_fwd_bidir: the reverse and accumulate flags are its own; pointers checked."""
+    a = args(dk=128, dv=128)
+    need = lib.gdr_chunk_fwd_bidir_workspace_size(ctypes.byref(a))
+    assert need > lib.gdr_chunk_fwd_workspace_size(ctypes.byref(a))  # scratch output (tc)
+    assert lib.gdr_chunk_fwd_bidir_workspace_size(ctypes.byref(args(reverse=1))) == 0
+    assert lib.gdr_chunk_fwd_bidir_workspace_size(ctypes.byref(args(o_accumulate=1))) == 0
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def bidir(a, wsb=need, **kw):
+        p = dict(q=FAKE, k=FAKE, v=FAKE, gf=FAKE, bf=FAKE, gb=FAKE, bb=FAKE, cu=None, o=FAKE,
+                 ws=FAKE)
+        p.update(kw)
+        return lib.gdr_chunk_fwd_bidir(ctypes.byref(a), *[vp(p[n]) for n in (
+            "q", "k", "v", "gf", "bf", "gb", "bb", "cu", "o", "ws")], ctypes.c_size_t(wsb), None)
+
+    assert bidir(args(dk=128, dv=128, reverse=1)) == _abi.GDR_ERR_INVALID_ARG
+    assert bidir(a, gb=None) == _abi.GDR_ERR_INVALID_ARG
+    assert bidir(a, bb=FAKE + 2) == _abi.GDR_ERR_ALIGNMENT
+    assert bidir(a, wsb=need - 1) == _abi.GDR_ERR_WORKSPACE
+    assert bidir(a, ws=None) == _abi.GDR_ERR_WORKSPACE
