@@ -690,11 +690,13 @@ __device__ __forceinline__ void load_rows4(float* dst, const float* src, int row
                                            const SimtParams& p, long long t0, long long t1,
                                            int p0, int h) {
     const int n4 = n / 4;
+    // read-only global loads: they may all be issued before the shared stores
+#pragma unroll 4
     for (int idx = threadIdx.x; idx < rows * n4; idx += kThreads) {
         const int i = idx / n4, d4 = idx % n4;
         const long long t = phys_token(t0, t1, p0 + i, p.reverse);
         reinterpret_cast<float4*>(dst + (size_t)i * n)[d4] =
-            reinterpret_cast<const float4*>(src + ((size_t)t * p.Hv + h) * n)[d4];
+            __ldg(reinterpret_cast<const float4*>(src + ((size_t)t * p.Hv + h) * n) + d4);
     }
 }
 
@@ -730,8 +732,9 @@ chunk_scan_rb(SimtParams p) {
         load_rows4(Ws, p.W, Cc, dk, p, t0, t1, p0, h);
         {
             const float4* src = reinterpret_cast<const float4*>(p.Pc + ((size_t)c * p.Hv + h) * C * C);
+#pragma unroll 4
             for (int idx = tid; idx < C * C / 4; idx += kThreads)
-                reinterpret_cast<float4*>(Ps)[idx] = src[idx];
+                reinterpret_cast<float4*>(Ps)[idx] = __ldg(src + idx);
         }
         for (int i = wid; i < Cc; i += kThreads / 32) {
             const long long t = phys_token(t0, t1, p0 + i, p.reverse);
