@@ -238,3 +238,23 @@ def test_bidirectional_host_validation(lib):
     assert bidir(a, bb=FAKE + 2) == _abi.GDR_ERR_ALIGNMENT
     assert bidir(a, wsb=need - 1) == _abi.GDR_ERR_WORKSPACE
     assert bidir(a, ws=None) == _abi.GDR_ERR_WORKSPACE
+
+
+def test_binding_refuses_host_tensors(lib):
+    """Every entry point of the binding refuses CPU tensors before reaching the library:
+    there is no CPU path to fall back on."""
+    import torch
+    import gated_delta_rule_146_b200 as gdr
+    q = torch.zeros((1, 8, 1, 64), dtype=torch.bfloat16)
+    v = torch.zeros((1, 8, 1, 64), dtype=torch.bfloat16)
+    g = torch.zeros((1, 8, 1), dtype=torch.bfloat16)
+    calls = [
+        lambda: gdr.chunk_fwd(q, q, v, g, g),
+        lambda: gdr.chunk_fwd_bidir(q, q, v, g, g, g, g),
+        lambda: gdr.chunk_bwd(q, q, v, g, g, v),
+        lambda: gdr.decode_step(q[:, 0], q[:, 0], v[:, 0], g[:, 0], g[:, 0],
+                                torch.zeros((1, 1, 64, 64))),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA tensors only"):
+            call()
