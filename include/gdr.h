@@ -29,7 +29,10 @@
  * - Inconsistencies only visible on the device (a cu_seqlens array that is not
  *   non-decreasing, does not start at 0 or does not end at T) are recorded in
  *   an error word inside the workspace; the kernels then skip the work.  Read
- *   it with gdr_read_device_error.  No kernel traps or waits without a bound.
+ *   it with gdr_read_device_error.  No kernel traps or waits without a bound
+ *   (the one wait not on a timer: in gdr_chunk_fwd_bidir the reverse scan's CTAs
+ *   wait, before they exit, for the forward scan's grid to complete, and every
+ *   CTA of that grid is already running and bounds its own waits).
  */
 #ifndef GDR_H
 #define GDR_H
