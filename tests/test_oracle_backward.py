@@ -35,6 +35,8 @@ def fd_grads(x, up, cu, h=1e-6, **kw):
     out = {}
     for name in ("q", "k", "v", "g", "beta", "S0"):
         base = x[name]
+        if base is None:
+            continue
         grad = np.zeros_like(base)
         for idx in np.ndindex(base.shape):
             keep = base[idx]
@@ -142,3 +144,29 @@ def test_checkpoint_invariance():
     b = oracle_grads(x, up, cu, scale=0.5, ckpt=3)
     for n in a:
         np.testing.assert_array_equal(a[n], b[n])
+
+
+def test_finite_differences_random_shapes():
+    """Random small shapes and options (key/value head counts, head sizes, varlen or batched,
+    both read modes, reversal, normalisation on or off, a state or none): every gradient
+    entry against central differences of the forward oracle."""
+    hyp = pytest.importorskip("hypothesis")
+    st = hyp.strategies
+
+    @hyp.settings(max_examples=12, deadline=None, derandomize=True)
+    @hyp.given(hk=st.integers(1, 2), group=st.integers(1, 2), dk=st.integers(1, 3),
+               dv=st.integers(1, 3), lens=st.lists(st.integers(0, 4), min_size=1, max_size=3),
+               varlen=st.booleans(), pre=st.booleans(), rev=st.booleans(), l2=st.booleans(),
+               s0=st.booleans(), scale=st.floats(0.25, 2.0))
+    def check(hk, group, dk, dv, lens, varlen, pre, rev, l2, s0, scale):
+        if varlen:
+            x, up, cu = problem(1, 0, hk, hk * group, dk, dv, lengths=lens, s0=s0)
+        else:
+            x, up, cu = problem(len(lens), max(lens), hk, hk * group, dk, dv, s0=s0)
+        kw = dict(read_mode="pre" if pre else "post", reverse=rev, qk_l2norm=l2, scale=scale)
+        got = oracle_grads(x, up, cu, **kw)
+        want = fd_grads(x, up, cu, **kw)
+        for name, ref in want.items():
+            np.testing.assert_allclose(got[name], ref, rtol=1e-5, atol=1e-6, err_msg=name)
+
+    check()
