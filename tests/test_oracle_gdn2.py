@@ -93,3 +93,30 @@ def test_product_of_transitions_without_writes():
         M = (np.eye(dk) - np.outer(kt, b[0, t, 0] * kt)) @ np.diag(np.exp(g[0, t, 0])) @ M
         assert np.allclose(o[0, t, 0], q[0, t, 0] @ M, rtol=1e-11, atol=1e-12)
     assert np.allclose(S[0, 0], M, rtol=1e-11, atol=1e-12)
+
+
+def test_matches_chunked_form_random_shapes():
+    """Random shapes, chunk sizes and read modes: the per-token GDN-2 oracle against the
+    independent chunked form."""
+    hyp = pytest.importorskip("hypothesis")
+    st = hyp.strategies
+
+    @hyp.settings(max_examples=20, deadline=None, derandomize=True)
+    @hyp.given(B=st.integers(1, 2), T=st.integers(1, 40), H=st.integers(1, 2),
+               dk=st.integers(1, 6), dv=st.integers(1, 5), chunk=st.sampled_from([1, 3, 8, 16]),
+               pre=st.booleans(), s0=st.booleans(), seed=st.integers(0, 1000))
+    def check(B, T, H, dk, dv, chunk, pre, s0, seed):
+        r = np.random.default_rng(seed)
+        q, k = r.normal(size=(B, T, H, dk)), r.normal(size=(B, T, H, dk))
+        v = r.normal(size=(B, T, H, dv))
+        g = -np.log1p(np.exp(r.normal(-2, 1, (B, T, H, dk))))
+        b = 1 / (1 + np.exp(-r.normal(0, 1, (B, T, H, dk))))
+        w = 1 / (1 + np.exp(-r.normal(0, 1, (B, T, H, dv))))
+        S0 = 0.3 * r.normal(size=(B, H, dk, dv)) if s0 else None
+        mode = "pre" if pre else "post"
+        o1, S1 = oracle.gdn2_forward(q, k, v, g, b, w, S0, read_mode=mode, scale=0.7)
+        o2, S2 = gdn2_chunked.forward(q, k, v, g, b, w, S0, chunk=chunk, read_mode=mode,
+                                      scale=0.7)
+        assert np.abs(o1 - o2).max() < 1e-11 and np.abs(S1 - S2).max() < 1e-11
+
+    check()
