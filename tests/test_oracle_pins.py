@@ -293,3 +293,36 @@ def test_decode_steps_equal_forward():
         ot, St = oracle.decode_step(q[:, t], k[:, t], v[:, t], g[:, t], beta[:, t], St)
         assert np.abs(ot - o[:, t]).max() < 1e-13
     assert np.abs(St - S).max() < 1e-13
+
+
+def test_matches_wy_form_random_shapes():
+    """Random shapes, GQA groups, chunk sizes, varlen layouts, read modes and reversal: the
+    per-token C oracle against the NumPy WY/UT chunk form."""
+    hyp = pytest.importorskip("hypothesis")
+    st = hyp.strategies
+
+    @hyp.settings(max_examples=25, deadline=None, derandomize=True)
+    @hyp.given(hk=st.integers(1, 3), group=st.integers(1, 3), dk=st.integers(1, 9),
+               dv=st.integers(1, 7), lens=st.lists(st.integers(0, 50), min_size=1, max_size=4),
+               varlen=st.booleans(), chunk=st.sampled_from([1, 2, 5, 16, 64]),
+               pre=st.booleans(), rev=st.booleans(), l2=st.booleans(), seed=st.integers(0, 999))
+    def check(hk, group, dk, dv, lens, varlen, chunk, pre, rev, l2, seed):
+        r = np.random.default_rng(seed)
+        Hv = hk * group
+        if varlen:
+            B, T = 1, sum(lens)
+            cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+            n = len(lens)
+        else:
+            B, T, cu, n = len(lens), max(lens), None, len(lens)
+        q, k = r.normal(size=(B, T, hk, dk)), r.normal(size=(B, T, hk, dk))
+        v = r.normal(size=(B, T, Hv, dv))
+        g = -np.log1p(np.exp(r.normal(-2, 1, (B, T, Hv))))
+        beta = 1 / (1 + np.exp(-r.normal(size=(B, T, Hv))))
+        S0 = 0.3 * r.normal(size=(n, Hv, dk, dv))
+        kw = dict(read_mode="pre" if pre else "post", scale=0.7, qk_l2norm=l2, reverse=rev)
+        o, S = oracle.forward(q, k, v, g, beta, S0, cu, **kw)
+        o2, S2 = wy_reference.chunked_forward(q, k, v, g, beta, S0, cu, chunk=chunk, **kw)
+        assert np.abs(o - o2).max(initial=0.0) < 1e-9 and np.abs(S - S2).max(initial=0.0) < 1e-9
+
+    check()
