@@ -382,8 +382,7 @@ chunk_local_simt_g2(SimtParams p) {
         for (int i = 0; i < Cc; ++i) { run += Gc[i * lg + d]; Gc[i * lg + d] = run; }
     }
     __syncthreads();
-    if (C <= 64) {
-        // A_ij = sum_d (b . k^)_id k^_jd e^{G_id - G_jd}, j < i
+    {   // A_ij = sum_d (b . k^)_id k^_jd e^{G_id - G_jd}, j < i (chunk <= 64)
         for (int idx = tid; idx < C * dk; idx += kThreads) {
             const int i = idx / dk, d = idx % dk;
             Bc[i * lg + d] *= R[i * ld + d];
@@ -409,54 +408,6 @@ chunk_local_simt_g2(SimtParams p) {
             const int i = idx / dk, d = idx % dk;
             R[i * ld + d] = Bc[i * lg + d] * expf(Gc[i * lg + d]);
         }
-    } else {
-    // A over rows 4 rg + ii and columns cg + 16 jj of this thread, in passes of 64 rows
-    {
-        const int rg = tid >> 4, cg = tid & 15;
-        for (int i0 = 0; i0 < C; i0 += 64)
-            for (int j0 = 0; j0 <= i0; j0 += 64) {
-                float acc[4][4] = {};
-                for (int d = 0; d < dk; ++d) {
-                    float a[4], b[4], ga[4], gb[4];
-#pragma unroll
-                    for (int ii = 0; ii < 4; ++ii) {
-                        const int i = i0 + 4 * rg + ii;
-                        a[ii] = i < C ? Bc[i * lg + d] * R[i * ld + d] : 0.f;
-                        ga[ii] = i < C ? Gc[i * lg + d] : 0.f;
-                    }
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const int j = j0 + cg + 16 * jj;
-                        b[jj] = j < C ? R[j * ld + d] : 0.f;
-                        gb[jj] = j < C ? Gc[j * lg + d] : 0.f;
-                    }
-#pragma unroll
-                    for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj)
-                            if (j0 + cg + 16 * jj < i0 + 4 * rg + ii)  // beyond the mask the
-                                acc[ii][jj] = fmaf(a[ii] * b[jj],   // factor may overflow
-                                                   expf(ga[ii] - gb[jj]), acc[ii][jj]);
-                }
-#pragma unroll
-                for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const int i = i0 + 4 * rg + ii, j = j0 + cg + 16 * jj;
-                        if (i < C && j < C) A[i * (C + 1) + j] = (j < i && i < Cc) ? acc[ii][jj] : 0.f;
-                    }
-            }
-        // blocks above the diagonal (j0 > i0) of a 128-token chunk are zero
-        for (int idx = tid; idx < C * C; idx += kThreads) {
-            const int i = idx / C, j = idx % C;
-            if ((j / 64) > (i / 64)) A[i * (C + 1) + j] = 0.f;
-        }
-    }
-    __syncthreads();
-    for (int idx = tid; idx < Cc * dk; idx += kThreads) {  // K rows -> e^{G} . b . k
-        const int i = idx / dk, d = idx % dk;
-        R[i * ld + d] *= Bc[i * lg + d] * expf(Gc[i * lg + d]);
-    }
     }
     __syncthreads();
     for (int col = tid; col < dk + dv; col += kThreads) {
@@ -919,6 +870,7 @@ size_t scan_smem(const gdr_chunk_args& a) {
 
 bool simt_supported(const gdr_chunk_args& a) {
     if (a.dv % kSlice != 0 || a.dk < 1 || a.dk > 256 || a.dv > 256) return false;
+    if (a.gdn2 && a.chunk > 64) return false;  // the GDN-2 local kernel tiles 64 rows
     if (simt_rb(a) && (prep_smem(a) > kMaxSmem || scan_rb_smem(a) > kMaxSmem)) return false;
     return local_smem(a) <= kMaxSmem && scan_smem(a) <= kMaxSmem;
 }

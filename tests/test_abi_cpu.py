@@ -170,6 +170,10 @@ def test_gdn2_host_validation(lib):
     assert need > lib.gdr_chunk_fwd_workspace_size(ctypes.byref(scalar))
     assert lib.gdr_chunk_fwd_path(ctypes.byref(g2)) == b"simt"
     assert lib.gdr_chunk_fwd_workspace_size(ctypes.byref(args(gdn2=2))) == 0
+    # GDN-2's local kernel tiles 64 rows: no path for chunks of 128
+    assert lib.gdr_chunk_fwd_workspace_size(ctypes.byref(args(gdn2=1, gdn2_w=FAKE, chunk=128))) == 0
+    assert lib.gdr_chunk_fwd_path(ctypes.byref(args(gdn2=1, gdn2_w=FAKE, chunk=128))) is None
+    assert lib.gdr_chunk_fwd_path(ctypes.byref(args(chunk=128))) == b"simt"  # scalar gates do
     assert lib.gdr_chunk_fwd_workspace_size(
         ctypes.byref(args(gdn2=1, gate_raw=1, gate_A=FAKE, gate_dt_bias=FAKE))) == 0
     assert call(lib, args(gdn2=1), wsb=need) == _abi.GDR_ERR_INVALID_ARG     # no write gate

@@ -92,10 +92,10 @@ def test_decode(dtype, read_mode, fused_norm):
     assert_close("S", S, S_ref, torch.float32 if dtype == "f32" else torch.bfloat16)
 
 
-@pytest.mark.parametrize("chunk", [16, 32, 128])
+@pytest.mark.parametrize("chunk", [16, 32])
 def test_chunk_sizes(chunk):
-    """Chunks of 32 (one factored block below the diagonal blocks), 16 (diagonal only) and
-    128 (one exp per term everywhere, the scan that forms P per column slice)."""
+    """Chunks of 32 (one factored block below the diagonal blocks) and 16 (diagonal only);
+    GDN-2 takes chunks up to 64."""
     x = workloads.chunk_inputs(1, 150, 2, 2, 64, 64, "f32", s0_std=0.05, seed=73)
     g, b, w = workloads.gdn2_gate_inputs(x["v"].shape[:3], 64, 64, "f32", seed=74)
     o, S = run_chunk(x, g, b, w, chunk=chunk, scale=0.125)
