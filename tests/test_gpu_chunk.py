@@ -12,7 +12,7 @@ import torch
 import oracle
 import workloads
 import gated_delta_rule_146_b200 as gdr
-from gpu_helpers import assert_close, oracle_units, to_dev, tol_for, max_err
+from gpu_helpers import assert_close, oracle_units, to_dev
 
 pytestmark = pytest.mark.gpu
 

@@ -18,7 +18,7 @@ g-logits, beta-logits), S0.
 from __future__ import annotations
 
 import math
-from dataclasses import dataclass, field
+from dataclasses import dataclass
 
 import torch
 
