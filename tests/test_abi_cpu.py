@@ -262,3 +262,15 @@ def test_binding_refuses_host_tensors(lib):
     for call in calls:
         with pytest.raises(ValueError, match="CUDA tensors only"):
             call()
+
+
+def test_binding_argument_counts_match_header(lib):
+    """Each prototype in include/gdr.h has as many parameters as the binding declares."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = re.findall(r"\b(gdr_[a-z_0-9]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S)
+    assert protos
+    for name, params in protos:
+        params = params.strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        argtypes = getattr(lib, name).argtypes
+        assert argtypes is not None and len(argtypes) == n, (name, n, argtypes)
