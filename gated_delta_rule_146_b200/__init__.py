@@ -22,7 +22,8 @@ from ._abi import GdrError, ChunkArgs, DecodeArgs, F32, BF16, READ_POST, READ_PR
 __all__ = ["chunk_fwd", "chunk_fwd_bidir", "chunk_bwd", "decode_step",
            "chunk_fwd_workspace_size", "chunk_fwd_bidir_workspace_size",
            "chunk_bwd_workspace_size", "chunk_fwd_path",
-           "read_device_error", "library", "GdrError"]
+           "read_device_error", "chunk_fwd_noalloc", "noalloc_read_device_error", "library",
+           "GdrError"]
 
 
 def library():
@@ -89,7 +90,7 @@ def _gdn2_fields(g, v, gdn2_w):
 
 def make_chunk_args(q, v, g, cu_seqlens=None, chunk=64, read_mode="post", scale=None,
                     qk_l2norm=True, reverse=False, o_accumulate=False, gate_A=None,
-                    gate_dt_bias=None, beta_scale=1.0, gdn2_w=None):
+                    gate_dt_bias=None, beta_scale=1.0, gdn2_w=None, status=None):
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     n_seqs = B if cu_seqlens is None else cu_seqlens.numel() - 1
@@ -98,7 +99,19 @@ def make_chunk_args(q, v, g, cu_seqlens=None, chunk=64, read_mode="post", scale=
     return ChunkArgs(B, T, Hk, Hv, dk, dv, n_seqs, chunk, _dtype_code(q), _dtype_code(g),
                      READ_PRE if read_mode == "pre" else READ_POST, float(scale),
                      int(bool(qk_l2norm)), int(bool(reverse)), int(bool(o_accumulate)),
-                     *_gating_fields(gate_A, gate_dt_bias, beta_scale), *_gdn2_fields(g, v, gdn2_w))
+                     *_gating_fields(gate_A, gate_dt_bias, beta_scale), *_gdn2_fields(g, v, gdn2_w),
+                     _status_field(status))
+
+
+def _status_field(status):
+    """Device address of the caller's optional status word (an int32 CUDA tensor that the
+    caller zeroes; a failed device-side check stores its gdr_status there), or None."""
+    if status is None:
+        return None
+    import torch
+    if status.dtype != torch.int32 or not status.is_cuda or status.numel() < 1:
+        raise TypeError("status must be an int32 CUDA tensor")
+    return status.data_ptr()
 
 
 def chunk_fwd_workspace_size(args: ChunkArgs) -> int:
@@ -113,19 +126,20 @@ def chunk_fwd_path(args: ChunkArgs):
 def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, *, chunk=64, read_mode="post",
               scale=None, qk_l2norm=True, reverse=False, o=None, o_accumulate=False,
               output_final_state=True, S_final=None, workspace=None, stream=None,
-              gate_A=None, gate_dt_bias=None, beta_scale=1.0, gdn2_w=None):
+              gate_A=None, gate_dt_bias=None, beta_scale=1.0, gdn2_w=None, status=None):
     """Chunk-parallel forward (gdr_chunk_fwd).  Shapes: q, k [B,T,Hk,dk]; v [B,T,Hv,dv];
     g, beta [B,T,Hv]; S0 [n_seqs,Hv,dk,dv] fp32 or None; cu_seqlens int32 [n_seqs+1] or
     None.  With gate_A and gate_dt_bias ([Hv] fp32) given, g and beta are the raw
     projections a and b of the fused gating prologue.  With gdn2_w ([B,T,Hv,dv]) given, the
     gates are GDN-2's: g the per-key-channel log decay and beta the erase gate, both
-    [B,T,Hv,dk], gdn2_w the write gate.  Returns (o [B,T,Hv,dv], S_final [n_seqs,Hv,dk,dv]
-    fp32 or None)."""
+    [B,T,Hv,dk], gdn2_w the write gate.  ``status``: an optional int32 CUDA tensor the
+    caller zeroes, where a failed device-side check stores its gdr_status without any
+    synchronisation.  Returns (o [B,T,Hv,dv], S_final [n_seqs,Hv,dk,dv] fp32 or None)."""
     import torch
     _check_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_final, workspace, gate_A, gate_dt_bias,
-                gdn2_w)
+                gdn2_w, status)
     args = make_chunk_args(q, v, g, cu_seqlens, chunk, read_mode, scale, qk_l2norm, reverse,
-                           o_accumulate, gate_A, gate_dt_bias, beta_scale, gdn2_w)
+                           o_accumulate, gate_A, gate_dt_bias, beta_scale, gdn2_w, status)
     if k.dtype != q.dtype or v.dtype != q.dtype or beta.dtype != g.dtype:
         raise TypeError("q, k, v share one dtype and g, beta another")
     if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
@@ -154,15 +168,16 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, *, chunk=64, read_mode
 
 def chunk_fwd_bidir(q, k, v, g_fwd, beta_fwd, g_bwd, beta_bwd, cu_seqlens=None, *, chunk=64,
                     read_mode="pre", scale=None, qk_l2norm=True, o=None, workspace=None,
-                    stream=None, gate_A=None, gate_dt_bias=None, beta_scale=1.0, gdn2_w=None):
+                    stream=None, gate_A=None, gate_dt_bias=None, beta_scale=1.0, gdn2_w=None,
+                    status=None):
     """Bidirectional forward (gdr_chunk_fwd_bidir): o = forward scan with (g_fwd, beta_fwd)
     + reverse scan within each sequence with (g_bwd, beta_bwd), from zero states, in one
-    call.  Shapes as for ``chunk_fwd``.  Returns o."""
+    call.  Shapes as for ``chunk_fwd``; ``status`` as there.  Returns o."""
     import torch
     _check_cuda(q, k, v, g_fwd, beta_fwd, g_bwd, beta_bwd, cu_seqlens, o, workspace, gate_A,
-                gate_dt_bias, gdn2_w)
+                gate_dt_bias, gdn2_w, status)
     args = make_chunk_args(q, v, g_fwd, cu_seqlens, chunk, read_mode, scale, qk_l2norm, False,
-                           False, gate_A, gate_dt_bias, beta_scale, gdn2_w)
+                           False, gate_A, gate_dt_bias, beta_scale, gdn2_w, status)
     if k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("q, k, v share one dtype")
     if len({t.dtype for t in (g_fwd, beta_fwd, g_bwd, beta_bwd)}) != 1:
@@ -194,14 +209,15 @@ def chunk_bwd_workspace_size(args: ChunkArgs) -> int:
 
 def chunk_bwd(q, k, v, g, beta, dO, S0=None, cu_seqlens=None, dS_final=None, *, chunk=64,
               read_mode="post", scale=None, qk_l2norm=True, reverse=False, dS0=True,
-              workspace=None, stream=None):
+              workspace=None, stream=None, status=None):
     """Backward pass of ``chunk_fwd`` (gdr_chunk_bwd): the gradients of
     <dO, o> + <dS_final, S_final> for the same inputs.  dO has the shape of v (io dtype);
     dS_final [n_seqs,Hv,dk,dv] fp32 or None.  Returns (dq, dk, dv, dg, dbeta, dS0) with the
     shapes and dtypes of q, k, v, g, beta and S0 (dS0 fp32, None when ``dS0=False``)."""
     import torch
-    _check_cuda(q, k, v, g, beta, dO, S0, cu_seqlens, dS_final, workspace)
-    args = make_chunk_args(q, v, g, cu_seqlens, chunk, read_mode, scale, qk_l2norm, reverse)
+    _check_cuda(q, k, v, g, beta, dO, S0, cu_seqlens, dS_final, workspace, status)
+    args = make_chunk_args(q, v, g, cu_seqlens, chunk, read_mode, scale, qk_l2norm, reverse,
+                           status=status)
     if k.dtype != q.dtype or v.dtype != q.dtype or dO.dtype != q.dtype or beta.dtype != g.dtype:
         raise TypeError("q, k, v, dO share one dtype and g, beta another")
     if tuple(dO.shape) != tuple(v.shape):
@@ -233,6 +249,23 @@ def read_device_error(args: ChunkArgs, workspace, stream=None) -> int:
     """Synchronising diagnostic: the device-side status recorded in `workspace`."""
     return int(_abi.lib().gdr_read_device_error(ctypes.byref(args), _ptr(workspace),
                                                 _stream(stream)))
+
+
+def chunk_fwd_noalloc(args: ChunkArgs, q, k, v, g, beta, S0, cu_seqlens, o, S_final,
+                      stream=None) -> int:
+    """gdr_chunk_fwd_noalloc: the forward with its scratch in the library's static device
+    array (no workspace).  ``args`` from ``make_chunk_args``; o and S_final are
+    caller-allocated outputs (S_final may be None).  Returns the gdr_status (not raised)."""
+    _check_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_final)
+    return int(_abi.lib().gdr_chunk_fwd_noalloc(
+        ctypes.byref(args), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+        _ptr(cu_seqlens), _ptr(o), _ptr(S_final), _stream(stream)))
+
+
+def noalloc_read_device_error(stream=None) -> int:
+    """Synchronising diagnostic: the device-side status the last gdr_chunk_fwd_noalloc call
+    left in the static scratch array of the current device."""
+    return int(_abi.lib().gdr_noalloc_read_device_error(_stream(stream)))
 
 
 def _norm_fields(q, norm_z, norm_weight, norm_eps):

@@ -16,6 +16,7 @@ READ_POST, READ_PRE = 0, 1
 
 # every symbol include/gdr.h declares
 EXPORTS = ["gdr_chunk_fwd_workspace_size", "gdr_chunk_fwd", "gdr_chunk_fwd_noalloc",
+           "gdr_noalloc_read_device_error",
            "gdr_chunk_bwd_workspace_size", "gdr_chunk_bwd",
            "gdr_chunk_fwd_bidir_workspace_size", "gdr_chunk_fwd_bidir",
            "gdr_chunk_fwd_path",
@@ -31,7 +32,8 @@ class ChunkArgs(ctypes.Structure):
                 ("reverse", ctypes.c_int), ("o_accumulate", ctypes.c_int),
                 ("gate_raw", ctypes.c_int), ("gate_A", ctypes.c_void_p),
                 ("gate_dt_bias", ctypes.c_void_p), ("beta_scale", ctypes.c_float),
-                ("gdn2", ctypes.c_int), ("gdn2_w", ctypes.c_void_p)]
+                ("gdn2", ctypes.c_int), ("gdn2_w", ctypes.c_void_p),
+                ("status", ctypes.c_void_p)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -64,6 +66,8 @@ def _declare(lib):
     lib.gdr_chunk_fwd.restype = ctypes.c_int
     lib.gdr_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(ChunkArgs)] + [vp] * 10
     lib.gdr_chunk_fwd_noalloc.restype = ctypes.c_int
+    lib.gdr_noalloc_read_device_error.argtypes = [vp]
+    lib.gdr_noalloc_read_device_error.restype = ctypes.c_int
     lib.gdr_chunk_fwd_bidir_workspace_size.argtypes = [ctypes.POINTER(ChunkArgs)]
     lib.gdr_chunk_fwd_bidir_workspace_size.restype = sz
     lib.gdr_chunk_fwd_bidir.argtypes = [ctypes.POINTER(ChunkArgs)] + [vp] * 10 + [sz, vp]

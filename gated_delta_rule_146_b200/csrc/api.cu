@@ -66,6 +66,25 @@ gdr_status check_chunk_args(const gdr_chunk_args* a) {
     return GDR_OK;
 }
 
+// The caller's optional device status word: 4-byte aligned when given.
+gdr_status check_status_word(const gdr_chunk_args* a) {
+    return (reinterpret_cast<uintptr_t>(a->status) & 3u) ? GDR_ERR_ALIGNMENT : GDR_OK;
+}
+
+// Copies a device-side status recorded in the workspace header into the caller's status
+// word, unless that word already holds an error.  Enqueued after a call's last kernel, so
+// it sees everything the call recorded.
+__global__ void publish_status_kernel(const WsHeader* __restrict__ hdr, int* __restrict__ status) {
+    const int e = hdr->err;
+    if (e != GDR_OK) atomicCAS(status, (int)GDR_OK, e);
+}
+
+gdr_status publish_status(const gdr_chunk_args& a, const void* ws, cudaStream_t s) {
+    if (!a.status) return GDR_OK;
+    publish_status_kernel<<<1, 1, 0, s>>>(reinterpret_cast<const WsHeader*>(ws), a.status);
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
 enum class Path { None, Tc, Simt };
 
 Path choose_path(const gdr_chunk_args& a) {
@@ -75,6 +94,16 @@ Path choose_path(const gdr_chunk_args& a) {
 }
 
 }  // namespace
+
+namespace gdr {
+// Host-side status of a forward call's arguments alone: what gdr_chunk_fwd would return
+// before looking at pointers, or GDR_ERR_UNSUPPORTED when no kernel path takes them.
+gdr_status chunk_args_status(const gdr_chunk_args* a) {
+    const gdr_status st = check_chunk_args(a);
+    if (st != GDR_OK) return st;
+    return choose_path(*a) == Path::None ? GDR_ERR_UNSUPPORTED : GDR_OK;
+}
+}  // namespace gdr
 
 extern "C" {
 
@@ -108,6 +137,7 @@ gdr_status gdr_chunk_fwd(const gdr_chunk_args* a, const void* q, const void* k, 
     const bool has_tokens = (long long)a->B * a->T > 0;
     if (has_tokens && (!q || !k || !v || !g || !beta || !o)) return GDR_ERR_INVALID_ARG;
     if ((st = check_gating(a, true)) != GDR_OK) return st;
+    if ((st = check_status_word(a)) != GDR_OK) return st;
     if (!workspace) return GDR_ERR_WORKSPACE;
     const void* ptrs[] = {q, k, v, g, beta, S0, cu_seqlens, o, S_final, workspace};
     for (const void* p : ptrs)
@@ -120,10 +150,13 @@ gdr_status gdr_chunk_fwd(const gdr_chunk_args* a, const void* q, const void* k, 
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (launch_plan(*a, cu_seqlens, workspace, L, s) != cudaSuccess) return GDR_ERR_CUDA;
-    if (path == Path::Tc)
-        return launch_chunk_tc(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s);
-    return launch_chunk_simt(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s);
+    st = path == Path::Tc
+             ? launch_chunk_tc(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s)
+             : launch_chunk_simt(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s);
+    if (st != GDR_OK) return st;
+    return publish_status(*a, workspace, s);
 }
+
 
 // Bidirectional forward: the plan, then the two scans; on the tensor-core path the reverse
 // scan is the forward scan's programmatic dependent (it fills the SMs the first grid leaves
@@ -163,6 +196,7 @@ gdr_status gdr_chunk_fwd_bidir(const gdr_chunk_args* a, const void* q, const voi
     if (has_tokens && (!q || !k || !v || !g_fwd || !beta_fwd || !g_bwd || !beta_bwd || !o))
         return GDR_ERR_INVALID_ARG;
     if ((st = check_gating(a, true)) != GDR_OK) return st;
+    if ((st = check_status_word(a)) != GDR_OK) return st;
     if (!workspace) return GDR_ERR_WORKSPACE;
     const void* ptrs[] = {q, k, v, g_fwd, beta_fwd, g_bwd, beta_bwd, cu_seqlens, o, workspace};
     for (const void* p : ptrs)
@@ -185,13 +219,19 @@ gdr_status gdr_chunk_fwd_bidir(const gdr_chunk_args* a, const void* q, const voi
         if ((st = launch_chunk_tc(rev, q, k, v, g_bwd, beta_bwd, nullptr, scratch, nullptr,
                                   workspace, L, s, /*dependent=*/true)) != GDR_OK)
             return st;
-        return launch_add_bf16(o, scratch, (long long)a->B * a->T * a->Hv * a->dv, s);
+        if ((st = launch_add_bf16(o, scratch, (long long)a->B * a->T * a->Hv * a->dv, s)) !=
+            GDR_OK)
+            return st;
+        return publish_status(*a, workspace, s);
     }
     if ((st = launch_chunk_simt(*a, q, k, v, g_fwd, beta_fwd, nullptr, o, nullptr, workspace, L,
                                 s)) != GDR_OK)
         return st;
     rev.o_accumulate = 1;  // the CUDA-core scan adds the reverse direction into o itself
-    return launch_chunk_simt(rev, q, k, v, g_bwd, beta_bwd, nullptr, o, nullptr, workspace, L, s);
+    if ((st = launch_chunk_simt(rev, q, k, v, g_bwd, beta_bwd, nullptr, o, nullptr, workspace, L,
+                                s)) != GDR_OK)
+        return st;
+    return publish_status(*a, workspace, s);
 }
 
 size_t gdr_chunk_bwd_workspace_size(const gdr_chunk_args* a) {
@@ -215,6 +255,7 @@ gdr_status gdr_chunk_bwd(const gdr_chunk_args* a, const void* q, const void* k, 
     const bool has_tokens = (long long)a->B * a->T > 0;
     if (has_tokens && (!q || !k || !v || !g || !beta || !dO || !dq || !dk || !dv || !dg || !dbeta))
         return GDR_ERR_INVALID_ARG;
+    if ((st = check_status_word(a)) != GDR_OK) return st;
     if (!workspace) return GDR_ERR_WORKSPACE;
     const void* ptrs[] = {q, k, v, g, beta, S0, cu_seqlens, dO, dS_final, dq, dk, dv, dg, dbeta,
                           dS0, workspace};
@@ -227,7 +268,8 @@ gdr_status gdr_chunk_bwd(const gdr_chunk_args* a, const void* q, const void* k, 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (launch_plan(*a, cu_seqlens, workspace, B.base, s) != cudaSuccess) return GDR_ERR_CUDA;
     const BwdPtrs x{q, k, v, g, beta, dO, S0, dS_final, dq, dk, dv, dg, dbeta, dS0};
-    return launch_chunk_bwd(*a, x, workspace, B, s);
+    if ((st = launch_chunk_bwd(*a, x, workspace, B, s)) != GDR_OK) return st;
+    return publish_status(*a, workspace, s);
 }
 
 gdr_status gdr_decode_step(const gdr_decode_args* a, const void* q, const void* k, const void* v,

@@ -119,6 +119,15 @@ typedef struct {
      *             gate_raw. */
     int gdn2;
     const void* gdn2_w;
+    /* Optional device status word (NULL: none).  A device int owned by the caller, who
+     * sets it to GDR_OK (0) before the call.  When a device-side check of the call fails
+     * (GDR_ERR_DEVICE_CHECK, GDR_ERR_TIMEOUT, GDR_ERR_RANGE), the call's last kernel stores
+     * that status here if the word still holds GDR_OK; the library never clears it.  The
+     * caller reads it whenever it likes (e.g. cudaMemcpyAsync into pinned host memory on
+     * the same stream), with no synchronisation inside the library, so one word can
+     * collect the status of many calls.  4-byte aligned.  Serves every entry point that
+     * takes these arguments, gdr_chunk_fwd_noalloc included. */
+    int* status;
 } gdr_chunk_args;
 
 /* Bytes of device workspace gdr_chunk_fwd needs for these arguments (0 on invalid
@@ -174,8 +183,13 @@ gdr_status gdr_chunk_fwd(const gdr_chunk_args* args,
  *   streams, or different host threads, without ordering between them) race and may
  *   corrupt each other's results.  Each call rewrites every scratch field it reads, so a
  *   previous call's contents never leak into the next.
- * - The device error word lives in the shared array, so gdr_read_device_error cannot be
- *   used with this entry point.
+ * - The device error word lives in the shared array: read it with
+ *   gdr_noalloc_read_device_error (which synchronises), or give args->status a device word
+ *   of the caller's to have it set without a synchronisation.
+ * - The array's address is cached per device and CUDA context; a call made after the
+ *   device's primary context was reset (cudaDeviceReset) looks it up again.
+ * - Arguments that are valid but have no kernel path return GDR_ERR_UNSUPPORTED, invalid
+ *   ones the status gdr_chunk_fwd would return; neither enqueues anything.
  */
 #define GDR_NOALLOC_SCRATCH_BYTES (4u << 20)
 gdr_status gdr_chunk_fwd_noalloc(const gdr_chunk_args* args,
@@ -183,6 +197,12 @@ gdr_status gdr_chunk_fwd_noalloc(const gdr_chunk_args* args,
                                  const void* g, const void* beta,
                                  const float* S0, const int32_t* cu_seqlens,
                                  void* o, float* S_final, void* stream);
+
+/* Test/diagnostic helper for gdr_chunk_fwd_noalloc, NOT for the hot path: copies the device
+ * error word out of the static scratch array of the current device (as the last
+ * gdr_chunk_fwd_noalloc call on `stream` left it), SYNCHRONISES `stream`, and returns GDR_OK
+ * or the recorded device-side status. */
+gdr_status gdr_noalloc_read_device_error(void* stream);
 
 /* Name of the kernel path gdr_chunk_fwd takes for these arguments: "tc" (tcgen05
  * tensor-core kernels), "simt" (fp32 CUDA-core kernels) or NULL if unsupported. */

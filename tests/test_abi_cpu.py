@@ -274,3 +274,20 @@ def test_binding_argument_counts_match_header(lib):
         n = 0 if params in ("", "void") else params.count(",") + 1
         argtypes = getattr(lib, name).argtypes
         assert argtypes is not None and len(argtypes) == n, (name, n, argtypes)
+
+
+def test_noalloc_and_status_word_host_validation(lib):
+    """gdr_chunk_fwd_noalloc names invalid arguments and valid ones without a kernel path
+    (GDN-2 with chunks of 128) as such, before touching the device; a misaligned status
+    word is refused by every entry point that takes the argument struct."""
+    vp = ctypes.c_void_p
+    na = lambda a: lib.gdr_chunk_fwd_noalloc(ctypes.byref(a), *[vp(FAKE)] * 9, None)
+    assert na(args(Hv=3)) == _abi.GDR_ERR_INVALID_ARG
+    g2 = args(dk=128, dv=128, chunk=128, gdn2=1, gdn2_w=FAKE)
+    assert lib.gdr_chunk_fwd_path(ctypes.byref(g2)) is None
+    assert na(g2) == _abi.GDR_ERR_UNSUPPORTED
+    a = args(status=FAKE + 2)
+    need = lib.gdr_chunk_fwd_workspace_size(ctypes.byref(a))
+    assert call(lib, a, wsb=need) == _abi.GDR_ERR_ALIGNMENT
+    assert lib.gdr_chunk_fwd_bidir(ctypes.byref(a), *[vp(FAKE)] * 7, None, vp(FAKE), vp(FAKE),
+                                   ctypes.c_size_t(1 << 30), None) == _abi.GDR_ERR_ALIGNMENT

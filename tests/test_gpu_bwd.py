@@ -1,9 +1,11 @@
 """GPU parity of the backward pass (gdr_chunk_bwd) against the fp64 reverse-mode oracle
 ``oracle.backward``, on the same seeded inputs and upstream gradients.
 
-Tolerance: bf16 as for the forward (2e-2 RMS(ref) + 2^-7 |ref| element-wise).  fp32: the
-pages ask the two forms to agree to 1e-4 on the forward and on the gradients; gradients
-scale with dO, T and the state, so the bound used is 1e-4 max(1, RMS(ref))."""
+Tolerance: bf16 as for the forward (2e-2 RMS(ref) + 2^-8 |ref| element-wise for a gradient
+written in bf16, 2e-2 RMS(ref) for the fp32 dS0).  fp32: the pages ask the two forms to
+agree to 1e-4 on the forward and on the gradients; gradients scale with dO, T and the
+state, so the bound used is 1e-4 max(1, RMS(ref)).  Every comparison's margin is recorded
+in the session's parity table."""
 import math
 
 import numpy as np
@@ -13,19 +15,22 @@ import torch
 import oracle.backward as obw
 import workloads
 import gated_delta_rule_146_b200 as gdr
-from gpu_helpers import assert_close, to_dev
+from gpu_helpers import assert_close, record, to_dev
 
 pytestmark = pytest.mark.gpu
 
 
 def grad_close(name, gpu, ref, dtype):
     if dtype == torch.bfloat16:
-        return assert_close(name, gpu, ref, dtype)
+        return assert_close(name, gpu, ref, dtype,
+                            kind="state" if name.startswith("dS0") else "out")
     g = gpu.detach().double().cpu().numpy()
     if not ref.size:
         return
-    tol = 1e-4 * max(1.0, float(np.sqrt(np.mean(ref * ref))))
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    tol = 1e-4 * max(1.0, rms)
     err = np.abs(g - ref)
+    record(name, float(err.max()), rms, float(err.max()) / tol)
     assert err.max() <= tol, f"{name}: max err {err.max():.3e} > {tol:.3e}"
 
 

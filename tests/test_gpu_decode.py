@@ -1,14 +1,13 @@
 """GPU parity of gdr_decode_step against the fp64 oracle."""
 import math
 
-import numpy as np
 import pytest
 import torch
 
 import oracle
 import workloads
 import gated_delta_rule_146_b200 as gdr
-from gpu_helpers import assert_close, to_dev
+from gpu_helpers import Accum, assert_close, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -28,7 +27,7 @@ def test_decode_steps_small(dtype, read_mode, dk, dv):
                                           S_ref, read_mode=read_mode, scale=scale)
         torch.cuda.synchronize()
         assert_close(f"o step {t}", o, o_ref, workloads.DTYPES[dtype])
-    assert_close("S", S, S_ref, torch.float32 if dtype == "f32" else torch.bfloat16)
+    assert_close("S", S, S_ref, torch.float32 if dtype == "f32" else torch.bfloat16, kind="state")
 
 
 def test_decode_matches_chunk_forward():
@@ -50,23 +49,32 @@ def test_decode_matches_chunk_forward():
     assert (S - S_c).abs().max().item() < 1e-4
 
 
-def test_decode_workload_sampled():
+def test_decode_workload_whole():
     """256 sequences x 32 v-heads (16 k-heads), 64 steps of fresh bf16 inputs from an
-    N(0, 0.02^2) fp32 state; the oracle follows 12 sampled sequences through all steps."""
+    N(0, 0.02^2) fp32 state: every output of every step and the whole final state against
+    the oracle, which follows groups of 32 sequences through all 64 steps."""
     w = workloads.DECODE_WORKLOADS["bf16_decode_n256_hk16_hv32_d128"]
     x = workloads.decode_workload_inputs(w)
     S = x["S"].clone().cuda()
-    seqs = np.random.default_rng(0).choice(w.N, 12, replace=False)
-    seqs.sort()
-    S_ref = x["S"][seqs].double().numpy()
+    outs = []
     for t in range(w.steps):
         o = gdr.decode_step(*(to_dev(x[n][t]) for n in ("q", "k", "v", "g", "beta")), S,
                             read_mode=w.read_mode, scale=w.scale)
-        o_ref, S_ref = oracle.decode_step(*(x[n][t][seqs] for n in ("q", "k", "v", "g", "beta")),
-                                          S_ref, read_mode=w.read_mode, scale=w.scale)
-        torch.cuda.synchronize()
-        assert_close(f"o step {t}", o[seqs], o_ref, torch.bfloat16)
-    assert_close("S final", S[seqs], S_ref, torch.bfloat16)
+        outs.append(o.cpu())
+    torch.cuda.synchronize()
+    S_gpu = S.cpu()
+    ao = Accum("o (every step)", torch.bfloat16, "out")
+    aS = Accum("S final", torch.bfloat16, "state")
+    for s0 in range(0, w.N, 32):
+        sl = slice(s0, s0 + 32)
+        S_ref = x["S"][sl].double().numpy()
+        for t in range(w.steps):
+            o_ref, S_ref = oracle.decode_step(*(x[n][t][sl] for n in ("q", "k", "v", "g", "beta")),
+                                              S_ref, read_mode=w.read_mode, scale=w.scale)
+            ao.add(outs[t][sl], o_ref, label=f" step {t} seqs {s0}+")
+        aS.add(S_gpu[sl], S_ref, label=f" seqs {s0}+")
+    ao.check()
+    aS.check()
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -89,4 +97,4 @@ def test_decode_fused_gated_rmsnorm(dtype, dk, dv):
         ref = oracle.gated_rmsnorm(o_core, z, w, 1e-6)
         torch.cuda.synchronize()
         assert_close(f"o step {t}", o, ref, workloads.DTYPES[dtype])
-    assert_close("S", S, S_ref, torch.float32 if dtype == "f32" else torch.bfloat16)
+    assert_close("S", S, S_ref, torch.float32 if dtype == "f32" else torch.bfloat16, kind="state")

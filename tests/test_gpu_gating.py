@@ -48,7 +48,7 @@ def test_tensor_core_path(beta_scale, read_mode):
     o_r, S_r = oracle.forward(x["q"], x["k"], x["v"], g, beta, x["S0"], read_mode=read_mode,
                               scale=scale)
     assert_close("o", o, o_r, torch.bfloat16)
-    assert_close("S", S, S_r, torch.bfloat16)
+    assert_close("S", S, S_r, torch.bfloat16, kind="state")
 
 
 def test_tensor_core_varlen_reverse_fp32_gates():
@@ -61,7 +61,7 @@ def test_tensor_core_varlen_reverse_fp32_gates():
     o_r, S_r = oracle.forward(x["q"], x["k"], x["v"], g, beta, x["S0"], x["cu_seqlens"],
                               read_mode="pre", scale=0.3, reverse=True)
     assert_close("o", o, o_r, torch.bfloat16)
-    assert_close("S", S, S_r, torch.bfloat16)
+    assert_close("S", S, S_r, torch.bfloat16, kind="state")
 
 
 def test_cuda_core_path():
@@ -74,7 +74,7 @@ def test_cuda_core_path():
     g, beta = oracle.gating(a, b, A, dt, 2.0)
     o_r, S_r = oracle.forward(x["q"], x["k"], x["v"], g, beta, x["S0"], scale=0.125)
     assert_close("o", o, o_r, torch.float32)
-    assert_close("S", S, S_r, torch.float32)
+    assert_close("S", S, S_r, torch.float32, kind="state")
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -93,4 +93,4 @@ def test_decode(dtype):
                                           scale=1 / math.sqrt(128))
         torch.cuda.synchronize()
         assert_close(f"o step {t}", o, o_ref, workloads.DTYPES[dtype])
-    assert_close("S", S, S_ref, torch.float32 if dtype == "f32" else torch.bfloat16)
+    assert_close("S", S, S_ref, torch.float32 if dtype == "f32" else torch.bfloat16, kind="state")

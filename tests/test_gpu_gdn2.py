@@ -36,7 +36,7 @@ def test_chunk(dtype, read_mode):
     o_r, S_r = oracle.gdn2_forward(x["q"], x["k"], x["v"], g, b, w, x["S0"],
                                    read_mode=read_mode, scale=scale)
     assert_close("o", o, o_r, workloads.DTYPES[dtype])
-    assert_close("S", S, S_r, workloads.DTYPES[dtype])
+    assert_close("S", S, S_r, workloads.DTYPES[dtype], kind="state")
 
 
 @pytest.mark.parametrize("reverse", [False, True])
@@ -48,7 +48,7 @@ def test_chunk_varlen_small_heads(reverse):
     o_r, S_r = oracle.gdn2_forward(x["q"], x["k"], x["v"], g, b, w, x["S0"], x["cu_seqlens"],
                                    read_mode="pre", scale=0.3, reverse=reverse)
     assert_close("o", o, o_r, torch.float32)
-    assert_close("S", S, S_r, torch.float32)
+    assert_close("S", S, S_r, torch.float32, kind="state")
 
 
 def test_chunk_scalar_gates_match_gated_delta_rule():
@@ -60,7 +60,7 @@ def test_chunk_scalar_gates_match_gated_delta_rule():
     o, S = run_chunk(x, g, b, b.clone(), scale=0.125)
     o_r, S_r = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], scale=0.125)
     assert_close("o", o, o_r, torch.float32)
-    assert_close("S", S, S_r, torch.float32)
+    assert_close("S", S, S_r, torch.float32, kind="state")
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -89,7 +89,7 @@ def test_decode(dtype, read_mode, fused_norm):
             o_ref = oracle.gated_rmsnorm(o_ref, z, weight, 1e-6)
         torch.cuda.synchronize()
         assert_close(f"o step {t}", o, o_ref, workloads.DTYPES[dtype])
-    assert_close("S", S, S_ref, torch.float32 if dtype == "f32" else torch.bfloat16)
+    assert_close("S", S, S_ref, torch.float32 if dtype == "f32" else torch.bfloat16, kind="state")
 
 
 @pytest.mark.parametrize("chunk", [16, 32])
@@ -101,7 +101,7 @@ def test_chunk_sizes(chunk):
     o, S = run_chunk(x, g, b, w, chunk=chunk, scale=0.125)
     o_r, S_r = oracle.gdn2_forward(x["q"], x["k"], x["v"], g, b, w, x["S0"], scale=0.125)
     assert_close("o", o, o_r, torch.float32)
-    assert_close("S", S, S_r, torch.float32)
+    assert_close("S", S, S_r, torch.float32, kind="state")
 
 
 def test_growing_and_strong_decays():
@@ -120,4 +120,4 @@ def test_growing_and_strong_decays():
         o_r, S_r = oracle.gdn2_forward(x["q"], x["k"], x["v"], g, b, w, x["S0"], read_mode=mode,
                                        scale=0.125)
         assert_close(f"o {mode}", o, o_r, torch.float32)
-        assert_close(f"S {mode}", S, S_r, torch.float32)
+        assert_close(f"S {mode}", S, S_r, torch.float32, kind="state")

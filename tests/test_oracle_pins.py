@@ -326,3 +326,38 @@ def test_matches_wy_form_random_shapes():
         assert np.abs(o - o2).max(initial=0.0) < 1e-9 and np.abs(S - S2).max(initial=0.0) < 1e-9
 
     check()
+
+
+@pytest.mark.parametrize("read_mode,read_mode_bwd,combine", [("pre", None, 1.0),
+                                                             ("post", "pre", 0.5)])
+def test_bidirectional_is_forward_plus_host_flipped_scan(read_mode, read_mode_bwd, combine):
+    """oracle.bidirectional against an independent assembly of its two directions
+    (Rondo-Exp tiny_gdn/fugue.py, BidirectionalGatedDeltaNet2.forward and scan): the
+    forward direction is the NumPy WY/UT form with (g_fwd, beta_fwd); the backward
+    direction flips every segment on the host, runs the same WY form FORWARD with
+    (g_bwd, beta_bwd), and flips the output back; the two are summed and scaled by the
+    combine factor.  Neither the C oracle nor its reversal flag is used on this side."""
+    lens = [9, 1, 30, 17]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    rng = np.random.default_rng(77)
+    q, k, v, g_f, b_f, _ = rand_problem(T=int(cu[-1]), Hk=1, Hv=2, dk=8, dv=6, rng=rng)
+    g_b = -np.log1p(np.exp(rng.standard_normal(g_f.shape) - 1.0))
+    b_b = 1.5 / (1.0 + np.exp(-rng.standard_normal(b_f.shape)))
+    got = oracle.bidirectional(q, k, v, g_f, b_f, g_b, b_b, cu, read_mode=read_mode,
+                               scale=0.6, read_mode_bwd=read_mode_bwd, combine=combine)
+    rev = np.concatenate([np.arange(cu[s + 1] - 1, cu[s] - 1, -1) for s in range(len(lens))])
+    flip = lambda x: x[:, rev]
+    o_f, _ = wy_reference.chunked_forward(q, k, v, g_f, b_f, None, cu, chunk=8,
+                                          read_mode=read_mode, scale=0.6)
+    o_b, _ = wy_reference.chunked_forward(flip(q), flip(k), flip(v), flip(g_b), flip(b_b), None,
+                                          cu, chunk=8, read_mode=read_mode_bwd or read_mode,
+                                          scale=0.6)
+    want = combine * (o_f + flip(o_b))
+    assert np.abs(got - want).max() < 1e-10
+    # the directions are not interchangeable: swapping the gate pairs changes the result,
+    # and so does dropping either direction
+    swapped = oracle.bidirectional(q, k, v, g_b, b_b, g_f, b_f, cu, read_mode=read_mode,
+                                   scale=0.6, read_mode_bwd=read_mode_bwd, combine=combine)
+    assert np.abs(swapped - want).max() > 1e-3
+    assert np.abs(combine * o_f - want).max() > 1e-3
+    assert np.abs(combine * flip(o_b) - want).max() > 1e-3
