@@ -33,6 +33,7 @@ METRIC = "gated-delta chunk-fwd tokens/s + %bf16 TC peak; decode state GB/s vs H
 CHUNK_WORKLOAD = "bf16_b8_h16_t4096_d128"
 DECODE_WORKLOAD = "bf16_decode_n256_hk16_hv32_d128"
 BIDIR_WORKLOAD = "bf16_bidir_16x2048_h12_d64"
+VARLEN_WORKLOAD = "bf16_varlen64_h16_d128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -294,6 +295,53 @@ def bench_ours(args, rank, world, local_rank):
                  "algorithmic_bytes": bbytes,
                  "hbm_frac": bbytes / (bms / 1e3) / 1e9 / peaks["hbm_gbs"]}
 
+    # ---------------- varlen workload: 64 sequences of 256-8192 tokens packed in one row,
+    # per-sequence initial state, S_final per sequence
+    varlen = None
+    if not args.no_varlen and args.only != "decode" and not args.rows:
+        vw = workloads.WORKLOADS[VARLEN_WORKLOAD]
+        vx = workloads.workload_inputs(vw, seed=rank)
+        vd = {n: (t.to(dev) if t is not None else None) for n, t in vx.items()}
+        vo = torch.empty_like(vd["v"])
+        vargs = gdr.make_chunk_args(vd["q"], vd["v"], vd["g"], vd["cu_seqlens"], vw.chunk,
+                                    vw.read_mode, vw.scale)
+        vS = torch.empty((vargs.n_seqs, vw.Hv, vw.dk, vw.dv), dtype=torch.float32, device=dev)
+        vws = torch.empty(gdr.chunk_fwd_workspace_size(vargs), dtype=torch.uint8, device=dev)
+
+        def vstep():
+            gdr.chunk_fwd(vd["q"], vd["k"], vd["v"], vd["g"], vd["beta"], vd["S0"],
+                          vd["cu_seqlens"], chunk=vw.chunk, read_mode=vw.read_mode,
+                          scale=vw.scale, o=vo, S_final=vS, workspace=vws)
+
+        for _ in range(args.warmup):
+            vstep()
+        torch.cuda.synchronize()
+        barrier()
+        v0, v1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        v0.record(stream)
+        vsteps = max(1, min(args.steps, 20))
+        for _ in range(vsteps):
+            vstep()
+        v1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        vms = max_over_ranks(v0.elapsed_time(v1) / vsteps, world)
+        vtok = int(vd["q"].shape[1])
+        vbytes = sum(t.numel() * t.element_size() for t in
+                     (vd["q"], vd["k"], vd["v"], vd["g"], vd["beta"], vo, vd["S0"], vS))
+        vgbs = vbytes / (vms / 1e3) / 1e9
+        vflops = vtok * vw.Hv * flops_per_head_token(vw.chunk, vw.dk, vw.dv)
+        varlen = {"workload": vw.name, "tokens": vtok, "sequences": vargs.n_seqs,
+                  "ms_per_step": vms, "steps": vsteps,
+                  "value": whole_job_rate(vtok, world, vms), "unit": "tokens/s",
+                  "path": gdr.chunk_fwd_path(vargs),
+                  "tflops": vflops / (vms / 1e3) / 1e12,
+                  "roofline": {"bound": "hbm", "achieved": vgbs, "peak": peaks["hbm_gbs"],
+                               "unit": "GB/s", "frac": vgbs / peaks["hbm_gbs"],
+                               "algorithmic_bytes": vbytes,
+                               "floor_ms": vbytes / (peaks["hbm_gbs"] * 1e9) * 1e3}}
+        del vws, vo, vS, vd
+
     # ---------------- decode step
     dec = None
     if not args.no_decode and args.only != "chunk":
@@ -461,38 +509,77 @@ def bench_ours(args, rank, world, local_rank):
                               "frac": g2gbs / peaks["hbm_gbs"]}
     clocks = sampler.stop()
 
-    # ---------------- end to end through the public API with host buffers
+    # ---------------- end to end through the public API with host buffers: the rows are cut
+    # into blocks; each block's inputs are copied in on one stream, its forward runs on a
+    # stream of its own once its copies have landed, and its o and S_final are copied out on a
+    # third stream, so copies in, kernels and copies out of different blocks overlap
     e2e = None
     if not args.no_e2e:
         pin = {n: x[n].pin_memory() for n in ("q", "k", "v", "g", "beta")}
         h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         h_S = torch.empty(S_final.shape, dtype=S_final.dtype).pin_memory()
         bufs = {n: torch.empty_like(d[n]) for n in pin}
+        nblk = 4 if w.B % 4 == 0 else 1
+        rb = w.B // nblk
+        h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        cstr = [torch.cuda.Stream(device=dev) for _ in range(nblk)]
+        sub = gdr.make_chunk_args(d["q"][:rb], d["v"][:rb], d["g"][:rb], None, w.chunk,
+                                  w.read_mode, w.scale)
+        wss = [torch.empty(gdr.chunk_fwd_workspace_size(sub), dtype=torch.uint8, device=dev)
+               for _ in range(nblk)]
 
-        def e2e_step():
-            for n in pin:
-                bufs[n].copy_(pin[n], non_blocking=True)
-            oo, SS = gdr.chunk_fwd(bufs["q"], bufs["k"], bufs["v"], bufs["g"], bufs["beta"],
-                                   None, None, chunk=w.chunk, read_mode=w.read_mode,
-                                   scale=w.scale, o=o, S_final=S_final, workspace=ws)
-            h_o.copy_(oo, non_blocking=True)
-            h_S.copy_(SS, non_blocking=True)
+        def e2e_step(start_ev):
+            h2d.wait_event(start_ev)
+            landed = []
+            with torch.cuda.stream(h2d):
+                for i in range(nblk):
+                    r = slice(i * rb, (i + 1) * rb)
+                    for n in pin:
+                        bufs[n][r].copy_(pin[n][r], non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(h2d)
+                    landed.append(ev)
+            for i in range(nblk):
+                r = slice(i * rb, (i + 1) * rb)
+                cstr[i].wait_event(landed[i])
+                with torch.cuda.stream(cstr[i]):
+                    gdr.chunk_fwd(bufs["q"][r], bufs["k"][r], bufs["v"][r], bufs["g"][r],
+                                  bufs["beta"][r], None, None, chunk=w.chunk,
+                                  read_mode=w.read_mode, scale=w.scale, o=o[r],
+                                  S_final=S_final[r], workspace=wss[i], stream=cstr[i])
+                    done = torch.cuda.Event()
+                    done.record(cstr[i])
+                d2h.wait_event(done)
+                with torch.cuda.stream(d2h):
+                    h_o[r].copy_(o[r], non_blocking=True)
+                    h_S[r].copy_(S_final[r], non_blocking=True)
+            fin = torch.cuda.Event()
+            fin.record(d2h)
+            stream.wait_event(fin)
+            return fin
 
+        # each step starts once the previous one has copied its results out (its buffers are
+        # reused), so a step's time is one batch from host memory to host memory
         n_e2e = max(1, min(args.steps, 5))
-        e2e_step()
+        s0 = torch.cuda.Event()
+        s0.record(stream)
+        e2e_step(s0)
         torch.cuda.synchronize()
         barrier()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
+        prev = a0
         for _ in range(n_e2e):
-            e2e_step()
+            prev = e2e_step(prev)
         a1.record(stream)
         torch.cuda.synchronize()
         barrier()
         ems = max_over_ranks(a0.elapsed_time(a1) / n_e2e, world)
         e2e = {"value": whole_job_rate(tokens, world, ems), "unit": "tokens/s", "ms_per_step": ems,
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin.values()),
-               "d2h_bytes_per_step": h_o.numel() * h_o.element_size() + h_S.numel() * 4}
+               "d2h_bytes_per_step": h_o.numel() * h_o.element_size() + h_S.numel() * 4,
+               "pipeline": f"{nblk} row blocks: copies in, forward and copies out overlapped "
+                           "on three streams"}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -514,7 +601,8 @@ def bench_ours(args, rank, world, local_rank):
                      "tensor_frac": tflops / peaks["bf16_tflops"],
                      "timed": "whole gdr_chunk_fwd call (plan + chunk kernels), CUDA events",
                      "peak_source": f"{peak_src} (hbm_gbs copy; bf16_tflops burst)"},
-        "decode": dec, "gating_prologue": gating, "bidirectional": bidir, "gdn2": gdn2, "backward": backward, "e2e": e2e,
+        "decode": dec, "varlen": varlen, "gating_prologue": gating, "bidirectional": bidir,
+        "gdn2": gdn2, "backward": backward, "e2e": e2e,
         "clocks": clocks,
         "gpu_launches": launches_per_call * args.steps,
     }
@@ -584,6 +672,8 @@ def main():
                     help="skip the GDN-2 (decoupled gates) chunk and decode measurements")
     ap.add_argument("--no-bidir", action="store_true",
                     help="skip the bidirectional workload (both directions summed)")
+    ap.add_argument("--no-varlen", action="store_true",
+                    help="skip the varlen workload (64 packed sequences of 256-8192 tokens)")
     ap.add_argument("--no-gating", action="store_true",
                     help="skip the forward through the fused gating prologue")
     ap.add_argument("--no-e2e", action="store_true")

@@ -36,12 +36,14 @@
 //
 // Operand precision: [K;Q] K^T is formed from the bf16 inputs as they arrive (exact
 // products, fp32 sums) and the L2 norms are applied to its rows and columns in fp32.
-// V and T diag(beta) are bf16 (V arrives in bf16); every other operand
-// (normalised k, Q~, T diag(beta e^G), W, the state copy, V', P) is rounded to fp16,
-// whose 11-bit significand keeps the chain of roundings well inside the bf16 parity bound
-// at long sequence lengths where bf16 operands do not.  Every fp16 operand is checked for
-// overflow (an infinite or NaN half); one sets GDR_ERR_RANGE.  Decay factors are
-// 2^(log2(e) (G_i - G_j)) by the hardware exp2 approximation (relative error ~2^-22).
+// Every other operand (normalised k, Q~, V, T diag(beta), T diag(beta e^G), W, the state
+// copy, V', P) is fp16, whose 11-bit significand keeps the chain of roundings well inside
+// the bf16 parity bound at long sequence lengths where bf16 operands do not; V is
+// converted to fp16 in shared memory, exactly for every bf16 value of the fp16 range.  A
+// value beyond the fp16 range becomes infinite and makes an output or the final state
+// non-finite; the chain checks both, and a non-finite one sets GDR_ERR_RANGE.  Decay
+// factors are 2^(log2(e) (G_i - G_j)) by the hardware exp2 approximation (relative error
+// ~2^-22).
 //
 // The state update uses V' with its rows scaled by e^(G_C - G_i) (a second fp16 copy in
 // tensor memory) against the unscaled K, so K is never rewritten after normalisation.
@@ -81,7 +83,7 @@ constexpr uint32_t OFF_TWU = 131072;   // T fp32 [64][64] (the solve)
 constexpr uint32_t OFF_AS = 147456;    // A fp32 [64][64]
 constexpr uint32_t OFF_RS = 163840;    // the four diagonal 16x16 blocks of A, transposed (fp32)
 constexpr uint32_t OFF_P = 167936;     // 2 x 8 KB: P fp16 [i][j]
-constexpr uint32_t OFF_WN = 184320;    // 2 x 16 KB: T diag(beta e^G) fp16 | T diag(beta) bf16
+constexpr uint32_t OFF_WN = 184320;    // 2 x 16 KB: T diag(beta e^G) fp16 | T diag(beta) fp16
                                        // during the solve, then -W^T fp16 [dk][tok]; output
                                        // staging
 constexpr uint32_t OFF_SMALL = 217088;
@@ -105,7 +107,8 @@ enum {
     MB_LD = 7,    // x3: K, Q, V tiles of a chunk landed (by K/Q buffer)
     MB_CD = 10,   // x2: chain finished with a chunk's buffers (by chunk parity)
     MB_MU = 12,   // U~ product of a chunk done (awaited by the chain's MMA issuer)
-    MB_COUNT = 13
+    MB_MO = 13,   // output products of a chunk done
+    MB_COUNT = 14
 };
 
 struct Small {
@@ -130,8 +133,8 @@ struct TcParams {
     const void* g; const void* beta; const float* S0;
     __nv_bfloat16* o; float* S_final;
     WsHeader* hdr; const int32_t* cu;
+    const int32_t* order;  // sequences in visiting order (longest first for varlen calls)
     int Hk, Hv, read_pre, qk_l2norm, reverse, o_acc, use_tma;
-    int tma_store;  // full output chunks leave through the output tensor map
     gdr_dtype gt;
     float scale;
 };
@@ -143,17 +146,24 @@ struct GateParams {
     float beta_scale;
 };
 
-// fp16 pair; `mx` keeps the running maximum magnitude of every half produced (NaN sticks),
-// tested once at the end: an infinite or NaN half means the value left the fp16 range.
-__device__ __forceinline__ uint32_t h2(float a, float b, __half2& mx) {
+// fp16 pair, rounded to nearest.  A value beyond the fp16 range becomes infinite; every
+// operand takes part in products that reach the outputs or the state, where it shows as a
+// non-finite value (an infinity, or NaN from infinity times zero), and those are checked.
+__device__ __forceinline__ uint32_t h2(float a, float b) {
     const __half2 v = __floats2half2_rn(a, b);
-    mx = __hmax2_nan(mx, __habs2(v));
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-__device__ __forceinline__ uint4 h8(const float* f, __half2& flags) {
-    return make_uint4(h2(f[0], f[1], flags), h2(f[2], f[3], flags), h2(f[4], f[5], flags),
-                      h2(f[6], f[7], flags));
+__device__ __forceinline__ uint4 h8(const float* f) {
+    return make_uint4(h2(f[0], f[1]), h2(f[2], f[3]), h2(f[4], f[5]), h2(f[6], f[7]));
+}
+
+// max(m, |x|) with NaN propagation: the running magnitude of the outputs and the final state,
+// non-finite exactly when one of them is
+__device__ __forceinline__ float max_abs_nan(float m, float x) {
+    float y;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(y) : "f"(m), "f"(fabsf(x)));
+    return y;
 }
 
 // element (i, j) of a fp32 [64][64] matrix stored with 16-byte chunks XOR-swizzled by row
@@ -182,7 +192,7 @@ template <bool kRaw, int kDh>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-               const __grid_constant__ CUtensorMap tm_o, const GateParams gp) {
+               const GateParams gp) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base, as a byte offset from the shared array so that every access
     // through it stays a shared-memory access (an integer round trip would make them generic)
@@ -198,7 +208,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     griddep_launch_dependents();
     if (p.hdr->err != GDR_OK) { griddep_wait(); return; }
 
-    const int s = blockIdx.x, h = blockIdx.y;
+    // one CTA per (sequence, value head), heads fastest, sequences in the plan's order
+    const int h = (int)(blockIdx.x % (unsigned)p.Hv);
+    const int s = p.order[blockIdx.x / (unsigned)p.Hv];
     // the gates as the recurrence uses them (fused gating prologue when kRaw)
     auto XG = [&](float a) -> float {
         if constexpr (kRaw) return gate_g_from_raw(gp.A[h], gp.dt_bias[h], a);
@@ -252,8 +264,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     tc_fence_after();
     const uint32_t tmem = SS.tmem_base;
     const uint32_t tlane = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's lanes
-    __half2 rflags = __float2half2_rn(0.f);  // running max |fp16 operand| (overflow test)
-    bool rbad = false;                       // a bound showed an operand out of the fp16 range
+    float omax = 0.f;     // chain: running max |output| and |final state| (NaN sticks)
     bool fail = false;    // a bounded wait gave up
 
     auto gate_at = [&](const void* arr, int pos) -> float {
@@ -469,8 +480,6 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     f = p.scale * ex2(Gr) * inv;
                 }
                 if (i >= Cc) f = 0.f;
-                // every element of the row is at most ||row|| f in magnitude (NaN fails too)
-                if (!(sqrtf(tot) * fabsf(f) < 65504.f)) rbad = true;
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
                     const uint32_t w[4] = {vals[c8].x, vals[c8].y, vals[c8].z, vals[c8].w};
@@ -480,10 +489,24 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         hv[c8 * 4 + e] = pack_f16x2(x.x * f, x.y * f);
                     }
                 }
-                for (int idx = pt; idx < (C - Cc) * 16; idx += kPrep) {  // V rows past the chunk
-                    const int iv = Cc + (idx >> 4), c16 = idx & 15;
-                    *reinterpret_cast<uint4*>(sm + OFF_V + pb * V_STRIDE + (c16 >> 3) * 8192 +
-                                              sw128(iv, c16 & 7)) = make_uint4(0, 0, 0, 0);
+                // V to fp16 in place (every bf16 value of the fp16 range is exact in fp16),
+                // rows past the chunk to zero; the swizzle only permutes the 16-byte pieces
+                // within a row, so a piece's row is its offset / 128
+                for (int idx = pt; idx < (kDh / 64) * 512; idx += kPrep) {
+                    uint4* vp = reinterpret_cast<uint4*>(sm + OFF_V + pb * V_STRIDE) + idx;
+                    if (((idx & 511) >> 3) >= Cc) {
+                        *vp = make_uint4(0, 0, 0, 0);
+                        continue;
+                    }
+                    const uint4 w = *vp;
+                    const uint32_t wi[4] = {w.x, w.y, w.z, w.w};
+                    uint32_t wo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 xv = unpack_bf16x2(wi[e]);
+                        wo[e] = h2(xv.x, xv.y);
+                    }
+                    *vp = make_uint4(wo[0], wo[1], wo[2], wo[3]);
                 }
             }
             if (!wg_wait(MB_M0, c & 1, kBarPrep)) { fail = true; break; }
@@ -593,7 +616,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                             pv[u] = on ? vals[e8 * 8 + u] : 0.f;
                         }
                         *reinterpret_cast<uint4*>(sm + OFF_P + pb * 8192 + sw128(i, hf * 4 + e8)) =
-                            h8(pv, rflags);
+                            h8(pv);
                     }
                 }
             }
@@ -649,7 +672,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         for (int e = 0; e < 4; ++e)
                             R[nt][e] = (add ? R[nt][e] : 0.f) + (t[0][nt][e] + t[1][nt][e]);
                 };
-                // T_w = T diag(beta e^G) (fp16) and T_u = T diag(beta) (bf16) as [i][j] K-major
+                // T_w = T diag(beta e^G) and T_u = T diag(beta) (fp16) as [i][j] K-major
                 // tiles, the B operands of the W and U~ products, in the -W^T buffer of this
                 // chunk (free from the chunk's start until the products have run); each block of
                 // T is written there by the warp that completes it
@@ -664,8 +687,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         for (int hh = 0; hh < 2; ++hh) {
                             const float t0 = -acc[nt][2 * hh], t1 = -acc[nt][2 * hh + 1];
                             const uint32_t off = sw128(16 * yr + gq + 8 * hh, cc >> 3) + (cc & 7) * 2;
-                            *reinterpret_cast<uint32_t*>(twu + off) = h2(t0 * bgp.x, t1 * bgp.y, rflags);
-                            *reinterpret_cast<uint32_t*>(twu + 8192 + off) = pack_bf16x2(t0 * bp.x, t1 * bp.y);
+                            *reinterpret_cast<uint32_t*>(twu + off) = h2(t0 * bgp.x, t1 * bgp.y);
+                            *reinterpret_cast<uint32_t*>(twu + 8192 + off) = h2(t0 * bp.x, t1 * bp.y);
                         }
                     }
                 };
@@ -724,8 +747,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                             uint32_t w4[4], u4[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                w4[e] = h2(tv[2 * e] * gv[2 * e], tv[2 * e + 1] * gv[2 * e + 1], rflags);
-                                u4[e] = pack_bf16x2(tv[2 * e] * bv[2 * e], tv[2 * e + 1] * bv[2 * e + 1]);
+                                w4[e] = h2(tv[2 * e] * gv[2 * e], tv[2 * e + 1] * gv[2 * e + 1]);
+                                u4[e] = h2(tv[2 * e] * bv[2 * e], tv[2 * e + 1] * bv[2 * e + 1]);
                             }
                             *reinterpret_cast<uint4*>(twu + sw128(i, 2 * b + m)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                             *reinterpret_cast<uint4*>(twu + 8192 + sw128(i, 2 * b + m)) = make_uint4(u4[0], u4[1], u4[2], u4[3]);
@@ -759,7 +782,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             named_bar(kBarPrep, kPrep);
             tc_fence_after();
 
-            // P5: W^T = K^T T_w^T (fp16, into D0) and U~^T = V^T T_u^T (bf16, into DU[pb])
+            // P5: W^T = K^T T_w^T (into D0) and U~^T = V^T T_u^T (into DU[pb]), fp16 operands
             if (pt == 0) {
                 const uint32_t idw = idesc_f32acc(128, 64, true, false, false);
 #pragma unroll
@@ -767,7 +790,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     mma_f32acc_ss(tmem + TM_D0, sdesc_sw128(KQ + kk * 2048, 16384, 1024),
                                   sdesc_sw128(sbase + OFF_WN + pb * 16384 + kk * 32, 16, 1024), idw, kk > 0);
                 mma_commit(&SS.mbar[MB_MW]);  // W^T: all P6 needs
-                const uint32_t idu = idesc_f32acc(128, 64, true, false, true);
+                const uint32_t idu = idesc_f32acc(128, 64, true, false, false);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f32acc_ss(tmem + TM_DU + pb * 64, sdesc_sw128(VV + kk * 2048, 8192, 1024),
@@ -788,7 +811,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                     for (int u = 0; u < 8; ++u) f[u] = -u2f(rr[e8 * 8 + u]);
                     *reinterpret_cast<uint4*>(sm + OFF_WN + pb * 16384 + sw128(r, hf * 4 + e8)) =
-                        h8(f, rflags);
+                        h8(f);
                 }
             }
             if (has_next && pt < C)
@@ -821,7 +844,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     const float x1 = in ? p.S0[sb + (size_t)(d0 + e + 1) * kDh + j] : 0.f;
                     r[e] = __float_as_uint(x0 * gam);
                     r[e + 1] = __float_as_uint(x1 * gam);
-                    hb[e >> 1] = h2(x0, x1, rflags);
+                    hb[e >> 1] = h2(x0, x1);
                 }
                 tmem_st32(tlane + TM_HM + d0, r);
                 tmem_st16(tlane + TM_HB + d0 / 2, hb);
@@ -831,10 +854,43 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             named_bar(kBarChain, 128);
             tc_fence_after();
         }
+        // The output of chunk c waits in TM_DO until iteration c + 1, which stores it straight
+        // from registers while its own V' product runs, off the state recursion's path.  It
+        // is held as bf16 pairs of consecutive tokens (one rounding of the fp32 result).
+        uint32_t ob[32];
+        auto load_o = [&]() {
+            uint32_t r[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                tmem_ld32(tlane + TM_DO + half * 32, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    omax = max_abs_nan(omax, u2f(r[2 * e]));
+                    omax = max_abs_nan(omax, u2f(r[2 * e + 1]));
+                    ob[half * 16 + e] = pack_bf16x2(u2f(r[2 * e]), u2f(r[2 * e + 1]));
+                }
+            }
+        };
+        // chunk cc's output, lane = dv index: each store of a warp writes 32 consecutive bf16 of
+        // one token's row (accumulating calls add the bf16 result to o and round the sum)
+        auto store_o = [&](int cc) {
+            const int Ccc = min(C, L - cc * C);
+            const long long tok0 = tokA + tstep * (long long)cc * C;
+#pragma unroll
+            for (int m = 0; m < C; ++m) {
+                if (m < Ccc && j < kDh) {
+                    const uint32_t pr = ob[m >> 1];
+                    __nv_bfloat16 y = __ushort_as_bfloat16((unsigned short)((m & 1) ? pr >> 16 : pr & 0xffffu));
+                    __nv_bfloat16* op = p.o + ((size_t)(tok0 + tstep * m) * p.Hv + h) * kDh + j;
+                    if (p.o_acc) y = __float2bfloat16_rn(__bfloat162float(y) + __bfloat162float(*op));
+                    *op = y;
+                }
+            }
+        };
         for (int c = 0; c < nchunks; ++c) {
             const int pb = c & 1;
             const uint32_t KQ = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
-            const int Cc = min(C, L - c * C);
             const bool has_next = c + 1 < nchunks;
             const int Cn = has_next ? min(C, L - (c + 1) * C) : 0;
             // loaded unconditionally from an in-bounds position, masked when reduced in C2
@@ -842,8 +898,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             if (has_next) g_raw = gate_bits_at(p.g, (c + 1) * C + min(lt & 63, Cn - 1));
 
             if (!wg_wait(MB_PREP + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
-            // C1: V'^T = U~^T + H^T (-W^T);  O^T = H^T Q~^T   (A = state copy in TMEM), once the
-            //     preparation's U~ product has landed (a failed wait skips the products: the
+            // C1: V'^T = U~^T + H^T (-W^T)  (A = fp16 state copy in TMEM), once the
+            //     preparation's U~ product has landed (a failed wait skips the product: the
             //     chain's next wait then gives up and the group agrees to stop)
             if (lt == 0 &&
                 mbar_wait_bounded(&SS.mbar[MB_MU], (uint32_t)(c & 1), kWaitLimitNs)) {
@@ -854,9 +910,15 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     mma_f32acc_ts(tmem + TM_DU + pb * 64, tmem + TM_HB + kk * 8,
                                   sdesc_sw128(sbase + OFF_WN + pb * 16384 + kk * 2048, 8192, 1024),
                                   id1, 1);
-                // V' is all C2 needs: its barrier fires before the output product runs; the
-                // commit after C3 covers the output product
                 mma_commit(&SS.mbar[MB_M1]);
+            }
+            // the previous chunk's output leaves TM_DO before this chunk's O^T = H^T Q~^T goes
+            // there; the state copy still holds this chunk's starting state
+            if (c > 0) load_o();
+            tc_fence_before();
+            named_bar(kBarChain, 128);
+            tc_fence_after();
+            if (lt == 0) {
                 const uint32_t id2 = idesc_f32acc(128, 64, false, false, false);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -865,6 +927,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                                   sdesc_sw128(KQ + off + 8192, 16, 1024), id2, kk > 0);
                 }
             }
+            if (c > 0) store_o(c - 1);
             if (!wg_wait(MB_M1, c & 1, kBarChain)) { fail = true; break; }
 
             // C2: V'^T -> fp16 packed in TMEM, plain (output) and scaled by Kd (state update)
@@ -880,12 +943,14 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
                         const float4 kd = *reinterpret_cast<const float4*>(&SS.Kd[pb][half * 32 + 4 * e4]);
-                        const float a0 = u2f(r[4 * e4]), b0 = u2f(r[4 * e4 + 1]);
-                        const float a1 = u2f(r[4 * e4 + 2]), b1 = u2f(r[4 * e4 + 3]);
-                        pk[2 * e4] = h2(a0, b0, rflags);
-                        pk[2 * e4 + 1] = h2(a1, b1, rflags);
-                        ps[2 * e4] = h2(a0 * kd.x, b0 * kd.y, rflags);
-                        ps[2 * e4 + 1] = h2(a1 * kd.z, b1 * kd.w, rflags);
+                        const float2 x0 = make_float2(u2f(r[4 * e4]), u2f(r[4 * e4 + 1]));
+                        const float2 x1 = make_float2(u2f(r[4 * e4 + 2]), u2f(r[4 * e4 + 3]));
+                        const float2 y0 = __fmul2_rn(x0, make_float2(kd.x, kd.y));
+                        const float2 y1 = __fmul2_rn(x1, make_float2(kd.z, kd.w));
+                        pk[2 * e4] = h2(x0.x, x0.y);
+                        pk[2 * e4 + 1] = h2(x1.x, x1.y);
+                        ps[2 * e4] = h2(y0.x, y0.y);
+                        ps[2 * e4 + 1] = h2(y1.x, y1.y);
                     }
                     tmem_st16(tlane + TM_VP + half * 16, pk);
                     tmem_st16(tlane + TM_VS + half * 16, ps);
@@ -900,75 +965,29 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             named_bar(kBarChain, 128);
             tc_fence_after();
 
-            // C3: O^T += V'^T P^T (N=64, K=64);  H^T += (Kd V')^T K (N=128, K=64, B MN-major)
+            // C3: H^T += (Kd V')^T K (N=128, K=64, B MN-major), committed on its own so the
+            //     state pass can start; then O^T += V'^T P^T (N=64, K=64)
             if (lt == 0) {
-                const uint32_t id3 = idesc_f32acc(128, 64, false, false, false);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_f32acc_ts(tmem + TM_DO, tmem + TM_VP + kk * 8,
-                                  sdesc_sw128(sbase + OFF_P + pb * 8192 + kk * 32, 16, 1024), id3, 1);
                 const uint32_t id4 = idesc_f32acc(128, 128, false, true, false);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f32acc_ts(tmem + TM_HM, tmem + TM_VS + kk * 8,
                                   sdesc_sw128(KQ + kk * 2048, 16384, 1024), id4, 1);
                 mma_commit(&SS.mbar[MB_M3 + pb]);
+                const uint32_t id3 = idesc_f32acc(128, 64, false, false, false);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f32acc_ts(tmem + TM_DO, tmem + TM_VP + kk * 8,
+                                  sdesc_sw128(sbase + OFF_P + pb * 8192 + kk * 32, 16, 1024), id3, 1);
+                mma_commit(&SS.mbar[MB_MO]);
             }
+            // the state update and everything issued before it (the products that read the
+            // state copy) are complete
             if (!wg_wait(MB_M3 + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
 
-            // C4: O -> staged in WN[pb] -> global (two tensor stores for a full chunk, else
-            //     coalesced 16-byte stores); state -> fp16 copy, pre-scaled for the next chunk
+            // C4: state -> fp16 copy, and the fp32 state pre-scaled by the next chunk's total
+            //     decay (the final state instead, after the last chunk)
             {
-                // staging: two [token][64] bf16 tiles (dv halves) in the 128-byte-swizzled
-                // layout of the output tensor map's box
-                uint8_t* stage = sm + OFF_WN + pb * 16384;
-                uint8_t* stage_j = stage + (j >> 6) * 8192 + (j & 7) * 2;
-                const int cj = (j & 63) >> 3;
-                uint32_t ro[2][32];
-                tmem_ld32(tlane + TM_DO, ro[0]);
-                tmem_ld32(tlane + TM_DO + 32, ro[1]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int half = 0; half < 2; ++half)
-#pragma unroll
-                    for (int m = 0; m < 32; ++m)
-                        *reinterpret_cast<__nv_bfloat16*>(stage_j + sw128(half * 32 + m, cj)) =
-                            __float2bfloat16_rn(u2f(ro[half][m]));
-                fence_proxy_async_smem();
-                named_bar(kBarChain, 128);
-                if (p.tma_store && Cc == C) {
-                    if (lt == 0) {
-                        const int z = (int)(t0 + (long long)c * C);
-                        const uint32_t src = sbase + OFF_WN + pb * 16384;
-                        tma_store_3d(&tm_o, src, 0, h, z);
-                        if (kDh > 64) tma_store_3d(&tm_o, src + 8192, 64, h, z);
-                        bulk_commit();
-                    }
-                } else {
-                // 16-byte chunks, consecutive threads on consecutive chunks of a row
-#pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const int idx = m * 128 + lt, row = idx >> 4, c16 = idx & 15;
-                    if (row < Cc && c16 < kDh / 8) {
-                        const long long tok = tokA + tstep * (long long)(c * C + row);
-                        uint4* dp = reinterpret_cast<uint4*>(p.o + ((size_t)tok * p.Hv + h) * kDh + c16 * 8);
-                        uint4 a = *reinterpret_cast<const uint4*>(stage + (c16 >> 3) * 8192 +
-                                                                  sw128(row, c16 & 7));
-                        if (p.o_acc) {
-                            const uint4 b = *dp;
-                            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
-                            uint32_t ow[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 x = unpack_bf16x2(aw[e]), y = unpack_bf16x2(bw[e]);
-                                ow[e] = pack_bf16x2(x.x + y.x, x.y + y.y);
-                            }
-                            a = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                        }
-                        *dp = a;
-                    }
-                }
-                }
                 const float gam = has_next ? ex2((SS.gsum_part[0] + SS.gsum_part[1]) * kLog2e) : 1.f;
 #pragma unroll
                 for (int d0 = 0; d0 < D; d0 += 64) {
@@ -980,37 +999,47 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     for (int hh = 0; hh < 2; ++hh) {
                         uint32_t (&r)[32] = r2[hh];
                         const int dd = d0 + hh * 32;
-                        uint32_t hb[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) hb[e] = h2(u2f(r[2 * e]), u2f(r[2 * e + 1]), rflags);
-                        tmem_st16(tlane + TM_HB + dd / 2, hb);
                         if (has_next) {
+                            uint32_t hb[16];
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(u2f(r[e]) * gam);
+                            for (int e = 0; e < 16; ++e) {
+                                const float2 x = make_float2(u2f(r[2 * e]), u2f(r[2 * e + 1]));
+                                hb[e] = h2(x.x, x.y);
+                                const float2 y = __fmul2_rn(x, make_float2(gam, gam));
+                                r[2 * e] = __float_as_uint(y.x);
+                                r[2 * e + 1] = __float_as_uint(y.y);
+                            }
+                            tmem_st16(tlane + TM_HB + dd / 2, hb);
                             tmem_st32(tlane + TM_HM + dd, r);
-                        } else if (p.S_final) {
+                        } else {
 #pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                if (dd + e < kDh && j < kDh)
+                            for (int e = 0; e < 32; ++e) {
+                                omax = max_abs_nan(omax, u2f(r[e]));
+                                if (p.S_final && dd + e < kDh && j < kDh)
                                     p.S_final[sb + (size_t)(dd + e) * kDh + j] = u2f(r[e]);
+                            }
                         }
                     }
                 }
                 tmem_wait_st();
-                if (lt == 0) bulk_wait_read();  // the staging buffer is free for reuse
-                mbar_arrive(&SS.mbar[MB_CD + pb]);
             }
+            // the output product has read P and Q~: the chunk's buffers are free
+            if (!wg_wait(MB_MO, c & 1, kBarChain)) { fail = true; break; }
             tc_fence_before();
+            mbar_arrive(&SS.mbar[MB_CD + pb]);
             named_bar(kBarChain, 128);
             tc_fence_after();
         }
+        if (!fail && nchunks > 0) {
+            load_o();
+            store_o(nchunks - 1);
+        }
     }
 
-    if (tid == 0) bulk_wait_all();  // output tiles written before the CTA exits
     if (fail && (tid == 0 || tid == 128 || tid == 256)) atomicExch(&p.hdr->err, (int)GDR_ERR_TIMEOUT);
     tc_fence_before();
-    rbad = rbad || !(__low2float(rflags) <= 65504.f) || !(__high2float(rflags) <= 65504.f);
-    if (__syncthreads_or(rbad ? 1 : 0) && tid == 0)
+    // an fp16 operand that left its range shows as a non-finite output or final state
+    if (__syncthreads_or(omax <= 3.4e38f ? 0 : 1) && tid == 0)
         atomicCAS(&p.hdr->err, (int)GDR_OK, (int)GDR_ERR_RANGE);
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
     griddep_wait();
@@ -1097,32 +1126,29 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
     p.o = static_cast<__nv_bfloat16*>(o); p.S_final = S_final;
     p.hdr = reinterpret_cast<WsHeader*>(base);
     p.cu = reinterpret_cast<const int32_t*>(base + L.cu);
+    p.order = reinterpret_cast<const int32_t*>(base + L.order);
     p.Hk = a.Hk; p.Hv = a.Hv; p.read_pre = a.read_mode == GDR_READ_PRE;
     p.qk_l2norm = a.qk_l2norm; p.reverse = a.reverse; p.o_acc = a.o_accumulate;
     p.gt = a.gate_dtype; p.scale = a.scale;
     const GateParams gp{a.gate_A, a.gate_dt_bias, a.beta_scale};
-    CUtensorMap tq, tk, tv, to;
+    CUtensorMap tq, tk, tv;
     memset(&tq, 0, sizeof(tq));
     memset(&tk, 0, sizeof(tk));
     memset(&tv, 0, sizeof(tv));
-    memset(&to, 0, sizeof(to));
     const long long T_tot = (long long)a.B * a.T;
     p.use_tma = 0;
-    p.tma_store = 0;
     if (!a.reverse && T_tot > 0) {  // reversed scans gather rows with cp.async instead
         if (!make_tile_map(&tq, q, a.Hk, T_tot, a.dk) || !make_tile_map(&tk, k, a.Hk, T_tot, a.dk) ||
             !make_tile_map(&tv, v, a.Hv, T_tot, a.dv))
             return GDR_ERR_CUDA;
         p.use_tma = 1;
-        // accumulating outputs are read back, so they keep the plain stores
-        p.tma_store = !a.o_accumulate && make_tile_map(&to, o, a.Hv, T_tot, a.dv);
     }
     auto kernel = a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D> : chunk_fused_tc<false, D>)
                             : (a.gate_raw ? chunk_fused_tc<true, 64> : chunk_fused_tc<false, 64>);
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
-    dim3 grid((unsigned)a.n_seqs, (unsigned)a.Hv);
+    dim3 grid((unsigned)a.n_seqs * (unsigned)a.Hv);
     if (dependent) {  // may start while the stream's previous grid finishes (see the kernel)
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = grid;
@@ -1134,10 +1160,10 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, kernel, p, tq, tk, tv, to, gp) != cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, kernel, p, tq, tk, tv, gp) != cudaSuccess)
             return GDR_ERR_CUDA;
     } else {
-        kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p, tq, tk, tv, to, gp);
+        kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p, tq, tk, tv, gp);
     }
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }

@@ -70,9 +70,14 @@ struct WsHeader {
 };
 
 struct WsLayout {
-    size_t cu, chunk_off, chunk_seq, W, U, G, Qt, Kt, Pc, total;
+    size_t cu, chunk_off, chunk_seq, order, W, U, G, Qt, Kt, Pc, total;
     long long max_chunks;
 };
+
+// Sequences a per-(sequence, head) kernel visits in order of decreasing length (varlen calls
+// of at most this many sequences; otherwise, and without cu_seqlens, in index order), so
+// that the longest sequences start in the first wave and none is left for the last.
+constexpr int kOrderMaxSeqs = 1024;
 
 // The register-blocked CUDA-core scan (chunk_scan_rb) splits a chunk's rows and the state's
 // dk rows over 8 warps, the latter in float4s: chunk <= 64, dk a multiple of 32 up to 128.
@@ -91,6 +96,7 @@ inline WsLayout ws_layout(const gdr_chunk_args& a, bool simt) {
     L.cu = off;        off = align_up(off + sizeof(int32_t) * (a.n_seqs + 1), 256);
     L.chunk_off = off; off = align_up(off + sizeof(int32_t) * (a.n_seqs + 1), 256);
     L.chunk_seq = off; off = align_up(off + sizeof(int32_t) * (size_t)L.max_chunks, 256);
+    L.order = off;     off = align_up(off + sizeof(int32_t) * (size_t)a.n_seqs, 256);
     if (simt) {
         L.W = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv * a.dk, 256);
         L.U = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv * a.dv, 256);

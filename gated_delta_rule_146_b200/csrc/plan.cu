@@ -1,11 +1,13 @@
 // plan.cu -- builds the chunk map of a forward call on the device.
 //
-// Chunks restart at every sequence start and the last chunk of a sequence may be
-// short (Prizma "seq/delta.py", chunked_delta: c1 = min(c0 + chunk, T); flashrt
-// fused_layer.py `_prefill_chain`: s1 = min(s0 + 64, S)).  Packed sequences are
-// delimited by cu_seqlens (tiny_gdn/fugue.py `segment_layout`).  The map is built
-// without any host synchronisation: grids downstream are sized by the upper bound
-// ceil(T_total / chunk) + n_seqs and surplus blocks exit.
+// Chunks restart at every sequence start and the last chunk of a sequence may be short
+// (Prizma "seq/delta.py", chunked_delta: the chunk loop clips each chunk's end at the
+// sequence length; flashrt fused_layer.py, `_prefill_chain`: the same clipping of its
+// 64-token spans).  Packed sequences are delimited by cu_seqlens (tiny_gdn/fugue.py
+// `segment_layout`).  The map is built without any host synchronisation: grids downstream
+// are sized by the upper bound ceil(T_total / chunk) + n_seqs and surplus blocks exit.
+// It also holds the order in which per-(sequence, head) kernels visit the sequences:
+// longest first for varlen calls, so the long ones do not end up in the last wave.
 #include "common.cuh"
 
 namespace gdr {
@@ -17,9 +19,10 @@ constexpr int kPlanThreads = 1024;
 __global__ void __launch_bounds__(kPlanThreads)
 plan_kernel(const int32_t* __restrict__ cu_in, int n_seqs, int B, int T, int chunk,
             WsHeader* __restrict__ hdr, int32_t* __restrict__ cu, int32_t* __restrict__ chunk_off,
-            int32_t* __restrict__ chunk_seq, long long max_chunks) {
+            int32_t* __restrict__ chunk_seq, int32_t* __restrict__ order, long long max_chunks) {
     __shared__ int s_bad;
     __shared__ int s_warp[kPlanThreads / 32];
+    __shared__ int s_len[kOrderMaxSeqs];
     const int tid = threadIdx.x;
     if (tid == 0) s_bad = 0;
     __syncthreads();
@@ -84,6 +87,23 @@ plan_kernel(const int32_t* __restrict__ cu_in, int n_seqs, int B, int T, int chu
         }
         chunk_seq[c] = lo;
     }
+    // 4. visiting order: by decreasing length, ties by index (a stable rank of each sequence
+    //    among all of them), for varlen calls of at most kOrderMaxSeqs sequences
+    if (cu_in && n_seqs <= kOrderMaxSeqs) {
+        for (int s = tid; s < n_seqs; s += kPlanThreads) s_len[s] = cu[s + 1] - cu[s];
+        __syncthreads();
+        for (int s = tid; s < n_seqs; s += kPlanThreads) {
+            const int ls = s_len[s];
+            int rank = 0;
+            for (int t = 0; t < n_seqs; ++t) {
+                const int lt = s_len[t];
+                rank += (lt > ls) | ((lt == ls) & (t < s));
+            }
+            order[rank] = s;
+        }
+    } else {
+        for (int s = tid; s < n_seqs; s += kPlanThreads) order[s] = s;
+    }
     if (tid == 0) {
         hdr->n_chunks = total;
         hdr->err = (total <= max_chunks) ? GDR_OK : GDR_ERR_DEVICE_CHECK;
@@ -98,7 +118,8 @@ cudaError_t launch_plan(const gdr_chunk_args& a, const int32_t* cu_in, void* ws,
     plan_kernel<<<1, kPlanThreads, 0, st>>>(
         cu_in, a.n_seqs, a.B, a.T, a.chunk, reinterpret_cast<WsHeader*>(base),
         reinterpret_cast<int32_t*>(base + L.cu), reinterpret_cast<int32_t*>(base + L.chunk_off),
-        reinterpret_cast<int32_t*>(base + L.chunk_seq), L.max_chunks);
+        reinterpret_cast<int32_t*>(base + L.chunk_seq), reinterpret_cast<int32_t*>(base + L.order),
+        L.max_chunks);
     return cudaGetLastError();
 }
 
