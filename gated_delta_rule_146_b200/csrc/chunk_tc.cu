@@ -107,8 +107,7 @@ enum {
     MB_LD = 7,    // x3: K, Q, V tiles of a chunk landed (by K/Q buffer)
     MB_CD = 10,   // x2: chain finished with a chunk's buffers (by chunk parity)
     MB_MU = 12,   // U~ product of a chunk done (awaited by the chain's MMA issuer)
-    MB_MO = 13,   // output products of a chunk done
-    MB_COUNT = 14
+    MB_COUNT = 13
 };
 
 struct Small {
@@ -119,7 +118,7 @@ struct Small {
     float Er[C];             // 2^(G_i - G_ref): row factor of the decay (K rows)
     float Eq[C];             // 2^(G'_i - G_ref): row factor for the read (G' = G_i or G_{i-1})
     float ck[C];             // column factor of [K;Q]K^T: 1/||k_j|| (x 2^(G_ref - G_j) when split)
-    float ssp[2][128];       // partial sums of squares of the [K;Q] row halves
+    float inv[128];          // 1 / ||row|| of [K;Q] (1 without normalisation)
     float gsum_part[2];      // chain: partial sums of the next chunk's g
     uint64_t mbar[MB_COUNT];
     uint32_t tmem_base;
@@ -135,6 +134,7 @@ struct TcParams {
     WsHeader* hdr; const int32_t* cu;
     const int32_t* order;  // sequences in visiting order (longest first for varlen calls)
     int Hk, Hv, read_pre, qk_l2norm, reverse, o_acc, use_tma;
+    int tma_store;  // full output chunks leave through the output tensor map
     gdr_dtype gt;
     float scale;
 };
@@ -192,7 +192,7 @@ template <bool kRaw, int kDh>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-               const GateParams gp) {
+               const __grid_constant__ CUtensorMap tm_o, const GateParams gp) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base, as a byte offset from the shared array so that every access
     // through it stays a shared-memory access (an integer round trip would make them generic)
@@ -300,6 +300,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
         const int r = pt & 127;        // TMEM lane / row of [K;Q] / dk or dv row
         const int hf = pt >> 7;        // which half of the columns this thread takes
         const int pw = pt >> 5;        // preparation warp 0..7
+        // P2's split of the rows: the two halves of a row sit in lanes l and l ^ 8 of one warp
+        // (eight rows per quarter warp, so the swizzled 16-byte accesses do not conflict)
+        const int r2 = ((pt >> 4) << 3) | (pt & 7), hf2 = (pt >> 3) & 1;
         // cp.async plan: this thread copies 16-byte column chunk `cd` of rows r0 + 16 m
         const int cd = pt & 15, r0 = pt >> 4;
         const bool cd_in = cd < kDh / 8;  // column chunks past a 64-wide head are zero-filled
@@ -378,6 +381,20 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 chunk_cumsum(2 * lane < Cc0 ? XG(gate_at(p.g, 2 * lane)) : 0.f,
                              2 * lane + 1 < Cc0 ? XG(gate_at(p.g, 2 * lane + 1)) : 0.f, 0);
         }
+        // P5, issued as the solve completes T's block columns: K-step kk of W^T = K^T T_w^T
+        // (into D0) and of U~^T = V^T T_u^T (into DU) reads block column kk of T_w and T_u
+        // only, so columns 3 and 2 go after phase 1, column 1 after phase 2 and column 0 (with
+        // the commits) after phase 3; the first K-step issued (kk = 3) starts each accumulator
+        auto issue_w = [&](uint32_t KQa, int pb_, int kk) {
+            mma_f32acc_ss(tmem + TM_D0, sdesc_sw128(KQa + kk * 2048, 16384, 1024),
+                          sdesc_sw128(sbase + OFF_WN + pb_ * 16384 + kk * 32, 16, 1024),
+                          idesc_f32acc(128, 64, true, false, false), kk < 3);
+        };
+        auto issue_u = [&](uint32_t VVa, int pb_, int kk) {
+            mma_f32acc_ss(tmem + TM_DU + pb_ * 64, sdesc_sw128(VVa + kk * 2048, 8192, 1024),
+                          sdesc_sw128(sbase + OFF_WN + pb_ * 16384 + 8192 + kk * 32, 16, 1024),
+                          idesc_f32acc(128, 64, true, false, false), kk < 3);
+        };
         // raw bits of the next chunk's gates: beta (one per thread), g (two per lane, warp 5)
         uint32_t b_nx = 0, g_nx0 = 0, g_nx1 = 0;
         for (int c = 0; c < nchunks; ++c) {
@@ -441,41 +458,41 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             //     (tensor tiles carry the following tokens there) become 0.  Stored over the
             //     bf16 tile once the product has read it.
             uint32_t hv[32];
-            float inv;  // 1 / ||row|| (1 without normalisation)
-            uint8_t* rowp = KQp + hf * 16384;
+            uint8_t* rowp = KQp + hf2 * 16384;  // this thread's half of row r2
             {
                 uint4 vals[8];
-                float ssq[4] = {0.f, 0.f, 0.f, 0.f};
+                float2 ssq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8)
-                    vals[c8] = *reinterpret_cast<const uint4*>(rowp + sw128(r, c8));
+                    vals[c8] = *reinterpret_cast<const uint4*>(rowp + sw128(r2, c8));
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
                     const uint32_t w[4] = {vals[c8].x, vals[c8].y, vals[c8].z, vals[c8].w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 x = unpack_bf16x2(w[e]);
-                        ssq[e] = fmaf(x.x, x.x, fmaf(x.y, x.y, ssq[e]));
+                        ssq[e & 1] = __ffma2_rn(x, x, ssq[e & 1]);
                     }
                 }
-                SS.ssp[hf][r] = (ssq[0] + ssq[1]) + (ssq[2] + ssq[3]);
-                named_bar(kBarPrep, kPrep);
-                const float tot = SS.ssp[0][r] + SS.ssp[1][r];
-                inv = p.qk_l2norm ? rsqrtf(fmaxf(tot, kNormEps * kNormEps)) : 1.f;
-                if (pt < C) {  // per-token factors; the column factor of D0 (K rows) is 1/||k_j||,
-                               // times 2^(G_ref - G_j) when split
+                float tot = (ssq[0].x + ssq[0].y) + (ssq[1].x + ssq[1].y);
+                tot += __shfl_xor_sync(0xffffffffu, tot, 8);  // the row's other half
+                const float inv = p.qk_l2norm ? rsqrtf(fmaxf(tot, kNormEps * kNormEps)) : 1.f;
+                if (hf2 == 0) SS.inv[r2] = inv;
+                if (hf2 == 0 && r2 < C) {  // per-token factors; the column factor of D0 (K rows)
+                                           // is 1/||k_j||, times 2^(G_ref - G_j) when split
+                    const int t = r2;
                     const float Gref = SS.G[pb][31];
-                    const float Gi = SS.G[pb][pt];
-                    const float Gr = p.read_pre ? (pt > 0 ? SS.G[pb][pt - 1] : 0.f) : Gi;
-                    SS.Kd[pb][pt] = pt < Cc ? ex2(SS.G[pb][Cc - 1] - Gi) : 0.f;
-                    SS.bg[pt] = SS.b[pb][pt] * ex2(Gi);
-                    SS.Er[pt] = ex2(Gi - Gref);
-                    SS.Eq[pt] = ex2(Gr - Gref);
-                    SS.ck[pt] = SS.split_ok[pb] ? ex2(Gref - Gi) * inv : inv;
+                    const float Gi = SS.G[pb][t];
+                    const float Gr = p.read_pre ? (t > 0 ? SS.G[pb][t - 1] : 0.f) : Gi;
+                    SS.Kd[pb][t] = t < Cc ? ex2(SS.G[pb][Cc - 1] - Gi) : 0.f;
+                    SS.bg[t] = SS.b[pb][t] * ex2(Gi);
+                    SS.Er[t] = ex2(Gi - Gref);
+                    SS.Eq[t] = ex2(Gr - Gref);
+                    SS.ck[t] = SS.split_ok[pb] ? ex2(Gref - Gi) * inv : inv;
                 }
-                const int i = r & 63;
+                const int i = r2 & 63;
                 float f = inv;
-                if (r >= C) {
+                if (r2 >= C) {
                     const float Gr = p.read_pre ? (i > 0 ? SS.G[pb][i - 1] : 0.f) : SS.G[pb][i];
                     f = p.scale * ex2(Gr) * inv;
                 }
@@ -485,28 +502,30 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     const uint32_t w[4] = {vals[c8].x, vals[c8].y, vals[c8].z, vals[c8].w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float2 x = unpack_bf16x2(w[e]);
-                        hv[c8 * 4 + e] = pack_f16x2(x.x * f, x.y * f);
+                        const float2 x = __fmul2_rn(unpack_bf16x2(w[e]), make_float2(f, f));
+                        hv[c8 * 4 + e] = pack_f16x2(x.x, x.y);
                     }
                 }
-                // V to fp16 in place (every bf16 value of the fp16 range is exact in fp16),
-                // rows past the chunk to zero; the swizzle only permutes the 16-byte pieces
-                // within a row, so a piece's row is its offset / 128
-                for (int idx = pt; idx < (kDh / 64) * 512; idx += kPrep) {
-                    uint4* vp = reinterpret_cast<uint4*>(sm + OFF_V + pb * V_STRIDE) + idx;
-                    if (((idx & 511) >> 3) >= Cc) {
-                        *vp = make_uint4(0, 0, 0, 0);
-                        continue;
-                    }
-                    const uint4 w = *vp;
-                    const uint32_t wi[4] = {w.x, w.y, w.z, w.w};
+                // V to fp16 in place, four 16-byte pieces per thread (every bf16 value of the
+                // fp16 range is exact in fp16), rows past the chunk to zero; the swizzle only
+                // permutes the pieces within a row, so a piece's row is its offset / 128
+                uint4* vt = reinterpret_cast<uint4*>(sm + OFF_V + pb * V_STRIDE);
+                constexpr int kVPieces = (kDh / 64) * 512 / kPrep;
+                uint4 vw[kVPieces];
+#pragma unroll
+                for (int m = 0; m < kVPieces; ++m) vw[m] = vt[pt + m * kPrep];
+#pragma unroll
+                for (int m = 0; m < kVPieces; ++m) {
+                    const int idx = pt + m * kPrep;
+                    const uint32_t wi[4] = {vw[m].x, vw[m].y, vw[m].z, vw[m].w};
                     uint32_t wo[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 xv = unpack_bf16x2(wi[e]);
                         wo[e] = h2(xv.x, xv.y);
                     }
-                    *vp = make_uint4(wo[0], wo[1], wo[2], wo[3]);
+                    vt[idx] = ((idx & 511) >> 3) < Cc ? make_uint4(wo[0], wo[1], wo[2], wo[3])
+                                                      : make_uint4(0, 0, 0, 0);
                 }
             }
             if (!wg_wait(MB_M0, c & 1, kBarPrep)) { fail = true; break; }
@@ -533,13 +552,13 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 }
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8)
-                    *reinterpret_cast<uint4*>(rowp + sw128(r, c8)) =
+                    *reinterpret_cast<uint4*>(rowp + sw128(r2, c8)) =
                         make_uint4(hv[c8 * 4], hv[c8 * 4 + 1], hv[c8 * 4 + 2], hv[c8 * 4 + 3]);
                 // row factor (beta_i / ||k_i|| or scale / ||q_i||, times 2^(G'_i - G_ref) when
                 // split) and, without the split, the per-element decay exponent's row part
                 const float Gi = r < C ? SS.G[pb][i]
                                        : (p.read_pre ? (i > 0 ? SS.G[pb][i - 1] : 0.f) : SS.G[pb][i]);
-                float fi = live ? (r < C ? SS.b[pb][i] : p.scale) * inv : 0.f;
+                float fi = live ? (r < C ? SS.b[pb][i] : p.scale) * SS.inv[r] : 0.f;
                 if (split) fi *= r < C ? SS.Er[i] : SS.Eq[i];
                 tmem_wait_ld();
                 float vals[32];
@@ -758,14 +777,30 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                             *reinterpret_cast<uint4*>(twu + 8192 + sw128(i, c8)) = make_uint4(0, 0, 0, 0);
                         }
                     }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
                     named_bar(kBarPrep, kPrep);
+                    if (pt == 192) {  // block columns 3 and 2 of T_w, T_u are complete
+                        tc_fence_after();
+                        issue_w(KQ, pb, 3);
+                        issue_w(KQ, pb, 2);
+                        issue_u(VV, pb, 3);
+                        issue_u(VV, pb, 2);
+                    }
                     if (pw >= 3 && pw < 6) {
                         frag_reg(a, E1);
                         if (pw == 3) { bprod(Y, a, Ts, 1, 0, true); store_neg(Ts, 2, 0, Y); put_twu(2, 0, Y); }
                         if (pw == 4) { bprod(Y, a, Ts, 2, 1, true); put_twu(3, 1, Y); }
                         if (pw == 5) bprod(Y, a, Ts, 1, 0, true);
                     }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
                     named_bar(kBarPrep, kPrep);
+                    if (pt == 192) {  // block column 1
+                        tc_fence_after();
+                        issue_w(KQ, pb, 1);
+                        issue_u(VV, pb, 1);
+                    }
                     if (pw == 5) {
                         const float4 x0 = *reinterpret_cast<const float4*>(e32);
                         const float4 x1 = *reinterpret_cast<const float4*>(e32 + 4);
@@ -782,21 +817,13 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             named_bar(kBarPrep, kPrep);
             tc_fence_after();
 
-            // P5: W^T = K^T T_w^T (into D0) and U~^T = V^T T_u^T (into DU[pb]), fp16 operands
-            if (pt == 0) {
-                const uint32_t idw = idesc_f32acc(128, 64, true, false, false);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_f32acc_ss(tmem + TM_D0, sdesc_sw128(KQ + kk * 2048, 16384, 1024),
-                                  sdesc_sw128(sbase + OFF_WN + pb * 16384 + kk * 32, 16, 1024), idw, kk > 0);
-                mma_commit(&SS.mbar[MB_MW]);  // W^T: all P6 needs
-                const uint32_t idu = idesc_f32acc(128, 64, true, false, false);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_f32acc_ss(tmem + TM_DU + pb * 64, sdesc_sw128(VV + kk * 2048, 8192, 1024),
-                                  sdesc_sw128(sbase + OFF_WN + pb * 16384 + 8192 + kk * 32, 16, 1024), idu,
-                                  kk > 0);
-                mma_commit(&SS.mbar[MB_MU]);  // U~^T: awaited by the chain before V' accumulates
+            // P5, last step: block column 0; the commit covers every K-step issued before (W^T
+            // for P6, U~^T for the chain, before V' accumulates onto it)
+            if (pt == 192) {
+                issue_w(KQ, pb, 0);
+                mma_commit(&SS.mbar[MB_MW]);
+                issue_u(VV, pb, 0);
+                mma_commit(&SS.mbar[MB_MU]);
             }
             if (!wg_wait(MB_MW, c & 1, kBarPrep)) { fail = true; break; }
 
@@ -834,7 +861,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             if (lane == 0 && warp < 2) SS.gsum_part[warp] = part;
             named_bar(kBarChain, 128);
             const float gam = ex2((SS.gsum_part[0] + SS.gsum_part[1]) * kLog2e);
-#pragma unroll
+#pragma unroll 1
             for (int d0 = 0; d0 < D; d0 += 32) {
                 uint32_t r[32], hb[16];
 #pragma unroll
@@ -854,43 +881,11 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             named_bar(kBarChain, 128);
             tc_fence_after();
         }
-        // The output of chunk c waits in TM_DO until iteration c + 1, which stores it straight
-        // from registers while its own V' product runs, off the state recursion's path.  It
-        // is held as bf16 pairs of consecutive tokens (one rounding of the fp32 result).
-        uint32_t ob[32];
-        auto load_o = [&]() {
-            uint32_t r[32];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tmem_ld32(tlane + TM_DO + half * 32, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    omax = max_abs_nan(omax, u2f(r[2 * e]));
-                    omax = max_abs_nan(omax, u2f(r[2 * e + 1]));
-                    ob[half * 16 + e] = pack_bf16x2(u2f(r[2 * e]), u2f(r[2 * e + 1]));
-                }
-            }
-        };
-        // chunk cc's output, lane = dv index: each store of a warp writes 32 consecutive bf16 of
-        // one token's row (accumulating calls add the bf16 result to o and round the sum)
-        auto store_o = [&](int cc) {
-            const int Ccc = min(C, L - cc * C);
-            const long long tok0 = tokA + tstep * (long long)cc * C;
-#pragma unroll
-            for (int m = 0; m < C; ++m) {
-                if (m < Ccc && j < kDh) {
-                    const uint32_t pr = ob[m >> 1];
-                    __nv_bfloat16 y = __ushort_as_bfloat16((unsigned short)((m & 1) ? pr >> 16 : pr & 0xffffu));
-                    __nv_bfloat16* op = p.o + ((size_t)(tok0 + tstep * m) * p.Hv + h) * kDh + j;
-                    if (p.o_acc) y = __float2bfloat16_rn(__bfloat162float(y) + __bfloat162float(*op));
-                    *op = y;
-                }
-            }
-        };
+        const bool check_o = !p.qk_l2norm || !(fabsf(p.scale) <= 1024.f);
         for (int c = 0; c < nchunks; ++c) {
             const int pb = c & 1;
             const uint32_t KQ = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
+            const int Cc = min(C, L - c * C);
             const bool has_next = c + 1 < nchunks;
             const int Cn = has_next ? min(C, L - (c + 1) * C) : 0;
             // loaded unconditionally from an in-bounds position, masked when reduced in C2
@@ -898,8 +893,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             if (has_next) g_raw = gate_bits_at(p.g, (c + 1) * C + min(lt & 63, Cn - 1));
 
             if (!wg_wait(MB_PREP + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
-            // C1: V'^T = U~^T + H^T (-W^T)  (A = fp16 state copy in TMEM), once the
-            //     preparation's U~ product has landed (a failed wait skips the product: the
+            // C1: V'^T = U~^T + H^T (-W^T);  O^T = H^T Q~^T   (A = state copy in TMEM), once the
+            //     preparation's U~ product has landed (a failed wait skips the products: the
             //     chain's next wait then gives up and the group agrees to stop)
             if (lt == 0 &&
                 mbar_wait_bounded(&SS.mbar[MB_MU], (uint32_t)(c & 1), kWaitLimitNs)) {
@@ -910,15 +905,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     mma_f32acc_ts(tmem + TM_DU + pb * 64, tmem + TM_HB + kk * 8,
                                   sdesc_sw128(sbase + OFF_WN + pb * 16384 + kk * 2048, 8192, 1024),
                                   id1, 1);
+                // V' is all C2 needs: its barrier fires before the output product runs; the
+                // commit after C3 covers the output product
                 mma_commit(&SS.mbar[MB_M1]);
-            }
-            // the previous chunk's output leaves TM_DO before this chunk's O^T = H^T Q~^T goes
-            // there; the state copy still holds this chunk's starting state
-            if (c > 0) load_o();
-            tc_fence_before();
-            named_bar(kBarChain, 128);
-            tc_fence_after();
-            if (lt == 0) {
                 const uint32_t id2 = idesc_f32acc(128, 64, false, false, false);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -927,7 +916,6 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                                   sdesc_sw128(KQ + off + 8192, 16, 1024), id2, kk > 0);
                 }
             }
-            if (c > 0) store_o(c - 1);
             if (!wg_wait(MB_M1, c & 1, kBarChain)) { fail = true; break; }
 
             // C2: V'^T -> fp16 packed in TMEM, plain (output) and scaled by Kd (state update)
@@ -943,14 +931,12 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
                         const float4 kd = *reinterpret_cast<const float4*>(&SS.Kd[pb][half * 32 + 4 * e4]);
-                        const float2 x0 = make_float2(u2f(r[4 * e4]), u2f(r[4 * e4 + 1]));
-                        const float2 x1 = make_float2(u2f(r[4 * e4 + 2]), u2f(r[4 * e4 + 3]));
-                        const float2 y0 = __fmul2_rn(x0, make_float2(kd.x, kd.y));
-                        const float2 y1 = __fmul2_rn(x1, make_float2(kd.z, kd.w));
-                        pk[2 * e4] = h2(x0.x, x0.y);
-                        pk[2 * e4 + 1] = h2(x1.x, x1.y);
-                        ps[2 * e4] = h2(y0.x, y0.y);
-                        ps[2 * e4 + 1] = h2(y1.x, y1.y);
+                        const float a0 = u2f(r[4 * e4]), b0 = u2f(r[4 * e4 + 1]);
+                        const float a1 = u2f(r[4 * e4 + 2]), b1 = u2f(r[4 * e4 + 3]);
+                        pk[2 * e4] = h2(a0, b0);
+                        pk[2 * e4 + 1] = h2(a1, b1);
+                        ps[2 * e4] = h2(a0 * kd.x, b0 * kd.y);
+                        ps[2 * e4 + 1] = h2(a1 * kd.z, b1 * kd.w);
                     }
                     tmem_st16(tlane + TM_VP + half * 16, pk);
                     tmem_st16(tlane + TM_VS + half * 16, ps);
@@ -965,41 +951,93 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             named_bar(kBarChain, 128);
             tc_fence_after();
 
-            // C3: H^T += (Kd V')^T K (N=128, K=64, B MN-major), committed on its own so the
-            //     state pass can start; then O^T += V'^T P^T (N=64, K=64)
+            // C3: O^T += V'^T P^T (N=64, K=64);  H^T += (Kd V')^T K (N=128, K=64, B MN-major)
             if (lt == 0) {
+                const uint32_t id3 = idesc_f32acc(128, 64, false, false, false);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f32acc_ts(tmem + TM_DO, tmem + TM_VP + kk * 8,
+                                  sdesc_sw128(sbase + OFF_P + pb * 8192 + kk * 32, 16, 1024), id3, 1);
                 const uint32_t id4 = idesc_f32acc(128, 128, false, true, false);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f32acc_ts(tmem + TM_HM, tmem + TM_VS + kk * 8,
                                   sdesc_sw128(KQ + kk * 2048, 16384, 1024), id4, 1);
                 mma_commit(&SS.mbar[MB_M3 + pb]);
-                const uint32_t id3 = idesc_f32acc(128, 64, false, false, false);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_f32acc_ts(tmem + TM_DO, tmem + TM_VP + kk * 8,
-                                  sdesc_sw128(sbase + OFF_P + pb * 8192 + kk * 32, 16, 1024), id3, 1);
-                mma_commit(&SS.mbar[MB_MO]);
             }
-            // the state update and everything issued before it (the products that read the
-            // state copy) are complete
             if (!wg_wait(MB_M3 + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
 
-            // C4: state -> fp16 copy, and the fp32 state pre-scaled by the next chunk's total
-            //     decay (the final state instead, after the last chunk)
+            // C4: O -> staged in WN[pb] -> global (two tensor stores for a full chunk, else
+            //     coalesced 16-byte stores); state -> fp16 copy, pre-scaled for the next chunk
             {
+                // staging: two [token][64] bf16 tiles (dv halves) in the 128-byte-swizzled
+                // layout of the output tensor map's box
+                uint8_t* stage = sm + OFF_WN + pb * 16384;
+                uint8_t* stage_j = stage + (j >> 6) * 8192 + (j & 7) * 2;
+                const int cj = (j & 63) >> 3;
+                uint32_t ro[2][32];
+                tmem_ld32(tlane + TM_DO, ro[0]);
+                tmem_ld32(tlane + TM_DO + 32, ro[1]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int half = 0; half < 2; ++half)
+#pragma unroll
+                    for (int m = 0; m < 32; ++m)
+                        *reinterpret_cast<__nv_bfloat16*>(stage_j + sw128(half * 32 + m, cj)) =
+                            __float2bfloat16_rn(u2f(ro[half][m]));
+                // with normalised q, k and |scale| <= 1024 the operands that reach only the
+                // output (P, Q~) are bounded by |scale|; otherwise every output is checked
+                if (check_o) {
+#pragma unroll
+                    for (int m = 0; m < 64; ++m) omax = max_abs_nan(omax, u2f(ro[m >> 5][m & 31]));
+                }
+                fence_proxy_async_smem();
+                named_bar(kBarChain, 128);
+                if (p.tma_store && Cc == C) {
+                    if (lt == 0) {
+                        const int z = (int)(t0 + (long long)c * C);
+                        const uint32_t src = sbase + OFF_WN + pb * 16384;
+                        tma_store_3d(&tm_o, src, 0, h, z);
+                        if (kDh > 64) tma_store_3d(&tm_o, src + 8192, 64, h, z);
+                        bulk_commit();
+                    }
+                } else {
+                // 16-byte chunks, consecutive threads on consecutive chunks of a row
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const int idx = m * 128 + lt, row = idx >> 4, c16 = idx & 15;
+                    if (row < Cc && c16 < kDh / 8) {
+                        const long long tok = tokA + tstep * (long long)(c * C + row);
+                        uint4* dp = reinterpret_cast<uint4*>(p.o + ((size_t)tok * p.Hv + h) * kDh + c16 * 8);
+                        uint4 a = *reinterpret_cast<const uint4*>(stage + (c16 >> 3) * 8192 +
+                                                                  sw128(row, c16 & 7));
+                        if (p.o_acc) {
+                            const uint4 b = *dp;
+                            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+                            uint32_t ow[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 x = unpack_bf16x2(aw[e]), y = unpack_bf16x2(bw[e]);
+                                ow[e] = pack_bf16x2(x.x + y.x, x.y + y.y);
+                            }
+                            a = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                        }
+                        *dp = a;
+                    }
+                }
+                }
                 const float gam = has_next ? ex2((SS.gsum_part[0] + SS.gsum_part[1]) * kLog2e) : 1.f;
+                if (has_next) {
 #pragma unroll
-                for (int d0 = 0; d0 < D; d0 += 64) {
-                    uint32_t r2[2][32];
-                    tmem_ld32(tlane + TM_HM + d0, r2[0]);
-                    tmem_ld32(tlane + TM_HM + d0 + 32, r2[1]);
-                    tmem_wait_ld();
+                    for (int d0 = 0; d0 < D; d0 += 64) {
+                        uint32_t r2[2][32];
+                        tmem_ld32(tlane + TM_HM + d0, r2[0]);
+                        tmem_ld32(tlane + TM_HM + d0 + 32, r2[1]);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t (&r)[32] = r2[hh];
-                        const int dd = d0 + hh * 32;
-                        if (has_next) {
+                        for (int hh = 0; hh < 2; ++hh) {
+                            uint32_t (&r)[32] = r2[hh];
+                            const int dd = d0 + hh * 32;
                             uint32_t hb[16];
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
@@ -1011,31 +1049,35 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                             }
                             tmem_st16(tlane + TM_HB + dd / 2, hb);
                             tmem_st32(tlane + TM_HM + dd, r);
-                        } else {
+                        }
+                    }
+                } else {
+                    // the final state, once per sequence (column j of the transposed state);
+                    // an operand that left the fp16 range on the state's path shows here
+#pragma unroll 1
+                    for (int d0 = 0; d0 < kDh; d0 += 32) {
+                        uint32_t r[32];
+                        tmem_ld32(tlane + TM_HM + d0, r);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) {
-                                omax = max_abs_nan(omax, u2f(r[e]));
-                                if (p.S_final && dd + e < kDh && j < kDh)
-                                    p.S_final[sb + (size_t)(dd + e) * kDh + j] = u2f(r[e]);
-                            }
+                        for (int e = 0; e < 32; ++e) {
+                            omax = max_abs_nan(omax, u2f(r[e]));
+                            if (p.S_final && j < kDh)
+                                p.S_final[sb + (size_t)(d0 + e) * kDh + j] = u2f(r[e]);
                         }
                     }
                 }
                 tmem_wait_st();
+                if (lt == 0) bulk_wait_read();  // the staging buffer is free for reuse
+                mbar_arrive(&SS.mbar[MB_CD + pb]);
             }
-            // the output product has read P and Q~: the chunk's buffers are free
-            if (!wg_wait(MB_MO, c & 1, kBarChain)) { fail = true; break; }
             tc_fence_before();
-            mbar_arrive(&SS.mbar[MB_CD + pb]);
             named_bar(kBarChain, 128);
             tc_fence_after();
         }
-        if (!fail && nchunks > 0) {
-            load_o();
-            store_o(nchunks - 1);
-        }
     }
 
+    if (tid == 0) bulk_wait_all();  // output tiles written before the CTA exits
     if (fail && (tid == 0 || tid == 128 || tid == 256)) atomicExch(&p.hdr->err, (int)GDR_ERR_TIMEOUT);
     tc_fence_before();
     // an fp16 operand that left its range shows as a non-finite output or final state
@@ -1131,17 +1173,21 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
     p.qk_l2norm = a.qk_l2norm; p.reverse = a.reverse; p.o_acc = a.o_accumulate;
     p.gt = a.gate_dtype; p.scale = a.scale;
     const GateParams gp{a.gate_A, a.gate_dt_bias, a.beta_scale};
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     memset(&tq, 0, sizeof(tq));
     memset(&tk, 0, sizeof(tk));
     memset(&tv, 0, sizeof(tv));
+    memset(&to, 0, sizeof(to));
     const long long T_tot = (long long)a.B * a.T;
     p.use_tma = 0;
+    p.tma_store = 0;
     if (!a.reverse && T_tot > 0) {  // reversed scans gather rows with cp.async instead
         if (!make_tile_map(&tq, q, a.Hk, T_tot, a.dk) || !make_tile_map(&tk, k, a.Hk, T_tot, a.dk) ||
             !make_tile_map(&tv, v, a.Hv, T_tot, a.dv))
             return GDR_ERR_CUDA;
         p.use_tma = 1;
+        // accumulating outputs are read back, so they keep the plain stores
+        p.tma_store = !a.o_accumulate && make_tile_map(&to, o, a.Hv, T_tot, a.dv);
     }
     auto kernel = a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D> : chunk_fused_tc<false, D>)
                             : (a.gate_raw ? chunk_fused_tc<true, 64> : chunk_fused_tc<false, 64>);
@@ -1160,10 +1206,10 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, kernel, p, tq, tk, tv, gp) != cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, kernel, p, tq, tk, tv, to, gp) != cudaSuccess)
             return GDR_ERR_CUDA;
     } else {
-        kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p, tq, tk, tv, gp);
+        kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p, tq, tk, tv, to, gp);
     }
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }

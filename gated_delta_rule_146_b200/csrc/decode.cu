@@ -10,7 +10,9 @@
 //     pre:  o = scale s_q
 // and, when the output epilogue is fused (the decode chain's gated RMSNorm, flashrt
 // fused_layer.py `_decode_one`), o <- o / sqrt(mean(o^2) + eps) * weight * silu(z) over
-// the head's dv values; that variant gives each block a whole head (DVS = DV).
+// the head's dv values; the blocks of one head's column slices then form a thread-block
+// cluster and add their partial sums of squares through distributed shared memory, so the
+// normalised variant keeps the plain one's slice size (and its registers and occupancy).
 // GDN-2 (decoupled gates, tiny_gdn/fugue.py BidirectionalGatedDeltaNet2) in the same pass:
 // with per-row decay e^{g_d} and erase gate b_d and per-column write gate w_j,
 //     s_k = H^T (e^g . b . k),  u = w . v - s_k,  H <- e^g . H + k u^T,
@@ -21,6 +23,8 @@
 // shared memory across warps), and writes the updated slice back from the same
 // registers.  Each block reads all of its slice before writing any of it, so the
 // update in place needs no scratch copy of the state.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 namespace gdr {
@@ -47,7 +51,7 @@ struct DecodeParams {
 template <int DK, int DV, int DVS, bool kNorm, bool kG2>
 __global__ void __launch_bounds__(kThreads)
 decode_kernel(DecodeParams p) {
-    static_assert(!kNorm || DVS == DV, "the normed epilogue needs the whole head in a block");
+    constexpr int CL = DV / DVS;           // blocks per head (the cluster, when kNorm)
     constexpr int CPR = DVS / 4;           // float4 column groups per row slice
     constexpr int RPW = 32 / CPR;          // rows a warp covers per pass
     constexpr int RPP = RPW * kWarps;      // rows per pass over the block
@@ -61,6 +65,7 @@ decode_kernel(DecodeParams p) {
     __shared__ float s_o[kNorm ? DVS : 1];        // recurrent output of the head (epilogue)
     __shared__ float s_eg[kG2 ? DK : 1], s_b[kG2 ? DK : 1];  // GDN-2: e^{g_d}, b_d per row
     __shared__ float s_ss[kWarps];
+    __shared__ float s_part[CL];                  // the cluster's partial sums of o^2
 
     const int nh = blockIdx.x;                   // n * Hv + h
     const int J = blockIdx.y;                    // column slice
@@ -164,21 +169,39 @@ decode_kernel(DecodeParams p) {
     }
     __syncthreads();
     if constexpr (kNorm) {
-        // gated RMSNorm over the head: o_j / sqrt(mean(o^2) + eps) * weight_j * silu(z_j)
-        if (wid * 32 < DV) {
-            const float x = tid < DV ? s_o[tid] : 0.f;
+        // gated RMSNorm over the head: o_j / sqrt(mean(o^2) + eps) * weight_j * silu(z_j);
+        // this block's slice gives a partial sum of o^2, which its first thread writes into
+        // slot J of every block of the cluster (the head's slices, J = rank in the cluster)
+        if (wid * 32 < DVS) {
+            const float x = tid < DVS ? s_o[tid] : 0.f;
             const float ss = warp_sum(x * x);
             if (lane == 0) s_ss[wid] = ss;
         }
         __syncthreads();
-        if (tid < DV) {
+        if (tid == 0) {
             float ss = 0.f;
 #pragma unroll
-            for (int w = 0; w < (DV + 31) / 32; ++w) ss += s_ss[w];
-            const float r = rsqrtf(ss / DV + p.norm_eps);
-            const float z = load_elem(p.norm_z, (size_t)nh * DV + tid, p.io);
+            for (int w = 0; w < (DVS + 31) / 32; ++w) ss += s_ss[w];
+            if constexpr (CL > 1) {
+                cooperative_groups::cluster_group cl = cooperative_groups::this_cluster();
+#pragma unroll
+                for (int r = 0; r < CL; ++r) cl.map_shared_rank(s_part, r)[J] = ss;
+            } else {
+                s_part[0] = ss;
+            }
+        }
+        // every block's partial has arrived (and nothing reads another block's memory after)
+        if constexpr (CL > 1) cooperative_groups::this_cluster().sync();
+        else __syncthreads();
+        if (tid < DVS) {
+            float ss = 0.f;
+#pragma unroll
+            for (int r = 0; r < CL; ++r) ss += s_part[r];
+            const int col = J * DVS + tid;
+            const float rr = rsqrtf(ss / DV + p.norm_eps);
+            const float z = load_elem(p.norm_z, (size_t)nh * DV + col, p.io);
             const float silu = z / (1.f + expf(-z));
-            store_elem(p.o, (size_t)nh * DV + tid, s_o[tid] * r * p.norm_weight[tid] * silu, p.io);
+            store_elem(p.o, (size_t)nh * DV + col, s_o[tid] * rr * p.norm_weight[col] * silu, p.io);
         }
     }
     const float4 u4 = *reinterpret_cast<const float4*>(&s_u[cg * 4]);
@@ -193,14 +216,33 @@ decode_kernel(DecodeParams p) {
     }
 }
 
+// The normed epilogue reduces over the head's dv values: its slices of one head run as one
+// thread-block cluster (DV / DVS blocks along y).
+template <int DK, int DV, int DVS, bool kG2>
+gdr_status launch_norm(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = DV / DVS;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_kernel<DK, DV, DVS, true, kG2>, p) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
 template <int DK, int DV>
 gdr_status launch_dv(const gdr_decode_args& a, const DecodeParams& p, cudaStream_t st) {
     constexpr int DVS = DV >= 64 ? 64 : 32;
-    const dim3 whole((unsigned)(a.N * a.Hv), 1), sliced((unsigned)(a.N * a.Hv), DV / DVS);
-    // the normed epilogue takes one block per (sequence, head): it reduces over dv
-    if (a.out_norm && a.gdn2) decode_kernel<DK, DV, DV, true, true><<<whole, kThreads, 0, st>>>(p);
-    else if (a.out_norm) decode_kernel<DK, DV, DV, true, false><<<whole, kThreads, 0, st>>>(p);
-    else if (a.gdn2) decode_kernel<DK, DV, DVS, false, true><<<sliced, kThreads, 0, st>>>(p);
+    const dim3 sliced((unsigned)(a.N * a.Hv), DV / DVS);
+    if (a.out_norm && a.gdn2) return launch_norm<DK, DV, DVS, true>(p, sliced, st);
+    if (a.out_norm) return launch_norm<DK, DV, DVS, false>(p, sliced, st);
+    if (a.gdn2) decode_kernel<DK, DV, DVS, false, true><<<sliced, kThreads, 0, st>>>(p);
     else decode_kernel<DK, DV, DVS, false, false><<<sliced, kThreads, 0, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
