@@ -101,13 +101,14 @@ constexpr uint32_t TM_COLS = 512;
 
 // mbarriers
 enum {
-    MB_M0 = 0, MB_MW = 1, MB_M1 = 2,
+    MB_M0 = 0, MB_M1 = 2,  // (index 1 unused)
     MB_M3 = 3,    // x2: state update of a chunk done (by chunk parity)
     MB_PREP = 5,  // x2: chunk prepared (by chunk parity)
     MB_LD = 7,    // x3: K, Q, V tiles of a chunk landed (by K/Q buffer)
     MB_CD = 10,   // x2: chain finished with a chunk's buffers (by chunk parity)
-    MB_MU = 12,   // U~ product of a chunk done (awaited by the chain's MMA issuer)
-    MB_COUNT = 13
+    MB_MU = 12,   // W and U~ products of a chunk done (awaited by the chain)
+    MB_D0F = 13,  // the chain has read W^T out of D0 (the next [K;Q]K^T may overwrite it)
+    MB_COUNT = 14
 };
 
 struct Small {
@@ -244,9 +245,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     }
     if (tid == 0) {
         for (int i = 0; i < MB_COUNT; ++i)
-            mbar_init(&SS.mbar[i], (i == MB_PREP || i == MB_PREP + 1) ? kPrep
-                                   : (i == MB_CD || i == MB_CD + 1)  ? 128
-                                                                     : 1);
+            mbar_init(&SS.mbar[i], (i == MB_PREP || i == MB_PREP + 1)              ? kPrep
+                                   : (i == MB_CD || i == MB_CD + 1 || i == MB_D0F) ? 128
+                                                                                   : 1);
         SS.gflag[0][0] = SS.gflag[0][1] = SS.gflag[1][0] = SS.gflag[1][1] = 0;
         mbar_init_fence();
     }
@@ -405,17 +406,16 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             const int Cc = min(C, L - c * C);
             const bool has_next = c + 1 < nchunks;
 
-            // P0: the buffers of chunk c-2 are released once the chain is done with them.  Either
-            //     barrier also publishes this chunk's beta and cumulative decay (stored during
-            //     the previous chunk's preparation, or before the loop).
-            if (c >= 2) {
-                if (!wg_wait(MB_CD + pb, ((c >> 1) & 1) ^ 1, kBarPrep)) { fail = true; break; }
-            } else {
-                named_bar(kBarPrep, kPrep);
-            }
+            // P0: the buffers of chunk c-2 are released once the chain is done with them (each
+            //     thread sees it on the mbarrier before its own copies into them); the one
+            //     group barrier below, after this chunk's tiles have landed, also publishes this
+            //     chunk's beta and cumulative decay (stored during the previous chunk's
+            //     preparation, or before the loop)
+            bool ok = true;
+            if (c >= 2) ok = mbar_wait_bounded(&SS.mbar[MB_CD + pb], ((c >> 1) & 1) ^ 1, kWaitLimitNs);
             int Cn = 0;
             if (has_next) {
-                if (!p.use_tma) load_chunk(c + 1);  // reversed scans: every thread's row copies
+                if (!p.use_tma && ok) load_chunk(c + 1);  // reversed scans: every thread's row copies
                 // in-bounds positions for every thread, masked only where the values are used
                 // (a select on a just-loaded value would wait for the load right here)
                 Cn = min(C, L - (c + 1) * C);
@@ -448,11 +448,15 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 cp_async_wait<1>();
             if (!p.use_tma) fence_proxy_async_smem();  // row copies land through the generic proxy
             if (landed && ld_pending == c) ld_pending = -1;
-            if (!group_agree(landed, kBarPrep)) {
+            if (!group_agree(ok && landed, kBarPrep)) {
                 fail = true;
                 break;
             }
-            if (pt == kPrep - 32) issue_mma0();
+            tc_fence_after();
+            // D0 held the previous chunk's W^T until the chain read it out
+            if (pt == kPrep - 32 &&
+                (c == 0 || mbar_wait_bounded(&SS.mbar[MB_D0F], (uint32_t)((c - 1) & 1), kWaitLimitNs)))
+                issue_mma0();
             // P2: half row of [K; Q] -> sum of squares -> fp16 operand in registers: K rows
             //     L2-normalised, Q rows as Q~ = scale e^(G') q / ||q||; rows past the chunk
             //     (tensor tiles carry the following tokens there) become 0.  Stored over the
@@ -817,29 +821,12 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             named_bar(kBarPrep, kPrep);
             tc_fence_after();
 
-            // P5, last step: block column 0; the commit covers every K-step issued before (W^T
-            // for P6, U~^T for the chain, before V' accumulates onto it)
+            // P5, last step: block column 0; the commit covers every K-step issued before.  The
+            // chain reads W^T out of D0 itself, so the chunk is handed over right away.
             if (pt == 192) {
                 issue_w(KQ, pb, 0);
-                mma_commit(&SS.mbar[MB_MW]);
                 issue_u(VV, pb, 0);
                 mma_commit(&SS.mbar[MB_MU]);
-            }
-            if (!wg_wait(MB_MW, c & 1, kBarPrep)) { fail = true; break; }
-
-            // P6: columns [32 hf, +32) of -W^T row r -> WN[pb] (B operand, MN-major)
-            {
-                uint32_t rr[32];
-                tmem_ld32(tlane + TM_D0 + hf * 32, rr);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e8 = 0; e8 < 4; ++e8) {
-                    float f[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) f[u] = -u2f(rr[e8 * 8 + u]);
-                    *reinterpret_cast<uint4*>(sm + OFF_WN + pb * 16384 + sw128(r, hf * 4 + e8)) =
-                        h8(f);
-                }
             }
             if (has_next && pt < C)
                 SS.b[pb ^ 1][pt] = pt < Cn ? XB(gate_bits_to_float(b_nx, p.gt)) : 0.f;
@@ -893,11 +880,32 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             if (has_next) g_raw = gate_bits_at(p.g, (c + 1) * C + min(lt & 63, Cn - 1));
 
             if (!wg_wait(MB_PREP + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
-            // C1: V'^T = U~^T + H^T (-W^T);  O^T = H^T Q~^T   (A = state copy in TMEM), once the
-            //     preparation's U~ product has landed (a failed wait skips the products: the
-            //     chain's next wait then gives up and the group agrees to stop)
-            if (lt == 0 &&
-                mbar_wait_bounded(&SS.mbar[MB_MU], (uint32_t)(c & 1), kWaitLimitNs)) {
+            // C0: -W^T (the preparation's W product, in D0; row = dk = this lane) into WN[pb] as
+            //     the B operand of V' (MN-major), once the W and U~ products are done (they read
+            //     T_w, T_u from the same buffer); D0 is then released for the next chunk
+            if (!wg_wait(MB_MU, c & 1, kBarChain)) { fail = true; break; }
+            {
+                uint32_t rw[2][32];
+                tmem_ld32(tlane + TM_D0, rw[0]);
+                tmem_ld32(tlane + TM_D0 + 32, rw[1]);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&SS.mbar[MB_D0F]);
+#pragma unroll
+                for (int half = 0; half < 2; ++half)
+#pragma unroll
+                    for (int e8 = 0; e8 < 4; ++e8) {
+                        float f[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) f[u] = -u2f(rw[half][e8 * 8 + u]);
+                        *reinterpret_cast<uint4*>(sm + OFF_WN + pb * 16384 + sw128(lt, half * 4 + e8)) =
+                            h8(f);
+                    }
+            }
+            fence_proxy_async_smem();
+            named_bar(kBarChain, 128);
+            // C1: V'^T = U~^T + H^T (-W^T);  O^T = H^T Q~^T   (A = state copy in TMEM)
+            if (lt == 0) {
                 tc_fence_after();
                 const uint32_t id1 = idesc_f32acc(128, 64, false, true, false);
 #pragma unroll
