@@ -606,13 +606,25 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         float acc[16];
 #pragma unroll
                         for (int m = 0; m < 16; ++m) acc[m] = 0.f;
+                        // column jc + 1 of A is loaded while column jc is applied, so each step
+                        // waits only on its own short chain of FMAs, not on shared memory
+                        float4 col[2][4];
+#pragma unroll
+                        for (int i4 = 0; i4 < 4; ++i4)
+                            col[0][i4] = *reinterpret_cast<const float4*>(atr + 4 * i4);
 #pragma unroll
                         for (int jc = 0; jc < 16; ++jc) {
+                            if (jc < 15) {
+#pragma unroll
+                                for (int i4 = (jc + 2) >> 2; i4 < 4; ++i4)
+                                    col[(jc + 1) & 1][i4] =
+                                        *reinterpret_cast<const float4*>(atr + (jc + 1) * 16 + 4 * i4);
+                            }
                             const float xj = jc < il ? 0.f : (jc == il ? 1.f : -acc[jc]);
                             acc[jc] = xj;
 #pragma unroll
                             for (int i4 = (jc + 1) >> 2; i4 < 4; ++i4) {
-                                const float4 a4 = *reinterpret_cast<const float4*>(atr + jc * 16 + 4 * i4);
+                                const float4 a4 = col[jc & 1][i4];
                                 const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
                                 for (int u = 0; u < 4; ++u)
