@@ -14,8 +14,8 @@ bool tc_supported(const gdr_chunk_args& a);
 gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k, const void* v,
                            const void* g, const void* beta, const float* S0, void* o,
                            float* S_final, void* ws, const WsLayout& L, cudaStream_t st,
-                           bool dependent = false);
-gdr_status launch_add_bf16(void* o, const void* x, long long n, cudaStream_t st);
+                           bool dependent = false, const void* g_rev = nullptr,
+                           const void* beta_rev = nullptr, size_t part_off = 0);
 }  // namespace gdr
 
 using namespace gdr;
@@ -158,9 +158,11 @@ gdr_status gdr_chunk_fwd(const gdr_chunk_args* a, const void* q, const void* k, 
 }
 
 
-// Bidirectional forward: the plan, then the two scans; on the tensor-core path the reverse
-// scan is the forward scan's programmatic dependent (it fills the SMs the first grid leaves
-// free) and writes a scratch output that one more kernel adds into o.
+// Bidirectional forward: the plan, then the two scans.  On the tensor-core path both run in
+// one grid, the two scans of a (sequence, head) as a cluster pair that sums the two outputs
+// of every chunk in fp32 through the workspace (one fp32 [64][head size] tile per chunk and
+// head) and rounds once; the CUDA-core path runs the reverse scan after the forward one and
+// accumulates into o.
 namespace {
 size_t bidir_scratch_offset(const gdr_chunk_args& a, Path path) {
     return align_up(ws_layout(a, path == Path::Simt).total, 256);
@@ -168,7 +170,8 @@ size_t bidir_scratch_offset(const gdr_chunk_args& a, Path path) {
 size_t bidir_workspace(const gdr_chunk_args& a, Path path) {
     const size_t base = bidir_scratch_offset(a, path);
     if (path != Path::Tc) return base;
-    return align_up(base + (size_t)2 * a.B * a.T * a.Hv * a.dv, 256);
+    const WsLayout L = ws_layout(a, false);
+    return align_up(base + sizeof(float) * (size_t)L.max_chunks * a.Hv * a.chunk * a.dv, 256);
 }
 }  // namespace
 
@@ -212,14 +215,8 @@ gdr_status gdr_chunk_fwd_bidir(const gdr_chunk_args* a, const void* q, const voi
     gdr_chunk_args rev = *a;
     rev.reverse = 1;
     if (path == Path::Tc) {
-        void* scratch = static_cast<char*>(workspace) + bidir_scratch_offset(*a, path);
         if ((st = launch_chunk_tc(*a, q, k, v, g_fwd, beta_fwd, nullptr, o, nullptr, workspace,
-                                  L, s)) != GDR_OK)
-            return st;
-        if ((st = launch_chunk_tc(rev, q, k, v, g_bwd, beta_bwd, nullptr, scratch, nullptr,
-                                  workspace, L, s, /*dependent=*/true)) != GDR_OK)
-            return st;
-        if ((st = launch_add_bf16(o, scratch, (long long)a->B * a->T * a->Hv * a->dv, s)) !=
+                                  L, s, false, g_bwd, beta_bwd, bidir_scratch_offset(*a, path))) !=
             GDR_OK)
             return st;
         return publish_status(*a, workspace, s);

@@ -125,6 +125,7 @@ struct Small {
     uint32_t tmem_base;
     int gflag[2][2];         // a bounded wait gave up: [chain, preparation][alternate waits]
     int split_ok[2];         // the chunk's decay factors factor into row x column exactly
+    uint32_t pair_cnt;       // bidirectional pair: chunks the partner has left for this CTA
 };
 static_assert(sizeof(Small) <= 5120, "small shared block");
 
@@ -138,6 +139,12 @@ struct TcParams {
     int tma_store;  // full output chunks leave through the output tensor map
     gdr_dtype gt;
     float scale;
+    // bidirectional pairs: the reverse scan's gates, the chunk map's first chunk of every
+    // sequence, and the fp32 output a pair's first scan of a chunk leaves for the second
+    // ([chunk][head][64 rows][head size], rows in forward order)
+    const void* g_rev; const void* beta_rev;
+    const int32_t* chunk_off;
+    float* part;
 };
 
 // The fused gating prologue's per-head arrays, a kernel argument of its own that only the
@@ -189,7 +196,7 @@ __device__ __forceinline__ float gate_bits_to_float(uint32_t b, gdr_dtype dt) {
 // kDh: the head size dk = dv in memory, 128 or 64.  A 64-wide head runs in the same 128-wide
 // tiles with feature columns 64-127 zero (never loaded): the normalisation is unchanged and
 // the state's extra rows and columns receive only zero updates, so they stay zero.
-template <bool kRaw, int kDh>
+template <bool kRaw, int kDh, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -207,11 +214,23 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     // bidirectional call) may start on the SMs this grid leaves free; every CTA waits for the
     // grid it depends on before it exits, so a later ordinary launch sees both grids' results
     griddep_launch_dependents();
-    if (p.hdr->err != GDR_OK) { griddep_wait(); return; }
+    // a bidirectional pair stops only on an error of the plan, which both of its CTAs see
+    // alike (an error another CTA records while this grid runs must not split a pair)
+    if (kPair ? p.hdr->err == GDR_ERR_DEVICE_CHECK : p.hdr->err != GDR_OK) {
+        griddep_wait();
+        return;
+    }
 
-    // one CTA per (sequence, value head), heads fastest, sequences in the plan's order
-    const int h = (int)(blockIdx.x % (unsigned)p.Hv);
-    const int s = p.order[blockIdx.x / (unsigned)p.Hv];
+    // one CTA per (sequence, value head), heads fastest, sequences in the plan's order; a
+    // bidirectional pair is two CTAs of one cluster, the forward scan (rank 0) and the reverse
+    // scan (rank 1) of one (sequence, head)
+    const unsigned unit = kPair ? blockIdx.x >> 1 : blockIdx.x;
+    const bool rev = kPair ? cluster_ctarank() == 1 : p.reverse != 0;
+    const void* const gsrc = kPair && rev ? p.g_rev : p.g;
+    const void* const bsrc = kPair && rev ? p.beta_rev : p.beta;
+    const bool use_tma = p.use_tma && !rev;  // reversed scans gather rows with cp.async
+    const int h = (int)(unit % (unsigned)p.Hv);
+    const int s = p.order[unit / (unsigned)p.Hv];
     // the gates as the recurrence uses them (fused gating prologue when kRaw)
     auto XG = [&](float a) -> float {
         if constexpr (kRaw) return gate_g_from_raw(gp.A[h], gp.dt_bias[h], a);
@@ -223,13 +242,20 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     };
     const int hk = h / (p.Hv / p.Hk);
     const long long t0 = p.cu[s], t1 = p.cu[s + 1];
-    const int L = (int)(t1 - t0);
+    const int Lseq = (int)(t1 - t0);
+    // The reverse scan of a pair aligns its chunks with the forward scan's, so both cover the
+    // same 64 tokens per chunk: its chunk 0 holds the sequence's last Lseq mod 64 tokens in
+    // rows rofs..63, and rows below rofs are empty (zero keys, queries, values and gates,
+    // which leave the recurrence unchanged).  The chunked form is exact for any chunking.
+    const int rofs = kPair && rev ? (C - Lseq % C) % C : 0;
+    const int L = Lseq + rofs;  // positions of the (row-offset) scan
     const int nchunks = (L + C - 1) / C;
+    auto row_lo = [&](int c) -> int { return c == 0 ? rofs : 0; };  // first live row of chunk c
     static_assert(kDh == 64 || kDh == D, "head size");
     const size_t sb = ((size_t)s * p.Hv + h) * kDh * kDh;
     // physical token of logical position 0, and the step between consecutive positions
-    const long long tokA = p.reverse ? t1 - 1 : t0;
-    const long long tstep = p.reverse ? -1 : 1;
+    const long long tstep = rev ? -1 : 1;
+    const long long tokA = (rev ? t1 - 1 : t0) - tstep * rofs;
 
     if (nchunks == 0) {  // empty sequence: the state passes through
         if (p.S_final)
@@ -249,6 +275,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                                    : (i == MB_CD || i == MB_CD + 1 || i == MB_D0F) ? 128
                                                                                    : 1);
         SS.gflag[0][0] = SS.gflag[0][1] = SS.gflag[1][0] = SS.gflag[1][1] = 0;
+        SS.pair_cnt = 0;
         mbar_init_fence();
     }
     if constexpr (kDh < D) {  // feature columns 64-127 of every K/Q and V tile stay zero
@@ -262,6 +289,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     }
     tc_fence_before();
     __syncthreads();
+    // a pair's counters start at zero before either CTA may advance its partner's
+    if constexpr (kPair) cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem = SS.tmem_base;
     const uint32_t tlane = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's lanes
@@ -312,7 +341,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
         const __nv_bfloat16* vbase = p.v + (size_t)h * kDh + (cd_in ? cd : 0) * 8;
         const long long kq_tok = (long long)p.Hk * kDh, v_tok = (long long)p.Hv * kDh;
         auto load_chunk = [&](int c) {
-            if (p.use_tma) {  // forward scans: six 8 KB tensor tiles, issued by one thread (pt 128)
+            if (use_tma) {  // forward scans: six 8 KB tensor tiles, issued by one thread (pt 128)
                 uint64_t* bar = &SS.mbar[MB_LD + c % 3];
                 const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
                 const uint32_t vv = sbase + OFF_V + (c & 1) * V_STRIDE;
@@ -332,7 +361,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int i = r0 + 16 * m;
-                const bool valid = i < Cc && cd_in;
+                const bool valid = i >= row_lo(c) && i < Cc && cd_in;
                 const long long tok = valid ? tokA + tstep * (c * C + i) : t0;
                 const uint32_t off = sw128(i, cd & 7);
                 cp_async16(kq + off, kbase + tok * kq_tok, valid);
@@ -340,16 +369,16 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 cp_async16(vv + off, vbase + tok * v_tok, valid);
             }
         };
-        if (p.use_tma && pt == 128) {
+        if (use_tma && pt == 128) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
         }
-        if (!p.use_tma || pt == 128) load_chunk(0);
+        if (!use_tma || pt == 128) load_chunk(0);
         // the chunk whose tensor loads this thread issued and nobody has waited for yet (-1:
         // none); on an early exit it waits for them, so no copy lands in released memory
-        int ld_pending = p.use_tma && pt == 128 ? 0 : -1;
-        if (!p.use_tma) cp_async_commit();
+        int ld_pending = use_tma && pt == 128 ? 0 : -1;
+        if (!use_tma) cp_async_commit();
         // in-chunk cumulative log decay (log2 units) of one chunk from its gates, two per lane
         // (positions 2 lane, 2 lane + 1; 0 past the chunk), into G[par], and whether every
         // decay factor 2^(G_i - G_j) splits into 2^(G_i - G_ref) 2^(G_ref - G_j) inside the
@@ -377,10 +406,11 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
         };
         {
             const int Cc0 = min(C, L);
-            if (pt < C) SS.b[0][pt] = pt < Cc0 ? XB(gate_at(p.beta, pt)) : 0.f;
+            auto live0 = [&](int i) { return i >= rofs && i < Cc0; };
+            if (pt < C) SS.b[0][pt] = live0(pt) ? XB(gate_at(bsrc, pt)) : 0.f;
             if (pw == 1)
-                chunk_cumsum(2 * lane < Cc0 ? XG(gate_at(p.g, 2 * lane)) : 0.f,
-                             2 * lane + 1 < Cc0 ? XG(gate_at(p.g, 2 * lane + 1)) : 0.f, 0);
+                chunk_cumsum(live0(2 * lane) ? XG(gate_at(gsrc, 2 * lane)) : 0.f,
+                             live0(2 * lane + 1) ? XG(gate_at(gsrc, 2 * lane + 1)) : 0.f, 0);
         }
         // P5, issued as the solve completes T's block columns: K-step kk of W^T = K^T T_w^T
         // (into D0) and of U~^T = V^T T_u^T (into DU) reads block column kk of T_w and T_u
@@ -415,17 +445,17 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             if (c >= 2) ok = mbar_wait_bounded(&SS.mbar[MB_CD + pb], ((c >> 1) & 1) ^ 1, kWaitLimitNs);
             int Cn = 0;
             if (has_next) {
-                if (!p.use_tma && ok) load_chunk(c + 1);  // reversed scans: every thread's row copies
+                if (!use_tma && ok) load_chunk(c + 1);  // reversed scans: every thread's row copies
                 // in-bounds positions for every thread, masked only where the values are used
                 // (a select on a just-loaded value would wait for the load right here)
                 Cn = min(C, L - (c + 1) * C);
-                b_nx = gate_bits_at(p.beta, (c + 1) * C + min(pt & 63, Cn - 1));
+                b_nx = gate_bits_at(bsrc, (c + 1) * C + min(pt & 63, Cn - 1));
                 if (pw == 1) {
-                    g_nx0 = gate_bits_at(p.g, (c + 1) * C + min(2 * lane, Cn - 1));
-                    g_nx1 = gate_bits_at(p.g, (c + 1) * C + min(2 * lane + 1, Cn - 1));
+                    g_nx0 = gate_bits_at(gsrc, (c + 1) * C + min(2 * lane, Cn - 1));
+                    g_nx1 = gate_bits_at(gsrc, (c + 1) * C + min(2 * lane + 1, Cn - 1));
                 }
             }
-            if (!p.use_tma) cp_async_commit();
+            if (!use_tma) cp_async_commit();
             // P1: D0 = [K;Q] K^T straight from the bf16 tiles (M=128, N=64, K=128), issued by
             //     warp 11 once the tiles have landed.  The L2 norms scale D0's rows and columns
             //     afterwards, so the product runs while the operands are normalised.
@@ -441,12 +471,12 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 mma_commit(&SS.mbar[MB_M0]);
             };
             bool landed = true;
-            if (p.use_tma)
+            if (use_tma)
                 landed = mbar_wait_bounded(&SS.mbar[MB_LD + c % 3], (uint32_t)((c / 3) & 1),
                                            kWaitLimitNs);
             else
                 cp_async_wait<1>();
-            if (!p.use_tma) fence_proxy_async_smem();  // row copies land through the generic proxy
+            if (!use_tma) fence_proxy_async_smem();  // row copies land through the generic proxy
             if (landed && ld_pending == c) ld_pending = -1;
             if (!group_agree(ok && landed, kBarPrep)) {
                 fail = true;
@@ -488,7 +518,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     const float Gref = SS.G[pb][31];
                     const float Gi = SS.G[pb][t];
                     const float Gr = p.read_pre ? (t > 0 ? SS.G[pb][t - 1] : 0.f) : Gi;
-                    SS.Kd[pb][t] = t < Cc ? ex2(SS.G[pb][Cc - 1] - Gi) : 0.f;
+                    SS.Kd[pb][t] = t >= row_lo(c) && t < Cc ? ex2(SS.G[pb][Cc - 1] - Gi) : 0.f;
                     SS.bg[t] = SS.b[pb][t] * ex2(Gi);
                     SS.Er[t] = ex2(Gi - Gref);
                     SS.Eq[t] = ex2(Gr - Gref);
@@ -500,7 +530,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     const float Gr = p.read_pre ? (i > 0 ? SS.G[pb][i - 1] : 0.f) : SS.G[pb][i];
                     f = p.scale * ex2(Gr) * inv;
                 }
-                if (i >= Cc) f = 0.f;
+                if (i < row_lo(c) || i >= Cc) f = 0.f;
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
                     const uint32_t w[4] = {vals[c8].x, vals[c8].y, vals[c8].z, vals[c8].w};
@@ -538,12 +568,12 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             //     (read by the product) while the accumulator load is in flight
             {
                 // warp 8 has no store here: it issues the next chunk's tensor loads
-                if (p.use_tma && has_next && pt == 128) {
+                if (use_tma && has_next && pt == 128) {
                     load_chunk(c + 1);
                     ld_pending = c + 1;
                 }
                 const int i = r & 63;
-                const bool live = i < Cc;
+                const bool live = i >= row_lo(c) && i < Cc;
                 const bool split = SS.split_ok[pb];
                 float* As = reinterpret_cast<float*>(sm + OFF_AS);
                 uint32_t rr[32];
@@ -855,7 +885,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
         const int j = lt;  // dv column = TMEM lane
         {
             // initial state -> TM_HM (pre-scaled by chunk 0's total decay), TM_HB (fp16)
-            const float gv = lt < min(C, L) ? XG(gate_at(p.g, lt)) : 0.f;
+            const float gv = lt >= rofs && lt < min(C, L) ? XG(gate_at(gsrc, lt)) : 0.f;
             const float part = warp_sum(gv);
             if (lane == 0 && warp < 2) SS.gsum_part[warp] = part;
             named_bar(kBarChain, 128);
@@ -881,6 +911,17 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             tc_fence_after();
         }
         const bool check_o = !p.qk_l2norm || !(fabsf(p.scale) <= 1024.f);
+        // bidirectional pair: a chunk's fp32 output left for the partner and not announced yet
+        bool sig_pending = false;
+        auto pair_flush = [&]() {
+            if (!sig_pending) return;
+            named_bar(kBarChain, 128);  // every thread's stores of the chunk precede the release
+            if (lt == 0) {
+                __threadfence();
+                cluster_add_release(cluster_map(smem_u32(&SS.pair_cnt), rev ? 0u : 1u), 1u);
+            }
+            sig_pending = false;
+        };
         for (int c = 0; c < nchunks; ++c) {
             const int pb = c & 1;
             const uint32_t KQ = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
@@ -889,7 +930,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             const int Cn = has_next ? min(C, L - (c + 1) * C) : 0;
             // loaded unconditionally from an in-bounds position, masked when reduced in C2
             uint32_t g_raw = 0;
-            if (has_next) g_raw = gate_bits_at(p.g, (c + 1) * C + min(lt & 63, Cn - 1));
+            if (has_next) g_raw = gate_bits_at(gsrc, (c + 1) * C + min(lt & 63, Cn - 1));
 
             if (!wg_wait(MB_PREP + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
             // C0: -W^T (the preparation's W product, in D0; row = dk = this lane) into WN[pb] as
@@ -985,6 +1026,20 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                                   sdesc_sw128(KQ + kk * 2048, 16384, 1024), id4, 1);
                 mma_commit(&SS.mbar[MB_M3 + pb]);
             }
+            // Bidirectional pair: chunk u of the forward order.  The scan that reaches it first
+            // (the forward one in the first half of the sequence, the reverse one in the second)
+            // leaves its fp32 output in the workspace and advances its partner's counter; the
+            // other adds it to its own and rounds the sum once.  Reverse row i is forward row
+            // 63 - i.  The counter moves one chunk late (a fence right after the stores would
+            // wait for all of them), always before this CTA waits for its partner.  Each waits
+            // only for chunks its partner reached at an earlier step and announced by the start
+            // of this step's wait, before which the partner waits for nothing from it, so the
+            // two CTAs of the cluster (resident together) cannot wait on each other.
+            const int u = kPair && rev ? nchunks - 1 - c : c;
+            const bool second = kPair && (rev ? 2 * u <= nchunks - 1 : 2 * u > nchunks - 1);
+            float* const part = kPair ? p.part + ((size_t)(p.chunk_off[s] + u) * p.Hv + h) * (C * kDh)
+                                      : nullptr;
+            if constexpr (kPair) pair_flush();
             if (!wg_wait(MB_M3 + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
 
             // C4: O -> staged in WN[pb] -> global (two tensor stores for a full chunk, else
@@ -999,12 +1054,45 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 tmem_ld32(tlane + TM_DO, ro[0]);
                 tmem_ld32(tlane + TM_DO + 32, ro[1]);
                 tmem_wait_ld();
+                // Output rows: this chunk's own (tok = tokA + tstep (64 c + row)), or in a
+                // bidirectional pair the forward chunk u both scans cover, in forward order.
+                const long long obase = kPair ? t0 + (long long)C * u : tokA + tstep * (long long)c * C;
+                const long long ostep = kPair ? 1 : tstep;
+                const int olo = kPair ? 0 : row_lo(c);
+                const int ohi = kPair ? min(C, Lseq - C * u) : Cc;
+                bool emit = true;  // this CTA writes the chunk's output
+                if constexpr (kPair) {
+                    if (!second) {
+                        if (j < kDh) {
+#pragma unroll
+                            for (int i = 0; i < C; ++i)
+                                __stcg(part + (rev ? C - 1 - i : i) * kDh + j, u2f(ro[i >> 5][i & 31]));
+                        }
+                        sig_pending = true;
+                        emit = false;
+                    } else {
+                        bool ok = true;
+                        if (lt == 0)
+                            ok = counter_wait_bounded(smem_u32(&SS.pair_cnt),
+                                                      (uint32_t)(rev ? u + 1 : nchunks - u), kWaitLimitNs);
+                        if (!group_agree(ok, kBarChain)) { fail = true; break; }
+                        if (j < kDh) {
+#pragma unroll
+                            for (int i = 0; i < C; ++i)
+                                ro[i >> 5][i & 31] = __float_as_uint(
+                                    u2f(ro[i >> 5][i & 31]) + __ldcg(part + (rev ? C - 1 - i : i) * kDh + j));
+                        }
+                    }
+                }
+                if (emit) {
 #pragma unroll
                 for (int half = 0; half < 2; ++half)
 #pragma unroll
-                    for (int m = 0; m < 32; ++m)
-                        *reinterpret_cast<__nv_bfloat16*>(stage_j + sw128(half * 32 + m, cj)) =
+                    for (int m = 0; m < 32; ++m) {
+                        const int row = kPair && rev ? C - 1 - (half * 32 + m) : half * 32 + m;
+                        *reinterpret_cast<__nv_bfloat16*>(stage_j + sw128(row, cj)) =
                             __float2bfloat16_rn(u2f(ro[half][m]));
+                    }
                 // with normalised q, k and |scale| <= 1024 the operands that reach only the
                 // output (P, Q~) are bounded by |scale|; otherwise every output is checked
                 if (check_o) {
@@ -1013,9 +1101,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 }
                 fence_proxy_async_smem();
                 named_bar(kBarChain, 128);
-                if (p.tma_store && Cc == C) {
+                if (p.tma_store && olo == 0 && ohi == C) {
                     if (lt == 0) {
-                        const int z = (int)(t0 + (long long)c * C);
+                        const int z = (int)obase;
                         const uint32_t src = sbase + OFF_WN + pb * 16384;
                         tma_store_3d(&tm_o, src, 0, h, z);
                         if (kDh > 64) tma_store_3d(&tm_o, src + 8192, 64, h, z);
@@ -1026,8 +1114,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {
                     const int idx = m * 128 + lt, row = idx >> 4, c16 = idx & 15;
-                    if (row < Cc && c16 < kDh / 8) {
-                        const long long tok = tokA + tstep * (long long)(c * C + row);
+                    if (row >= olo && row < ohi && c16 < kDh / 8) {
+                        const long long tok = obase + ostep * row;
                         uint4* dp = reinterpret_cast<uint4*>(p.o + ((size_t)tok * p.Hv + h) * kDh + c16 * 8);
                         uint4 a = *reinterpret_cast<const uint4*>(stage + (c16 >> 3) * 8192 +
                                                                   sw128(row, c16 & 7));
@@ -1044,6 +1132,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         }
                         *dp = a;
                     }
+                }
                 }
                 }
                 const float gam = has_next ? ex2((SS.gsum_part[0] + SS.gsum_part[1]) * kLog2e) : 1.f;
@@ -1095,6 +1184,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             named_bar(kBarChain, 128);
             tc_fence_after();
         }
+        if constexpr (kPair) pair_flush();  // the last chunk left for the partner
     }
 
     if (tid == 0) bulk_wait_all();  // output tiles written before the CTA exits
@@ -1103,6 +1193,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     // an fp16 operand that left its range shows as a non-finite output or final state
     if (__syncthreads_or(omax <= 3.4e38f ? 0 : 1) && tid == 0)
         atomicCAS(&p.hdr->err, (int)GDR_OK, (int)GDR_ERR_RANGE);
+    // no CTA of a pair leaves while its partner may still advance its counter
+    if constexpr (kPair) cluster_sync_all();
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
     griddep_wait();
 }
@@ -1149,36 +1241,12 @@ bool tc_supported(const gdr_chunk_args& a) {
            !a.gdn2;
 }
 
-// sum of two bf16 arrays of n8 groups of 8, rounded once: o += x
-__global__ void add_bf16_kernel(__nv_bfloat16* o, const __nv_bfloat16* x, long long n8) {
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
-         i += (long long)gridDim.x * blockDim.x) {
-        uint4 a = reinterpret_cast<uint4*>(o)[i];
-        const uint4 b = reinterpret_cast<const uint4*>(x)[i];
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
-        uint32_t ow[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 u = unpack_bf16x2(aw[e]), w = unpack_bf16x2(bw[e]);
-            ow[e] = pack_bf16x2(u.x + w.x, u.y + w.y);
-        }
-        reinterpret_cast<uint4*>(o)[i] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-    }
-}
-
-gdr_status launch_add_bf16(void* o, const void* x, long long n, cudaStream_t st) {
-    const long long n8 = n / 8;
-    if (n8 == 0) return GDR_OK;
-    const unsigned blocks = (unsigned)std::min<long long>((n8 + 255) / 256, 148LL * 8);
-    add_bf16_kernel<<<blocks, 256, 0, st>>>(static_cast<__nv_bfloat16*>(o),
-                                            static_cast<const __nv_bfloat16*>(x), n8);
-    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
-}
-
 gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k, const void* v,
                            const void* g, const void* beta, const float* S0, void* o,
                            float* S_final, void* ws, const WsLayout& L, cudaStream_t st,
-                           bool dependent) {
+                           bool dependent, const void* g_rev, const void* beta_rev,
+                           size_t part_off) {
+    const bool pair = g_rev != nullptr;  // bidirectional: both scans, one cluster per pair
     char* base = static_cast<char*>(ws);
     TcParams p;
     p.q = static_cast<const __nv_bfloat16*>(q);
@@ -1192,6 +1260,9 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
     p.Hk = a.Hk; p.Hv = a.Hv; p.read_pre = a.read_mode == GDR_READ_PRE;
     p.qk_l2norm = a.qk_l2norm; p.reverse = a.reverse; p.o_acc = a.o_accumulate;
     p.gt = a.gate_dtype; p.scale = a.scale;
+    p.g_rev = g_rev; p.beta_rev = beta_rev;
+    p.chunk_off = reinterpret_cast<const int32_t*>(base + L.chunk_off);
+    p.part = pair ? reinterpret_cast<float*>(base + part_off) : nullptr;
     const GateParams gp{a.gate_A, a.gate_dt_bias, a.beta_scale};
     CUtensorMap tq, tk, tv, to;
     memset(&tq, 0, sizeof(tq));
@@ -1201,7 +1272,9 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
     const long long T_tot = (long long)a.B * a.T;
     p.use_tma = 0;
     p.tma_store = 0;
-    if (!a.reverse && T_tot > 0) {  // reversed scans gather rows with cp.async instead
+    // tensor maps for forward scans (a pair's forward CTA included); reversed scans gather
+    // rows with cp.async instead.  A pair writes whole forward chunks from either CTA.
+    if ((!a.reverse || pair) && T_tot > 0) {
         if (!make_tile_map(&tq, q, a.Hk, T_tot, a.dk) || !make_tile_map(&tk, k, a.Hk, T_tot, a.dk) ||
             !make_tile_map(&tv, v, a.Hv, T_tot, a.dv))
             return GDR_ERR_CUDA;
@@ -1209,28 +1282,35 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
         // accumulating outputs are read back, so they keep the plain stores
         p.tma_store = !a.o_accumulate && make_tile_map(&to, o, a.Hv, T_tot, a.dv);
     }
-    auto kernel = a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D> : chunk_fused_tc<false, D>)
-                            : (a.gate_raw ? chunk_fused_tc<true, 64> : chunk_fused_tc<false, 64>);
+    auto kernel = pair ? (a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D, true> : chunk_fused_tc<false, D, true>)
+                                    : (a.gate_raw ? chunk_fused_tc<true, 64, true> : chunk_fused_tc<false, 64, true>))
+                       : (a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D, false> : chunk_fused_tc<false, D, false>)
+                                    : (a.gate_raw ? chunk_fused_tc<true, 64, false> : chunk_fused_tc<false, 64, false>));
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
-    dim3 grid((unsigned)a.n_seqs * (unsigned)a.Hv);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)a.n_seqs * (unsigned)a.Hv * (pair ? 2u : 1u));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
     if (dependent) {  // may start while the stream's previous grid finishes (see the kernel)
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = grid;
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = SMEM_BYTES;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, kernel, p, tq, tk, tv, to, gp) != cudaSuccess)
-            return GDR_ERR_CUDA;
-    } else {
-        kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p, tq, tk, tv, to, gp);
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
     }
+    if (pair) {  // the two scans of a (sequence, head) run together on one cluster
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 2;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    if (cudaLaunchKernelEx(&cfg, kernel, p, tq, tk, tv, to, gp) != cudaSuccess) return GDR_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

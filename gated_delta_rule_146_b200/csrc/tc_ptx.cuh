@@ -69,6 +69,45 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     return true;
 }
 
+// ---- thread-block cluster: partner shared memory, release/acquire counters ---------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// shared::cluster address of the variable at shared::cta address `saddr` in CTA `rank`
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+    uint32_t d;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(saddr), "r"(rank));
+    return d;
+}
+__device__ __forceinline__ void cluster_add_release(uint32_t caddr, uint32_t v) {
+    asm volatile("red.release.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(caddr), "r"(v)
+                 : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_cluster(uint32_t saddr) {
+    uint32_t v;
+    asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(saddr) : "memory");
+    return v;
+}
+// every thread of every CTA of the cluster
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                     "memory");
+}
+// Wait until a counter in this CTA's shared memory, advanced by another CTA of the cluster,
+// reaches `need`; gives up after `limit_ns`.
+__device__ __forceinline__ bool counter_wait_bounded(uint32_t saddr, uint32_t need,
+                                                     uint64_t limit_ns) {
+    if (ld_acquire_cluster(saddr) >= need) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_cluster(saddr) < need) {
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+        __nanosleep(100);
+    }
+    return true;
+}
+
 // ---- proxy / tcgen05 ordering fences ----------------------------------------------------
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -30,9 +30,9 @@
  *   non-decreasing, does not start at 0 or does not end at T) are recorded in
  *   an error word inside the workspace; the kernels then skip the work.  Read
  *   it with gdr_read_device_error.  No kernel traps or waits without a bound
- *   (the one wait not on a timer: in gdr_chunk_fwd_bidir the reverse scan's CTAs
- *   wait, before they exit, for the forward scan's grid to complete, and every
- *   CTA of that grid is already running and bounds its own waits).
+ *   (the one wait not on a timer: in gdr_chunk_fwd_bidir the two CTAs of a
+ *   cluster meet at a cluster barrier before they exit, and each bounds every
+ *   wait that could keep it from getting there).
  */
 #ifndef GDR_H
 #define GDR_H
@@ -219,14 +219,19 @@ const char* gdr_chunk_fwd_path(const gdr_chunk_args* args);
  *   g_*, beta_* [B, T, Hv] gate_dtype, or the raw projections with gate_raw (both
  *               directions share gate_A, gate_dt_bias, beta_scale); GDN-2 layouts with gdn2
  *               (both directions share gdn2_w)
- *   o           [B, T, Hv, dv] io_dtype; with bf16 on the tensor-core path each direction's
- *               output is rounded to bf16 and the sum rounded once more, as two gdr_chunk_fwd
- *               calls (the second with reverse and o_accumulate) give
+ *   o           [B, T, Hv, dv] io_dtype; on the tensor-core path the two directions are
+ *               summed in fp32 and the sum rounded once (two gdr_chunk_fwd calls, the second
+ *               with reverse and o_accumulate, round each direction first)
  *   workspace   at least gdr_chunk_fwd_bidir_workspace_size(args) bytes, 256-byte aligned
  *
- * On the tensor-core path the reverse scan's CTAs start while the forward scan's last CTAs
- * run (programmatic dependent launch) and write a scratch output in the workspace, which a
- * final kernel adds into o.  Errors: as gdr_chunk_fwd.
+ * On the tensor-core path one grid runs both scans: the two scans of a (sequence, head) are
+ * the two CTAs of a thread-block cluster.  The reverse scan's 64-token chunks are aligned
+ * with the forward scan's (its first chunk holds the sequence's last T mod 64 tokens), so
+ * both produce the output of the same 64 tokens per chunk; the scan that gets to a chunk
+ * first leaves its fp32 output there in the workspace, and the other adds it to its own and
+ * writes o.  The two CTAs read the same q, k, v tiles within one residency, so the second
+ * read is served mostly from L2.  The CUDA-core path runs the reverse scan after the forward
+ * one, accumulating into o.  Errors: as gdr_chunk_fwd.
  */
 size_t gdr_chunk_fwd_bidir_workspace_size(const gdr_chunk_args* args);
 gdr_status gdr_chunk_fwd_bidir(const gdr_chunk_args* args,
