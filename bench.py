@@ -62,9 +62,12 @@ def source_digest(sources) -> str:
 
 
 def measured_traffic(kernel: str, sources, units: float):
-    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu summary
-    (profiles/traffic.json), scaled from the captured case to `units` (rows or sequences);
-    None when a kernel source has changed since the counters were taken."""
+    """Memory traffic per launch of `kernel` from the committed ncu summary
+    (profiles/traffic.json): DRAM bytes read plus the bytes the SMs wrote into L2 (each write
+    counted once where it enters L2; dram__bytes_write misses the lines still dirty in L2
+    when the kernel ends), scaled from the captured case to `units` (rows or sequences; 1
+    for a capture of the full workload); None when a kernel source has changed since the
+    counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -76,8 +79,8 @@ def measured_traffic(kernel: str, sources, units: float):
         return None
     if not rec or digest != rec["source_sha256_16"]:
         return None
-    captured = rec.get("rows_captured") or rec.get("seqs_captured")
-    return (rec["dram_read_bytes"] + rec["dram_write_bytes"]) * units / captured
+    captured = rec.get("rows_captured") or rec.get("seqs_captured") or rec.get("calls_captured")
+    return (rec["dram_read_bytes"] + rec["write_bytes_into_l2"]) * units / captured
 
 
 def flops_per_head_token(C, dk, dv):
@@ -288,7 +291,9 @@ def bench_ours(args, rank, world, local_rank):
         bbytes = sum(bd[n].numel() * bd[n].element_size() for n in ("q", "k", "v")) + sum(
             bd[n].numel() * bd[n].element_size() for n in ("g", "beta", "g_bwd", "beta_bwd")) + (
             bo.numel() * bo.element_size())
+        btraffic = measured_traffic("chunk_fused_tc_pair", CHUNK_TC_SOURCES, 1)
         bidir = {"workload": bw.name, "ms_per_step": bms, "value": whole_job_rate(btok, world, bms),
+                 "traffic": btraffic,
                  "unit": "tokens/s", "path": gdr.chunk_fwd_path(bargs),
                  "call": "gdr_chunk_fwd_bidir: one grid, forward and reverse scan of a "
                          "(sequence, head) as a 2-CTA cluster, fp32 sum rounded once",
