@@ -9,11 +9,12 @@
  *     post-write read  o_t = scale * H_t^T q_t
  *     pre-write read   o_t = scale * H_{t-1}^T q_t
  *
- * (Prizma "seq/delta.py", module docstring: S_t = alpha_t S_{t-1} + u_t k_t^T
- * with u_t = beta_t (v_t - alpha_t S_{t-1} k_t) and the strictly causal read
- * o_t = S_{t-1} q_t; sparse_delta_memory/layer.py, SparseDeltaMemory docstring:
- * memory *= exp(g), memory += beta k (v - memory k)^T; tiny_gdn/fugue.py,
- * BidirectionalGatedDeltaNet2 docstring: the forward read q_t^T S_t.)
+ * (Prizma "seq/delta.py", module docstring: the same update on the untransposed
+ * state, and the strictly causal read from the state before the token's write;
+ * sparse_delta_memory/layer.py, SparseDeltaMemory docstring: the memory decays by
+ * the gate's exponential, then takes a write of beta times the key and the
+ * prediction error; tiny_gdn/fugue.py, BidirectionalGatedDeltaNet2 docstring: the
+ * forward scan reads the state after the token's write.)
  *
  * Conventions shared by every entry point
  * ---------------------------------------

@@ -12,9 +12,9 @@
  *       S_t = alpha_t S_{t-1} + u_t k_t^T,
  *       u_t = beta_t (v_t - alpha_t S_{t-1} k_t),
  *       pre-write read o_t = S_{t-1} q_t.
- *   sparse_delta_memory/layer.py, `SparseDeltaMemory` docstring:
- *       memory *= exp(g);  memory += beta * k (v - memory k)^T,
- *     i.e. alpha_t = exp(g_t).
+ *   sparse_delta_memory/layer.py, `SparseDeltaMemory` docstring: the memory
+ *     decays by the exponential of the gate, then takes the delta write of beta
+ *     times k and the prediction error, i.e. alpha_t = exp(g_t).
  *   tiny_gdn/fugue.py, `BidirectionalGatedDeltaNet2` docstring: the forward
  *     scan reads q_t^T S_t (post-write read).
  *
