@@ -195,3 +195,13 @@ def compare_whole(x, o, S, read_mode, scale, dtype, name="", reverse=False, gkey
     ao.check()
     if S_c is not None:
         aS.check()
+
+
+def oracle_backward_sequence(job):
+    """One sequence of a fixed-length workload through the fp64 backward oracle (a process
+    pool's task: the arrays arrive and leave as NumPy, the reference as float32, whose
+    rounding is far below any bound it is compared with)."""
+    import oracle.backward as obw
+    arrays, kw = job
+    ref = obw.backward(*arrays, **kw)
+    return {n: a.astype(np.float32) for n, a in ref.items()}

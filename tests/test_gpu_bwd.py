@@ -15,7 +15,7 @@ import torch
 import oracle.backward as obw
 import workloads
 import gated_delta_rule_146_b200 as gdr
-from gpu_helpers import assert_close, record, to_dev
+from gpu_helpers import Accum, assert_close, oracle_backward_sequence, record, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -99,12 +99,12 @@ def test_bidirectional_workload_rows():
     run_and_check(x, dO, None, "bf16", read_mode="pre", scale=1.0, reverse=True)
 
 
-def test_training_shape_workload_sampled():
+def test_training_shape_workload_whole():
     """The backward at the training workload's full size (8 x 4096 tokens, 16 heads, d=128,
-    bf16), checked on sampled (sequence, head) units that the oracle computes one by one
-    (key heads = value heads here, so dq and dk of a unit are its own)."""
+    bf16): every element of dq, dk, dv, dg, dbeta and dS0 against the oracle, which runs one
+    sequence per process of a spawned pool (about a minute on the host's cores)."""
+    import multiprocessing as mp
     w = workloads.WORKLOADS["bf16_b8_h16_t4096_d128"]
-    assert w.Hk == w.Hv
     x = workloads.workload_inputs(w)
     gen = torch.Generator("cpu").manual_seed(71)
     dO = torch.randn(x["v"].shape, generator=gen).to(torch.bfloat16)
@@ -113,12 +113,20 @@ def test_training_shape_workload_sampled():
                         dev["S0"], None, None, chunk=w.chunk, read_mode=w.read_mode,
                         scale=w.scale)
     torch.cuda.synchronize()
-    assert all(torch.isfinite(t.float()).all() for t in got)
-    for b, h in [(0, 0), (w.B - 1, w.Hv - 1), (3, 7)]:
-        sl = lambda t: t[b:b + 1, :, h:h + 1]
-        ref = obw.backward(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]), sl(x["beta"]),
-                           sl(dO), None if x["S0"] is None else x["S0"][b:b + 1, h:h + 1],
-                           None, read_mode=w.read_mode, scale=w.scale)
-        for name, g in zip(("dq", "dk", "dv", "dg", "dbeta"), got[:5]):
-            grad_close(f"{name}[{b},{h}]", sl(g), ref[name], torch.bfloat16)
-        grad_close(f"dS0[{b},{h}]", got[5][b:b + 1, h:h + 1], ref["dS0"], torch.bfloat16)
+    got = [t.detach().cpu() for t in got]
+    f32 = lambda t: None if t is None else t.float().numpy()
+    jobs = []
+    for b in range(w.B):
+        sl = lambda t: f32(t[b:b + 1])
+        arrays = (sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]), sl(x["beta"]), sl(dO),
+                  None if x["S0"] is None else f32(x["S0"][b:b + 1]), None)
+        jobs.append((arrays, {"read_mode": w.read_mode, "scale": w.scale}))
+    acc = {n: Accum(n, torch.bfloat16, "state" if n == "dS0" else "out")
+           for n in ("dq", "dk", "dv", "dg", "dbeta", "dS0")}
+    with mp.get_context("spawn").Pool(min(w.B, max(1, mp.cpu_count()))) as pool:
+        for b, ref in enumerate(pool.imap(oracle_backward_sequence, jobs)):
+            for i, n in enumerate(("dq", "dk", "dv", "dg", "dbeta")):
+                acc[n].add(got[i][b:b + 1], ref[n].astype(np.float64), label=f" row {b}")
+            acc["dS0"].add(got[5][b:b + 1], ref["dS0"].astype(np.float64), label=f" row {b}")
+    for a in acc.values():
+        a.check()
