@@ -10,6 +10,10 @@
 
 namespace gdr {
 bool tc_supported(const gdr_chunk_args& a);
+bool tc_g2_supported(const gdr_chunk_args& a);
+gdr_status launch_chunk_g2_tc(const gdr_chunk_args& a, const void* q, const void* k, const void* v,
+                              const void* g, const void* b, const float* S0, void* o,
+                              float* S_final, void* ws, const WsLayout& L, cudaStream_t st);
 // `dependent`: launched as the programmatic dependent of the stream's previous grid
 gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k, const void* v,
                            const void* g, const void* beta, const float* S0, void* o,
@@ -85,12 +89,20 @@ gdr_status publish_status(const gdr_chunk_args& a, const void* ws, cudaStream_t 
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 
-enum class Path { None, Tc, Simt };
+enum class Path { None, Tc, TcG2, Simt };
 
 Path choose_path(const gdr_chunk_args& a) {
     if (tc_supported(a)) return Path::Tc;
+    if (tc_g2_supported(a)) return Path::TcG2;
     if (simt_supported(a)) return Path::Simt;
     return Path::None;
+}
+
+// The bidirectional call: GDN-2 gates take the CUDA-core scans (the tensor-core GDN-2 path
+// runs forward scans only).
+Path bidir_path(const gdr_chunk_args& a) {
+    const Path p = choose_path(a);
+    return p == Path::TcG2 ? Path::Simt : p;
 }
 
 }  // namespace
@@ -118,6 +130,7 @@ const char* gdr_chunk_fwd_path(const gdr_chunk_args* a) {
     if (check_chunk_args(a) != GDR_OK) return nullptr;
     switch (choose_path(*a)) {
         case Path::Tc: return "tc";
+        case Path::TcG2: return "tc";
         case Path::Simt: return "simt";
         default: return nullptr;
     }
@@ -150,9 +163,9 @@ gdr_status gdr_chunk_fwd(const gdr_chunk_args* a, const void* q, const void* k, 
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (launch_plan(*a, cu_seqlens, workspace, L, s) != cudaSuccess) return GDR_ERR_CUDA;
-    st = path == Path::Tc
-             ? launch_chunk_tc(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s)
-             : launch_chunk_simt(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s);
+    st = path == Path::Tc     ? launch_chunk_tc(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s)
+         : path == Path::TcG2 ? launch_chunk_g2_tc(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s)
+                              : launch_chunk_simt(*a, q, k, v, g, beta, S0, o, S_final, workspace, L, s);
     if (st != GDR_OK) return st;
     return publish_status(*a, workspace, s);
 }
@@ -177,7 +190,7 @@ size_t bidir_workspace(const gdr_chunk_args& a, Path path) {
 
 size_t gdr_chunk_fwd_bidir_workspace_size(const gdr_chunk_args* a) {
     if (check_chunk_args(a) != GDR_OK || a->reverse || a->o_accumulate) return 0;
-    const Path path = choose_path(*a);
+    const Path path = bidir_path(*a);
     if (path == Path::None) return 0;
     return bidir_workspace(*a, path);
 }
@@ -205,7 +218,7 @@ gdr_status gdr_chunk_fwd_bidir(const gdr_chunk_args* a, const void* q, const voi
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDR_ERR_ALIGNMENT;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return GDR_ERR_ALIGNMENT;
-    const Path path = choose_path(*a);
+    const Path path = bidir_path(*a);
     if (path == Path::None) return GDR_ERR_UNSUPPORTED;
     if (workspace_bytes < bidir_workspace(*a, path)) return GDR_ERR_WORKSPACE;
     const WsLayout L = ws_layout(*a, path == Path::Simt);

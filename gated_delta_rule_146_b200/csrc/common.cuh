@@ -70,7 +70,7 @@ struct WsHeader {
 };
 
 struct WsLayout {
-    size_t cu, chunk_off, chunk_seq, order, W, U, G, Qt, Kt, Pc, total;
+    size_t cu, chunk_off, chunk_seq, order, W, U, G, Qt, Kt, Pc, rec, total;
     long long max_chunks;
 };
 
@@ -87,6 +87,10 @@ inline bool simt_rb(const gdr_chunk_args& a) {
 }
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Bytes of one (chunk, head) record of the tensor-core GDN-2 path: the shared-memory image of
+// the recursion's operands (q~, -W, K~, U~^T, P in fp16, e^{G_C} in fp32).
+constexpr size_t kG2RecordBytes = 74240;
 
 inline WsLayout ws_layout(const gdr_chunk_args& a, bool simt) {
     WsLayout L{};
@@ -109,6 +113,10 @@ inline WsLayout ws_layout(const gdr_chunk_args& a, bool simt) {
             L.Pc = off;
             off = align_up(off + sizeof(float) * (size_t)L.max_chunks * a.Hv * a.chunk * a.chunk, 256);
         }
+    }
+    if (!simt && a.gdn2) {  // tensor-core GDN-2: one record per (chunk, head)
+        L.rec = off;
+        off = align_up(off + kG2RecordBytes * (size_t)L.max_chunks * a.Hv, 256);
     }
     L.total = off;
     return L;
