@@ -82,6 +82,12 @@ __device__ __forceinline__ float bf(const uint8_t* base, uint32_t off) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
 }
 
+// eight consecutive fp32 values (16-byte aligned) into registers
+__device__ __forceinline__ void load_row8(float (&v)[8], const float* src) {
+    const float4 a = reinterpret_cast<const float4*>(src)[0], b = reinterpret_cast<const float4*>(src)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
 // ----------------------------------------------------------------------------------------
 // chunk_g2_prep_tc: per (chunk, value head) item, 256 threads
 // shared memory (bytes from a 1024-aligned base)
@@ -92,47 +98,52 @@ constexpr uint32_t P_G = 49152;     // g bf16, then b . e^G . k^ fp16 (A operand
 constexpr uint32_t P_B = 65536;     // b bf16, then -W staging
 constexpr uint32_t P_W = 81920;     // w bf16, then U~^T staging
 constexpr uint32_t P_GF = 98304;    // G (log2 units) fp32 [64][128]
-constexpr uint32_t P_X = 131072;    // row operands of one row block: A [16][128], P [16][128]
-constexpr uint32_t P_Y = 147456;    // column operand [<= 64][128]; then T_w | T_u (fp16)
-constexpr uint32_t P_A = 180224;    // A fp32 [64][64], swizzled
-constexpr uint32_t P_T = 196608;    // P staging (fp16 record layout), then T fp32
-constexpr uint32_t P_RS = 212992;   // transposed diagonal blocks, then E_32
-constexpr uint32_t P_SMALL = 217088;
+constexpr int kLdXY = 136;          // padded row of the tf32 operands (conflict-free fragments)
+constexpr uint32_t P_X = 131072;    // row operands of one row block: A [16][136], P [16][136]
+constexpr uint32_t P_Y = 148480;    // column operand [<= 64][136]; then T_w | T_u (fp16)
+constexpr uint32_t P_A = 183296;    // A fp32 [64][64], swizzled
+constexpr uint32_t P_T = 199680;    // T fp32
+constexpr uint32_t P_RS = 216064;   // transposed diagonal blocks, then E_32
+constexpr uint32_t P_SMALL = 220160;
 constexpr uint32_t P_SMEM = P_SMALL + 2048 + 1024;
 
 struct PrepSmall {
     float inv_q[C], inv_k[C];
     float dec[D];         // e^{G_C} per channel
     float ones[C];        // column scales of the solve's T tiles (1: T itself)
+    float half_tot[D];    // the cumulative log decay over the first 32 tokens, per channel
     uint64_t mbar[2];     // tiles landed, W^T and U~^T done
     uint32_t tmem_base;
     int range_bad;
 };
 static_assert(sizeof(PrepSmall) <= 2048, "prep small block");
 
-// fp32 [rows][128] operand rows with 16-byte chunks XOR-swizzled by row, for the tf32
-// fragment loads (rows gq and gq + 8 of a fragment hit different banks)
-__device__ __forceinline__ float* opsw(float* base, int r, int c) {
-    return base + r * D + ((((c >> 2) ^ (r & 7)) << 2) | (c & 3));
-}
-
 // One tf32 warp-MMA product of a 16-row block: acc (16 x 8, n-tile) = X (16 x 128) Y^T
-// (8 x 128), X and Y fp32 rows in the opsw layout.  Each thread's two k slots of a step are
-// two adjacent columns (any pairing the A and B fragments share gives the same sum).
-__device__ __forceinline__ void rowblock_ntile(float (&acc)[4], float* X, float* Y, int n0,
-                                               int lane) {
+// (8 x 128).  X and Y hold tf32 bit patterns in rows padded to kLdXY words, so a fragment's
+// eight rows fall in distinct banks and every load is a fixed offset from the lane's base.
+// Each thread's two k slots of a step are two adjacent columns (any pairing the A and B
+// fragments share gives the same sum); even and odd steps accumulate separately.
+__device__ __forceinline__ void rowblock_ntile(float (&acc)[4], const uint32_t* X,
+                                               const uint32_t* Y, int n0, int lane) {
     const int gq = lane >> 2, tq = lane & 3;
+    const uint32_t* x0p = X + gq * kLdXY + 2 * tq;
+    const uint32_t* x1p = x0p + 8 * kLdXY;
+    const uint32_t* yp = Y + (n0 + gq) * kLdXY + 2 * tq;
+    float acc2[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[e] = 0.f;
-#pragma unroll 4
+    for (int e = 0; e < 4; ++e) acc[e] = acc2[e] = 0.f;
+#pragma unroll
     for (int k0 = 0; k0 < D; k0 += 8) {
-        const float2 x0 = *reinterpret_cast<const float2*>(opsw(X, gq, k0 + 2 * tq));
-        const float2 x1 = *reinterpret_cast<const float2*>(opsw(X, gq + 8, k0 + 2 * tq));
-        const float2 y = *reinterpret_cast<const float2*>(opsw(Y, n0 + gq, k0 + 2 * tq));
-        const uint32_t a[4] = {to_tf32(x0.x), to_tf32(x1.x), to_tf32(x0.y), to_tf32(x1.y)};
-        const uint32_t bb[2] = {to_tf32(y.x), to_tf32(y.y)};
-        mma_tf32_16x8x8(acc, a, bb);
+        const uint2 x0 = *reinterpret_cast<const uint2*>(x0p + k0);
+        const uint2 x1 = *reinterpret_cast<const uint2*>(x1p + k0);
+        const uint2 y = *reinterpret_cast<const uint2*>(yp + k0);
+        const uint32_t a[4] = {x0.x, x1.x, x0.y, x1.y};
+        const uint32_t bb[2] = {y.x, y.y};
+        if ((k0 >> 3) & 1) mma_tf32_16x8x8(acc2, a, bb);
+        else mma_tf32_16x8x8(acc, a, bb);
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] += acc2[e];
 }
 
 __global__ void __launch_bounds__(kPrepThreads, 1)
@@ -166,9 +177,9 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
     tc_fence_after();
     const uint32_t tmem = SS.tmem_base;
     float* GF = reinterpret_cast<float*>(sm + P_GF);
-    float* Xa = reinterpret_cast<float*>(sm + P_X);
-    float* Xp = Xa + 16 * D;
-    float* Yc = reinterpret_cast<float*>(sm + P_Y);
+    uint32_t* Xa = reinterpret_cast<uint32_t*>(sm + P_X);
+    uint32_t* Xp = Xa + 16 * kLdXY;
+    uint32_t* Yc = reinterpret_cast<uint32_t*>(sm + P_Y);
     float* As = reinterpret_cast<float*>(sm + P_A);
     float* Ts = reinterpret_cast<float*>(sm + P_T);
     float* RS = reinterpret_cast<float*>(sm + P_RS);
@@ -203,23 +214,50 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
         const bool landed = mbar_wait_bounded(&SS.mbar[0], (uint32_t)(it & 1), kWaitNs);
         if (__syncthreads_or(landed ? 0 : 1)) { fail = true; break; }
 
-        // N: per-channel cumulative log decay (log2 units) and its span, threads 0-127; the
-        //    norms of the q and k rows, threads 128-255
-        if (pt < D) {
-            const int d = pt;
-            float G = 0.f;
-#pragma unroll 1
-            for (int t0 = 0; t0 < C; t0 += 16) {
-                float gv[16];
+        // N: per-channel cumulative log decay (log2 units): thread (channel d, half hh) scans
+        //    its 32 tokens, the second half then adds the first half's total
+        {
+            const int d = pt & 127, hh = pt >> 7;
+            float gv[32];
 #pragma unroll
-                for (int u = 0; u < 16; ++u)
-                    gv[u] = t0 + u <= last ? bf(sm + P_G, tile16(t0 + u, d, 8192)) : 0.f;
+            for (int u = 0; u < 32; ++u) {
+                const int t = 32 * hh + u;
+                gv[u] = t <= last ? bf(sm + P_G, tile16(t, d, 8192)) * kLog2e : 0.f;
+            }
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    G = fmaf(gv[u], kLog2e, G);
-                    GF[(t0 + u) * D + d] = G;
+            for (int u = 1; u < 32; ++u) gv[u] += gv[u - 1];
+            if (hh == 0) SS.half_tot[d] = gv[31];
+            __syncthreads();
+            const float add = hh ? SS.half_tot[d] : 0.f;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) GF[(32 * hh + u) * D + d] = gv[u] + add;
+        }
+        // the q and k row norms: thread (row r of [q; k], half hf2) sums 64 squares, the two
+        // halves of a row in lanes l and l ^ 8
+        {
+            const int r2 = ((pt >> 4) << 3) | (pt & 7), hf2 = (pt >> 3) & 1;  // row 0..127
+            const int t = r2 & 63;
+            const uint8_t* tile = sm + (r2 < C ? P_Q : P_K) + hf2 * 8192;
+            float ss = 0.f;
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {
+                const uint4 u = *reinterpret_cast<const uint4*>(tile + sw128(t, c8));
+                const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 x = unpack_bf16x2(wv[e]);
+                    ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
                 }
             }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+            const float inv = t > last ? 0.f : (p.qk_l2norm ? rsqrtf(fmaxf(ss, kNormEps * kNormEps)) : 1.f);
+            if (hf2 == 0) {
+                if (r2 < C) SS.inv_q[t] = inv; else SS.inv_k[t] = inv;
+            }
+        }
+        __syncthreads();
+        if (pt < D) {
+            const int d = pt;
             SS.dec[d] = ex2(GF[last * D + d]);
             // the exponents of the pair-sum factors this channel will use: row factors
             // G_t - R_I over block I, column factors R_I - G_s over s <= 16 I + 15
@@ -236,25 +274,7 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
                 worst = fmaxf(worst, R - lo);
             }
             if (!(worst <= 100.f)) SS.range_bad = 1;
-        } else {
-            const int r = pt - D;          // 0..127: q rows 0-63, k rows 64-127
-            const int t = r & 63;
-            const uint8_t* tile = sm + (r < C ? P_Q : P_K);
-            float ss = 0.f;
-#pragma unroll 4
-            for (int c8 = 0; c8 < 16; ++c8) {
-                const uint4 u = *reinterpret_cast<const uint4*>(tile + (c8 >> 3) * 8192 + sw128(t, c8 & 7));
-                const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 x = unpack_bf16x2(wv[e]);
-                    ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
-                }
-            }
-            const float inv = t > last ? 0.f : (p.qk_l2norm ? rsqrtf(fmaxf(ss, kNormEps * kNormEps)) : 1.f);
-            if (r < C) SS.inv_q[t] = inv; else SS.inv_k[t] = inv;
         }
-        __syncthreads();
 
         // O: the A operands of W^T and U~^T over the consumed g and the v tile:
         //    b . e^G . k^ (fp16) and w . v (fp16); eight elements (16 bytes) per step
@@ -268,12 +288,12 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
                 const uint4 bb = *reinterpret_cast<const uint4*>(sm + P_B + off);
                 const float ik = SS.inv_k[t];
                 const uint32_t kw[4] = {bk.x, bk.y, bk.z, bk.w}, gw[4] = {bb.x, bb.y, bb.z, bb.w};
+                float Gv[8];
+                load_row8(Gv, GF + t * D + c16 * 8);
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int d = c16 * 8 + 2 * u;
                     const float2 kk = unpack_bf16x2(kw[u]), gb = unpack_bf16x2(gw[u]);
-                    outw[u] = h2(gb.x * kk.x * ik * ex2(GF[t * D + d]),
-                                 gb.y * kk.y * ik * ex2(GF[t * D + d + 1]));
+                    outw[u] = h2(gb.x * kk.x * ik * ex2(Gv[2 * u]), gb.y * kk.y * ik * ex2(Gv[2 * u + 1]));
                 }
                 *reinterpret_cast<uint4*>(sm + P_G + off) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
             } else {
@@ -310,7 +330,7 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
                     Rv[0] = r0.x; Rv[1] = r0.y; Rv[2] = r0.z; Rv[3] = r0.w;
                     Rv[4] = r1.x; Rv[5] = r1.y; Rv[6] = r1.z; Rv[7] = r1.w;
                 }
-                float* ob;  // destination rows
+                uint32_t* ob;  // destination rows
                 int orow;
                 if (row < 16) {               // A rows: b_t k^_t e^{G_t - R}
                     const int t = 16 * I + row;
@@ -371,8 +391,9 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
                     ob = Yc;
                     orow = sidx;
                 }
-                *reinterpret_cast<float4*>(opsw(ob, orow, d0)) = make_float4(f[0], f[1], f[2], f[3]);
-                *reinterpret_cast<float4*>(opsw(ob, orow, d0 + 4)) = make_float4(f[4], f[5], f[6], f[7]);
+                uint32_t* op = ob + orow * kLdXY + d0;
+                *reinterpret_cast<uint4*>(op) = make_uint4(to_tf32(f[0]), to_tf32(f[1]), to_tf32(f[2]), to_tf32(f[3]));
+                *reinterpret_cast<uint4*>(op + 4) = make_uint4(to_tf32(f[4]), to_tf32(f[5]), to_tf32(f[6]), to_tf32(f[7]));
             }
             __syncthreads();
             const int ntA = 2 * (I + 1);
@@ -413,22 +434,27 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
             const uint4 raw = *reinterpret_cast<const uint4*>(tile + off);
             const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
             uint32_t outw[4];
+            float ev[8];  // exponents (log2)
+            if (which == 0) {
+                const int tg = p.read_pre ? t - 1 : t;
+                if (tg >= 0) {
+                    load_row8(ev, GF + tg * D + c16 * 8);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) ev[u] = 0.f;
+                }
+            } else {
+                float gl[8];
+                load_row8(ev, GF + t * D + c16 * 8);
+                load_row8(gl, GF + last * D + c16 * 8);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) ev[u] = gl[u] - ev[u];
+            }
+            const float sc = which == 0 ? p.scale * SS.inv_q[t] : SS.inv_k[t];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int d = c16 * 8 + 2 * u;
                 const float2 x = unpack_bf16x2(rw[u]);
-                float f0, f1;
-                if (which == 0) {
-                    const float sc = p.scale * SS.inv_q[t];
-                    const float G0 = p.read_pre ? (t > 0 ? GF[(t - 1) * D + d] : 0.f) : GF[t * D + d];
-                    const float G1 = p.read_pre ? (t > 0 ? GF[(t - 1) * D + d + 1] : 0.f) : GF[t * D + d + 1];
-                    f0 = sc * ex2(G0);
-                    f1 = sc * ex2(G1);
-                } else {
-                    f0 = SS.inv_k[t] * ex2(GF[last * D + d] - GF[t * D + d]);
-                    f1 = SS.inv_k[t] * ex2(GF[last * D + d + 1] - GF[t * D + d + 1]);
-                }
-                outw[u] = h2(x.x * f0, x.y * f1);
+                outw[u] = h2(x.x * sc * ex2(ev[2 * u]), x.y * sc * ex2(ev[2 * u + 1]));
             }
             *reinterpret_cast<uint4*>(tile + off) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
         }
