@@ -112,7 +112,7 @@ struct PrepSmall {
     float dec[D];         // e^{G_C} per channel
     float ones[C];        // column scales of the solve's T tiles (1: T itself)
     float half_tot[D];    // the cumulative log decay over the first 32 tokens, per channel
-    uint64_t mbar[2];     // tiles landed, W^T and U~^T done
+    uint64_t mbar[3];     // q, k, b, w tiles landed; W^T and U~^T done; v, g tiles landed
     uint32_t tmem_base;
     int range_bad;
 };
@@ -166,8 +166,7 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
         tmem_relinquish();
     }
     if (pt == 0) {
-        mbar_init(&SS.mbar[0], 1);
-        mbar_init(&SS.mbar[1], 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&SS.mbar[i], 1);
         mbar_init_fence();
         SS.range_bad = 0;
     }
@@ -185,33 +184,60 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
     float* RS = reinterpret_cast<float*>(sm + P_RS);
     bool fail = false;
 
-    int it = 0;
-    for (long long item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
+    // An item's tiles are loaded while the previous item finishes: q, k, b, w once its q~
+    // and K~ are out, v and g once its W and U~ products have read them.
+    struct ItemPos { int h, hk, last; long long t0; };
+    auto decode = [&](long long item) -> ItemPos {
+        ItemPos ip;
         const int cg = (int)(item / p.Hv);
-        const int h = (int)(item - (long long)cg * p.Hv);
-        const int hk = h / (p.Hv / p.Hk);
+        ip.h = (int)(item - (long long)cg * p.Hv);
+        ip.hk = ip.h / (p.Hv / p.Hk);
         const int s = p.chunk_seq[cg];
         const int c = cg - p.chunk_off[s];
-        const long long t0 = (long long)p.cu[s] + (long long)c * C;
-        const int Cc = (int)min((long long)C, (long long)p.cu[s + 1] - t0);
-        const int last = Cc - 1;
-
-        // L: the six tiles (tokens t0 .. t0 + 63; rows past the chunk are masked below)
-        if (pt == 0) {
-            uint64_t* bar = &SS.mbar[0];
-            mbar_expect_tx(bar, 12 * 8192);
-            const int z = (int)t0;
+        ip.t0 = (long long)p.cu[s] + (long long)c * C;
+        ip.last = (int)min((long long)C, (long long)p.cu[s + 1] - ip.t0) - 1;
+        return ip;
+    };
+    auto load_qkbw = [&](const ItemPos& ip) {  // thread 0
+        uint64_t* bar = &SS.mbar[0];
+        mbar_expect_tx(bar, 8 * 8192);
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                tma_load_3d(sbase + P_Q + hh * 8192, &tm_q, hh * 64, hk, z, bar);
-                tma_load_3d(sbase + P_K + hh * 8192, &tm_k, hh * 64, hk, z, bar);
-                tma_load_3d(sbase + P_V + hh * 8192, &tm_v, hh * 64, h, z, bar);
-                tma_load_3d(sbase + P_G + hh * 8192, &tm_g, hh * 64, h, z, bar);
-                tma_load_3d(sbase + P_B + hh * 8192, &tm_b, hh * 64, h, z, bar);
-                tma_load_3d(sbase + P_W + hh * 8192, &tm_w, hh * 64, h, z, bar);
-            }
+        for (int hh = 0; hh < 2; ++hh) {
+            tma_load_3d(sbase + P_Q + hh * 8192, &tm_q, hh * 64, ip.hk, (int)ip.t0, bar);
+            tma_load_3d(sbase + P_K + hh * 8192, &tm_k, hh * 64, ip.hk, (int)ip.t0, bar);
+            tma_load_3d(sbase + P_B + hh * 8192, &tm_b, hh * 64, ip.h, (int)ip.t0, bar);
+            tma_load_3d(sbase + P_W + hh * 8192, &tm_w, hh * 64, ip.h, (int)ip.t0, bar);
         }
-        const bool landed = mbar_wait_bounded(&SS.mbar[0], (uint32_t)(it & 1), kWaitNs);
+    };
+    auto load_vg = [&](const ItemPos& ip) {  // thread 0
+        uint64_t* bar = &SS.mbar[2];
+        mbar_expect_tx(bar, 4 * 8192);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            tma_load_3d(sbase + P_V + hh * 8192, &tm_v, hh * 64, ip.h, (int)ip.t0, bar);
+            tma_load_3d(sbase + P_G + hh * 8192, &tm_g, hh * 64, ip.h, (int)ip.t0, bar);
+        }
+    };
+    ItemPos cur = decode(blockIdx.x);
+    if (pt == 0) {
+        load_qkbw(cur);
+        load_vg(cur);
+    }
+    int pend = pt == 0 ? 3 : 0;  // tile groups in flight that nobody has waited for (bits 0, 1)
+
+    int it = 0;
+    for (long long item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
+        const int h = cur.h;
+        const int last = cur.last;
+        const long long nitem = item + gridDim.x;
+        const bool has_next = nitem < n_items;
+        ItemPos nx = cur;
+        if (has_next) nx = decode(nitem);  // its loads resolve while this item runs
+
+        // L: this item's six tiles (tokens t0 .. t0 + 63; rows past the chunk are masked)
+        bool landed = mbar_wait_bounded(&SS.mbar[0], (uint32_t)(it & 1), kWaitNs);
+        landed = mbar_wait_bounded(&SS.mbar[2], (uint32_t)(it & 1), kWaitNs) && landed;
+        if (landed) pend = 0;
         if (__syncthreads_or(landed ? 0 : 1)) { fail = true; break; }
 
         // N: per-channel cumulative log decay (log2 units): thread (channel d, half hh) scans
@@ -456,8 +482,11 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
                 const float2 x = unpack_bf16x2(rw[u]);
                 outw[u] = h2(x.x * sc * ex2(ev[2 * u]), x.y * sc * ex2(ev[2 * u + 1]));
             }
-            *reinterpret_cast<uint4*>(tile + off) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+            *reinterpret_cast<uint4*>(rec + (which == 0 ? REC_Q : REC_K) + off) =
+                make_uint4(outw[0], outw[1], outw[2], outw[3]);
         }
+        // q, k, b, w are consumed: the next item's land there during the solve
+        fence_proxy_async_smem();
         __syncthreads();
 
         // S: T = (I + A)^-1 (the blocked solve of the scalar kernel), T in fp16 over Y
@@ -472,7 +501,14 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
             wy_diag_stage0(vals, i, lane, hf, As, RS, Ts);
         }
         uint8_t* twu = sm + P_Y;
-        wy_solve_offdiag(As, Ts, RS, twu, SS.ones, SS.ones, pt, kBarG2, kPrepThreads, [](int) {});
+        // (the solve's first barrier also orders every read of the q, k, b, w tiles before
+        // the next item's tensor loads into them, issued after it)
+        wy_solve_offdiag(As, Ts, RS, twu, SS.ones, SS.ones, pt, kBarG2, kPrepThreads, [&](int phase) {
+            if (phase == 1 && has_next && pt == 0) {
+                load_qkbw(nx);
+                pend |= 1;
+            }
+        });
         fence_proxy_async_smem();
         tc_fence_before();
         named_bar(kBarG2, kPrepThreads);  // block column 0 of T complete
@@ -505,7 +541,7 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
             if (pt < 128) {
 #pragma unroll
                 for (int t = 0; t < C; ++t)
-                    *reinterpret_cast<__half*>(sm + P_B + tile16(t, j, 8192)) =
+                    *reinterpret_cast<__half*>(rec + REC_W + tile16(t, j, 8192)) =
                         __float2half_rn(-u2f(r2[t >> 5][t & 31]));
             } else {
 #pragma unroll
@@ -513,33 +549,30 @@ chunk_g2_prep_tc(G2Params p, const __grid_constant__ CUtensorMap tm_q,
                     float f[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) f[u] = u2f(r2[c8 >> 2][(c8 & 3) * 8 + u]);
-                    *reinterpret_cast<uint4*>(sm + P_W + sw128(j, c8)) = h8(f);
+                    *reinterpret_cast<uint4*>(rec + REC_U + sw128(j, c8)) = h8(f);
                 }
             }
         }
         tc_fence_before();
         if (__syncthreads_or(mdone ? 0 : 1)) { fail = true; break; }
-
-        // R: the rest of the record (q~, -W, K~, U~^T, e^{G_C}), 16-byte pieces
-        for (int e = pt; e < 4 * 1024 + 32; e += kPrepThreads) {
-            if (e < 4 * 1024) {
-                const int part = e >> 10, idx = e & 1023;
-                const uint32_t src = part == 0 ? P_Q : part == 1 ? P_B : part == 2 ? P_K : P_W;
-                const uint32_t dst = part == 0 ? REC_Q : part == 1 ? REC_W : part == 2 ? REC_K : REC_U;
-                reinterpret_cast<uint4*>(rec + dst)[idx] = reinterpret_cast<const uint4*>(sm + src)[idx];
-            } else {
-                reinterpret_cast<float4*>(rec + REC_D)[e - 4 * 1024] =
-                    reinterpret_cast<const float4*>(SS.dec)[e - 4 * 1024];
-            }
+        // the W and U~ products have read b e^G k^ and w v: the next item's v, g land there
+        if (has_next && pt == 0) {
+            load_vg(nx);
+            pend |= 2;
         }
+        // R: the per-channel decay of the chunk
+        if (pt < 32) reinterpret_cast<float4*>(rec + REC_D)[pt] = reinterpret_cast<const float4*>(SS.dec)[pt];
         if (SS.range_bad && pt == 0) atomicCAS(&p.hdr->err, (int)GDR_OK, (int)GDR_ERR_RANGE);
-        __syncthreads();  // the next item's tiles land over this one's
+        cur = nx;
     }
 
     if (fail && pt == 0) {
         atomicExch(&p.hdr->err, (int)GDR_ERR_TIMEOUT);
-        // no tile may land after the CTA has left its shared memory
-        mbar_wait_bounded(&SS.mbar[0], (uint32_t)(it & 1), kWaitNs);
+        // no tile may land after the CTA has left its shared memory (the groups in flight
+        // belong to item `it`, or to `it + 1` when this item's were waited for)
+        const uint32_t par = (uint32_t)(it & 1);
+        if (pend & 1) mbar_wait_bounded(&SS.mbar[0], par, kWaitNs) || mbar_wait_bounded(&SS.mbar[0], par ^ 1u, kWaitNs);
+        if (pend & 2) mbar_wait_bounded(&SS.mbar[2], par, kWaitNs) || mbar_wait_bounded(&SS.mbar[2], par ^ 1u, kWaitNs);
     }
     tc_fence_before();
     __syncthreads();
