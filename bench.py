@@ -481,9 +481,18 @@ def bench_ours(args, rank, world, local_rank):
             torch.cuda.synchronize()
             barrier()
             cms = max_over_ranks(c0.elapsed_time(c1) / g2steps, world)
+            # the least HBM traffic of the call: q, k, v and the three gate tensors read once,
+            # o and S_final written once (the tensor-core path's per-chunk records, written
+            # and read back through the workspace, are not counted)
+            g2bytes = sum(d[n].numel() * d[n].element_size() for n in ("q", "k", "v")) + sum(
+                t.numel() * t.element_size() for t in (gg, gb, gw)) + (
+                o.numel() * o.element_size() + S_final.numel() * 4)
             gdn2["chunk"] = {"workload": w.name, "ms_per_step": cms, "steps": g2steps,
                              "value": whole_job_rate(tokens, world, cms), "unit": "tokens/s",
-                             "path": gdr.chunk_fwd_path(g2args)}
+                             "path": gdr.chunk_fwd_path(g2args),
+                             "algorithmic_bytes": g2bytes,
+                             "hbm_frac": g2bytes / (cms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                             "vs_scalar_forward": cms / ms}
             del g2ws
         if dec is not None:
             dg, db, dwg = (t.to(dev) for t in workloads.gdn2_gate_inputs(

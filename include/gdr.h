@@ -117,7 +117,10 @@ typedef struct {
      *             erase gate b [.., Hv, dk], and gdn2_w the per-value-channel write gate
      *             [.., Hv, dv], all gate_dtype and 16-byte aligned.  With g = log(alpha),
      *             b = w = beta on every channel this is the scalar rule.  Not combined with
-     *             gate_raw. */
+     *             gate_raw.  bf16 inputs and gates with dk = dv = 128, chunk 64 and forward
+     *             scans take the tensor cores (a preparation kernel over every chunk and
+     *             head, then the recursion); a chunk whose per-channel decay grows by more
+     *             than 2^100 within 16 tokens is refused there with GDR_ERR_RANGE. */
     int gdn2;
     const void* gdn2_w;
     /* Optional device status word (NULL: none).  A device int owned by the caller, who
@@ -174,7 +177,8 @@ gdr_status gdr_chunk_fwd(const gdr_chunk_args* args,
  *
  * - Calls whose scratch need (gdr_chunk_fwd_workspace_size) exceeds the array return
  *   GDR_ERR_WORKSPACE and enqueue nothing.  The tensor-core path needs only
- *   256 + 8 (n_seqs + 1) + 4 (ceil(B*T / chunk) + n_seqs) bytes; the CUDA-core path
+ *   256 + 8 (n_seqs + 1) + 4 (ceil(B*T / chunk) + n_seqs) bytes (with gdn2 another 74240
+ *   bytes per chunk and value head); the CUDA-core path
  *   additionally 4 B*T Hv (dk + dv + 1) bytes (4 B*T Hv (2 dk + dv) with gdn2), and for
  *   chunk <= 64 with dk a multiple of 32 up to 128 another 8 B*T Hv dk +
  *   4 (ceil(B*T / chunk) + n_seqs) Hv chunk^2 bytes, so it fits only small problems.
