@@ -46,7 +46,8 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-CHUNK_TC_SOURCES = ("chunk_tc.cu", "tc_ptx.cuh", "common.cuh")
+CHUNK_TC_SOURCES = ("chunk_tc.cu", "wy_solve.cuh", "tc_ptx.cuh", "common.cuh")
+G2_TC_SOURCES = ("chunk_g2_tc.cu", "wy_solve.cuh", "tc_ptx.cuh", "common.cuh")
 DECODE_SOURCES = ("decode.cu", "common.cuh")
 
 
@@ -453,7 +454,7 @@ def bench_ours(args, rank, world, local_rank):
     # ---------------- GDN-2 (decoupled per-channel gates): the chunk workload on the CUDA-core
     # path and the decode steps, same inputs with g, beta per key channel and a write gate
     gdn2 = None
-    if args.gdn2 and not args.rows:
+    if args.gdn2:
         gdn2 = {}
         if args.only != "decode":
             gg, gb, gw = (t.to(dev) for t in workloads.gdn2_gate_inputs(
@@ -493,8 +494,13 @@ def bench_ours(args, rank, world, local_rank):
                              "algorithmic_bytes": g2bytes,
                              "hbm_frac": g2bytes / (cms / 1e3) / 1e9 / peaks["hbm_gbs"],
                              "vs_scalar_forward": cms / ms}
+            if gdn2["chunk"]["path"] == "tc":
+                # measured traffic of the two kernels of a call (the records included)
+                tp = [measured_traffic(k, G2_TC_SOURCES, w.B)
+                      for k in ("chunk_g2_prep_tc", "chunk_g2_chain_tc")]
+                gdn2["chunk"]["traffic"] = None if None in tp else sum(tp)
             del g2ws
-        if dec is not None:
+        if dec is not None and not args.rows:
             dg, db, dwg = (t.to(dev) for t in workloads.gdn2_gate_inputs(
                 (dw.steps, dw.N, dw.Hv), dw.dk, dw.dv, dw.gate_dtype, seed=rank))
 

@@ -205,3 +205,11 @@ def oracle_backward_sequence(job):
     arrays, kw = job
     ref = obw.backward(*arrays, **kw)
     return {n: a.astype(np.float32) for n, a in ref.items()}
+
+
+def oracle_gdn2_sequence(job):
+    """One sequence of a fixed-length workload through the fp64 GDN-2 oracle (a process
+    pool's task; the reference returns as float32, far below any bound it meets)."""
+    arrays, kw = job
+    o, S = oracle.gdn2_forward(*arrays, **kw)
+    return o.astype(np.float32), S.astype(np.float32)

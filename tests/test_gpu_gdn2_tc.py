@@ -10,7 +10,9 @@ import torch
 import oracle
 import workloads
 import gated_delta_rule_146_b200 as gdr
-from gpu_helpers import assert_close, to_dev
+import numpy as np
+
+from gpu_helpers import Accum, assert_close, oracle_gdn2_sequence, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -69,3 +71,29 @@ def test_tensor_core_gdn2_scalar_gates_match_gated_delta_rule():
     o_r, S_r = oracle.forward(x["q"], x["k"], x["v"], g[..., 0], b[..., 0], x["S0"], scale=0.1)
     assert_close("o", o, o_r, torch.bfloat16)
     assert_close("S", S, S_r, torch.bfloat16, kind="state")
+
+
+def test_training_shape_workload_whole():
+    """The GDN-2 forward at the training workload's full size (8 x 4096 tokens, 16 heads,
+    d = 128, bf16, the bench's GDN-2 gates): every element of o and S_final against the
+    oracle, one sequence per process of a spawned pool."""
+    import multiprocessing as mp
+    w = workloads.WORKLOADS["bf16_b8_h16_t4096_d128"]
+    x = workloads.workload_inputs(w)
+    g, b, wg = workloads.gdn2_gate_inputs(x["v"].shape[:3], w.dk, w.dv, w.gate_dtype, seed=0)
+    o, S = run(x, g, b, wg, read_mode=w.read_mode, scale=w.scale)
+    o, S = o.cpu(), S.cpu()
+    f32 = lambda t: None if t is None else t.float().numpy()
+    jobs = []
+    for r in range(w.B):
+        sl = lambda t: f32(t[r:r + 1])
+        arrays = (sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(g), sl(b), sl(wg),
+                  None if x["S0"] is None else f32(x["S0"][r:r + 1]))
+        jobs.append((arrays, {"read_mode": w.read_mode, "scale": w.scale}))
+    ao, aS = Accum("o", torch.bfloat16, "out"), Accum("S_final", torch.bfloat16, "state")
+    with mp.get_context("spawn").Pool(min(w.B, max(1, mp.cpu_count()))) as pool:
+        for r, (o_r, S_r) in enumerate(pool.imap(oracle_gdn2_sequence, jobs)):
+            ao.add(o[r:r + 1], o_r.astype(np.float64), label=f" row {r}")
+            aS.add(S[r:r + 1], S_r.astype(np.float64), label=f" row {r}")
+    ao.check()
+    aS.check()
