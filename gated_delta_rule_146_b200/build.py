@@ -18,6 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgdr.so")
 SOURCES = ["api.cu", "plan.cu", "chunk_simt.cu", "chunk_tc.cu", "chunk_g2_tc.cu", "chunk_bwd.cu",
+           "chunk_bwd_tc.cu",
            "decode.cu", "noalloc.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]

@@ -34,7 +34,7 @@
 //   bwd_reduce_heads       dq, dk summed over each key head's v-heads
 #include <algorithm>
 
-#include "common.cuh"
+#include "chunk_bwd.cuh"
 
 namespace gdr {
 
@@ -44,23 +44,7 @@ constexpr int kThreads = 256;  // state passes and the head reduction
 constexpr int kNT = 512;       // per-(chunk, head) kernels: 16 warps over 64 rows
 constexpr int kSlice = 32;     // dv columns per state-pass block (one per lane)
 
-struct BwdParams {
-    const void *q, *k, *v, *g, *beta, *dO;
-    const float *S0, *dS_final;
-    void *dq_out, *dk_out, *dv_out, *dg_out, *dbeta_out;
-    float* dS0;
-    const WsHeader* hdr; const int32_t *cu, *chunk_off, *chunk_seq;
-    const float *W, *U, *G;         // from chunk_local_simt: [T][Hv][dk], [T][Hv][dv], [T][Hv]
-    float *Hc, *dHc;                // [max_chunks][Hv][dk][dv]: H at chunk start, dH+
-    float *Vp, *dVp;                // [T][Hv][dv]: V', dV'
-    float *dW, *dKp, *dqh, *dkh;    // [T][Hv][dk]
-    float* dGp;                     // [T][Hv]
-    const float *Qt, *Kt;           // [T][Hv][dk]: s e^{G'} q^, e^{G_C - G} k^ (chunk_prep_simt)
-    const float* Pc;                // [max_chunks][Hv][C][C]: P, zero off the mask
-    int Hk, Hv, dk, dv, chunk, read_pre, qk_l2norm, reverse;
-    gdr_dtype io, gt;
-    float scale;
-};
+
 
 // Normalise `rows` rows of length n (stride ld) in shared memory, one warp per row, and
 // record each row's norm |x| (needed by the adjoint).
@@ -97,22 +81,6 @@ struct Tile {
     __device__ int col(int jj) const { return cg + 32 * jj; }
 };
 
-struct ChunkPos {
-    int s, c, jc, p0, Cc;
-    long long t0, t1;
-};
-
-__device__ __forceinline__ bool chunk_pos(const BwdParams& p, ChunkPos& cp) {
-    cp.c = blockIdx.x;
-    if (cp.c >= p.hdr->n_chunks) return false;
-    cp.s = p.chunk_seq[cp.c];
-    cp.t0 = p.cu[cp.s];
-    cp.t1 = p.cu[cp.s + 1];
-    cp.jc = cp.c - p.chunk_off[cp.s];
-    cp.p0 = cp.jc * p.chunk;
-    cp.Cc = (int)min((long long)p.chunk, (cp.t1 - cp.t0) - cp.p0);
-    return true;
-}
 
 // ---- state passes: one block per (sequence, v-head, 32-column slice of dv) ---------------
 //
@@ -980,7 +948,11 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
     const dim3 gs((unsigned)a.n_seqs, (unsigned)a.Hv, (unsigned)(a.dv / kSlice));
     if ((s = launch_states(a, p, gs, st)) != GDR_OK) return s;
     if (L.max_chunks > 0) {
-        bwd_chunk_dqk<<<gc, kNT, sm_q, st>>>(p);
+        if (bwd_dqk_tc_supported(a)) {
+            if ((s = launch_bwd_dqk_tc(p, gc, st)) != GDR_OK) return s;
+        } else {
+            bwd_chunk_dqk<<<gc, kNT, sm_q, st>>>(p);
+        }
         bwd_chunk_wy<<<gc, kNT, sm_w, st>>>(p);
         const long long n = (long long)a.B * a.T * a.Hk * a.dk;
         const unsigned blocks = (unsigned)std::min<long long>((n + kThreads - 1) / kThreads, 148LL * 16);
