@@ -950,10 +950,11 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
     if (L.max_chunks > 0) {
         if (bwd_dqk_tc_supported(a)) {
             if ((s = launch_bwd_dqk_tc(p, gc, st)) != GDR_OK) return s;
+            if ((s = launch_bwd_wy_tc(p, gc, st)) != GDR_OK) return s;
         } else {
             bwd_chunk_dqk<<<gc, kNT, sm_q, st>>>(p);
+            bwd_chunk_wy<<<gc, kNT, sm_w, st>>>(p);
         }
-        bwd_chunk_wy<<<gc, kNT, sm_w, st>>>(p);
         const long long n = (long long)a.B * a.T * a.Hk * a.dk;
         const unsigned blocks = (unsigned)std::min<long long>((n + kThreads - 1) / kThreads, 148LL * 16);
         if (n > 0) bwd_reduce_heads<<<blocks, kThreads, 0, st>>>(p, n);

@@ -42,8 +42,10 @@ __device__ __forceinline__ bool chunk_pos(const BwdParams& p, ChunkPos& cp) {
     return true;
 }
 
-// The tensor-core dq / dK / dW step: bf16 inputs, dk = dv = 128, chunk 64.
+// The tensor-core per-chunk steps (dq / dK / dW, then the WY step): bf16 inputs,
+// dk = dv = 128, chunk 64.
 bool bwd_dqk_tc_supported(const gdr_chunk_args& a);
 gdr_status launch_bwd_dqk_tc(const BwdParams& p, dim3 grid, cudaStream_t st);
+gdr_status launch_bwd_wy_tc(const BwdParams& p, dim3 grid, cudaStream_t st);
 
 }  // namespace gdr

@@ -30,6 +30,7 @@
 // folded into the other operand.  fp16 keeps 11 significant bits against bf16's 8.
 #include "chunk_bwd.cuh"
 #include "tc_ptx.cuh"
+#include "wy_solve.cuh"
 
 namespace gdr {
 
@@ -75,8 +76,6 @@ struct DqkSmall {
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + sizeof(DqkSmall) + 1024;
 static_assert(OFF_SMALL + sizeof(DqkSmall) + 1024 <= 227 * 1024, "shared memory");
 
-__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
-
 __device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return sdesc_sw128(saddr, 16, 1024); }
 
 // The power of two that maps a row whose largest magnitude is m into [2^14, 2^15): 2^(15 - e)
@@ -97,6 +96,12 @@ __device__ __forceinline__ float max16(float m) {
 __device__ __forceinline__ float sum16(float m) {
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) m += __shfl_xor_sync(0xffffffffu, m, o);
+    return m;
+}
+
+__device__ __forceinline__ float warp_max(float m) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     return m;
 }
 
@@ -552,6 +557,486 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
     if (fail && tid == 0) atomicExch(const_cast<int*>(&p.hdr->err), (int)GDR_ERR_TIMEOUT);
 }
 
+
+// ============================================================================================
+// The WY step: what bwd_chunk_wy (chunk_bwd.cu) computes, on the tensor cores.
+//     A     = strict_lower(diag(beta) (K^ K^T) . e^{G_i - G_j}),  T = (I + A)^-1 (blocked solve)
+//     dR    = [dR_w | dR_u] = T^T [dW | dV']
+//     dA    = -(dR_w W^T + dR_u U~^T) on the strict lower triangle, D = dA . e^{G_i - G_j}
+//     dK^   = (beta D + (beta D)^T) K^ + diag(beta e^G) dR_w + (the P and carry parts)
+//     dv    = diag(beta) dR_u,  dbeta, dg (reverse cumulative sum of dG within the chunk)
+// Products (tcgen05, fp16 operands, fp32 accumulators):
+//     P1  [k; -] k^T             rows 0-63: k_i . k_j
+//     P2  [dW | dV']^T T         two M = 128 blocks: dR_w^T, dR_u^T (lane = feature, column = i)
+//     P3  [dR; -] [W | U~]^T     rows 0-63: -dA
+//     P4  K^T (beta D + (beta D)^T)^T     dK^T (lane = d, column = i)
+// The solve is the forward's (wy_solve.cuh): the diagonal 16x16 inverses by substitution,
+// the blocks below them by tf32 warp MMAs, T written as an fp16 tile.  [dW | dV'] and dR take
+// one power-of-two factor per tile (their rows run along a K index); the rows of k and of
+// [W | U~] and of the combined beta D take one each.
+
+constexpr int kBarWy = 1, kBarSolve = 2;
+constexpr uint32_t W_K = 0;         // k rows (K = d): 2 groups x 8 KB
+constexpr uint32_t W_R = 16384;     // [dW | dV'] rows j: 4 groups x 8 KB (x = feature)
+constexpr uint32_t W_WF = 49152;    // [W | U~] rows j: 4 groups x 8 KB
+constexpr uint32_t W_T = 81920;     // T (fp16, [i][j]), a second copy 8 KB on
+constexpr uint32_t W_DR = 98304;    // dR rows i (K = x): 4 groups x 8 KB
+constexpr uint32_t W_AS = 131072;   // A below the diagonal (fp32), then beta D (fp32)
+constexpr uint32_t W_TS = 147456;   // T (fp32) of the solve
+constexpr uint32_t W_RS = 163840;   // the solve's diagonal blocks
+constexpr uint32_t W_BS = 167936;   // (beta D + (beta D)^T) diag(1/|k|) rows i (K = j): 8 KB
+constexpr uint32_t W_SMALL = 176128;
+constexpr uint32_t WT_SK = 0, WT_DRW = 64, WT_DRU = 128, WT_DA = 192, WT_DK = 0;
+
+struct WySmall {
+    float G[64], beta[64], ones[64], invk[64], nk[64];
+    float rk[64], rw[64], rbs[64];    // reciprocal row factors: k, [W | U~], beta D + ...
+    float rr[2], rdr;                 // reciprocal tile factors: dW, dV' halves; dR
+    float mx[8][3];                   // per-warp largest magnitudes (dW, dV'; dR)
+    float bsmax[2][64];               // largest |Bs'| of row i, by column half
+    float dgr[2][64], dgc[2][64], db[2][64];  // from dA: row sums, column sums, beta parts
+    float rred[4][64], pred[4][64], vred[4][64];  // k^ . dR_w, k^ . acc, v . dR_u by lane quarter
+    uint64_t mbar[4];
+    uint32_t tmem;
+    int range_bad;
+};
+constexpr uint32_t W_SMEM = W_SMALL + sizeof(WySmall) + 1024;
+static_assert(W_SMALL + sizeof(WySmall) + 1024 <= 227 * 1024, "shared memory");
+
+__global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(sm);
+    WySmall& SS = *reinterpret_cast<WySmall*>(sm + W_SMALL);
+    if (p.hdr->err != GDR_OK) return;
+    ChunkPos cp;
+    if (!chunk_pos(p, cp)) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int sp = warp & 3, ch = warp >> 2;
+    const int h = blockIdx.y, hk = h / (p.Hv / p.Hk), Cc = cp.Cc;
+    const bool on = p.qk_l2norm != 0;
+    auto tok = [&](int i) { return phys_token(cp.t0, cp.t1, cp.p0 + i, p.reverse); };
+    float* As = reinterpret_cast<float*>(sm + W_AS);
+    float* Ts = reinterpret_cast<float*>(sm + W_TS);
+
+    if (warp == 0) {
+        tmem_alloc(&SS.tmem, 256);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    if (tid == 0) {
+        for (int b = 0; b < 4; ++b) mbar_init(&SS.mbar[b], 1);
+        mbar_init_fence();
+        SS.range_bad = 0;
+    }
+    if (tid < 64) {
+        const bool lt = tid < Cc;
+        const size_t gi = lt ? (size_t)tok(tid) * p.Hv + h : 0;
+        SS.G[tid] = lt ? p.G[gi] : 0.f;
+        SS.beta[tid] = lt ? load_elem(p.beta, gi, p.gt) : 0.f;
+        SS.ones[tid] = 1.f;
+    }
+
+    // ---- staging
+    {
+        // k rows (bf16), with their norms
+        uint4 raw[4];
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int idx = tid + it * kTh, i = idx >> 4, c = idx & 15;
+            raw[it] = make_uint4(0, 0, 0, 0);
+            if (i < Cc)
+                raw[it] = __ldg(static_cast<const uint4*>(p.k) + ((size_t)tok(i) * p.Hk + hk) * 16 + c);
+        }
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int idx = tid + it * kTh, i = idx >> 4, c = idx & 15;
+            float f[8];
+            bf16x8_to_f32(raw[it], f);
+            const float sc = pow2_scale(max16(amax8(f)));
+            *reinterpret_cast<uint4*>(sm + W_K + (c >> 3) * 8192 + sw128(i, c & 7)) = f16x8(f, sc);
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+            ss = sum16(ss);
+            if (c == 0) {
+                const float n = sqrtf(ss);
+                SS.rk[i] = __frcp_rn(sc);
+                SS.nk[i] = n;
+                SS.invk[i] = on ? 1.f / fmaxf(n, kNormEps) : 1.f;
+            }
+        }
+    }
+    {
+        // [W | U~] rows j (fp32): one factor per row over both halves
+#pragma unroll 1
+        for (int it0 = 0; it0 < 4; it0 += 2) {
+            float4 a[2][4];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int idx = tid + (it0 + u) * kTh, j = idx >> 4, c = idx & 15;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) a[u][v] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (j < Cc) {
+                    const size_t row = ((size_t)tok(j) * p.Hv + h) * 128 + c * 8;
+                    const float4* w4 = reinterpret_cast<const float4*>(p.W + row);
+                    const float4* u4 = reinterpret_cast<const float4*>(p.U + row);
+                    a[u][0] = __ldg(w4); a[u][1] = __ldg(w4 + 1);
+                    a[u][2] = __ldg(u4); a[u][3] = __ldg(u4 + 1);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int idx = tid + (it0 + u) * kTh, j = idx >> 4, c = idx & 15;
+                float fw[8], fu[8];
+                f4x2_to_f32(a[u][0], a[u][1], fw);
+                f4x2_to_f32(a[u][2], a[u][3], fu);
+                const float sc = pow2_scale(max16(fmaxf(amax8(fw), amax8(fu))));
+                *reinterpret_cast<uint4*>(sm + W_WF + (c >> 3) * 8192 + sw128(j, c & 7)) = f16x8(fw, sc);
+                *reinterpret_cast<uint4*>(sm + W_WF + (2 + (c >> 3)) * 8192 + sw128(j, c & 7)) = f16x8(fu, sc);
+                if (c == 0) SS.rw[j] = __frcp_rn(sc);
+            }
+        }
+    }
+    // [dW | dV'] (fp32) held in registers until the tile's largest magnitudes are known
+    float4 rv[4][2][2];  // [piece][dW, dV'][half]
+    {
+        float mw = 0.f, mv = 0.f;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int idx = tid + it * kTh, j = idx >> 4, c = idx & 15;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) rv[it][t][0] = rv[it][t][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (j < Cc) {
+                const size_t row = ((size_t)tok(j) * p.Hv + h) * 128 + c * 8;
+                const float4* w4 = reinterpret_cast<const float4*>(p.dW + row);
+                const float4* v4 = reinterpret_cast<const float4*>(p.dVp + row);
+                rv[it][0][0] = __ldg(w4); rv[it][0][1] = __ldg(w4 + 1);
+                rv[it][1][0] = __ldg(v4); rv[it][1][1] = __ldg(v4 + 1);
+            }
+            float f[8];
+            f4x2_to_f32(rv[it][0][0], rv[it][0][1], f);
+            mw = fmaxf(mw, amax8(f));
+            f4x2_to_f32(rv[it][1][0], rv[it][1][1], f);
+            mv = fmaxf(mv, amax8(f));
+        }
+        mw = warp_max(mw);
+        mv = warp_max(mv);
+        if (lane == 0) { SS.mx[warp][0] = mw; SS.mx[warp][1] = mv; }
+    }
+    __syncthreads();
+    {
+        float mw = 0.f, mv = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) { mw = fmaxf(mw, SS.mx[w][0]); mv = fmaxf(mv, SS.mx[w][1]); }
+        const float sw = pow2_scale(mw), sv = pow2_scale(mv);
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int idx = tid + it * kTh, j = idx >> 4, c = idx & 15;
+            float f[8];
+            f4x2_to_f32(rv[it][0][0], rv[it][0][1], f);
+            *reinterpret_cast<uint4*>(sm + W_R + (c >> 3) * 8192 + sw128(j, c & 7)) = f16x8(f, sw);
+            f4x2_to_f32(rv[it][1][0], rv[it][1][1], f);
+            *reinterpret_cast<uint4*>(sm + W_R + (2 + (c >> 3)) * 8192 + sw128(j, c & 7)) = f16x8(f, sv);
+        }
+        if (tid == 0) { SS.rr[0] = __frcp_rn(sw); SS.rr[1] = __frcp_rn(sv); }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = SS.tmem;
+    const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
+
+    // ---- P1: k . k
+    if (tid == 0) {
+        const uint32_t id = idesc_f32acc(128, 64, false, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t o = (kk >> 2) * 8192 + (kk & 3) * 32;
+            mma_f32acc_ss(tmem + WT_SK, kdesc(sbase + W_K + o), kdesc(sbase + W_K + o), id, kk > 0);
+        }
+        mma_commit(&SS.mbar[0]);
+    }
+    bool fail = !mbar_wait_bounded(&SS.mbar[0], 0, kWaitNs);
+    fail = __syncthreads_or(fail);
+    tc_fence_after();
+
+    // ---- A (rows i = 0-63: warps 0, 1 and 4, 5) and the solve T = (I + A)^-1
+    if (!fail) {
+        if (sp < 2) {
+            const int i = sp * 32 + lane;
+            uint32_t rs[32];
+            tmem_ld32(tl + WT_SK + ch * 32, rs);
+            tmem_wait_ld();
+            const float f = SS.beta[i] * SS.rk[i] * SS.invk[i], gi = SS.G[i];
+            float vals[32];
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                const int j = ch * 32 + u;
+                const bool m = i < Cc && j < i;
+                vals[u] = m ? f * u2f(rs[u]) * SS.rk[j] * SS.invk[j] * exp2f((gi - SS.G[j]) * kLog2e) : 0.f;
+            }
+            // the solve's layout: warp 1 holds only blocks below the diagonal, warps 0 and 5 the
+            // diagonal blocks (and A_10, A_32), warp 4 none that it reads
+            if (warp == 1) {
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4)
+                    *reinterpret_cast<float4*>(f32sw(As, i, e4 * 4)) =
+                        make_float4(vals[e4 * 4], vals[e4 * 4 + 1], vals[e4 * 4 + 2], vals[e4 * 4 + 3]);
+            } else if (warp == 0 || warp == 5) {
+                wy_diag_stage0(vals, i, lane, ch, As, reinterpret_cast<float*>(sm + W_RS), Ts);
+            }
+        }
+        wy_solve_offdiag(As, Ts, reinterpret_cast<float*>(sm + W_RS), sm + W_T, SS.ones, SS.ones, tid,
+                         kBarSolve, kTh, [](int) {});
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- P2: dR^T = [dW | dV']^T T (A and B MN-major)
+    if (tid == 0 && !fail) {
+        const uint32_t id = idesc_f32acc(128, 64, true, true, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t b = sdesc_sw128(sbase + W_T + kk * 2048, 8192, 1024);
+            mma_f32acc_ss(tmem + WT_DRW, sdesc_sw128(sbase + W_R + kk * 2048, 8192, 1024), b, id, kk > 0);
+            mma_f32acc_ss(tmem + WT_DRU, sdesc_sw128(sbase + W_R + 16384 + kk * 2048, 8192, 1024), b, id, kk > 0);
+        }
+        mma_commit(&SS.mbar[1]);
+    }
+    if (!fail) fail = !mbar_wait_bounded(&SS.mbar[1], 0, kWaitNs);
+    fail = __syncthreads_or(fail);
+    tc_fence_after();
+    // dR into shared memory as rows i (K = feature x), one factor for the tile; every warp
+    // (lanes: the feature within its block, columns: positions 32 ch .. 32 ch + 31)
+    if (!fail) {
+        uint32_t ra[32], rb[32];
+        tmem_ld32(tl + WT_DRW + ch * 32, ra);
+        tmem_ld32(tl + WT_DRU + ch * 32, rb);
+        tmem_wait_ld();
+        const float r0 = SS.rr[0], r1 = SS.rr[1];
+        float m = 0.f;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            m = max_abs_nan(m, u2f(ra[u]) * r0);
+            m = max_abs_nan(m, u2f(rb[u]) * r1);
+        }
+        m = warp_max(m);
+        if (lane == 0) SS.mx[warp][2] = m;
+        __syncthreads();
+        float mt = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) mt = max_abs_nan(mt, SS.mx[w][2]);
+        if (!(mt <= 3.402823e38f) && tid == 0) SS.range_bad = 1;
+        const float sd = pow2_scale(mt);
+        uint16_t* dr = reinterpret_cast<uint16_t*>(sm + W_DR);
+        const int xa = sp * 32 + lane;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            const int i = ch * 32 + u;
+            const __half ha = __float2half_rn(u2f(ra[u]) * r0 * sd);
+            const __half hb = __float2half_rn(u2f(rb[u]) * r1 * sd);
+            dr[((xa >> 6) * 8192 + sw128(i, (xa >> 3) & 7)) / 2 + (xa & 7)] = *reinterpret_cast<const uint16_t*>(&ha);
+            dr[((2 + (xa >> 6)) * 8192 + sw128(i, (xa >> 3) & 7)) / 2 + (xa & 7)] = *reinterpret_cast<const uint16_t*>(&hb);
+        }
+        if (tid == 0) SS.rdr = __frcp_rn(sd);
+    } else {
+        __syncthreads();  // the barrier every thread of the branch above takes
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- P3: -dA = dR [W | U~]^T (K = 256)
+    if (tid == 0 && !fail) {
+        const uint32_t id = idesc_f32acc(128, 64, false, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            const uint32_t o = (kk >> 2) * 8192 + (kk & 3) * 32;
+            mma_f32acc_ss(tmem + WT_DA, kdesc(sbase + W_DR + o), kdesc(sbase + W_WF + o), id, kk > 0);
+        }
+        mma_commit(&SS.mbar[2]);
+    }
+    if (!fail) fail = !mbar_wait_bounded(&SS.mbar[2], 0, kWaitNs);
+    fail = __syncthreads_or(fail);
+    tc_fence_after();
+    // dA -> D, the decay and beta gradients it carries, beta D (rows i: warps 0, 1, 4, 5)
+    if (!fail && sp < 2) {
+        const int i = sp * 32 + lane;
+        uint32_t rd[32], rs[32];
+        tmem_ld32(tl + WT_DA + ch * 32, rd);
+        tmem_ld32(tl + WT_SK + ch * 32, rs);
+        tmem_wait_ld();
+        const float bi = SS.beta[i], gi = SS.G[i], fk = SS.rk[i] * SS.invk[i], rdr = SS.rdr;
+        float col[32], bd[32], db = 0.f, dg = 0.f;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            const int j = ch * 32 + u;
+            const bool m = i < Cc && j < i;
+            const float dA = -u2f(rd[u]) * rdr * SS.rw[j];
+            const float sk = u2f(rs[u]) * fk * SS.rk[j] * SS.invk[j];
+            const float e = exp2f((gi - SS.G[j]) * kLog2e);
+            const float D = m ? dA * e : 0.f;
+            db = fmaf(D, sk, db);
+            const float ga = m ? dA * (bi * sk * e) : 0.f;
+            dg += ga;
+            col[u] = -ga;
+            bd[u] = bi * D;
+        }
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4)
+            *reinterpret_cast<float4*>(f32sw(As, i, ch * 32 + e4 * 4)) =
+                make_float4(bd[e4 * 4], bd[e4 * 4 + 1], bd[e4 * 4 + 2], bd[e4 * 4 + 3]);
+        SS.db[ch][i] = db;
+        SS.dgr[ch][i] = dg;
+        const float cs = transpose_reduce32<false>(col, lane);
+        SS.dgc[sp][ch * 32 + lane] = cs;
+        named_bar(kBarWy, 128);
+        // Bs'_ij = (beta_i D_ij + beta_j D_ji) / |k_j| / (k_j's factor): the B operand of P4
+        float bm = 0.f;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            const int j = ch * 32 + u;
+            bd[u] = (bd[u] + *f32sw(As, j, i)) * SS.invk[j] * SS.rk[j];
+            bm = fmaxf(bm, fabsf(bd[u]));
+        }
+        SS.bsmax[ch][i] = bm;
+        named_bar(kBarWy, 128);
+        const float sb = pow2_scale(fmaxf(SS.bsmax[0][i], SS.bsmax[1][i]));
+#pragma unroll
+        for (int e8 = 0; e8 < 4; ++e8) {
+            float f[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) f[u] = bd[e8 * 8 + u];
+            *reinterpret_cast<uint4*>(sm + W_BS + sw128(i, ch * 4 + e8)) = f16x8(f, sb);
+        }
+        if (ch == 0) SS.rbs[i] = __frcp_rn(sb);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- P4: dK^T = K^T Bs'^T (A = the k tile, MN-major; B = Bs' rows i)
+    if (tid == 0 && !fail) {
+        const uint32_t id = idesc_f32acc(128, 64, true, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            mma_f32acc_ss(tmem + WT_DK, sdesc_sw128(sbase + W_K + kk * 2048, 8192, 1024),
+                          kdesc(sbase + W_BS + kk * 32), id, kk > 0);
+        mma_commit(&SS.mbar[3]);
+    }
+    const int x = sp * 32 + lane;  // feature: d of dR_w and dK, e of dR_u and dv
+    // dv = beta dR_u and v . dR_u while P4 runs (every warp: lanes = e, columns = i)
+    if (!fail) {
+        uint32_t rb[32];
+        tmem_ld32(tl + WT_DRU + ch * 32, rb);
+        tmem_wait_ld();
+        const float r1 = SS.rr[1];
+        float vp[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            const int i = ch * 32 + u;
+            vp[u] = 0.f;
+            if (i < Cc) {
+                const float du = u2f(rb[u]) * r1;
+                const size_t o = ((size_t)tok(i) * p.Hv + h) * 128 + x;
+                store_elem(p.dv_out, o, SS.beta[i] * du, p.io);
+                vp[u] = load_elem(p.v, o, p.io) * du;
+            }
+        }
+        const float vs = transpose_reduce32<false>(vp, lane);
+        SS.vred[sp][ch * 32 + lane] = vs;
+    }
+    if (!fail) fail = !mbar_wait_bounded(&SS.mbar[3], 0, kWaitNs);
+    fail = __syncthreads_or(fail);
+    tc_fence_after();
+    // dK^ = P4 + beta e^G dR_w + (the P and carry parts), then the normalisation's adjoint
+    float acc[32];
+    if (!fail) {
+        uint32_t rk4[32], ra[32];
+        tmem_ld32(tl + WT_DK + ch * 32, rk4);
+        tmem_ld32(tl + WT_DRW + ch * 32, ra);
+        tmem_wait_ld();
+        const float r0 = SS.rr[0];
+        const uint16_t* kt = reinterpret_cast<const uint16_t*>(sm + W_K);
+        float rp[32], pp[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            const int i = ch * 32 + u;
+            rp[u] = pp[u] = acc[u] = 0.f;
+            if (i < Cc) {
+                const uint16_t kb = kt[((x >> 6) * 8192 + sw128(i, (x >> 3) & 7)) / 2 + (x & 7)];
+                const float kh = __half2float(*reinterpret_cast<const __half*>(&kb)) * SS.rk[i] * SS.invk[i];
+                const float dr = u2f(ra[u]) * r0;
+                const float a = u2f(rk4[u]) * SS.rbs[i] + SS.beta[i] * exp2f(SS.G[i] * kLog2e) * dr +
+                                p.dKp[((size_t)tok(i) * p.Hv + h) * 128 + x];
+                rp[u] = kh * dr;
+                pp[u] = kh * a;
+                acc[u] = a;
+            }
+        }
+        const float rs = transpose_reduce32<false>(rp, lane);
+        SS.rred[sp][ch * 32 + lane] = rs;
+        const float ps = transpose_reduce32<false>(pp, lane);
+        SS.pred[sp][ch * 32 + lane] = ps;
+    }
+    __syncthreads();
+    if (!fail) {
+        const uint16_t* kt = reinterpret_cast<const uint16_t*>(sm + W_K);
+#pragma unroll 4
+        for (int u = 0; u < 32; ++u) {
+            const int i = ch * 32 + u;
+            if (i >= Cc) break;
+            const float proj = SS.pred[0][i] + SS.pred[1][i] + SS.pred[2][i] + SS.pred[3][i];
+            const float n = SS.nk[i];
+            const uint16_t kb = kt[((x >> 6) * 8192 + sw128(i, (x >> 3) & 7)) / 2 + (x & 7)];
+            const float kh = __half2float(*reinterpret_cast<const __half*>(&kb)) * SS.rk[i] * SS.invk[i];
+            const float a = acc[u];
+            p.dkh[((size_t)tok(i) * p.Hv + h) * 128 + x] =
+                on ? (n > kNormEps ? (a - kh * proj) / n : a / kNormEps) : a;
+        }
+    }
+    // ---- dG, dbeta per position and dg = the reverse cumulative sum of dG within the chunk
+    float* dgf = reinterpret_cast<float*>(sm + W_AS);  // beta D is no longer read
+    float* dbf = dgf + 64;
+    if (!fail && tid < 64) {
+        const int t = tid;
+        if (t < Cc) {
+            const float r = SS.rred[0][t] + SS.rred[1][t] + SS.rred[2][t] + SS.rred[3][t];
+            const float eg = exp2f(SS.G[t] * kLog2e);
+            dgf[t] = p.dGp[(size_t)tok(t) * p.Hv + h] + (SS.dgr[0][t] + SS.dgr[1][t]) +
+                     (SS.dgc[0][t] + SS.dgc[1][t]) + SS.beta[t] * eg * r;
+            dbf[t] = (SS.db[0][t] + SS.db[1][t]) + eg * r +
+                     (SS.vred[0][t] + SS.vred[1][t] + SS.vred[2][t] + SS.vred[3][t]);
+        }
+    }
+    __syncthreads();
+    if (!fail && tid == 0) {
+        float run = 0.f;
+        for (int t = Cc - 1; t >= 0; --t) {
+            run += dgf[t];
+            const size_t gi = (size_t)tok(t) * p.Hv + h;
+            store_elem(p.dg_out, gi, run, p.gt);
+            store_elem(p.dbeta_out, gi, dbf[t], p.gt);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+    if (tid == 0) {
+        if (fail) atomicExch(const_cast<int*>(&p.hdr->err), (int)GDR_ERR_TIMEOUT);
+        else if (SS.range_bad) atomicCAS(const_cast<int*>(&p.hdr->err), (int)GDR_OK, (int)GDR_ERR_RANGE);
+    }
+}
+
 }  // namespace
 
 bool bwd_dqk_tc_supported(const gdr_chunk_args& a) {
@@ -563,6 +1048,14 @@ gdr_status launch_bwd_dqk_tc(const BwdParams& p, dim3 grid, cudaStream_t st) {
                              (int)SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
     bwd_chunk_dqk_tc<<<grid, kTh, SMEM_BYTES, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+gdr_status launch_bwd_wy_tc(const BwdParams& p, dim3 grid, cudaStream_t st) {
+    if (cudaFuncSetAttribute(bwd_chunk_wy_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)W_SMEM) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    bwd_chunk_wy_tc<<<grid, kTh, W_SMEM, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 
