@@ -46,7 +46,7 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-CHUNK_TC_SOURCES = ("chunk_tc.cu", "wy_solve.cuh", "tc_ptx.cuh", "common.cuh")
+CHUNK_TC_SOURCES = ("chunk_tc.cu", "chunk_tc.cuh", "wy_solve.cuh", "tc_ptx.cuh", "common.cuh")
 G2_TC_SOURCES = ("chunk_g2_tc.cu", "wy_solve.cuh", "tc_ptx.cuh", "common.cuh")
 DECODE_SOURCES = ("decode.cu", "common.cuh")
 

@@ -6,20 +6,14 @@
 #include <cmath>
 #include <cstring>
 
+#include "chunk_tc.cuh"
 #include "common.cuh"
 
 namespace gdr {
-bool tc_supported(const gdr_chunk_args& a);
 bool tc_g2_supported(const gdr_chunk_args& a);
 gdr_status launch_chunk_g2_tc(const gdr_chunk_args& a, const void* q, const void* k, const void* v,
                               const void* g, const void* b, const float* S0, void* o,
                               float* S_final, void* ws, const WsLayout& L, cudaStream_t st);
-// `dependent`: launched as the programmatic dependent of the stream's previous grid
-gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k, const void* v,
-                           const void* g, const void* beta, const float* S0, void* o,
-                           float* S_final, void* ws, const WsLayout& L, cudaStream_t st,
-                           bool dependent = false, const void* g_rev = nullptr,
-                           const void* beta_rev = nullptr, size_t part_off = 0);
 }  // namespace gdr
 
 using namespace gdr;

@@ -864,6 +864,24 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
     if (!fail) fail = !mbar_wait_bounded(&SS.mbar[2], 0, kWaitNs);
     fail = __syncthreads_or(fail);
     tc_fence_after();
+    // the products have read [dW | dV'] and [W | U~]: their regions take the P and carry parts
+    // of dK^ (fp32 rows of 512 bytes) and v (bf16 rows of 256 bytes), copied in while the
+    // next steps run
+    {
+        const long long tok0 = tok(0);
+#pragma unroll
+        for (int it = 0; it < 12; ++it) {
+            const int idx = tid + it * kTh;
+            const bool isv = idx >= 2048;
+            const int i = isv ? (idx - 2048) >> 4 : idx >> 5, c = isv ? idx & 15 : idx & 31;
+            const bool valid = i < Cc;
+            const size_t row = (size_t)(valid ? tok(i) : tok0) * p.Hv + h;
+            const void* src = isv ? static_cast<const void*>(static_cast<const uint4*>(p.v) + row * 16 + c)
+                                  : static_cast<const void*>(reinterpret_cast<const uint4*>(p.dKp) + row * 32 + c);
+            cp_async16(sbase + (isv ? W_WF + i * 256 : W_R + i * 512) + c * 16, src, valid);
+        }
+        cp_async_commit();
+    }
     // dA -> D, the decay and beta gradients it carries, beta D (rows i: warps 0, 1, 4, 5)
     if (!fail && sp < 2) {
         const int i = sp * 32 + lane;
@@ -931,8 +949,11 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
         mma_commit(&SS.mbar[3]);
     }
     const int x = sp * 32 + lane;  // feature: d of dR_w and dK, e of dR_u and dv
+    cp_async_wait<0>();
+    __syncthreads();
     // dv = beta dR_u and v . dR_u while P4 runs (every warp: lanes = e, columns = i)
     if (!fail) {
+        const __nv_bfloat16* vsm = reinterpret_cast<const __nv_bfloat16*>(sm + W_WF);
         uint32_t rb[32];
         tmem_ld32(tl + WT_DRU + ch * 32, rb);
         tmem_wait_ld();
@@ -946,7 +967,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
                 const float du = u2f(rb[u]) * r1;
                 const size_t o = ((size_t)tok(i) * p.Hv + h) * 128 + x;
                 store_elem(p.dv_out, o, SS.beta[i] * du, p.io);
-                vp[u] = load_elem(p.v, o, p.io) * du;
+                vp[u] = __bfloat162float(vsm[i * 128 + x]) * du;
             }
         }
         const float vs = transpose_reduce32<false>(vp, lane);
@@ -974,7 +995,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
                 const float kh = __half2float(*reinterpret_cast<const __half*>(&kb)) * SS.rk[i] * SS.invk[i];
                 const float dr = u2f(ra[u]) * r0;
                 const float a = u2f(rk4[u]) * SS.rbs[i] + SS.beta[i] * exp2f(SS.G[i] * kLog2e) * dr +
-                                p.dKp[((size_t)tok(i) * p.Hv + h) * 128 + x];
+                                reinterpret_cast<const float*>(sm + W_R)[i * 128 + x];
                 rp[u] = kh * dr;
                 pp[u] = kh * a;
                 acc[u] = a;
@@ -988,10 +1009,10 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
     __syncthreads();
     if (!fail) {
         const uint16_t* kt = reinterpret_cast<const uint16_t*>(sm + W_K);
-#pragma unroll 4
+#pragma unroll
         for (int u = 0; u < 32; ++u) {
             const int i = ch * 32 + u;
-            if (i >= Cc) break;
+            if (i >= Cc) continue;
             const float proj = SS.pred[0][i] + SS.pred[1][i] + SS.pred[2][i] + SS.pred[3][i];
             const float n = SS.nk[i];
             const uint16_t kb = kt[((x >> 6) * 8192 + sw128(i, (x >> 3) & 7)) / 2 + (x & 7)];
@@ -1016,13 +1037,26 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
         }
     }
     __syncthreads();
-    if (!fail && tid == 0) {
-        float run = 0.f;
-        for (int t = Cc - 1; t >= 0; --t) {
-            run += dgf[t];
-            const size_t gi = (size_t)tok(t) * p.Hv + h;
-            store_elem(p.dg_out, gi, run, p.gt);
-            store_elem(p.dbeta_out, gi, dbf[t], p.gt);
+    if (!fail && warp == 0) {
+        // lane l takes positions 2l and 2l + 1: a suffix sum of the pair sums over the lanes
+        const int t0 = 2 * lane, t1 = 2 * lane + 1;
+        const float a = t0 < Cc ? dgf[t0] : 0.f, b = t1 < Cc ? dgf[t1] : 0.f;
+        float incl = a + b;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_down_sync(0xffffffffu, incl, o);
+            if (lane + o < 32) incl += y;
+        }
+        const float after = incl - (a + b);  // positions 2l + 2 on
+        if (t0 < Cc) {
+            const size_t gi = (size_t)tok(t0) * p.Hv + h;
+            store_elem(p.dg_out, gi, after + b + a, p.gt);
+            store_elem(p.dbeta_out, gi, dbf[t0], p.gt);
+        }
+        if (t1 < Cc) {
+            const size_t gi = (size_t)tok(t1) * p.Hv + h;
+            store_elem(p.dg_out, gi, after + b, p.gt);
+            store_elem(p.dbeta_out, gi, dbf[t1], p.gt);
         }
     }
     tc_fence_before();

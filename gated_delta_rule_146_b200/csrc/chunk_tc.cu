@@ -56,6 +56,7 @@
 #include <algorithm>
 #include <cstring>
 
+#include "chunk_tc.cuh"
 #include "common.cuh"
 
 #include "tc_ptx.cuh"
@@ -146,6 +147,10 @@ struct TcParams {
     const void* g_rev; const void* beta_rev;
     const int32_t* chunk_off;
     float* part;
+    // the saving instantiation (kSave) leaves what the backward reads, fp32: W and U~ by
+    // token ([token][head][d]), the in-chunk cumulative log decay G ([token][head]), the state
+    // at every chunk start ([chunk][head][dk][dv]) and V' ([token][head][dv]); no output
+    float *sv_W, *sv_U, *sv_G, *sv_H, *sv_V;
 };
 
 // The fused gating prologue's per-head arrays, a kernel argument of its own that only the
@@ -170,7 +175,9 @@ __device__ __forceinline__ float gate_bits_to_float(uint32_t b, gdr_dtype dt) {
 // kDh: the head size dk = dv in memory, 128 or 64.  A 64-wide head runs in the same 128-wide
 // tiles with feature columns 64-127 zero (never loaded): the normalisation is unchanged and
 // the state's extra rows and columns receive only zero updates, so they stay zero.
-template <bool kRaw, int kDh, bool kPair>
+// kSave: the forward of the backward pass (see TcParams); plain gates, head size 128, single
+// scans only.
+template <bool kRaw, int kDh, bool kPair, bool kSave>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -497,6 +504,10 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     SS.Er[t] = ex2(Gi - Gref);
                     SS.Eq[t] = ex2(Gr - Gref);
                     SS.ck[t] = SS.split_ok[pb] ? ex2(Gref - Gi) * inv : inv;
+                    if constexpr (kSave) {
+                        if (t >= row_lo(c) && t < Cc)
+                            p.sv_G[(size_t)(tokA + tstep * (c * C + t)) * p.Hv + h] = Gi * (1.f / kLog2e);
+                    }
                 }
                 const int i = r2 & 63;
                 float f = inv;
@@ -674,6 +685,11 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     r[e] = __float_as_uint(x0 * gam);
                     r[e + 1] = __float_as_uint(x1 * gam);
                     hb[e >> 1] = h2(x0, x1);
+                    if constexpr (kSave) {
+                        float* hc = p.sv_H + ((size_t)p.chunk_off[s] * p.Hv + h) * (D * D) + j;
+                        hc[(size_t)(d0 + e) * D] = x0;
+                        hc[(size_t)(d0 + e + 1) * D] = x1;
+                    }
                 }
                 tmem_st32(tlane + TM_HM + d0, r);
                 tmem_st16(tlane + TM_HB + d0 / 2, hb);
@@ -717,6 +733,25 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&SS.mbar[MB_D0F]);
+                if constexpr (kSave) {  // W (lane = d) and U~ (lane = e), rows of live tokens
+                    float* wrow = p.sv_W + ((size_t)(tokA + tstep * c * C) * p.Hv + h) * D + lt;
+                    float* urow = p.sv_U + ((size_t)(tokA + tstep * c * C) * p.Hv + h) * D + lt;
+                    const long long rstep = tstep * (long long)p.Hv * D;
+#pragma unroll
+                    for (int i = 0; i < C; ++i)
+                        if (i >= row_lo(c) && i < Cc) wrow[rstep * i] = u2f(rw[i >> 5][i & 31]);
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t ru[32];
+                        tmem_ld32(tlane + TM_DU + pb * 64 + half * 32, ru);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int m = 0; m < 32; ++m) {
+                            const int i = half * 32 + m;
+                            if (i >= row_lo(c) && i < Cc) urow[rstep * i] = u2f(ru[m]);
+                        }
+                    }
+                }
 #pragma unroll
                 for (int half = 0; half < 2; ++half)
 #pragma unroll
@@ -758,6 +793,13 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 tmem_ld32(tlane + TM_DU + pb * 64, rv[0]);
                 tmem_ld32(tlane + TM_DU + pb * 64 + 32, rv[1]);
                 tmem_wait_ld();
+                if constexpr (kSave) {
+                    float* vrow = p.sv_V + ((size_t)(tokA + tstep * c * C) * p.Hv + h) * D + lt;
+                    const long long rstep = tstep * (long long)p.Hv * D;
+#pragma unroll
+                    for (int i = 0; i < C; ++i)
+                        if (i >= row_lo(c) && i < Cc) vrow[rstep * i] = u2f(rv[i >> 5][i & 31]);
+                }
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[16], ps[16];
@@ -833,7 +875,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 const long long ostep = kPair ? 1 : tstep;
                 const int olo = kPair ? 0 : row_lo(c);
                 const int ohi = kPair ? min(C, Lseq - C * u) : Cc;
-                bool emit = true;  // this CTA writes the chunk's output
+                bool emit = !kSave;  // this CTA writes the chunk's output
                 if constexpr (kPair) {
                     if (!second) {
                         if (j < kDh) {
@@ -924,6 +966,11 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
                                 const float2 x = make_float2(u2f(r[2 * e]), u2f(r[2 * e + 1]));
+                                if constexpr (kSave) {
+                                    float* hc = p.sv_H + ((size_t)(p.chunk_off[s] + c + 1) * p.Hv + h) * (D * D) + lt;
+                                    hc[(size_t)(dd + 2 * e) * D] = x.x;
+                                    hc[(size_t)(dd + 2 * e + 1) * D] = x.y;
+                                }
                                 hb[e] = h2(x.x, x.y);
                                 const float2 y = __fmul2_rn(x, make_float2(gam, gam));
                                 r[2 * e] = __float_as_uint(y.x);
@@ -1018,7 +1065,7 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
                            const void* g, const void* beta, const float* S0, void* o,
                            float* S_final, void* ws, const WsLayout& L, cudaStream_t st,
                            bool dependent, const void* g_rev, const void* beta_rev,
-                           size_t part_off) {
+                           size_t part_off, const TcSave* save) {
     const bool pair = g_rev != nullptr;  // bidirectional: both scans, one cluster per pair
     char* base = static_cast<char*>(ws);
     TcParams p;
@@ -1036,6 +1083,11 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
     p.g_rev = g_rev; p.beta_rev = beta_rev;
     p.chunk_off = reinterpret_cast<const int32_t*>(base + L.chunk_off);
     p.part = pair ? reinterpret_cast<float*>(base + part_off) : nullptr;
+    p.sv_W = save ? save->W : nullptr;
+    p.sv_U = save ? save->U : nullptr;
+    p.sv_G = save ? save->G : nullptr;
+    p.sv_H = save ? save->H : nullptr;
+    p.sv_V = save ? save->V : nullptr;
     const GateParams gp{a.gate_A, a.gate_dt_bias, a.beta_scale};
     CUtensorMap tq, tk, tv, to;
     memset(&tq, 0, sizeof(tq));
@@ -1053,12 +1105,13 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
             return GDR_ERR_CUDA;
         p.use_tma = 1;
         // accumulating outputs are read back, so they keep the plain stores
-        p.tma_store = !a.o_accumulate && make_tile_map(&to, o, a.Hv, T_tot, a.dv);
+        p.tma_store = !save && !a.o_accumulate && make_tile_map(&to, o, a.Hv, T_tot, a.dv);
     }
-    auto kernel = pair ? (a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D, true> : chunk_fused_tc<false, D, true>)
-                                    : (a.gate_raw ? chunk_fused_tc<true, 64, true> : chunk_fused_tc<false, 64, true>))
-                       : (a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D, false> : chunk_fused_tc<false, D, false>)
-                                    : (a.gate_raw ? chunk_fused_tc<true, 64, false> : chunk_fused_tc<false, 64, false>));
+    auto kernel = pair ? (a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D, true, false> : chunk_fused_tc<false, D, true, false>)
+                                    : (a.gate_raw ? chunk_fused_tc<true, 64, true, false> : chunk_fused_tc<false, 64, true, false>))
+                       : (a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D, false, false> : chunk_fused_tc<false, D, false, false>)
+                                    : (a.gate_raw ? chunk_fused_tc<true, 64, false, false> : chunk_fused_tc<false, 64, false, false>));
+    if (save) kernel = chunk_fused_tc<false, D, false, true>;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
