@@ -837,38 +837,37 @@ constexpr size_t kMaxSmem = 227 * 1024;
 
 template <int RP, int DR>
 gdr_status launch_states_t(const gdr_chunk_args& a, const BwdParams& p, dim3 grid,
-                           cudaStream_t st, bool with_fwd) {
+                           cudaStream_t st) {
     const size_t sf = states_fwd_smem(a), sb = states_bwd_smem(a);
     if (cudaFuncSetAttribute(bwd_states_fwd<RP, DR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sf) != cudaSuccess ||
         cudaFuncSetAttribute(bwd_states_bwd<RP, DR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sb) != cudaSuccess)
         return GDR_ERR_CUDA;
-    if (with_fwd) bwd_states_fwd<RP, DR><<<grid, kThreads, sf, st>>>(p);
+    bwd_states_fwd<RP, DR><<<grid, kThreads, sf, st>>>(p);
     bwd_states_bwd<RP, DR><<<grid, kThreads, sb, st>>>(p);
     return GDR_OK;
 }
 
 template <int RP>
 gdr_status launch_states_dk(const gdr_chunk_args& a, const BwdParams& p, dim3 grid,
-                            cudaStream_t st, bool with_fwd) {
+                            cudaStream_t st) {
     switch (a.dk) {
-        case 32: return launch_states_t<RP, 4>(a, p, grid, st, with_fwd);
-        case 64: return launch_states_t<RP, 8>(a, p, grid, st, with_fwd);
-        case 96: return launch_states_t<RP, 12>(a, p, grid, st, with_fwd);
-        case 128: return launch_states_t<RP, 16>(a, p, grid, st, with_fwd);
+        case 32: return launch_states_t<RP, 4>(a, p, grid, st);
+        case 64: return launch_states_t<RP, 8>(a, p, grid, st);
+        case 96: return launch_states_t<RP, 12>(a, p, grid, st);
+        case 128: return launch_states_t<RP, 16>(a, p, grid, st);
     }
     return GDR_ERR_UNSUPPORTED;
 }
 
-// State passes for C rows per chunk (C/8 per warp) and dk state rows (dk/8 per warp); the
-// forward pass only when the saving tensor-core forward has not left H and V' already.
+// State passes for C rows per chunk (C/8 per warp) and dk state rows (dk/8 per warp).
 gdr_status launch_states(const gdr_chunk_args& a, const BwdParams& p, dim3 grid,
-                         cudaStream_t st, bool with_fwd) {
+                         cudaStream_t st) {
     switch (a.chunk) {
-        case 16: return launch_states_dk<2>(a, p, grid, st, with_fwd);
-        case 32: return launch_states_dk<4>(a, p, grid, st, with_fwd);
-        case 64: return launch_states_dk<8>(a, p, grid, st, with_fwd);
+        case 16: return launch_states_dk<2>(a, p, grid, st);
+        case 32: return launch_states_dk<4>(a, p, grid, st);
+        case 64: return launch_states_dk<8>(a, p, grid, st);
     }
     return GDR_ERR_UNSUPPORTED;
 }
@@ -944,13 +943,18 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
     const bool tc = bwd_dqk_tc_supported(a) && tc_supported(a);
     gdr_status s;
     if (tc) {
-        const TcSave sv{W, U, G, p.Hc, p.Vp};
+        // the forward, then the reverse state pass (dH+ per chunk, dV', dS0) on the same kernel
+        const TcSave fw{W, U, G, p.Hc, p.Vp, false};
+        const TcSave ad{nullptr, nullptr, nullptr, p.dHc, p.dVp, true};
         s = launch_chunk_tc(a, x.q, x.k, x.v, x.g, x.beta, x.S0, nullptr, nullptr, ws, L, st,
-                            false, nullptr, nullptr, 0, &sv);
+                            false, nullptr, nullptr, 0, &fw);
+        if (s == GDR_OK)
+            s = launch_chunk_tc(a, x.q, x.k, x.dO, x.g, x.beta, x.dS_final, nullptr, x.dS0, ws, L,
+                                st, false, nullptr, nullptr, 0, &ad);
     } else {
         s = launch_wy_local_simt(a, x.k, x.v, x.g, x.beta, ws, L, W, U, G, st);
+        if (s == GDR_OK) s = launch_prep_simt(a, x.q, x.k, ws, L, st);
     }
-    if (s == GDR_OK) s = launch_prep_simt(a, x.q, x.k, ws, L, st);
     if (s != GDR_OK) return s;
     const size_t sm_q = dqk_smem(a), sm_w = wy_smem(a);
     if (cudaFuncSetAttribute(bwd_chunk_dqk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_q) != cudaSuccess ||
@@ -958,7 +962,7 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
         return GDR_ERR_CUDA;
     const dim3 gc((unsigned)L.max_chunks, (unsigned)a.Hv);
     const dim3 gs((unsigned)a.n_seqs, (unsigned)a.Hv, (unsigned)(a.dv / kSlice));
-    if ((s = launch_states(a, p, gs, st, !tc)) != GDR_OK) return s;
+    if (!tc && (s = launch_states(a, p, gs, st)) != GDR_OK) return s;
     if (L.max_chunks > 0) {
         if (tc) {
             if ((s = launch_bwd_dqk_tc(p, gc, st)) != GDR_OK) return s;

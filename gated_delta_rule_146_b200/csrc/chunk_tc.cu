@@ -123,6 +123,7 @@ struct Small {
     float ck[C];             // column factor of [K;Q]K^T: 1/||k_j|| (x 2^(G_ref - G_j) when split)
     float inv[128];          // 1 / ||row|| of [K;Q] (1 without normalisation)
     float gsum_part[2];      // chain: partial sums of the next chunk's g
+    float gam_adj[2];        // adjoint: e^(G_last) of the chunk, by step parity
     uint64_t mbar[MB_COUNT];
     uint32_t tmem_base;
     int gflag[2][2];         // a bounded wait gave up: [chain, preparation][alternate waits]
@@ -177,7 +178,11 @@ __device__ __forceinline__ float gate_bits_to_float(uint32_t b, gdr_dtype dt) {
 // the state's extra rows and columns receive only zero updates, so they stay zero.
 // kSave: the forward of the backward pass (see TcParams); plain gates, head size 128, single
 // scans only.
-template <bool kRaw, int kDh, bool kPair, bool kSave>
+// kAdj: the backward's reverse state pass on the same preparation.  The chunks are visited
+// last to first; the value tiles carry dO, the initial state is dS_final and the final one
+// dS0; the chain keeps dH^T in tensor memory and leaves dH+ at every chunk and dV' (sv_H,
+// sv_V).  Plain gates, head size 128, single scans.
+template <bool kRaw, int kDh, bool kPair, bool kSave, bool kAdj>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -232,6 +237,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     const int L = Lseq + rofs;  // positions of the (row-offset) scan
     const int nchunks = (L + C - 1) / C;
     auto row_lo = [&](int c) -> int { return c == 0 ? rofs : 0; };  // first live row of chunk c
+    // the chunk taken at step `step` (the adjoint pass walks the chunks backwards)
+    auto chunk_of = [&](int step) -> int { return kAdj ? nchunks - 1 - step : step; };
     static_assert(kDh == 64 || kDh == D, "head size");
     const size_t sb = ((size_t)s * p.Hv + h) * kDh * kDh;
     // physical token of logical position 0, and the step between consecutive positions
@@ -321,11 +328,12 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
         const __nv_bfloat16* qbase = p.q + (size_t)hk * kDh + (cd_in ? cd : 0) * 8;
         const __nv_bfloat16* vbase = p.v + (size_t)h * kDh + (cd_in ? cd : 0) * 8;
         const long long kq_tok = (long long)p.Hk * kDh, v_tok = (long long)p.Hv * kDh;
-        auto load_chunk = [&](int c) {
+        auto load_chunk = [&](int step) {  // buffers by step, positions by chunk
+            const int c = chunk_of(step);
             if (use_tma) {  // forward scans: six 8 KB tensor tiles, issued by one thread (pt 128)
-                uint64_t* bar = &SS.mbar[MB_LD + c % 3];
-                const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
-                const uint32_t vv = sbase + OFF_V + (c & 1) * V_STRIDE;
+                uint64_t* bar = &SS.mbar[MB_LD + step % 3];
+                const uint32_t kq = sbase + OFF_KQ + (step % 3) * KQ_STRIDE;
+                const uint32_t vv = sbase + OFF_V + (step & 1) * V_STRIDE;
                 const int z = (int)(t0 + (long long)c * C);
                 mbar_expect_tx(bar, 3 * (kDh / 64) * 8192);
 #pragma unroll
@@ -337,8 +345,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 return;
             }
             const int Cc = min(C, L - c * C);
-            const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_STRIDE + (cd >> 3) * 16384;
-            const uint32_t vv = sbase + OFF_V + (c & 1) * V_STRIDE + (cd >> 3) * 8192;
+            const uint32_t kq = sbase + OFF_KQ + (step % 3) * KQ_STRIDE + (cd >> 3) * 16384;
+            const uint32_t vv = sbase + OFF_V + (step & 1) * V_STRIDE + (cd >> 3) * 8192;
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int i = r0 + 16 * m;
@@ -386,12 +394,12 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             if (lane == 0) SS.split_ok[par] = dev <= 110.f;
         };
         {
-            const int Cc0 = min(C, L);
-            auto live0 = [&](int i) { return i >= rofs && i < Cc0; };
-            if (pt < C) SS.b[0][pt] = live0(pt) ? XB(gate_at(bsrc, pt)) : 0.f;
+            const int p0 = chunk_of(0) * C, Cc0 = min(C, L - p0);
+            auto live0 = [&](int i) { return i >= row_lo(chunk_of(0)) && i < Cc0; };
+            if (pt < C) SS.b[0][pt] = live0(pt) ? XB(gate_at(bsrc, p0 + pt)) : 0.f;
             if (pw == 1)
-                chunk_cumsum(live0(2 * lane) ? XG(gate_at(gsrc, 2 * lane)) : 0.f,
-                             live0(2 * lane + 1) ? XG(gate_at(gsrc, 2 * lane + 1)) : 0.f, 0);
+                chunk_cumsum(live0(2 * lane) ? XG(gate_at(gsrc, p0 + 2 * lane)) : 0.f,
+                             live0(2 * lane + 1) ? XG(gate_at(gsrc, p0 + 2 * lane + 1)) : 0.f, 0);
         }
         // P5, issued as the solve completes T's block columns: K-step kk of W^T = K^T T_w^T
         // (into D0) and of U~^T = V^T T_u^T (into DU) reads block column kk of T_w and T_u
@@ -414,7 +422,8 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             const uint32_t KQ = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
             uint8_t* KQp = sm + OFF_KQ + (c % 3) * KQ_STRIDE;
             const uint32_t VV = sbase + OFF_V + pb * V_STRIDE;
-            const int Cc = min(C, L - c * C);
+            const int cc = chunk_of(c);  // the chunk of this step
+            const int Cc = min(C, L - cc * C);
             const bool has_next = c + 1 < nchunks;
 
             // P0: the buffers of chunk c-2 are released once the chain is done with them (each
@@ -426,14 +435,19 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             if (c >= 2) ok = mbar_wait_bounded(&SS.mbar[MB_CD + pb], ((c >> 1) & 1) ^ 1, kWaitLimitNs);
             int Cn = 0;
             if (has_next) {
+                // the loads of step c + 1 rewrite the value tile of step c - 1: its last reader
+                // (the U~ product, or in the adjoint the chain's first products) must be done
+                if (!use_tma && ok && c >= 1)
+                    ok = mbar_wait_bounded(&SS.mbar[kAdj ? MB_M1 : MB_MU], (uint32_t)((c - 1) & 1), kWaitLimitNs);
                 if (!use_tma && ok) load_chunk(c + 1);  // reversed scans: every thread's row copies
                 // in-bounds positions for every thread, masked only where the values are used
                 // (a select on a just-loaded value would wait for the load right here)
-                Cn = min(C, L - (c + 1) * C);
-                b_nx = gate_bits_at(bsrc, (c + 1) * C + min(pt & 63, Cn - 1));
+                const int pn = chunk_of(c + 1) * C;
+                Cn = min(C, L - pn);
+                b_nx = gate_bits_at(bsrc, pn + min(pt & 63, Cn - 1));
                 if (pw == 1) {
-                    g_nx0 = gate_bits_at(gsrc, (c + 1) * C + min(2 * lane, Cn - 1));
-                    g_nx1 = gate_bits_at(gsrc, (c + 1) * C + min(2 * lane + 1, Cn - 1));
+                    g_nx0 = gate_bits_at(gsrc, pn + min(2 * lane, Cn - 1));
+                    g_nx1 = gate_bits_at(gsrc, pn + min(2 * lane + 1, Cn - 1));
                 }
             }
             if (!use_tma) cp_async_commit();
@@ -499,14 +513,15 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     const float Gref = SS.G[pb][31];
                     const float Gi = SS.G[pb][t];
                     const float Gr = p.read_pre ? (t > 0 ? SS.G[pb][t - 1] : 0.f) : Gi;
-                    SS.Kd[pb][t] = t >= row_lo(c) && t < Cc ? ex2(SS.G[pb][Cc - 1] - Gi) : 0.f;
+                    SS.Kd[pb][t] = t >= row_lo(cc) && t < Cc ? ex2(SS.G[pb][Cc - 1] - Gi) : 0.f;
+                    if (kAdj && t == 0) SS.gam_adj[pb] = ex2(SS.G[pb][Cc - 1]);
                     SS.bg[t] = SS.b[pb][t] * ex2(Gi);
                     SS.Er[t] = ex2(Gi - Gref);
                     SS.Eq[t] = ex2(Gr - Gref);
                     SS.ck[t] = SS.split_ok[pb] ? ex2(Gref - Gi) * inv : inv;
                     if constexpr (kSave) {
-                        if (t >= row_lo(c) && t < Cc)
-                            p.sv_G[(size_t)(tokA + tstep * (c * C + t)) * p.Hv + h] = Gi * (1.f / kLog2e);
+                        if (t >= row_lo(cc) && t < Cc)
+                            p.sv_G[(size_t)(tokA + tstep * (cc * C + t)) * p.Hv + h] = Gi * (1.f / kLog2e);
                     }
                 }
                 const int i = r2 & 63;
@@ -515,7 +530,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                     const float Gr = p.read_pre ? (i > 0 ? SS.G[pb][i - 1] : 0.f) : SS.G[pb][i];
                     f = p.scale * ex2(Gr) * inv;
                 }
-                if (i < row_lo(c) || i >= Cc) f = 0.f;
+                if (i < row_lo(cc) || i >= Cc) f = 0.f;
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
                     const uint32_t w[4] = {vals[c8].x, vals[c8].y, vals[c8].z, vals[c8].w};
@@ -554,11 +569,14 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             {
                 // warp 8 has no store here: it issues the next chunk's tensor loads
                 if (use_tma && has_next && pt == 128) {
-                    load_chunk(c + 1);
-                    ld_pending = c + 1;
+                    // (adjoint: the chain's first products of step c - 1 read the value tile)
+                    if (!kAdj || c == 0 || mbar_wait_bounded(&SS.mbar[MB_M1], (uint32_t)((c - 1) & 1), kWaitLimitNs)) {
+                        load_chunk(c + 1);
+                        ld_pending = c + 1;
+                    }
                 }
                 const int i = r & 63;
-                const bool live = i >= row_lo(c) && i < Cc;
+                const bool live = i >= row_lo(cc) && i < Cc;
                 const bool split = SS.split_ok[pb];
                 float* As = reinterpret_cast<float*>(sm + OFF_AS);
                 uint32_t rr[32];
@@ -635,11 +653,13 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                                  if (phase == 1) {
                                      issue_w(KQ, pb, 3);
                                      issue_w(KQ, pb, 2);
-                                     issue_u(VV, pb, 3);
-                                     issue_u(VV, pb, 2);
+                                     if (!kAdj) {
+                                         issue_u(VV, pb, 3);
+                                         issue_u(VV, pb, 2);
+                                     }
                                  } else {
                                      issue_w(KQ, pb, 1);
-                                     issue_u(VV, pb, 1);
+                                     if (!kAdj) issue_u(VV, pb, 1);
                                  }
                              });
             fence_proxy_async_smem();
@@ -651,7 +671,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             // chain reads W^T out of D0 itself, so the chunk is handed over right away.
             if (pt == 192) {
                 issue_w(KQ, pb, 0);
-                issue_u(VV, pb, 0);
+                if (!kAdj) issue_u(VV, pb, 0);
                 mma_commit(&SS.mbar[MB_MU]);
             }
             if (has_next && pt < C)
@@ -667,6 +687,163 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
     } else {
         // =============================== chain warpgroup ===============================
         const int j = lt;  // dv column = TMEM lane
+
+        if constexpr (kAdj) {
+            // ---------------- adjoint chain: dH^T (lane = dv column e) from dS_final back
+            // to dS0.  Per chunk (last to first), with dH+ the gradient of its final state:
+            //   dV'^T = dO^T P + diag-free (dH+^T K^T) diag(Kd)     (dV' = P^T dO + K~ dH+)
+            //   dH^T  = e^(G_last) dH+^T + dO^T Q~ + dV'^T (-W)
+#pragma unroll 1
+            for (int d0 = 0; d0 < D; d0 += 32) {
+                uint32_t r[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    r[e] = __float_as_uint(p.S0 ? p.S0[sb + (size_t)(d0 + e) * D + j] : 0.f);
+                tmem_st32(tlane + TM_HM + d0, r);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            named_bar(kBarChain, 128);
+            tc_fence_after();
+            for (int c = 0; c < nchunks; ++c) {
+                const int pb = c & 1, cc = chunk_of(c);
+                const uint32_t KQ = sbase + OFF_KQ + (c % 3) * KQ_STRIDE;
+                const uint32_t VV = sbase + OFF_V + pb * V_STRIDE;
+                const int Cc = min(C, L - cc * C);
+                if (!wg_wait(MB_PREP + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
+                if (!wg_wait(MB_MU, c & 1, kBarChain)) { fail = true; break; }
+                // -W^T into WN[pb] (rows d): the B operand of dV'^T (-W), K-major
+                {
+                    uint32_t rw[2][32];
+                    tmem_ld32(tlane + TM_D0, rw[0]);
+                    tmem_ld32(tlane + TM_D0 + 32, rw[1]);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive(&SS.mbar[MB_D0F]);
+#pragma unroll
+                    for (int half = 0; half < 2; ++half)
+#pragma unroll
+                        for (int e8 = 0; e8 < 4; ++e8) {
+                            float f[8];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) f[u] = -u2f(rw[half][e8 * 8 + u]);
+                            *reinterpret_cast<uint4*>(sm + OFF_WN + pb * 16384 + sw128(lt, half * 4 + e8)) =
+                                h8(f);
+                        }
+                }
+                // dH+ -> this chunk's slot of sv_H ([d][e]), an fp16 copy (A operand), and
+                // e^(G_last) dH+ back into the accumulator
+                {
+                    const float gam = SS.gam_adj[pb];
+                    float* hc = p.sv_H + ((size_t)(p.chunk_off[s] + cc) * p.Hv + h) * (D * D) + j;
+#pragma unroll 1
+                    for (int d0 = 0; d0 < D; d0 += 32) {
+                        uint32_t r[32], hb[16];
+                        tmem_ld32(tlane + TM_HM + d0, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const float x0 = u2f(r[2 * e]), x1 = u2f(r[2 * e + 1]);
+                            omax = max_abs_nan(omax, x0);
+                            omax = max_abs_nan(omax, x1);
+                            hc[(size_t)(d0 + 2 * e) * D] = x0;
+                            hc[(size_t)(d0 + 2 * e + 1) * D] = x1;
+                            hb[e] = h2(x0, x1);
+                            r[2 * e] = __float_as_uint(x0 * gam);
+                            r[2 * e + 1] = __float_as_uint(x1 * gam);
+                        }
+                        tmem_st16(tlane + TM_HB + d0 / 2, hb);
+                        tmem_st32(tlane + TM_HM + d0, r);
+                    }
+                    tmem_wait_st();
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar(kBarChain, 128);
+                // dO^T P (DU half 0; A = the fp16 dO tile, MN-major; B = P, MN-major) and
+                // dH+^T K^T (DU half 1; A = the fp16 dH+ copy; B = the K^ rows, K-major)
+                if (lt == 0) {
+                    tc_fence_after();
+                    const uint32_t i1 = idesc_f32acc(128, 64, true, true, false);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f32acc_ss(tmem + TM_DU, sdesc_sw128(VV + kk * 2048, 8192, 1024),
+                                      sdesc_sw128(sbase + OFF_P + pb * 8192 + kk * 2048, 8192, 1024), i1, kk > 0);
+                    const uint32_t i2 = idesc_f32acc(128, 64, false, false, false);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        mma_f32acc_ts(tmem + TM_DU + 64, tmem + TM_HB + kk * 8,
+                                      sdesc_sw128(KQ + off, 16, 1024), i2, kk > 0);
+                    }
+                    // dH^T += dO^T Q~ (B = the Q~ rows, MN-major): the dO tile's last reader, so
+                    // this commit also frees it for the preparation's next loads
+                    const uint32_t i3 = idesc_f32acc(128, 128, true, true, false);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f32acc_ss(tmem + TM_HM, sdesc_sw128(VV + kk * 2048, 8192, 1024),
+                                      sdesc_sw128(KQ + 8192 + kk * 2048, 16384, 1024), i3, 1);
+                    mma_commit(&SS.mbar[MB_M1]);
+                }
+                if (!wg_wait(MB_M1, c & 1, kBarChain)) { fail = true; break; }
+                // dV'^T = dO^T P + (dH+^T K^T) diag(Kd) -> sv_V and the fp16 copy TM_VP
+                {
+                    float* vrow = p.sv_V + ((size_t)(tokA + tstep * cc * C) * p.Hv + h) * D + j;
+                    const long long rstep = tstep * (long long)p.Hv * D;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t r1[32], r2[32], pk[16];
+                        tmem_ld32(tlane + TM_DU + half * 32, r1);
+                        tmem_ld32(tlane + TM_DU + 64 + half * 32, r2);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int i0 = half * 32 + 2 * e;
+                            const float a0 = fmaf(SS.Kd[pb][i0], u2f(r2[2 * e]), u2f(r1[2 * e]));
+                            const float a1 = fmaf(SS.Kd[pb][i0 + 1], u2f(r2[2 * e + 1]), u2f(r1[2 * e + 1]));
+                            omax = max_abs_nan(omax, a0);
+                            omax = max_abs_nan(omax, a1);
+                            if (i0 < Cc) vrow[rstep * i0] = a0;
+                            if (i0 + 1 < Cc) vrow[rstep * (i0 + 1)] = a1;
+                            pk[e] = h2(a0, a1);
+                        }
+                        tmem_st16(tlane + TM_VP + half * 16, pk);
+                    }
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                named_bar(kBarChain, 128);
+                // dH^T += dV'^T (-W) (B = WN[pb], K-major)
+                if (lt == 0) {
+                    tc_fence_after();
+                    const uint32_t i4 = idesc_f32acc(128, 128, false, false, false);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f32acc_ts(tmem + TM_HM, tmem + TM_VP + kk * 8,
+                                      sdesc_sw128(sbase + OFF_WN + pb * 16384 + kk * 32, 16, 1024), i4, 1);
+                    mma_commit(&SS.mbar[MB_M3 + pb]);
+                }
+                if (!wg_wait(MB_M3 + pb, (c >> 1) & 1, kBarChain)) { fail = true; break; }
+                mbar_arrive(&SS.mbar[MB_CD + pb]);  // the step's buffers are free
+                tc_fence_before();
+                named_bar(kBarChain, 128);
+                tc_fence_after();
+            }
+            // dS0: dH^T after the first chunk ([d][e])
+            if (!fail) {
+#pragma unroll 1
+                for (int d0 = 0; d0 < D; d0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tlane + TM_HM + d0, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        omax = max_abs_nan(omax, u2f(r[e]));
+                        if (p.S_final) p.S_final[sb + (size_t)(d0 + e) * D + j] = u2f(r[e]);
+                    }
+                }
+            }
+        } else {
         {
             // initial state -> TM_HM (pre-scaled by chunk 0's total decay), TM_HB (fp16)
             const float gv = lt >= rofs && lt < min(C, L) ? XG(gate_at(gsrc, lt)) : 0.f;
@@ -1005,6 +1182,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
             tc_fence_after();
         }
         if constexpr (kPair) pair_flush();  // the last chunk left for the partner
+        }  // forward chain
     }
 
     if (tid == 0) bulk_wait_all();  // output tiles written before the CTA exits
@@ -1107,11 +1285,12 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
         // accumulating outputs are read back, so they keep the plain stores
         p.tma_store = !save && !a.o_accumulate && make_tile_map(&to, o, a.Hv, T_tot, a.dv);
     }
-    auto kernel = pair ? (a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D, true, false> : chunk_fused_tc<false, D, true, false>)
-                                    : (a.gate_raw ? chunk_fused_tc<true, 64, true, false> : chunk_fused_tc<false, 64, true, false>))
-                       : (a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D, false, false> : chunk_fused_tc<false, D, false, false>)
-                                    : (a.gate_raw ? chunk_fused_tc<true, 64, false, false> : chunk_fused_tc<false, 64, false, false>));
-    if (save) kernel = chunk_fused_tc<false, D, false, true>;
+    auto kernel = pair ? (a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D, true, false, false> : chunk_fused_tc<false, D, true, false, false>)
+                                    : (a.gate_raw ? chunk_fused_tc<true, 64, true, false, false> : chunk_fused_tc<false, 64, true, false, false>))
+                       : (a.dk == D ? (a.gate_raw ? chunk_fused_tc<true, D, false, false, false> : chunk_fused_tc<false, D, false, false, false>)
+                                    : (a.gate_raw ? chunk_fused_tc<true, 64, false, false, false> : chunk_fused_tc<false, 64, false, false, false>));
+    if (save) kernel = save->adjoint ? chunk_fused_tc<false, D, false, false, true>
+                                     : chunk_fused_tc<false, D, false, true, false>;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
