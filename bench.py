@@ -446,7 +446,7 @@ def bench_ours(args, rank, world, local_rank):
             kbytes += 2 * d["S0"].numel() * 4
         backward = {"workload": w.name, "ms_per_step": kms, "steps": bwsteps,
                     "value": whole_job_rate(tokens, world, kms), "unit": "tokens/s",
-                    "path": "simt (fp32 CUDA cores)", "algorithmic_bytes": kbytes,
+                    "path": gdr.chunk_bwd_path(cargs), "algorithmic_bytes": kbytes,
                     "hbm_frac": kbytes / (kms / 1e3) / 1e9 / peaks["hbm_gbs"],
                     "workspace_bytes": bws_.numel()}
         del bws_

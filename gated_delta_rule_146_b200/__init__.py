@@ -8,7 +8,8 @@ fallback: if the compiled library is missing, importing the entry points raises.
 Entry points (names follow the C ABI):
   chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, ...) -> (o, S_final)
   decode_step(q, k, v, g, beta, S, ...) -> o           (S updated in place)
-  chunk_fwd_workspace_size(...), chunk_fwd_path(...), read_device_error(...)
+  chunk_fwd_workspace_size(...), chunk_fwd_path(...), chunk_bwd_path(...),
+  read_device_error(...)
 """
 from __future__ import annotations
 
@@ -21,7 +22,7 @@ from ._abi import GdrError, ChunkArgs, DecodeArgs, F32, BF16, READ_POST, READ_PR
 
 __all__ = ["chunk_fwd", "chunk_fwd_bidir", "chunk_bwd", "decode_step",
            "chunk_fwd_workspace_size", "chunk_fwd_bidir_workspace_size",
-           "chunk_bwd_workspace_size", "chunk_fwd_path",
+           "chunk_bwd_workspace_size", "chunk_fwd_path", "chunk_bwd_path",
            "read_device_error", "chunk_fwd_noalloc", "noalloc_read_device_error", "library",
            "GdrError"]
 
@@ -120,6 +121,12 @@ def chunk_fwd_workspace_size(args: ChunkArgs) -> int:
 
 def chunk_fwd_path(args: ChunkArgs):
     r = _abi.lib().gdr_chunk_fwd_path(ctypes.byref(args))
+    return None if r is None else r.decode()
+
+
+def chunk_bwd_path(args: ChunkArgs):
+    """gdr_chunk_bwd_path: "tc", "simt" or None (unsupported)."""
+    r = _abi.lib().gdr_chunk_bwd_path(ctypes.byref(args))
     return None if r is None else r.decode()
 
 

@@ -19,7 +19,7 @@ EXPORTS = ["gdr_chunk_fwd_workspace_size", "gdr_chunk_fwd", "gdr_chunk_fwd_noall
            "gdr_noalloc_read_device_error",
            "gdr_chunk_bwd_workspace_size", "gdr_chunk_bwd",
            "gdr_chunk_fwd_bidir_workspace_size", "gdr_chunk_fwd_bidir",
-           "gdr_chunk_fwd_path",
+           "gdr_chunk_fwd_path", "gdr_chunk_bwd_path",
            "gdr_decode_step", "gdr_status_string", "gdr_read_device_error", "gdr_version"]
 
 
@@ -78,6 +78,8 @@ def _declare(lib):
     lib.gdr_chunk_bwd.restype = ctypes.c_int
     lib.gdr_chunk_fwd_path.argtypes = [ctypes.POINTER(ChunkArgs)]
     lib.gdr_chunk_fwd_path.restype = ctypes.c_char_p
+    lib.gdr_chunk_bwd_path.argtypes = [ctypes.POINTER(ChunkArgs)]
+    lib.gdr_chunk_bwd_path.restype = ctypes.c_char_p
     lib.gdr_decode_step.argtypes = [ctypes.POINTER(DecodeArgs)] + [vp] * 8
     lib.gdr_decode_step.restype = ctypes.c_int
     lib.gdr_status_string.argtypes = [ctypes.c_int]

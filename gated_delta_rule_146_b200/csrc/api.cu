@@ -10,6 +10,7 @@
 #include "common.cuh"
 
 namespace gdr {
+bool bwd_tc_path(const gdr_chunk_args& a);  // chunk_bwd.cu
 bool tc_g2_supported(const gdr_chunk_args& a);
 gdr_status launch_chunk_g2_tc(const gdr_chunk_args& a, const void* q, const void* k, const void* v,
                               const void* g, const void* b, const float* S0, void* o,
@@ -241,6 +242,11 @@ gdr_status gdr_chunk_fwd_bidir(const gdr_chunk_args* a, const void* q, const voi
 size_t gdr_chunk_bwd_workspace_size(const gdr_chunk_args* a) {
     if (check_chunk_args(a) != GDR_OK || !bwd_supported(*a)) return 0;
     return bwd_layout(*a).total;
+}
+
+const char* gdr_chunk_bwd_path(const gdr_chunk_args* a) {
+    if (check_chunk_args(a) != GDR_OK || !bwd_supported(*a)) return nullptr;
+    return bwd_tc_path(*a) ? "tc" : "simt";
 }
 
 gdr_status gdr_chunk_bwd(const gdr_chunk_args* a, const void* q, const void* k, const void* v,

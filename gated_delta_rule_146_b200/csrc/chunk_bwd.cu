@@ -905,6 +905,10 @@ bool bwd_supported(const gdr_chunk_args& a) {
            states_bwd_smem(a) <= kMaxSmem && dqk_smem(a) <= kMaxSmem && wy_smem(a) <= kMaxSmem;
 }
 
+// bf16, head size 128, chunk 64: the tensor-core kernels (both recurrences on the fused
+// forward kernel, the per-chunk steps in chunk_bwd_tc.cu)
+bool bwd_tc_path(const gdr_chunk_args& a) { return bwd_dqk_tc_supported(a) && tc_supported(a); }
+
 gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
                             const BwdLayout& B, cudaStream_t st) {
     char* base = static_cast<char*>(ws);
@@ -940,7 +944,7 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
 
     // bf16, head size 128, chunk 64: the tensor-core forward leaves W, U~, G, H and V' (its
     // saving instantiation), and the per-chunk steps run on the tensor cores
-    const bool tc = bwd_dqk_tc_supported(a) && tc_supported(a);
+    const bool tc = bwd_tc_path(a);
     gdr_status s;
     if (tc) {
         // the forward, then the reverse state pass (dH+ per chunk, dV', dS0) on the same kernel

@@ -266,6 +266,14 @@ gdr_status gdr_chunk_fwd_bidir(const gdr_chunk_args* args,
  *   workspace   device scratch of at least gdr_chunk_bwd_workspace_size(args) bytes,
  *               256-byte aligned, no initialisation needed
  *
+ * Kernels.  bf16, dk = dv = 128, chunk 64 ("tc"): the tensor-core forward kernel runs twice,
+ * once leaving W, U~, the in-chunk decay, the state at every chunk start and V', once as the
+ * adjoint recurrence from dS_final back to dS0 (dH+ at every chunk, dV'); two per-(chunk,
+ * head) tcgen05 kernels then form dq, dk, dv, dg and dbeta.  Their operands are fp16, each row
+ * (or tile) scaled by a power of two; an fp16 operand of the recurrences that leaves its range
+ * (|dO| or a gradient of the state beyond 65504) is reported as GDR_ERR_RANGE through the
+ * workspace, as in gdr_chunk_fwd.  Other sizes and fp32 ("simt"): fp32 CUDA-core kernels.
+ *
  * Outputs are written, never accumulated.  Errors: as gdr_chunk_fwd; GDR_ERR_UNSUPPORTED
  * for sizes or options outside the kernels' range.
  */
@@ -277,6 +285,10 @@ gdr_status gdr_chunk_bwd(const gdr_chunk_args* args,
                          const void* dO, const float* dS_final,
                          void* dq, void* dk, void* dv, void* dg, void* dbeta, float* dS0,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Name of the kernel path gdr_chunk_bwd takes for these arguments: "tc" (tcgen05
+ * tensor-core kernels), "simt" (fp32 CUDA-core kernels) or NULL if unsupported. */
+const char* gdr_chunk_bwd_path(const gdr_chunk_args* args);
 
 /*
  * One-token recurrent decode step (flashrt fused_layer.py `_decode_one`, the

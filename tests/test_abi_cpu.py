@@ -291,3 +291,15 @@ def test_noalloc_and_status_word_host_validation(lib):
     assert call(lib, a, wsb=need) == _abi.GDR_ERR_ALIGNMENT
     assert lib.gdr_chunk_fwd_bidir(ctypes.byref(a), *[vp(FAKE)] * 7, None, vp(FAKE), vp(FAKE),
                                    ctypes.c_size_t(1 << 30), None) == _abi.GDR_ERR_ALIGNMENT
+
+
+def test_backward_path(lib):
+    """gdr_chunk_bwd_path: the tensor-core kernels for bf16, d = 128, chunk 64; the CUDA-core
+    ones for fp32 inputs and for other sizes; none where the backward is not built."""
+    path = lambda **kw: lib.gdr_chunk_bwd_path(ctypes.byref(args(**kw)))
+    assert path(dk=128, dv=128) == b"tc"
+    assert path(dk=128, dv=128, io_dtype=_abi.F32, gate_dtype=_abi.F32) == b"simt"
+    assert path(dk=64, dv=64) == b"simt"
+    assert path(dk=128, dv=128, chunk=32) == b"simt"
+    assert path(dk=128, dv=128, gate_raw=1) is None
+    assert path(dk=128, dv=128, o_accumulate=1) is None

@@ -47,6 +47,10 @@ def upstream(x, dtype, seed, with_dS=True):
 def run_and_check(x, dO, dS, dtype, *, read_mode="post", scale=0.1, reverse=False, chunk=64,
                   qk_l2norm=True):
     dev = {n: to_dev(t) if t is not None else None for n, t in x.items()}
+    a = gdr.make_chunk_args(dev["q"], dev["v"], dev["g"], dev["cu_seqlens"], chunk, read_mode,
+                            scale, qk_l2norm, reverse)
+    tc = dtype == "bf16" and x["q"].shape[3] == 128 and x["v"].shape[3] == 128 and chunk == 64
+    assert gdr.chunk_bwd_path(a) == ("tc" if tc else "simt")
     got = gdr.chunk_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], to_dev(dO),
                         dev["S0"], dev["cu_seqlens"], to_dev(dS), chunk=chunk,
                         read_mode=read_mode, scale=scale, reverse=reverse, qk_l2norm=qk_l2norm)
@@ -109,6 +113,8 @@ def test_training_shape_workload_whole():
     gen = torch.Generator("cpu").manual_seed(71)
     dO = torch.randn(x["v"].shape, generator=gen).to(torch.bfloat16)
     dev = {n: to_dev(t) if t is not None else None for n, t in x.items()}
+    a = gdr.make_chunk_args(dev["q"], dev["v"], dev["g"], None, w.chunk, w.read_mode, w.scale)
+    assert gdr.chunk_bwd_path(a) == "tc"  # the tensor-core kernels
     got = gdr.chunk_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], to_dev(dO),
                         dev["S0"], None, None, chunk=w.chunk, read_mode=w.read_mode,
                         scale=w.scale)
