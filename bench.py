@@ -48,6 +48,12 @@ def load_peaks():
 
 CHUNK_TC_SOURCES = ("chunk_tc.cu", "chunk_tc.cuh", "wy_solve.cuh", "tc_ptx.cuh", "common.cuh")
 G2_TC_SOURCES = ("chunk_g2_tc.cu", "wy_solve.cuh", "tc_ptx.cuh", "common.cuh")
+BWD_TC_SOURCES = ("chunk_bwd_tc.cu", "chunk_bwd.cuh", "wy_solve.cuh", "tc_ptx.cuh", "common.cuh")
+BWD_SOURCES = ("chunk_bwd.cu", "chunk_bwd.cuh", "common.cuh")
+# the kernels of one tensor-core backward call, with the sources of their traffic records
+BWD_TC_KERNELS = (("chunk_fused_tc_save", CHUNK_TC_SOURCES), ("chunk_fused_tc_adj", CHUNK_TC_SOURCES),
+                  ("bwd_chunk_dqk_tc", BWD_TC_SOURCES), ("bwd_chunk_wy_tc", BWD_TC_SOURCES),
+                  ("bwd_reduce_heads", BWD_SOURCES))
 DECODE_SOURCES = ("decode.cu", "common.cuh")
 
 
@@ -414,7 +420,7 @@ def bench_ours(args, rank, world, local_rank):
     # ---------------- backward pass (gdr_chunk_bwd) on the same workload and inputs, with a
     # seeded upstream gradient dO; gradients of q, k, v, g, beta and S0
     backward = None
-    if args.backward and args.only != "decode" and not args.rows:
+    if args.backward and args.only != "decode":
         gen = torch.Generator("cpu").manual_seed(1000 + rank)
         dOb = torch.randn(tuple(d["v"].shape), generator=gen).to(d["v"].dtype).to(dev)
         bargs_ = gdr.make_chunk_args(d["q"], d["v"], d["g"], d["cu_seqlens"], w.chunk,
@@ -449,6 +455,10 @@ def bench_ours(args, rank, world, local_rank):
                     "path": gdr.chunk_bwd_path(cargs), "algorithmic_bytes": kbytes,
                     "hbm_frac": kbytes / (kms / 1e3) / 1e9 / peaks["hbm_gbs"],
                     "workspace_bytes": bws_.numel()}
+        if backward["path"] == "tc":
+            # measured traffic of the call's kernels, the intermediate arrays included
+            tp = [measured_traffic(k, src, w.B) for k, src in BWD_TC_KERNELS]
+            backward["traffic"] = None if None in tp else sum(tp)
         del bws_
 
     # ---------------- GDN-2 (decoupled per-channel gates): the chunk workload on the CUDA-core
