@@ -966,7 +966,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
             if (i < Cc) {
                 const float du = u2f(rb[u]) * r1;
                 const size_t o = ((size_t)tok(i) * p.Hv + h) * 128 + x;
-                store_elem(p.dv_out, o, SS.beta[i] * du, p.io);
+                static_cast<__nv_bfloat16*>(p.dv_out)[o] = __float2bfloat16_rn(SS.beta[i] * du);
                 vp[u] = __bfloat162float(vsm[i * 128 + x]) * du;
             }
         }
