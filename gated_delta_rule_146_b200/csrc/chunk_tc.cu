@@ -1140,13 +1140,22 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                             uint32_t (&r)[32] = r2[hh];
                             const int dd = d0 + hh * 32;
                             uint32_t hb[16];
+                            // the saving forward's state leaves through the free staging slab WN[pb]
+                            // by bulk stores (off the chain's path); the slab is rewritten once
+                            // the previous slab's store has read it
+                            if constexpr (kSave) {
+                                if (dd > 0) {
+                                    if (lt == 0) bulk_wait_read();
+                                    named_bar(kBarChain, 128);
+                                }
+                            }
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
                                 const float2 x = make_float2(u2f(r[2 * e]), u2f(r[2 * e + 1]));
                                 if constexpr (kSave) {
-                                    float* hc = p.sv_H + ((size_t)(p.chunk_off[s] + c + 1) * p.Hv + h) * (D * D) + lt;
-                                    hc[(size_t)(dd + 2 * e) * D] = x.x;
-                                    hc[(size_t)(dd + 2 * e + 1) * D] = x.y;
+                                    float* stg = reinterpret_cast<float*>(sm + OFF_WN + pb * 16384);
+                                    stg[(2 * e) * D + lt] = x.x;
+                                    stg[(2 * e + 1) * D + lt] = x.y;
                                 }
                                 hb[e] = h2(x.x, x.y);
                                 const float2 y = __fmul2_rn(x, make_float2(gam, gam));
@@ -1155,6 +1164,15 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                             }
                             tmem_st16(tlane + TM_HB + dd / 2, hb);
                             tmem_st32(tlane + TM_HM + dd, r);
+                            if constexpr (kSave) {  // rows dd .. dd + 31 of the state, 16 KB contiguous
+                                fence_proxy_async_smem();
+                                named_bar(kBarChain, 128);
+                                if (lt == 0) {
+                                    float* hc = p.sv_H + ((size_t)(p.chunk_off[s] + c + 1) * p.Hv + h) * (D * D) + (size_t)dd * D;
+                                    bulk_store(hc, sbase + OFF_WN + pb * 16384, 16384u);
+                                    bulk_commit();
+                                }
+                            }
                         }
                     }
                 } else {

@@ -136,3 +136,62 @@ def test_training_shape_workload_whole():
             acc["dS0"].add(got[5][b:b + 1], ref["dS0"].astype(np.float64), label=f" row {b}")
     for a in acc.values():
         a.check()
+
+
+@pytest.mark.parametrize("read_mode", ["post", "pre"])
+@pytest.mark.parametrize("reverse", [False, True])
+def test_tensor_core_varlen_reverse(reverse, read_mode):
+    """The tensor-core backward (bf16, d = 128, chunk 64) over packed sequences with an empty
+    one, a one-token one and ragged tails, GQA 2 -> 4, S0 and dS_final, both directions and
+    both read modes."""
+    lengths = [1, 0, 64, 65, 130, 200]
+    x = workloads.chunk_inputs(1, 0, 2, 4, 128, 128, "bf16", lengths=lengths, s0_std=0.1, seed=81)
+    dO, dS = upstream(x, "bf16", 82)
+    run_and_check(x, dO, dS, "bf16", read_mode=read_mode, scale=1 / math.sqrt(128),
+                  reverse=reverse)
+
+
+def test_tensor_core_no_norm_no_state():
+    """The tensor-core backward without the in-kernel normalisation, S0 = None and
+    dS_final = None."""
+    x = workloads.chunk_inputs(2, 150, 2, 2, 128, 128, "bf16", seed=83)
+    x["q"] = (x["q"].float() * 0.08).to(torch.bfloat16)
+    x["k"] = (x["k"].float() * 0.08).to(torch.bfloat16)
+    dO, _ = upstream(x, "bf16", 84, with_dS=False)
+    run_and_check(x, dO, None, "bf16", scale=1.0, qk_l2norm=False)
+
+
+def test_tensor_core_deterministic():
+    """Two tensor-core backward calls on the same inputs agree bit for bit (every sum has a
+    fixed order; no atomics)."""
+    x = workloads.chunk_inputs(2, 300, 2, 4, 128, 128, "bf16", s0_std=0.05, seed=85)
+    dO, dS = upstream(x, "bf16", 86)
+    dev = {n: to_dev(t) if t is not None else None for n, t in x.items()}
+    outs = []
+    for _ in range(2):
+        got = gdr.chunk_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], to_dev(dO),
+                            dev["S0"], None, to_dev(dS), scale=0.1)
+        torch.cuda.synchronize()
+        outs.append([t.detach().cpu() for t in got])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_tensor_core_range_reported():
+    """An upstream gradient beyond the fp16 range of the recurrences' operands is reported as
+    GDR_ERR_RANGE through the workspace (the outputs are then not valid)."""
+    x = workloads.chunk_inputs(1, 130, 2, 2, 128, 128, "bf16", seed=87)
+    dO, _ = upstream(x, "bf16", 88, with_dS=False)
+    dO = (dO.float() * 1e6).to(torch.bfloat16)
+    dev = {n: to_dev(t) if t is not None else None for n, t in x.items()}
+    a = gdr.make_chunk_args(dev["q"], dev["v"], dev["g"], None, 64, "post", 0.1, True, False)
+    assert gdr.chunk_bwd_path(a) == "tc"
+    ws = torch.empty(gdr.chunk_bwd_workspace_size(a), dtype=torch.uint8, device="cuda")
+    gdr.chunk_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], to_dev(dO), None, None,
+                  None, scale=0.1, workspace=ws)
+    assert gdr.read_device_error(a, ws) == gdr._abi.GDR_ERR_RANGE
+    # the same call at a normal scale is clean
+    gdr.chunk_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"],
+                  to_dev((dO.float() * 1e-6).to(torch.bfloat16)), None, None, None, scale=0.1,
+                  workspace=ws)
+    assert gdr.read_device_error(a, ws) == 0
