@@ -53,7 +53,7 @@ BWD_SOURCES = ("chunk_bwd.cu", "chunk_bwd.cuh", "common.cuh")
 # the kernels of one tensor-core backward call, with the sources of their traffic records
 BWD_TC_KERNELS = (("chunk_fused_tc_save", CHUNK_TC_SOURCES), ("chunk_fused_tc_adj", CHUNK_TC_SOURCES),
                   ("bwd_chunk_dqk_tc", BWD_TC_SOURCES), ("bwd_chunk_wy_tc", BWD_TC_SOURCES),
-                  ("bwd_reduce_heads", BWD_SOURCES))
+                  ("bwd_reduce_heads4", BWD_SOURCES))
 DECODE_SOURCES = ("decode.cu", "common.cuh")
 
 

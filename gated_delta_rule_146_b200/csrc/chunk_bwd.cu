@@ -31,7 +31,7 @@
 //   bwd_chunk_dqk          per (chunk, head): dq (normalised adjoint), the P and carry parts
 //                          of dK^ and dG, dW
 //   bwd_chunk_wy           per (chunk, head): the transposed solve, dA, dbeta, dv, dg, dk
-//   bwd_reduce_heads       dq, dk summed over each key head's v-heads
+//   bwd_reduce_heads4      dq, dk summed over each key head's v-heads
 #include <algorithm>
 
 #include "chunk_bwd.cuh"
@@ -791,21 +791,35 @@ bwd_chunk_wy(BwdParams p) {
     }
 }
 
-// dq, dk per key head: the sum over the v-heads that read it.
-__global__ void bwd_reduce_heads(BwdParams p, long long n) {
-    const int group = p.Hv / p.Hk;
-    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+// dq, dk per key head: the sum over the v-heads that read it.  Four consecutive features per
+// thread (dk is a multiple of 32): 16-byte loads of the fp32 per-v-head parts, one 8- or
+// 16-byte store of the io-dtype result.
+__global__ void bwd_reduce_heads4(BwdParams p, long long n4) {
+    const int group = p.Hv / p.Hk, dk4 = p.dk / 4;
+    const float4* qh = reinterpret_cast<const float4*>(p.dqh);
+    const float4* kh = reinterpret_cast<const float4*>(p.dkh);
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n4;
          idx += (long long)gridDim.x * blockDim.x) {
-        const long long d = idx % p.dk, r = idx / p.dk;  // r = t * Hk + hk
+        const long long d4 = idx % dk4, r = idx / dk4;  // r = t * Hk + hk
         const long long t = r / p.Hk, hk = r % p.Hk;
-        float sq = 0.f, sk = 0.f;
+        float4 sq = make_float4(0.f, 0.f, 0.f, 0.f), sk = sq;
+        const size_t src = ((size_t)t * p.Hv + hk * group) * dk4 + d4;
         for (int j = 0; j < group; ++j) {
-            const size_t src = ((size_t)t * p.Hv + hk * group + j) * p.dk + d;
-            sq += p.dqh[src];
-            sk += p.dkh[src];
+            const float4 a = __ldcs(qh + src + (size_t)j * dk4), b = __ldcs(kh + src + (size_t)j * dk4);
+            sq.x += a.x; sq.y += a.y; sq.z += a.z; sq.w += a.w;
+            sk.x += b.x; sk.y += b.y; sk.z += b.z; sk.w += b.w;
         }
-        store_elem(p.dq_out, (size_t)idx, sq, p.io);
-        store_elem(p.dk_out, (size_t)idx, sk, p.io);
+        if (p.io == GDR_BF16) {
+            const __nv_bfloat162 q0 = __floats2bfloat162_rn(sq.x, sq.y), q1 = __floats2bfloat162_rn(sq.z, sq.w);
+            const __nv_bfloat162 k0 = __floats2bfloat162_rn(sk.x, sk.y), k1 = __floats2bfloat162_rn(sk.z, sk.w);
+            reinterpret_cast<uint2*>(p.dq_out)[idx] =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&q0), *reinterpret_cast<const uint32_t*>(&q1));
+            reinterpret_cast<uint2*>(p.dk_out)[idx] =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&k0), *reinterpret_cast<const uint32_t*>(&k1));
+        } else {
+            reinterpret_cast<float4*>(p.dq_out)[idx] = sq;
+            reinterpret_cast<float4*>(p.dk_out)[idx] = sk;
+        }
     }
 }
 
@@ -975,9 +989,9 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
             bwd_chunk_dqk<<<gc, kNT, sm_q, st>>>(p);
             bwd_chunk_wy<<<gc, kNT, sm_w, st>>>(p);
         }
-        const long long n = (long long)a.B * a.T * a.Hk * a.dk;
-        const unsigned blocks = (unsigned)std::min<long long>((n + kThreads - 1) / kThreads, 148LL * 16);
-        if (n > 0) bwd_reduce_heads<<<blocks, kThreads, 0, st>>>(p, n);
+        const long long n4 = (long long)a.B * a.T * a.Hk * (a.dk / 4);
+        const unsigned blocks = (unsigned)std::min<long long>((n4 + kThreads - 1) / kThreads, 148LL * 16);
+        if (n4 > 0) bwd_reduce_heads4<<<blocks, kThreads, 0, st>>>(p, n4);
     }
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
