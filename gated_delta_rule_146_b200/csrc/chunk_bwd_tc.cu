@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
             const bool m = li && j < Cc && (pre ? j < i : j <= i);
             const float ik = SS.invk[j], rkj = SS.rk[j];
             const float dp = u2f(rp[u]) * rdoi * SS.rv[j];
-            const float d1 = m ? p.scale * dp * exp2f((gri - SS.G[j]) * kLog2e) : 0.f;
+            const float d1 = m ? p.scale * dp * ex2((gri - SS.G[j]) * kLog2e) : 0.f;
             const float ev = d1 * (u2f(rs[u]) * rqi * rkj * iq * ik);
             rsum += ev;
             e[u] = -ev;
@@ -427,7 +427,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
     if (!fail && sp < 2) {
         const int i = sp * 32 + lane;
         const bool li = i < Cc;
-        const float rd = li ? p.scale * exp2f(SS.Gr[i] * kLog2e) : 0.f;
+        const float rd = li ? p.scale * ex2(SS.Gr[i] * kLog2e) : 0.f;
         const float rdoi = SS.rdo[i], rqi = SS.rq[i], rd1i = SS.rd1[i];
         const uint8_t* qrow = sm + OFF_QK + ch * G16;
         float gs = 0.f, pq = 0.f;
@@ -460,7 +460,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
     // ---- rows 64-127: the P and carry parts of dK^, the carry's decay gradient
     if (!fail && sp >= 2) {
         const bool lj = j < Cc;
-        const float kd = lj ? exp2f((SS.G[Cc - 1] - SS.G[j]) * kLog2e) : 0.f;
+        const float kd = lj ? ex2((SS.G[Cc - 1] - SS.G[j]) * kLog2e) : 0.f;
         const float rvj = SS.rv[j], rkj = SS.rk[j], rd1tj = SS.rd1t[j];
         const uint8_t* krow = sm + OFF_QK + ch * G16 + 8192;
         float* dst = p.dKp + ((size_t)(lj ? tok(j) : 0) * p.Hv + h) * 128 + ch * 64;
@@ -524,7 +524,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
     if (!fail && tid < 64) {
         const int t = tid;
         const bool lt = t < Cc;
-        const float kd = lt ? exp2f((SS.G[Cc - 1] - SS.G[t]) * kLog2e) : 0.f;
+        const float kd = lt ? ex2((SS.G[Cc - 1] - SS.G[t]) * kLog2e) : 0.f;
         const float c = lt ? kd * SS.invk[t] * (SS.ck[0][t] + SS.ck[1][t]) : 0.f;
         SS.c[t] = c;
         const float cs = warp_sum(c);
@@ -534,7 +534,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
     if (!fail && tid < 64 && tid < Cc) {
         const int t = tid;
         auto dgr = [&](int i) {
-            const float rd = p.scale * exp2f(SS.Gr[i] * kLog2e);
+            const float rd = p.scale * ex2(SS.Gr[i] * kLog2e);
             return SS.dGr[0][i] + SS.dGr[1][i] + rd * SS.invq[i] * (SS.gsum[0][i] + SS.gsum[1][i]);
         };
         float g = SS.dGs[0][t] + SS.dGs[1][t] - SS.c[t];
@@ -542,7 +542,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
             float hd = 0.f;
 #pragma unroll
             for (int w = 0; w < 8; ++w) hd += SS.hdot[w];
-            g += (SS.csum[0] + SS.csum[1]) + exp2f(SS.G[Cc - 1] * kLog2e) * hd;
+            g += (SS.csum[0] + SS.csum[1]) + ex2(SS.G[Cc - 1] * kLog2e) * hd;
         }
         if (!pre) g += dgr(t);
         else if (t + 1 < Cc) g += dgr(t + 1);
@@ -775,7 +775,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
             for (int u = 0; u < 32; ++u) {
                 const int j = ch * 32 + u;
                 const bool m = i < Cc && j < i;
-                vals[u] = m ? f * u2f(rs[u]) * SS.rk[j] * SS.invk[j] * exp2f((gi - SS.G[j]) * kLog2e) : 0.f;
+                vals[u] = m ? f * u2f(rs[u]) * SS.rk[j] * SS.invk[j] * ex2((gi - SS.G[j]) * kLog2e) : 0.f;
             }
             // the solve's layout: warp 1 holds only blocks below the diagonal, warps 0 and 5 the
             // diagonal blocks (and A_10, A_32), warp 4 none that it reads
@@ -897,7 +897,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
             const bool m = i < Cc && j < i;
             const float dA = -u2f(rd[u]) * rdr * SS.rw[j];
             const float sk = u2f(rs[u]) * fk * SS.rk[j] * SS.invk[j];
-            const float e = exp2f((gi - SS.G[j]) * kLog2e);
+            const float e = ex2((gi - SS.G[j]) * kLog2e);
             const float D = m ? dA * e : 0.f;
             db = fmaf(D, sk, db);
             const float ga = m ? dA * (bi * sk * e) : 0.f;
@@ -994,7 +994,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
                 const uint16_t kb = kt[((x >> 6) * 8192 + sw128(i, (x >> 3) & 7)) / 2 + (x & 7)];
                 const float kh = __half2float(*reinterpret_cast<const __half*>(&kb)) * SS.rk[i] * SS.invk[i];
                 const float dr = u2f(ra[u]) * r0;
-                const float a = u2f(rk4[u]) * SS.rbs[i] + SS.beta[i] * exp2f(SS.G[i] * kLog2e) * dr +
+                const float a = u2f(rk4[u]) * SS.rbs[i] + SS.beta[i] * ex2(SS.G[i] * kLog2e) * dr +
                                 reinterpret_cast<const float*>(sm + W_R)[i * 128 + x];
                 rp[u] = kh * dr;
                 pp[u] = kh * a;
@@ -1017,9 +1017,9 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
             const float n = SS.nk[i];
             const uint16_t kb = kt[((x >> 6) * 8192 + sw128(i, (x >> 3) & 7)) / 2 + (x & 7)];
             const float kh = __half2float(*reinterpret_cast<const __half*>(&kb)) * SS.rk[i] * SS.invk[i];
-            const float a = acc[u];
+            const float a = acc[u], rn = SS.invk[i];  // 1 / max(|k|, eps) when normalising
             p.dkh[((size_t)tok(i) * p.Hv + h) * 128 + x] =
-                on ? (n > kNormEps ? (a - kh * proj) / n : a / kNormEps) : a;
+                on ? (n > kNormEps ? (a - kh * proj) * rn : a * rn) : a;
         }
     }
     // ---- dG, dbeta per position and dg = the reverse cumulative sum of dG within the chunk
@@ -1029,7 +1029,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
         const int t = tid;
         if (t < Cc) {
             const float r = SS.rred[0][t] + SS.rred[1][t] + SS.rred[2][t] + SS.rred[3][t];
-            const float eg = exp2f(SS.G[t] * kLog2e);
+            const float eg = ex2(SS.G[t] * kLog2e);
             dgf[t] = p.dGp[(size_t)tok(t) * p.Hv + h] + (SS.dgr[0][t] + SS.dgr[1][t]) +
                      (SS.dgc[0][t] + SS.dgc[1][t]) + SS.beta[t] * eg * r;
             dbf[t] = (SS.db[0][t] + SS.db[1][t]) + eg * r +
