@@ -90,6 +90,13 @@ def measured_traffic(kernel: str, sources, units: float):
     return (rec["dram_read_bytes"] + rec["write_bytes_into_l2"]) * units / captured
 
 
+def device_status(a, ws) -> str:
+    """The device-side status a call left in its workspace (read after the timed region; it
+    synchronises): "ok", or the status name (e.g. an fp16 operand out of range)."""
+    st = gdr.read_device_error(a, ws)
+    return "ok" if st == 0 else gdr._abi.status_string(st)
+
+
 def flops_per_head_token(C, dk, dv):
     """Dense chunk-form FLOPs per token per head: KK^T, QK^T, W (2C dk each), U and the
     intra output (2C dv each), W H, the state update and Q H (2 dk dv each)."""
@@ -222,6 +229,7 @@ def bench_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world)
+    statuses = {"chunk": device_status(cargs, ws)}
 
     tokens = int(d["q"].shape[0] * d["q"].shape[1])
     head_tokens = tokens * w.Hv
@@ -257,6 +265,7 @@ def bench_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         gms = max_over_ranks(g0.elapsed_time(g1) / args.steps, world)
+        statuses["gating_prologue"] = device_status(cargs, ws)
         gating = {"ms_per_step": gms, "value": whole_job_rate(tokens, world, gms),
                   "unit": "tokens/s", "overhead_vs_given_gates": gms / ms - 1.0,
                   "inputs": "raw a ~ N(-2,1), b ~ N(0,1) with A = -1, dt_bias = 0 "
@@ -292,6 +301,7 @@ def bench_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         bms = max_over_ranks(b0.elapsed_time(b1) / args.steps, world)
+        statuses["bidirectional"] = device_status(bargs, bws)
         btok = int(bd["q"].shape[1])
         # the least HBM traffic of the call: q, k, v and both directions' gates read once,
         # o written once (the fp32 hand-off between the two scans of a pair is not counted)
@@ -338,6 +348,7 @@ def bench_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         vms = max_over_ranks(v0.elapsed_time(v1) / vsteps, world)
+        statuses["varlen"] = device_status(vargs, vws)
         vtok = int(vd["q"].shape[1])
         vbytes = sum(t.numel() * t.element_size() for t in
                      (vd["q"], vd["k"], vd["v"], vd["g"], vd["beta"], vo, vd["S0"], vS))
@@ -445,6 +456,7 @@ def bench_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         kms = max_over_ranks(k0.elapsed_time(k1) / bwsteps, world)
+        statuses["backward"] = device_status(bargs_, bws_)
         # read q, k, v, g, beta, dO (and S0); write dq, dk, dv, dg, dbeta (and dS0)
         kbytes = 2 * sum(d[n].numel() * d[n].element_size() for n in ("q", "k", "v", "g", "beta"))
         kbytes += dOb.numel() * dOb.element_size()
@@ -492,6 +504,7 @@ def bench_ours(args, rank, world, local_rank):
             torch.cuda.synchronize()
             barrier()
             cms = max_over_ranks(c0.elapsed_time(c1) / g2steps, world)
+            statuses["gdn2.chunk"] = device_status(g2args, g2ws)
             # the least HBM traffic of the call: q, k, v and the three gate tensors read once,
             # o and S_final written once (the tensor-core path's per-chunk records, written
             # and read back through the workspace, are not counted)
@@ -633,6 +646,8 @@ def bench_ours(args, rank, world, local_rank):
                      "peak_source": f"{peak_src} (hbm_gbs copy; bf16_tflops burst)"},
         "decode": dec, "varlen": varlen, "gating_prologue": gating, "bidirectional": bidir,
         "gdn2": gdn2, "backward": backward, "e2e": e2e,
+        # every timed call's device-side status word (workspace), read after the timing
+        "device_status": statuses,
         "clocks": clocks,
         "gpu_launches": launches_per_call * args.steps,
     }
