@@ -93,6 +93,7 @@ def measured_traffic(kernel: str, sources, units: float):
 def device_status(a, ws) -> str:
     """The device-side status a call left in its workspace (read after the timed region; it
     synchronises): "ok", or the status name (e.g. an fp16 operand out of range)."""
+    import gated_delta_rule_146_b200 as gdr
     st = gdr.read_device_error(a, ws)
     return "ok" if st == 0 else gdr._abi.status_string(st)
 
