@@ -888,7 +888,11 @@ gdr_status launch_states(const gdr_chunk_args& a, const BwdParams& p, dim3 grid,
 
 }  // namespace
 
-// Backward workspace: the forward's plan and CUDA-core arrays, then the backward's own.
+bool bwd_tc_path(const gdr_chunk_args& a);
+
+// Backward workspace: the forward's plan and CUDA-core arrays, then the backward's own.  The
+// tensor-core path reads none of the CUDA-core scan's operands (Q~, K~, P, the layout's last
+// three arrays), so its own arrays start where those would.
 BwdLayout bwd_layout(const gdr_chunk_args& a) {
     BwdLayout B{};
     B.base = ws_layout(a, true);
@@ -896,7 +900,7 @@ BwdLayout bwd_layout(const gdr_chunk_args& a) {
     const size_t tk = sizeof(float) * (size_t)T_tot * a.Hv * a.dk;
     const size_t tv = sizeof(float) * (size_t)T_tot * a.Hv * a.dv;
     const size_t st = sizeof(float) * (size_t)B.base.max_chunks * a.Hv * a.dk * a.dv;
-    size_t off = B.base.total;
+    size_t off = bwd_tc_path(a) && B.base.Qt > 0 ? B.base.Qt : B.base.total;
     B.Hc = off;  off = align_up(off + st, 256);
     B.dHc = off; off = align_up(off + st, 256);
     B.Vp = off;  off = align_up(off + tv, 256);
