@@ -587,6 +587,11 @@ constexpr uint32_t W_RS = 163840;   // the solve's diagonal blocks
 constexpr uint32_t W_BS = 167936;   // (beta D + (beta D)^T) diag(1/|k|) rows i (K = j): 8 KB
 constexpr uint32_t W_SMALL = 176128;
 constexpr uint32_t WT_SK = 0, WT_DRW = 64, WT_DRU = 128, WT_DA = 192, WT_DK = 0;
+// the tail's fp32 rows [64][128], over regions no product reads by then: dR_u over the
+// upper half of [W | U~] (v takes the lower) and T, dR_w over dR, the P4 part over A and
+// the solve's T
+constexpr uint32_t W_DRU_S = W_WF + 16384, W_DRW_S = W_DR, W_DK_S = W_AS;
+static_assert(W_DRU_S + 32768 <= W_DR && W_DK_S + 32768 <= W_RS, "tail rows");
 
 struct WySmall {
     float G[64], beta[64], ones[64], invk[64], nk[64];
@@ -595,7 +600,8 @@ struct WySmall {
     float mx[8][3];                   // per-warp largest magnitudes (dW, dV'; dR)
     float bsmax[2][64];               // largest |Bs'| of row i, by column half
     float dgr[2][64], dgc[2][64], db[2][64];  // from dA: row sums, column sums, beta parts
-    float rred[4][64], pred[4][64], vred[4][64];  // k^ . dR_w, k^ . acc, v . dR_u by lane quarter
+    float rsum[64], vsum[64];         // k^ . dR_w, v . dR_u per position
+    float dgf[64], dbf[64];           // dG and dbeta per position
     uint64_t mbar[4];
     uint32_t tmem;
     int range_bad;
@@ -948,99 +954,122 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
                           kdesc(sbase + W_BS + kk * 32), id, kk > 0);
         mma_commit(&SS.mbar[3]);
     }
-    const int x = sp * 32 + lane;  // feature: d of dR_w and dK, e of dR_u and dv
-    cp_async_wait<0>();
-    __syncthreads();
-    // dv = beta dR_u and v . dR_u while P4 runs (every warp: lanes = e, columns = i)
+    // dR_w and dR_u (lane = feature, column = position) into shared memory as fp32 rows i
+    // while P4 runs; the row passes below read them back one row per warp
+    float* drw_s = reinterpret_cast<float*>(sm + W_DRW_S);
+    float* dru_s = reinterpret_cast<float*>(sm + W_DRU_S);
+    float* dk_s = reinterpret_cast<float*>(sm + W_DK_S);
     if (!fail) {
-        const __nv_bfloat16* vsm = reinterpret_cast<const __nv_bfloat16*>(sm + W_WF);
-        uint32_t rb[32];
+        const int x = sp * 32 + lane;  // feature: d of dR_w, e of dR_u
+        uint32_t ra[32], rb[32];
+        tmem_ld32(tl + WT_DRW + ch * 32, ra);
         tmem_ld32(tl + WT_DRU + ch * 32, rb);
         tmem_wait_ld();
-        const float r1 = SS.rr[1];
-        float vp[32];
+        const float r0 = SS.rr[0], r1 = SS.rr[1];
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-            const int i = ch * 32 + u;
-            vp[u] = 0.f;
-            if (i < Cc) {
-                const float du = u2f(rb[u]) * r1;
-                const size_t o = ((size_t)tok(i) * p.Hv + h) * 128 + x;
-                static_cast<__nv_bfloat16*>(p.dv_out)[o] = __float2bfloat16_rn(SS.beta[i] * du);
-                vp[u] = __bfloat162float(vsm[i * 128 + x]) * du;
-            }
+            drw_s[(ch * 32 + u) * 128 + x] = u2f(ra[u]) * r0;
+            dru_s[(ch * 32 + u) * 128 + x] = u2f(rb[u]) * r1;
         }
-        const float vs = transpose_reduce32<false>(vp, lane);
-        SS.vred[sp][ch * 32 + lane] = vs;
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    // Row passes: warp w takes positions 8w .. 8w + 7, lane l the features 4l .. 4l + 3.
+    // k^ of those features: four fp16 values of the staged k tile, times the row's factors.
+    const uint16_t* kt = reinterpret_cast<const uint16_t*>(sm + W_K);
+    auto khat4 = [&](int i, float (&kh)[4]) {
+        const int x0 = 4 * lane;
+        const uint2 raw = *reinterpret_cast<const uint2*>(
+            kt + ((x0 >> 6) * 8192 + sw128(i, (x0 >> 3) & 7)) / 2 + (x0 & 7));
+        const float f = SS.rk[i] * SS.invk[i];
+        const __half2 h01 = *reinterpret_cast<const __half2*>(&raw.x);
+        const __half2 h23 = *reinterpret_cast<const __half2*>(&raw.y);
+        kh[0] = __low2float(h01) * f; kh[1] = __high2float(h01) * f;
+        kh[2] = __low2float(h23) * f; kh[3] = __high2float(h23) * f;
+    };
+    // dv = beta dR_u; v . dR_u and k^ . dR_w per position
+    if (!fail) {
+        const __nv_bfloat16* vsm = reinterpret_cast<const __nv_bfloat16*>(sm + W_WF);
+#pragma unroll 2
+        for (int r = 0; r < 8; ++r) {
+            const int i = warp * 8 + r;
+            if (i >= Cc) break;
+            const float4 du = reinterpret_cast<const float4*>(dru_s + i * 128)[lane];
+            const float4 dr = reinterpret_cast<const float4*>(drw_s + i * 128)[lane];
+            const uint2 vr = *reinterpret_cast<const uint2*>(vsm + i * 128 + 4 * lane);
+            const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vr.x));
+            const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vr.y));
+            float kh[4];
+            khat4(i, kh);
+            const float bi = SS.beta[i];
+            const __nv_bfloat162 o01 = __floats2bfloat162_rn(bi * du.x, bi * du.y);
+            const __nv_bfloat162 o23 = __floats2bfloat162_rn(bi * du.z, bi * du.w);
+            uint2 ov;
+            ov.x = *reinterpret_cast<const uint32_t*>(&o01);
+            ov.y = *reinterpret_cast<const uint32_t*>(&o23);
+            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.dv_out) +
+                                      ((size_t)tok(i) * p.Hv + h) * 128 + 4 * lane) = ov;
+            float vs = v01.x * du.x + v01.y * du.y + v23.x * du.z + v23.y * du.w;
+            float rs = kh[0] * dr.x + kh[1] * dr.y + kh[2] * dr.z + kh[3] * dr.w;
+            vs = warp_sum(vs);
+            rs = warp_sum(rs);
+            if (lane == 0) { SS.vsum[i] = vs; SS.rsum[i] = rs; }
+        }
     }
     if (!fail) fail = !mbar_wait_bounded(&SS.mbar[3], 0, kWaitNs);
     fail = __syncthreads_or(fail);
     tc_fence_after();
-    // dK^ = P4 + beta e^G dR_w + (the P and carry parts), then the normalisation's adjoint
-    float acc[32];
+    // the P4 part of dK^ (lane = d, column = i) as fp32 rows i, times the rows' factors of Bs'
     if (!fail) {
-        uint32_t rk4[32], ra[32];
+        const int x = sp * 32 + lane;
+        uint32_t rk4[32];
         tmem_ld32(tl + WT_DK + ch * 32, rk4);
-        tmem_ld32(tl + WT_DRW + ch * 32, ra);
         tmem_wait_ld();
-        const float r0 = SS.rr[0];
-        const uint16_t* kt = reinterpret_cast<const uint16_t*>(sm + W_K);
-        float rp[32], pp[32];
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-            const int i = ch * 32 + u;
-            rp[u] = pp[u] = acc[u] = 0.f;
-            if (i < Cc) {
-                const uint16_t kb = kt[((x >> 6) * 8192 + sw128(i, (x >> 3) & 7)) / 2 + (x & 7)];
-                const float kh = __half2float(*reinterpret_cast<const __half*>(&kb)) * SS.rk[i] * SS.invk[i];
-                const float dr = u2f(ra[u]) * r0;
-                const float a = u2f(rk4[u]) * SS.rbs[i] + SS.beta[i] * ex2(SS.G[i] * kLog2e) * dr +
-                                reinterpret_cast<const float*>(sm + W_R)[i * 128 + x];
-                rp[u] = kh * dr;
-                pp[u] = kh * a;
-                acc[u] = a;
-            }
-        }
-        const float rs = transpose_reduce32<false>(rp, lane);
-        SS.rred[sp][ch * 32 + lane] = rs;
-        const float ps = transpose_reduce32<false>(pp, lane);
-        SS.pred[sp][ch * 32 + lane] = ps;
+        for (int u = 0; u < 32; ++u) dk_s[(ch * 32 + u) * 128 + x] = u2f(rk4[u]) * SS.rbs[ch * 32 + u];
     }
     __syncthreads();
+    // dK^ = P4 + beta e^G dR_w + (the P and carry parts), then the normalisation's adjoint
+    // dk = (dK^ - k^ (k^ . dK^)) / |k| (plain 1 / max(|k|, eps) below eps, dK^ without it)
     if (!fail) {
-        const uint16_t* kt = reinterpret_cast<const uint16_t*>(sm + W_K);
+        const float* dkp = reinterpret_cast<const float*>(sm + W_R);
+#pragma unroll 2
+        for (int r = 0; r < 8; ++r) {
+            const int i = warp * 8 + r;
+            if (i >= Cc) break;
+            const float4 k4 = reinterpret_cast<const float4*>(dk_s + i * 128)[lane];
+            const float4 dr = reinterpret_cast<const float4*>(drw_s + i * 128)[lane];
+            const float4 cp4 = reinterpret_cast<const float4*>(dkp + i * 128)[lane];
+            const float be = SS.beta[i] * ex2(SS.G[i] * kLog2e);
+            float a[4] = {k4.x + be * dr.x + cp4.x, k4.y + be * dr.y + cp4.y,
+                          k4.z + be * dr.z + cp4.z, k4.w + be * dr.w + cp4.w};
+            float kh[4];
+            khat4(i, kh);
+            const float proj = warp_sum(kh[0] * a[0] + kh[1] * a[1] + kh[2] * a[2] + kh[3] * a[3]);
+            const float n = SS.nk[i], rn = SS.invk[i];  // 1 / max(|k|, eps) when normalising
+            float o[4];
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-            const int i = ch * 32 + u;
-            if (i >= Cc) continue;
-            const float proj = SS.pred[0][i] + SS.pred[1][i] + SS.pred[2][i] + SS.pred[3][i];
-            const float n = SS.nk[i];
-            const uint16_t kb = kt[((x >> 6) * 8192 + sw128(i, (x >> 3) & 7)) / 2 + (x & 7)];
-            const float kh = __half2float(*reinterpret_cast<const __half*>(&kb)) * SS.rk[i] * SS.invk[i];
-            const float a = acc[u], rn = SS.invk[i];  // 1 / max(|k|, eps) when normalising
-            p.dkh[((size_t)tok(i) * p.Hv + h) * 128 + x] =
-                on ? (n > kNormEps ? (a - kh * proj) * rn : a * rn) : a;
+            for (int e = 0; e < 4; ++e) o[e] = on ? (n > kNormEps ? (a[e] - kh[e] * proj) * rn : a[e] * rn) : a[e];
+            reinterpret_cast<float4*>(p.dkh + ((size_t)tok(i) * p.Hv + h) * 128)[lane] =
+                make_float4(o[0], o[1], o[2], o[3]);
         }
     }
     // ---- dG, dbeta per position and dg = the reverse cumulative sum of dG within the chunk
-    float* dgf = reinterpret_cast<float*>(sm + W_AS);  // beta D is no longer read
-    float* dbf = dgf + 64;
     if (!fail && tid < 64) {
         const int t = tid;
         if (t < Cc) {
-            const float r = SS.rred[0][t] + SS.rred[1][t] + SS.rred[2][t] + SS.rred[3][t];
+            const float r = SS.rsum[t];
             const float eg = ex2(SS.G[t] * kLog2e);
-            dgf[t] = p.dGp[(size_t)tok(t) * p.Hv + h] + (SS.dgr[0][t] + SS.dgr[1][t]) +
-                     (SS.dgc[0][t] + SS.dgc[1][t]) + SS.beta[t] * eg * r;
-            dbf[t] = (SS.db[0][t] + SS.db[1][t]) + eg * r +
-                     (SS.vred[0][t] + SS.vred[1][t] + SS.vred[2][t] + SS.vred[3][t]);
+            SS.dgf[t] = p.dGp[(size_t)tok(t) * p.Hv + h] + (SS.dgr[0][t] + SS.dgr[1][t]) +
+                        (SS.dgc[0][t] + SS.dgc[1][t]) + SS.beta[t] * eg * r;
+            SS.dbf[t] = (SS.db[0][t] + SS.db[1][t]) + eg * r + SS.vsum[t];
         }
     }
     __syncthreads();
     if (!fail && warp == 0) {
         // lane l takes positions 2l and 2l + 1: a suffix sum of the pair sums over the lanes
         const int t0 = 2 * lane, t1 = 2 * lane + 1;
-        const float a = t0 < Cc ? dgf[t0] : 0.f, b = t1 < Cc ? dgf[t1] : 0.f;
+        const float a = t0 < Cc ? SS.dgf[t0] : 0.f, b = t1 < Cc ? SS.dgf[t1] : 0.f;
         float incl = a + b;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -1051,12 +1080,12 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
         if (t0 < Cc) {
             const size_t gi = (size_t)tok(t0) * p.Hv + h;
             store_elem(p.dg_out, gi, after + b + a, p.gt);
-            store_elem(p.dbeta_out, gi, dbf[t0], p.gt);
+            store_elem(p.dbeta_out, gi, SS.dbf[t0], p.gt);
         }
         if (t1 < Cc) {
             const size_t gi = (size_t)tok(t1) * p.Hv + h;
             store_elem(p.dg_out, gi, after + b, p.gt);
-            store_elem(p.dbeta_out, gi, dbf[t1], p.gt);
+            store_elem(p.dbeta_out, gi, SS.dbf[t1], p.gt);
         }
     }
     tc_fence_before();
