@@ -910,7 +910,21 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&SS.mbar[MB_D0F]);
-                if constexpr (kSave) {  // W (lane = d) and U~ (lane = e), rows of live tokens
+#pragma unroll
+                for (int half = 0; half < 2; ++half)
+#pragma unroll
+                    for (int e8 = 0; e8 < 4; ++e8) {
+                        float f[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) f[u] = -u2f(rw[half][e8 * 8 + u]);
+                        *reinterpret_cast<uint4*>(sm + OFF_WN + pb * 16384 + sw128(lt, half * 4 + e8)) =
+                            h8(f);
+                    }
+                // a proxy fence waits for this thread's global stores in flight: the saving
+                // forward's stores of W (lane = d) and U~ (lane = e) come after it, and U~ is
+                // read out before the group barrier that lets V' accumulate over it
+                fence_proxy_async_smem();
+                if constexpr (kSave) {
                     float* wrow = p.sv_W + ((size_t)(tokA + tstep * c * C) * p.Hv + h) * D + lt;
                     float* urow = p.sv_U + ((size_t)(tokA + tstep * c * C) * p.Hv + h) * D + lt;
                     const long long rstep = tstep * (long long)p.Hv * D;
@@ -928,19 +942,9 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                             if (i >= row_lo(c) && i < Cc) urow[rstep * i] = u2f(ru[m]);
                         }
                     }
+                    tc_fence_before();
                 }
-#pragma unroll
-                for (int half = 0; half < 2; ++half)
-#pragma unroll
-                    for (int e8 = 0; e8 < 4; ++e8) {
-                        float f[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) f[u] = -u2f(rw[half][e8 * 8 + u]);
-                        *reinterpret_cast<uint4*>(sm + OFF_WN + pb * 16384 + sw128(lt, half * 4 + e8)) =
-                            h8(f);
-                    }
             }
-            fence_proxy_async_smem();
             named_bar(kBarChain, 128);
             // C1: V'^T = U~^T + H^T (-W^T);  O^T = H^T Q~^T   (A = state copy in TMEM)
             if (lt == 0) {
@@ -970,13 +974,6 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                 tmem_ld32(tlane + TM_DU + pb * 64, rv[0]);
                 tmem_ld32(tlane + TM_DU + pb * 64 + 32, rv[1]);
                 tmem_wait_ld();
-                if constexpr (kSave) {
-                    float* vrow = p.sv_V + ((size_t)(tokA + tstep * c * C) * p.Hv + h) * D + lt;
-                    const long long rstep = tstep * (long long)p.Hv * D;
-#pragma unroll
-                    for (int i = 0; i < C; ++i)
-                        if (i >= row_lo(c) && i < Cc) vrow[rstep * i] = u2f(rv[i >> 5][i & 31]);
-                }
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[16], ps[16];
@@ -1190,6 +1187,24 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                                 p.S_final[sb + (size_t)(d0 + e) * kDh + j] = u2f(r[e]);
                         }
                     }
+                }
+                if constexpr (kSave) {
+                    // V' (lane = e), after the state slabs' proxy fences: V'^T stays in DU[pb]
+                    // until the release below lets the preparation's U~ product reuse it
+                    float* vrow = p.sv_V + ((size_t)(tokA + tstep * c * C) * p.Hv + h) * D + lt;
+                    const long long rstep = tstep * (long long)p.Hv * D;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t rv[32];
+                        tmem_ld32(tlane + TM_DU + pb * 64 + half * 32, rv);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int m = 0; m < 32; ++m) {
+                            const int i = half * 32 + m;
+                            if (i >= row_lo(c) && i < Cc) vrow[rstep * i] = u2f(rv[m]);
+                        }
+                    }
+                    tc_fence_before();
                 }
                 tmem_wait_st();
                 if (lt == 0) bulk_wait_read();  // the staging buffer is free for reuse
