@@ -57,6 +57,7 @@ constexpr uint32_t OFF_SMALL = 163840;
 constexpr uint32_t TM_X = 0, TM_Z = 128, TM_P = 256, TM_S = 320, TM_DQ = 256, TM_DK = 384;
 
 struct DqkSmall {
+    float4 jf[64];      // per column j: |k_j|^-1 rk_j, rv_j, G_j
     float G[64], Gr[64], invq[64], invk[64], nq[64];
     // reciprocal row factors: 1 / (power of two) of each stored fp16 row
     float rq[64], rk[64], rdo[64], rv[64], rdv[64], rh[128], rdh[128], rd1[64], rd1t[64];
@@ -303,7 +304,10 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
     fence_proxy_async_smem();
     __syncthreads();
     tc_fence_after();
-    if (tid < 64) SS.Gr[tid] = pre ? (tid > 0 ? SS.G[tid - 1] : 0.f) : SS.G[tid];
+    if (tid < 64) {
+        SS.Gr[tid] = pre ? (tid > 0 ? SS.G[tid - 1] : 0.f) : SS.G[tid];
+        SS.jf[tid] = make_float4(SS.invk[tid] * SS.rk[tid], SS.rv[tid], SS.G[tid], 0.f);
+    }
     const uint32_t tmem = SS.tmem;
     const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);  // this warp's TMEM lanes
 
@@ -333,21 +337,20 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
         tmem_ld32(tl + TM_P + ch * 32, rp);
         tmem_ld32(tl + TM_S + ch * 32, rs);
         tmem_wait_ld();
-        const bool li = i < Cc;
-        const float gri = SS.Gr[i], iq = SS.invq[i], rqi = SS.rq[i], rdoi = SS.rdo[i];
+        // columns inside the mask: j < Cc and j <= i (j < i for the pre-write read)
+        const int jend = i < Cc ? min(Cc, pre ? i : i + 1) : 0;
+        const float gri = SS.Gr[i], qi = SS.invq[i] * SS.rq[i], ci = p.scale * SS.rdo[i];
         float e[32], bm[32], rsum = 0.f, am = 0.f;
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
             const int j = ch * 32 + u;
-            const bool m = li && j < Cc && (pre ? j < i : j <= i);
-            const float ik = SS.invk[j], rkj = SS.rk[j];
-            const float dp = u2f(rp[u]) * rdoi * SS.rv[j];
-            const float d1 = m ? p.scale * dp * ex2((gri - SS.G[j]) * kLog2e) : 0.f;
-            const float ev = d1 * (u2f(rs[u]) * rqi * rkj * iq * ik);
+            const float4 f = SS.jf[j];
+            const float d1 = j < jend ? ci * u2f(rp[u]) * f.y * ex2((gri - f.z) * kLog2e) : 0.f;
+            a1[u] = d1 * f.x;
+            b1[u] = d1 * qi;
+            const float ev = a1[u] * (u2f(rs[u]) * qi);
             rsum += ev;
             e[u] = -ev;
-            a1[u] = d1 * ik * rkj;
-            b1[u] = d1 * iq * rqi;
             am = fmaxf(am, fabsf(a1[u]));
             bm[u] = fabsf(b1[u]);
         }
@@ -358,7 +361,8 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
         const float cmax = transpose_reduce32<true>(bm, lane);
         SS.bmax[sp][ch * 32 + lane] = cmax;
         named_bar(kBarEpi, 128);
-        // D1k row i and D1q^T rows j in fp16, each with its row's factor
+        // D1k row i and D1q^T rows j in fp16, each with its row's factor (lane u holds row
+        // j = 32 ch + u's)
         const float sd = pow2_scale(fmaxf(SS.amax[0][i], SS.amax[1][i]));
 #pragma unroll
         for (int e8 = 0; e8 < 4; ++e8) {
@@ -367,19 +371,16 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
             for (int u = 0; u < 8; ++u) f[u] = a1[e8 * 8 + u];
             *reinterpret_cast<uint4*>(sm + OFF_D + sw128(i, ch * 4 + e8)) = f16x8(f, sd);
         }
+        const float stl = pow2_scale(fmaxf(SS.bmax[0][ch * 32 + lane], SS.bmax[1][ch * 32 + lane]));
         uint16_t* d1t = reinterpret_cast<uint16_t*>(sm + OFF_D);
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
             const int j = ch * 32 + u;
-            const float st = pow2_scale(fmaxf(SS.bmax[0][j], SS.bmax[1][j]));
-            const __half hv = __float2half_rn(b1[u] * st);
+            const __half hv = __float2half_rn(b1[u] * __shfl_sync(0xffffffffu, stl, u));
             d1t[(sw128(64 + j, i >> 3) >> 1) + (i & 7)] = *reinterpret_cast<const uint16_t*>(&hv);
         }
         if (ch == 0) SS.rd1[i] = __frcp_rn(sd);
-        if (sp == 0) {
-            const int j = ch * 32 + lane;
-            SS.rd1t[j] = __frcp_rn(pow2_scale(fmaxf(SS.bmax[0][j], SS.bmax[1][j])));
-        }
+        if (sp == 0) SS.rd1t[ch * 32 + lane] = __frcp_rn(stl);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -594,6 +595,7 @@ constexpr uint32_t W_DRU_S = W_WF + 16384, W_DRW_S = W_DR, W_DK_S = W_AS;
 static_assert(W_DRU_S + 32768 <= W_DR && W_DK_S + 32768 <= W_RS, "tail rows");
 
 struct WySmall {
+    float4 jf[64];                    // per column j: |k_j|^-1 rk_j, rw_j, G_j
     float G[64], beta[64], ones[64], invk[64], nk[64];
     float rk[64], rw[64], rbs[64];    // reciprocal row factors: k, [W | U~], beta D + ...
     float rr[2], rdr;                 // reciprocal tile factors: dW, dV' halves; dR
@@ -753,6 +755,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
     tc_fence_after();
     const uint32_t tmem = SS.tmem;
     const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
+    if (tid < 64) SS.jf[tid] = make_float4(SS.invk[tid] * SS.rk[tid], SS.rw[tid], SS.G[tid], 0.f);
 
     // ---- P1: k . k
     if (tid == 0) {
@@ -776,12 +779,13 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
             tmem_ld32(tl + WT_SK + ch * 32, rs);
             tmem_wait_ld();
             const float f = SS.beta[i] * SS.rk[i] * SS.invk[i], gi = SS.G[i];
+            const int jend = i < Cc ? i : 0;  // strictly lower: j < i
             float vals[32];
 #pragma unroll
             for (int u = 0; u < 32; ++u) {
                 const int j = ch * 32 + u;
-                const bool m = i < Cc && j < i;
-                vals[u] = m ? f * u2f(rs[u]) * SS.rk[j] * SS.invk[j] * ex2((gi - SS.G[j]) * kLog2e) : 0.f;
+                const float4 fj = SS.jf[j];
+                vals[u] = j < jend ? f * u2f(rs[u]) * fj.x * ex2((gi - fj.z) * kLog2e) : 0.f;
             }
             // the solve's layout: warp 1 holds only blocks below the diagonal, warps 0 and 5 the
             // diagonal blocks (and A_10, A_32), warp 4 none that it reads
@@ -895,18 +899,18 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
         tmem_ld32(tl + WT_DA + ch * 32, rd);
         tmem_ld32(tl + WT_SK + ch * 32, rs);
         tmem_wait_ld();
-        const float bi = SS.beta[i], gi = SS.G[i], fk = SS.rk[i] * SS.invk[i], rdr = SS.rdr;
+        const float bi = SS.beta[i], gi = SS.G[i], fk = SS.rk[i] * SS.invk[i], rdr = -SS.rdr;
+        const int jend = i < Cc ? i : 0;  // strictly lower: j < i
         float col[32], bd[32], db = 0.f, dg = 0.f;
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
             const int j = ch * 32 + u;
-            const bool m = i < Cc && j < i;
-            const float dA = -u2f(rd[u]) * rdr * SS.rw[j];
-            const float sk = u2f(rs[u]) * fk * SS.rk[j] * SS.invk[j];
-            const float e = ex2((gi - SS.G[j]) * kLog2e);
-            const float D = m ? dA * e : 0.f;
+            const float4 fj = SS.jf[j];
+            const float dA = u2f(rd[u]) * rdr * fj.y;
+            const float sk = u2f(rs[u]) * fk * fj.x;
+            const float D = j < jend ? dA * ex2((gi - fj.z) * kLog2e) : 0.f;
             db = fmaf(D, sk, db);
-            const float ga = m ? dA * (bi * sk * e) : 0.f;
+            const float ga = bi * sk * D;
             dg += ga;
             col[u] = -ga;
             bd[u] = bi * D;
@@ -925,7 +929,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
             const int j = ch * 32 + u;
-            bd[u] = (bd[u] + *f32sw(As, j, i)) * SS.invk[j] * SS.rk[j];
+            bd[u] = (bd[u] + *f32sw(As, j, i)) * SS.jf[j].x;
             bm = fmaxf(bm, fabsf(bd[u]));
         }
         SS.bsmax[ch][i] = bm;
