@@ -50,7 +50,10 @@ constexpr uint32_t OFF_H = 49152;        // H as B (rows d, K = e), two groups o
 constexpr uint32_t OFF_DH = 81920;       // dH+ as B, same
 constexpr uint32_t OFF_QK = 114688;      // per group: q rows 0-63 | k rows (K = d)
 constexpr uint32_t G16 = 16384;          // group stride of the H, dH+ and q/k regions
-constexpr uint32_t OFF_D = 147456;       // D1k rows 0-63 (K = j) | D1q^T rows 64-127 (K = i)
+constexpr uint32_t OFF_D = 147456;
+// fp32 row tiles of the stores, over the first products' operands (E, H, dH+)
+constexpr uint32_t OFF_TW = 0, OFF_TK = 32768, OFF_TQ = 65536;
+static_assert(OFF_TQ + 32768 <= OFF_QK, "row tiles");       // D1k rows 0-63 (K = j) | D1q^T rows 64-127 (K = i)
 constexpr uint32_t OFF_SMALL = 163840;
 
 // tensor memory columns (fp32 accumulators, lane = row of the stacked product)
@@ -66,7 +69,6 @@ struct DqkSmall {
     float dGr[2][64];   // row sums of E, by column half
     float dGs[2][64];   // column sums of -E, by row warp
     float gsum[2][64];  // sum_d q_d X_d, by d half
-    float projq[2][64]; // sum_d q_d acc_d, by d half
     float ck[2][64];    // sum_d k_d Z_d, by d half
     float c[64];        // the carry's decay gradient per position
     float hdot[8];      // <dH+, H> by warp
@@ -398,40 +400,43 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
         }
         mma_commit(&SS.mbar[1]);
     }
+    // dW, the P and carry parts of dK^ and dQ^ leave as fp32 rows [64][128] staged over the
+    // operands the first products read (dO, dV', V', H, dH+); a row's 16-byte piece pc sits
+    // at pc ^ (row & 7), so that 32 rows' same piece and one row's 32 pieces both spread over
+    // the banks.  One warp per row stores them below.
+    auto tile_at = [&](uint32_t off, int row, int pc) {
+        return reinterpret_cast<float4*>(sm + off + row * 512 + ((pc ^ (row & 7)) << 4));
+    };
     // rows 64-127 (warps 2, 3, 6, 7): dW = -(dV' H^T) while the second products run.  The
     // TMEM loads are warp-wide instructions: every lane issues them, live row or not.
     const int j = (sp - 2) * 32 + lane;  // the row's position, for sp >= 2
     if (!fail && sp >= 2) {
-        const float rdvj = SS.rdv[j & 63];
-        float* dst = p.dW + ((size_t)(j < Cc ? tok(j) : 0) * p.Hv + h) * 128 + ch * 64;
+        const float rdvj = -SS.rdv[j & 63];
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
             uint32_t r[32];
             tmem_ld32(tl + TM_X + ch * 64 + s * 32, r);
             tmem_wait_ld();
-            if (j < Cc) {
-                const float* rh = SS.rh + ch * 64 + s * 32;
+            const float* rh = SS.rh + ch * 64 + s * 32;
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4)
-                    reinterpret_cast<float4*>(dst + s * 32)[e4] = make_float4(
-                        -u2f(r[4 * e4]) * rdvj * rh[4 * e4], -u2f(r[4 * e4 + 1]) * rdvj * rh[4 * e4 + 1],
-                        -u2f(r[4 * e4 + 2]) * rdvj * rh[4 * e4 + 2], -u2f(r[4 * e4 + 3]) * rdvj * rh[4 * e4 + 3]);
-            }
+            for (int e4 = 0; e4 < 8; ++e4)
+                *tile_at(OFF_TW, j, ch * 16 + s * 8 + e4) = make_float4(
+                    u2f(r[4 * e4]) * rdvj * rh[4 * e4], u2f(r[4 * e4 + 1]) * rdvj * rh[4 * e4 + 1],
+                    u2f(r[4 * e4 + 2]) * rdvj * rh[4 * e4 + 2], u2f(r[4 * e4 + 3]) * rdvj * rh[4 * e4 + 3]);
         }
     }
     if (!fail) fail = !mbar_wait_bounded(&SS.mbar[1], 0, kWaitNs);
     fail = __syncthreads_or(fail);
     tc_fence_after();
 
-    // ---- rows 0-63: dQ^ = D1 K^ + s e^{G'} X, its inter-read decay gradient, then dq
-    float acc[64];
+    // ---- rows 0-63: dQ^ = D1 K^ + s e^{G'} X and its inter-read decay gradient
     if (!fail && sp < 2) {
         const int i = sp * 32 + lane;
         const bool li = i < Cc;
         const float rd = li ? p.scale * ex2(SS.Gr[i] * kLog2e) : 0.f;
         const float rdoi = SS.rdo[i], rqi = SS.rq[i], rd1i = SS.rd1[i];
         const uint8_t* qrow = sm + OFF_QK + ch * G16;
-        float gs = 0.f, pq = 0.f;
+        float gs = 0.f;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
             uint32_t rx[32], rk[32];
@@ -441,22 +446,20 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
             const float* rh = SS.rh + ch * 64 + s * 32;
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8) {
-                float qf[8];
+                float qf[8], a[8];
                 f16x8_to_f32(*reinterpret_cast<const uint4*>(qrow + sw128(i, s * 4 + c8)), qf);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int u = c8 * 8 + e;
                     const float x = u2f(rx[u]) * rdoi * rh[u];
-                    const float a = fmaf(rd, x, u2f(rk[u]) * rd1i);
-                    const float qv = qf[e] * rqi;
-                    gs = fmaf(qv, x, gs);
-                    pq = fmaf(qv, a, pq);
-                    acc[s * 32 + u] = a;
+                    a[e] = fmaf(rd, x, u2f(rk[u]) * rd1i);
+                    gs = fmaf(qf[e] * rqi, x, gs);
                 }
+                *tile_at(OFF_TQ, i, ch * 16 + s * 8 + 2 * c8) = make_float4(a[0], a[1], a[2], a[3]);
+                *tile_at(OFF_TQ, i, ch * 16 + s * 8 + 2 * c8 + 1) = make_float4(a[4], a[5], a[6], a[7]);
             }
         }
         SS.gsum[ch][i] = gs;
-        SS.projq[ch][i] = pq;
     }
     // ---- rows 64-127: the P and carry parts of dK^, the carry's decay gradient
     if (!fail && sp >= 2) {
@@ -464,7 +467,6 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
         const float kd = lj ? ex2((SS.G[Cc - 1] - SS.G[j]) * kLog2e) : 0.f;
         const float rvj = SS.rv[j], rkj = SS.rk[j], rd1tj = SS.rd1t[j];
         const uint8_t* krow = sm + OFF_QK + ch * G16 + 8192;
-        float* dst = p.dKp + ((size_t)(lj ? tok(j) : 0) * p.Hv + h) * 128 + ch * 64;
         float c = 0.f;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
@@ -473,52 +475,49 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
             tmem_ld32(tl + TM_DQ + ch * 64 + s * 32, rq);
             tmem_wait_ld();
             const float* rdh = SS.rdh + ch * 64 + s * 32;
-            float out[32];
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8) {
-                float kf[8];
+                float kf[8], out[8];
                 f16x8_to_f32(*reinterpret_cast<const uint4*>(krow + sw128(j, s * 4 + c8)), kf);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int u = c8 * 8 + e;
                     const float z = u2f(rz[u]) * rvj * rdh[u];
                     c = fmaf(kf[e] * rkj, z, c);
-                    out[u] = fmaf(kd, z, u2f(rq[u]) * rd1tj);
+                    out[e] = fmaf(kd, z, u2f(rq[u]) * rd1tj);
                 }
-            }
-            if (lj) {
-#pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4)
-                    reinterpret_cast<float4*>(dst + s * 32)[e4] =
-                        make_float4(out[4 * e4], out[4 * e4 + 1], out[4 * e4 + 2], out[4 * e4 + 3]);
+                *tile_at(OFF_TK, j, ch * 16 + s * 8 + 2 * c8) = make_float4(out[0], out[1], out[2], out[3]);
+                *tile_at(OFF_TK, j, ch * 16 + s * 8 + 2 * c8 + 1) = make_float4(out[4], out[5], out[6], out[7]);
             }
         }
         SS.ck[ch][j] = c;
     }
     __syncthreads();
-    if (!fail && sp < 2) {
-        const int i = sp * 32 + lane;
-        if (i < Cc) {
-            const float iq = SS.invq[i], rqi = SS.rq[i];
-            // the CUDA-core kernel's projection sum_d q^_d acc_d = |q|^-1 sum_d q_d acc_d
-            const float proj = iq * (SS.projq[0][i] + SS.projq[1][i]);
+    // Row passes: warp w takes positions 8w .. 8w + 7, lane l the features 4l .. 4l + 3.
+    // dq = (dQ^ - q^ (q^ . dQ^)) / |q| (plain 1 / max(|q|, eps) below eps, dQ^ without it)
+    if (!fail) {
+#pragma unroll 2
+        for (int r = 0; r < 8; ++r) {
+            const int i = warp * 8 + r;
+            if (i >= Cc) break;
+            const size_t row = ((size_t)tok(i) * p.Hv + h) * 128;
+            reinterpret_cast<float4*>(p.dW + row)[lane] = *tile_at(OFF_TW, i, lane);
+            reinterpret_cast<float4*>(p.dKp + row)[lane] = *tile_at(OFF_TK, i, lane);
+            const float4 a4 = *tile_at(OFF_TQ, i, lane);
+            const int x0 = 4 * lane;
+            const uint2 raw = *reinterpret_cast<const uint2*>(
+                sm + OFF_QK + (x0 >> 6) * G16 + sw128(i, (x0 >> 3) & 7) + (x0 & 7) * 2);
+            const float f = SS.rq[i] * SS.invq[i];
+            const float2 q01 = unpack_f16x2(raw.x), q23 = unpack_f16x2(raw.y);
+            const float a[4] = {a4.x, a4.y, a4.z, a4.w};
+            const float qh[4] = {q01.x * f, q01.y * f, q23.x * f, q23.y * f};
+            const float proj = warp_sum(qh[0] * a[0] + qh[1] * a[1] + qh[2] * a[2] + qh[3] * a[3]);
             const float n = SS.nq[i];
             const float rn = n > kNormEps ? 1.f / n : 1.f / kNormEps;
-            const uint8_t* qrow = sm + OFF_QK + ch * G16;
-            float* dst = p.dqh + ((size_t)tok(i) * p.Hv + h) * 128 + ch * 64;
+            float o[4];
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-                float qf[8];
-                f16x8_to_f32(*reinterpret_cast<const uint4*>(qrow + sw128(i, c8)), qf);
-                float o[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float a = acc[c8 * 8 + e];
-                    o[e] = on ? (n > kNormEps ? (a - qf[e] * rqi * iq * proj) * rn : a * rn) : a;
-                }
-                reinterpret_cast<float4*>(dst)[2 * c8] = make_float4(o[0], o[1], o[2], o[3]);
-                reinterpret_cast<float4*>(dst)[2 * c8 + 1] = make_float4(o[4], o[5], o[6], o[7]);
-            }
+            for (int e = 0; e < 4; ++e) o[e] = on ? (n > kNormEps ? (a[e] - qh[e] * proj) * rn : a[e] * rn) : a[e];
+            reinterpret_cast<float4*>(p.dqh + row)[lane] = make_float4(o[0], o[1], o[2], o[3]);
         }
     }
     // ---- decay gradient per position, assembled as bwd_chunk_dqk does
