@@ -891,8 +891,8 @@ gdr_status launch_states(const gdr_chunk_args& a, const BwdParams& p, dim3 grid,
 bool bwd_tc_path(const gdr_chunk_args& a);
 
 // Backward workspace: the forward's plan and CUDA-core arrays, then the backward's own.  The
-// tensor-core path reads none of the CUDA-core scan's operands (Q~, K~, P, the layout's last
-// three arrays), so its own arrays start where those would.
+// tensor-core path reads none of the CUDA-core arrays (W, U~, and the scan's Q~, K~, P), so
+// its own arrays, G first, start where those would.
 BwdLayout bwd_layout(const gdr_chunk_args& a) {
     BwdLayout B{};
     B.base = ws_layout(a, true);
@@ -900,7 +900,13 @@ BwdLayout bwd_layout(const gdr_chunk_args& a) {
     const size_t tk = sizeof(float) * (size_t)T_tot * a.Hv * a.dk;
     const size_t tv = sizeof(float) * (size_t)T_tot * a.Hv * a.dv;
     const size_t st = sizeof(float) * (size_t)B.base.max_chunks * a.Hv * a.dk * a.dv;
-    size_t off = bwd_tc_path(a) && B.base.Qt > 0 ? B.base.Qt : B.base.total;
+    const bool tc = bwd_tc_path(a) && B.base.W > 0;
+    size_t off = tc ? B.base.W : B.base.total;
+    if (tc) {
+        B.G = off; off = align_up(off + sizeof(float) * (size_t)T_tot * a.Hv, 256);
+    } else {
+        B.G = B.base.G;
+    }
     B.Hc = off;  off = align_up(off + st, 256);
     B.dHc = off; off = align_up(off + st, 256);
     B.Vp = off;  off = align_up(off + tv, 256);
@@ -942,7 +948,7 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
     p.chunk_seq = reinterpret_cast<const int32_t*>(base + L.chunk_seq);
     float* W = reinterpret_cast<float*>(base + L.W);
     float* U = reinterpret_cast<float*>(base + L.U);
-    float* G = reinterpret_cast<float*>(base + L.G);
+    float* G = reinterpret_cast<float*>(base + B.G);
     p.W = W; p.U = U; p.G = G;
     p.Hc = reinterpret_cast<float*>(base + B.Hc);
     p.dHc = reinterpret_cast<float*>(base + B.dHc);
@@ -960,14 +966,15 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
     p.read_pre = a.read_mode == GDR_READ_PRE; p.qk_l2norm = a.qk_l2norm; p.reverse = a.reverse;
     p.io = a.io_dtype; p.gt = a.gate_dtype; p.scale = a.scale;
 
-    // bf16, head size 128, chunk 64: the tensor-core forward leaves W, U~, G, H and V' (its
-    // saving instantiation), and the per-chunk steps run on the tensor cores
+    // bf16, head size 128, chunk 64: the tensor-core forward leaves G, H and V' (its saving
+    // instantiation), and the per-chunk steps run on the tensor cores (the WY step forms W
+    // and U~ again from its own T)
     const bool tc = bwd_tc_path(a);
     gdr_status s;
     if (tc) {
         // the forward, then the reverse state pass (dH+ per chunk, dV', dS0) on the same kernel
-        const TcSave fw{W, U, G, p.Hc, p.Vp, false};
-        const TcSave ad{nullptr, nullptr, nullptr, p.dHc, p.dVp, true};
+        const TcSave fw{G, p.Hc, p.Vp, false};
+        const TcSave ad{nullptr, p.dHc, p.dVp, true};
         s = launch_chunk_tc(a, x.q, x.k, x.v, x.g, x.beta, x.S0, nullptr, nullptr, ws, L, st,
                             false, nullptr, nullptr, 0, &fw);
         if (s == GDR_OK)

@@ -587,6 +587,8 @@ constexpr uint32_t W_RS = 163840;   // the solve's diagonal blocks
 constexpr uint32_t W_BS = 167936;   // (beta D + (beta D)^T) diag(1/|k|) rows i (K = j): 8 KB
 constexpr uint32_t W_SMALL = 176128;
 constexpr uint32_t WT_SK = 0, WT_DRW = 64, WT_DRU = 128, WT_DA = 192, WT_DK = 0;
+constexpr uint32_t WT_W = WT_DRW, WT_U = WT_DRU;  // W^T, U~^T until P2 takes the columns
+constexpr uint32_t W_V = W_DR;     // beta v rows (K = feature) until the dR epilogue
 // the tail's fp32 rows [64][128], over regions no product reads by then: dR_u over the
 // upper half of [W | U~] (v takes the lower) and T, dR_w over dR, the P4 part over A and
 // the solve's T
@@ -595,6 +597,9 @@ static_assert(W_DRU_S + 32768 <= W_DR && W_DK_S + 32768 <= W_RS, "tail rows");
 
 struct WySmall {
     float4 jf[64];                    // per column j: |k_j|^-1 rk_j, rw_j, G_j
+    // column factors of T for W: beta e^G rk |k|^-1 2^16 (the solve reads column factors in
+    // pairs, so this array and `ones` are 8-byte aligned)
+    alignas(16) float sw[64];
     float G[64], beta[64], ones[64], invk[64], nk[64];
     float rk[64], rw[64], rbs[64];    // reciprocal row factors: k, [W | U~], beta D + ...
     float rr[2], rdr;                 // reciprocal tile factors: dW, dV' halves; dR
@@ -603,11 +608,13 @@ struct WySmall {
     float dgr[2][64], dgc[2][64], db[2][64];  // from dA: row sums, column sums, beta parts
     float rsum[64], vsum[64];         // k^ . dR_w, v . dR_u per position
     float dgf[64], dbf[64];           // dG and dbeta per position
-    uint64_t mbar[4];
+    float wmx[4][64];                 // largest |W|, |U~| of row j, by feature quarter
+    uint64_t mbar[5];
     uint32_t tmem;
     int range_bad;
 };
 constexpr uint32_t W_SMEM = W_SMALL + sizeof(WySmall) + 1024;
+static_assert(offsetof(WySmall, sw) % 8 == 0 && offsetof(WySmall, ones) % 8 == 0, "pair loads");
 static_assert(W_SMALL + sizeof(WySmall) + 1024 <= 227 * 1024, "shared memory");
 
 __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
@@ -633,7 +640,7 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
         tc_fence_before();
     }
     if (tid == 0) {
-        for (int b = 0; b < 4; ++b) mbar_init(&SS.mbar[b], 1);
+        for (int b = 0; b < 5; ++b) mbar_init(&SS.mbar[b], 1);
         mbar_init_fence();
         SS.range_bad = 0;
     }
@@ -675,36 +682,14 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
             }
         }
     }
-    {
-        // [W | U~] rows j (fp32): one factor per row over both halves
-#pragma unroll 1
-        for (int it0 = 0; it0 < 4; it0 += 2) {
-            float4 a[2][4];
+    // v rows (bf16) in registers, converted to fp16 times beta once beta is visible: the
+    // operand of U~ = T (diag(beta) V)
+    uint4 vraw[4];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int idx = tid + (it0 + u) * kTh, j = idx >> 4, c = idx & 15;
-#pragma unroll
-                for (int v = 0; v < 4; ++v) a[u][v] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (j < Cc) {
-                    const size_t row = ((size_t)tok(j) * p.Hv + h) * 128 + c * 8;
-                    const float4* w4 = reinterpret_cast<const float4*>(p.W + row);
-                    const float4* u4 = reinterpret_cast<const float4*>(p.U + row);
-                    a[u][0] = __ldg(w4); a[u][1] = __ldg(w4 + 1);
-                    a[u][2] = __ldg(u4); a[u][3] = __ldg(u4 + 1);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int idx = tid + (it0 + u) * kTh, j = idx >> 4, c = idx & 15;
-                float fw[8], fu[8];
-                f4x2_to_f32(a[u][0], a[u][1], fw);
-                f4x2_to_f32(a[u][2], a[u][3], fu);
-                const float sc = pow2_scale(max16(fmaxf(amax8(fw), amax8(fu))));
-                *reinterpret_cast<uint4*>(sm + W_WF + (c >> 3) * 8192 + sw128(j, c & 7)) = f16x8(fw, sc);
-                *reinterpret_cast<uint4*>(sm + W_WF + (2 + (c >> 3)) * 8192 + sw128(j, c & 7)) = f16x8(fu, sc);
-                if (c == 0) SS.rw[j] = __frcp_rn(sc);
-            }
-        }
+    for (int it = 0; it < 4; ++it) {
+        const int idx = tid + it * kTh, i = idx >> 4, c = idx & 15;
+        vraw[it] = make_uint4(0, 0, 0, 0);
+        if (i < Cc) vraw[it] = __ldg(static_cast<const uint4*>(p.v) + ((size_t)tok(i) * p.Hv + h) * 16 + c);
     }
     // [dW | dV'] (fp32) held in registers until the tile's largest magnitudes are known
     float4 rv[4][2][2];  // [piece][dW, dV'][half]
@@ -748,13 +733,32 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
             *reinterpret_cast<uint4*>(sm + W_R + (2 + (c >> 3)) * 8192 + sw128(j, c & 7)) = f16x8(f, sv);
         }
         if (tid == 0) { SS.rr[0] = __frcp_rn(sw); SS.rr[1] = __frcp_rn(sv); }
+        // beta v rows in fp16, laid out as the k tile (rows i, K = feature); a value beyond
+        // the fp16 range is reported
+        bool vbad = false;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int idx = tid + it * kTh, i = idx >> 4, c = idx & 15;
+            float f[8];
+            bf16x8_to_f32(vraw[it], f);
+            const float bi = SS.beta[i];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] *= bi;
+            vbad |= !(amax8(f) <= 65504.f);
+            *reinterpret_cast<uint4*>(sm + W_V + (c >> 3) * 8192 + sw128(i, c & 7)) = f16x8(f, 1.f);
+        }
+        if (vbad) SS.range_bad = 1;
     }
     fence_proxy_async_smem();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = SS.tmem;
     const uint32_t tl = tmem + ((uint32_t)(sp * 32) << 16);
-    if (tid < 64) SS.jf[tid] = make_float4(SS.invk[tid] * SS.rk[tid], SS.rw[tid], SS.G[tid], 0.f);
+    if (tid < 64) {
+        const float kf = SS.invk[tid] * SS.rk[tid];
+        SS.jf[tid] = make_float4(kf, 0.f, SS.G[tid], 0.f);  // .y = rw once W, U~ are formed
+        SS.sw[tid] = SS.beta[tid] * ex2(SS.G[tid] * kLog2e) * kf * 65536.f;
+    }
 
     // ---- P1: k . k
     if (tid == 0) {
@@ -797,8 +801,68 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
                 wy_diag_stage0(vals, i, lane, ch, As, reinterpret_cast<float*>(sm + W_RS), Ts);
             }
         }
-        wy_solve_offdiag(As, Ts, reinterpret_cast<float*>(sm + W_RS), sm + W_T, SS.ones, SS.ones, tid,
+        // T at W_T (dR and U~), T diag(sw) 8 KB on (W)
+        wy_solve_offdiag(As, Ts, reinterpret_cast<float*>(sm + W_RS), sm + W_T, SS.ones, SS.sw, tid,
                          kBarSolve, kTh, [](int) {});
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- P1b: W^T = K^T (T diag(sw))^T 2^-16 and U~^T = (diag(beta) V)^T T^T (A = the k or
+    //      beta v tile, MN-major; B = T rows j, K-major), into the dR columns
+    if (tid == 0 && !fail) {
+        const uint32_t id = idesc_f32acc(128, 64, true, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            mma_f32acc_ss(tmem + WT_W, sdesc_sw128(sbase + W_K + kk * 2048, 8192, 1024),
+                          kdesc(sbase + W_T + 8192 + kk * 32), id, kk > 0);
+            mma_f32acc_ss(tmem + WT_U, sdesc_sw128(sbase + W_V + kk * 2048, 8192, 1024),
+                          kdesc(sbase + W_T + kk * 32), id, kk > 0);
+        }
+        mma_commit(&SS.mbar[4]);
+    }
+    if (!fail) fail = !mbar_wait_bounded(&SS.mbar[4], 0, kWaitNs);
+    fail = __syncthreads_or(fail);
+    tc_fence_after();
+    // [W | U~] rows j in fp16 with one factor per row, the B operand of P3 (every warp: lanes
+    // = the feature within its quarter, columns = positions 32 ch .. 32 ch + 31)
+    if (!fail) {
+        uint32_t rwv[32], ruv[32];
+        tmem_ld32(tl + WT_W + ch * 32, rwv);
+        tmem_ld32(tl + WT_U + ch * 32, ruv);
+        tmem_wait_ld();
+        float m[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u)
+            m[u] = max_abs_nan(max_abs_nan(0.f, u2f(rwv[u]) * 0x1p-16f), u2f(ruv[u]));
+        bool bad = false;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) bad |= !(m[u] <= 3.402823e38f);
+        if (bad) SS.range_bad = 1;
+        SS.wmx[sp][ch * 32 + lane] = transpose_reduce32<true>(m, lane);
+        __syncthreads();
+        const int jl = ch * 32 + lane;
+        const float scl = pow2_scale(fmaxf(fmaxf(SS.wmx[0][jl], SS.wmx[1][jl]), fmaxf(SS.wmx[2][jl], SS.wmx[3][jl])));
+        if (sp == 0) {
+            SS.rw[jl] = __frcp_rn(scl);
+            SS.jf[jl].y = __frcp_rn(scl);
+        }
+        uint16_t* wf = reinterpret_cast<uint16_t*>(sm + W_WF);
+        const int x = sp * 32 + lane;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            const int j = ch * 32 + u;
+            const float sc = __shfl_sync(0xffffffffu, scl, u);
+            const __half hw = __float2half_rn(u2f(rwv[u]) * 0x1p-16f * sc);
+            const __half hu = __float2half_rn(u2f(ruv[u]) * sc);
+            const int o = ((x >> 6) * 8192 + sw128(j, (x >> 3) & 7)) / 2 + (x & 7);
+            wf[o] = *reinterpret_cast<const uint16_t*>(&hw);
+            wf[o + 8192] = *reinterpret_cast<const uint16_t*>(&hu);
+        }
+    } else {
+        __syncthreads();  // the barrier every thread of the branch above takes
     }
     fence_proxy_async_smem();
     tc_fence_before();

@@ -151,7 +151,7 @@ struct TcParams {
     // the saving instantiation (kSave) leaves what the backward reads, fp32: W and U~ by
     // token ([token][head][d]), the in-chunk cumulative log decay G ([token][head]), the state
     // at every chunk start ([chunk][head][dk][dv]) and V' ([token][head][dv]); no output
-    float *sv_W, *sv_U, *sv_G, *sv_H, *sv_V;
+    float *sv_G, *sv_H, *sv_V;
 };
 
 // The fused gating prologue's per-head arrays, a kernel argument of its own that only the
@@ -920,30 +920,7 @@ chunk_fused_tc(TcParams p, const __grid_constant__ CUtensorMap tm_q,
                         *reinterpret_cast<uint4*>(sm + OFF_WN + pb * 16384 + sw128(lt, half * 4 + e8)) =
                             h8(f);
                     }
-                // a proxy fence waits for this thread's global stores in flight: the saving
-                // forward's stores of W (lane = d) and U~ (lane = e) come after it, and U~ is
-                // read out before the group barrier that lets V' accumulate over it
                 fence_proxy_async_smem();
-                if constexpr (kSave) {
-                    float* wrow = p.sv_W + ((size_t)(tokA + tstep * c * C) * p.Hv + h) * D + lt;
-                    float* urow = p.sv_U + ((size_t)(tokA + tstep * c * C) * p.Hv + h) * D + lt;
-                    const long long rstep = tstep * (long long)p.Hv * D;
-#pragma unroll
-                    for (int i = 0; i < C; ++i)
-                        if (i >= row_lo(c) && i < Cc) wrow[rstep * i] = u2f(rw[i >> 5][i & 31]);
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t ru[32];
-                        tmem_ld32(tlane + TM_DU + pb * 64 + half * 32, ru);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int m = 0; m < 32; ++m) {
-                            const int i = half * 32 + m;
-                            if (i >= row_lo(c) && i < Cc) urow[rstep * i] = u2f(ru[m]);
-                        }
-                    }
-                    tc_fence_before();
-                }
             }
             named_bar(kBarChain, 128);
             // C1: V'^T = U~^T + H^T (-W^T);  O^T = H^T Q~^T   (A = state copy in TMEM)
@@ -1294,8 +1271,6 @@ gdr_status launch_chunk_tc(const gdr_chunk_args& a, const void* q, const void* k
     p.g_rev = g_rev; p.beta_rev = beta_rev;
     p.chunk_off = reinterpret_cast<const int32_t*>(base + L.chunk_off);
     p.part = pair ? reinterpret_cast<float*>(base + part_off) : nullptr;
-    p.sv_W = save ? save->W : nullptr;
-    p.sv_U = save ? save->U : nullptr;
     p.sv_G = save ? save->G : nullptr;
     p.sv_H = save ? save->H : nullptr;
     p.sv_V = save ? save->V : nullptr;

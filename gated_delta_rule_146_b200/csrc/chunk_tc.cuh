@@ -7,12 +7,12 @@
 namespace gdr {
 
 // The backward's two passes on the fused kernel (fp32 outputs, see TcParams in chunk_tc.cu).
-// Forward (adjoint = false): W and U~ ([token][head][128]), G ([token][head]), the state at
-// every chunk start H ([chunk][head][128][128]) and V' ([token][head][128]).  Adjoint
+// Forward (adjoint = false): G ([token][head]), the state at every chunk start H
+// ([chunk][head][128][128]) and V' ([token][head][128]).  Adjoint
 // (adjoint = true; the launch's v is dO, S0 is dS_final and S_final is dS0): dH+ of every
 // chunk in H and dV' in V.
 struct TcSave {
-    float *W, *U, *G, *H, *V;
+    float *G, *H, *V;
     bool adjoint;
 };
 

@@ -158,6 +158,7 @@ gdr_status launch_prep_simt(const gdr_chunk_args& a, const void* q, const void* 
 // Backward pass (chunk_bwd.cu).
 struct BwdLayout {
     WsLayout base;  // the forward's plan and CUDA-core arrays
+    size_t G;       // the in-chunk log decay (the base layout's, or the backward's own)
     size_t Hc, dHc, Vp, dVp, dW, dKp, dqh, dkh, dGp, total;
 };
 struct BwdPtrs {
