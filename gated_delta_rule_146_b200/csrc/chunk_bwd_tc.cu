@@ -182,18 +182,6 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
     const uint4* kg = static_cast<const uint4*>(p.k);
     const uint4* dog = static_cast<const uint4*>(p.dO);
 
-    if (warp == 0) {
-        tmem_alloc(&SS.tmem, 512);
-        tmem_relinquish();
-        tc_fence_before();
-    }
-    if (tid == 0) {
-        mbar_init(&SS.mbar[0], 1);
-        mbar_init(&SS.mbar[1], 1);
-        mbar_init_fence();
-    }
-    if (tid < 64) SS.G[tid] = tid < Cc ? p.G[(size_t)tok(tid) * p.Hv + h] : 0.f;
-
     // ---- staging.  Each row of 128 values is 16 pieces of 8, held by 16 consecutive lanes,
     // which agree on the row's factor; rows past the chunk are zero.
     {
@@ -208,6 +196,18 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
                 raw[it] = __ldg((t == 2 ? dog : t ? kg : qg) + row * 16 + c);
             }
         }
+        // the setup that no staged value needs goes after the first loads are in flight
+        if (warp == 0) {
+            tmem_alloc(&SS.tmem, 512);
+            tmem_relinquish();
+            tc_fence_before();
+        }
+        if (tid == 0) {
+            mbar_init(&SS.mbar[0], 1);
+            mbar_init(&SS.mbar[1], 1);
+            mbar_init_fence();
+        }
+        if (tid < 64) SS.G[tid] = tid < Cc ? p.G[(size_t)tok(tid) * p.Hv + h] : 0.f;
 #pragma unroll
         for (int it = 0; it < 12; ++it) {
             const int idx = tid + it * kTh, t = idx >> 10, i = (idx >> 4) & 63, c = idx & 15;
@@ -634,24 +634,6 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
     float* As = reinterpret_cast<float*>(sm + W_AS);
     float* Ts = reinterpret_cast<float*>(sm + W_TS);
 
-    if (warp == 0) {
-        tmem_alloc(&SS.tmem, 256);
-        tmem_relinquish();
-        tc_fence_before();
-    }
-    if (tid == 0) {
-        for (int b = 0; b < 5; ++b) mbar_init(&SS.mbar[b], 1);
-        mbar_init_fence();
-        SS.range_bad = 0;
-    }
-    if (tid < 64) {
-        const bool lt = tid < Cc;
-        const size_t gi = lt ? (size_t)tok(tid) * p.Hv + h : 0;
-        SS.G[tid] = lt ? p.G[gi] : 0.f;
-        SS.beta[tid] = lt ? load_elem(p.beta, gi, p.gt) : 0.f;
-        SS.ones[tid] = 1.f;
-    }
-
     // ---- staging
     {
         // k rows (bf16), with their norms
@@ -662,6 +644,24 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
             raw[it] = make_uint4(0, 0, 0, 0);
             if (i < Cc)
                 raw[it] = __ldg(static_cast<const uint4*>(p.k) + ((size_t)tok(i) * p.Hk + hk) * 16 + c);
+        }
+        // the setup that no staged value needs goes after the first loads are in flight
+        if (warp == 0) {
+            tmem_alloc(&SS.tmem, 256);
+            tmem_relinquish();
+            tc_fence_before();
+        }
+        if (tid == 0) {
+            for (int b = 0; b < 5; ++b) mbar_init(&SS.mbar[b], 1);
+            mbar_init_fence();
+            SS.range_bad = 0;
+        }
+        if (tid < 64) {
+            const bool lt = tid < Cc;
+            const size_t gi = lt ? (size_t)tok(tid) * p.Hv + h : 0;
+            SS.G[tid] = lt ? p.G[gi] : 0.f;
+            SS.beta[tid] = lt ? load_elem(p.beta, gi, p.gt) : 0.f;
+            SS.ones[tid] = 1.f;
         }
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
