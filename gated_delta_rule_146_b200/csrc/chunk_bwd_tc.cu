@@ -384,22 +384,6 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
         if (ch == 0) SS.rd1[i] = __frcp_rn(sd);
         if (sp == 0) SS.rd1t[ch * 32 + lane] = __frcp_rn(stl);
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    // ---- second products: D1 K^ and D1^T Q^ (B = the k or q tile, MN-major)
-    if (tid == 0 && !fail) {
-        const uint32_t ib = idesc_f32acc(128, 128, false, true, false);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            mma_f32acc_ss(tmem + TM_DK, kdesc(sbase + OFF_D + kk * 32),
-                          sdesc_sw128(sbase + OFF_QK + 8192 + kk * 2048, G16, 1024), ib, kk > 0);
-            mma_f32acc_ss(tmem + TM_DQ, kdesc(sbase + OFF_D + kk * 32),
-                          sdesc_sw128(sbase + OFF_QK + kk * 2048, G16, 1024), ib, kk > 0);
-        }
-        mma_commit(&SS.mbar[1]);
-    }
     // dW, the P and carry parts of dK^ and dQ^ leave as fp32 rows [64][128] staged over the
     // operands the first products read (dO, dV', V', H, dH+); a row's 16-byte piece pc sits
     // at pc ^ (row & 7), so that 32 rows' same piece and one row's 32 pieces both spread over
@@ -407,8 +391,8 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
     auto tile_at = [&](uint32_t off, int row, int pc) {
         return reinterpret_cast<float4*>(sm + off + row * 512 + ((pc ^ (row & 7)) << 4));
     };
-    // rows 64-127 (warps 2, 3, 6, 7): dW = -(dV' H^T) while the second products run.  The
-    // TMEM loads are warp-wide instructions: every lane issues them, live row or not.
+    // rows 64-127 (warps 2, 3, 6, 7, idle in D1, which only rows 0-63 take): dW = -(dV' H^T).
+    // The TMEM loads are warp-wide instructions: every lane issues them, live row or not.
     const int j = (sp - 2) * 32 + lane;  // the row's position, for sp >= 2
     if (!fail && sp >= 2) {
         const float rdvj = -SS.rdv[j & 63];
@@ -424,6 +408,22 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
                     u2f(r[4 * e4]) * rdvj * rh[4 * e4], u2f(r[4 * e4 + 1]) * rdvj * rh[4 * e4 + 1],
                     u2f(r[4 * e4 + 2]) * rdvj * rh[4 * e4 + 2], u2f(r[4 * e4 + 3]) * rdvj * rh[4 * e4 + 3]);
         }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // ---- second products: D1 K^ and D1^T Q^ (B = the k or q tile, MN-major)
+    if (tid == 0 && !fail) {
+        const uint32_t ib = idesc_f32acc(128, 128, false, true, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            mma_f32acc_ss(tmem + TM_DK, kdesc(sbase + OFF_D + kk * 32),
+                          sdesc_sw128(sbase + OFF_QK + 8192 + kk * 2048, G16, 1024), ib, kk > 0);
+            mma_f32acc_ss(tmem + TM_DQ, kdesc(sbase + OFF_D + kk * 32),
+                          sdesc_sw128(sbase + OFF_QK + kk * 2048, G16, 1024), ib, kk > 0);
+        }
+        mma_commit(&SS.mbar[1]);
     }
     if (!fail) fail = !mbar_wait_bounded(&SS.mbar[1], 0, kWaitNs);
     fail = __syncthreads_or(fail);
