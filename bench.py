@@ -50,7 +50,8 @@ CHUNK_TC_SOURCES = ("chunk_tc.cu", "chunk_tc.cuh", "wy_solve.cuh", "tc_ptx.cuh",
 G2_TC_SOURCES = ("chunk_g2_tc.cu", "wy_solve.cuh", "tc_ptx.cuh", "common.cuh")
 BWD_TC_SOURCES = ("chunk_bwd_tc.cu", "chunk_bwd.cuh", "wy_solve.cuh", "tc_ptx.cuh", "common.cuh")
 BWD_SOURCES = ("chunk_bwd.cu", "chunk_bwd.cuh", "common.cuh")
-# the kernels of one tensor-core backward call, with the sources of their traffic records
+# the kernels of one tensor-core backward call, with the sources of their traffic records (the
+# head reduction only where several v-heads share a key head)
 BWD_TC_KERNELS = (("chunk_fused_tc_save", CHUNK_TC_SOURCES), ("chunk_fused_tc_adj", CHUNK_TC_SOURCES),
                   ("bwd_chunk_dqk_tc", BWD_TC_SOURCES), ("bwd_chunk_wy_tc", BWD_TC_SOURCES),
                   ("bwd_reduce_heads4", BWD_SOURCES))
@@ -470,7 +471,9 @@ def bench_ours(args, rank, world, local_rank):
                     "workspace_bytes": bws_.numel()}
         if backward["path"] == "tc":
             # measured traffic of the call's kernels, the intermediate arrays included
-            tp = [measured_traffic(k, src, w.B) for k, src in BWD_TC_KERNELS]
+            # (with one v-head per key head the head reduction is not launched)
+            tp = [measured_traffic(k, src, w.B) for k, src in BWD_TC_KERNELS
+                  if k != "bwd_reduce_heads4" or w.Hv != w.Hk]
             backward["traffic"] = None if None in tp else sum(tp)
         del bws_
 

@@ -970,6 +970,7 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
     // instantiation), and the per-chunk steps run on the tensor cores (the WY step forms W
     // and U~ again from its own T)
     const bool tc = bwd_tc_path(a);
+    p.direct_out = tc && a.Hv == a.Hk;
     gdr_status s;
     if (tc) {
         // the forward, then the reverse state pass (dH+ per chunk, dV', dS0) on the same kernel
@@ -1000,9 +1001,11 @@ gdr_status launch_chunk_bwd(const gdr_chunk_args& a, const BwdPtrs& x, void* ws,
             bwd_chunk_dqk<<<gc, kNT, sm_q, st>>>(p);
             bwd_chunk_wy<<<gc, kNT, sm_w, st>>>(p);
         }
+        // with one v-head per key head there is nothing to sum: the tensor-core kernels
+        // write dq and dk themselves
         const long long n4 = (long long)a.B * a.T * a.Hk * (a.dk / 4);
         const unsigned blocks = (unsigned)std::min<long long>((n4 + kThreads - 1) / kThreads, 148LL * 16);
-        if (n4 > 0) bwd_reduce_heads4<<<blocks, kThreads, 0, st>>>(p, n4);
+        if (n4 > 0 && !p.direct_out) bwd_reduce_heads4<<<blocks, kThreads, 0, st>>>(p, n4);
     }
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }

@@ -23,6 +23,7 @@ struct BwdParams {
     int Hk, Hv, dk, dv, chunk, read_pre, qk_l2norm, reverse;
     gdr_dtype io, gt;
     float scale;
+    int direct_out;  // tensor cores with Hv == Hk: dq, dk leave the per-chunk kernels in bf16
 };
 
 struct ChunkPos {

@@ -141,6 +141,12 @@ __device__ __forceinline__ void f16x8_to_f32(const uint4& v, float (&f)[8]) {
     }
 }
 
+// four values -> four bf16, rounded to nearest, as one 8-byte word
+__device__ __forceinline__ uint2 bf16x4(const float (&o)[4]) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(o[0], o[1]), b = __floats2bfloat162_rn(o[2], o[3]);
+    return make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+}
+
 __device__ __forceinline__ void f4x2_to_f32(const float4& a, const float4& b, float (&f)[8]) {
     f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
     f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
@@ -517,7 +523,10 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_dqk_tc(BwdParams p) {
             float o[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[e] = on ? (n > kNormEps ? (a[e] - qh[e] * proj) * rn : a[e] * rn) : a[e];
-            reinterpret_cast<float4*>(p.dqh + row)[lane] = make_float4(o[0], o[1], o[2], o[3]);
+            if (p.direct_out)  // one v-head per key head: dq itself, in bf16
+                reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.dq_out) + row)[lane] = bf16x4(o);
+            else
+                reinterpret_cast<float4*>(p.dqh + row)[lane] = make_float4(o[0], o[1], o[2], o[3]);
         }
     }
     // ---- decay gradient per position, assembled as bwd_chunk_dqk does
@@ -1117,8 +1126,11 @@ __global__ void __launch_bounds__(kTh, 1) bwd_chunk_wy_tc(BwdParams p) {
             float o[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[e] = on ? (n > kNormEps ? (a[e] - kh[e] * proj) * rn : a[e] * rn) : a[e];
-            reinterpret_cast<float4*>(p.dkh + ((size_t)tok(i) * p.Hv + h) * 128)[lane] =
-                make_float4(o[0], o[1], o[2], o[3]);
+            const size_t row = ((size_t)tok(i) * p.Hv + h) * 128;
+            if (p.direct_out)  // one v-head per key head: dk itself, in bf16
+                reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.dk_out) + row)[lane] = bf16x4(o);
+            else
+                reinterpret_cast<float4*>(p.dkh + row)[lane] = make_float4(o[0], o[1], o[2], o[3]);
         }
     }
     // ---- dG, dbeta per position and dg = the reverse cumulative sum of dG within the chunk
