@@ -267,9 +267,11 @@ gdr_status gdr_chunk_fwd_bidir(const gdr_chunk_args* args,
  *               256-byte aligned, no initialisation needed
  *
  * Kernels.  bf16, dk = dv = 128, chunk 64 ("tc"): the tensor-core forward kernel runs twice,
- * once leaving W, U~, the in-chunk decay, the state at every chunk start and V', once as the
- * adjoint recurrence from dS_final back to dS0 (dH+ at every chunk, dV'); two per-(chunk,
- * head) tcgen05 kernels then form dq, dk, dv, dg and dbeta.  Their operands are fp16, each row
+ * once leaving the in-chunk decay, the state at every chunk start and V', once as the adjoint
+ * recurrence from dS_final back to dS0 (dH+ at every chunk, dV'); two per-(chunk, head)
+ * tcgen05 kernels then form dq, dk, dv, dg and dbeta, the second forming W and U~ again from
+ * its own solve.  With one v-head per key head they write dq and dk themselves; otherwise a
+ * last kernel sums them over each key head's v-heads.  Their operands are fp16, each row
  * (or tile) scaled by a power of two; an fp16 operand of the recurrences that leaves its range
  * (|dO| or a gradient of the state beyond 65504) is reported as GDR_ERR_RANGE through the
  * workspace, as in gdr_chunk_fwd.  Other sizes and fp32 ("simt"): fp32 CUDA-core kernels.
